@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Benchmark of the TurboQuant decode hot path on B200.
+
+A step is one decode step of the long-context workload (B=4, Hq=16/Hkv=8,
+d=128, 102400 compressed tokens per sequence) through the library's C ABI:
+encode one new K and one new V vector per (batch, kv head) into the cache
+(tq_encode_k / tq_encode_v) and attend over the whole compressed cache
+(tq_attend_decode: query prologue, split-K attention, combine).  The headline
+metric is the achieved bandwidth on the compressed-cache bytes the step must
+read (118 B per token per kv head); the encode-only workload (B=1, 8 kv heads,
+32768 bf16 tokens) gives the KV encode throughput in Mvectors/s.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs an independent
+replica on its own GPU (the workload shards by sequence with no exchange), and
+rank 0 prints one JSON line with the whole-job numbers (max time over ranks).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_vector_14_b200 import synthetic  # noqa: E402
+
+METRIC = "decode-attn achieved HBM GB/s (% of B200 peak); KV encode Mvectors/s"
+UNIT = "GB/s"
+BYTES_PER_TOKEN_HEAD = {128: 68 + 50, 256: 132 + 98}      # packed K + V record per token per kv head
+ENCODE_BYTES_PER_VECTOR = {("k", 128): 68, ("v", 128): 50}
+
+# DRAM traffic of the split-K kernel from one ncu capture, valid only while the
+# kernel source is unchanged (sha256 of csrc/tq_decode.cu at capture time).
+NCU_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None, "capture": None}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def source_sha(rel: str) -> str:
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.proc = None
+        self.out = None
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+            if uuid:
+                cmd += ["-i", uuid]
+            self.out = open(os.devnull if not os.path.isdir("/tmp") else f"/tmp/tq_clocks_{os.getpid()}.csv", "w+")
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.seek(0)
+        rows = [r.split(",") for r in self.out.read().strip().splitlines() if r.count(",") >= 8]
+        self.out.close()
+        try:
+            os.unlink(self.out.name)
+        except Exception:
+            pass
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" == r[5 + i].strip()})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle (baseline)
+
+def oracle_decode_rate(w, seconds: float, tokens: int | None = None):
+    """Time the float64 oracle's decode attention on host cores over a bounded
+    sample: the G query heads of kv head 0 of sequence 0, over its first
+    `tokens` compressed tokens (the oracle encodes them itself).  Returns
+    (GB/s on the algorithmic bytes, threads, sample text, seconds of work)."""
+    import oracle as O
+    tokens = tokens or w.T
+    prm = O.params(w.d, 0)
+    xk = synthetic.kv(w, "k", 0, tokens, batches=[0])[0, 0].astype(np.float64)
+    xv = synthetic.kv(w, "v", 0, tokens, batches=[0])[0, 0].astype(np.float64)
+    ek, ev = O.encode(xk, prm, True), O.encode(xv, prm, False)
+    kc = {"idx": ek["idx"], "sig": ek["sig"], "nh": ek["nh"], "gh": ek["gh"]}
+    vc = {"idx": ev["idx"], "nh": ev["nh"]}
+    G = w.Hq // w.Hkv
+    q = synthetic.queries(w)[0, :G].astype(np.float64)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        O.attend(prm, q, kc, vc, w.scale)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    nbytes = n * tokens * BYTES_PER_TOKEN_HEAD[w.d]
+    threads = min(G, O.num_threads())
+    sample = (f"oracle attention of {G} query heads over {tokens} tokens of one kv head "
+              f"(float64, {n} repetitions, {el:.1f} s)")
+    return nbytes / el / 1e9, threads, sample, el
+
+
+def oracle_encode_rate(w, seconds: float):
+    import oracle as O
+    prm = O.params(w.d, 0)
+    x = synthetic.kv(w, "k", 0, 4096, batches=[0])[0].reshape(-1, w.d).astype(np.float64)
+    t0 = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t0 < seconds:
+        O.encode(x, prm, True)
+        O.encode(x, prm, False)
+        n += 2 * x.shape[0]
+    el = time.perf_counter() - t0
+    return n / el / 1e6, O.num_threads(), f"oracle encode of {x.shape[0]} K and V vectors, repeated ({el:.1f} s)"
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    w = synthetic.WORKLOADS["c4"]
+    budget = 120.0 / max(args.steps + args.warmup, 1)       # seconds per step
+    # calibrate tokens per step so the whole run stays within a few minutes
+    probe = 2048
+    rate, _, _, _ = oracle_decode_rate(w, 0.5, probe)
+    tok = int(max(256, min(w.T, rate * 1e9 * budget * 0.8 / BYTES_PER_TOKEN_HEAD[w.d])))
+    tok = tok // 64 * 64
+    import oracle as O
+    prm = O.params(w.d, 0)
+    xk = synthetic.kv(w, "k", 0, tok, batches=[0])[0, 0].astype(np.float64)
+    xv = synthetic.kv(w, "v", 0, tok, batches=[0])[0, 0].astype(np.float64)
+    ek, ev = O.encode(xk, prm, True), O.encode(xv, prm, False)
+    kc = {"idx": ek["idx"], "sig": ek["sig"], "nh": ek["nh"], "gh": ek["gh"]}
+    vc = {"idx": ev["idx"], "nh": ev["nh"]}
+    G = w.Hq // w.Hkv
+    q = synthetic.queries(w)[0, :G].astype(np.float64)
+    for _ in range(args.warmup):
+        O.attend(prm, q, kc, vc, w.scale)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.attend(prm, q, kc, vc, w.scale)
+    el = time.perf_counter() - t0
+    value = args.steps * tok * BYTES_PER_TOKEN_HEAD[w.d] / el / 1e9
+    threads = min(G, O.num_threads())
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.title, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.d, "T": w.T,
+                   "l2": "n/a (host)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"per step: oracle attention of {G} query heads over {tok} tokens of one kv head"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank: int, world: int, dist):
+    import torch
+    from kv_cache_vector_14_b200 import build, tq
+
+    build.build()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    w = synthetic.WORKLOADS["c4"]
+    d, B, Hq, Hkv, T = w.d, w.B, w.Hq, w.Hkv, w.T
+    h = tq.tq_init(d, 0)
+    kc, vc = tq.Cache(d, True, B, Hkv, T), tq.Cache(d, False, B, Hkv, T)
+    for which, cache in (("k", kc), ("v", vc)):
+        x = torch.from_numpy(synthetic.kv(w, which)).to(dev)
+        (tq.tq_encode_k if which == "k" else tq.tq_encode_v)(h, x, cache, 0)
+        torch.cuda.synchronize()
+        if which == "k":
+            k_new = x[:, :, T - 1:T].clone()
+        else:
+            v_new = x[:, :, T - 1:T].clone()
+        del x
+    q = torch.from_numpy(synthetic.queries(w)).to(dev).to(torch.bfloat16)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    ws = torch.empty(tq.tq_attend_workspace_bytes(h, B, Hq, Hkv, T), dtype=torch.uint8, device=dev)
+    path = tq.tq_attend_path(h, Hq, Hkv)
+
+    def step(kn, vn, qq, o):
+        tq.tq_encode_k(h, kn, kc, T - 1)
+        tq.tq_encode_v(h, vn, vc, T - 1)
+        tq.tq_attend_decode(h, qq, kc, vc, o, ws, T=T, scale=w.scale)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step(k_new, v_new, q, out)
+    torch.cuda.synchronize()
+
+    # ---- timed region (device-resident inputs); the split-K kernel timed alone by events
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        tq.tq_set_decode_events(h, kev[i][0], kev[i][1])
+        step(k_new, v_new, q, out)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    tq.tq_set_decode_events(h, None, None)
+    clocks = sampler.stop() if sampler else None
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = max_over_ranks(ms)
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    bytes_step = B * Hkv * T * BYTES_PER_TOKEN_HEAD[d]
+    value = world * bytes_step / (ms_max * 1e-3) / 1e9
+
+    # ---- end to end: pinned host inputs copied in, the output read back, every step
+    kh = k_new.cpu().pin_memory()
+    vh = v_new.cpu().pin_memory()
+    qh = q.cpu().pin_memory()
+    oh = torch.empty_like(out, device="cpu").pin_memory()
+    kd, vd, qd = torch.empty_like(k_new), torch.empty_like(v_new), torch.empty_like(q)
+    n_e2e = max(1, min(args.steps, 2000))
+    for _ in range(3):
+        kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True); qd.copy_(qh, non_blocking=True)
+        step(kd, vd, qd, out)
+        oh.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record()
+    for _ in range(n_e2e):
+        kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True); qd.copy_(qh, non_blocking=True)
+        step(kd, vd, qd, out)
+        oh.copy_(out, non_blocking=True)
+    e3.record()
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e2.elapsed_time(e3) / n_e2e)
+    e2e_value = world * bytes_step / (ms_e2e * 1e-3) / 1e9
+    h2d = (kh.numel() + vh.numel()) * 4 + qh.numel() * 2
+    d2h = oh.numel() * 4
+
+    # ---- encode-only workload: KV encode throughput
+    we = synthetic.WORKLOADS["c2"]
+    xk = torch.from_numpy(synthetic.kv(we, "k")).to(dev).to(torch.bfloat16)
+    xv = torch.from_numpy(synthetic.kv(we, "v")).to(dev).to(torch.bfloat16)
+    ekc = tq.Cache(we.d, True, we.B, we.Hkv, we.T)
+    evc = tq.Cache(we.d, False, we.B, we.Hkv, we.T)
+    for _ in range(3):
+        tq.tq_encode_k(h, xk, ekc, 0)
+        tq.tq_encode_v(h, xv, evc, 0)
+    n_enc = 30
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)      # 2x L2: evict between passes
+    enc_ms = []
+    for _ in range(n_enc):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        tq.tq_encode_k(h, xk, ekc, 0)
+        tq.tq_encode_v(h, xv, evc, 0)
+        b.record()
+        torch.cuda.synchronize()
+        enc_ms.append(a.elapsed_time(b))
+    enc_med = statistics.median(enc_ms)
+    nvec = 2 * we.B * we.Hkv * we.T
+    enc_bytes = we.B * we.Hkv * we.T * (2 * we.d * 2 + ENCODE_BYTES_PER_VECTOR[("k", 128)] +
+                                        ENCODE_BYTES_PER_VECTOR[("v", 128)])
+    enc_mvps = max_over_ranks(enc_med)
+    enc_mvps = world * nvec / (enc_mvps * 1e-3) / 1e6
+    del xk, xv, flush
+
+    peak, peak_kind = peaks()
+    achieved = bytes_step / (kern_ms * 1e-3) / 1e9
+    traffic = NCU_TRAFFIC["bytes_per_launch"] if NCU_TRAFFIC["source_sha256"] == source_sha(
+        "kv_cache_vector_14_b200/csrc/tq_decode.cu") else None
+
+    cpu = None
+    enc_cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample, _ = oracle_decode_rate(w, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        ev_, ecores, esample = oracle_encode_rate(we, min(10.0, args.cpu_seconds))
+        enc_cpu = {"value": ev_, "unit": "Mvectors/s", "cores": ecores, "kind": "oracle", "sample": esample}
+
+    status = tq.tq_device_status(h)
+    tq.tq_destroy(h)
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.title, "B": B, "Hq": Hq, "Hkv": Hkv, "head_dim": d, "T": T,
+                   "step": "encode 1 K + 1 V per (batch, kv head), then attention over the compressed cache",
+                   "algorithmic_bytes_per_step": bytes_step, "decode_path": path,
+                   "l2": "inputs larger than L2 (386.7 MB compressed cache read per step vs 126 MB L2)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "kernel": f"tq_decode ({path})",
+                     "kernel_ms": kern_ms, "peak_kind": f"{peak_kind} (copy bandwidth, burst)",
+                     "frac_of_8000": achieved / 8000.0},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": ms_e2e},
+        "gpu_launches": 5 * args.steps,
+        "clocks": clocks,
+        "encode": {"workload": we.title, "value": enc_mvps, "unit": "Mvectors/s", "ms_per_pass": enc_med,
+                   "vectors_per_pass": nvec, "algorithmic_bytes_per_pass": enc_bytes,
+                   "achieved_gbs": enc_bytes / (enc_med * 1e-3) / 1e9,
+                   "frac": enc_bytes / (enc_med * 1e-3) / 1e9 / peak, "l2": "256 MB buffer written between passes",
+                   "cpu_baseline": enc_cpu},
+        "device_status": tq.tq_status_string(status),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    try:
+        run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,191 @@
+/*
+ * tq.h -- C ABI of libtq: TurboQuant KV-cache compression and decode attention
+ * over the compressed cache, for NVIDIA B200 (sm_100a).
+ *
+ * The method (page "Apple Silicon向けSwiftLM、TurboQuant KVキャッシュ圧縮とSSD
+ * Expert Streamingを実装", ai-heartland.com):
+ *   K cache, section "K-Cache圧縮：3-bit PolarQuant + 1-bit QJL = 4.25 bits/dim":
+ *     1. L2-norm extraction and normalisation, x_hat = x / ||x||;
+ *     2. a fast Walsh-Hadamard rotation that spreads outliers (applied here
+ *        after a fixed random sign diagonal D: y = H D x_hat);
+ *     3. a 3-bit non-linear Lloyd-Max codebook per coordinate;
+ *     4. the residual of step 3;
+ *     5. a Johnson-Lindenstrauss (QJL) projection of the residual, keeping one
+ *        sign bit per projection.
+ *   V cache, section "V-Cache圧縮：3-bit PolarQuant = 3.125 bits/dim":
+ *     steps 1-3 only; V is not used for scoring, so it carries no QJL bit.
+ *   Attention, section on the hybrid V2+V3 design: dequantisation is fused
+ *     into the attention kernel, which reads the packed cache directly.
+ *
+ * Conventions.  d = head_dim (128 or 256); m = d JL rows; tokens per cache
+ * block = 64.  All data buffers (inputs, caches, outputs, workspace) are
+ * device memory owned by the caller; the library owns only the constants
+ * created by tq_init.  Hot calls (encode, attend) allocate nothing, do not
+ * synchronise and copy nothing to the host; they enqueue kernels on the
+ * caller's stream and return.  Errors in the arguments are detected on the
+ * host before anything is launched and leave all buffers untouched.
+ * Asynchronous device faults surface at the caller's next synchronisation.
+ * A handle is read-only after tq_init, so concurrent calls on different
+ * streams are safe; calls whose outputs overlap race.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifndef TQ_API
+#define TQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tq_handle tq_handle;
+
+/* Status codes.  TQ_ERR_CUDA: a CUDA runtime call or a launch failed.
+ * TQ_ERR_WORKSPACE: the workspace passed is smaller than required.
+ * TQ_ERR_DEVICE_CHECK: a kernel recorded a failed device-side check (a bounded
+ * wait that ran out); reported by tq_device_status. */
+typedef enum {
+    TQ_OK = 0,
+    TQ_ERR_INVALID_ARG = 1,
+    TQ_ERR_UNSUPPORTED = 2,
+    TQ_ERR_CUDA = 3,
+    TQ_ERR_WORKSPACE = 4,
+    TQ_ERR_DEVICE_CHECK = 5
+} tq_status;
+
+/* Element type of K/V inputs and of queries. */
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
+
+/* A compressed cache: caller-owned device buffer of tq_cache_bytes() bytes,
+ * 16-byte aligned, laid out as [B][Hkv][Tcap/64] blocks (Tcap a multiple of 64).
+ * K block (64 tokens): codes 64 x 3d/8 B | signs 64 x d/8 B | ||k|| fp16 x 64 |
+ *                      gamma = ||residual|| fp16 x 64
+ * V block (64 tokens): codes 64 x 3d/8 B | ||v|| fp16 x 64
+ * Per token the 3-bit codes are 3d/32 little-endian uint32 words.  Slice s
+ * (128 coordinates) and slot t (0..3) own words 12s+3t+{0,1,2} (Wa, Wb, Wc)
+ * holding slot codes i = 0..31, where slot code i is coordinate
+ *     j = 128 s + 16 (i >> 2) + 2 t + (i & 1) + 8 ((i >> 1) & 1).
+ * Nibble k of Wa: bits 0-2 = code(i = k), bit 3 = bit 0 of code(24 + k);
+ * Wb: code(8 + k) and bit 1 of code(24 + k); Wc: code(16 + k) and bit 2 of
+ * code(24 + k).  Signs are d/32 words per token; word 4s+t holds the sign of
+ * JL row i = 2q at bit q and of row 2q+1 at bit 16+q (q = 0..15), rows mapped
+ * to indices exactly as coordinates above.  A sign bit is 1 when the
+ * projection is >= 0.  Storage: (3d + m + 32)/d bits/dim for K (4.25 at
+ * d = 128) and (3d + 16)/d for V (3.125 at d = 128). */
+typedef struct {
+    void* base;
+    int64_t B;
+    int64_t Hkv;
+    int64_t Tcap;
+} tq_cache;
+
+/* ---- constants -------------------------------------------------------- */
+
+/* Compute the method's constants on the host, with no device involved:
+ * D (d signs, +-1), S (m x d fp32, row-major, iid N(0,1)), the 8 codebook
+ * centroids (ascending) and the 7 decision boundaries (midpoints).
+ * Readings: counter-based SplitMix64 stream `seed`; D_j = -1 iff the top bit of
+ * draw j is set; S from Box-Muller on draws d+2p, d+2p+1 (cosine output to
+ * element 2p, sine output to 2p+1), rounded to fp32; centroids = the 8-level
+ * Lloyd-Max quantiser of N(0,1) (K flow step 3), scaled by 1/sqrt(d), rounded
+ * to fp16.  Any output pointer may be NULL.  Errors: INVALID_ARG (d not 128 or
+ * 256). */
+TQ_API tq_status tq_params_host(int head_dim, uint64_t seed, int8_t* D, float* S, float* centroids8,
+                         float* bounds7);
+
+/* Create a handle on the current CUDA device: computes the constants as
+ * tq_params_host does and uploads them (the only allocating call).
+ * Errors: INVALID_ARG (bad d or NULL out), CUDA. */
+TQ_API tq_status tq_init(int head_dim, uint64_t seed, tq_handle** out);
+
+/* Free the handle's device constants.  NULL is accepted. */
+TQ_API tq_status tq_destroy(tq_handle* h);
+
+/* Copy the handle's constants to host arrays (any may be NULL); synchronous. */
+TQ_API tq_status tq_get_params(const tq_handle* h, int8_t* D, float* S, float* centroids8,
+                        float* bounds7);
+
+TQ_API int tq_head_dim(const tq_handle* h);
+
+/* ---- sizes ------------------------------------------------------------ */
+
+/* Bytes of one 64-token block; 0 for an unsupported d. */
+TQ_API size_t tq_block_bytes(int head_dim, int is_k);
+
+/* Bytes of a cache [B][Hkv][Tcap/64 blocks]; 0 if Tcap is not a positive
+ * multiple of 64 or d is unsupported. */
+TQ_API size_t tq_cache_bytes(int head_dim, int is_k, int64_t B, int64_t Hkv, int64_t Tcap);
+
+/* ---- encode (K flow steps 1-5 / V steps 1-3) --------------------------- */
+
+/* Encode Tnew new vectors per (batch, kv head) into token positions
+ * [t0, t0 + Tnew) of the cache.  x is a device tensor of `dtype` with element
+ * strides (sb, sh, st) for (batch, head, token) and a contiguous last
+ * dimension of d elements: vector (b, h, t) starts at x + b*sb + h*sh + t*st.
+ * Each vector is normalised (n = ||x||, stored as fp16), rotated, quantised
+ * to 3-bit codes against the boundaries (a coordinate equal to a boundary
+ * takes the upper cell), and for K the residual's norm gamma (fp16) and the
+ * sign bits of S * residual are stored.  A zero vector stores code 4, gamma 0,
+ * all signs 1.  Tokens outside [t0, t0+Tnew) are not touched.
+ * Errors: INVALID_ARG (NULL pointers, B/Hkv mismatch with the cache, Tnew < 0,
+ * t0 < 0, t0 + Tnew > Tcap, misaligned x or cache), CUDA. */
+TQ_API tq_status tq_encode_k(const tq_handle* h, const void* x, tq_dtype dtype, int64_t B, int64_t Hkv,
+                      int64_t Tnew, int64_t sb, int64_t sh, int64_t st, const tq_cache* kc,
+                      int64_t t0, void* stream);
+TQ_API tq_status tq_encode_v(const tq_handle* h, const void* x, tq_dtype dtype, int64_t B, int64_t Hkv,
+                      int64_t Tnew, int64_t sb, int64_t sh, int64_t st, const tq_cache* vc,
+                      int64_t t0, void* stream);
+
+/* ---- decode attention --------------------------------------------------- */
+
+/* Workspace bytes tq_attend_decode needs for these sizes on this handle's
+ * device (query rotation, per-split softmax partials).  0 on bad arguments. */
+TQ_API size_t tq_attend_workspace_bytes(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv,
+                                 int64_t Tmax);
+
+/* One decode step of attention for B x Hq queries (q [B][Hq][d] contiguous,
+ * `qdtype`) over the compressed caches kc (K) and vc (V).  Query head h uses
+ * kv head h / (Hq/Hkv).  Sequence b attends over tokens [0, seq_lens[b]) when
+ * seq_lens (device int32[B]) is not NULL, else over [0, T).  Computes, per
+ * query head, q' = H D q, u = S q' and
+ *   s_t = scale * n_t * (<q', c[idx_t]> + gamma_t * sqrt(pi/2)/m * <u, 2 sigma_t - 1>),
+ *   out = D H sum_t softmax(s)_t * nv_t * c[idxv_t],
+ * with n_t, gamma_t, nv_t the stored fp16 values, in fp32 with split-K
+ * (flash-decoding) partials in `ws` merged by a final kernel.  out is fp32
+ * [B][Hq][d]; an empty sequence gives zeros.  Supported: d in {128, 256},
+ * Hq/Hkv in {1, 2, 4, 8}.  ws must be 256-byte aligned with at least
+ * tq_attend_workspace_bytes(h, B, Hq, Hkv, T or max seq_len) bytes.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+TQ_API tq_status tq_attend_decode(const tq_handle* h, const void* q, tq_dtype qdtype, int64_t B,
+                           int64_t Hq, const tq_cache* kc, const tq_cache* vc,
+                           const int32_t* seq_lens, int64_t T, float scale, float* out, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/* ---- diagnostics -------------------------------------------------------- */
+
+/* Synchronise `stream`, then report and clear the handle's device check word:
+ * TQ_ERR_DEVICE_CHECK if a kernel gave up a bounded wait since the last call. */
+TQ_API tq_status tq_device_status(const tq_handle* h, void* stream);
+
+/* Diagnostics: when ev_start/ev_stop (cudaEvent_t, created by the caller) are
+ * not NULL, each later tq_attend_decode records ev_start just before its
+ * split-K attention kernel and ev_stop just after it, on the call's stream, so
+ * the caller can time that kernel alone.  Pass NULLs to stop.  Not thread-safe
+ * with concurrent tq_attend_decode calls on the same handle. */
+TQ_API tq_status tq_set_decode_events(tq_handle* h, void* ev_start, void* ev_stop);
+
+/* Name of the kernel path tq_attend_decode uses for these sizes ("mma" or
+ * "simt"); static string. */
+TQ_API const char* tq_attend_path(const tq_handle* h, int64_t Hq, int64_t Hkv);
+
+TQ_API const char* tq_status_string(tq_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

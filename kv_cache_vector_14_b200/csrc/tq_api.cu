@@ -1,0 +1,300 @@
+// C ABI of libtq (declared in include/tq.h): argument validation, the handle
+// with its device constants, and the launch sequences of encode and decode.
+#include <cmath>
+#include <cstring>
+#include <new>
+
+#include "tq_internal.h"
+
+using namespace tqi;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+size_t dtype_size(tq_dtype dt) { return dt == TQ_F32 ? 4 : 2; }
+bool dtype_ok(int dt) { return dt == TQ_F32 || dt == TQ_BF16 || dt == TQ_F16; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Pick the split count for decode: among a few candidate wave counts, the one
+// that best fills the GPU (whole waves of CTAs, balanced 64-token blocks).
+int choose_nsplit(int num_sms, int ctas_per_sm, int64_t pairs, int64_t Tmax) {
+    const int64_t nblk = Tmax > 0 ? (Tmax + kBlockT - 1) / kBlockT : 1;
+    const int64_t cap = (int64_t)num_sms * ctas_per_sm;
+    int64_t best = 1;
+    double best_score = -1.0;
+    for (int w = 1; w <= 8; ++w) {
+        int64_t ns = (int64_t)llround((double)w * cap / (double)pairs);
+        if (ns < 1) ns = 1;
+        if (ns > nblk) ns = nblk;
+        const int64_t per = (nblk + ns - 1) / ns;            // blocks per split
+        const int64_t used = (nblk + per - 1) / per;         // splits that get work
+        const int64_t ctas = pairs * used;
+        const int64_t waves = (ctas + cap - 1) / cap;
+        const double fill = (double)ctas / (double)(waves * cap);
+        const double bal = (double)nblk / (double)(used * per);
+        const double score = fill * bal - 1e-3 * w;           // prefer fewer partials on ties
+        if (score > best_score + 1e-9) { best_score = score; best = ns; }
+    }
+    const int64_t per = (nblk + best - 1) / best;
+    return (int)((nblk + per - 1) / per);
+}
+
+struct DecodePlan {
+    int G = 0;
+    bool use_mma = false;
+    int nsplit = 0;
+    int64_t split_tokens = 0;
+    size_t off_qp = 0, off_up = 0, off_ml = 0, off_acc = 0, bytes = 0;
+};
+
+// Largest split count choose_nsplit can return for any T <= Tmax.
+int nsplit_upper(int num_sms, int ctas_per_sm, int64_t pairs, int64_t Tmax) {
+    const int64_t nblk = Tmax > 0 ? (Tmax + kBlockT - 1) / kBlockT : 1;
+    int64_t ns = (int64_t)llround(8.0 * num_sms * ctas_per_sm / (double)pairs) + 1;
+    return (int)(ns < nblk ? ns : nblk);
+}
+
+void layout_ws(int d, size_t BHq, int nsplit, DecodePlan* p) {
+    size_t off = 0;
+    p->off_qp = off; off = round_up(off + BHq * d * 4, 256);
+    p->off_up = off; off = round_up(off + BHq * d * 4, 256);
+    p->off_ml = off; off = round_up(off + BHq * nsplit * 2 * 4, 256);
+    p->off_acc = off; off = round_up(off + BHq * nsplit * d * 4, 256);
+    p->bytes = off;
+}
+
+bool make_plan(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t Tmax, DecodePlan* p,
+               bool upper_bound) {
+    if (!h || B < 0 || Hq <= 0 || Hkv <= 0 || Tmax < 0 || Hq % Hkv) return false;
+    const int d = h->d;
+    p->G = (int)(Hq / Hkv);
+    p->use_mma = mma_supported(d, p->G);
+    const int64_t pairs = B * Hkv > 0 ? B * Hkv : 1;
+    const int cps = decode_ctas_per_sm(p->use_mma);
+    p->nsplit = upper_bound ? nsplit_upper(h->num_sms, cps, pairs, Tmax)
+                            : choose_nsplit(h->num_sms, cps, pairs, Tmax);
+    const int64_t nblk = Tmax > 0 ? (Tmax + kBlockT - 1) / kBlockT : 1;
+    p->split_tokens = ((nblk + p->nsplit - 1) / p->nsplit) * kBlockT;
+    layout_ws(d, (size_t)(B * Hq), p->nsplit, p);
+    return true;
+}
+
+tq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
+
+bool cache_ok(const tq_handle* h, const tq_cache* c) {
+    return c && c->base && aligned(c->base, 16) && c->B >= 0 && c->Hkv > 0 && c->Tcap > 0 &&
+           c->Tcap % kBlockT == 0 && h;
+}
+
+tq_status encode_common(const tq_handle* h, const void* x, tq_dtype dt, int64_t B, int64_t Hkv, int64_t Tnew,
+                        int64_t sb, int64_t sh, int64_t st, const tq_cache* c, int64_t t0, void* stream, bool is_k) {
+    if (!h || !dtype_ok(dt) || !cache_ok(h, c)) return TQ_ERR_INVALID_ARG;
+    if (B != c->B || Hkv != c->Hkv || Tnew < 0 || t0 < 0 || t0 + Tnew > c->Tcap) return TQ_ERR_INVALID_ARG;
+    if (B == 0 || Tnew == 0) return TQ_OK;
+    if (!x || !aligned(x, dtype_size(dt)) || sb < 0 || sh < 0 || st < 0) return TQ_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
+    if (dev != h->device) return TQ_ERR_INVALID_ARG;
+    EncArgs a{};
+    a.x = x; a.sb = sb; a.sh = sh; a.st = st;
+    a.B = B; a.Hkv = Hkv; a.Tnew = Tnew; a.t0 = t0;
+    a.NB = c->Tcap / kBlockT;
+    a.cache = static_cast<uint8_t*>(c->base);
+    a.dsign = h->dsign; a.sthr = h->dSThr; a.cb = h->cb;
+    return cuda_status(launch_encode(h->d, is_k, dt, a, h->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tq_status_string(tq_status s) {
+    switch (s) {
+        case TQ_OK: return "ok";
+        case TQ_ERR_INVALID_ARG: return "invalid argument";
+        case TQ_ERR_UNSUPPORTED: return "unsupported configuration";
+        case TQ_ERR_CUDA: return "CUDA error";
+        case TQ_ERR_WORKSPACE: return "workspace too small";
+        case TQ_ERR_DEVICE_CHECK: return "device-side check failed";
+    }
+    return "unknown status";
+}
+
+tq_status tq_params_host(int head_dim, uint64_t seed, int8_t* D, float* S, float* c8, float* b7) {
+    return make_params(head_dim, seed, D, S, c8, b7) ? TQ_OK : TQ_ERR_INVALID_ARG;
+}
+
+size_t tq_block_bytes(int head_dim, int is_k) {
+    if (head_dim != 128 && head_dim != 256) return 0;
+    return (size_t)block_bytes(head_dim, is_k != 0);
+}
+
+size_t tq_cache_bytes(int head_dim, int is_k, int64_t B, int64_t Hkv, int64_t Tcap) {
+    if ((head_dim != 128 && head_dim != 256) || B < 0 || Hkv < 0 || Tcap <= 0 || Tcap % kBlockT) return 0;
+    return (size_t)(B * Hkv * (Tcap / kBlockT)) * (size_t)block_bytes(head_dim, is_k != 0);
+}
+
+tq_status tq_init(int head_dim, uint64_t seed, tq_handle** out) {
+    if (!out || (head_dim != 128 && head_dim != 256)) return TQ_ERR_INVALID_ARG;
+    *out = nullptr;
+    tq_handle* h = new (std::nothrow) tq_handle();
+    if (!h) return TQ_ERR_CUDA;
+    const int d = head_dim;
+    h->d = d;
+    h->seed = seed;
+    h->hD.resize(d);
+    h->hS.resize((size_t)d * d);
+    make_params(d, seed, h->hD.data(), h->hS.data(), h->hc, h->hb);
+    for (int k = 0; k < 8; ++k) h->cb.c[k] = h->hc[k];
+    for (int k = 0; k < 7; ++k) h->cb.b[k] = h->hb[k];
+    uint32_t lo[2] = {0, 0}, hi[2] = {0, 0};
+    for (int k = 0; k < 8; ++k) {
+        const uint16_t bits = double_to_half_bits((double)h->hc[k]);
+        lo[k >> 2] |= (uint32_t)(bits & 0xFF) << (8 * (k & 3));
+        hi[k >> 2] |= (uint32_t)(bits >> 8) << (8 * (k & 3));
+    }
+    h->cb.lut_lo[0] = lo[0]; h->cb.lut_lo[1] = lo[1];
+    h->cb.lut_hi[0] = hi[0]; h->cb.lut_hi[1] = hi[1];
+
+    std::vector<float> sign(d), st((size_t)d * d), sthr((size_t)d * d);
+    for (int j = 0; j < d; ++j) sign[j] = (float)h->hD[j];
+    for (int i = 0; i < d; ++i)
+        for (int j = 0; j < d; ++j) st[(size_t)j * d + i] = h->hS[(size_t)i * d + j];
+    const int R = d / 32;
+    for (int j = 0; j < d; ++j)
+        for (int r = 0; r < R; ++r)
+            for (int l = 0; l < 32; ++l) {
+                const int row = slot_coord(r / 4, r % 4, 2 * (l & 15) + (l >> 4));
+                sthr[((size_t)j * R + r) * 32 + l] = h->hS[(size_t)row * d + j];
+            }
+    cudaError_t e = cudaGetDevice(&h->device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
+    if (e == cudaSuccess) e = cudaMalloc(&h->dsign, sizeof(float) * d);
+    if (e == cudaSuccess) e = cudaMalloc(&h->dST, sizeof(float) * d * d);
+    if (e == cudaSuccess) e = cudaMalloc(&h->dSThr, sizeof(float) * d * d);
+    if (e == cudaSuccess) e = cudaMalloc(&h->derr, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemcpy(h->dsign, sign.data(), sizeof(float) * d, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(h->dST, st.data(), sizeof(float) * d * d, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(h->dSThr, sthr.data(), sizeof(float) * d * d, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemset(h->derr, 0, sizeof(int));
+    if (e != cudaSuccess) {
+        tq_destroy(h);
+        return TQ_ERR_CUDA;
+    }
+    *out = h;
+    return TQ_OK;
+}
+
+tq_status tq_destroy(tq_handle* h) {
+    if (!h) return TQ_OK;
+    cudaFree(h->dsign);
+    cudaFree(h->dST);
+    cudaFree(h->dSThr);
+    cudaFree(h->derr);
+    delete h;
+    return TQ_OK;
+}
+
+tq_status tq_get_params(const tq_handle* h, int8_t* D, float* S, float* c8, float* b7) {
+    if (!h) return TQ_ERR_INVALID_ARG;
+    const int d = h->d;
+    if (D) std::memcpy(D, h->hD.data(), d);
+    if (S) std::memcpy(S, h->hS.data(), sizeof(float) * d * d);
+    if (c8) std::memcpy(c8, h->hc, sizeof(h->hc));
+    if (b7) std::memcpy(b7, h->hb, sizeof(h->hb));
+    return TQ_OK;
+}
+
+int tq_head_dim(const tq_handle* h) { return h ? h->d : 0; }
+
+tq_status tq_encode_k(const tq_handle* h, const void* x, tq_dtype dt, int64_t B, int64_t Hkv, int64_t Tnew,
+                      int64_t sb, int64_t sh, int64_t st, const tq_cache* kc, int64_t t0, void* stream) {
+    return encode_common(h, x, dt, B, Hkv, Tnew, sb, sh, st, kc, t0, stream, true);
+}
+
+tq_status tq_encode_v(const tq_handle* h, const void* x, tq_dtype dt, int64_t B, int64_t Hkv, int64_t Tnew,
+                      int64_t sb, int64_t sh, int64_t st, const tq_cache* vc, int64_t t0, void* stream) {
+    return encode_common(h, x, dt, B, Hkv, Tnew, sb, sh, st, vc, t0, stream, false);
+}
+
+size_t tq_attend_workspace_bytes(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t Tmax) {
+    DecodePlan p;
+    if (!make_plan(h, B, Hq, Hkv, Tmax, &p, true)) return 0;
+    return p.bytes;
+}
+
+const char* tq_attend_path(const tq_handle* h, int64_t Hq, int64_t Hkv) {
+    if (!h || Hq <= 0 || Hkv <= 0 || Hq % Hkv) return "invalid";
+    return mma_supported(h->d, (int)(Hq / Hkv)) ? "mma" : "simt";
+}
+
+tq_status tq_attend_decode(const tq_handle* h, const void* q, tq_dtype qdt, int64_t B, int64_t Hq,
+                           const tq_cache* kc, const tq_cache* vc, const int32_t* seq_lens, int64_t T,
+                           float scale, float* out, void* ws, size_t ws_bytes, void* stream) {
+    if (!h || !dtype_ok(qdt) || !cache_ok(h, kc) || !cache_ok(h, vc)) return TQ_ERR_INVALID_ARG;
+    if (B < 0 || Hq <= 0 || kc->B != B || vc->B != B || kc->Hkv != vc->Hkv || kc->Tcap != vc->Tcap)
+        return TQ_ERR_INVALID_ARG;
+    const int64_t Hkv = kc->Hkv;
+    if (Hq % Hkv) return TQ_ERR_INVALID_ARG;
+    const int G = (int)(Hq / Hkv);
+    if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_ERR_UNSUPPORTED;
+    if (!seq_lens && (T < 0 || T > kc->Tcap)) return TQ_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
+    if (B == 0) return TQ_OK;
+    if (!q || !out || !ws || !aligned(q, dtype_size(qdt)) || !aligned(out, 16) || !aligned(ws, 256))
+        return TQ_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
+    if (dev != h->device) return TQ_ERR_INVALID_ARG;
+    const int64_t Tmax = seq_lens ? kc->Tcap : T;
+    DecodePlan p;
+    if (!make_plan(h, B, Hq, Hkv, Tmax, &p, false)) return TQ_ERR_INVALID_ARG;
+    if (ws_bytes < p.bytes) return TQ_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    DecArgs a{};
+    a.qp = reinterpret_cast<float*>(w + p.off_qp);
+    a.up = reinterpret_cast<float*>(w + p.off_up);
+    a.kc = static_cast<const uint8_t*>(kc->base);
+    a.vc = static_cast<const uint8_t*>(vc->base);
+    a.NB = kc->Tcap / kBlockT;
+    a.seq_lens = seq_lens;
+    a.T = T;
+    a.Tcap = kc->Tcap;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv;
+    a.nsplit = p.nsplit;
+    a.split_tokens = p.split_tokens;
+    a.scale_log2 = scale * kLog2e;
+    a.part_ml = reinterpret_cast<float*>(w + p.off_ml);
+    a.part_acc = reinterpret_cast<float*>(w + p.off_acc);
+    a.err = h->derr;
+    a.cb = h->cb;
+    cudaError_t e = launch_prologue(h->d, q, qdt, B * Hq, h->dsign, h->dST,
+                                    const_cast<float*>(a.qp), const_cast<float*>(a.up), s);
+    if (e == cudaSuccess && h->ev_start) e = cudaEventRecord(h->ev_start, s);
+    if (e == cudaSuccess) e = launch_decode(h->d, G, p.use_mma, a, s);
+    if (e == cudaSuccess && h->ev_stop) e = cudaEventRecord(h->ev_stop, s);
+    if (e == cudaSuccess) e = launch_combine(h->d, B * Hq, p.nsplit, a.part_ml, a.part_acc, h->dsign, out, s);
+    return cuda_status(e);
+}
+
+tq_status tq_set_decode_events(tq_handle* h, void* ev_start, void* ev_stop) {
+    if (!h || (ev_start == nullptr) != (ev_stop == nullptr)) return TQ_ERR_INVALID_ARG;
+    h->ev_start = static_cast<cudaEvent_t>(ev_start);
+    h->ev_stop = static_cast<cudaEvent_t>(ev_stop);
+    return TQ_OK;
+}
+
+tq_status tq_device_status(const tq_handle* h, void* stream) {
+    if (!h) return TQ_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TQ_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, h->derr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TQ_ERR_CUDA;
+    if (v != 0) {
+        if (cudaMemset(h->derr, 0, sizeof(int)) != cudaSuccess) return TQ_ERR_CUDA;
+        return TQ_ERR_DEVICE_CHECK;
+    }
+    return TQ_OK;
+}
+
+}  // extern "C"

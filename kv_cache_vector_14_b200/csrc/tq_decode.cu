@@ -1,0 +1,309 @@
+// Decode attention over the packed TurboQuant cache, for sm_100a.
+//
+// Page "Apple Silicon向けSwiftLM、TurboQuant KVキャッシュ圧縮とSSD Expert
+// Streamingを実装" (ai-heartland.com): hybrid V2+V3 section (dequantisation fused
+// into the attention kernel), K section (the QJL bit corrects inner-product
+// scores), V section (V carries no QJL bit).  Per query head, with
+// q' = H D q and u = S q':
+//   s_t = scale * n_t * (<q', c[idx_t]> + gamma_t * sqrt(pi/2)/m * <u, 2 sigma_t - 1>)
+//   out = D H sum_t softmax(s)_t * nv_t * c[idxv_t]
+// Three kernels: the query prologue (q', u), split-K attention over token
+// ranges writing (max, sum, rotated accumulator) partials, and the combine
+// kernel (log-sum-exp merge, one inverse transform per head).
+#include "tq_internal.h"
+
+namespace tqi {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+template <int DT>
+__device__ __forceinline__ float load_q(const void* p, int64_t i) {
+    if constexpr (DT == TQ_F32) return __ldg(static_cast<const float*>(p) + i);
+    else if constexpr (DT == TQ_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+    else return __half2float(static_cast<const __half*>(p)[i]);
+}
+
+// In-place unnormalised Walsh-Hadamard butterflies of NH vectors [NH][D] in
+// shared memory, D threads; caller synchronises before and after.
+template <int D, int NH>
+__device__ void smem_fwht(float* v) {
+    const int j = threadIdx.x;
+#pragma unroll 1
+    for (int h = 1; h < D; h <<= 1) {
+        if ((j & h) == 0) {
+#pragma unroll
+            for (int k = 0; k < NH; ++k) {
+                const float a = v[k * D + j], b = v[k * D + j + h];
+                v[k * D + j] = a + b;
+                v[k * D + j + h] = a - b;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------- prologue
+// q' = H D q / sqrt(d) and up = sqrt(pi/2)/m * S q' for QH query heads per CTA.
+constexpr int kQH = 8;
+
+template <int D, int DT>
+__global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t BHq, const float* dsign,
+                                                        const float* ST, float* qp, float* up) {
+    __shared__ float v[kQH * D];
+    const int j = threadIdx.x;
+    const int64_t h0 = (int64_t)blockIdx.x * kQH;
+    const float ds = dsign[j];
+#pragma unroll
+    for (int k = 0; k < kQH; ++k) {
+        const int64_t h = h0 + k;
+        v[k * D + j] = (h < BHq) ? ds * load_q<DT>(q, h * D + j) : 0.f;
+    }
+    __syncthreads();
+    smem_fwht<D, kQH>(v);
+    const float inv = 1.0f / sqrtf((float)D);
+#pragma unroll
+    for (int k = 0; k < kQH; ++k) v[k * D + j] *= inv;
+    __syncthreads();
+    float u[kQH];
+#pragma unroll
+    for (int k = 0; k < kQH; ++k) u[k] = 0.f;
+    for (int jj = 0; jj < D; ++jj) {
+        const float s = __ldg(ST + (size_t)jj * D + j);   // S[j][jj], coalesced over j
+#pragma unroll
+        for (int k = 0; k < kQH; ++k) u[k] = fmaf(s, v[k * D + jj], u[k]);
+    }
+    const float cq = 1.2533141373155003f / (float)D;       // sqrt(pi/2) / m
+#pragma unroll
+    for (int k = 0; k < kQH; ++k) {
+        const int64_t h = h0 + k;
+        if (h < BHq) {
+            qp[h * D + j] = v[k * D + j];
+            up[h * D + j] = cq * u[k];
+        }
+    }
+}
+
+// ---------------------------------------------------------------- SIMT decode
+// One CTA (4 warps) per (split, kv head, batch).  Each warp walks a quarter of
+// the split's token range one token at a time; lane l owns coordinates
+// j = l + 32 r.  Partial scores are reduced across the warp, the online
+// softmax runs in log2 units, and the four warps are merged through shared
+// memory into one partial per query head.
+__device__ __forceinline__ int code_from_words(const uint32_t* w, int j) {
+    const int s = j >> 7, t = slot_of(j), i = slot_pos(j);
+    const uint32_t* W = w + 12 * s + 3 * t;
+    if (i < 24) return (int)((W[i >> 3] >> (4 * (i & 7))) & 7u);
+    const int k = i - 24;
+    return (int)(((W[0] >> (4 * k + 3)) & 1u) | (((W[1] >> (4 * k + 3)) & 1u) << 1) |
+                 (((W[2] >> (4 * k + 3)) & 1u) << 2));
+}
+__device__ __forceinline__ int sign_from_words(const uint32_t* w, int j) {
+    const int s = j >> 7, t = slot_of(j), i = slot_pos(j);
+    const int bit = (i & 1) ? 16 + (i >> 1) : (i >> 1);
+    return (int)((w[4 * s + t] >> bit) & 1u);
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
+    constexpr int R = D / 32;
+    __shared__ float sC[8];
+    __shared__ float sm[4][G][2];
+    __shared__ float sacc[4][G][D];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int split = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
+    if (threadIdx.x < 8) sC[threadIdx.x] = a.cb.c[threadIdx.x];
+
+    int64_t Tb = a.seq_lens ? (int64_t)a.seq_lens[b] : a.T;
+    Tb = Tb < 0 ? 0 : (Tb > a.Tcap ? a.Tcap : Tb);
+    const int64_t s0 = (int64_t)split * a.split_tokens;
+    const int64_t s1 = (s0 + a.split_tokens < Tb) ? s0 + a.split_tokens : Tb;
+    const int64_t len = s1 > s0 ? s1 - s0 : 0;
+    const int64_t per = (len + 3) / 4;
+    const int64_t w0 = s0 + warp * per;
+    const int64_t w1 = (w0 + per < s1) ? w0 + per : s1;
+
+    const int64_t seq = (int64_t)b * a.Hkv + hkv;
+    const int64_t kbb = block_bytes(D, true), vbb = block_bytes(D, false);
+    float q[G][R], u[G][R], acc[G][R], mrun[G], lrun[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        const int64_t bh = (int64_t)b * a.Hq + (int64_t)hkv * G + g;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            q[g][r] = a.qp[bh * D + lane + 32 * r];
+            u[g][r] = a.up[bh * D + lane + 32 * r];
+            acc[g][r] = 0.f;
+        }
+        mrun[g] = -INFINITY;
+        lrun[g] = 0.f;
+    }
+    __syncthreads();
+
+    for (int64_t t = w0; t < w1; ++t) {
+        const uint8_t* kb = a.kc + (seq * a.NB + (t >> 6)) * kbb;
+        const uint8_t* vb = a.vc + (seq * a.NB + (t >> 6)) * vbb;
+        const int tau = (int)(t & 63);
+        const uint32_t* kw = reinterpret_cast<const uint32_t*>(kb + tau * code_bytes(D));
+        const uint32_t* sw = reinterpret_cast<const uint32_t*>(kb + kBlockT * code_bytes(D) + tau * sign_bytes(D));
+        const uint32_t* vw = reinterpret_cast<const uint32_t*>(vb + tau * code_bytes(D));
+        const float nk = __half2float(reinterpret_cast<const __half*>(kb + kBlockT * (code_bytes(D) + sign_bytes(D)))[tau]);
+        const float gk = __half2float(reinterpret_cast<const __half*>(kb + kBlockT * (code_bytes(D) + sign_bytes(D)) + 2 * kBlockT)[tau]);
+        const float nv = __half2float(reinterpret_cast<const __half*>(vb + kBlockT * code_bytes(D))[tau]);
+        float part[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) part[g] = 0.f;
+        float cv[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int j = lane + 32 * r;
+            const float ck = sC[code_from_words(kw, j)];
+            const float sg = sign_from_words(sw, j) ? gk : -gk;
+            cv[r] = sC[code_from_words(vw, j)];
+#pragma unroll
+            for (int g = 0; g < G; ++g) part[g] = fmaf(q[g][r], ck, fmaf(u[g][r], sg, part[g]));
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) part[g] += __shfl_xor_sync(kFull, part[g], o);
+            const float s = a.scale_log2 * nk * part[g];
+            const float mnew = fmaxf(mrun[g], s);
+            const float corr = exp2f(mrun[g] - mnew);
+            const float p = exp2f(s - mnew);
+            lrun[g] = lrun[g] * corr + p;
+            const float pv = p * nv;
+#pragma unroll
+            for (int r = 0; r < R; ++r) acc[g][r] = fmaf(pv, cv[r], acc[g][r] * corr);
+            mrun[g] = mnew;
+        }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        if (lane == 0) { sm[warp][g][0] = mrun[g]; sm[warp][g][1] = lrun[g]; }
+#pragma unroll
+        for (int r = 0; r < R; ++r) sacc[warp][g][lane + 32 * r] = acc[g][r];
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * D; idx += 128) {
+        const int g = idx / D, j = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, sm[w][g][0]);
+        float L = 0.f, A = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float f = exp2f(sm[w][g][0] - M);   // empty warps: exp2(-inf) = 0
+                L = fmaf(f, sm[w][g][1], L);
+                A = fmaf(f, sacc[w][g][j], A);
+            }
+        }
+        const int64_t bh = (int64_t)b * a.Hq + (int64_t)hkv * G + g;
+        const int64_t pidx = bh * a.nsplit + split;
+        a.part_acc[pidx * D + j] = A;
+        if (j == 0) { a.part_ml[2 * pidx] = M; a.part_ml[2 * pidx + 1] = L; }
+    }
+}
+
+// ---------------------------------------------------------------- combine
+// One CTA of D threads per (batch, query head): log-sum-exp merge of the
+// split partials, division by the softmax sum, one inverse transform D H.
+template <int D>
+__global__ void __launch_bounds__(D) tq_combine_kernel(const float* part_ml, const float* part_acc, int nsplit,
+                                                       const float* dsign, float* out) {
+    __shared__ float v[D];
+    const int j = threadIdx.x;
+    const int64_t bh = blockIdx.x;
+    const float* ml = part_ml + bh * nsplit * 2;
+    float M = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, ml[2 * s]);
+    float L = 0.f, A = 0.f;
+    if (M != -INFINITY) {
+        for (int s = 0; s < nsplit; ++s) {
+            const float f = exp2f(ml[2 * s] - M);
+            L = fmaf(f, ml[2 * s + 1], L);
+            A = fmaf(f, part_acc[(bh * nsplit + s) * D + j], A);
+        }
+    }
+    v[j] = (L > 0.f) ? A / L : 0.f;
+    __syncthreads();
+    smem_fwht<D, 1>(v);
+    out[bh * D + j] = dsign[j] * v[j] * (1.0f / sqrtf((float)D));
+}
+
+template <int D>
+cudaError_t launch_prologue_d(const void* q, tq_dtype dt, int64_t BHq, const float* dsign, const float* st,
+                              float* qp, float* up, cudaStream_t s) {
+    const int grid = (int)((BHq + kQH - 1) / kQH);
+    if (grid == 0) return cudaSuccess;
+    switch (dt) {
+        case TQ_F32: tq_prologue_kernel<D, TQ_F32><<<grid, D, 0, s>>>(q, BHq, dsign, st, qp, up); break;
+        case TQ_BF16: tq_prologue_kernel<D, TQ_BF16><<<grid, D, 0, s>>>(q, BHq, dsign, st, qp, up); break;
+        case TQ_F16: tq_prologue_kernel<D, TQ_F16><<<grid, D, 0, s>>>(q, BHq, dsign, st, qp, up); break;
+    }
+    return cudaGetLastError();
+}
+
+template <int D, int G>
+cudaError_t launch_simt(const DecArgs& a, cudaStream_t s) {
+    dim3 grid(a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
+    tq_decode_simt_kernel<D, G><<<grid, 128, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_simt_g(int G, const DecArgs& a, cudaStream_t s) {
+    switch (G) {
+        case 1: return launch_simt<D, 1>(a, s);
+        case 2: return launch_simt<D, 2>(a, s);
+        case 4: return launch_simt<D, 4>(a, s);
+        case 8: return launch_simt<D, 8>(a, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, const float* dsign, const float* st,
+                            float* qp, float* up, cudaStream_t s) {
+    if (d == 128) return launch_prologue_d<128>(q, dt, BHq, dsign, st, qp, up, s);
+    if (d == 256) return launch_prologue_d<256>(q, dt, BHq, dsign, st, qp, up, s);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_simt(int d, int G, const DecArgs& a, cudaStream_t s) {
+    if (a.B * a.Hkv == 0) return cudaSuccess;
+    if (d == 128) return launch_simt_g<128>(G, a, s);
+    if (d == 256) return launch_simt_g<256>(G, a, s);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml, const float* part_acc,
+                           const float* dsign, float* out, cudaStream_t s) {
+    if (BHq == 0) return cudaSuccess;
+    if (d == 128) tq_combine_kernel<128><<<(unsigned)BHq, 128, 0, s>>>(part_ml, part_acc, nsplit, dsign, out);
+    else if (d == 256) tq_combine_kernel<256><<<(unsigned)BHq, 256, 0, s>>>(part_ml, part_acc, nsplit, dsign, out);
+    else return cudaErrorInvalidValue;
+    return cudaGetLastError();
+}
+
+}  // namespace tqi
+
+namespace tqi {
+
+cudaError_t launch_decode_simt(int d, int G, const DecArgs& a, cudaStream_t s);
+
+bool mma_supported(int d, int G) {
+    (void)d; (void)G;
+    return false;
+}
+
+int decode_ctas_per_sm(bool use_mma) { return use_mma ? 1 : 4; }
+
+cudaError_t launch_decode(int d, int G, bool use_mma, const DecArgs& a, cudaStream_t s) {
+    (void)use_mma;
+    return launch_decode_simt(d, G, a, s);
+}
+
+}  // namespace tqi

@@ -1,0 +1,273 @@
+// TurboQuant K/V encode kernels for sm_100a.
+//
+// Page "Apple Silicon向けSwiftLM、TurboQuant KVキャッシュ圧縮とSSD Expert
+// Streamingを実装" (ai-heartland.com), section "K-Cache圧縮：3-bit PolarQuant +
+// 1-bit QJL = 4.25 bits/dim" (steps 1-5) and section "V-Cache圧縮：3-bit
+// PolarQuant = 3.125 bits/dim" (steps 1-3, no QJL).
+//
+// One CTA of 8 warps handles tiles of 32 vectors (4 per warp):
+//   phase 1, one warp per vector: coalesced load, ||x|| by warp reduction,
+//     sign flip + Walsh-Hadamard butterflies (register stages for the lane's
+//     own coordinates j = lane + 32 r, shuffle stages across lanes), scale by
+//     1 / (||x|| sqrt(d)), bucketize against the 7 boundaries, residual and
+//     its norm gamma (K).  Codes are staged in shared memory in slot order.
+//   phase 2 (K only): the JL projection Z = R S^T of the tile as an fp32
+//     contraction from shared memory, each lane owning the JL rows whose sign
+//     bits form one packed word, so one ballot yields each stored word.
+//   phase 3: the staged codes are packed into the nibble words of the layout
+//     and stored with coalesced 4-byte stores.
+#include "tq_internal.h"
+
+namespace tqi {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr int kThreads = 256;
+constexpr int kTileV = 32;                  // vectors per tile
+constexpr int kVecPerWarp = kTileV / 8;
+
+template <int DT>
+__device__ __forceinline__ float load_x(const void* p, int64_t i) {
+    if constexpr (DT == TQ_F32) return __ldg(static_cast<const float*>(p) + i);
+    else if constexpr (DT == TQ_BF16)
+        return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+    else return __half2float(static_cast<const __half*>(p)[i]);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
+// Pack 8 byte-sized values (< 16) held in two words into 8 nibbles.
+__device__ __forceinline__ uint32_t nibbles8(uint32_t lo4, uint32_t hi4) {
+    uint32_t a = (lo4 | (lo4 >> 4)) & 0x00FF00FFu;
+    a = (a | (a >> 8)) & 0x0000FFFFu;
+    uint32_t b = (hi4 | (hi4 >> 4)) & 0x00FF00FFu;
+    b = (b | (b >> 8)) & 0x0000FFFFu;
+    return a | (b << 16);
+}
+
+template <int D, bool IS_K>
+struct EncSmem {
+    static constexpr int R = D / 32;
+    static constexpr int JC = (D == 128) ? 128 : 64;           // JL columns resident at once
+    static constexpr size_t s_bytes = IS_K ? (size_t)JC * D * 4 : 0;
+    static constexpr size_t r_bytes = IS_K ? (size_t)kTileV * D * 4 : 0;
+    static constexpr size_t code_bytes = (size_t)kTileV * D;
+    static constexpr size_t total = s_bytes + r_bytes + code_bytes;
+};
+
+template <int D, bool IS_K, int DT>
+__global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
+    using SM = EncSmem<D, IS_K>;
+    constexpr int R = SM::R;
+    constexpr int JC = SM::JC;
+    extern __shared__ __align__(16) unsigned char smem[];
+    float* sS = reinterpret_cast<float*>(smem);                        // [JC][R][32]
+    float* sR = reinterpret_cast<float*>(smem + SM::s_bytes);          // [kTileV][D]
+    uint8_t* sCode = smem + SM::s_bytes + SM::r_bytes;                 // [kTileV][D], slot order
+    __shared__ float sC[8];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t N = a.B * a.Hkv * a.Tnew;
+    const int64_t ntiles = (N + kTileV - 1) / kTileV;
+    const int64_t bb = block_bytes(D, IS_K);
+    const float sqrt_d = sqrtf((float)D);
+
+    if (threadIdx.x < 8) sC[threadIdx.x] = a.cb.c[threadIdx.x];
+    float dsg[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) dsg[r] = __ldg(a.dsign + lane + 32 * r);
+    if constexpr (IS_K && D == 128) {
+        for (int i = threadIdx.x; i < JC * D / 4; i += kThreads)
+            reinterpret_cast<float4*>(sS)[i] = __ldg(reinterpret_cast<const float4*>(a.sthr) + i);
+    }
+    __syncthreads();
+
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        // ---------------- phase 1: one warp per vector
+        for (int vv = 0; vv < kVecPerWarp; ++vv) {
+            const int v = warp * kVecPerWarp + vv;
+            const int64_t gv = tile * kTileV + v;
+            const bool valid = gv < N;
+            float x[R];
+            float ss = 0.f;
+            int64_t tt = 0, bh = 0;
+            if (valid) {
+                tt = gv % a.Tnew;
+                bh = gv / a.Tnew;
+                const int64_t h = bh % a.Hkv, b = bh / a.Hkv;
+                const int64_t base = b * a.sb + h * a.sh + tt * a.st;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    x[r] = load_x<DT>(a.x, base + lane + 32 * r);
+                    ss = fmaf(x[r], x[r], ss);
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < R; ++r) x[r] = 0.f;
+            }
+            ss = warp_sum(ss);
+            const float n = sqrtf(ss);
+#pragma unroll
+            for (int r = 0; r < R; ++r) x[r] *= dsg[r];
+            // butterflies over lane bits (coordinate bits 0..4)
+#pragma unroll
+            for (int hb = 1; hb < 32; hb <<= 1) {
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const float p = __shfl_xor_sync(kFull, x[r], hb);
+                    x[r] = (lane & hb) ? (p - x[r]) : (x[r] + p);
+                }
+            }
+            // butterflies over register bits (coordinate bits 5..)
+#pragma unroll
+            for (int hb = 1; hb < R; hb <<= 1) {
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    if ((r & hb) == 0) {
+                        const float u = x[r], w = x[r | hb];
+                        x[r] = u + w;
+                        x[r | hb] = u - w;
+                    }
+                }
+            }
+            const float nsd = n * sqrt_d;
+            float g2 = 0.f;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int j = lane + 32 * r;
+                const float y = (n > 0.f) ? __fdiv_rn(x[r], nsd) : 0.f;
+                int code = 0;
+#pragma unroll
+                for (int i = 0; i < 7; ++i) code += (y >= a.cb.b[i]) ? 1 : 0;
+                const float res = (n > 0.f) ? (y - sC[code]) : 0.f;
+                g2 = fmaf(res, res, g2);
+                if constexpr (IS_K) sR[v * D + j] = res;
+                sCode[v * D + (j >> 7) * 128 + slot_of(j) * 32 + slot_pos(j)] = (uint8_t)code;
+            }
+            if constexpr (IS_K) g2 = warp_sum(g2);
+            if (valid && lane == 0) {
+                const int64_t t = a.t0 + tt;
+                uint8_t* blk = a.cache + (bh * a.NB + (t >> 6)) * bb;
+                const int tau = (int)(t & 63);
+                const int64_t norm_off = kBlockT * code_bytes(D) + (IS_K ? kBlockT * sign_bytes(D) : 0);
+                reinterpret_cast<__half*>(blk + norm_off)[tau] = __float2half_rn(n);
+                if constexpr (IS_K)
+                    reinterpret_cast<__half*>(blk + norm_off + 2 * kBlockT)[tau] = __float2half_rn(sqrtf(g2));
+            }
+        }
+        __syncthreads();
+
+        // ---------------- phase 2 (K): z = S r for the tile, signs by ballot
+        if constexpr (IS_K) {
+            float z[kVecPerWarp][R];
+#pragma unroll
+            for (int vv = 0; vv < kVecPerWarp; ++vv)
+#pragma unroll
+                for (int r = 0; r < R; ++r) z[vv][r] = 0.f;
+            for (int j0 = 0; j0 < D; j0 += JC) {
+                if constexpr (D != 128) {
+                    __syncthreads();
+                    const float4* src = reinterpret_cast<const float4*>(a.sthr + (size_t)j0 * D);
+                    for (int i = threadIdx.x; i < JC * D / 4; i += kThreads)
+                        reinterpret_cast<float4*>(sS)[i] = __ldg(src + i);
+                    __syncthreads();
+                }
+#pragma unroll 2
+                for (int jj = 0; jj < JC; jj += 4) {
+                    float4 rv[kVecPerWarp];
+#pragma unroll
+                    for (int vv = 0; vv < kVecPerWarp; ++vv)
+                        rv[vv] = *reinterpret_cast<const float4*>(sR + (warp * kVecPerWarp + vv) * D + j0 + jj);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                        for (int r = 0; r < R; ++r) {
+                            const float s = sS[((jj + q) * R + r) * 32 + lane];
+#pragma unroll
+                            for (int vv = 0; vv < kVecPerWarp; ++vv) {
+                                const float rq = (q == 0) ? rv[vv].x : (q == 1) ? rv[vv].y : (q == 2) ? rv[vv].z : rv[vv].w;
+                                z[vv][r] = fmaf(rq, s, z[vv][r]);
+                            }
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int vv = 0; vv < kVecPerWarp; ++vv) {
+                const int64_t gv = tile * kTileV + warp * kVecPerWarp + vv;
+                uint32_t mine = 0;
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const uint32_t w = __ballot_sync(kFull, z[vv][r] >= 0.f);
+                    if (lane == r) mine = w;
+                }
+                if (gv < N && lane < R) {
+                    const int64_t tt = gv % a.Tnew, bh = gv / a.Tnew, t = a.t0 + tt;
+                    uint8_t* blk = a.cache + (bh * a.NB + (t >> 6)) * bb;
+                    uint32_t* sw = reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(D) +
+                                                               (t & 63) * sign_bytes(D));
+                    sw[lane] = mine;
+                }
+            }
+        }
+
+        // ---------------- phase 3: pack staged codes into the layout's words
+        constexpr int W = 3 * D / 32;
+#pragma unroll
+        for (int vv = 0; vv < kVecPerWarp; ++vv) {
+            const int v = warp * kVecPerWarp + vv;
+            const int64_t gv = tile * kTileV + v;
+            if (gv < N && lane < W) {
+                const int s = lane / 12, t = (lane % 12) / 3, g = lane % 3;
+                const uint8_t* slot = sCode + v * D + s * 128 + t * 32;
+                const uint32_t* sw = reinterpret_cast<const uint32_t*>(slot);
+                const uint32_t main = nibbles8(sw[2 * g], sw[2 * g + 1]);
+                const uint32_t tail = nibbles8(sw[6], sw[7]);
+                const uint32_t word = main | (((tail >> g) & 0x11111111u) << 3);
+                const int64_t tt = gv % a.Tnew, bh = gv / a.Tnew, tok = a.t0 + tt;
+                uint8_t* blk = a.cache + (bh * a.NB + (tok >> 6)) * bb;
+                reinterpret_cast<uint32_t*>(blk + (tok & 63) * code_bytes(D))[lane] = word;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+template <int D, bool IS_K, int DT>
+cudaError_t launch_enc_t(const EncArgs& a, int num_sms, cudaStream_t s) {
+    using SM = EncSmem<D, IS_K>;
+    auto kern = tq_encode_kernel<D, IS_K, DT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::total);
+    if (e != cudaSuccess) return e;
+    const int64_t N = a.B * a.Hkv * a.Tnew;
+    const int64_t ntiles = (N + kTileV - 1) / kTileV;
+    const int64_t cap = (int64_t)num_sms * 2;
+    const int grid = (int)(ntiles < cap ? ntiles : cap);
+    if (grid <= 0) return cudaSuccess;
+    kern<<<grid, kThreads, SM::total, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D, bool IS_K>
+cudaError_t launch_enc_dt(tq_dtype dt, const EncArgs& a, int num_sms, cudaStream_t s) {
+    switch (dt) {
+        case TQ_F32: return launch_enc_t<D, IS_K, TQ_F32>(a, num_sms, s);
+        case TQ_BF16: return launch_enc_t<D, IS_K, TQ_BF16>(a, num_sms, s);
+        case TQ_F16: return launch_enc_t<D, IS_K, TQ_F16>(a, num_sms, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, cudaStream_t s) {
+    if (d == 128) return is_k ? launch_enc_dt<128, true>(dt, a, num_sms, s) : launch_enc_dt<128, false>(dt, a, num_sms, s);
+    if (d == 256) return is_k ? launch_enc_dt<256, true>(dt, a, num_sms, s) : launch_enc_dt<256, false>(dt, a, num_sms, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace tqi

@@ -1,0 +1,108 @@
+// Internal declarations shared by the libtq translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+#define TQ_API __attribute__((visibility("default")))
+#include "tq.h"
+
+namespace tqi {
+
+constexpr int kBlockT = 64;      // tokens per cache block
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Codebook passed by value to every kernel (it lands in the constant bank).
+struct Codebook {
+    float c[8];         // centroids, ascending (fp16-exact values)
+    float b[7];         // decision boundaries (midpoints)
+    uint32_t lut_lo[2]; // low bytes of the fp16 bit patterns of c[0..7]
+    uint32_t lut_hi[2]; // high bytes of the fp16 bit patterns of c[0..7]
+};
+
+// Host-side generation of the constants (tq_params.cpp).
+bool make_params(int d, uint64_t seed, int8_t* D, float* S, float* c8, float* b7);
+uint16_t double_to_half_bits(double x);
+
+// Byte sizes of the block fields.
+__host__ __device__ inline int64_t code_bytes(int d) { return 3LL * d / 8; }          // per token
+__host__ __device__ inline int64_t sign_bytes(int d) { return (int64_t)d / 8; }       // per token
+__host__ __device__ inline int64_t block_bytes(int d, bool is_k) {
+    return kBlockT * code_bytes(d) + (is_k ? kBlockT * sign_bytes(d) + 4 * kBlockT : 2 * kBlockT);
+}
+
+// Slot order of coordinate j inside a token record: slot t (0..3) of slice
+// j >> 7 owns 32 coordinates; position i inside the slot.
+__host__ __device__ inline int slot_of(int j) { return (j >> 1) & 3; }
+__host__ __device__ inline int slot_pos(int j) {
+    int jj = j & 127;
+    return ((jj >> 4) << 2) | (((jj >> 3) & 1) << 1) | (jj & 1);
+}
+__host__ __device__ inline int slot_coord(int s, int t, int i) {
+    return 128 * s + 16 * (i >> 2) + 2 * t + (i & 1) + 8 * ((i >> 1) & 1);
+}
+
+struct EncArgs {
+    const void* x;
+    int64_t sb, sh, st;
+    int64_t B, Hkv, Tnew, t0;
+    int64_t NB;               // blocks per sequence (Tcap / 64)
+    uint8_t* cache;
+    const float* dsign;       // [d] +-1
+    const float* sthr;        // [d][d/32][32] JL matrix, encode lane order
+    Codebook cb;
+};
+
+struct DecArgs {
+    const float* qp;          // [B*Hq][d] rotated queries q' = H D q
+    const float* up;          // [B*Hq][d] sqrt(pi/2)/m * S q'
+    const uint8_t* kc;
+    const uint8_t* vc;
+    int64_t NB;               // blocks per sequence
+    const int32_t* seq_lens;  // device or null
+    int64_t T;                // used when seq_lens is null
+    int64_t Tcap;
+    int64_t B, Hq, Hkv;
+    int nsplit;
+    int64_t split_tokens;     // tokens per split, multiple of 64
+    float scale_log2;         // softmax scale * log2(e)
+    float* part_ml;           // [B*Hq][nsplit][2] (running max in log2 units, sum)
+    float* part_acc;          // [B*Hq][nsplit][d] rotated-domain accumulators
+    int* err;                 // device check word
+    Codebook cb;
+};
+
+// Kernel launchers (tq_encode.cu, tq_decode.cu); return a CUDA error code.
+cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms,
+                          cudaStream_t s);
+cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, const float* dsign,
+                            const float* st, float* qp, float* up, cudaStream_t s);
+cudaError_t launch_decode(int d, int G, bool use_mma, const DecArgs& a, cudaStream_t s);
+cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml,
+                           const float* part_acc, const float* dsign, float* out, cudaStream_t s);
+bool mma_supported(int d, int G);
+int decode_ctas_per_sm(bool use_mma);
+
+}  // namespace tqi
+
+struct tq_handle {
+    int d = 0;
+    uint64_t seed = 0;
+    int device = -1;
+    int num_sms = 0;
+    std::vector<int8_t> hD;
+    std::vector<float> hS;    // [m][d]
+    float hc[8] = {};
+    float hb[7] = {};
+    float* dsign = nullptr;   // [d]
+    float* dST = nullptr;     // [d][m] transposed S (query prologue)
+    float* dSThr = nullptr;   // [d][d/32][32] encode lane order
+    int* derr = nullptr;
+    tqi::Codebook cb{};
+    cudaEvent_t ev_start = nullptr;   // optional timing of the split-K kernel
+    cudaEvent_t ev_stop = nullptr;
+};

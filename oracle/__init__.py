@@ -60,6 +60,8 @@ def _L():
             lib.orc_fwht.argtypes = [P, C.c_int]
             lib.orc_encode.restype = None
             lib.orc_encode.argtypes = [C.c_int, P, P, P, P, P, i64, C.c_int, P, P, P, P, P, P]
+            lib.orc_sketch_given_codes.restype = None
+            lib.orc_sketch_given_codes.argtypes = [C.c_int, P, P, P, P, P, i64, P, P, P]
             lib.orc_block_bytes.restype = i64
             lib.orc_block_bytes.argtypes = [C.c_int, C.c_int]
             lib.orc_pack.restype = None
@@ -154,6 +156,21 @@ def encode(x, prm: dict, with_qjl: bool) -> dict:
     if with_qjl:
         out.update(sig=sig, gamma=g, gh=to_fp16_bits(g), z=z)
     return out
+
+
+def sketch_given_codes(prm: dict, y, idx, nonzero) -> dict:
+    """Residual norm and JL signs of rows y ([N, d]) quantised to the given codes."""
+    d = prm["d"]
+    y = np.ascontiguousarray(y, dtype=np.float64).reshape(-1, d)
+    idx = np.ascontiguousarray(idx, dtype=np.uint8).reshape(-1, d)
+    nz = np.ascontiguousarray(nonzero, dtype=np.uint8).reshape(-1)
+    N = y.shape[0]
+    sig = np.zeros((N, d), dtype=np.uint8)
+    g = np.zeros(N, dtype=np.float64)
+    z = np.zeros((N, d), dtype=np.float64)
+    _L().orc_sketch_given_codes(d, _p(prm["S"]), _p(prm["c8"]), _p(y), _p(idx), _p(nz), N,
+                                _p(sig), _p(g), _p(z))
+    return {"sig": sig, "gamma": g, "gh": to_fp16_bits(g), "z": z}
 
 
 def block_bytes(d: int, is_k: bool) -> int:

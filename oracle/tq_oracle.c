@@ -182,43 +182,65 @@ void orc_fwht(double* v, int d) {
  * y and z are returned for the boundary-window accounting of the tests.
  * with_qjl = 0 gives the V path (sig, gam and z untouched).
  * ---------------------------------------------------------------------- */
+/* Steps 4-5 for one vector whose codes are given: r = y - c[idx] (r = 0 for a
+ * zero input), gamma = ||r||, z = S r, sigma_i = [z_i >= 0]. */
+static void orc_residual_sketch(int d, const double* S, const double* c8, const double* y,
+                                const uint8_t* idx, int nonzero, uint8_t* sig, double* gam,
+                                double* z_out) {
+    const int m = d;
+    double* r = (double*)malloc(sizeof(double) * (size_t)d);
+    double g2 = 0.0;
+    for (int j = 0; j < d; ++j) {
+        r[j] = nonzero ? y[j] - c8[idx[j]] : 0.0;
+        g2 += r[j] * r[j];
+    }
+    *gam = sqrt(g2);
+    for (int i = 0; i < m; ++i) {
+        double z = 0.0;
+        for (int j = 0; j < d; ++j) z += S[(size_t)i * d + j] * r[j];
+        sig[i] = (z >= 0.0) ? 1 : 0;
+        if (z_out) z_out[i] = z;
+    }
+    free(r);
+}
+
 void orc_encode(int d, const int8_t* D, const double* S, const double* c8, const double* b7,
                 const double* x, int64_t N, int with_qjl,
                 uint8_t* idx, uint8_t* sig, double* nrm, double* gam,
                 double* y_out, double* z_out) {
-    const int m = d;
 #pragma omp parallel for schedule(static)
     for (int64_t v = 0; v < N; ++v) {
         const double* xv = x + v * d;
         double* y = (double*)malloc(sizeof(double) * (size_t)d);
-        double* r = (double*)malloc(sizeof(double) * (size_t)d);
         double ss = 0.0;
         for (int j = 0; j < d; ++j) ss += xv[j] * xv[j];
-        double n = sqrt(ss);
+        double n = sqrt(ss);                                   /* step 1 */
         nrm[v] = n;
         for (int j = 0; j < d; ++j) y[j] = (n > 0.0) ? D[j] * (xv[j] / n) : 0.0;
-        orc_fwht(y, d);
-        double g2 = 0.0;
-        for (int j = 0; j < d; ++j) {
+        orc_fwht(y, d);                                        /* step 2 */
+        for (int j = 0; j < d; ++j) {                          /* step 3 */
             int k = 0;
             for (int i = 0; i < 7; ++i) k += (b7[i] <= y[j]) ? 1 : 0;
             idx[v * d + j] = (uint8_t)k;
-            r[j] = (n > 0.0) ? y[j] - c8[k] : 0.0;
-            g2 += r[j] * r[j];
             if (y_out) y_out[v * d + j] = y[j];
         }
-        if (with_qjl) {
-            gam[v] = sqrt(g2);
-            for (int i = 0; i < m; ++i) {
-                double z = 0.0;
-                for (int j = 0; j < d; ++j) z += S[(size_t)i * d + j] * r[j];
-                sig[v * m + i] = (z >= 0.0) ? 1 : 0;
-                if (z_out) z_out[v * m + i] = z;
-            }
-        }
+        if (with_qjl)                                          /* steps 4-5 */
+            orc_residual_sketch(d, S, c8, y, idx + v * d, n > 0.0, sig + v * d, &gam[v],
+                                z_out ? z_out + v * d : NULL);
         free(y);
-        free(r);
     }
+}
+
+/* Steps 4-5 for N vectors with y and the codes supplied (y [N][d], idx [N][d],
+ * nonzero [N]): lets a test compare sign bits where the two sides took a
+ * different code decision inside the boundary window. */
+void orc_sketch_given_codes(int d, const double* S, const double* c8, const double* y,
+                            const uint8_t* idx, const uint8_t* nonzero, int64_t N,
+                            uint8_t* sig, double* gam, double* z_out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t v = 0; v < N; ++v)
+        orc_residual_sketch(d, S, c8, y + v * d, idx + v * d, nonzero[v], sig + v * d, &gam[v],
+                            z_out ? z_out + v * d : NULL);
 }
 
 /* ------------------------------------------------------------------------

@@ -25,3 +25,11 @@ def read_golden(name):
 @pytest.fixture(scope="session")
 def golden():
     return read_golden
+
+
+@pytest.fixture(scope="session")
+def libtq():
+    """Build (if stale) and load the in-tree libtq.so."""
+    from kv_cache_vector_14_b200 import build, tq
+    build.build()
+    return tq.lib()

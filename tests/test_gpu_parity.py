@@ -1,0 +1,286 @@
+"""GPU parity: the CUDA library (through its C ABI) against the float64 oracle on
+the same seeded inputs, for the five workloads and their edge cases."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from kv_cache_vector_14_b200 import synthetic, tq
+from gpu_util import (ATT_TOL, attend_gpu, check_encode, encode_gpu, oracle_attend, rel_err_rows,
+                      torch_input, unpack_cache)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def handles(libtq):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    hs = {d: tq.tq_init(d, 0) for d in (128, 256)}
+    yield hs
+    torch.cuda.synchronize()
+    for h in hs.values():
+        tq.tq_destroy(h)
+
+
+@pytest.fixture(scope="module")
+def prms():
+    return {d: O.params(d, 0) for d in (128, 256)}
+
+
+def _flat(u: dict) -> dict:
+    return {k: v.reshape((-1,) + v.shape[2:]) for k, v in u.items()}
+
+
+def _x64(x: np.ndarray) -> np.ndarray:
+    return x.astype(np.float64).reshape(-1, x.shape[-1])
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_params_on_device(handles, d):
+    p, hp = tq.tq_get_params(handles[d]), tq.tq_params_host(d, 0)
+    for k in ("D", "S", "c8", "b7"):
+        assert np.array_equal(p[k], hp[k])
+
+
+# ------------------------------------------------------------------ encode
+
+def test_encode_single_head_fp32(handles, prms):
+    w = synthetic.WORKLOADS["c1"]
+    for which in ("k", "v"):
+        x = synthetic.kv(w, which)
+        kc, vc = encode_gpu(handles[128], 128, torch_input(x, w.kv_dtype), Tcap=w.T, which=which)
+        g = _flat(unpack_cache(kc if which == "k" else vc, 0, w.T))
+        st = check_encode(prms[128], _x64(x), g if which == "k" else None, g if which == "v" else None)
+        print(which, st)
+
+
+def test_encode_bf16_8heads_32768_full(handles, prms):
+    """The encode-only workload at full size: every vector is compared."""
+    w = synthetic.WORKLOADS["c2"]
+    xk, xv = synthetic.kv(w, "k"), synthetic.kv(w, "v")
+    kc, _ = encode_gpu(handles[128], 128, torch_input(xk, "bf16"), Tcap=w.T, which="k")
+    _, vc = encode_gpu(handles[128], 128, torch_input(xv, "bf16"), Tcap=w.T, which="v")
+    print("K", check_encode(prms[128], _x64(xk), _flat(unpack_cache(kc, 0, w.T)), None))
+    print("V", check_encode(prms[128], _x64(xv), None, _flat(unpack_cache(vc, 0, w.T))))
+
+
+def test_encode_d256_sampled(handles, prms):
+    """d = 256 (append-and-attend workload's initial cache), two heads compared in full."""
+    w = synthetic.WORKLOADS["c5"]
+    x = synthetic.kv(w, "k", 0, w.T, batches=[0, 5])
+    kc, vc = encode_gpu(handles[256], 256, torch_input(x, "f32"), Tcap=w.T)
+    seqs = [(0, 0), (1, 7)]
+    gk, gv = unpack_cache(kc, 0, w.T, seqs), unpack_cache(vc, 0, w.T, seqs)
+    xs = np.stack([x[0, 0], x[1, 7]])
+    print(check_encode(prms[256], _x64(xs), _flat(gk), _flat(gv)))
+
+
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+def test_encode_ragged_offsets_strides(handles, prms, d, dtype):
+    B, Hkv, T, t0, Tcap = 2, 3, 77, 50, 192
+    base = synthetic.gaussian((B, T, Hkv, d), seed=d + len(dtype))     # [B, T, H, d]: strided heads
+    base[..., 3] *= 20.0
+    if dtype == "bf16":
+        base = synthetic.bf16_round(base)
+    elif dtype == "f16":
+        base = base.astype(np.float16).astype(np.float32)
+    xt = torch_input(base, dtype).permute(0, 2, 1, 3)                    # view [B, H, T, d]
+    assert not xt.is_contiguous()
+    kc, vc = encode_gpu(handles[d], d, xt, Tcap=Tcap, t0=t0)
+    x = base.transpose(0, 2, 1, 3)
+    print(check_encode(prms[d], _x64(x), _flat(unpack_cache(kc, t0, T)), _flat(unpack_cache(vc, t0, T))))
+    # tokens outside [t0, t0 + T) are untouched (buffers started as zeros)
+    for c in (kc, vc):
+        u = unpack_cache(c, 0, Tcap)
+        for k, v in u.items():
+            assert not np.any(v[:, :t0]) and not np.any(v[:, t0 + T:]), k
+
+
+def test_encode_zero_and_special_vectors(handles, prms):
+    d = 128
+    x = np.zeros((1, 1, 5, d), np.float32)
+    x[0, 0, 1, 7] = 3.0
+    x[0, 0, 2] = 1e-3
+    x[0, 0, 3] = synthetic.gaussian((d,), seed=1) * 1000.0
+    x[0, 0, 4, :64] = -2.0
+    kc, vc = encode_gpu(handles[d], d, torch_input(x, "f32"), Tcap=64)
+    gk, gv = _flat(unpack_cache(kc, 0, 5)), _flat(unpack_cache(vc, 0, 5))
+    assert np.all(gk["idx"][0] == 4) and np.all(gk["sig"][0] == 1)
+    assert gk["nh"][0] == 0 and gk["gh"][0] == 0 and gv["nh"][0] == 0
+    print(check_encode(prms[d], _x64(x), gk, gv))
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_append_one_token_at_a_time_equals_bulk(handles, d):
+    B, Hkv, T, Tcap = 2, 2, 130, 192
+    x = torch_input(synthetic.gaussian((B, Hkv, T, d), seed=3), "f32")
+    kb, vb = encode_gpu(handles[d], d, x, Tcap=Tcap)
+    ka, va = tq.Cache(d, True, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
+    for t in range(T):
+        encode_gpu(handles[d], d, x[:, :, t:t + 1], Tcap=Tcap, t0=t, kc=ka, vc=va)
+    torch.cuda.synchronize()
+    assert torch.equal(ka.buf, kb.buf) and torch.equal(va.buf, vb.buf)
+
+
+# ------------------------------------------------------------------ attention
+
+def _attend_case(h, prm, w, x_k, x_v, q, T, Tcap, seq_lens=None):
+    d = w.d
+    kc, _ = encode_gpu(h, d, torch_input(x_k, w.kv_dtype), Tcap=Tcap, which="k")
+    _, vc = encode_gpu(h, d, torch_input(x_v, w.kv_dtype), Tcap=Tcap, which="v")
+    qt = torch_input(q, w.q_dtype)
+    sl = torch.tensor(seq_lens, dtype=torch.int32, device="cuda") if seq_lens is not None else None
+    out = attend_gpu(h, qt, kc, vc, T=T, seq_lens=sl, scale=w.scale).cpu().numpy()
+    ku, vu = unpack_cache(kc, 0, Tcap), unpack_cache(vc, 0, Tcap)
+    lens = seq_lens if seq_lens is not None else [T] * q.shape[0]
+    ref = oracle_attend(prm, q.astype(np.float64), ku, vu, kc.Hkv, lens, w.scale)
+    err = rel_err_rows(out, ref)
+    return out, ref, err
+
+
+def test_attend_single_head(handles, prms):
+    w = synthetic.WORKLOADS["c1"]
+    out, ref, err = _attend_case(handles[128], prms[128], w, synthetic.kv(w, "k"), synthetic.kv(w, "v"),
+                                 synthetic.queries(w), w.T, w.T)
+    print("max rel err", err.max())
+    assert err.max() <= ATT_TOL
+
+
+def test_attend_gqa_32_8_40960_full(handles, prms):
+    w = synthetic.WORKLOADS["c3"]
+    out, ref, err = _attend_case(handles[128], prms[128], w, synthetic.kv(w, "k"), synthetic.kv(w, "v"),
+                                 synthetic.queries(w), w.T, w.T)
+    print("max rel err", err.max())
+    assert err.max() <= ATT_TOL
+
+
+def test_attend_long_context_b4_102400_full(handles, prms):
+    """The benchmark's workload and launch configuration, every output compared."""
+    w = synthetic.WORKLOADS["c4"]
+    out, ref, err = _attend_case(handles[128], prms[128], w, synthetic.kv(w, "k"), synthetic.kv(w, "v"),
+                                 synthetic.queries(w), w.T, w.T)
+    print("max rel err", err.max(), "path", tq.tq_attend_path(handles[128], w.Hq, w.Hkv))
+    assert err.max() <= ATT_TOL
+
+
+def test_append_and_attend_loop_d256(handles, prms):
+    """256 append-and-attend steps from 8192 tokens (B=16, Hq=32/Hkv=8, d=256);
+    several steps checked against the oracle; the grown cache equals a bulk encode."""
+    w = synthetic.WORKLOADS["c5"]
+    h, d = handles[256], 256
+    Tend = w.T + w.steps
+    Tcap = (Tend + 63) // 64 * 64
+    xk = torch_input(synthetic.kv(w, "k"), "f32")
+    xv = torch_input(synthetic.kv(w, "v"), "f32")
+    kc, vc = tq.Cache(d, True, w.B, w.Hkv, Tcap), tq.Cache(d, False, w.B, w.Hkv, Tcap)
+    tq.tq_encode_k(h, xk[:, :, :w.T], kc, 0)
+    tq.tq_encode_v(h, xv[:, :, :w.T], vc, 0)
+    check = {0: None, 1: None, 127: None, w.steps - 1: None}
+    ws = torch.empty(tq.tq_attend_workspace_bytes(h, w.B, w.Hq, w.Hkv, Tend), dtype=torch.uint8, device="cuda")
+    out = torch.empty((w.B, w.Hq, d), dtype=torch.float32, device="cuda")
+    for s in range(w.steps):
+        T = w.T + s
+        tq.tq_encode_k(h, xk[:, :, T:T + 1], kc, T)
+        tq.tq_encode_v(h, xv[:, :, T:T + 1], vc, T)
+        q = torch_input(synthetic.queries(w, s), w.q_dtype)
+        tq.tq_attend_decode(h, q, kc, vc, out, ws, T=T + 1, scale=w.scale)
+        if s in check:
+            check[s] = out.cpu().numpy().copy()
+    ku, vu = unpack_cache(kc, 0, Tend), unpack_cache(vc, 0, Tend)
+    for s, o in check.items():
+        T = w.T + s + 1
+        ref = oracle_attend(prms[d], synthetic.queries(w, s).astype(np.float64), ku, vu, w.Hkv, [T] * w.B, w.scale)
+        err = rel_err_rows(o, ref)
+        print("step", s, "max rel err", err.max())
+        assert err.max() <= ATT_TOL
+    kb, vb = encode_gpu(h, d, xk, Tcap=Tcap)
+    _, vb = encode_gpu(h, d, xv, Tcap=Tcap, which="v")
+    torch.cuda.synchronize()
+    assert torch.equal(kb.buf, kc.buf) and torch.equal(vb.buf, vc.buf)
+
+
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_attend_group_sizes_and_ragged_lengths(handles, prms, d, G):
+    Hkv, B, Tcap = 2, 3, 320
+    w = synthetic.Workload("t", "edge", B=B, Hq=Hkv * G, Hkv=Hkv, d=d, T=Tcap, kv_dtype="f32", q_dtype="f32",
+                           lognormal_norms=False, seed=d + G, scale=1.0 / math.sqrt(d))
+    xk, xv = synthetic.kv(w, "k"), synthetic.kv(w, "v")
+    q = synthetic.queries(w)
+    lens = [1, 65, Tcap]
+    out, ref, err = _attend_case(handles[d], prms[d], w, xk, xv, q, 0, Tcap, seq_lens=lens)
+    assert err.max() <= ATT_TOL
+    lens = [0, 200, 17]
+    out, ref, err = _attend_case(handles[d], prms[d], w, xk, xv, q, 0, Tcap, seq_lens=lens)
+    assert np.all(out[0] == 0.0)
+    assert err.max() <= ATT_TOL
+
+
+@pytest.mark.parametrize("qdt", ["f32", "bf16", "f16"])
+def test_attend_query_dtypes(handles, prms, qdt):
+    w = synthetic.Workload("t", "qdt", B=1, Hq=8, Hkv=2, d=128, T=500, kv_dtype="bf16", q_dtype=qdt,
+                           lognormal_norms=True, seed=9, scale=0.1)
+    q = synthetic.queries(w)
+    if qdt == "f16":
+        q = q.astype(np.float16).astype(np.float32)
+    out, ref, err = _attend_case(handles[128], prms[128], w, synthetic.kv(w, "k"), synthetic.kv(w, "v"), q,
+                                 w.T, 512)
+    assert err.max() <= ATT_TOL
+
+
+def test_split_count_invariance(handles):
+    """Different split plans (by T, or by Tcap through seq_lens) agree within 1e-5."""
+    d, B, Hq, Hkv, T, Tcap = 128, 2, 8, 2, 3000, 8192
+    h = handles[d]
+    x = torch_input(synthetic.gaussian((B, Hkv, Tcap, d), seed=4), "f32")
+    kc, vc = encode_gpu(h, d, x, Tcap=Tcap)
+    q = torch_input(synthetic.gaussian((B, Hq, d), seed=5), "f32")
+    a = attend_gpu(h, q, kc, vc, T=T, scale=0.2).cpu().numpy()
+    b = attend_gpu(h, q, kc, vc, seq_lens=torch.full((B,), T, dtype=torch.int32, device="cuda"),
+                   scale=0.2).cpu().numpy()
+    assert tq.tq_attend_workspace_bytes(h, B, Hq, Hkv, T) != tq.tq_attend_workspace_bytes(h, B, Hq, Hkv, Tcap)
+    assert rel_err_rows(a, b).max() <= 1e-5
+
+
+def test_group_heads_equal_separate_heads(handles):
+    """Query heads sharing a KV head give what each gives alone against that head."""
+    d, T = 128, 700
+    h = handles[d]
+    x = synthetic.gaussian((1, 2, T, d), seed=6)
+    kc, vc = encode_gpu(h, d, torch_input(x, "f32"), Tcap=768)
+    q = torch_input(synthetic.gaussian((1, 8, d), seed=7), "f32")
+    full = attend_gpu(h, q, kc, vc, T=T, scale=0.3).cpu().numpy()
+    k1, v1 = encode_gpu(h, d, torch_input(x[:, 1:2], "f32"), Tcap=768)
+    for g in range(4):
+        one = attend_gpu(h, q[:, 4 + g:5 + g].contiguous(), k1, v1, T=T, scale=0.3).cpu().numpy()
+        assert rel_err_rows(one[0, 0], full[0, 4 + g]).max() <= 1e-5
+
+
+def test_attend_argument_errors(handles):
+    h = handles[128]
+    kc, vc = tq.Cache(128, True, 1, 2, 64), tq.Cache(128, False, 1, 2, 64)
+    q = torch.zeros((1, 6, 128), device="cuda")
+    out = torch.empty((1, 6, 128), device="cuda")
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_attend_decode(h, q, kc, vc, out, ws, T=10)           # G = 3
+    assert e.value.status == tq.TQ_ERR_UNSUPPORTED
+    q = torch.zeros((1, 4, 128), device="cuda")
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_attend_decode(h, q, kc, vc, out, ws[:16], T=10)
+    assert e.value.status == tq.TQ_ERR_WORKSPACE
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_attend_decode(h, q, kc, vc, out, ws, T=65)           # T > Tcap
+    assert e.value.status == tq.TQ_ERR_INVALID_ARG
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_attend_decode(h, q, kc, vc, out, ws[1:], T=10)       # misaligned workspace
+    assert e.value.status == tq.TQ_ERR_INVALID_ARG
+    x = torch.zeros((1, 2, 10, 128), device="cuda")
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_encode_k(h, x, kc, t0=60)                            # past Tcap
+    assert e.value.status == tq.TQ_ERR_INVALID_ARG
+    assert tq.tq_device_status(h) == tq.TQ_OK
