@@ -243,6 +243,10 @@ def run_ours(args, rank: int, world: int, dist):
 
     # ---- timed region (device-resident inputs); the split-K kernel timed alone by events
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a_, b_ in kev:           # torch creates the CUDA events on first record; the library re-records them
+        a_.record()
+        b_.record()
+    torch.cuda.synchronize()
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)

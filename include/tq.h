@@ -178,8 +178,13 @@ TQ_API tq_status tq_device_status(const tq_handle* h, void* stream);
  * with concurrent tq_attend_decode calls on the same handle. */
 TQ_API tq_status tq_set_decode_events(tq_handle* h, void* ev_start, void* ev_stop);
 
-/* Name of the kernel path tq_attend_decode uses for these sizes ("mma" or
- * "simt"); static string. */
+/* Diagnostics: choose the decode kernel of later tq_attend_decode calls on this
+ * handle: 0 = automatic (tensor-core kernel where supported), 1 = the SIMT
+ * kernel.  Changes the workspace size tq_attend_workspace_bytes reports. */
+TQ_API tq_status tq_set_decode_path(tq_handle* h, int path);
+
+/* Name of the kernel path tq_attend_decode uses for these sizes on this handle
+ * ("mma" or "simt"); static string. */
 TQ_API const char* tq_attend_path(const tq_handle* h, int64_t Hq, int64_t Hkv);
 
 TQ_API const char* tq_status_string(tq_status s);

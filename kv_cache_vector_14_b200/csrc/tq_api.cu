@@ -15,28 +15,31 @@ size_t dtype_size(tq_dtype dt) { return dt == TQ_F32 ? 4 : 2; }
 bool dtype_ok(int dt) { return dt == TQ_F32 || dt == TQ_BF16 || dt == TQ_F16; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Pick the split count for decode: among a few candidate wave counts, the one
-// that best fills the GPU (whole waves of CTAs, balanced 64-token blocks).
-int choose_nsplit(int num_sms, int ctas_per_sm, int64_t pairs, int64_t Tmax) {
-    const int64_t nblk = Tmax > 0 ? (Tmax + kBlockT - 1) / kBlockT : 1;
-    const int64_t cap = (int64_t)num_sms * ctas_per_sm;
+// Split count for decode.  Work is `pairs` sequences of nchunk chunks; a CTA
+// handles `per` consecutive chunks spread over its warps, so its time is
+// ceil(per / warps) chunk-steps and the kernel's time is waves * that.  The
+// count maximising ideal / actual time wins (ties: fewer partials).  The loop
+// bound is also the workspace's upper bound (split_upper_bound).
+int64_t split_loop_bound(int64_t cap, int64_t pairs, int64_t nchunk) {
+    const int64_t bound = 16 * cap / pairs + 1;
+    return bound < nchunk ? bound : nchunk;
+}
+
+int choose_nsplit(int64_t cap, int warps, int64_t pairs, int64_t nchunk) {
+    const int64_t hi = split_loop_bound(cap, pairs, nchunk);
+    const double ideal = (double)pairs * nchunk / ((double)cap * warps);
     int64_t best = 1;
-    double best_score = -1.0;
-    for (int w = 1; w <= 8; ++w) {
-        int64_t ns = (int64_t)llround((double)w * cap / (double)pairs);
-        if (ns < 1) ns = 1;
-        if (ns > nblk) ns = nblk;
-        const int64_t per = (nblk + ns - 1) / ns;            // blocks per split
-        const int64_t used = (nblk + per - 1) / per;         // splits that get work
-        const int64_t ctas = pairs * used;
-        const int64_t waves = (ctas + cap - 1) / cap;
-        const double fill = (double)ctas / (double)(waves * cap);
-        const double bal = (double)nblk / (double)(used * per);
-        const double score = fill * bal - 1e-3 * w;           // prefer fewer partials on ties
-        if (score > best_score + 1e-9) { best_score = score; best = ns; }
+    double best_eff = -1.0;
+    for (int64_t ns = 1; ns <= hi; ++ns) {
+        const int64_t per = (nchunk + ns - 1) / ns;
+        const int64_t used = (nchunk + per - 1) / per;
+        if (used != ns) continue;
+        const int64_t waves = (pairs * used + cap - 1) / cap;
+        const double t = (double)waves * (double)((per + warps - 1) / warps);
+        const double eff = ideal / t - 1e-4 * (double)ns;
+        if (eff > best_eff + 1e-12) { best_eff = eff; best = ns; }
     }
-    const int64_t per = (nblk + best - 1) / best;
-    return (int)((nblk + per - 1) / per);
+    return (int)best;
 }
 
 struct DecodePlan {
@@ -46,13 +49,6 @@ struct DecodePlan {
     int64_t split_tokens = 0;
     size_t off_qp = 0, off_up = 0, off_ml = 0, off_acc = 0, bytes = 0;
 };
-
-// Largest split count choose_nsplit can return for any T <= Tmax.
-int nsplit_upper(int num_sms, int ctas_per_sm, int64_t pairs, int64_t Tmax) {
-    const int64_t nblk = Tmax > 0 ? (Tmax + kBlockT - 1) / kBlockT : 1;
-    int64_t ns = (int64_t)llround(8.0 * num_sms * ctas_per_sm / (double)pairs) + 1;
-    return (int)(ns < nblk ? ns : nblk);
-}
 
 void layout_ws(int d, size_t BHq, int nsplit, DecodePlan* p) {
     size_t off = 0;
@@ -68,13 +64,14 @@ bool make_plan(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t T
     if (!h || B < 0 || Hq <= 0 || Hkv <= 0 || Tmax < 0 || Hq % Hkv) return false;
     const int d = h->d;
     p->G = (int)(Hq / Hkv);
-    p->use_mma = mma_supported(d, p->G);
+    p->use_mma = !h->force_simt && mma_supported(d, p->G);
     const int64_t pairs = B * Hkv > 0 ? B * Hkv : 1;
-    const int cps = decode_ctas_per_sm(p->use_mma);
-    p->nsplit = upper_bound ? nsplit_upper(h->num_sms, cps, pairs, Tmax)
-                            : choose_nsplit(h->num_sms, cps, pairs, Tmax);
-    const int64_t nblk = Tmax > 0 ? (Tmax + kBlockT - 1) / kBlockT : 1;
-    p->split_tokens = ((nblk + p->nsplit - 1) / p->nsplit) * kBlockT;
+    const int64_t cap = (int64_t)h->num_sms * decode_ctas_per_sm(p->use_mma);
+    const int chunk = decode_chunk_tokens(p->use_mma);
+    const int64_t nchunk = Tmax > 0 ? (Tmax + chunk - 1) / chunk : 1;
+    p->nsplit = upper_bound ? (int)split_loop_bound(cap, pairs, nchunk)
+                            : choose_nsplit(cap, decode_warps(p->use_mma), pairs, nchunk);
+    p->split_tokens = ((nchunk + p->nsplit - 1) / p->nsplit) * chunk;
     layout_ws(d, (size_t)(B * Hq), p->nsplit, p);
     return true;
 }
@@ -225,7 +222,7 @@ size_t tq_attend_workspace_bytes(const tq_handle* h, int64_t B, int64_t Hq, int6
 
 const char* tq_attend_path(const tq_handle* h, int64_t Hq, int64_t Hkv) {
     if (!h || Hq <= 0 || Hkv <= 0 || Hq % Hkv) return "invalid";
-    return mma_supported(h->d, (int)(Hq / Hkv)) ? "mma" : "simt";
+    return (!h->force_simt && mma_supported(h->d, (int)(Hq / Hkv))) ? "mma" : "simt";
 }
 
 tq_status tq_attend_decode(const tq_handle* h, const void* q, tq_dtype qdt, int64_t B, int64_t Hq,
@@ -282,6 +279,12 @@ tq_status tq_set_decode_events(tq_handle* h, void* ev_start, void* ev_stop) {
     if (!h || (ev_start == nullptr) != (ev_stop == nullptr)) return TQ_ERR_INVALID_ARG;
     h->ev_start = static_cast<cudaEvent_t>(ev_start);
     h->ev_stop = static_cast<cudaEvent_t>(ev_stop);
+    return TQ_OK;
+}
+
+tq_status tq_set_decode_path(tq_handle* h, int path) {
+    if (!h || path < 0 || path > 1) return TQ_ERR_INVALID_ARG;
+    h->force_simt = path;
     return TQ_OK;
 }
 

@@ -293,17 +293,20 @@ cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml,
 namespace tqi {
 
 cudaError_t launch_decode_simt(int d, int G, const DecArgs& a, cudaStream_t s);
+cudaError_t launch_decode_mma(int d, int G, const DecArgs& a, cudaStream_t s);
+int decode_mma_chunk_tokens();
+int decode_mma_warps();
 
-bool mma_supported(int d, int G) {
-    (void)d; (void)G;
-    return false;
-}
+// The tensor-core kernel covers head_dim 128 with up to 8 query heads per kv
+// head; other shapes take the SIMT kernel.
+bool mma_supported(int d, int G) { return d == 128 && G >= 1 && G <= 8; }
 
 int decode_ctas_per_sm(bool use_mma) { return use_mma ? 1 : 4; }
+int decode_chunk_tokens(bool use_mma) { return use_mma ? decode_mma_chunk_tokens() : kBlockT; }
+int decode_warps(bool use_mma) { return use_mma ? decode_mma_warps() : 4; }
 
 cudaError_t launch_decode(int d, int G, bool use_mma, const DecArgs& a, cudaStream_t s) {
-    (void)use_mma;
-    return launch_decode_simt(d, G, a, s);
+    return use_mma ? launch_decode_mma(d, G, a, s) : launch_decode_simt(d, G, a, s);
 }
 
 }  // namespace tqi

@@ -86,6 +86,8 @@ cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml,
                            const float* part_acc, const float* dsign, float* out, cudaStream_t s);
 bool mma_supported(int d, int G);
 int decode_ctas_per_sm(bool use_mma);
+int decode_chunk_tokens(bool use_mma);   // split ranges are multiples of this
+int decode_warps(bool use_mma);          // warps sharing one split
 
 }  // namespace tqi
 
@@ -105,4 +107,5 @@ struct tq_handle {
     tqi::Codebook cb{};
     cudaEvent_t ev_start = nullptr;   // optional timing of the split-K kernel
     cudaEvent_t ev_stop = nullptr;
+    int force_simt = 0;               // diagnostics: always use the SIMT decode kernel
 };

@@ -22,7 +22,7 @@ TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 
 EXPORTED = ("tq_params_host", "tq_init", "tq_destroy", "tq_get_params", "tq_head_dim", "tq_block_bytes",
             "tq_cache_bytes", "tq_encode_k", "tq_encode_v", "tq_attend_workspace_bytes", "tq_attend_decode",
-            "tq_device_status", "tq_set_decode_events", "tq_attend_path", "tq_status_string")
+            "tq_device_status", "tq_set_decode_events", "tq_set_decode_path", "tq_attend_path", "tq_status_string")
 
 
 class TQError(RuntimeError):
@@ -75,6 +75,8 @@ def lib() -> C.CDLL:
             L.tq_device_status.restype = st
             L.tq_set_decode_events.argtypes = [P, P, P]
             L.tq_set_decode_events.restype = st
+            L.tq_set_decode_path.argtypes = [P, i32]
+            L.tq_set_decode_path.restype = st
             L.tq_attend_path.argtypes = [P, i64, i64]
             L.tq_attend_path.restype = C.c_char_p
             L.tq_status_string.argtypes = [i32]
@@ -219,6 +221,11 @@ def tq_set_decode_events(h, ev_start=None, ev_stop=None) -> None:
     a = C.c_void_p(ev_start.cuda_event) if ev_start is not None else None
     b = C.c_void_p(ev_stop.cuda_event) if ev_stop is not None else None
     _check(lib().tq_set_decode_events(h, a, b), "tq_set_decode_events")
+
+
+def tq_set_decode_path(h, path: str) -> None:
+    """"auto" (tensor-core kernel where supported) or "simt"."""
+    _check(lib().tq_set_decode_path(h, {"auto": 0, "simt": 1}[path]), "tq_set_decode_path")
 
 
 def tq_attend_path(h, Hq: int, Hkv: int) -> str:

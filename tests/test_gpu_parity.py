@@ -25,6 +25,17 @@ def handles(libtq):
         tq.tq_destroy(h)
 
 
+@pytest.fixture(params=["auto", "simt"])
+def decode_path(request, handles):
+    """Run a test once with the default (tensor-core where supported) decode
+    kernel and once with the SIMT kernel forced."""
+    for h in handles.values():
+        tq.tq_set_decode_path(h, request.param)
+    yield request.param
+    for h in handles.values():
+        tq.tq_set_decode_path(h, "auto")
+
+
 @pytest.fixture(scope="module")
 def prms():
     return {d: O.params(d, 0) for d in (128, 256)}
@@ -142,7 +153,7 @@ def _attend_case(h, prm, w, x_k, x_v, q, T, Tcap, seq_lens=None):
     return out, ref, err
 
 
-def test_attend_single_head(handles, prms):
+def test_attend_single_head(decode_path, handles, prms):
     w = synthetic.WORKLOADS["c1"]
     out, ref, err = _attend_case(handles[128], prms[128], w, synthetic.kv(w, "k"), synthetic.kv(w, "v"),
                                  synthetic.queries(w), w.T, w.T)
@@ -150,7 +161,7 @@ def test_attend_single_head(handles, prms):
     assert err.max() <= ATT_TOL
 
 
-def test_attend_gqa_32_8_40960_full(handles, prms):
+def test_attend_gqa_32_8_40960_full(decode_path, handles, prms):
     w = synthetic.WORKLOADS["c3"]
     out, ref, err = _attend_case(handles[128], prms[128], w, synthetic.kv(w, "k"), synthetic.kv(w, "v"),
                                  synthetic.queries(w), w.T, w.T)
@@ -158,12 +169,12 @@ def test_attend_gqa_32_8_40960_full(handles, prms):
     assert err.max() <= ATT_TOL
 
 
-def test_attend_long_context_b4_102400_full(handles, prms):
+def test_attend_long_context_b4_102400_full(decode_path, handles, prms):
     """The benchmark's workload and launch configuration, every output compared."""
     w = synthetic.WORKLOADS["c4"]
     out, ref, err = _attend_case(handles[128], prms[128], w, synthetic.kv(w, "k"), synthetic.kv(w, "v"),
                                  synthetic.queries(w), w.T, w.T)
-    print("max rel err", err.max(), "path", tq.tq_attend_path(handles[128], w.Hq, w.Hkv))
+    print("max rel err", err.max(), "path", tq.tq_attend_path(handles[128], w.Hq, w.Hkv), decode_path)
     assert err.max() <= ATT_TOL
 
 
@@ -205,7 +216,7 @@ def test_append_and_attend_loop_d256(handles, prms):
 
 @pytest.mark.parametrize("d", [128, 256])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
-def test_attend_group_sizes_and_ragged_lengths(handles, prms, d, G):
+def test_attend_group_sizes_and_ragged_lengths(decode_path, handles, prms, d, G):
     Hkv, B, Tcap = 2, 3, 320
     w = synthetic.Workload("t", "edge", B=B, Hq=Hkv * G, Hkv=Hkv, d=d, T=Tcap, kv_dtype="f32", q_dtype="f32",
                            lognormal_norms=False, seed=d + G, scale=1.0 / math.sqrt(d))
@@ -221,7 +232,7 @@ def test_attend_group_sizes_and_ragged_lengths(handles, prms, d, G):
 
 
 @pytest.mark.parametrize("qdt", ["f32", "bf16", "f16"])
-def test_attend_query_dtypes(handles, prms, qdt):
+def test_attend_query_dtypes(decode_path, handles, prms, qdt):
     w = synthetic.Workload("t", "qdt", B=1, Hq=8, Hkv=2, d=128, T=500, kv_dtype="bf16", q_dtype=qdt,
                            lognormal_norms=True, seed=9, scale=0.1)
     q = synthetic.queries(w)
@@ -232,7 +243,7 @@ def test_attend_query_dtypes(handles, prms, qdt):
     assert err.max() <= ATT_TOL
 
 
-def test_split_count_invariance(handles):
+def test_split_count_invariance(decode_path, handles):
     """Different split plans (by T, or by Tcap through seq_lens) agree within 1e-5."""
     d, B, Hq, Hkv, T, Tcap = 128, 2, 8, 2, 3000, 8192
     h = handles[d]
@@ -246,7 +257,7 @@ def test_split_count_invariance(handles):
     assert rel_err_rows(a, b).max() <= 1e-5
 
 
-def test_group_heads_equal_separate_heads(handles):
+def test_group_heads_equal_separate_heads(decode_path, handles):
     """Query heads sharing a KV head give what each gives alone against that head."""
     d, T = 128, 700
     h = handles[d]

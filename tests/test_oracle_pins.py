@@ -327,3 +327,26 @@ def test_attend_empty_and_gqa_independence():
     allh = O.attend(p, q, kc, vc, 0.2)
     for g in range(4):
         assert np.array_equal(allh[g], O.attend(p, q[g:g + 1], kc, vc, 0.2)[0])
+
+
+def test_layout_hand_worked_entries(golden):
+    """Single-entry records against words worked out by hand from the written layout."""
+    rows = golden("layout_single_entries.txt")
+    cases = {}
+    for kind, hd, j, val, widx, whex in rows:
+        cases.setdefault((kind, int(hd), int(j), int(val)), {})[int(widx)] = int(whex, 16)
+    for (kind, d, j, val), words in cases.items():
+        idx = np.zeros((1, d), np.uint8)
+        sig = np.zeros((1, d), np.uint8)
+        (idx if kind == "code" else sig)[0, j] = val
+        blocks = np.zeros(O.block_bytes(d, True), dtype=np.uint8)
+        O.pack(d, True, 0, idx, sig, np.zeros(1, np.uint16), np.zeros(1, np.uint16), blocks)
+        if kind == "code":
+            rec = blocks[: 3 * d // 8].view(np.uint32)
+        else:
+            off = 64 * 3 * d // 8
+            rec = blocks[off: off + d // 8].view(np.uint32)
+        expect = np.zeros_like(rec)
+        for w, v in words.items():
+            expect[w] = v
+        assert np.array_equal(rec, expect), (kind, d, j, val, [hex(x) for x in rec])
