@@ -165,6 +165,37 @@ TQ_API tq_status tq_attend_decode(const tq_handle* h, const void* q, tq_dtype qd
                            const int32_t* seq_lens, int64_t T, float scale, float* out, void* ws,
                            size_t ws_bytes, void* stream);
 
+/* ---- decode attention without device allocation ------------------------- */
+
+/* Size of the scratch array inside the library used by tq_attend_decode_static. */
+#define TQ_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* The method's pages have no counterpart to this call; it exists for callers.
+ * Same computation, arguments and results as tq_attend_decode, but with no
+ * workspace argument: the scratch (rotated queries, split-K partials) is a
+ * fixed TQ_STATIC_SCRATCH_BYTES (8 MiB) array inside the library, which every
+ * GPU that loads the library keeps until the process exits.  It is for callers
+ * that cannot allocate device memory when they run a decode step: a plugin or
+ * custom operator handed only input and output pointers by a host framework
+ * that owns the allocator, a serving loop that fixes its memory budget at
+ * start-up and must not grow it or pay an allocation's implicit
+ * synchronisation per token, or a deployment that forbids dynamic device
+ * allocation after initialisation.  Nothing here calls cudaMalloc or cudaFree.
+ * The first call on each device resolves the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  Sizes that need more scratch than
+ * the array holds (tq_attend_workspace_bytes(...) above 8 MiB) are rejected
+ * with TQ_ERR_WORKSPACE before anything is launched.  All calls on a device
+ * share the one array and it keeps the last call's contents (every byte a call
+ * reads is written by that call first, so nothing needs clearing); calls that
+ * overlap on the GPU -- on different streams, or from different threads --
+ * race on it and must be serialised by the caller.
+ * Errors: those of tq_attend_decode; CUDA if the address cannot be resolved. */
+TQ_API tq_status tq_attend_decode_static(const tq_handle* h, const void* q, tq_dtype qdtype, int64_t B,
+                                         int64_t Hq, const tq_cache* kc, const tq_cache* vc,
+                                         const int32_t* seq_lens, int64_t T, float scale, float* out,
+                                         void* stream);
+
 /* ---- diagnostics -------------------------------------------------------- */
 
 /* Synchronise `stream`, then report and clear the handle's device check word:

@@ -22,7 +22,7 @@ TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 
 EXPORTED = ("tq_params_host", "tq_init", "tq_destroy", "tq_get_params", "tq_head_dim", "tq_block_bytes",
             "tq_cache_bytes", "tq_encode_k", "tq_encode_v", "tq_attend_workspace_bytes", "tq_attend_decode",
-            "tq_device_status", "tq_set_decode_events", "tq_set_decode_path", "tq_attend_path", "tq_status_string")
+            "tq_attend_decode_static", "tq_device_status", "tq_set_decode_events", "tq_set_decode_path", "tq_attend_path", "tq_status_string")
 
 
 class TQError(RuntimeError):
@@ -71,6 +71,9 @@ def lib() -> C.CDLL:
             L.tq_attend_decode.argtypes = [P, P, i32, i64, i64, C.POINTER(tq_cache), C.POINTER(tq_cache), P, i64,
                                            C.c_float, P, P, C.c_size_t, P]
             L.tq_attend_decode.restype = st
+            L.tq_attend_decode_static.argtypes = [P, P, i32, i64, i64, C.POINTER(tq_cache), C.POINTER(tq_cache), P,
+                                                  i64, C.c_float, P, P]
+            L.tq_attend_decode_static.restype = st
             L.tq_device_status.argtypes = [P, P]
             L.tq_device_status.restype = st
             L.tq_set_decode_events.argtypes = [P, P, P]
