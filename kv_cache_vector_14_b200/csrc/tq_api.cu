@@ -21,11 +21,15 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // count maximising ideal / actual time wins (ties: fewer partials).  The loop
 // bound is also the workspace's upper bound (split_upper_bound).
 int64_t split_loop_bound(int64_t cap, int64_t pairs, int64_t nchunk) {
-    const int64_t bound = 16 * cap / pairs + 1;
+    int64_t bound = 16 * cap / pairs + 1;
+    if (bound > kMaxSplits) bound = kMaxSplits;
     return bound < nchunk ? bound : nchunk;
 }
 
 int choose_nsplit(int64_t cap, int warps, int64_t pairs, int64_t nchunk) {
+    // A CTA also pays a fixed cost (constants, barrier set-up, the merge of its
+    // warps, the partial it writes), about kSetup chunk-steps per warp.
+    const double kSetup = 2.0;
     const int64_t hi = split_loop_bound(cap, pairs, nchunk);
     const double ideal = (double)pairs * nchunk / ((double)cap * warps);
     int64_t best = 1;
@@ -35,8 +39,8 @@ int choose_nsplit(int64_t cap, int warps, int64_t pairs, int64_t nchunk) {
         const int64_t used = (nchunk + per - 1) / per;
         if (used != ns) continue;
         const int64_t waves = (pairs * used + cap - 1) / cap;
-        const double t = (double)waves * (double)((per + warps - 1) / warps);
-        const double eff = ideal / t - 1e-4 * (double)ns;
+        const double t = (double)waves * ((double)((per + warps - 1) / warps) + kSetup);
+        const double eff = ideal / t;
         if (eff > best_eff + 1e-12) { best_eff = eff; best = ns; }
     }
     return (int)best;
@@ -70,7 +74,7 @@ bool make_plan(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t T
     const int chunk = decode_chunk_tokens(p->use_mma);
     const int64_t nchunk = Tmax > 0 ? (Tmax + chunk - 1) / chunk : 1;
     p->nsplit = upper_bound ? (int)split_loop_bound(cap, pairs, nchunk)
-                            : choose_nsplit(cap, decode_warps(p->use_mma), pairs, nchunk);
+                            : choose_nsplit(cap, decode_warps(p->use_mma, p->G), pairs, nchunk);
     p->split_tokens = ((nchunk + p->nsplit - 1) / p->nsplit) * chunk;
     layout_ws(d, (size_t)(B * Hq), p->nsplit, p);
     return true;
@@ -152,6 +156,7 @@ tq_status tq_init(int head_dim, uint64_t seed, tq_handle** out) {
     }
     h->cb.lut_lo[0] = lo[0]; h->cb.lut_lo[1] = lo[1];
     h->cb.lut_hi[0] = hi[0]; h->cb.lut_hi[1] = hi[1];
+    for (int k = 0; k < 32; ++k) h->cb.pow2[k] = 1u << k;
 
     std::vector<float> sign(d), st((size_t)d * d), sthr((size_t)d * d);
     for (int j = 0; j < d; ++j) sign[j] = (float)h->hD[j];

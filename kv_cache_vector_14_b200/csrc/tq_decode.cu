@@ -44,13 +44,17 @@ __device__ void smem_fwht(float* v) {
 }
 
 // ---------------------------------------------------------------- prologue
-// q' = H D q / sqrt(d) and up = sqrt(pi/2)/m * S q' for QH query heads per CTA.
+// q' = H D q / sqrt(d) and up = sqrt(pi/2)/m * S q' for kQH query heads per
+// CTA.  S^T is staged through shared memory in chunks of kJC rows with wide,
+// independent loads; each thread then owns one JL row i for all kQH heads.
 constexpr int kQH = 8;
+constexpr int kJC = 64;
 
 template <int D, int DT>
 __global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t BHq, const float* dsign,
                                                         const float* ST, float* qp, float* up) {
     __shared__ float v[kQH * D];
+    extern __shared__ __align__(16) float sst[];          // [kJC][D] rows of S^T
     const int j = threadIdx.x;
     const int64_t h0 = (int64_t)blockIdx.x * kQH;
     const float ds = dsign[j];
@@ -64,14 +68,21 @@ __global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t B
     const float inv = 1.0f / sqrtf((float)D);
 #pragma unroll
     for (int k = 0; k < kQH; ++k) v[k * D + j] *= inv;
-    __syncthreads();
     float u[kQH];
 #pragma unroll
     for (int k = 0; k < kQH; ++k) u[k] = 0.f;
-    for (int jj = 0; jj < D; ++jj) {
-        const float s = __ldg(ST + (size_t)jj * D + j);   // S[j][jj], coalesced over j
+    for (int j0 = 0; j0 < D; j0 += kJC) {
+        __syncthreads();
+        const float4* src = reinterpret_cast<const float4*>(ST + (size_t)j0 * D);
+#pragma unroll 8
+        for (int i = j; i < kJC * D / 4; i += D) reinterpret_cast<float4*>(sst)[i] = __ldg(src + i);
+        __syncthreads();
+#pragma unroll 8
+        for (int jj = 0; jj < kJC; ++jj) {
+            const float sv = sst[jj * D + j];                 // S[j][j0 + jj]
 #pragma unroll
-        for (int k = 0; k < kQH; ++k) u[k] = fmaf(s, v[k * D + jj], u[k]);
+            for (int k = 0; k < kQH; ++k) u[k] = fmaf(sv, v[k * D + j0 + jj], u[k]);
+        }
     }
     const float cq = 1.2533141373155003f / (float)D;       // sqrt(pi/2) / m
 #pragma unroll
@@ -209,27 +220,76 @@ __global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
 // ---------------------------------------------------------------- combine
 // One CTA of D threads per (batch, query head): log-sum-exp merge of the
 // split partials, division by the softmax sum, one inverse transform D H.
+// The per-split (max, sum) pairs go through shared memory once; each thread
+// then sums its coordinate over the splits with independent loads.
+constexpr int kMaxSplitSmem = kMaxSplits;
+
 template <int D>
 __global__ void __launch_bounds__(D) tq_combine_kernel(const float* part_ml, const float* part_acc, int nsplit,
                                                        const float* dsign, float* out) {
     __shared__ float v[D];
-    const int j = threadIdx.x;
+    __shared__ float wgt[kMaxSplitSmem];
+    __shared__ float red[D / 32];
+    __shared__ float sM, sL;
+    const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
     const int64_t bh = blockIdx.x;
     const float* ml = part_ml + bh * nsplit * 2;
-    float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, ml[2 * s]);
-    float L = 0.f, A = 0.f;
-    if (M != -INFINITY) {
-        for (int s = 0; s < nsplit; ++s) {
-            const float f = exp2f(ml[2 * s] - M);
-            L = fmaf(f, ml[2 * s + 1], L);
-            A = fmaf(f, part_acc[(bh * nsplit + s) * D + j], A);
-        }
+    const int ns = nsplit < kMaxSplitSmem ? nsplit : kMaxSplitSmem;
+    float m = -INFINITY;
+    for (int s = j; s < ns; s += D) m = fmaxf(m, ml[2 * s]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    if (j == 0) {
+        float M = -INFINITY;
+        for (int w = 0; w < D / 32; ++w) M = fmaxf(M, red[w]);
+        sM = M;
     }
-    v[j] = (L > 0.f) ? A / L : 0.f;
+    __syncthreads();
+    const float M = sM;
+    float l = 0.f;
+    for (int s = j; s < ns; s += D) {
+        const float f = (M == -INFINITY) ? 0.f : exp2f(ml[2 * s] - M);
+        wgt[s] = f;
+        l = fmaf(f, ml[2 * s + 1], l);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(kFull, l, o);
+    __syncthreads();
+    if (lane == 0) red[warp] = l;
+    __syncthreads();
+    if (j == 0) {
+        float L = 0.f;
+        for (int w = 0; w < D / 32; ++w) L += red[w];
+        sL = L;
+    }
+    __syncthreads();
+    const float* acc = part_acc + bh * nsplit * D + j;
+    float A0 = 0.f, A1 = 0.f, A2 = 0.f, A3 = 0.f;
+    int s = 0;
+    for (; s + 4 <= ns; s += 4) {
+        A0 = fmaf(wgt[s], acc[(size_t)s * D], A0);
+        A1 = fmaf(wgt[s + 1], acc[(size_t)(s + 1) * D], A1);
+        A2 = fmaf(wgt[s + 2], acc[(size_t)(s + 2) * D], A2);
+        A3 = fmaf(wgt[s + 3], acc[(size_t)(s + 3) * D], A3);
+    }
+    for (; s < ns; ++s) A0 = fmaf(wgt[s], acc[(size_t)s * D], A0);
+    const float L = sL;
+    v[j] = (L > 0.f) ? ((A0 + A1) + (A2 + A3)) / L : 0.f;
     __syncthreads();
     smem_fwht<D, 1>(v);
     out[bh * D + j] = dsign[j] * v[j] * (1.0f / sqrtf((float)D));
+}
+
+template <int D, int DT>
+cudaError_t launch_prologue_t(int grid, size_t smem, const void* q, int64_t BHq, const float* dsign, const float* st,
+                              float* qp, float* up, cudaStream_t s) {
+    auto kern = tq_prologue_kernel<D, DT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, D, smem, s>>>(q, BHq, dsign, st, qp, up);
+    return cudaGetLastError();
 }
 
 template <int D>
@@ -237,12 +297,13 @@ cudaError_t launch_prologue_d(const void* q, tq_dtype dt, int64_t BHq, const flo
                               float* qp, float* up, cudaStream_t s) {
     const int grid = (int)((BHq + kQH - 1) / kQH);
     if (grid == 0) return cudaSuccess;
+    const size_t smem = (size_t)kJC * D * sizeof(float);
     switch (dt) {
-        case TQ_F32: tq_prologue_kernel<D, TQ_F32><<<grid, D, 0, s>>>(q, BHq, dsign, st, qp, up); break;
-        case TQ_BF16: tq_prologue_kernel<D, TQ_BF16><<<grid, D, 0, s>>>(q, BHq, dsign, st, qp, up); break;
-        case TQ_F16: tq_prologue_kernel<D, TQ_F16><<<grid, D, 0, s>>>(q, BHq, dsign, st, qp, up); break;
+        case TQ_F32: return launch_prologue_t<D, TQ_F32>(grid, smem, q, BHq, dsign, st, qp, up, s);
+        case TQ_BF16: return launch_prologue_t<D, TQ_BF16>(grid, smem, q, BHq, dsign, st, qp, up, s);
+        case TQ_F16: return launch_prologue_t<D, TQ_F16>(grid, smem, q, BHq, dsign, st, qp, up, s);
     }
-    return cudaGetLastError();
+    return cudaErrorInvalidValue;
 }
 
 template <int D, int G>
@@ -295,7 +356,7 @@ namespace tqi {
 cudaError_t launch_decode_simt(int d, int G, const DecArgs& a, cudaStream_t s);
 cudaError_t launch_decode_mma(int d, int G, const DecArgs& a, cudaStream_t s);
 int decode_mma_chunk_tokens();
-int decode_mma_warps();
+int decode_mma_warps(int G);
 
 // The tensor-core kernel covers head_dim 128 with up to 8 query heads per kv
 // head; other shapes take the SIMT kernel.
@@ -303,7 +364,7 @@ bool mma_supported(int d, int G) { return d == 128 && G >= 1 && G <= 8; }
 
 int decode_ctas_per_sm(bool use_mma) { return use_mma ? 1 : 4; }
 int decode_chunk_tokens(bool use_mma) { return use_mma ? decode_mma_chunk_tokens() : kBlockT; }
-int decode_warps(bool use_mma) { return use_mma ? decode_mma_warps() : 4; }
+int decode_warps(bool use_mma, int G) { return use_mma ? decode_mma_warps(G) : 4; }
 
 cudaError_t launch_decode(int d, int G, bool use_mma, const DecArgs& a, cudaStream_t s) {
     return use_mma ? launch_decode_mma(d, G, a, s) : launch_decode_simt(d, G, a, s);

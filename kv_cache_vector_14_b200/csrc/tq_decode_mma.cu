@@ -38,8 +38,7 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kD = 128;
-constexpr int kNW = 8;                 // warps per CTA
-constexpr int kStages = 4;             // ring depth per warp
+constexpr int kStages = 3;             // ring depth per warp
 constexpr int kChunk = 32;             // tokens per stage
 constexpr int kCodeB = 48;             // code bytes per token (d = 128)
 constexpr int kSignB = 16;             // sign bytes per token
@@ -94,15 +93,20 @@ __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
     uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+// 2^x on the special-function unit (relative error ~2^-22); -inf gives 0
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
@@ -115,16 +119,25 @@ __device__ __forceinline__ void split_hilo(float x0, float x1, uint32_t& hi, uin
     lo = h2_bits(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
 }
 
+// Left shifts as integer multiplies, x << k = x * 2^k (IMAD): the powers of two
+// come from the kernel parameters, so the compiler cannot turn them back into
+// shifts; they run on the FMA pipe and leave the ALU pipe (prmt, lop3) to the
+// dequantisation.  Right shifts stay shifts (the multiply-high form is a
+// quarter-rate instruction).
+__device__ __forceinline__ uint32_t shl_m(uint32_t x, const uint32_t* pw, int k) { return x * pw[k]; }
+__device__ __forceinline__ uint32_t shr_m(uint32_t x, const uint32_t* pw, int k) { (void)pw; return x >> k; }
+
 // Selector words for the 32 slot codes of one token: sel[w] holds, in its
 // nibbles, the codes of slot positions 8w .. 8w+7.
-__device__ __forceinline__ void code_selectors(const uint8_t* rec, uint32_t (&sel)[4]) {
+__device__ __forceinline__ void code_selectors(const uint8_t* rec, const uint32_t* pw, uint32_t (&sel)[4]) {
     const uint32_t wa = *reinterpret_cast<const uint32_t*>(rec);
     const uint32_t wb = *reinterpret_cast<const uint32_t*>(rec + 4);
     const uint32_t wc = *reinterpret_cast<const uint32_t*>(rec + 8);
     sel[0] = wa & 0x77777777u;
     sel[1] = wb & 0x77777777u;
     sel[2] = wc & 0x77777777u;
-    sel[3] = ((wa >> 3) & 0x11111111u) | ((wb >> 2) & 0x22222222u) | ((wc >> 1) & 0x44444444u);
+    sel[3] = (shr_m(wa, pw, 3) & 0x11111111u) | (shr_m(wb, pw, 2) & 0x22222222u) |
+             (shr_m(wc, pw, 1) & 0x44444444u);
 }
 
 // fp16 centroid pairs for slot positions 4kc .. 4kc+3: e=0,1 -> x0, e=2,3 -> x1
@@ -135,14 +148,23 @@ __device__ __forceinline__ void dequant4(uint32_t sel16, const uint32_t (&lut)[4
     x1 = __byte_perm(lo4, hi4, 0x7362);
 }
 
-__device__ __forceinline__ uint32_t sel_for(const uint32_t (&sel)[4], int kc) {
-    return (kc & 1) ? (sel[kc >> 1] >> 16) : sel[kc >> 1];
+__device__ __forceinline__ uint32_t sel_for(const uint32_t (&sel)[4], const uint32_t* pw, int kc) {
+    return (kc & 1) ? shr_m(sel[kc >> 1], pw, 16) : sel[kc >> 1];
 }
 
 // ---------------------------------------------------------------- kernel
-__global__ void __launch_bounds__(kNW * 32, 1) tq_decode_mma128_kernel(const DecArgs a, int G) {
+// Token-row orientation: each mma tile has 16 tokens on M and the (head,
+// hi|lo) columns on N (NT n-tiles of 4 heads), so no M rows are wasted:
+//   scores  S[16 tok][8] += Kdeq[16 tok][16 coords] * Q'[16 coords][8]   (8 coordinate chunks)
+//                         + Sgn[16 tok][16 signs] * U'[16 signs][8]       (8 sign chunks)
+//   values  O^T[16 coords][8] += Vdeq^T[16 coords][16 tok] * P[16 tok][8] (8 coordinate tiles)
+// Lane (g, t) = (lane / 4, lane % 4) dequantises tokens g and g + 8 of each
+// 16-token tile; its score columns are head t (hi, lo), so its softmax state
+// and output rows belong to head t (and head 4 + t when NT = 2).
+template <int NT, int NW>
+__global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecArgs a, int G) {
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kNW * kStages * kStageB);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)NW * kStages * kStageB);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gr = lane >> 2, tq4 = lane & 3;
     uint8_t* ring = smem + (size_t)warp * kStages * kStageB;
@@ -153,7 +175,7 @@ __global__ void __launch_bounds__(kNW * 32, 1) tq_decode_mma128_kernel(const Dec
     const int64_t s0 = (int64_t)split * a.split_tokens;
     const int64_t s1 = (s0 + a.split_tokens < Tb) ? s0 + a.split_tokens : Tb;
     const int nchunk = s1 > s0 ? (int)((s1 - s0 + kChunk - 1) / kChunk) : 0;
-    const int nmine = nchunk > warp ? (nchunk - warp + kNW - 1) / kNW : 0;
+    const int nmine = nchunk > warp ? (nchunk - warp + NW - 1) / NW : 0;
     const int64_t seq = (int64_t)b * a.Hkv + hkv;
     const int64_t kbb = block_bytes(kD, true), vbb = block_bytes(kD, false);
 
@@ -162,9 +184,8 @@ __global__ void __launch_bounds__(kNW * 32, 1) tq_decode_mma128_kernel(const Dec
     fence_mbar_init();
     __syncwarp();
 
-    // issue the six bulk copies of chunk i of this warp into stage i % kStages
     auto issue = [&](int i) {
-        const int64_t t0 = s0 + (int64_t)(warp + i * kNW) * kChunk;     // multiple of 32
+        const int64_t t0 = s0 + (int64_t)(warp + i * NW) * kChunk;     // multiple of 32
         const int64_t blk = seq * a.NB + (t0 >> 6);
         const int half = (int)((t0 >> 5) & 1);
         const uint8_t* kb = a.kc + blk * kbb;
@@ -183,33 +204,45 @@ __global__ void __launch_bounds__(kNW * 32, 1) tq_decode_mma128_kernel(const Dec
         for (int i = 0; i < kStages && i < nmine; ++i) issue(i);
     }
 
-    // A operands: rows gr (hi) and gr + 8 (lo) of query head gr of this kv head
-    uint32_t aq[8][4], au[8][4];
-    {
-        const bool live = gr < G;
-        const int64_t bh = (int64_t)b * a.Hq + (int64_t)hkv * G + (live ? gr : 0);
+    // B operands (constant): column n = gr of n-tile nt is head 4 nt + gr / 2, limb gr % 2
+    uint32_t bq[NT][8][2], bu[NT][8][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int hcol = 4 * nt + (gr >> 1);
+        const bool live = hcol < G;
+        const int64_t bh = (int64_t)b * a.Hq + (int64_t)hkv * G + (live ? hcol : 0);
         const float* qp = a.qp + bh * kD;
         const float* up = a.up + bh * kD;
 #pragma unroll
         for (int kc = 0; kc < 8; ++kc) {
             const int c0 = 16 * kc + 2 * tq4;
-            float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f, y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+            float x[4] = {0.f, 0.f, 0.f, 0.f}, y[4] = {0.f, 0.f, 0.f, 0.f};
             if (live) {
-                x0 = qp[c0]; x1 = qp[c0 + 1]; x2 = qp[c0 + 8]; x3 = qp[c0 + 9];
-                y0 = up[c0]; y1 = up[c0 + 1]; y2 = up[c0 + 8]; y3 = up[c0 + 9];
+                x[0] = qp[c0]; x[1] = qp[c0 + 1]; x[2] = qp[c0 + 8]; x[3] = qp[c0 + 9];
+                y[0] = up[c0]; y[1] = up[c0 + 1]; y[2] = up[c0 + 8]; y[3] = up[c0 + 9];
             }
-            split_hilo(x0, x1, aq[kc][0], aq[kc][1]);
-            split_hilo(x2, x3, aq[kc][2], aq[kc][3]);
-            split_hilo(y0, y1, au[kc][0], au[kc][1]);
-            split_hilo(y2, y3, au[kc][2], au[kc][3]);
+            uint32_t h0, l0, h1, l1;
+            split_hilo(x[0], x[1], h0, l0);
+            split_hilo(x[2], x[3], h1, l1);
+            bq[nt][kc][0] = (gr & 1) ? l0 : h0;
+            bq[nt][kc][1] = (gr & 1) ? l1 : h1;
+            split_hilo(y[0], y[1], h0, l0);
+            split_hilo(y[2], y[3], h1, l1);
+            bu[nt][kc][0] = (gr & 1) ? l0 : h0;
+            bu[nt][kc][1] = (gr & 1) ? l1 : h1;
         }
     }
     const uint32_t lut[4] = {a.cb.lut_lo[0], a.cb.lut_lo[1], a.cb.lut_hi[0], a.cb.lut_hi[1]};
+    const uint32_t* pw = a.cb.pow2;
 
-    float o[16][4];
+    float o[NT][8][4];
 #pragma unroll
-    for (int ct = 0; ct < 16; ++ct) o[ct][0] = o[ct][1] = o[ct][2] = o[ct][3] = 0.f;
-    float mrun = -INFINITY, lrun = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+    float mrun[NT], lrun[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) { mrun[nt] = -INFINITY; lrun[nt] = 0.f; }
     bool failed = false;
 
     for (int i = 0; i < nmine; ++i) {
@@ -217,91 +250,103 @@ __global__ void __launch_bounds__(kNW * 32, 1) tq_decode_mma128_kernel(const Dec
         if (!mbar_wait_bounded(bar, (uint32_t)((i / kStages) & 1))) {
             failed = true;
             if (lane == 0) atomicExch(a.err, 1);
-            // bounded wait for this warp's copies still in flight, then stop
             for (int j = i; j < nmine && j < i + kStages; ++j)
                 mbar_wait_bounded(smem_u32(&bars[warp * kStages + (j % kStages)]), (uint32_t)((j / kStages) & 1));
             break;
         }
         const uint8_t* st = ring + (i % kStages) * kStageB;
-        const int64_t tok0 = s0 + (int64_t)(warp + i * kNW) * kChunk;
+        const int64_t tok0 = s0 + (int64_t)(warp + i * NW) * kChunk;
         const int nvalid = (int)((s1 - tok0) < kChunk ? (s1 - tok0) : kChunk);
 
-#pragma unroll 1
+#pragma unroll
         for (int kt = 0; kt < kChunk / 16; ++kt) {
             if (kt * 16 >= nvalid) break;
-            // ---------------- scores for the two 8-token tiles
-            float sc[2][4];
+            const int tA = kt * 16 + gr, tB = tA + 8;            // this lane's two tokens
+            // ---------------- scores
+            uint32_t selA[4], selB[4];
+            code_selectors(st + kOffKc + tA * kCodeB + tq4 * 12, pw, selA);
+            code_selectors(st + kOffKc + tB * kCodeB + tq4 * 12, pw, selB);
+            const uint32_t sgA = *reinterpret_cast<const uint32_t*>(st + kOffKs + tA * kSignB + tq4 * 4);
+            const uint32_t sgB = *reinterpret_cast<const uint32_t*>(st + kOffKs + tB * kSignB + tq4 * 4);
+            const uint32_t gA = *reinterpret_cast<const uint16_t*>(st + kOffKg + 2 * tA);
+            const uint32_t gB = *reinterpret_cast<const uint16_t*>(st + kOffKg + 2 * tB);
+            const uint32_t ggA = gA | (gA << 16), ggB = gB | (gB << 16);
+            float acc[NT][4];
 #pragma unroll
-            for (int tt = 0; tt < 2; ++tt) {
-                const int tok = kt * 16 + tt * 8 + gr;                      // B column of this lane
-                uint32_t sel[4];
-                code_selectors(st + kOffKc + tok * kCodeB + tq4 * 12, sel);
-                const uint32_t nsg = ~*reinterpret_cast<const uint32_t*>(st + kOffKs + tok * kSignB + tq4 * 4);
-                const uint32_t gb = *reinterpret_cast<const uint16_t*>(st + kOffKg + 2 * tok);
-                const uint32_t gg = gb | (gb << 16);
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll
-                for (int kc = 0; kc < 8; ++kc) {
-                    uint32_t b0, b1;
-                    dequant4(sel_for(sel, kc), lut, b0, b1);
-                    mma16816(acc, aq[kc], b0, b1);
+            for (int kc = 0; kc < 8; ++kc) {
+                uint32_t ka[4];
+                dequant4(sel_for(selA, pw, kc), lut, ka[0], ka[2]);
+                dequant4(sel_for(selB, pw, kc), lut, ka[1], ka[3]);
+                uint32_t sa[4];
+                // sign bit 1 -> +gamma: the pair (2kc | 2kc+1) of a slot sits at bits (q, 16 + q)
+                sa[0] = ggA ^ (~shl_m(sgA, pw, 15 - 2 * kc) & 0x80008000u);
+                sa[1] = ggB ^ (~shl_m(sgB, pw, 15 - 2 * kc) & 0x80008000u);
+                sa[2] = ggA ^ (~shl_m(sgA, pw, 14 - 2 * kc) & 0x80008000u);
+                sa[3] = ggB ^ (~shl_m(sgB, pw, 14 - 2 * kc) & 0x80008000u);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    mma16816(acc[nt], ka, bq[nt][kc][0], bq[nt][kc][1]);
+                    mma16816(acc[nt], sa, bu[nt][kc][0], bu[nt][kc][1]);
                 }
+            }
+            // ---------------- online softmax per head (this lane: head 4 nt + tq4)
+            const float2 nkA = __half22float2(__halves2half2(*reinterpret_cast<const __half*>(st + kOffKn + 2 * tA),
+                                                             *reinterpret_cast<const __half*>(st + kOffKn + 2 * tB)));
+            float2 nv = __half22float2(__halves2half2(*reinterpret_cast<const __half*>(st + kOffVn + 2 * tA),
+                                                      *reinterpret_cast<const __half*>(st + kOffVn + 2 * tB)));
+            const bool okA = tA < nvalid, okB = tB < nvalid;
+            if (nvalid < kChunk) {
+                if (!okA) nv.x = 0.f;
+                if (!okB) nv.y = 0.f;
+            }
+            uint32_t pb[NT][2];
 #pragma unroll
-                for (int kc = 0; kc < 8; ++kc) {
-                    const uint32_t b0 = gg ^ ((nsg << (15 - 2 * kc)) & 0x80008000u);
-                    const uint32_t b1 = gg ^ ((nsg << (14 - 2 * kc)) & 0x80008000u);
-                    mma16816(acc, au[kc], b0, b1);
+            for (int nt = 0; nt < NT; ++nt) {
+                float sA = a.scale_log2 * nkA.x * (acc[nt][0] + acc[nt][1]);
+                float sB = a.scale_log2 * nkA.y * (acc[nt][2] + acc[nt][3]);
+                if (nvalid < kChunk) {
+                    if (!okA) sA = -INFINITY;
+                    if (!okB) sB = -INFINITY;
                 }
-                sc[tt][0] = acc[0] + acc[2];                                 // token 2 tq4, head gr
-                sc[tt][1] = acc[1] + acc[3];                                 // token 2 tq4 + 1
-            }
-            // ---------------- online softmax (log2 units), per head gr
-            float s[4], nvv[4];
+                float mt = fmaxf(sA, sB);
+                mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 4));
+                mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 8));
+                mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 16));
+                const float mnew = fmaxf(mrun[nt], mt);
+                if (__any_sync(kFull, mnew > mrun[nt])) {
+                    const float corr = (mnew == -INFINITY) ? 1.f : fast_exp2(mrun[nt] - mnew);
+                    lrun[nt] *= corr;
 #pragma unroll
-            for (int tt = 0; tt < 2; ++tt) {
-                const int t0 = kt * 16 + tt * 8 + 2 * tq4;
-                const float2 nk = __half22float2(*reinterpret_cast<const __half2*>(st + kOffKn + 2 * t0));
-                const float2 nv = __half22float2(*reinterpret_cast<const __half2*>(st + kOffVn + 2 * t0));
-                s[2 * tt] = (t0 < nvalid) ? a.scale_log2 * nk.x * sc[tt][0] : -INFINITY;
-                s[2 * tt + 1] = (t0 + 1 < nvalid) ? a.scale_log2 * nk.y * sc[tt][1] : -INFINITY;
-                nvv[2 * tt] = nv.x;
-                nvv[2 * tt + 1] = nv.y;
-            }
-            float mt = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3]));
-            mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 1));
-            mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 2));
-            const float mnew = fmaxf(mrun, mt);
-            if (__any_sync(kFull, mnew > mrun)) {
-                const float corr = (mnew == -INFINITY) ? 1.f : exp2f(mrun - mnew);
-                lrun *= corr;
-#pragma unroll
-                for (int ct = 0; ct < 16; ++ct) {
-                    o[ct][0] *= corr; o[ct][1] *= corr; o[ct][2] *= corr; o[ct][3] *= corr;
+                    for (int mt2 = 0; mt2 < 8; ++mt2) {
+                        o[nt][mt2][0] *= corr; o[nt][mt2][1] *= corr; o[nt][mt2][2] *= corr; o[nt][mt2][3] *= corr;
+                    }
+                    mrun[nt] = mnew;
                 }
-                mrun = mnew;
+                const float pA = (sA == -INFINITY) ? 0.f : fast_exp2(sA - mrun[nt]);
+                const float pB = (sB == -INFINITY) ? 0.f : fast_exp2(sB - mrun[nt]);
+                lrun[nt] += pA + pB;
+                uint32_t hi, lo, xA, xB;
+                split_hilo(pA * nv.x, pB * nv.y, hi, lo);
+                // (hi, lo) of token A and of token B as the two columns of head tq4
+                xA = __byte_perm(hi, lo, 0x5410);
+                xB = __byte_perm(hi, lo, 0x7632);
+                if (4 * nt + tq4 >= G) xA = xB = 0u;
+                pb[nt][0] = movmatrix_t(xA);
+                pb[nt][1] = movmatrix_t(xB);
             }
-            float pv[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float p = (s[k] == -INFINITY) ? 0.f : exp2f(s[k] - mrun);
-                lrun += p;
-                pv[k] = (p == 0.f) ? 0.f : p * nvv[k];
-            }
-            uint32_t ap[4];
-            split_hilo(pv[0], pv[1], ap[0], ap[1]);
-            split_hilo(pv[2], pv[3], ap[2], ap[3]);
-            if (gr >= G) ap[0] = ap[1] = ap[2] = ap[3] = 0u;
-            // ---------------- values: O += P V
-            uint32_t vs0[4], vs1[4];
-            code_selectors(st + kOffVc + (kt * 16 + gr) * kCodeB + tq4 * 12, vs0);
-            code_selectors(st + kOffVc + (kt * 16 + 8 + gr) * kCodeB + tq4 * 12, vs1);
+            // ---------------- values: O^T += Vdeq^T P
+            code_selectors(st + kOffVc + tA * kCodeB + tq4 * 12, pw, selA);
+            code_selectors(st + kOffVc + tB * kCodeB + tq4 * 12, pw, selB);
 #pragma unroll
             for (int kc = 0; kc < 8; ++kc) {
                 uint32_t x0, x1, y0, y1;
-                dequant4(sel_for(vs0, kc), lut, x0, x1);       // tokens 0..7 of the tile
-                dequant4(sel_for(vs1, kc), lut, y0, y1);       // tokens 8..15
-                mma16816(o[2 * kc], ap, movmatrix_t(x0), movmatrix_t(y0));
-                mma16816(o[2 * kc + 1], ap, movmatrix_t(x1), movmatrix_t(y1));
+                dequant4(sel_for(selA, pw, kc), lut, x0, x1);      // token tA: coords 16kc+2t(+1), +8
+                dequant4(sel_for(selB, pw, kc), lut, y0, y1);      // token tB
+                const uint32_t va[4] = {movmatrix_t(x0), movmatrix_t(x1), movmatrix_t(y0), movmatrix_t(y1)};
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma16816(o[nt][kc], va, pb[nt][0], pb[nt][1]);
             }
         }
         __syncwarp();
@@ -310,39 +355,43 @@ __global__ void __launch_bounds__(kNW * 32, 1) tq_decode_mma128_kernel(const Dec
             issue(i + kStages);
         }
     }
-    if (failed) {
-        mrun = -INFINITY;
-        lrun = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        if (failed) { mrun[nt] = -INFINITY; lrun[nt] = 0.f; }
+        lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 4);
+        lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 8);
+        lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 16);
     }
-    lrun += __shfl_xor_sync(kFull, lrun, 1);
-    lrun += __shfl_xor_sync(kFull, lrun, 2);
 
     // ---------------- merge the warps of the CTA into one partial per head
     __syncwarp();
     float* wbuf = reinterpret_cast<float*>(ring);             // [G][kD + 2], in this warp's own ring
-    if (gr < G) {
 #pragma unroll
-        for (int ct = 0; ct < 16; ++ct) {
-            const int c = 8 * ct + 2 * tq4;
-            wbuf[gr * (kD + 2) + c] = o[ct][0] + o[ct][2];
-            wbuf[gr * (kD + 2) + c + 1] = o[ct][1] + o[ct][3];
-        }
-        if (tq4 == 0) {
-            wbuf[gr * (kD + 2) + kD] = mrun;
-            wbuf[gr * (kD + 2) + kD + 1] = lrun;
+    for (int nt = 0; nt < NT; ++nt) {
+        const int h = 4 * nt + tq4;
+        if (h < G) {
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                wbuf[h * (kD + 2) + 16 * mt + gr] = o[nt][mt][0] + o[nt][mt][1];
+                wbuf[h * (kD + 2) + 16 * mt + 8 + gr] = o[nt][mt][2] + o[nt][mt][3];
+            }
+            if (gr == 0) {
+                wbuf[h * (kD + 2) + kD] = mrun[nt];
+                wbuf[h * (kD + 2) + kD + 1] = lrun[nt];
+            }
         }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * kD; idx += kNW * 32) {
+    for (int idx = threadIdx.x; idx < G * kD; idx += NW * 32) {
         const int g = idx / kD, j = idx % kD;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kNW; ++w)
+        for (int w = 0; w < NW; ++w)
             M = fmaxf(M, reinterpret_cast<const float*>(smem + (size_t)w * kStages * kStageB)[g * (kD + 2) + kD]);
         float L = 0.f, A = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < kNW; ++w) {
+            for (int w = 0; w < NW; ++w) {
                 const float* wb = reinterpret_cast<const float*>(smem + (size_t)w * kStages * kStageB) + g * (kD + 2);
                 const float f = exp2f(wb[kD] - M);
                 L = fmaf(f, wb[kD + 1], L);
@@ -361,20 +410,27 @@ __global__ void __launch_bounds__(kNW * 32, 1) tq_decode_mma128_kernel(const Dec
 
 }  // namespace
 
-size_t decode_mma_smem_bytes() { return (size_t)kNW * kStages * kStageB + (size_t)kNW * kStages * 8; }
+constexpr int kNW1 = 16;   // warps per CTA, up to 4 heads per kv head (one n-tile)
+constexpr int kNW2 = 8;    // warps per CTA, 8 heads per kv head (two n-tiles, more registers)
+
+template <int NT, int NW>
+cudaError_t launch_mma_t(const DecArgs& a, int G, cudaStream_t s) {
+    const size_t smem = (size_t)NW * kStages * kStageB + (size_t)NW * kStages * 8;
+    auto kern = tq_decode_mma128_kernel<NT, NW>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
+    kern<<<grid, NW * 32, smem, s>>>(a, G);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_decode_mma(int d, int G, const DecArgs& a, cudaStream_t s) {
     if (d != kD || G < 1 || G > 8) return cudaErrorInvalidValue;
     if (a.B * a.Hkv == 0) return cudaSuccess;
-    const size_t smem = decode_mma_smem_bytes();
-    cudaError_t e = cudaFuncSetAttribute(tq_decode_mma128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    dim3 grid(a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
-    tq_decode_mma128_kernel<<<grid, kNW * 32, smem, s>>>(a, G);
-    return cudaGetLastError();
+    return G <= 4 ? launch_mma_t<1, kNW1>(a, G, s) : launch_mma_t<2, kNW2>(a, G, s);
 }
 
 int decode_mma_chunk_tokens() { return kChunk; }
-int decode_mma_warps() { return kNW; }
+int decode_mma_warps(int G) { return G <= 4 ? kNW1 : kNW2; }
 
 }  // namespace tqi

@@ -23,8 +23,6 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kThreads = 256;
-constexpr int kTileV = 32;                  // vectors per tile
-constexpr int kVecPerWarp = kTileV / 8;
 
 template <int DT>
 __device__ __forceinline__ float load_x(const void* p, int64_t i) {
@@ -49,19 +47,23 @@ __device__ __forceinline__ uint32_t nibbles8(uint32_t lo4, uint32_t hi4) {
     return a | (b << 16);
 }
 
-template <int D, bool IS_K>
+template <int D, bool IS_K, int TV>
 struct EncSmem {
     static constexpr int R = D / 32;
     static constexpr int JC = (D == 128) ? 128 : 64;           // JL columns resident at once
     static constexpr size_t s_bytes = IS_K ? (size_t)JC * D * 4 : 0;
-    static constexpr size_t r_bytes = IS_K ? (size_t)kTileV * D * 4 : 0;
-    static constexpr size_t code_bytes = (size_t)kTileV * D;
+    static constexpr size_t r_bytes = IS_K ? (size_t)TV * D * 4 : 0;
+    static constexpr size_t code_bytes = (size_t)TV * D;
     static constexpr size_t total = s_bytes + r_bytes + code_bytes;
 };
 
-template <int D, bool IS_K, int DT>
+// TV vectors per tile (32 for bulk encodes, 8 when there are too few tiles to
+// fill the GPU, e.g. appending one token per head).
+template <int D, bool IS_K, int DT, int TV>
 __global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
-    using SM = EncSmem<D, IS_K>;
+    using SM = EncSmem<D, IS_K, TV>;
+    constexpr int kTileV = TV;
+    constexpr int kVecPerWarp = TV / 8;
     constexpr int R = SM::R;
     constexpr int JC = SM::JC;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -87,76 +89,93 @@ __global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
     __syncthreads();
 
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-        // ---------------- phase 1: one warp per vector
+        // ---------------- phase 1: one warp per vector, the warp's vectors
+        // processed together so their shuffle chains overlap
+        float x[kVecPerWarp][R], ss[kVecPerWarp];
+        int64_t tt[kVecPerWarp], bh[kVecPerWarp];
+        bool valid[kVecPerWarp];
+#pragma unroll
+        for (int vv = 0; vv < kVecPerWarp; ++vv) {
+            const int64_t gv = tile * kTileV + warp * kVecPerWarp + vv;
+            valid[vv] = gv < N;
+            ss[vv] = 0.f;
+            tt[vv] = valid[vv] ? gv % a.Tnew : 0;
+            bh[vv] = valid[vv] ? gv / a.Tnew : 0;
+            const int64_t h = bh[vv] % a.Hkv, b = bh[vv] / a.Hkv;
+            const int64_t base = b * a.sb + h * a.sh + tt[vv] * a.st;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                x[vv][r] = valid[vv] ? load_x<DT>(a.x, base + lane + 32 * r) : 0.f;
+                ss[vv] = fmaf(x[vv][r], x[vv][r], ss[vv]);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int vv = 0; vv < kVecPerWarp; ++vv) ss[vv] += __shfl_xor_sync(kFull, ss[vv], o);
+        // sign flip, then butterflies over lane bits (coordinate bits 0..4)
+#pragma unroll
+        for (int vv = 0; vv < kVecPerWarp; ++vv)
+#pragma unroll
+            for (int r = 0; r < R; ++r) x[vv][r] *= dsg[r];
+#pragma unroll
+        for (int hb = 1; hb < 32; hb <<= 1) {
+#pragma unroll
+            for (int vv = 0; vv < kVecPerWarp; ++vv)
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    const float p = __shfl_xor_sync(kFull, x[vv][r], hb);
+                    x[vv][r] = (lane & hb) ? (p - x[vv][r]) : (x[vv][r] + p);
+                }
+        }
+        // butterflies over register bits (coordinate bits 5..)
+#pragma unroll
+        for (int hb = 1; hb < R; hb <<= 1)
+#pragma unroll
+            for (int vv = 0; vv < kVecPerWarp; ++vv)
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+                    if ((r & hb) == 0) {
+                        const float u = x[vv][r], w = x[vv][r | hb];
+                        x[vv][r] = u + w;
+                        x[vv][r | hb] = u - w;
+                    }
+        float g2[kVecPerWarp];
+#pragma unroll
         for (int vv = 0; vv < kVecPerWarp; ++vv) {
             const int v = warp * kVecPerWarp + vv;
-            const int64_t gv = tile * kTileV + v;
-            const bool valid = gv < N;
-            float x[R];
-            float ss = 0.f;
-            int64_t tt = 0, bh = 0;
-            if (valid) {
-                tt = gv % a.Tnew;
-                bh = gv / a.Tnew;
-                const int64_t h = bh % a.Hkv, b = bh / a.Hkv;
-                const int64_t base = b * a.sb + h * a.sh + tt * a.st;
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    x[r] = load_x<DT>(a.x, base + lane + 32 * r);
-                    ss = fmaf(x[r], x[r], ss);
-                }
-            } else {
-#pragma unroll
-                for (int r = 0; r < R; ++r) x[r] = 0.f;
-            }
-            ss = warp_sum(ss);
-            const float n = sqrtf(ss);
-#pragma unroll
-            for (int r = 0; r < R; ++r) x[r] *= dsg[r];
-            // butterflies over lane bits (coordinate bits 0..4)
-#pragma unroll
-            for (int hb = 1; hb < 32; hb <<= 1) {
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const float p = __shfl_xor_sync(kFull, x[r], hb);
-                    x[r] = (lane & hb) ? (p - x[r]) : (x[r] + p);
-                }
-            }
-            // butterflies over register bits (coordinate bits 5..)
-#pragma unroll
-            for (int hb = 1; hb < R; hb <<= 1) {
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    if ((r & hb) == 0) {
-                        const float u = x[r], w = x[r | hb];
-                        x[r] = u + w;
-                        x[r | hb] = u - w;
-                    }
-                }
-            }
+            const float n = sqrtf(ss[vv]);
             const float nsd = n * sqrt_d;
-            float g2 = 0.f;
+            g2[vv] = 0.f;
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 const int j = lane + 32 * r;
-                const float y = (n > 0.f) ? __fdiv_rn(x[r], nsd) : 0.f;
+                const float y = (n > 0.f) ? __fdiv_rn(x[vv][r], nsd) : 0.f;
                 int code = 0;
 #pragma unroll
                 for (int i = 0; i < 7; ++i) code += (y >= a.cb.b[i]) ? 1 : 0;
                 const float res = (n > 0.f) ? (y - sC[code]) : 0.f;
-                g2 = fmaf(res, res, g2);
+                g2[vv] = fmaf(res, res, g2[vv]);
                 if constexpr (IS_K) sR[v * D + j] = res;
                 sCode[v * D + (j >> 7) * 128 + slot_of(j) * 32 + slot_pos(j)] = (uint8_t)code;
             }
-            if constexpr (IS_K) g2 = warp_sum(g2);
-            if (valid && lane == 0) {
-                const int64_t t = a.t0 + tt;
-                uint8_t* blk = a.cache + (bh * a.NB + (t >> 6)) * bb;
+        }
+        if constexpr (IS_K) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int vv = 0; vv < kVecPerWarp; ++vv) g2[vv] += __shfl_xor_sync(kFull, g2[vv], o);
+        }
+#pragma unroll
+        for (int vv = 0; vv < kVecPerWarp; ++vv) {
+            if (valid[vv] && lane == 0) {
+                const int64_t t = a.t0 + tt[vv];
+                uint8_t* blk = a.cache + (bh[vv] * a.NB + (t >> 6)) * bb;
                 const int tau = (int)(t & 63);
                 const int64_t norm_off = kBlockT * code_bytes(D) + (IS_K ? kBlockT * sign_bytes(D) : 0);
-                reinterpret_cast<__half*>(blk + norm_off)[tau] = __float2half_rn(n);
+                reinterpret_cast<__half*>(blk + norm_off)[tau] = __float2half_rn(sqrtf(ss[vv]));
                 if constexpr (IS_K)
-                    reinterpret_cast<__half*>(blk + norm_off + 2 * kBlockT)[tau] = __float2half_rn(sqrtf(g2));
+                    reinterpret_cast<__half*>(blk + norm_off + 2 * kBlockT)[tau] = __float2half_rn(sqrtf(g2[vv]));
             }
         }
         __syncthreads();
@@ -237,19 +256,28 @@ __global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
     }
 }
 
-template <int D, bool IS_K, int DT>
-cudaError_t launch_enc_t(const EncArgs& a, int num_sms, cudaStream_t s) {
-    using SM = EncSmem<D, IS_K>;
-    auto kern = tq_encode_kernel<D, IS_K, DT>;
+template <int D, bool IS_K, int DT, int TV>
+cudaError_t launch_enc_tv(const EncArgs& a, int num_sms, cudaStream_t s) {
+    using SM = EncSmem<D, IS_K, TV>;
+    auto kern = tq_encode_kernel<D, IS_K, DT, TV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::total);
     if (e != cudaSuccess) return e;
     const int64_t N = a.B * a.Hkv * a.Tnew;
-    const int64_t ntiles = (N + kTileV - 1) / kTileV;
-    const int64_t cap = (int64_t)num_sms * 2;
+    const int64_t ntiles = (N + TV - 1) / TV;
+    // K kernels stage S once per CTA, so they run persistent (two CTAs per SM);
+    // V kernels are small and take as many CTAs as fit.
+    const int64_t cap = (int64_t)num_sms * (IS_K ? 2 : 8);
     const int grid = (int)(ntiles < cap ? ntiles : cap);
     if (grid <= 0) return cudaSuccess;
     kern<<<grid, kThreads, SM::total, s>>>(a);
     return cudaGetLastError();
+}
+
+template <int D, bool IS_K, int DT>
+cudaError_t launch_enc_t(const EncArgs& a, int num_sms, cudaStream_t s) {
+    const int64_t N = a.B * a.Hkv * a.Tnew;
+    if (N < (int64_t)32 * num_sms) return launch_enc_tv<D, IS_K, DT, 8>(a, num_sms, s);
+    return launch_enc_tv<D, IS_K, DT, 32>(a, num_sms, s);
 }
 
 template <int D, bool IS_K>

@@ -14,6 +14,7 @@
 namespace tqi {
 
 constexpr int kBlockT = 64;      // tokens per cache block
+constexpr int kMaxSplits = 2048; // split-K partials per query head (combine keeps their weights in smem)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Codebook passed by value to every kernel (it lands in the constant bank).
@@ -22,6 +23,7 @@ struct Codebook {
     float b[7];         // decision boundaries (midpoints)
     uint32_t lut_lo[2]; // low bytes of the fp16 bit patterns of c[0..7]
     uint32_t lut_hi[2]; // high bytes of the fp16 bit patterns of c[0..7]
+    uint32_t pow2[32];  // 1 << k: shifts done as integer multiplies (FMA pipe, not ALU)
 };
 
 // Host-side generation of the constants (tq_params.cpp).
@@ -87,7 +89,7 @@ cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml,
 bool mma_supported(int d, int G);
 int decode_ctas_per_sm(bool use_mma);
 int decode_chunk_tokens(bool use_mma);   // split ranges are multiples of this
-int decode_warps(bool use_mma);          // warps sharing one split
+int decode_warps(bool use_mma, int G);   // warps sharing one split
 
 }  // namespace tqi
 
