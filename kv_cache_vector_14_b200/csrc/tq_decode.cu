@@ -47,7 +47,7 @@ __device__ void smem_fwht(float* v) {
 // q' = H D q / sqrt(d) and up = sqrt(pi/2)/m * S q' for kQH query heads per
 // CTA.  S^T is staged through shared memory in chunks of kJC rows with wide,
 // independent loads; each thread then owns one JL row i for all kQH heads.
-constexpr int kQH = 8;
+constexpr int kQH = 1;
 constexpr int kJC = 64;
 
 template <int D, int DT>
@@ -55,6 +55,7 @@ __global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t B
                                                         const float* ST, float* qp, float* up) {
     __shared__ float v[kQH * D];
     extern __shared__ __align__(16) float sst[];          // [kJC][D] rows of S^T
+    pdl_trigger();                                        // the split-K kernel may start its prefetch
     const int j = threadIdx.x;
     const int64_t h0 = (int64_t)blockIdx.x * kQH;
     const float ds = dsign[j];
@@ -136,6 +137,7 @@ __global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
 
     const int64_t seq = (int64_t)b * a.Hkv + hkv;
     const int64_t kbb = block_bytes(D, true), vbb = block_bytes(D, false);
+    pdl_wait();                                           // q' and u' from the prologue
     float q[G][R], u[G][R], acc[G][R], mrun[G], lrun[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -233,6 +235,7 @@ __global__ void __launch_bounds__(D) tq_combine_kernel(const float* part_ml, con
     __shared__ float sM, sL;
     const int j = threadIdx.x, lane = j & 31, warp = j >> 5;
     const int64_t bh = blockIdx.x;
+    pdl_wait();                                           // partials of the split-K kernel
     const float* ml = part_ml + bh * nsplit * 2;
     const int ns = nsplit < kMaxSplitSmem ? nsplit : kMaxSplitSmem;
     float m = -INFINITY;
@@ -309,8 +312,7 @@ cudaError_t launch_prologue_d(const void* q, tq_dtype dt, int64_t BHq, const flo
 template <int D, int G>
 cudaError_t launch_simt(const DecArgs& a, cudaStream_t s) {
     dim3 grid(a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
-    tq_decode_simt_kernel<D, G><<<grid, 128, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(tq_decode_simt_kernel<D, G>, grid, dim3(128), 0, s, a);
 }
 
 template <int D>
@@ -343,10 +345,11 @@ cudaError_t launch_decode_simt(int d, int G, const DecArgs& a, cudaStream_t s) {
 cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml, const float* part_acc,
                            const float* dsign, float* out, cudaStream_t s) {
     if (BHq == 0) return cudaSuccess;
-    if (d == 128) tq_combine_kernel<128><<<(unsigned)BHq, 128, 0, s>>>(part_ml, part_acc, nsplit, dsign, out);
-    else if (d == 256) tq_combine_kernel<256><<<(unsigned)BHq, 256, 0, s>>>(part_ml, part_acc, nsplit, dsign, out);
-    else return cudaErrorInvalidValue;
-    return cudaGetLastError();
+    if (d == 128)
+        return launch_pdl(tq_combine_kernel<128>, dim3((unsigned)BHq), dim3(128), 0, s, part_ml, part_acc, nsplit, dsign, out);
+    if (d == 256)
+        return launch_pdl(tq_combine_kernel<256>, dim3((unsigned)BHq), dim3(256), 0, s, part_ml, part_acc, nsplit, dsign, out);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace tqi

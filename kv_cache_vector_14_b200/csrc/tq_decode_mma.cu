@@ -203,6 +203,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
     if (lane == 0) {
         for (int i = 0; i < kStages && i < nmine; ++i) issue(i);
     }
+    pdl_wait();                           // q' and u' come from the prologue kernel
 
     // B operands (constant): column n = gr of n-tile nt is head 4 nt + gr / 2, limb gr % 2
     uint32_t bq[NT][8][2], bu[NT][8][2];
@@ -363,6 +364,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
         lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 16);
     }
 
+    pdl_trigger();                        // the combine kernel may start launching
     // ---------------- merge the warps of the CTA into one partial per head
     __syncwarp();
     float* wbuf = reinterpret_cast<float*>(ring);             // [G][kD + 2], in this warp's own ring
@@ -420,8 +422,7 @@ cudaError_t launch_mma_t(const DecArgs& a, int G, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
-    kern<<<grid, NW * 32, smem, s>>>(a, G);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(NW * 32), smem, s, a, G);
 }
 
 cudaError_t launch_decode_mma(int d, int G, const DecArgs& a, cudaStream_t s) {

@@ -256,6 +256,114 @@ __global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
     }
 }
 
+// ---------------------------------------------------------------- small batches (K)
+// Appends of a few vectors per head: one warp per vector and four warps per
+// CTA, so a 32-vector append runs on 8 SMs at once instead of one.  S is
+// staged through shared memory (all of it at d = 128, 64-column chunks at
+// d = 256) and the projection accumulates over columns in the same order as
+// the tiled kernel, so both give bit-identical sign words.
+constexpr int kSmallWarps = 4;
+
+template <int D, int DT>
+__global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(const EncArgs a) {
+    constexpr int R = D / 32;
+    constexpr int JC = (D == 128) ? 128 : 64;      // columns of S resident at once
+    extern __shared__ __align__(16) float sS[];     // [JC][R][32]
+    __shared__ __align__(16) float sr[kSmallWarps][D];
+    __shared__ __align__(16) uint8_t scode[kSmallWarps][D];
+    __shared__ float sC[8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x < 8) sC[threadIdx.x] = a.cb.c[threadIdx.x];
+    __syncthreads();
+    const int64_t N = a.B * a.Hkv * a.Tnew;
+    const int64_t gv0 = (int64_t)blockIdx.x * kSmallWarps + warp;
+    const bool valid = gv0 < N;                     // idle warps still take part in the staging
+    const int64_t gv = valid ? gv0 : N - 1;
+    const int64_t tt = gv % a.Tnew, bh = gv / a.Tnew;
+    const int64_t t = a.t0 + tt;
+    uint8_t* blk = a.cache + (bh * a.NB + (t >> 6)) * block_bytes(D, true);
+    const int64_t h = bh % a.Hkv, b = bh / a.Hkv;
+    const int64_t base = b * a.sb + h * a.sh + tt * a.st;
+    float x[R];
+    float ss = 0.f;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        x[r] = load_x<DT>(a.x, base + lane + 32 * r);
+        ss = fmaf(x[r], x[r], ss);
+        x[r] *= __ldg(a.dsign + lane + 32 * r);
+    }
+    ss = warp_sum(ss);
+#pragma unroll
+    for (int hb = 1; hb < 32; hb <<= 1)
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const float p = __shfl_xor_sync(kFull, x[r], hb);
+            x[r] = (lane & hb) ? (p - x[r]) : (x[r] + p);
+        }
+#pragma unroll
+    for (int hb = 1; hb < R; hb <<= 1)
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            if ((r & hb) == 0) {
+                const float u = x[r], w = x[r | hb];
+                x[r] = u + w;
+                x[r | hb] = u - w;
+            }
+    const float n = sqrtf(ss);
+    const float nsd = n * sqrtf((float)D);
+    float g2 = 0.f;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int j = lane + 32 * r;
+        const float y = (n > 0.f) ? __fdiv_rn(x[r], nsd) : 0.f;
+        int code = 0;
+#pragma unroll
+        for (int i = 0; i < 7; ++i) code += (y >= a.cb.b[i]) ? 1 : 0;
+        const float res = (n > 0.f) ? (y - sC[code]) : 0.f;
+        g2 = fmaf(res, res, g2);
+        sr[warp][j] = res;
+        scode[warp][(j >> 7) * 128 + slot_of(j) * 32 + slot_pos(j)] = (uint8_t)code;
+    }
+    g2 = warp_sum(g2);
+    if (valid && lane == 0) {
+        const int64_t norm_off = kBlockT * code_bytes(D) + kBlockT * sign_bytes(D);
+        reinterpret_cast<__half*>(blk + norm_off)[t & 63] = __float2half_rn(n);
+        reinterpret_cast<__half*>(blk + norm_off + 2 * kBlockT)[t & 63] = __float2half_rn(sqrtf(g2));
+    }
+    float z[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) z[r] = 0.f;
+    for (int j0 = 0; j0 < D; j0 += JC) {
+        __syncthreads();
+        const float4* src = reinterpret_cast<const float4*>(a.sthr + (size_t)j0 * D);
+#pragma unroll 8
+        for (int i = threadIdx.x; i < JC * D / 4; i += kSmallWarps * 32) reinterpret_cast<float4*>(sS)[i] = __ldg(src + i);
+        __syncthreads();
+#pragma unroll 4
+        for (int jj = 0; jj < JC; ++jj) {
+            const float rj = sr[warp][j0 + jj];
+#pragma unroll
+            for (int r = 0; r < R; ++r) z[r] = fmaf(rj, sS[(jj * R + r) * 32 + lane], z[r]);
+        }
+    }
+    if (!valid) return;
+    uint32_t mine = 0;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const uint32_t word = __ballot_sync(kFull, z[r] >= 0.f);
+        if (lane == r) mine = word;
+    }
+    if (lane < R) reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(D) + (t & 63) * sign_bytes(D))[lane] = mine;
+    constexpr int W = 3 * D / 32;
+    if (lane < W) {
+        const int sl = lane / 12, st = (lane % 12) / 3, g = lane % 3;
+        const uint32_t* sw = reinterpret_cast<const uint32_t*>(&scode[warp][sl * 128 + st * 32]);
+        const uint32_t main = nibbles8(sw[2 * g], sw[2 * g + 1]);
+        const uint32_t tail = nibbles8(sw[6], sw[7]);
+        reinterpret_cast<uint32_t*>(blk + (t & 63) * code_bytes(D))[lane] = main | (((tail >> g) & 0x11111111u) << 3);
+    }
+}
+
 template <int D, bool IS_K, int DT, int TV>
 cudaError_t launch_enc_tv(const EncArgs& a, int num_sms, cudaStream_t s) {
     using SM = EncSmem<D, IS_K, TV>;
@@ -276,6 +384,17 @@ cudaError_t launch_enc_tv(const EncArgs& a, int num_sms, cudaStream_t s) {
 template <int D, bool IS_K, int DT>
 cudaError_t launch_enc_t(const EncArgs& a, int num_sms, cudaStream_t s) {
     const int64_t N = a.B * a.Hkv * a.Tnew;
+    if constexpr (IS_K) {
+        if (N <= (int64_t)4 * num_sms) {        // appends: one warp per vector
+            const unsigned grid = (unsigned)((N + kSmallWarps - 1) / kSmallWarps);
+            const size_t smem = (size_t)((D == 128) ? 128 : 64) * D * sizeof(float);
+            auto kern = tq_encode_k_small_kernel<D, DT>;
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            kern<<<grid, kSmallWarps * 32, smem, s>>>(a);
+            return cudaGetLastError();
+        }
+    }
     if (N < (int64_t)32 * num_sms) return launch_enc_tv<D, IS_K, DT, 8>(a, num_sms, s);
     return launch_enc_tv<D, IS_K, DT, 32>(a, num_sms, s);
 }

@@ -127,7 +127,9 @@ def test_encode_zero_and_special_vectors(handles, prms):
 
 @pytest.mark.parametrize("d", [128, 256])
 def test_append_one_token_at_a_time_equals_bulk(handles, d):
-    B, Hkv, T, Tcap = 2, 2, 130, 192
+    """Bulk encodes (over 4 vectors per SM: the tiled kernel) and one-token
+    appends (the small-batch kernel) write identical bytes."""
+    B, Hkv, T, Tcap = 2, 4, 130, 192
     x = torch_input(synthetic.gaussian((B, Hkv, T, d), seed=3), "f32")
     kb, vb = encode_gpu(handles[d], d, x, Tcap=Tcap)
     ka, va = tq.Cache(d, True, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
