@@ -31,6 +31,8 @@
 // cp.async.bulk with an mbarrier transaction count, no multicast).  Waits are
 // bounded: on timeout the kernel sets the handle's check word, waits (bounded)
 // for its own copies, and contributes an empty partial.
+#include <type_traits>
+
 #include "tq_internal.h"
 
 namespace tqi {
@@ -136,6 +138,7 @@ __device__ __forceinline__ void code_selectors(const uint8_t* rec, const uint32_
     sel[0] = wa & 0x77777777u;
     sel[1] = wb & 0x77777777u;
     sel[2] = wc & 0x77777777u;
+    // bit 3 of each nibble of wa, wb, wc holds bits 0, 1, 2 of codes 24..31
     sel[3] = (shr_m(wa, pw, 3) & 0x11111111u) | (shr_m(wb, pw, 2) & 0x22222222u) |
              (shr_m(wc, pw, 1) & 0x44444444u);
 }
@@ -241,9 +244,13 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
-    float mrun[NT], lrun[NT];
+    float mrun[NT], lrun[NT], live[NT];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) { mrun[nt] = -INFINITY; lrun[nt] = 0.f; }
+    for (int nt = 0; nt < NT; ++nt) {
+        mrun[nt] = -INFINITY;
+        lrun[nt] = 0.f;
+        live[nt] = (4 * nt + tq4 < G) ? 1.f : 0.f;   // this lane's head exists
+    }
     bool failed = false;
 
     for (int i = 0; i < nmine; ++i) {
@@ -259,9 +266,10 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
         const int64_t tok0 = s0 + (int64_t)(warp + i * NW) * kChunk;
         const int nvalid = (int)((s1 - tok0) < kChunk ? (s1 - tok0) : kChunk);
 
-#pragma unroll
-        for (int kt = 0; kt < kChunk / 16; ++kt) {
-            if (kt * 16 >= nvalid) break;
+        // one 16-token tile; PARTIAL masks tokens beyond nvalid (only the last
+        // chunk of a split can be partial)
+        auto tile = [&](const int kt, auto partial_tag) {
+            constexpr bool PARTIAL = decltype(partial_tag)::value;
             const int tA = kt * 16 + gr, tB = tA + 8;            // this lane's two tokens
             // ---------------- scores
             uint32_t selA[4], selB[4];
@@ -298,7 +306,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
             float2 nv = __half22float2(__halves2half2(*reinterpret_cast<const __half*>(st + kOffVn + 2 * tA),
                                                       *reinterpret_cast<const __half*>(st + kOffVn + 2 * tB)));
             const bool okA = tA < nvalid, okB = tB < nvalid;
-            if (nvalid < kChunk) {
+            if constexpr (PARTIAL) {
                 if (!okA) nv.x = 0.f;
                 if (!okB) nv.y = 0.f;
             }
@@ -307,7 +315,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
             for (int nt = 0; nt < NT; ++nt) {
                 float sA = a.scale_log2 * nkA.x * (acc[nt][0] + acc[nt][1]);
                 float sB = a.scale_log2 * nkA.y * (acc[nt][2] + acc[nt][3]);
-                if (nvalid < kChunk) {
+                if constexpr (PARTIAL) {
                     if (!okA) sA = -INFINITY;
                     if (!okB) sB = -INFINITY;
                 }
@@ -316,7 +324,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
                 mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 8));
                 mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 16));
                 const float mnew = fmaxf(mrun[nt], mt);
-                if (__any_sync(kFull, mnew > mrun[nt])) {
+                if (__any_sync(kFull, mnew > mrun[nt])) {   // a new running maximum
                     const float corr = (mnew == -INFINITY) ? 1.f : fast_exp2(mrun[nt] - mnew);
                     lrun[nt] *= corr;
 #pragma unroll
@@ -325,15 +333,15 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
                     }
                     mrun[nt] = mnew;
                 }
-                const float pA = (sA == -INFINITY) ? 0.f : fast_exp2(sA - mrun[nt]);
-                const float pB = (sB == -INFINITY) ? 0.f : fast_exp2(sB - mrun[nt]);
+                // mrun >= sA, sB here, so the exponent is <= 0 (masked: -inf -> 0)
+                const float pA = fast_exp2(sA - mrun[nt]);
+                const float pB = fast_exp2(sB - mrun[nt]);
                 lrun[nt] += pA + pB;
                 uint32_t hi, lo, xA, xB;
-                split_hilo(pA * nv.x, pB * nv.y, hi, lo);
+                split_hilo(pA * nv.x * live[nt], pB * nv.y * live[nt], hi, lo);
                 // (hi, lo) of token A and of token B as the two columns of head tq4
                 xA = __byte_perm(hi, lo, 0x5410);
                 xB = __byte_perm(hi, lo, 0x7632);
-                if (4 * nt + tq4 >= G) xA = xB = 0u;
                 pb[nt][0] = movmatrix_t(xA);
                 pb[nt][1] = movmatrix_t(xB);
             }
@@ -349,6 +357,13 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) mma16816(o[nt][kc], va, pb[nt][0], pb[nt][1]);
             }
+        };
+        if (nvalid == kChunk) {
+            tile(0, std::false_type{});
+            tile(1, std::false_type{});
+        } else {
+            tile(0, std::true_type{});
+            if (nvalid > 16) tile(1, std::true_type{});
         }
         __syncwarp();
         if (lane == 0 && i + kStages < nmine) {
