@@ -41,8 +41,10 @@ BYTES_PER_TOKEN_HEAD = {128: 68 + 50, 256: 132 + 98}      # packed K + V record 
 ENCODE_BYTES_PER_VECTOR = {("k", 128): 68, ("v", 128): 50}
 
 # DRAM traffic of the split-K kernel from one ncu capture, valid only while the
-# kernel source is unchanged (sha256 of csrc/tq_decode.cu at capture time).
-NCU_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None, "capture": None}
+# kernel source is unchanged (sha256 of csrc/tq_decode_mma.cu at capture time).
+NCU_TRAFFIC = {"source_sha256": "376492f8052cd60f6a3cdf698519890fad13557c45bc940f971ee97d98da8081",
+               "bytes_per_launch": 390568192,
+               "capture": "profiles/tq_decode_mma128_long_context_b4_hq16_hkv8_t102400.md"}
 
 
 def peaks():
@@ -328,8 +330,8 @@ def run_ours(args, rank: int, world: int, dist):
 
     peak, peak_kind = peaks()
     achieved = bytes_step / (kern_ms * 1e-3) / 1e9
-    traffic = NCU_TRAFFIC["bytes_per_launch"] if NCU_TRAFFIC["source_sha256"] == source_sha(
-        "kv_cache_vector_14_b200/csrc/tq_decode.cu") else None
+    traffic = NCU_TRAFFIC["bytes_per_launch"] if (path == "mma" and NCU_TRAFFIC["source_sha256"] == source_sha(
+        "kv_cache_vector_14_b200/csrc/tq_decode_mma.cu")) else None
 
     cpu = None
     enc_cpu = None
