@@ -107,6 +107,23 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# ----------------------------------------------------------------------------- multi-rank plumbing
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """Largest value of x over all ranks (x itself without a process group)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, seconds_local: float, world: int, dist, device) -> float:
+    """Units per second of the whole job: every rank's units over the slowest rank's time."""
+    return world * units_per_rank / max_over_ranks(seconds_local, dist, device)
+
+
 # ----------------------------------------------------------------------------- CPU oracle (baseline)
 
 def oracle_decode_rate(w, seconds: float, tokens: int | None = None):
@@ -232,12 +249,6 @@ def run_ours(args, rank: int, world: int, dist):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     for _ in range(args.warmup):
         step(k_new, v_new, q, out)
@@ -268,10 +279,10 @@ def run_ours(args, rank: int, world: int, dist):
     tq.tq_set_decode_events(h, None, None)
     clocks = sampler.stop() if sampler else None
     ms = e0.elapsed_time(e1) / args.steps
-    ms_max = max_over_ranks(ms)
+    ms_max = max_over_ranks(ms, dist, dev)
     kern_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
     bytes_step = B * Hkv * T * BYTES_PER_TOKEN_HEAD[d]
-    value = world * bytes_step / (ms_max * 1e-3) / 1e9
+    value = whole_job_rate(bytes_step, ms * 1e-3, world, dist, dev) / 1e9
 
     # ---- end to end: pinned host inputs copied in, the output read back, every step
     kh = k_new.cpu().pin_memory()
@@ -294,8 +305,9 @@ def run_ours(args, rank: int, world: int, dist):
         oh.copy_(out, non_blocking=True)
     e3.record()
     torch.cuda.synchronize()
-    ms_e2e = max_over_ranks(e2.elapsed_time(e3) / n_e2e)
-    e2e_value = world * bytes_step / (ms_e2e * 1e-3) / 1e9
+    ms_e2e_local = e2.elapsed_time(e3) / n_e2e
+    ms_e2e = max_over_ranks(ms_e2e_local, dist, dev)
+    e2e_value = whole_job_rate(bytes_step, ms_e2e_local * 1e-3, world, dist, dev) / 1e9
     h2d = (kh.numel() + vh.numel()) * 4 + qh.numel() * 2
     d2h = oh.numel() * 4
 
@@ -324,8 +336,7 @@ def run_ours(args, rank: int, world: int, dist):
     nvec = 2 * we.B * we.Hkv * we.T
     enc_bytes = we.B * we.Hkv * we.T * (2 * we.d * 2 + ENCODE_BYTES_PER_VECTOR[("k", 128)] +
                                         ENCODE_BYTES_PER_VECTOR[("v", 128)])
-    enc_mvps = max_over_ranks(enc_med)
-    enc_mvps = world * nvec / (enc_mvps * 1e-3) / 1e6
+    enc_mvps = whole_job_rate(nvec, enc_med * 1e-3, world, dist, dev) / 1e6
     del xk, xv, flush
 
     peak, peak_kind = peaks()
