@@ -101,7 +101,9 @@ tq_status encode_common(const tq_handle* h, const void* x, tq_dtype dt, int64_t 
     a.B = B; a.Hkv = Hkv; a.Tnew = Tnew; a.t0 = t0;
     a.NB = c->Tcap / kBlockT;
     a.cache = static_cast<uint8_t*>(c->base);
-    a.dsign = h->dsign; a.sthr = h->dSThr; a.cb = h->cb;
+    a.dsign = h->dsign; a.sthr = h->dSThr; a.bimg = h->dSB; a.err = h->derr; a.cb = h->cb;
+    const int64_t es = (int64_t)dtype_size(dt);
+    a.vec16 = (aligned(x, 16) && (sb * es) % 16 == 0 && (sh * es) % 16 == 0 && (st * es) % 16 == 0) ? 1 : 0;
     return cuda_status(launch_encode(h->d, is_k, dt, a, h->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
@@ -169,12 +171,32 @@ tq_status tq_init(int head_dim, uint64_t seed, tq_handle** out) {
                 const int row = slot_coord(r / 4, r % 4, 2 * (l & 15) + (l >> 4));
                 sthr[((size_t)j * R + r) * 32 + l] = h->hS[(size_t)row * d + j];
             }
+    // d = 128: the JL matrix as the B operand of the tensor-core encode, rows
+    // permuted into sign-word order, fp16 hi and lo limbs of each fp32 entry
+    std::vector<uint16_t> simg;
+    if (d == 128) {
+        simg.assign((size_t)2 * kTcRows * d, 0);
+        for (int n = 0; n < d; ++n) {
+            const int row = qjl_row_of_column(n);
+            for (int k = 0; k < d; ++k) {
+                const double sv = (double)h->hS[(size_t)row * d + k];
+                const uint16_t hi = double_to_half_bits(sv);
+                const uint16_t lo = double_to_half_bits(sv - half_bits_to_double(hi));
+                const size_t at = sw128_k_offset(n, k) / 2;
+                simg[at] = hi;
+                simg[(size_t)kTcRows * d + at] = lo;
+            }
+        }
+    }
     cudaError_t e = cudaGetDevice(&h->device);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device);
     if (e == cudaSuccess) e = cudaMalloc(&h->dsign, sizeof(float) * d);
     if (e == cudaSuccess) e = cudaMalloc(&h->dST, sizeof(float) * d * d);
     if (e == cudaSuccess) e = cudaMalloc(&h->dSThr, sizeof(float) * d * d);
     if (e == cudaSuccess) e = cudaMalloc(&h->derr, sizeof(int));
+    if (e == cudaSuccess && !simg.empty()) e = cudaMalloc(&h->dSB, simg.size() * sizeof(uint16_t));
+    if (e == cudaSuccess && !simg.empty())
+        e = cudaMemcpy(h->dSB, simg.data(), simg.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(h->dsign, sign.data(), sizeof(float) * d, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(h->dST, st.data(), sizeof(float) * d * d, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(h->dSThr, sthr.data(), sizeof(float) * d * d, cudaMemcpyHostToDevice);
@@ -192,6 +214,7 @@ tq_status tq_destroy(tq_handle* h) {
     cudaFree(h->dsign);
     cudaFree(h->dST);
     cudaFree(h->dSThr);
+    cudaFree(h->dSB);
     cudaFree(h->derr);
     delete h;
     return TQ_OK;

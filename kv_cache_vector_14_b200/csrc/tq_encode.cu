@@ -412,7 +412,7 @@ cudaError_t launch_enc_dt(tq_dtype dt, const EncArgs& a, int num_sms, cudaStream
 }  // namespace
 
 cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, cudaStream_t s) {
-    if (d == 128) return is_k ? launch_enc_dt<128, true>(dt, a, num_sms, s) : launch_enc_dt<128, false>(dt, a, num_sms, s);
+    if (d == 128) return launch_encode128(is_k, dt, a, num_sms, s);
     if (d == 256) return is_k ? launch_enc_dt<256, true>(dt, a, num_sms, s) : launch_enc_dt<256, false>(dt, a, num_sms, s);
     return cudaErrorInvalidValue;
 }

@@ -29,6 +29,7 @@ struct Codebook {
 // Host-side generation of the constants (tq_params.cpp).
 bool make_params(int d, uint64_t seed, int8_t* D, float* S, float* c8, float* b7);
 uint16_t double_to_half_bits(double x);
+double half_bits_to_double(uint16_t h);
 
 // Byte sizes of the block fields.
 __host__ __device__ inline int64_t code_bytes(int d) { return 3LL * d / 8; }          // per token
@@ -48,6 +49,23 @@ __host__ __device__ inline int slot_coord(int s, int t, int i) {
     return 128 * s + 16 * (i >> 2) + 2 * t + (i & 1) + 8 * ((i >> 1) & 1);
 }
 
+// Tensor-core K encode (d = 128): operands of 128 rows x 128 fp16 columns in
+// the 128-byte-swizzled K-major shared-memory layout (8-row groups of 1024
+// bytes; 16-byte chunk c of row r stored at chunk c ^ (r & 7); columns 64..127
+// in a second 16 KB half).
+constexpr int kTcRows = 128;
+__host__ __device__ inline uint32_t sw128_k_offset(int row, int k) {
+    return (uint32_t)((k >> 6) * (kTcRows * 128) + (row >> 3) * 1024 + (row & 7) * 128 +
+                      ((((k & 63) >> 3) ^ (row & 7)) << 4) + (k & 7) * 2);
+}
+// JL row whose projection lands in column n of the product: bit n % 32 of
+// stored sign word n / 32 (d = 128: word t = slot t, bit q -> position 2q,
+// bit 16 + q -> position 2q + 1).
+__host__ __device__ inline int qjl_row_of_column(int n) {
+    const int b = n & 31;
+    return slot_coord(0, n >> 5, b < 16 ? 2 * b : 2 * (b - 16) + 1);
+}
+
 struct EncArgs {
     const void* x;
     int64_t sb, sh, st;
@@ -56,6 +74,9 @@ struct EncArgs {
     uint8_t* cache;
     const float* dsign;       // [d] +-1
     const float* sthr;        // [d][d/32][32] JL matrix, encode lane order
+    const uint8_t* bimg;      // d = 128: JL matrix as tensor-core operand (hi, lo fp16 limbs)
+    int* err;                 // device check word
+    int vec16;                // every input row starts on a 16-byte boundary
     Codebook cb;
 };
 
@@ -103,6 +124,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 // Kernel launchers (tq_encode.cu, tq_decode.cu); return a CUDA error code.
 cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms,
                           cudaStream_t s);
+cudaError_t launch_encode128(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, cudaStream_t s);
 cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, const float* dsign,
                             const float* st, float* qp, float* up, cudaStream_t s);
 cudaError_t launch_decode(int d, int G, bool use_mma, const DecArgs& a, cudaStream_t s);
@@ -127,6 +149,7 @@ struct tq_handle {
     float* dsign = nullptr;   // [d]
     float* dST = nullptr;     // [d][m] transposed S (query prologue)
     float* dSThr = nullptr;   // [d][d/32][32] encode lane order
+    uint8_t* dSB = nullptr;   // d = 128: JL operand image for the tensor-core encode (64 KB)
     int* derr = nullptr;
     tqi::Codebook cb{};
     cudaEvent_t ev_start = nullptr;   // optional timing of the split-K kernel

@@ -81,7 +81,7 @@ uint16_t double_to_half_bits(double x) {
     return (uint16_t)(sgn | q);                      // q == 1024 is the smallest normal
 }
 
-static double half_bits_to_double(uint16_t h) {
+double half_bits_to_double(uint16_t h) {
     int e = (h >> 10) & 31, f = h & 1023;
     double v = (e == 0) ? std::ldexp((double)f, -24) : std::ldexp((double)(1024 + f), e - 25);
     return (h & 0x8000) ? -v : v;
