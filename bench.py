@@ -215,6 +215,44 @@ def run_reference(args, rank: int, world: int):
 
 # ----------------------------------------------------------------------------- our arm
 
+def measure_encode(h, dev, world: int, dist, passes: int = 30) -> dict:
+    """Encode-only workload (B=1, 8 kv heads, 32768 bf16 tokens): K and V of
+    every token per pass, L2 flushed between passes.  Returns the fields of the
+    'encode' object."""
+    import torch
+    from kv_cache_vector_14_b200 import tq
+    we = synthetic.WORKLOADS["c2"]
+    xk = torch.from_numpy(synthetic.kv(we, "k")).to(dev).to(torch.bfloat16)
+    xv = torch.from_numpy(synthetic.kv(we, "v")).to(dev).to(torch.bfloat16)
+    ekc = tq.Cache(we.d, True, we.B, we.Hkv, we.T)
+    evc = tq.Cache(we.d, False, we.B, we.Hkv, we.T)
+    for _ in range(3):
+        tq.tq_encode_k(h, xk, ekc, 0)
+        tq.tq_encode_v(h, xv, evc, 0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)      # 2x L2: evict between passes
+    enc_ms, k_ms = [], []
+    for _ in range(passes):
+        flush.zero_()
+        a, m, b = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record()
+        tq.tq_encode_k(h, xk, ekc, 0)
+        m.record()
+        tq.tq_encode_v(h, xv, evc, 0)
+        b.record()
+        torch.cuda.synchronize()
+        enc_ms.append(a.elapsed_time(b))
+        k_ms.append(a.elapsed_time(m))
+    enc_med = statistics.median(enc_ms)
+    nvec = 2 * we.B * we.Hkv * we.T
+    enc_bytes = we.B * we.Hkv * we.T * (2 * we.d * 2 + ENCODE_BYTES_PER_VECTOR[("k", 128)] +
+                                        ENCODE_BYTES_PER_VECTOR[("v", 128)])
+    enc_mvps = whole_job_rate(nvec, enc_med * 1e-3, world, dist, dev) / 1e6
+    return {"workload": we.title, "value": enc_mvps, "unit": "Mvectors/s", "ms_per_pass": enc_med,
+            "k_ms": statistics.median(k_ms), "vectors_per_pass": nvec, "algorithmic_bytes_per_pass": enc_bytes,
+            "achieved_gbs": enc_bytes / (enc_med * 1e-3) / 1e9,
+            "l2": "256 MB buffer written between passes"}
+
+
 def run_ours(args, rank: int, world: int, dist):
     import torch
     from kv_cache_vector_14_b200 import build, tq
@@ -225,6 +263,12 @@ def run_ours(args, rank: int, world: int, dist):
     w = synthetic.WORKLOADS["c4"]
     d, B, Hq, Hkv, T = w.d, w.B, w.Hq, w.Hkv, w.T
     h = tq.tq_init(d, 0)
+    if args.only == "encode":          # profiling aid: the encode-only workload alone
+        enc = measure_encode(h, dev, world, dist, passes=args.steps)
+        tq.tq_destroy(h)
+        if rank == 0:
+            print(json.dumps({"encode": enc}), flush=True)
+        return
     kc, vc = tq.Cache(d, True, B, Hkv, T), tq.Cache(d, False, B, Hkv, T)
     for which, cache in (("k", kc), ("v", vc)):
         x = torch.from_numpy(synthetic.kv(w, which)).to(dev)
@@ -311,33 +355,7 @@ def run_ours(args, rank: int, world: int, dist):
     h2d = (kh.numel() + vh.numel()) * 4 + qh.numel() * 2
     d2h = oh.numel() * 4
 
-    # ---- encode-only workload: KV encode throughput
-    we = synthetic.WORKLOADS["c2"]
-    xk = torch.from_numpy(synthetic.kv(we, "k")).to(dev).to(torch.bfloat16)
-    xv = torch.from_numpy(synthetic.kv(we, "v")).to(dev).to(torch.bfloat16)
-    ekc = tq.Cache(we.d, True, we.B, we.Hkv, we.T)
-    evc = tq.Cache(we.d, False, we.B, we.Hkv, we.T)
-    for _ in range(3):
-        tq.tq_encode_k(h, xk, ekc, 0)
-        tq.tq_encode_v(h, xv, evc, 0)
-    n_enc = 30
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)      # 2x L2: evict between passes
-    enc_ms = []
-    for _ in range(n_enc):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        tq.tq_encode_k(h, xk, ekc, 0)
-        tq.tq_encode_v(h, xv, evc, 0)
-        b.record()
-        torch.cuda.synchronize()
-        enc_ms.append(a.elapsed_time(b))
-    enc_med = statistics.median(enc_ms)
-    nvec = 2 * we.B * we.Hkv * we.T
-    enc_bytes = we.B * we.Hkv * we.T * (2 * we.d * 2 + ENCODE_BYTES_PER_VECTOR[("k", 128)] +
-                                        ENCODE_BYTES_PER_VECTOR[("v", 128)])
-    enc_mvps = whole_job_rate(nvec, enc_med * 1e-3, world, dist, dev) / 1e6
-    del xk, xv, flush
+    enc = measure_encode(h, dev, world, dist)
 
     peak, peak_kind = peaks()
     achieved = bytes_step / (kern_ms * 1e-3) / 1e9
@@ -349,7 +367,7 @@ def run_ours(args, rank: int, world: int, dist):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample, _ = oracle_decode_rate(w, args.cpu_seconds)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
-        ev_, ecores, esample = oracle_encode_rate(we, min(10.0, args.cpu_seconds))
+        ev_, ecores, esample = oracle_encode_rate(synthetic.WORKLOADS["c2"], min(10.0, args.cpu_seconds))
         enc_cpu = {"value": ev_, "unit": "Mvectors/s", "cores": ecores, "kind": "oracle", "sample": esample}
 
     status = tq.tq_device_status(h)
@@ -374,11 +392,7 @@ def run_ours(args, rank: int, world: int, dist):
                 "ms_per_step": ms_e2e},
         "gpu_launches": 5 * args.steps,
         "clocks": clocks,
-        "encode": {"workload": we.title, "value": enc_mvps, "unit": "Mvectors/s", "ms_per_pass": enc_med,
-                   "vectors_per_pass": nvec, "algorithmic_bytes_per_pass": enc_bytes,
-                   "achieved_gbs": enc_bytes / (enc_med * 1e-3) / 1e9,
-                   "frac": enc_bytes / (enc_med * 1e-3) / 1e9 / peak, "l2": "256 MB buffer written between passes",
-                   "cpu_baseline": enc_cpu},
+        "encode": {**enc, "frac": enc["achieved_gbs"] / peak, "cpu_baseline": enc_cpu},
         "device_status": tq.tq_status_string(status),
     }
     print(json.dumps(line), flush=True)
@@ -392,6 +406,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["encode"], default=None,
+                    help="run only the encode-only workload (--steps passes); for profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

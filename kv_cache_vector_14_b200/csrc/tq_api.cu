@@ -104,6 +104,9 @@ tq_status encode_common(const tq_handle* h, const void* x, tq_dtype dt, int64_t 
     a.dsign = h->dsign; a.sthr = h->dSThr; a.bimg = h->dSB; a.err = h->derr; a.cb = h->cb;
     const int64_t es = (int64_t)dtype_size(dt);
     a.vec16 = (aligned(x, 16) && (sb * es) % 16 == 0 && (sh * es) % 16 == 0 && (st * es) % 16 == 0) ? 1 : 0;
+    if (B * Hkv * Tnew >= (int64_t)1 << 31) return TQ_ERR_UNSUPPORTED;      // vector indices are 32-bit
+    a.fdT = make_fastdiv((uint32_t)Tnew);
+    a.fdH = make_fastdiv((uint32_t)Hkv);
     return cuda_status(launch_encode(h->d, is_k, dt, a, h->num_sms, static_cast<cudaStream_t>(stream)));
 }
 

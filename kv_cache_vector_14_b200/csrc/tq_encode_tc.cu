@@ -29,7 +29,10 @@
 // segment of Z (one sign word of one vector) and sets bit b when z >= 0.
 //
 // One tile of tile_rows vectors per CTA iteration; the CTA (16 warps, one per
-// SM) stages the JL limbs once (one bulk copy) and loops over tiles.  Small
+// SM) stages the JL limbs once (one bulk copy) and loops over tiles.  The
+// residual operand and the accumulator are double-buffered: the mma of tile i
+// runs while the warps compute steps 1-4 of tile i + 1, and its sign words are
+// read out after that.  Small
 // encodes (one new token per head) use short tiles so that they spread over
 // many SMs; every vector goes through the same instructions whatever its row,
 // so bulk encodes and one-token appends store identical bytes.
@@ -45,12 +48,13 @@ constexpr int kOpBytes = kTcRows * kD * 2;      // one fp16 limb of a 128 x 128 
 constexpr float kRScale = 4096.f;               // residual scale before the fp16 split
 constexpr int kWaitLimit = 1 << 20;
 
-constexpr int kOffAhi = 0;
-constexpr int kOffAlo = kOpBytes;
-constexpr int kOffBhi = 2 * kOpBytes;           // B image (hi then lo), one bulk copy
-constexpr int kOffCode = 4 * kOpBytes;          // [128 rows][128] code bytes in slot order
-constexpr int kOffBar = kOffCode + kTcRows * 128;
+constexpr int kOffA = 0;                        // two residual buffers, each hi then lo limb
+constexpr int kABytes = 2 * kOpBytes;
+constexpr int kOffBhi = 2 * kABytes;            // B image (hi then lo), one bulk copy
+constexpr int kOffCode = kOffBhi + 2 * kOpBytes; // [16 warps][4 vectors][128] code bytes in slot order
+constexpr int kOffBar = kOffCode + kWarps * 4 * 128;
 constexpr int kSmemK = kOffBar + 64 + 1024;     // + slack to align the base to 1024 bytes
+static_assert(kSmemK <= 227 * 1024, "shared memory per CTA");
 
 // instruction descriptor: D fp32, A and B fp16, both K-major, N = 128, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kD >> 3) << 17) | ((uint32_t)(kTcRows >> 4) << 24);
@@ -292,14 +296,31 @@ __device__ __forceinline__ uint32_t pack_code_word(const uint8_t* rec, int w) {
     return main | (((tail >> g) & 0x11111111u) << 3);
 }
 
-__device__ __forceinline__ int64_t x_offset(const EncArgs& a, int64_t gv) {
-    const int64_t tt = gv % a.Tnew, bh = gv / a.Tnew;
-    return (bh / a.Hkv) * a.sb + (bh % a.Hkv) * a.sh + tt * a.st;
-}
-__device__ __forceinline__ uint8_t* token_block(const EncArgs& a, int64_t gv, int64_t bb, int& tau) {
-    const int64_t tt = gv % a.Tnew, bh = gv / a.Tnew, t = a.t0 + tt;
+// Input offset and cache block of vector gv (b, h, token order).
+__device__ __forceinline__ void locate(const EncArgs& a, uint32_t gv, int64_t bb, int64_t& xoff, uint8_t*& blk,
+                                       int& tau) {
+    const uint32_t bh = fdiv(gv, a.fdT);
+    const uint32_t tt = gv - bh * (uint32_t)a.Tnew;
+    const uint32_t b = fdiv(bh, a.fdH);
+    const uint32_t hh = bh - b * (uint32_t)a.Hkv;
+    xoff = (int64_t)b * a.sb + (int64_t)hh * a.sh + (int64_t)tt * a.st;
+    const int64_t t = a.t0 + tt;
     tau = (int)(t & 63);
-    return a.cache + (bh * a.NB + (t >> 6)) * bb;
+    blk = a.cache + ((int64_t)bh * a.NB + (t >> 6)) * bb;
+}
+
+// The 12 code words of each of the warp's four vectors (group g holds vector
+// g; my_rec is the code record of this lane's vector) from the staged bytes.
+__device__ __forceinline__ void store_code_words(const uint8_t* stage, uint8_t* my_rec, int nvalid, int lane) {
+    const unsigned long long mine = reinterpret_cast<unsigned long long>(my_rec);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int idx = lane + 32 * k;                 // 4 vectors x 12 words
+        const int vv = idx / 12, w = idx % 12;
+        const unsigned long long rec = __shfl_sync(kFull, mine, 8 * (vv < 4 ? vv : 3));
+        if (idx < 48 && vv < nvalid)
+            reinterpret_cast<uint32_t*>(rec)[w] = pack_code_word(stage + vv * 128, w);
+    }
 }
 
 // ---------------------------------------------------------------- K kernel
@@ -309,8 +330,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     const uint32_t sbase = smem_u32(sm);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);     // [0] JL image copy, [1] mma done
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffBar + 16);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);     // [0] JL image copy, [1..2] mma done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffBar + 32);
     uint8_t* scode = sm + kOffCode;
     __shared__ float sC[8];
 
@@ -318,16 +339,17 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
     const int64_t N = a.B * a.Hkv * a.Tnew;
     const int64_t ntiles = (N + tile_rows - 1) / tile_rows;
     const int64_t bb = block_bytes(kD, true);
-    const uint32_t bar_b = smem_u32(&bars[0]), bar_mma = smem_u32(&bars[1]);
+    const uint32_t bar_b = smem_u32(&bars[0]);
 
     if (threadIdx.x < 8) sC[threadIdx.x] = a.cb.c[threadIdx.x];
     if (threadIdx.x == 0) {
         mbar_init(bar_b, 1);
-        mbar_init(bar_mma, 1);
+        mbar_init(smem_u32(&bars[1]), 1);
+        mbar_init(smem_u32(&bars[2]), 1);
         fence_mbar_init();
     }
     if (warp == 0) {
-        tc_alloc(smem_u32(tmem_slot), kTcRows);        // 128 fp32 columns: Z for one tile
+        tc_alloc(smem_u32(tmem_slot), 2 * kTcRows);    // two 128-column fp32 accumulators
         tc_relinquish();
     }
     tc_fence_before();
@@ -348,37 +370,75 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
         if (threadIdx.x == 0) atomicExch(a.err, 1);
         mbar_wait_bounded(bar_b, 0);
     }
-    uint32_t phase = 0;
+    uint32_t phases = 0;                 // bit j: parity of the next completion of buffer j
+    int64_t prev_row0 = -1;
+    int prev_nrows = 0, buf = 0;
+
+    // sign words of the tile held in accumulator pb: warp w reads lanes
+    // 32 (w & 3) .. + 31 and columns 32 (w >> 2) .. + 31 (one word per thread)
+    auto finish = [&](int pb, int64_t r0, int nr) -> bool {
+        const uint32_t bar = smem_u32(&bars[1 + pb]);
+        const bool ok = mbar_wait_bounded(bar, (phases >> pb) & 1u);
+        if (__syncthreads_or(!ok)) {
+            if (threadIdx.x == 0) atomicExch(a.err, 1);
+            mbar_wait_bounded(bar, (phases >> pb) & 1u);
+            return false;
+        }
+        phases ^= 1u << pb;
+        tc_fence_after();
+        uint32_t z[32];
+        tc_load32(tmem + (uint32_t)(pb * kTcRows) + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(32 * (warp >> 2)),
+                  z);
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 32; ++b) word |= (__uint_as_float(z[b]) >= 0.f ? 1u : 0u) << b;
+        const int v = 32 * (warp & 3) + lane;
+        if (v < nr) {
+            int64_t xoff;
+            uint8_t* blk;
+            int tau;
+            locate(a, (uint32_t)(r0 + v), bb, xoff, blk, tau);
+            reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(kD) + tau * sign_bytes(kD))[warp >> 2] = word;
+        }
+        tc_fence_before();
+        return true;
+    };
+
     for (int64_t tile = blockIdx.x; tile < ntiles && !failed; tile += gridDim.x) {
         const int64_t row0 = tile * tile_rows;
         const int nrows = (int)((N - row0) < tile_rows ? (N - row0) : tile_rows);
-        // ---- steps 1-4: pass p, warp w: tile rows 64 p + 4 w + g
+        uint8_t* A = sm + kOffA + buf * kABytes;
+        // ---- steps 1-4: pass p, warp w: tile rows 64 p + 4 w + g; code words stored per pass
+        uint8_t* stage = scode + warp * 4 * 128;
 #pragma unroll
         for (int p = 0; p < 2; ++p) {
             const int r0 = 64 * p + 4 * warp;
             if (r0 >= nrows) break;                        // warp-uniform
             const int v = r0 + g;
             const bool valid = v < nrows;
-            const int64_t gv = row0 + (valid ? v : 0);
+            int64_t xoff;
+            uint8_t* blk;
+            int tau;
+            locate(a, (uint32_t)(row0 + (valid ? v : r0)), bb, xoff, blk, tau);
             GroupOut o;
-            encode_group<DT, true>(a.x, x_offset(a, gv), valid, vec, l, dsg, a.cb, sC, o);
-            *reinterpret_cast<uint4*>(sm + kOffAhi + sw128_k_offset(v, 16 * l)) =
-                make_uint4(o.rh[0], o.rh[1], o.rh[2], o.rh[3]);
-            *reinterpret_cast<uint4*>(sm + kOffAhi + sw128_k_offset(v, 16 * l + 8)) =
+            encode_group<DT, true>(a.x, xoff, valid, vec, l, dsg, a.cb, sC, o);
+            *reinterpret_cast<uint4*>(A + sw128_k_offset(v, 16 * l)) = make_uint4(o.rh[0], o.rh[1], o.rh[2], o.rh[3]);
+            *reinterpret_cast<uint4*>(A + sw128_k_offset(v, 16 * l + 8)) =
                 make_uint4(o.rh[4], o.rh[5], o.rh[6], o.rh[7]);
-            *reinterpret_cast<uint4*>(sm + kOffAlo + sw128_k_offset(v, 16 * l)) =
+            *reinterpret_cast<uint4*>(A + kOpBytes + sw128_k_offset(v, 16 * l)) =
                 make_uint4(o.rl[0], o.rl[1], o.rl[2], o.rl[3]);
-            *reinterpret_cast<uint4*>(sm + kOffAlo + sw128_k_offset(v, 16 * l + 8)) =
+            *reinterpret_cast<uint4*>(A + kOpBytes + sw128_k_offset(v, 16 * l + 8)) =
                 make_uint4(o.rl[4], o.rl[5], o.rl[6], o.rl[7]);
 #pragma unroll
-            for (int t = 0; t < 4; ++t) *reinterpret_cast<uint32_t*>(scode + v * 128 + t * 32 + 4 * l) = o.cw[t];
+            for (int t = 0; t < 4; ++t) *reinterpret_cast<uint32_t*>(stage + g * 128 + t * 32 + 4 * l) = o.cw[t];
             if (valid && l == 0) {
-                int tau;
-                uint8_t* blk = token_block(a, gv, bb, tau);
                 __half* nf = reinterpret_cast<__half*>(blk + kBlockT * (code_bytes(kD) + sign_bytes(kD)));
                 nf[tau] = __float2half_rn(o.n);
                 nf[kBlockT + tau] = __float2half_rn(sqrtf(o.g2));
             }
+            __syncwarp();
+            store_code_words(stage, blk + tau * code_bytes(kD), nrows - r0, lane);
+            __syncwarp();
         }
         // ---- step 5 on the tensor core: Z = R_hi S_hi^T + R_hi S_lo^T + R_lo S_hi^T
         fence_proxy_async();
@@ -386,60 +446,39 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
         __syncthreads();
         if (threadIdx.x == 0) {
             tc_fence_after();
+            const uint32_t abase = sbase + kOffA + buf * kABytes, d_tmem = tmem + (uint32_t)(buf * kTcRows);
 #pragma unroll
             for (int ks = 0; ks < kD / 16; ++ks) {
                 const uint32_t koff = (uint32_t)((ks >> 2) * (kTcRows * 128) + (ks & 3) * 32);
-                const uint64_t ah = sw128_desc(sbase + kOffAhi + koff), al = sw128_desc(sbase + kOffAlo + koff);
+                const uint64_t ah = sw128_desc(abase + koff), al = sw128_desc(abase + kOpBytes + koff);
                 const uint64_t bh = sw128_desc(sbase + kOffBhi + koff);
                 const uint64_t bl = sw128_desc(sbase + kOffBhi + kOpBytes + koff);
-                tc_mma(tmem, ah, bh, ks > 0 ? 1u : 0u);
-                tc_mma(tmem, ah, bl, 1u);
-                tc_mma(tmem, al, bh, 1u);
+                tc_mma(d_tmem, ah, bh, ks > 0 ? 1u : 0u);
+                tc_mma(d_tmem, ah, bl, 1u);
+                tc_mma(d_tmem, al, bh, 1u);
             }
-            tc_commit(bar_mma);
+            tc_commit(smem_u32(&bars[1 + buf]));
         }
-        // ---- code words of this warp's rows (overlaps the mma)
-        __syncwarp();
-#pragma unroll
-        for (int k = 0; k < 3; ++k) {
-            const int idx = lane + 32 * k;                 // 8 rows x 12 words
-            const int vv = idx / 12, w = idx % 12;
-            const int v = 64 * (vv >> 2) + 4 * warp + (vv & 3);
-            if (v < nrows) {
-                int tau;
-                uint8_t* blk = token_block(a, row0 + v, bb, tau);
-                reinterpret_cast<uint32_t*>(blk + tau * code_bytes(kD))[w] = pack_code_word(scode + v * 128, w);
-            }
-        }
-        // ---- sign words: warp w reads lanes 32 (w & 3) .. + 31, columns 32 (w >> 2) .. + 31
-        const bool ok = mbar_wait_bounded(bar_mma, phase);
-        if (__syncthreads_or(!ok)) {
+        // ---- sign words of the previous tile (its mma ran under steps 1-4 above)
+        if (prev_row0 >= 0 && !finish(buf ^ 1, prev_row0, prev_nrows)) {
             failed = true;
-            if (threadIdx.x == 0) atomicExch(a.err, 1);
-            mbar_wait_bounded(bar_mma, phase);
             break;
         }
-        phase ^= 1u;
-        tc_fence_after();
-        uint32_t z[32];
-        tc_load32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(32 * (warp >> 2)), z);
-        uint32_t word = 0;
-#pragma unroll
-        for (int b = 0; b < 32; ++b) word |= (__uint_as_float(z[b]) >= 0.f ? 1u : 0u) << b;
-        const int v = 32 * (warp & 3) + lane;
-        if (v < nrows) {
-            int tau;
-            uint8_t* blk = token_block(a, row0 + v, bb, tau);
-            reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(kD) + tau * sign_bytes(kD))[warp >> 2] = word;
-        }
-        tc_fence_before();
-        __syncthreads();
+        prev_row0 = row0;
+        prev_nrows = nrows;
+        buf ^= 1;
+    }
+    if (failed) {
+        // a timed-out wait: let any mma still in flight finish before releasing tensor memory
+        for (int pb = 0; pb < 2; ++pb) mbar_wait_bounded(smem_u32(&bars[1 + pb]), (phases >> pb) & 1u);
+    } else if (prev_row0 >= 0) {
+        failed = !finish(buf ^ 1, prev_row0, prev_nrows);
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tc_dealloc(tmem, kTcRows);
+        tc_dealloc(tmem, 2 * kTcRows);
     }
 }
 
@@ -447,7 +486,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
 constexpr int kVWarps = 8;
 
 template <int DT>
-__global__ void __launch_bounds__(kVWarps * 32) tq_encode_v128_kernel(const EncArgs a) {
+__global__ void __launch_bounds__(kVWarps * 32, 3) tq_encode_v128_kernel(const EncArgs a) {
     __shared__ __align__(16) uint8_t scode[kVWarps][4][128];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 3, l = lane & 7;
     const int64_t N = a.B * a.Hkv * a.Tnew;
@@ -460,27 +499,17 @@ __global__ void __launch_bounds__(kVWarps * 32) tq_encode_v128_kernel(const EncA
     for (int64_t q = (int64_t)blockIdx.x * kVWarps + warp; q < nquads; q += (int64_t)gridDim.x * kVWarps) {
         const int64_t gv0 = 4 * q;
         const bool valid = gv0 + g < N;
-        const int64_t gv = valid ? gv0 + g : gv0;
+        int64_t xoff;
+        uint8_t* blk;
+        int tau;
+        locate(a, (uint32_t)(valid ? gv0 + g : gv0), bb, xoff, blk, tau);
         GroupOut o;
-        encode_group<DT, false>(a.x, x_offset(a, gv), valid, vec, l, dsg, a.cb, nullptr, o);
+        encode_group<DT, false>(a.x, xoff, valid, vec, l, dsg, a.cb, nullptr, o);
 #pragma unroll
         for (int t = 0; t < 4; ++t) *reinterpret_cast<uint32_t*>(&scode[warp][g][t * 32 + 4 * l]) = o.cw[t];
-        if (valid && l == 0) {
-            int tau;
-            uint8_t* blk = token_block(a, gv, bb, tau);
-            reinterpret_cast<__half*>(blk + kBlockT * code_bytes(kD))[tau] = __float2half_rn(o.n);
-        }
+        if (valid && l == 0) reinterpret_cast<__half*>(blk + kBlockT * code_bytes(kD))[tau] = __float2half_rn(o.n);
         __syncwarp();
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const int idx = lane + 32 * k;                 // 4 vectors x 12 words
-            const int vv = idx / 12, w = idx % 12;
-            if (idx < 48 && gv0 + vv < N) {
-                int tau;
-                uint8_t* blk = token_block(a, gv0 + vv, bb, tau);
-                reinterpret_cast<uint32_t*>(blk + tau * code_bytes(kD))[w] = pack_code_word(&scode[warp][vv][0], w);
-            }
-        }
+        store_code_words(&scode[warp][0][0], blk + tau * code_bytes(kD), (int)(N - gv0 < 4 ? N - gv0 : 4), lane);
         __syncwarp();
     }
 }

@@ -66,6 +66,22 @@ __host__ __device__ inline int qjl_row_of_column(int n) {
     return slot_coord(0, n >> 5, b < 16 ? 2 * b : 2 * (b - 16) + 1);
 }
 
+// Division by a fixed divisor d >= 1 for dividends below 2^31:
+// q = umulhi(n, m) >> s with m = ceil(2^(31 + ceil(log2 d)) / d); m = 0 marks d = 1.
+struct FastDiv {
+    uint32_t m, s;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+    if (d <= 1) return {0u, 0u};
+    uint32_t l = 0;
+    while ((1ull << l) < d) ++l;
+    const uint64_t p = 31 + l;
+    return {(uint32_t)(((1ull << p) + d - 1) / d), (uint32_t)(p - 32)};
+}
+#ifdef __CUDACC__
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, FastDiv f) { return f.m ? (__umulhi(n, f.m) >> f.s) : n; }
+#endif
+
 struct EncArgs {
     const void* x;
     int64_t sb, sh, st;
@@ -77,6 +93,7 @@ struct EncArgs {
     const uint8_t* bimg;      // d = 128: JL matrix as tensor-core operand (hi, lo fp16 limbs)
     int* err;                 // device check word
     int vec16;                // every input row starts on a 16-byte boundary
+    FastDiv fdT, fdH;         // division by Tnew and by Hkv (vector counts below 2^31)
     Codebook cb;
 };
 
