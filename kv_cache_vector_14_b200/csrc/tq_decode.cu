@@ -289,7 +289,7 @@ template <int D, int DT>
 cudaError_t launch_prologue_t(int grid, size_t smem, const void* q, int64_t BHq, const float* dsign, const float* st,
                               float* qp, float* up, cudaStream_t s) {
     auto kern = tq_prologue_kernel<D, DT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_once<tq_prologue_kernel<D, DT>>((int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, D, smem, s>>>(q, BHq, dsign, st, qp, up);
     return cudaGetLastError();

@@ -434,7 +434,7 @@ template <int NT, int NW>
 cudaError_t launch_mma_t(const DecArgs& a, int G, cudaStream_t s) {
     const size_t smem = (size_t)NW * kStages * kStageB + (size_t)NW * kStages * 8;
     auto kern = tq_decode_mma128_kernel<NT, NW>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_smem_once<tq_decode_mma128_kernel<NT, NW>>((int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
     return launch_pdl(kern, grid, dim3(NW * 32), smem, s, a, G);

@@ -368,7 +368,7 @@ template <int D, bool IS_K, int DT, int TV>
 cudaError_t launch_enc_tv(const EncArgs& a, int num_sms, cudaStream_t s) {
     using SM = EncSmem<D, IS_K, TV>;
     auto kern = tq_encode_kernel<D, IS_K, DT, TV>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::total);
+    cudaError_t e = set_smem_once<tq_encode_kernel<D, IS_K, DT, TV>>((int)SM::total);
     if (e != cudaSuccess) return e;
     const int64_t N = a.B * a.Hkv * a.Tnew;
     const int64_t ntiles = (N + TV - 1) / TV;
@@ -389,7 +389,7 @@ cudaError_t launch_enc_t(const EncArgs& a, int num_sms, cudaStream_t s) {
             const unsigned grid = (unsigned)((N + kSmallWarps - 1) / kSmallWarps);
             const size_t smem = (size_t)((D == 128) ? 128 : 64) * D * sizeof(float);
             auto kern = tq_encode_k_small_kernel<D, DT>;
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            cudaError_t e = set_smem_once<tq_encode_k_small_kernel<D, DT>>((int)smem);
             if (e != cudaSuccess) return e;
             kern<<<grid, kSmallWarps * 32, smem, s>>>(a);
             return cudaGetLastError();

@@ -526,7 +526,7 @@ cudaError_t launch_t(bool is_k, const EncArgs& a, int num_sms, cudaStream_t s) {
         const int64_t ntiles = (N + rows - 1) / rows;
         const int grid = (int)(ntiles < num_sms ? ntiles : num_sms);
         auto kern = tq_encode_k128_tc_kernel<DT>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemK);
+        cudaError_t e = set_smem_once<tq_encode_k128_tc_kernel<DT>>(kSmemK);
         if (e != cudaSuccess) return e;
         kern<<<grid, kWarps * 32, kSmemK, s>>>(a, (int)rows);
         return cudaGetLastError();

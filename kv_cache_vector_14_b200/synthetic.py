@@ -130,6 +130,15 @@ def queries(w: Workload, step: int | None = None) -> np.ndarray:
     return np.ascontiguousarray(q)
 
 
+def queries_all(w: Workload) -> np.ndarray:
+    """Every step's queries at once, [steps, B, Hq, d] (same values as queries(w, s))."""
+    g = _streams(w.seed)[_Q]
+    qa = g.standard_normal((max(w.steps, 1), w.B, w.Hq, w.d), dtype=np.float32)
+    if w.q_dtype == "bf16":
+        qa = bf16_round(qa)
+    return np.ascontiguousarray(qa)
+
+
 def gaussian(shape, seed: int) -> np.ndarray:
     """Plain iid N(0,1) fp32 array for small ad-hoc cases."""
     return np.random.Generator(np.random.PCG64(seed)).standard_normal(shape, dtype=np.float32)

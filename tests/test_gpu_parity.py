@@ -217,6 +217,49 @@ def test_append_and_attend_loop_d256(handles, prms):
 
 
 @pytest.mark.parametrize("d", [128, 256])
+def test_append_and_attend_graph_replay_equals_eager(handles, d):
+    """The append-and-attend step sequence captured in a CUDA graph and
+    replayed gives the same outputs, bit for bit, as launching it eagerly."""
+    h = handles[d]
+    B, Hq, Hkv, T0, S = 2, 8, 2, 200, 12
+    Tcap = (T0 + S + 63) // 64 * 64
+    xk = torch_input(synthetic.gaussian((B, Hkv, T0 + S, d), seed=5), "f32")
+    xv = torch_input(synthetic.gaussian((B, Hkv, T0 + S, d), seed=6), "f32")
+    q = torch_input(synthetic.gaussian((S, B, Hq, d), seed=7), "bf16")
+    kc, vc = tq.Cache(d, True, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
+    tq.tq_encode_k(h, xk[:, :, :T0], kc, 0)
+    tq.tq_encode_v(h, xv[:, :, :T0], vc, 0)
+    ws = torch.empty(tq.tq_attend_workspace_bytes(h, B, Hq, Hkv, T0 + S), dtype=torch.uint8, device="cuda")
+    out = torch.zeros((S, B, Hq, d), dtype=torch.float32, device="cuda")
+
+    def sequence():
+        for s in range(S):
+            T = T0 + s
+            tq.tq_encode_k(h, xk[:, :, T:T + 1], kc, T)
+            tq.tq_encode_v(h, xv[:, :, T:T + 1], vc, T)
+            tq.tq_attend_decode(h, q[s], kc, vc, out[s], ws, T=T + 1, scale=1.0 / np.sqrt(d))
+
+    sequence()
+    torch.cuda.synchronize()
+    ref, kref, vref = out.clone(), kc.buf.clone(), vc.buf.clone()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        sequence()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        sequence()
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    assert torch.equal(kc.buf, kref) and torch.equal(vc.buf, vref)
+    assert tq.tq_device_status(h) == tq.TQ_OK
+    del g
+
+
+@pytest.mark.parametrize("d", [128, 256])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_attend_group_sizes_and_ragged_lengths(decode_path, handles, prms, d, G):
     Hkv, B, Tcap = 2, 3, 320
