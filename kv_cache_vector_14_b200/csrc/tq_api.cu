@@ -71,7 +71,7 @@ bool make_plan(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t T
     p->use_mma = !h->force_simt && mma_supported(d, p->G);
     const int64_t pairs = B * Hkv > 0 ? B * Hkv : 1;
     const int64_t cap = (int64_t)h->num_sms * decode_ctas_per_sm(p->use_mma);
-    const int chunk = decode_chunk_tokens(p->use_mma);
+    const int chunk = decode_chunk_tokens(d, p->use_mma);
     const int64_t nchunk = Tmax > 0 ? (Tmax + chunk - 1) / chunk : 1;
     p->nsplit = upper_bound ? (int)split_loop_bound(cap, pairs, nchunk)
                             : choose_nsplit(cap, decode_warps(p->use_mma, p->G), pairs, nchunk);

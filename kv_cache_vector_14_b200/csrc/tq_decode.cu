@@ -358,15 +358,15 @@ namespace tqi {
 
 cudaError_t launch_decode_simt(int d, int G, const DecArgs& a, cudaStream_t s);
 cudaError_t launch_decode_mma(int d, int G, const DecArgs& a, cudaStream_t s);
-int decode_mma_chunk_tokens();
+int decode_mma_chunk_tokens(int d);
 int decode_mma_warps(int G);
 
-// The tensor-core kernel covers head_dim 128 with up to 8 query heads per kv
-// head; other shapes take the SIMT kernel.
-bool mma_supported(int d, int G) { return d == 128 && G >= 1 && G <= 8; }
+// The tensor-core kernel covers head_dim 128 and 256 with up to 8 query heads
+// per kv head; other group sizes take the SIMT kernel.
+bool mma_supported(int d, int G) { return (d == 128 || d == 256) && G >= 1 && G <= 8; }
 
 int decode_ctas_per_sm(bool use_mma) { return use_mma ? 1 : 4; }
-int decode_chunk_tokens(bool use_mma) { return use_mma ? decode_mma_chunk_tokens() : kBlockT; }
+int decode_chunk_tokens(int d, bool use_mma) { return use_mma ? decode_mma_chunk_tokens(d) : kBlockT; }
 int decode_warps(bool use_mma, int G) { return use_mma ? decode_mma_warps(G) : 4; }
 
 cudaError_t launch_decode(int d, int G, bool use_mma, const DecArgs& a, cudaStream_t s) {

@@ -1,5 +1,5 @@
 // Tensor-core split-K decode attention over the packed TurboQuant cache
-// (head_dim 128, up to 8 query heads per kv head), for sm_100a.
+// (head_dim 128 or 256, up to 8 query heads per kv head), for sm_100a.
 //
 // Page "Apple Silicon向けSwiftLM、TurboQuant KVキャッシュ圧縮とSSD Expert
 // Streamingを実装" (ai-heartland.com), hybrid V2+V3 section: dequantisation is
@@ -26,11 +26,17 @@
 // bits come as one word shifted into the fp16 sign positions.  Value
 // fragments are produced key-style and transposed in registers (movmatrix).
 //
-// Data movement: each warp owns a ring of STAGES shared-memory buffers of 32
-// tokens (K codes, signs, norms, gammas, V codes, norms: six bulk copies,
-// cp.async.bulk with an mbarrier transaction count, no multicast).  Waits are
-// bounded: on timeout the kernel sets the handle's check word, waits (bounded)
-// for its own copies, and contributes an empty partial.
+// Data movement: each warp owns a ring of STAGES shared-memory buffers of a
+// chunk of tokens (32 at d = 128, 16 at d = 256; K codes, signs, norms,
+// gammas, V codes, norms: six bulk copies, cp.async.bulk with an mbarrier
+// transaction count, no multicast).  Waits are bounded: on timeout the kernel
+// sets the handle's check word, waits (bounded) for its own copies, and
+// contributes an empty partial.
+//
+// head_dim 256 is two 128-coordinate slices of the same record layout: the
+// k-loop runs over 16 coordinate chunks and 16 sign chunks, the value tile
+// over 16 coordinate tiles.  Its q'/u' fragments are read from shared memory
+// (filled once per CTA) instead of being held in registers.
 #include <type_traits>
 
 #include "tq_internal.h"
@@ -39,22 +45,31 @@ namespace tqi {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kD = 128;
 constexpr int kStages = 3;             // ring depth per warp
-constexpr int kChunk = 32;             // tokens per stage
-constexpr int kCodeB = 48;             // code bytes per token (d = 128)
-constexpr int kSignB = 16;             // sign bytes per token
-// stage layout (bytes)
-constexpr int kOffKc = 0;
-constexpr int kOffKs = kOffKc + kChunk * kCodeB;      // 1536
-constexpr int kOffKn = kOffKs + kChunk * kSignB;      // 2048
-constexpr int kOffKg = kOffKn + 2 * kChunk;           // 2112
-constexpr int kOffVc = kOffKg + 2 * kChunk;           // 2176
-constexpr int kOffVn = kOffVc + kChunk * kCodeB;      // 3712
-constexpr int kStageB = kOffVn + 2 * kChunk;          // 3776
 constexpr int kWaitLimit = 1 << 20;
 
-static_assert(kStageB % 16 == 0, "stage must keep 16-byte alignment");
+// Per-head-dim shape of a ring stage (bytes).
+template <int D>
+struct Cfg {
+    static constexpr int kS = D / 128;                        // 128-coordinate slices
+    static constexpr int kKC = D / 16;                        // coordinate chunks (mma k-steps)
+    static constexpr int kCodeB = 3 * D / 8;                  // code bytes per token
+    static constexpr int kSignB = D / 8;                      // sign bytes per token
+    static constexpr int kChunk = D == 128 ? 32 : 16;         // tokens per stage
+    static constexpr int kTiles = kChunk / 16;
+    static constexpr int kOffKc = 0;
+    static constexpr int kOffKs = kOffKc + kChunk * kCodeB;
+    static constexpr int kOffKn = kOffKs + kChunk * kSignB;
+    static constexpr int kOffKg = kOffKn + 2 * kChunk;
+    static constexpr int kOffVc = kOffKg + 2 * kChunk;
+    static constexpr int kOffVn = kOffVc + kChunk * kCodeB;
+    static constexpr int kStageB = kOffVn + 2 * kChunk;
+    static constexpr bool kBRegs = D == 128;                   // q'/u' fragments in registers
+    static_assert(kStageB % 16 == 0 && kOffKn % 16 == 0 && kOffKg % 16 == 0 && kOffVc % 16 == 0 &&
+                      kOffVn % 16 == 0,
+                  "stage fields must keep 16-byte alignment");
+};
+
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -158,29 +173,33 @@ __device__ __forceinline__ uint32_t sel_for(const uint32_t (&sel)[4], const uint
 // ---------------------------------------------------------------- kernel
 // Token-row orientation: each mma tile has 16 tokens on M and the (head,
 // hi|lo) columns on N (NT n-tiles of 4 heads), so no M rows are wasted:
-//   scores  S[16 tok][8] += Kdeq[16 tok][16 coords] * Q'[16 coords][8]   (8 coordinate chunks)
-//                         + Sgn[16 tok][16 signs] * U'[16 signs][8]       (8 sign chunks)
-//   values  O^T[16 coords][8] += Vdeq^T[16 coords][16 tok] * P[16 tok][8] (8 coordinate tiles)
+//   scores  S[16 tok][8] += Kdeq[16 tok][16 coords] * Q'[16 coords][8]   (D/16 coordinate chunks)
+//                         + Sgn[16 tok][16 signs] * U'[16 signs][8]       (D/16 sign chunks)
+//   values  O^T[16 coords][8] += Vdeq^T[16 coords][16 tok] * P[16 tok][8] (D/16 coordinate tiles)
 // Lane (g, t) = (lane / 4, lane % 4) dequantises tokens g and g + 8 of each
 // 16-token tile; its score columns are head t (hi, lo), so its softmax state
 // and output rows belong to head t (and head 4 + t when NT = 2).
-template <int NT, int NW>
-__global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecArgs a, int G) {
+template <int D, int NT, int NW>
+__global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs a, int G) {
+    using C = Cfg<D>;
+    constexpr int kKC = C::kKC;
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)NW * kStages * kStageB);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)NW * kStages * C::kStageB);
+    // d = 256: q'/u' fragments per (operand, n-tile, k-step, lane), filled once per CTA
+    uint2* sB = reinterpret_cast<uint2*>(smem + (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gr = lane >> 2, tq4 = lane & 3;
-    uint8_t* ring = smem + (size_t)warp * kStages * kStageB;
+    uint8_t* ring = smem + (size_t)warp * kStages * C::kStageB;
     const int split = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
 
     int64_t Tb = a.seq_lens ? (int64_t)a.seq_lens[b] : a.T;
     Tb = Tb < 0 ? 0 : (Tb > a.Tcap ? a.Tcap : Tb);
     const int64_t s0 = (int64_t)split * a.split_tokens;
     const int64_t s1 = (s0 + a.split_tokens < Tb) ? s0 + a.split_tokens : Tb;
-    const int nchunk = s1 > s0 ? (int)((s1 - s0 + kChunk - 1) / kChunk) : 0;
+    const int nchunk = s1 > s0 ? (int)((s1 - s0 + C::kChunk - 1) / C::kChunk) : 0;
     const int nmine = nchunk > warp ? (nchunk - warp + NW - 1) / NW : 0;
     const int64_t seq = (int64_t)b * a.Hkv + hkv;
-    const int64_t kbb = block_bytes(kD, true), vbb = block_bytes(kD, false);
+    const int64_t kbb = block_bytes(D, true), vbb = block_bytes(D, false);
 
     if (lane == 0)
         for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&bars[warp * kStages + s]), 1);
@@ -188,62 +207,71 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
     __syncwarp();
 
     auto issue = [&](int i) {
-        const int64_t t0 = s0 + (int64_t)(warp + i * NW) * kChunk;     // multiple of 32
+        const int64_t t0 = s0 + (int64_t)(warp + i * NW) * C::kChunk;     // multiple of the chunk
         const int64_t blk = seq * a.NB + (t0 >> 6);
-        const int half = (int)((t0 >> 5) & 1);
+        const int sub = (int)((t0 & 63) / C::kChunk);
         const uint8_t* kb = a.kc + blk * kbb;
         const uint8_t* vb = a.vc + blk * vbb;
-        uint8_t* st = ring + (i % kStages) * kStageB;
+        uint8_t* st = ring + (i % kStages) * C::kStageB;
         const uint32_t bar = smem_u32(&bars[warp * kStages + (i % kStages)]);
-        mbar_expect_tx(bar, kStageB);
-        bulk_g2s(smem_u32(st + kOffKc), kb + half * kChunk * kCodeB, kChunk * kCodeB, bar);
-        bulk_g2s(smem_u32(st + kOffKs), kb + 64 * kCodeB + half * kChunk * kSignB, kChunk * kSignB, bar);
-        bulk_g2s(smem_u32(st + kOffKn), kb + 64 * (kCodeB + kSignB) + half * 2 * kChunk, 2 * kChunk, bar);
-        bulk_g2s(smem_u32(st + kOffKg), kb + 64 * (kCodeB + kSignB) + 128 + half * 2 * kChunk, 2 * kChunk, bar);
-        bulk_g2s(smem_u32(st + kOffVc), vb + half * kChunk * kCodeB, kChunk * kCodeB, bar);
-        bulk_g2s(smem_u32(st + kOffVn), vb + 64 * kCodeB + half * 2 * kChunk, 2 * kChunk, bar);
+        constexpr int cb = C::kCodeB, sb = C::kSignB, ch = C::kChunk;
+        mbar_expect_tx(bar, C::kStageB);
+        bulk_g2s(smem_u32(st + C::kOffKc), kb + sub * ch * cb, ch * cb, bar);
+        bulk_g2s(smem_u32(st + C::kOffKs), kb + 64 * cb + sub * ch * sb, ch * sb, bar);
+        bulk_g2s(smem_u32(st + C::kOffKn), kb + 64 * (cb + sb) + sub * 2 * ch, 2 * ch, bar);
+        bulk_g2s(smem_u32(st + C::kOffKg), kb + 64 * (cb + sb) + 128 + sub * 2 * ch, 2 * ch, bar);
+        bulk_g2s(smem_u32(st + C::kOffVc), vb + sub * ch * cb, ch * cb, bar);
+        bulk_g2s(smem_u32(st + C::kOffVn), vb + 64 * cb + sub * 2 * ch, 2 * ch, bar);
     };
     if (lane == 0) {
         for (int i = 0; i < kStages && i < nmine; ++i) issue(i);
     }
     pdl_wait();                           // q' and u' come from the prologue kernel
 
-    // B operands (constant): column n = gr of n-tile nt is head 4 nt + gr / 2, limb gr % 2
-    uint32_t bq[NT][8][2], bu[NT][8][2];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+    // B-operand fragment of k-step kc: column n = gr of n-tile nt is head
+    // 4 nt + gr / 2, limb gr % 2; rows 16 kc + 2 tq4 (+1), +8 (+9)
+    auto b_frag = [&](const float* base, int nt, int kc, uint32_t& r0, uint32_t& r1) {
         const int hcol = 4 * nt + (gr >> 1);
-        const bool live = hcol < G;
-        const int64_t bh = (int64_t)b * a.Hq + (int64_t)hkv * G + (live ? hcol : 0);
-        const float* qp = a.qp + bh * kD;
-        const float* up = a.up + bh * kD;
-#pragma unroll
-        for (int kc = 0; kc < 8; ++kc) {
-            const int c0 = 16 * kc + 2 * tq4;
-            float x[4] = {0.f, 0.f, 0.f, 0.f}, y[4] = {0.f, 0.f, 0.f, 0.f};
-            if (live) {
-                x[0] = qp[c0]; x[1] = qp[c0 + 1]; x[2] = qp[c0 + 8]; x[3] = qp[c0 + 9];
-                y[0] = up[c0]; y[1] = up[c0 + 1]; y[2] = up[c0 + 8]; y[3] = up[c0 + 9];
-            }
-            uint32_t h0, l0, h1, l1;
-            split_hilo(x[0], x[1], h0, l0);
-            split_hilo(x[2], x[3], h1, l1);
-            bq[nt][kc][0] = (gr & 1) ? l0 : h0;
-            bq[nt][kc][1] = (gr & 1) ? l1 : h1;
-            split_hilo(y[0], y[1], h0, l0);
-            split_hilo(y[2], y[3], h1, l1);
-            bu[nt][kc][0] = (gr & 1) ? l0 : h0;
-            bu[nt][kc][1] = (gr & 1) ? l1 : h1;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (hcol < G) {
+            const float* p = base + ((int64_t)b * a.Hq + (int64_t)hkv * G + hcol) * D + 16 * kc + 2 * tq4;
+            x[0] = p[0]; x[1] = p[1]; x[2] = p[8]; x[3] = p[9];
         }
+        uint32_t h0, l0, h1, l1;
+        split_hilo(x[0], x[1], h0, l0);
+        split_hilo(x[2], x[3], h1, l1);
+        r0 = (gr & 1) ? l0 : h0;
+        r1 = (gr & 1) ? l1 : h1;
+    };
+    uint32_t bq[C::kBRegs ? NT : 1][C::kBRegs ? kKC : 1][2], bu[C::kBRegs ? NT : 1][C::kBRegs ? kKC : 1][2];
+    if constexpr (C::kBRegs) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int kc = 0; kc < kKC; ++kc) {
+                b_frag(a.qp, nt, kc, bq[nt][kc][0], bq[nt][kc][1]);
+                b_frag(a.up, nt, kc, bu[nt][kc][0], bu[nt][kc][1]);
+            }
+    } else {
+        for (int kc = warp; kc < kKC; kc += NW)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                uint32_t r0, r1;
+                b_frag(a.qp, nt, kc, r0, r1);
+                sB[((0 * NT + nt) * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
+                b_frag(a.up, nt, kc, r0, r1);
+                sB[((1 * NT + nt) * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
+            }
+        __syncthreads();
     }
     const uint32_t lut[4] = {a.cb.lut_lo[0], a.cb.lut_lo[1], a.cb.lut_hi[0], a.cb.lut_hi[1]};
     const uint32_t* pw = a.cb.pow2;
 
-    float o[NT][8][4];
+    float o[NT][kKC][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+        for (int mt = 0; mt < kKC; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
     float mrun[NT], lrun[NT], live[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -262,9 +290,9 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
                 mbar_wait_bounded(smem_u32(&bars[warp * kStages + (j % kStages)]), (uint32_t)((j / kStages) & 1));
             break;
         }
-        const uint8_t* st = ring + (i % kStages) * kStageB;
-        const int64_t tok0 = s0 + (int64_t)(warp + i * NW) * kChunk;
-        const int nvalid = (int)((s1 - tok0) < kChunk ? (s1 - tok0) : kChunk);
+        const uint8_t* st = ring + (i % kStages) * C::kStageB;
+        const int64_t tok0 = s0 + (int64_t)(warp + i * NW) * C::kChunk;
+        const int nvalid = (int)((s1 - tok0) < C::kChunk ? (s1 - tok0) : C::kChunk);
 
         // one 16-token tile; PARTIAL masks tokens beyond nvalid (only the last
         // chunk of a split can be partial)
@@ -272,39 +300,50 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
             constexpr bool PARTIAL = decltype(partial_tag)::value;
             const int tA = kt * 16 + gr, tB = tA + 8;            // this lane's two tokens
             // ---------------- scores
-            uint32_t selA[4], selB[4];
-            code_selectors(st + kOffKc + tA * kCodeB + tq4 * 12, pw, selA);
-            code_selectors(st + kOffKc + tB * kCodeB + tq4 * 12, pw, selB);
-            const uint32_t sgA = *reinterpret_cast<const uint32_t*>(st + kOffKs + tA * kSignB + tq4 * 4);
-            const uint32_t sgB = *reinterpret_cast<const uint32_t*>(st + kOffKs + tB * kSignB + tq4 * 4);
-            const uint32_t gA = *reinterpret_cast<const uint16_t*>(st + kOffKg + 2 * tA);
-            const uint32_t gB = *reinterpret_cast<const uint16_t*>(st + kOffKg + 2 * tB);
+            uint32_t selA[C::kS][4], selB[C::kS][4], sgA[C::kS], sgB[C::kS];
+#pragma unroll
+            for (int sl = 0; sl < C::kS; ++sl) {
+                code_selectors(st + C::kOffKc + tA * C::kCodeB + sl * 48 + tq4 * 12, pw, selA[sl]);
+                code_selectors(st + C::kOffKc + tB * C::kCodeB + sl * 48 + tq4 * 12, pw, selB[sl]);
+                sgA[sl] = *reinterpret_cast<const uint32_t*>(st + C::kOffKs + tA * C::kSignB + sl * 16 + tq4 * 4);
+                sgB[sl] = *reinterpret_cast<const uint32_t*>(st + C::kOffKs + tB * C::kSignB + sl * 16 + tq4 * 4);
+            }
+            const uint32_t gA = *reinterpret_cast<const uint16_t*>(st + C::kOffKg + 2 * tA);
+            const uint32_t gB = *reinterpret_cast<const uint16_t*>(st + C::kOffKg + 2 * tB);
             const uint32_t ggA = gA | (gA << 16), ggB = gB | (gB << 16);
             float acc[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll
-            for (int kc = 0; kc < 8; ++kc) {
+            for (int kc = 0; kc < kKC; ++kc) {
+                const int sl = kc >> 3, kk = kc & 7;
                 uint32_t ka[4];
-                dequant4(sel_for(selA, pw, kc), lut, ka[0], ka[2]);
-                dequant4(sel_for(selB, pw, kc), lut, ka[1], ka[3]);
+                dequant4(sel_for(selA[sl], pw, kk), lut, ka[0], ka[2]);
+                dequant4(sel_for(selB[sl], pw, kk), lut, ka[1], ka[3]);
                 uint32_t sa[4];
-                // sign bit 1 -> +gamma: the pair (2kc | 2kc+1) of a slot sits at bits (q, 16 + q)
-                sa[0] = ggA ^ (~shl_m(sgA, pw, 15 - 2 * kc) & 0x80008000u);
-                sa[1] = ggB ^ (~shl_m(sgB, pw, 15 - 2 * kc) & 0x80008000u);
-                sa[2] = ggA ^ (~shl_m(sgA, pw, 14 - 2 * kc) & 0x80008000u);
-                sa[3] = ggB ^ (~shl_m(sgB, pw, 14 - 2 * kc) & 0x80008000u);
+                // sign bit 1 -> +gamma: the pair (2kk | 2kk+1) of a slot sits at bits (q, 16 + q)
+                sa[0] = ggA ^ (~shl_m(sgA[sl], pw, 15 - 2 * kk) & 0x80008000u);
+                sa[1] = ggB ^ (~shl_m(sgB[sl], pw, 15 - 2 * kk) & 0x80008000u);
+                sa[2] = ggA ^ (~shl_m(sgA[sl], pw, 14 - 2 * kk) & 0x80008000u);
+                sa[3] = ggB ^ (~shl_m(sgB[sl], pw, 14 - 2 * kk) & 0x80008000u);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    mma16816(acc[nt], ka, bq[nt][kc][0], bq[nt][kc][1]);
-                    mma16816(acc[nt], sa, bu[nt][kc][0], bu[nt][kc][1]);
+                    if constexpr (C::kBRegs) {
+                        mma16816(acc[nt], ka, bq[nt][kc][0], bq[nt][kc][1]);
+                        mma16816(acc[nt], sa, bu[nt][kc][0], bu[nt][kc][1]);
+                    } else {
+                        const uint2 fq = sB[((0 * NT + nt) * kKC + kc) * 32 + lane];
+                        const uint2 fu = sB[((1 * NT + nt) * kKC + kc) * 32 + lane];
+                        mma16816(acc[nt], ka, fq.x, fq.y);
+                        mma16816(acc[nt], sa, fu.x, fu.y);
+                    }
                 }
             }
             // ---------------- online softmax per head (this lane: head 4 nt + tq4)
-            const float2 nkA = __half22float2(__halves2half2(*reinterpret_cast<const __half*>(st + kOffKn + 2 * tA),
-                                                             *reinterpret_cast<const __half*>(st + kOffKn + 2 * tB)));
-            float2 nv = __half22float2(__halves2half2(*reinterpret_cast<const __half*>(st + kOffVn + 2 * tA),
-                                                      *reinterpret_cast<const __half*>(st + kOffVn + 2 * tB)));
+            const float2 nkA = __half22float2(__halves2half2(*reinterpret_cast<const __half*>(st + C::kOffKn + 2 * tA),
+                                                             *reinterpret_cast<const __half*>(st + C::kOffKn + 2 * tB)));
+            float2 nv = __half22float2(__halves2half2(*reinterpret_cast<const __half*>(st + C::kOffVn + 2 * tA),
+                                                      *reinterpret_cast<const __half*>(st + C::kOffVn + 2 * tB)));
             const bool okA = tA < nvalid, okB = tB < nvalid;
             if constexpr (PARTIAL) {
                 if (!okA) nv.x = 0.f;
@@ -314,12 +353,12 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 float sA = a.scale_log2 * nkA.x * (acc[nt][0] + acc[nt][1]);
-                float sB = a.scale_log2 * nkA.y * (acc[nt][2] + acc[nt][3]);
+                float sB_ = a.scale_log2 * nkA.y * (acc[nt][2] + acc[nt][3]);
                 if constexpr (PARTIAL) {
                     if (!okA) sA = -INFINITY;
-                    if (!okB) sB = -INFINITY;
+                    if (!okB) sB_ = -INFINITY;
                 }
-                float mt = fmaxf(sA, sB);
+                float mt = fmaxf(sA, sB_);
                 mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 4));
                 mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 8));
                 mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 16));
@@ -328,14 +367,14 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
                     const float corr = (mnew == -INFINITY) ? 1.f : fast_exp2(mrun[nt] - mnew);
                     lrun[nt] *= corr;
 #pragma unroll
-                    for (int mt2 = 0; mt2 < 8; ++mt2) {
+                    for (int mt2 = 0; mt2 < kKC; ++mt2) {
                         o[nt][mt2][0] *= corr; o[nt][mt2][1] *= corr; o[nt][mt2][2] *= corr; o[nt][mt2][3] *= corr;
                     }
                     mrun[nt] = mnew;
                 }
                 // mrun >= sA, sB here, so the exponent is <= 0 (masked: -inf -> 0)
                 const float pA = fast_exp2(sA - mrun[nt]);
-                const float pB = fast_exp2(sB - mrun[nt]);
+                const float pB = fast_exp2(sB_ - mrun[nt]);
                 lrun[nt] += pA + pB;
                 uint32_t hi, lo, xA, xB;
                 split_hilo(pA * nv.x * live[nt], pB * nv.y * live[nt], hi, lo);
@@ -346,24 +385,28 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
                 pb[nt][1] = movmatrix_t(xB);
             }
             // ---------------- values: O^T += Vdeq^T P
-            code_selectors(st + kOffVc + tA * kCodeB + tq4 * 12, pw, selA);
-            code_selectors(st + kOffVc + tB * kCodeB + tq4 * 12, pw, selB);
 #pragma unroll
-            for (int kc = 0; kc < 8; ++kc) {
+            for (int sl = 0; sl < C::kS; ++sl) {
+                code_selectors(st + C::kOffVc + tA * C::kCodeB + sl * 48 + tq4 * 12, pw, selA[sl]);
+                code_selectors(st + C::kOffVc + tB * C::kCodeB + sl * 48 + tq4 * 12, pw, selB[sl]);
+            }
+#pragma unroll
+            for (int kc = 0; kc < kKC; ++kc) {
+                const int sl = kc >> 3, kk = kc & 7;
                 uint32_t x0, x1, y0, y1;
-                dequant4(sel_for(selA, pw, kc), lut, x0, x1);      // token tA: coords 16kc+2t(+1), +8
-                dequant4(sel_for(selB, pw, kc), lut, y0, y1);      // token tB
+                dequant4(sel_for(selA[sl], pw, kk), lut, x0, x1);      // token tA: coords 16kc+2t(+1), +8
+                dequant4(sel_for(selB[sl], pw, kk), lut, y0, y1);      // token tB
                 const uint32_t va[4] = {movmatrix_t(x0), movmatrix_t(x1), movmatrix_t(y0), movmatrix_t(y1)};
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) mma16816(o[nt][kc], va, pb[nt][0], pb[nt][1]);
             }
         };
-        if (nvalid == kChunk) {
-            tile(0, std::false_type{});
-            tile(1, std::false_type{});
+        if (nvalid == C::kChunk) {
+#pragma unroll
+            for (int kt = 0; kt < C::kTiles; ++kt) tile(kt, std::false_type{});
         } else {
             tile(0, std::true_type{});
-            if (nvalid > 16) tile(1, std::true_type{});
+            if (C::kTiles > 1 && nvalid > 16) tile(1, std::true_type{});
         }
         __syncwarp();
         if (lane == 0 && i + kStages < nmine) {
@@ -382,42 +425,42 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
     pdl_trigger();                        // the combine kernel may start launching
     // ---------------- merge the warps of the CTA into one partial per head
     __syncwarp();
-    float* wbuf = reinterpret_cast<float*>(ring);             // [G][kD + 2], in this warp's own ring
+    float* wbuf = reinterpret_cast<float*>(ring);             // [G][D + 2], in this warp's own ring
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         const int h = 4 * nt + tq4;
         if (h < G) {
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                wbuf[h * (kD + 2) + 16 * mt + gr] = o[nt][mt][0] + o[nt][mt][1];
-                wbuf[h * (kD + 2) + 16 * mt + 8 + gr] = o[nt][mt][2] + o[nt][mt][3];
+            for (int mt = 0; mt < kKC; ++mt) {
+                wbuf[h * (D + 2) + 16 * mt + gr] = o[nt][mt][0] + o[nt][mt][1];
+                wbuf[h * (D + 2) + 16 * mt + 8 + gr] = o[nt][mt][2] + o[nt][mt][3];
             }
             if (gr == 0) {
-                wbuf[h * (kD + 2) + kD] = mrun[nt];
-                wbuf[h * (kD + 2) + kD + 1] = lrun[nt];
+                wbuf[h * (D + 2) + D] = mrun[nt];
+                wbuf[h * (D + 2) + D + 1] = lrun[nt];
             }
         }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * kD; idx += NW * 32) {
-        const int g = idx / kD, j = idx % kD;
+    for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
+        const int g = idx / D, j = idx % D;
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < NW; ++w)
-            M = fmaxf(M, reinterpret_cast<const float*>(smem + (size_t)w * kStages * kStageB)[g * (kD + 2) + kD]);
+            M = fmaxf(M, reinterpret_cast<const float*>(smem + (size_t)w * kStages * C::kStageB)[g * (D + 2) + D]);
         float L = 0.f, A = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
             for (int w = 0; w < NW; ++w) {
-                const float* wb = reinterpret_cast<const float*>(smem + (size_t)w * kStages * kStageB) + g * (kD + 2);
-                const float f = exp2f(wb[kD] - M);
-                L = fmaf(f, wb[kD + 1], L);
+                const float* wb = reinterpret_cast<const float*>(smem + (size_t)w * kStages * C::kStageB) + g * (D + 2);
+                const float f = exp2f(wb[D] - M);
+                L = fmaf(f, wb[D + 1], L);
                 A = fmaf(f, wb[j], A);
             }
         }
         const int64_t bh = (int64_t)b * a.Hq + (int64_t)hkv * G + g;
         const int64_t pidx = bh * a.nsplit + split;
-        a.part_acc[pidx * kD + j] = A;
+        a.part_acc[pidx * D + j] = A;
         if (j == 0) {
             a.part_ml[2 * pidx] = M;
             a.part_ml[2 * pidx + 1] = L;
@@ -430,23 +473,26 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma128_kernel(const DecA
 constexpr int kNW1 = 16;   // warps per CTA, up to 4 heads per kv head (one n-tile)
 constexpr int kNW2 = 8;    // warps per CTA, 8 heads per kv head (two n-tiles, more registers)
 
-template <int NT, int NW>
+template <int D, int NT, int NW>
 cudaError_t launch_mma_t(const DecArgs& a, int G, cudaStream_t s) {
-    const size_t smem = (size_t)NW * kStages * kStageB + (size_t)NW * kStages * 8;
-    auto kern = tq_decode_mma128_kernel<NT, NW>;
-    cudaError_t e = set_smem_once<tq_decode_mma128_kernel<NT, NW>>((int)smem);
+    using C = Cfg<D>;
+    const size_t smem = (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
+                        (C::kBRegs ? 0 : (size_t)2 * NT * C::kKC * 32 * sizeof(uint2));
+    auto kern = tq_decode_mma_kernel<D, NT, NW>;
+    cudaError_t e = set_smem_once<tq_decode_mma_kernel<D, NT, NW>>((int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
     return launch_pdl(kern, grid, dim3(NW * 32), smem, s, a, G);
 }
 
 cudaError_t launch_decode_mma(int d, int G, const DecArgs& a, cudaStream_t s) {
-    if (d != kD || G < 1 || G > 8) return cudaErrorInvalidValue;
+    if ((d != 128 && d != 256) || G < 1 || G > 8) return cudaErrorInvalidValue;
     if (a.B * a.Hkv == 0) return cudaSuccess;
-    return G <= 4 ? launch_mma_t<1, kNW1>(a, G, s) : launch_mma_t<2, kNW2>(a, G, s);
+    if (d == 128) return G <= 4 ? launch_mma_t<128, 1, kNW1>(a, G, s) : launch_mma_t<128, 2, kNW2>(a, G, s);
+    return G <= 4 ? launch_mma_t<256, 1, kNW1>(a, G, s) : launch_mma_t<256, 2, kNW2>(a, G, s);
 }
 
-int decode_mma_chunk_tokens() { return kChunk; }
+int decode_mma_chunk_tokens(int d) { return d == 128 ? Cfg<128>::kChunk : Cfg<256>::kChunk; }
 int decode_mma_warps(int G) { return G <= 4 ? kNW1 : kNW2; }
 
 }  // namespace tqi

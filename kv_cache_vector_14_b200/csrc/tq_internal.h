@@ -166,7 +166,7 @@ cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml,
                            const float* part_acc, const float* dsign, float* out, cudaStream_t s);
 bool mma_supported(int d, int G);
 int decode_ctas_per_sm(bool use_mma);
-int decode_chunk_tokens(bool use_mma);   // split ranges are multiples of this
+int decode_chunk_tokens(int d, bool use_mma);   // split ranges are multiples of this
 int decode_warps(bool use_mma, int G);   // warps sharing one split
 
 }  // namespace tqi
