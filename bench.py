@@ -2,10 +2,10 @@
 """Benchmark of the TurboQuant decode hot path on B200.
 
 A step is one decode step of the long-context workload (B=4, Hq=16/Hkv=8,
-d=128, 102400 compressed tokens per sequence) through the library's C ABI:
-encode one new K and one new V vector per (batch, kv head) into the cache
-(tq_encode_k / tq_encode_v) and attend over the whole compressed cache
-(tq_attend_decode: query prologue, split-K attention, combine).  The headline
+d=128, 102400 compressed tokens per sequence) through the library's C ABI,
+tq_append_attend: encode one new K and one new V vector per (batch, kv head)
+into the cache and attend over the whole compressed cache (query prologue,
+split-K attention, combine), the five kernels chained on one stream.  The headline
 metric is the achieved bandwidth on the compressed-cache bytes the step must
 read (118 B per token per kv head); the encode-only workload (B=1, 8 kv heads,
 32768 bf16 tokens) gives the KV encode throughput in Mvectors/s.
@@ -255,11 +255,12 @@ def measure_encode(h, dev, world: int, dist, passes: int = 30) -> dict:
 
 def measure_loop(dev, world: int, dist, replays: int = 5) -> dict:
     """Append-and-attend workload (B=16, Hq=32/Hkv=8, d=256, cache from 8192
-    tokens, 256 steps of: encode the step's K and V per (batch, kv head) at
-    position T, attend over T+1 tokens).  The 256-step sequence is captured
-    once in a CUDA graph and replayed; each replay rewrites the same cache
-    positions with the same values, so every replay does the full work.  The
-    ~250 MB cache exceeds L2.  Also timed eagerly (launch by launch)."""
+    tokens, 256 steps of tq_append_attend: encode the step's K and V per
+    (batch, kv head) at position T, attend over T+1 tokens).  The 256-step
+    sequence is captured once in a CUDA graph and replayed; each replay
+    rewrites the same cache positions with the same values, so every replay
+    does the full work.  The ~250 MB cache exceeds L2.  Also timed eagerly, and
+    as a graph of the same steps made of three separate calls each."""
     import torch
     from kv_cache_vector_14_b200 import tq
     w = synthetic.WORKLOADS["c5"]
@@ -280,9 +281,13 @@ def measure_loop(dev, world: int, dist, replays: int = 5) -> dict:
     out = torch.empty((S, B, Hq, d), dtype=torch.float32, device=dev)
     ws = torch.empty(tq.tq_attend_workspace_bytes(h, B, Hq, Hkv, Tend), dtype=torch.uint8, device=dev)
 
-    def sequence():
+    def sequence(fused=True):
         for s in range(S):
             T = T0 + s
+            if fused:
+                tq.tq_append_attend(h, kn[:, :, s:s + 1], vn[:, :, s:s + 1], kc, vc, T, q[s], out[s], ws,
+                                    scale=w.scale)
+                continue
             tq.tq_encode_k(h, kn[:, :, s:s + 1], kc, T)
             tq.tq_encode_v(h, vn[:, :, s:s + 1], vc, T)
             tq.tq_attend_decode(h, q[s], kc, vc, out[s], ws, T=T + 1, scale=w.scale)
@@ -317,6 +322,21 @@ def measure_loop(dev, world: int, dist, replays: int = 5) -> dict:
         times.append(e0.elapsed_time(e1))
     graph_ms = statistics.median(times)
     graph_ms_max = max_over_ranks(graph_ms, dist, dev)
+    del graph
+    graph = torch.cuda.CUDAGraph()              # the same steps as three separate calls each
+    with torch.cuda.graph(graph):
+        sequence(fused=False)
+    graph.replay()
+    torch.cuda.synchronize()
+    same_sep = bool(torch.equal(out, ref))
+    times = []
+    for _ in range(replays):
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    graph_sep_ms = statistics.median(times)
     path = tq.tq_attend_path(h, Hq, Hkv)
     status = tq.tq_status_string(tq.tq_device_status(h))
     del graph
@@ -325,6 +345,8 @@ def measure_loop(dev, world: int, dist, replays: int = 5) -> dict:
     return {"workload": w.title, "steps": S, "decode_path": path,
             "graph_ms_total": graph_ms, "graph_us_per_step": graph_ms * 1e3 / S,
             "eager_ms_total": eager_ms, "eager_us_per_step": eager_ms * 1e3 / S,
+            "graph_us_per_step_separate_calls": graph_sep_ms * 1e3 / S,
+            "separate_calls_output_equal": same_sep,
             "achieved_gbs": whole_job_rate(nbytes, graph_ms * 1e-3, world, dist, dev) / 1e9,
             "decode_tokens_per_s": world * S * B / (graph_ms_max * 1e-3),
             "kernels_per_step": 5, "graph_output_equals_eager": same,
@@ -369,6 +391,9 @@ def run_ours(args, rank: int, world: int, dist):
     path = tq.tq_attend_path(h, Hq, Hkv)
 
     def step(kn, vn, qq, o):
+        tq.tq_append_attend(h, kn, vn, kc, vc, T - 1, qq, o, ws, scale=w.scale)
+
+    def step_separate(kn, vn, qq, o):
         tq.tq_encode_k(h, kn, kc, T - 1)
         tq.tq_encode_v(h, vn, vc, T - 1)
         tq.tq_attend_decode(h, qq, kc, vc, o, ws, T=T, scale=w.scale)
@@ -380,37 +405,60 @@ def run_ours(args, rank: int, world: int, dist):
 
     for _ in range(args.warmup):
         step(k_new, v_new, q, out)
+        step_separate(k_new, v_new, q, out)
     torch.cuda.synchronize()
 
-    # ---- timed region (device-resident inputs); the split-K kernel timed alone by events
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for a_, b_ in kev:           # torch creates the CUDA events on first record; the library re-records them
-        a_.record()
-        b_.record()
-    torch.cuda.synchronize()
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         pass
+    # ---- timed region (device-resident inputs): the fused step, nothing else on the stream
     sampler = ClockSampler(uuid) if rank == 0 else None
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for i in range(args.steps):
-        tq.tq_set_decode_events(h, kev[i][0], kev[i][1])
         step(k_new, v_new, q, out)
     e1.record()
     torch.cuda.synchronize()
     barrier()
-    tq.tq_set_decode_events(h, None, None)
     clocks = sampler.stop() if sampler else None
     ms = e0.elapsed_time(e1) / args.steps
     ms_max = max_over_ranks(ms, dist, dev)
-    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
     bytes_step = B * Hkv * T * BYTES_PER_TOKEN_HEAD[d]
     value = whole_job_rate(bytes_step, ms * 1e-3, world, dist, dev) / 1e9
+
+    # ---- the split-K kernel alone, timed by events the library records around
+    # it (the events break the launch chain, so this is a separate pass)
+    n_kern = max(1, min(args.steps, 500))
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_kern)]
+    for a_, b_ in kev:           # torch creates the CUDA events on first record; the library re-records them
+        a_.record()
+        b_.record()
+    torch.cuda.synchronize()
+    for i in range(n_kern):
+        tq.tq_set_decode_events(h, kev[i][0], kev[i][1])
+        step(k_new, v_new, q, out)
+    torch.cuda.synchronize()
+    tq.tq_set_decode_events(h, None, None)
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+
+    # ---- the same step as three separate calls (encode K, encode V, attend)
+    e0.record()
+    for i in range(n_kern):
+        step_separate(k_new, v_new, q, out)
+    e1.record()
+    torch.cuda.synchronize()
+    ms_separate = e0.elapsed_time(e1) / n_kern
+
+    if args.only == "step":            # profiling aid: the timed decode steps alone
+        tq.tq_destroy(h)
+        if rank == 0:
+            print(json.dumps({"ms_per_step": ms_max, "kernel_ms": kern_ms, "ms_per_step_separate_calls": ms_separate,
+                              "decode_path": path}), flush=True)
+        return
 
     # ---- end to end: pinned host inputs copied in, the output read back, every step
     kh = k_new.cpu().pin_memory()
@@ -464,7 +512,9 @@ def run_ours(args, rank: int, world: int, dist):
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.title, "B": B, "Hq": Hq, "Hkv": Hkv, "head_dim": d, "T": T,
-                   "step": "encode 1 K + 1 V per (batch, kv head), then attention over the compressed cache",
+                   "step": "tq_append_attend: encode 1 K + 1 V per (batch, kv head) at position T-1, then "
+                           "attention over the T-token compressed cache",
+                   "ms_per_step_separate_calls": ms_separate,
                    "algorithmic_bytes_per_step": bytes_step, "decode_path": path,
                    "l2": "inputs larger than L2 (386.7 MB compressed cache read per step vs 126 MB L2)",
                    "parallelism": f"replicas x{world}"},
@@ -492,9 +542,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["encode", "loop"], default=None,
-                    help="run only the encode-only workload (--steps passes) or the append-and-attend "
-                         "workload (--steps graph replays); for profiling")
+    ap.add_argument("--only", choices=["step", "encode", "loop"], default=None,
+                    help="run only the decode step (--steps steps), the encode-only workload (--steps "
+                         "passes) or the append-and-attend workload (--steps graph replays); for profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

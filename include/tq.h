@@ -165,6 +165,31 @@ TQ_API tq_status tq_attend_decode(const tq_handle* h, const void* q, tq_dtype qd
                            const int32_t* seq_lens, int64_t T, float scale, float* out, void* ws,
                            size_t ws_bytes, void* stream);
 
+/* ---- fused append-and-attend step ---------------------------------------- */
+
+/* One decode step of a serving loop: encode Tnew new K and V vectors per
+ * (batch, kv head) into token positions [t0, t0 + Tnew) of kc and vc, then
+ * attend for B x Hq queries over tokens [0, t0 + Tnew) of every sequence.
+ * The page's decode loop appends each generated token's K/V to the
+ * compressed cache and attends over it (page "Apple Silicon向けSwiftLM ...",
+ * K/V sections and the hybrid V2+V3 section); this call does both in one
+ * launch chain.  Results (cache bytes and out) are identical to
+ * tq_encode_k + tq_encode_v + tq_attend_decode with T = t0 + Tnew.
+ * k_new and v_new share `kv_dtype` and the element strides (sb, sh, st) as in
+ * tq_encode_k; B and Hkv are the caches'.  q, out, ws and scale as in
+ * tq_attend_decode (ws sized by tq_attend_workspace_bytes(h, B, Hq, Hkv,
+ * t0 + Tnew)).  The kernels are chained with programmatic dependent launch:
+ * the query prologue runs alongside the encodes and the attention kernel
+ * prefetches every cached chunk except the ones holding the new tokens
+ * before they are written; every kernel completes only after the one before
+ * it, so the next work on the stream sees the finished step.
+ * Errors: those of tq_encode_k and tq_attend_decode (checked before any
+ * launch). */
+TQ_API tq_status tq_append_attend(const tq_handle* h, const void* k_new, const void* v_new, tq_dtype kv_dtype,
+                                  int64_t Tnew, int64_t sb, int64_t sh, int64_t st, const tq_cache* kc,
+                                  const tq_cache* vc, int64_t t0, const void* q, tq_dtype q_dtype, int64_t Hq,
+                                  float scale, float* out, void* ws, size_t ws_bytes, void* stream);
+
 /* ---- decode attention without device allocation ------------------------- */
 
 /* Size of the scratch array inside the library used by tq_attend_decode_static. */

@@ -87,27 +87,98 @@ bool cache_ok(const tq_handle* h, const tq_cache* c) {
            c->Tcap % kBlockT == 0 && h;
 }
 
-tq_status encode_common(const tq_handle* h, const void* x, tq_dtype dt, int64_t B, int64_t Hkv, int64_t Tnew,
-                        int64_t sb, int64_t sh, int64_t st, const tq_cache* c, int64_t t0, void* stream, bool is_k) {
+tq_status prepare_encode(const tq_handle* h, const void* x, tq_dtype dt, int64_t B, int64_t Hkv, int64_t Tnew,
+                         int64_t sb, int64_t sh, int64_t st, const tq_cache* c, int64_t t0, EncArgs* a,
+                         bool* empty) {
+    *empty = false;
     if (!h || !dtype_ok(dt) || !cache_ok(h, c)) return TQ_ERR_INVALID_ARG;
     if (B != c->B || Hkv != c->Hkv || Tnew < 0 || t0 < 0 || t0 + Tnew > c->Tcap) return TQ_ERR_INVALID_ARG;
-    if (B == 0 || Tnew == 0) return TQ_OK;
+    if (B == 0 || Tnew == 0) {
+        *empty = true;
+        return TQ_OK;
+    }
     if (!x || !aligned(x, dtype_size(dt)) || sb < 0 || sh < 0 || st < 0) return TQ_ERR_INVALID_ARG;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
     if (dev != h->device) return TQ_ERR_INVALID_ARG;
-    EncArgs a{};
-    a.x = x; a.sb = sb; a.sh = sh; a.st = st;
-    a.B = B; a.Hkv = Hkv; a.Tnew = Tnew; a.t0 = t0;
-    a.NB = c->Tcap / kBlockT;
-    a.cache = static_cast<uint8_t*>(c->base);
-    a.dsign = h->dsign; a.sthr = h->dSThr; a.bimg = h->dSB; a.err = h->derr; a.cb = h->cb;
-    const int64_t es = (int64_t)dtype_size(dt);
-    a.vec16 = (aligned(x, 16) && (sb * es) % 16 == 0 && (sh * es) % 16 == 0 && (st * es) % 16 == 0) ? 1 : 0;
     if (B * Hkv * Tnew >= (int64_t)1 << 31) return TQ_ERR_UNSUPPORTED;      // vector indices are 32-bit
-    a.fdT = make_fastdiv((uint32_t)Tnew);
-    a.fdH = make_fastdiv((uint32_t)Hkv);
-    return cuda_status(launch_encode(h->d, is_k, dt, a, h->num_sms, static_cast<cudaStream_t>(stream)));
+    *a = EncArgs{};
+    a->x = x; a->sb = sb; a->sh = sh; a->st = st;
+    a->B = B; a->Hkv = Hkv; a->Tnew = Tnew; a->t0 = t0;
+    a->NB = c->Tcap / kBlockT;
+    a->cache = static_cast<uint8_t*>(c->base);
+    a->dsign = h->dsign; a->sthr = h->dSThr; a->bimg = h->dSB; a->err = h->derr; a->cb = h->cb;
+    const int64_t es = (int64_t)dtype_size(dt);
+    a->vec16 = (aligned(x, 16) && (sb * es) % 16 == 0 && (sh * es) % 16 == 0 && (st * es) % 16 == 0) ? 1 : 0;
+    a->fdT = make_fastdiv((uint32_t)Tnew);
+    a->fdH = make_fastdiv((uint32_t)Hkv);
+    return TQ_OK;
+}
+
+tq_status encode_common(const tq_handle* h, const void* x, tq_dtype dt, int64_t B, int64_t Hkv, int64_t Tnew,
+                        int64_t sb, int64_t sh, int64_t st, const tq_cache* c, int64_t t0, void* stream, bool is_k) {
+    EncArgs a;
+    bool empty;
+    const tq_status r = prepare_encode(h, x, dt, B, Hkv, Tnew, sb, sh, st, c, t0, &a, &empty);
+    if (r != TQ_OK || empty) return r;
+    return cuda_status(launch_encode(h->d, is_k, dt, a, h->num_sms, false, static_cast<cudaStream_t>(stream)));
+}
+
+// Checks of an attention call and its kernel arguments; *G receives the group size.
+tq_status prepare_attend(const tq_handle* h, const void* q, tq_dtype qdt, int64_t B, int64_t Hq, const tq_cache* kc,
+                         const tq_cache* vc, const int32_t* seq_lens, int64_t T, float scale, float* out, void* ws,
+                         size_t ws_bytes, DecodePlan* p, DecArgs* a) {
+    if (!h || !dtype_ok(qdt) || !cache_ok(h, kc) || !cache_ok(h, vc)) return TQ_ERR_INVALID_ARG;
+    if (B < 0 || Hq <= 0 || kc->B != B || vc->B != B || kc->Hkv != vc->Hkv || kc->Tcap != vc->Tcap)
+        return TQ_ERR_INVALID_ARG;
+    const int64_t Hkv = kc->Hkv;
+    if (Hq % Hkv) return TQ_ERR_INVALID_ARG;
+    const int G = (int)(Hq / Hkv);
+    if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_ERR_UNSUPPORTED;
+    if (!seq_lens && (T < 0 || T > kc->Tcap)) return TQ_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
+    if (B == 0) return TQ_OK;
+    if (!q || !out || !ws || !aligned(q, dtype_size(qdt)) || !aligned(out, 16) || !aligned(ws, 256))
+        return TQ_ERR_INVALID_ARG;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
+    if (dev != h->device) return TQ_ERR_INVALID_ARG;
+    const int64_t Tmax = seq_lens ? kc->Tcap : T;
+    if (!make_plan(h, B, Hq, Hkv, Tmax, p, false)) return TQ_ERR_INVALID_ARG;
+    if (ws_bytes < p->bytes) return TQ_ERR_WORKSPACE;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    *a = DecArgs{};
+    a->qp = reinterpret_cast<float*>(w + p->off_qp);
+    a->up = reinterpret_cast<float*>(w + p->off_up);
+    a->kc = static_cast<const uint8_t*>(kc->base);
+    a->vc = static_cast<const uint8_t*>(vc->base);
+    a->NB = kc->Tcap / kBlockT;
+    a->seq_lens = seq_lens;
+    a->T = T;
+    a->Tcap = kc->Tcap;
+    a->B = B; a->Hq = Hq; a->Hkv = Hkv;
+    a->nsplit = p->nsplit;
+    a->split_tokens = p->split_tokens;
+    a->scale_log2 = scale * kLog2e;
+    a->part_ml = reinterpret_cast<float*>(w + p->off_ml);
+    a->part_acc = reinterpret_cast<float*>(w + p->off_acc);
+    a->err = h->derr;
+    a->cb = h->cb;
+    return TQ_OK;
+}
+
+// Prologue, split-K attention, combine.  chained: the prologue is a
+// programmatic dependent of the kernel before it (the fused step's encodes).
+cudaError_t launch_attend(const tq_handle* h, const void* q, tq_dtype qdt, const DecodePlan& p, const DecArgs& a,
+                          float* out, bool chained, cudaStream_t s) {
+    const int64_t BHq = a.B * a.Hq;
+    cudaError_t e = launch_prologue(h->d, q, qdt, BHq, h->dsign, h->dST, const_cast<float*>(a.qp),
+                                    const_cast<float*>(a.up), chained, s);
+    if (e == cudaSuccess && h->ev_start) e = cudaEventRecord(h->ev_start, s);
+    if (e == cudaSuccess) e = launch_decode(h->d, p.G, p.use_mma, a, s);
+    if (e == cudaSuccess && h->ev_stop) e = cudaEventRecord(h->ev_stop, s);
+    if (e == cudaSuccess) e = launch_combine(h->d, BHq, p.nsplit, a.part_ml, a.part_acc, h->dsign, out, s);
+    return e;
 }
 
 }  // namespace
@@ -259,50 +330,42 @@ const char* tq_attend_path(const tq_handle* h, int64_t Hq, int64_t Hkv) {
 tq_status tq_attend_decode(const tq_handle* h, const void* q, tq_dtype qdt, int64_t B, int64_t Hq,
                            const tq_cache* kc, const tq_cache* vc, const int32_t* seq_lens, int64_t T,
                            float scale, float* out, void* ws, size_t ws_bytes, void* stream) {
-    if (!h || !dtype_ok(qdt) || !cache_ok(h, kc) || !cache_ok(h, vc)) return TQ_ERR_INVALID_ARG;
-    if (B < 0 || Hq <= 0 || kc->B != B || vc->B != B || kc->Hkv != vc->Hkv || kc->Tcap != vc->Tcap)
-        return TQ_ERR_INVALID_ARG;
-    const int64_t Hkv = kc->Hkv;
-    if (Hq % Hkv) return TQ_ERR_INVALID_ARG;
-    const int G = (int)(Hq / Hkv);
-    if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_ERR_UNSUPPORTED;
-    if (!seq_lens && (T < 0 || T > kc->Tcap)) return TQ_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
-    if (B == 0) return TQ_OK;
-    if (!q || !out || !ws || !aligned(q, dtype_size(qdt)) || !aligned(out, 16) || !aligned(ws, 256))
-        return TQ_ERR_INVALID_ARG;
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
-    if (dev != h->device) return TQ_ERR_INVALID_ARG;
-    const int64_t Tmax = seq_lens ? kc->Tcap : T;
     DecodePlan p;
-    if (!make_plan(h, B, Hq, Hkv, Tmax, &p, false)) return TQ_ERR_INVALID_ARG;
-    if (ws_bytes < p.bytes) return TQ_ERR_WORKSPACE;
+    DecArgs a;
+    const tq_status r = prepare_attend(h, q, qdt, B, Hq, kc, vc, seq_lens, T, scale, out, ws, ws_bytes, &p, &a);
+    if (r != TQ_OK || B == 0) return r;
+    return cuda_status(launch_attend(h, q, qdt, p, a, out, false, static_cast<cudaStream_t>(stream)));
+}
+
+tq_status tq_append_attend(const tq_handle* h, const void* k_new, const void* v_new, tq_dtype kv_dtype,
+                           int64_t Tnew, int64_t sb, int64_t sh, int64_t st, const tq_cache* kc,
+                           const tq_cache* vc, int64_t t0, const void* q, tq_dtype q_dtype, int64_t Hq,
+                           float scale, float* out, void* ws, size_t ws_bytes, void* stream) {
+    if (!kc || !vc) return TQ_ERR_INVALID_ARG;
+    const int64_t B = kc->B, Hkv = kc->Hkv;
+    EncArgs ek, ev;
+    bool empty_k, empty_v;
+    tq_status r = prepare_encode(h, k_new, kv_dtype, B, Hkv, Tnew, sb, sh, st, kc, t0, &ek, &empty_k);
+    if (r == TQ_OK) r = prepare_encode(h, v_new, kv_dtype, B, Hkv, Tnew, sb, sh, st, vc, t0, &ev, &empty_v);
+    if (r != TQ_OK) return r;
+    DecodePlan p;
+    DecArgs a;
+    r = prepare_attend(h, q, q_dtype, B, Hq, kc, vc, nullptr, t0 + Tnew, scale, out, ws, ws_bytes, &p, &a);
+    if (r != TQ_OK || B == 0) return r;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t* w = static_cast<uint8_t*>(ws);
-    DecArgs a{};
-    a.qp = reinterpret_cast<float*>(w + p.off_qp);
-    a.up = reinterpret_cast<float*>(w + p.off_up);
-    a.kc = static_cast<const uint8_t*>(kc->base);
-    a.vc = static_cast<const uint8_t*>(vc->base);
-    a.NB = kc->Tcap / kBlockT;
-    a.seq_lens = seq_lens;
-    a.T = T;
-    a.Tcap = kc->Tcap;
-    a.B = B; a.Hq = Hq; a.Hkv = Hkv;
-    a.nsplit = p.nsplit;
-    a.split_tokens = p.split_tokens;
-    a.scale_log2 = scale * kLog2e;
-    a.part_ml = reinterpret_cast<float*>(w + p.off_ml);
-    a.part_acc = reinterpret_cast<float*>(w + p.off_acc);
-    a.err = h->derr;
-    a.cb = h->cb;
-    cudaError_t e = launch_prologue(h->d, q, qdt, B * Hq, h->dsign, h->dST,
-                                    const_cast<float*>(a.qp), const_cast<float*>(a.up), s);
-    if (e == cudaSuccess && h->ev_start) e = cudaEventRecord(h->ev_start, s);
-    if (e == cudaSuccess) e = launch_decode(h->d, G, p.use_mma, a, s);
-    if (e == cudaSuccess && h->ev_stop) e = cudaEventRecord(h->ev_stop, s);
-    if (e == cudaSuccess) e = launch_combine(h->d, B * Hq, p.nsplit, a.part_ml, a.part_acc, h->dsign, out, s);
+    cudaError_t e = cudaSuccess;
+    const bool chained = !empty_k;
+    if (chained) {
+        // K encode as a plain launch, V encode and the prologue as its
+        // programmatic dependents (each completes only after its predecessor);
+        // the split-K kernel prefetches every chunk but the appended tokens'
+        // before it waits.
+        e = launch_encode(h->d, true, kv_dtype, ek, h->num_sms, false, s);
+        if (e == cudaSuccess) e = launch_encode(h->d, false, kv_dtype, ev, h->num_sms, true, s);
+        a.fresh_lo = t0;
+        a.fresh_hi = t0 + Tnew;
+    }
+    if (e == cudaSuccess) e = launch_attend(h, q, q_dtype, p, a, out, chained, s);
     return cuda_status(e);
 }
 

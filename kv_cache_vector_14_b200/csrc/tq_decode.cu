@@ -44,56 +44,56 @@ __device__ void smem_fwht(float* v) {
 }
 
 // ---------------------------------------------------------------- prologue
-// q' = H D q / sqrt(d) and up = sqrt(pi/2)/m * S q' for kQH query heads per
-// CTA.  S^T is staged through shared memory in chunks of kJC rows with wide,
-// independent loads; each thread then owns one JL row i for all kQH heads.
-constexpr int kQH = 1;
-constexpr int kJC = 64;
+// q' = H D q / sqrt(d) and up = sqrt(pi/2)/m * S q'.  A CTA takes kPQH(D) =
+// D / kRC query heads and one chunk of kRC rows of S: it transforms its heads
+// in shared memory, stages the kRC columns of S^T it needs (one L2 read of S
+// per head group, not per head), and thread t computes row t % kRC of head
+// t / kRC.  The CTAs of row chunk 0 also store q'.
+constexpr int kRC = 32;
 
 template <int D, int DT>
 __global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t BHq, const float* dsign,
                                                         const float* ST, float* qp, float* up) {
-    __shared__ float v[kQH * D];
-    extern __shared__ __align__(16) float sst[];          // [kJC][D] rows of S^T
+    constexpr int QH = D / kRC;
+    __shared__ float v[QH * D];
+    __shared__ __align__(16) float sst[D * kRC];           // sst[j][i] = S[rc*kRC + i][j]
     pdl_trigger();                                        // the split-K kernel may start its prefetch
-    const int j = threadIdx.x;
-    const int64_t h0 = (int64_t)blockIdx.x * kQH;
-    const float ds = dsign[j];
+    const int t = threadIdx.x;
+    const int64_t h0 = (int64_t)blockIdx.x * QH;
+    const int rc = blockIdx.y;
+    // S^T columns of this row chunk: D rows of kRC floats
+    for (int i = t; i < D * kRC / 4; i += D) {
+        const int jr = i / (kRC / 4), c4 = i % (kRC / 4);
+        reinterpret_cast<float4*>(sst)[i] = __ldg(reinterpret_cast<const float4*>(ST + (size_t)jr * D + rc * kRC) + c4);
+    }
+    const float ds = dsign[t];
 #pragma unroll
-    for (int k = 0; k < kQH; ++k) {
+    for (int k = 0; k < QH; ++k) {
         const int64_t h = h0 + k;
-        v[k * D + j] = (h < BHq) ? ds * load_q<DT>(q, h * D + j) : 0.f;
+        v[k * D + t] = (h < BHq) ? ds * load_q<DT>(q, h * D + t) : 0.f;
     }
     __syncthreads();
-    smem_fwht<D, kQH>(v);
+    smem_fwht<D, QH>(v);
     const float inv = 1.0f / sqrtf((float)D);
 #pragma unroll
-    for (int k = 0; k < kQH; ++k) v[k * D + j] *= inv;
-    float u[kQH];
-#pragma unroll
-    for (int k = 0; k < kQH; ++k) u[k] = 0.f;
-    for (int j0 = 0; j0 < D; j0 += kJC) {
-        __syncthreads();
-        const float4* src = reinterpret_cast<const float4*>(ST + (size_t)j0 * D);
+    for (int k = 0; k < QH; ++k) v[k * D + t] *= inv;
+    __syncthreads();
+    const int i = t % kRC, k = t / kRC;
+    float u0 = 0.f, u1 = 0.f;
 #pragma unroll 8
-        for (int i = j; i < kJC * D / 4; i += D) reinterpret_cast<float4*>(sst)[i] = __ldg(src + i);
-        __syncthreads();
-#pragma unroll 8
-        for (int jj = 0; jj < kJC; ++jj) {
-            const float sv = sst[jj * D + j];                 // S[j][j0 + jj]
-#pragma unroll
-            for (int k = 0; k < kQH; ++k) u[k] = fmaf(sv, v[k * D + j0 + jj], u[k]);
-        }
+    for (int jj = 0; jj < D; jj += 2) {
+        u0 = fmaf(sst[jj * kRC + i], v[k * D + jj], u0);
+        u1 = fmaf(sst[(jj + 1) * kRC + i], v[k * D + jj + 1], u1);
     }
     const float cq = 1.2533141373155003f / (float)D;       // sqrt(pi/2) / m
+    const int64_t h = h0 + k;
+    if (h < BHq) up[h * D + rc * kRC + i] = cq * (u0 + u1);
+    if (rc == 0) {
 #pragma unroll
-    for (int k = 0; k < kQH; ++k) {
-        const int64_t h = h0 + k;
-        if (h < BHq) {
-            qp[h * D + j] = v[k * D + j];
-            up[h * D + j] = cq * u[k];
-        }
+        for (int kk = 0; kk < QH; ++kk)
+            if (h0 + kk < BHq) qp[(h0 + kk) * D + t] = v[kk * D + t];
     }
+    pdl_wait();          // chained after an encode (fused step): complete only after it
 }
 
 // ---------------------------------------------------------------- SIMT decode
@@ -286,25 +286,23 @@ __global__ void __launch_bounds__(D) tq_combine_kernel(const float* part_ml, con
 }
 
 template <int D, int DT>
-cudaError_t launch_prologue_t(int grid, size_t smem, const void* q, int64_t BHq, const float* dsign, const float* st,
+cudaError_t launch_prologue_t(dim3 grid, bool pdl, const void* q, int64_t BHq, const float* dsign, const float* st,
                               float* qp, float* up, cudaStream_t s) {
-    auto kern = tq_prologue_kernel<D, DT>;
-    cudaError_t e = set_smem_once<tq_prologue_kernel<D, DT>>((int)smem);
-    if (e != cudaSuccess) return e;
-    kern<<<grid, D, smem, s>>>(q, BHq, dsign, st, qp, up);
+    if (pdl) return launch_pdl(tq_prologue_kernel<D, DT>, grid, dim3(D), 0, s, q, BHq, dsign, st, qp, up);
+    tq_prologue_kernel<D, DT><<<grid, D, 0, s>>>(q, BHq, dsign, st, qp, up);
     return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_prologue_d(const void* q, tq_dtype dt, int64_t BHq, const float* dsign, const float* st,
-                              float* qp, float* up, cudaStream_t s) {
-    const int grid = (int)((BHq + kQH - 1) / kQH);
-    if (grid == 0) return cudaSuccess;
-    const size_t smem = (size_t)kJC * D * sizeof(float);
+                              float* qp, float* up, bool pdl, cudaStream_t s) {
+    const int64_t groups = (BHq + D / kRC - 1) / (D / kRC);
+    if (groups == 0) return cudaSuccess;
+    const dim3 grid((unsigned)groups, D / kRC);
     switch (dt) {
-        case TQ_F32: return launch_prologue_t<D, TQ_F32>(grid, smem, q, BHq, dsign, st, qp, up, s);
-        case TQ_BF16: return launch_prologue_t<D, TQ_BF16>(grid, smem, q, BHq, dsign, st, qp, up, s);
-        case TQ_F16: return launch_prologue_t<D, TQ_F16>(grid, smem, q, BHq, dsign, st, qp, up, s);
+        case TQ_F32: return launch_prologue_t<D, TQ_F32>(grid, pdl, q, BHq, dsign, st, qp, up, s);
+        case TQ_BF16: return launch_prologue_t<D, TQ_BF16>(grid, pdl, q, BHq, dsign, st, qp, up, s);
+        case TQ_F16: return launch_prologue_t<D, TQ_F16>(grid, pdl, q, BHq, dsign, st, qp, up, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -329,9 +327,9 @@ cudaError_t launch_simt_g(int G, const DecArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, const float* dsign, const float* st,
-                            float* qp, float* up, cudaStream_t s) {
-    if (d == 128) return launch_prologue_d<128>(q, dt, BHq, dsign, st, qp, up, s);
-    if (d == 256) return launch_prologue_d<256>(q, dt, BHq, dsign, st, qp, up, s);
+                            float* qp, float* up, bool pdl, cudaStream_t s) {
+    if (d == 128) return launch_prologue_d<128>(q, dt, BHq, dsign, st, qp, up, pdl, s);
+    if (d == 256) return launch_prologue_d<256>(q, dt, BHq, dsign, st, qp, up, pdl, s);
     return cudaErrorInvalidValue;
 }
 

@@ -223,10 +223,25 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         bulk_g2s(smem_u32(st + C::kOffVc), vb + sub * ch * cb, ch * cb, bar);
         bulk_g2s(smem_u32(st + C::kOffVn), vb + 64 * cb + sub * 2 * ch, 2 * ch, bar);
     };
+    // chunks holding tokens that a chained encode writes are fetched only after pdl_wait
+    auto fresh = [&](int i) {
+        const int64_t t0 = s0 + (int64_t)(warp + i * NW) * C::kChunk;
+        return t0 < a.fresh_hi && a.fresh_lo < t0 + C::kChunk;
+    };
     if (lane == 0) {
-        for (int i = 0; i < kStages && i < nmine; ++i) issue(i);
+        for (int i = 0; i < kStages && i < nmine; ++i)
+            if (!fresh(i)) issue(i);
     }
     pdl_wait();                           // q' and u' come from the prologue kernel
+    if (lane == 0) {
+        bool any = false;
+        for (int i = 0; i < kStages && i < nmine; ++i) any |= fresh(i);
+        if (any) {
+            asm volatile("fence.proxy.async;" ::: "memory");
+            for (int i = 0; i < kStages && i < nmine; ++i)
+                if (fresh(i)) issue(i);
+        }
+    }
 
     // B-operand fragment of k-step kc: column n = gr of n-tile nt is head
     // 4 nt + gr / 2, limb gr % 2; rows 16 kc + 2 tq4 (+1), +8 (+9)

@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
     uint8_t* sCode = smem + SM::s_bytes + SM::r_bytes;                 // [kTileV][D], slot order
     __shared__ float sC[8];
 
+    pdl_trigger();                 // a chained kernel may start (it waits for this one's writes)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t N = a.B * a.Hkv * a.Tnew;
     const int64_t ntiles = (N + kTileV - 1) / kTileV;
@@ -254,6 +255,7 @@ __global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
         }
         __syncthreads();
     }
+    pdl_wait();                    // when chained: complete only after the previous kernel
 }
 
 // ---------------------------------------------------------------- small batches (K)
@@ -272,6 +274,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(con
     __shared__ __align__(16) float sr[kSmallWarps][D];
     __shared__ __align__(16) uint8_t scode[kSmallWarps][D];
     __shared__ float sC[8];
+    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x < 8) sC[threadIdx.x] = a.cb.c[threadIdx.x];
     __syncthreads();
@@ -346,7 +349,10 @@ __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(con
             for (int r = 0; r < R; ++r) z[r] = fmaf(rj, sS[(jj * R + r) * 32 + lane], z[r]);
         }
     }
-    if (!valid) return;
+    if (!valid) {
+        pdl_wait();
+        return;
+    }
     uint32_t mine = 0;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -362,10 +368,11 @@ __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(con
         const uint32_t tail = nibbles8(sw[6], sw[7]);
         reinterpret_cast<uint32_t*>(blk + (t & 63) * code_bytes(D))[lane] = main | (((tail >> g) & 0x11111111u) << 3);
     }
+    pdl_wait();
 }
 
 template <int D, bool IS_K, int DT, int TV>
-cudaError_t launch_enc_tv(const EncArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_enc_tv(const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
     using SM = EncSmem<D, IS_K, TV>;
     auto kern = tq_encode_kernel<D, IS_K, DT, TV>;
     cudaError_t e = set_smem_once<tq_encode_kernel<D, IS_K, DT, TV>>((int)SM::total);
@@ -377,12 +384,13 @@ cudaError_t launch_enc_tv(const EncArgs& a, int num_sms, cudaStream_t s) {
     const int64_t cap = (int64_t)num_sms * (IS_K ? 2 : 8);
     const int grid = (int)(ntiles < cap ? ntiles : cap);
     if (grid <= 0) return cudaSuccess;
+    if (pdl) return launch_pdl(kern, dim3(grid), dim3(kThreads), SM::total, s, a);
     kern<<<grid, kThreads, SM::total, s>>>(a);
     return cudaGetLastError();
 }
 
 template <int D, bool IS_K, int DT>
-cudaError_t launch_enc_t(const EncArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_enc_t(const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
     const int64_t N = a.B * a.Hkv * a.Tnew;
     if constexpr (IS_K) {
         if (N <= (int64_t)4 * num_sms) {        // appends: one warp per vector
@@ -391,29 +399,31 @@ cudaError_t launch_enc_t(const EncArgs& a, int num_sms, cudaStream_t s) {
             auto kern = tq_encode_k_small_kernel<D, DT>;
             cudaError_t e = set_smem_once<tq_encode_k_small_kernel<D, DT>>((int)smem);
             if (e != cudaSuccess) return e;
+            if (pdl) return launch_pdl(kern, dim3(grid), dim3(kSmallWarps * 32), smem, s, a);
             kern<<<grid, kSmallWarps * 32, smem, s>>>(a);
             return cudaGetLastError();
         }
     }
-    if (N < (int64_t)32 * num_sms) return launch_enc_tv<D, IS_K, DT, 8>(a, num_sms, s);
-    return launch_enc_tv<D, IS_K, DT, 32>(a, num_sms, s);
+    if (N < (int64_t)32 * num_sms) return launch_enc_tv<D, IS_K, DT, 8>(a, num_sms, pdl, s);
+    return launch_enc_tv<D, IS_K, DT, 32>(a, num_sms, pdl, s);
 }
 
 template <int D, bool IS_K>
-cudaError_t launch_enc_dt(tq_dtype dt, const EncArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_enc_dt(tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
     switch (dt) {
-        case TQ_F32: return launch_enc_t<D, IS_K, TQ_F32>(a, num_sms, s);
-        case TQ_BF16: return launch_enc_t<D, IS_K, TQ_BF16>(a, num_sms, s);
-        case TQ_F16: return launch_enc_t<D, IS_K, TQ_F16>(a, num_sms, s);
+        case TQ_F32: return launch_enc_t<D, IS_K, TQ_F32>(a, num_sms, pdl, s);
+        case TQ_BF16: return launch_enc_t<D, IS_K, TQ_BF16>(a, num_sms, pdl, s);
+        case TQ_F16: return launch_enc_t<D, IS_K, TQ_F16>(a, num_sms, pdl, s);
     }
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, cudaStream_t s) {
-    if (d == 128) return launch_encode128(is_k, dt, a, num_sms, s);
-    if (d == 256) return is_k ? launch_enc_dt<256, true>(dt, a, num_sms, s) : launch_enc_dt<256, false>(dt, a, num_sms, s);
+cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
+    if (d == 128) return launch_encode128(is_k, dt, a, num_sms, pdl, s);
+    if (d == 256)
+        return is_k ? launch_enc_dt<256, true>(dt, a, num_sms, pdl, s) : launch_enc_dt<256, false>(dt, a, num_sms, pdl, s);
     return cudaErrorInvalidValue;
 }
 

@@ -334,6 +334,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffBar + 32);
     uint8_t* scode = sm + kOffCode;
     __shared__ float sC[8];
+    pdl_trigger();                 // a chained kernel may start (it waits for this one's writes)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 3, l = lane & 7;
     const int64_t N = a.B * a.Hkv * a.Tnew;
@@ -480,6 +481,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
         tc_fence_after();
         tc_dealloc(tmem, 2 * kTcRows);
     }
+    pdl_wait();                    // when chained: complete only after the previous kernel
 }
 
 // ---------------------------------------------------------------- V kernel
@@ -488,6 +490,7 @@ constexpr int kVWarps = 8;
 template <int DT>
 __global__ void __launch_bounds__(kVWarps * 32, 3) tq_encode_v128_kernel(const EncArgs a) {
     __shared__ __align__(16) uint8_t scode[kVWarps][4][128];
+    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 3, l = lane & 7;
     const int64_t N = a.B * a.Hkv * a.Tnew;
     const int64_t nquads = (N + 3) / 4;
@@ -512,10 +515,11 @@ __global__ void __launch_bounds__(kVWarps * 32, 3) tq_encode_v128_kernel(const E
         store_code_words(&scode[warp][0][0], blk + tau * code_bytes(kD), (int)(N - gv0 < 4 ? N - gv0 : 4), lane);
         __syncwarp();
     }
+    pdl_wait();
 }
 
 template <int DT>
-cudaError_t launch_t(bool is_k, const EncArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_t(bool is_k, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
     const int64_t N = a.B * a.Hkv * a.Tnew;
     if (N <= 0) return cudaSuccess;
     if (is_k) {
@@ -528,23 +532,26 @@ cudaError_t launch_t(bool is_k, const EncArgs& a, int num_sms, cudaStream_t s) {
         auto kern = tq_encode_k128_tc_kernel<DT>;
         cudaError_t e = set_smem_once<tq_encode_k128_tc_kernel<DT>>(kSmemK);
         if (e != cudaSuccess) return e;
+        if (pdl) return launch_pdl(kern, dim3(grid), dim3(kWarps * 32), kSmemK, s, a, (int)rows);
         kern<<<grid, kWarps * 32, kSmemK, s>>>(a, (int)rows);
         return cudaGetLastError();
     }
     const int64_t nquads = (N + 3) / 4;
     const int64_t ctas = (nquads + kVWarps - 1) / kVWarps;
     const int64_t cap = (int64_t)num_sms * 8;
-    tq_encode_v128_kernel<DT><<<(unsigned)(ctas < cap ? ctas : cap), kVWarps * 32, 0, s>>>(a);
+    const unsigned grid = (unsigned)(ctas < cap ? ctas : cap);
+    if (pdl) return launch_pdl(tq_encode_v128_kernel<DT>, dim3(grid), dim3(kVWarps * 32), 0, s, a);
+    tq_encode_v128_kernel<DT><<<grid, kVWarps * 32, 0, s>>>(a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_encode128(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_encode128(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
     switch (dt) {
-        case TQ_F32: return launch_t<TQ_F32>(is_k, a, num_sms, s);
-        case TQ_BF16: return launch_t<TQ_BF16>(is_k, a, num_sms, s);
-        case TQ_F16: return launch_t<TQ_F16>(is_k, a, num_sms, s);
+        case TQ_F32: return launch_t<TQ_F32>(is_k, a, num_sms, pdl, s);
+        case TQ_BF16: return launch_t<TQ_BF16>(is_k, a, num_sms, pdl, s);
+        case TQ_F16: return launch_t<TQ_F16>(is_k, a, num_sms, pdl, s);
     }
     return cudaErrorInvalidValue;
 }

@@ -114,6 +114,7 @@ struct DecArgs {
     float* part_ml;           // [B*Hq][nsplit][2] (running max in log2 units, sum)
     float* part_acc;          // [B*Hq][nsplit][d] rotated-domain accumulators
     int* err;                 // device check word
+    int64_t fresh_lo, fresh_hi;   // tokens written by a chained encode: read only after pdl_wait
     Codebook cb;
 };
 
@@ -156,11 +157,13 @@ cudaError_t set_smem_once(int bytes) {
 }
 
 // Kernel launchers (tq_encode.cu, tq_decode.cu); return a CUDA error code.
-cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms,
+cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl,
                           cudaStream_t s);
-cudaError_t launch_encode128(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_encode128(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s);
+// pdl: launched as a programmatic dependent of the previous kernel (fused
+// append-and-attend step); the kernels then complete only after it.
 cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, const float* dsign,
-                            const float* st, float* qp, float* up, cudaStream_t s);
+                            const float* st, float* qp, float* up, bool pdl, cudaStream_t s);
 cudaError_t launch_decode(int d, int G, bool use_mma, const DecArgs& a, cudaStream_t s);
 cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml,
                            const float* part_acc, const float* dsign, float* out, cudaStream_t s);

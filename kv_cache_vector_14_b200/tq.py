@@ -22,6 +22,7 @@ TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 
 EXPORTED = ("tq_params_host", "tq_init", "tq_destroy", "tq_get_params", "tq_head_dim", "tq_block_bytes",
             "tq_cache_bytes", "tq_encode_k", "tq_encode_v", "tq_attend_workspace_bytes", "tq_attend_decode",
+            "tq_append_attend",
             "tq_attend_decode_static", "tq_device_status", "tq_set_decode_events", "tq_set_decode_path", "tq_attend_path", "tq_status_string")
 
 
@@ -74,6 +75,9 @@ def lib() -> C.CDLL:
             L.tq_attend_decode_static.argtypes = [P, P, i32, i64, i64, C.POINTER(tq_cache), C.POINTER(tq_cache), P,
                                                   i64, C.c_float, P, P]
             L.tq_attend_decode_static.restype = st
+            L.tq_append_attend.argtypes = [P, P, P, i32, i64, i64, i64, i64, C.POINTER(tq_cache),
+                                           C.POINTER(tq_cache), i64, P, i32, i64, C.c_float, P, P, C.c_size_t, P]
+            L.tq_append_attend.restype = st
             L.tq_device_status.argtypes = [P, P]
             L.tq_device_status.restype = st
             L.tq_set_decode_events.argtypes = [P, P, P]
@@ -213,6 +217,24 @@ def tq_attend_decode(h, q, kc: Cache, vc: Cache, out, ws, T: int = 0, seq_lens=N
                                   C.byref(vc.struct), sl, T, float(scale), C.c_void_p(out.data_ptr()),
                                   C.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(), _stream(stream)),
            "tq_attend_decode")
+
+
+def tq_append_attend(h, k_new, v_new, kc: Cache, vc: Cache, t0: int, q, out, ws, scale: float = 1.0,
+                     stream=None) -> None:
+    """Fused decode step: append k_new/v_new ([B, Hkv, Tnew, d], same dtype and
+    strides) at positions [t0, t0 + Tnew), then attend over t0 + Tnew tokens."""
+    if k_new.dim() != 4 or k_new.stride(-1) != 1 or k_new.shape != v_new.shape or \
+            k_new.stride() != v_new.stride() or k_new.dtype != v_new.dtype:
+        raise ValueError("tq_append_attend: k_new, v_new must be [B, Hkv, Tnew, d] with equal dtype and strides")
+    if q.dim() != 3 or not q.is_contiguous():
+        raise ValueError("tq_append_attend: q must be contiguous [B, Hq, d]")
+    Tnew = k_new.shape[2]
+    sb, sh, st, _ = k_new.stride()
+    _check(lib().tq_append_attend(h, C.c_void_p(k_new.data_ptr()), C.c_void_p(v_new.data_ptr()),
+                                  _dtype_code(k_new), Tnew, sb, sh, st, C.byref(kc.struct), C.byref(vc.struct), t0,
+                                  C.c_void_p(q.data_ptr()), _dtype_code(q), q.shape[1], float(scale),
+                                  C.c_void_p(out.data_ptr()), C.c_void_p(ws.data_ptr()),
+                                  ws.numel() * ws.element_size(), _stream(stream)), "tq_append_attend")
 
 
 def tq_device_status(h, stream=None) -> int:

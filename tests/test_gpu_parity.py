@@ -217,9 +217,48 @@ def test_append_and_attend_loop_d256(handles, prms):
 
 
 @pytest.mark.parametrize("d", [128, 256])
-def test_append_and_attend_graph_replay_equals_eager(handles, d):
-    """The append-and-attend step sequence captured in a CUDA graph and
-    replayed gives the same outputs, bit for bit, as launching it eagerly."""
+@pytest.mark.parametrize("G,T0,Tnew", [(2, 0, 1), (4, 63, 1), (1, 64, 3), (8, 200, 2), (4, 1000, 1)])
+def test_fused_append_attend_equals_separate_calls(handles, d, G, T0, Tnew):
+    """tq_append_attend writes the same cache bytes and outputs, bit for bit, as
+    tq_encode_k + tq_encode_v + tq_attend_decode, over several steps, with the
+    new tokens at the start, middle and end of chunks and splits."""
+    h = handles[d]
+    B, Hkv, S = 2, 2, 4
+    Hq = Hkv * G
+    Tend = T0 + S * Tnew
+    Tcap = (Tend + 63) // 64 * 64
+    x = torch_input(synthetic.gaussian((2, B, Hkv, Tend, d), seed=11 + G), "bf16")
+    q = torch_input(synthetic.gaussian((S, B, Hq, d), seed=12), "f32")
+    caches = []
+    for _ in range(2):
+        kc, vc = tq.Cache(d, True, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
+        if T0:
+            tq.tq_encode_k(h, x[0, :, :, :T0], kc, 0)
+            tq.tq_encode_v(h, x[1, :, :, :T0], vc, 0)
+        caches.append((kc, vc))
+    ws = torch.empty(tq.tq_attend_workspace_bytes(h, B, Hq, Hkv, Tend), dtype=torch.uint8, device="cuda")
+    for s in range(S):
+        t0 = T0 + s * Tnew
+        (kc, vc), (kf, vf) = caches
+        ref = torch.empty((B, Hq, d), dtype=torch.float32, device="cuda")
+        out = torch.full((B, Hq, d), float("nan"), dtype=torch.float32, device="cuda")
+        tq.tq_encode_k(h, x[0, :, :, t0:t0 + Tnew], kc, t0)
+        tq.tq_encode_v(h, x[1, :, :, t0:t0 + Tnew], vc, t0)
+        tq.tq_attend_decode(h, q[s], kc, vc, ref, ws, T=t0 + Tnew, scale=1.0 / np.sqrt(d))
+        tq.tq_append_attend(h, x[0, :, :, t0:t0 + Tnew], x[1, :, :, t0:t0 + Tnew], kf, vf, t0, q[s], out, ws,
+                            scale=1.0 / np.sqrt(d))
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref), f"step {s}"
+        assert torch.equal(kf.buf, kc.buf) and torch.equal(vf.buf, vc.buf), f"step {s}"
+    assert tq.tq_device_status(h) == tq.TQ_OK
+
+
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("fused", [False, True])
+def test_append_and_attend_graph_replay_equals_eager(handles, d, fused):
+    """The append-and-attend step sequence (separate calls, or the fused
+    tq_append_attend) captured in a CUDA graph and replayed gives the same
+    outputs, bit for bit, as launching it eagerly."""
     h = handles[d]
     B, Hq, Hkv, T0, S = 2, 8, 2, 200, 12
     Tcap = (T0 + S + 63) // 64 * 64
@@ -235,6 +274,10 @@ def test_append_and_attend_graph_replay_equals_eager(handles, d):
     def sequence():
         for s in range(S):
             T = T0 + s
+            if fused:
+                tq.tq_append_attend(h, xk[:, :, T:T + 1], xv[:, :, T:T + 1], kc, vc, T, q[s], out[s], ws,
+                                    scale=1.0 / np.sqrt(d))
+                continue
             tq.tq_encode_k(h, xk[:, :, T:T + 1], kc, T)
             tq.tq_encode_v(h, xv[:, :, T:T + 1], vc, T)
             tq.tq_attend_decode(h, q[s], kc, vc, out[s], ws, T=T + 1, scale=1.0 / np.sqrt(d))
