@@ -353,6 +353,71 @@ def measure_loop(dev, world: int, dist, replays: int = 5) -> dict:
             "l2": "cache (~250 MB) larger than L2; no flush between replays", "device_status": status}
 
 
+def exact_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.ndarray:
+    """Softmax attention in float64 over unquantised keys and values (ground
+    truth for the quality comparison, not the method): q [G, d], k, v [T, d]."""
+    s = (q.astype(np.float64) @ k.astype(np.float64).T) * scale
+    s -= s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    return (p / p.sum(axis=1, keepdims=True)) @ v.astype(np.float64)
+
+
+def measure_polar(h, dev, w, vc, q, out_qjl, ws, n_calls: int) -> dict:
+    """PolarQuant-only K on the long-context workload: the K vectors encoded
+    without the QJL bit (V layout, 50 B per token at d=128), attention timed
+    on its own (split-K kernel by events, and the whole call), and the output
+    error of both K flows against exact attention over the unquantised data
+    for one sequence and kv head."""
+    import torch
+    from kv_cache_vector_14_b200 import tq
+    d, B, Hq, Hkv, T = w.d, w.B, w.Hq, w.Hkv, w.T
+    kp = tq.Cache(d, False, B, Hkv, T)
+    x = torch.from_numpy(synthetic.kv(w, "k")).to(dev)
+    tq.tq_encode_v(h, x, kp, 0)
+    del x
+    out = torch.empty_like(out_qjl)
+    for _ in range(5):
+        tq.tq_attend_decode_polar(h, q, kp, vc, out, ws, T=T, scale=w.scale)
+    torch.cuda.synchronize()
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_calls)]
+    for a_, b_ in kev:
+        a_.record()
+        b_.record()
+    torch.cuda.synchronize()
+    for i in range(n_calls):
+        tq.tq_set_decode_events(h, kev[i][0], kev[i][1])
+        tq.tq_attend_decode_polar(h, q, kp, vc, out, ws, T=T, scale=w.scale)
+    torch.cuda.synchronize()
+    tq.tq_set_decode_events(h, None, None)
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_calls):
+        tq.tq_attend_decode_polar(h, q, kp, vc, out, ws, T=T, scale=w.scale)
+    e1.record()
+    torch.cuda.synchronize()
+    call_ms = e0.elapsed_time(e1) / n_calls
+    G = Hq // Hkv
+    kx = synthetic.kv(w, "k", batches=[0])[0, 0]
+    vx = synthetic.kv(w, "v", batches=[0])[0, 0]
+    qx = q[0, :G].float().cpu().numpy()
+    ref = exact_attention(qx, kx, vx, w.scale)
+
+    def rel(o):        # mean over the query heads of ||o - ref||_2 / ||ref||_2
+        return float((np.linalg.norm(o - ref, axis=1) / np.linalg.norm(ref, axis=1)).mean())
+
+    nbytes = B * Hkv * T * 100          # 50 B K + 50 B V per token per kv head at d=128
+    del kp
+    return {"workload": w.title + ", K without the QJL bit (3.125 b/dim)", "bytes_per_token_head": 100,
+            "kernel_ms": kern_ms, "call_ms": call_ms, "achieved_gbs": nbytes / (kern_ms * 1e-3) / 1e9,
+            "quality_vs_exact_attention": {
+                "sample": f"batch 0, kv head 0: {G} query heads over {T} tokens, float64 softmax attention "
+                          "over the unquantised K and V",
+                "metric": "mean over query heads of relative L2 error of the attention output",
+                "qjl_k": rel(out_qjl[0, :G].cpu().numpy().astype(np.float64)),
+                "polar_k": rel(out[0, :G].cpu().numpy().astype(np.float64))}}
+
+
 def run_ours(args, rank: int, world: int, dist):
     import torch
     from kv_cache_vector_14_b200 import build, tq
@@ -487,6 +552,9 @@ def run_ours(args, rank: int, world: int, dist):
     h2d = (kh.numel() + vh.numel()) * 4 + qh.numel() * 2
     d2h = oh.numel() * 4
 
+    tq.tq_attend_decode(h, q, kc, vc, out, ws, T=T, scale=w.scale)     # QJL output for the quality check
+    torch.cuda.synchronize()
+    polar = measure_polar(h, dev, w, vc, q, out.clone(), ws, n_kern)
     enc = measure_encode(h, dev, world, dist)
     loop = measure_loop(dev, world, dist)
 
@@ -529,6 +597,7 @@ def run_ours(args, rank: int, world: int, dist):
         "clocks": clocks,
         "encode": {**enc, "frac": enc["achieved_gbs"] / peak, "cpu_baseline": enc_cpu},
         "loop": {**loop, "frac": loop["achieved_gbs"] / peak},
+        "polar_k": {**polar, "frac": polar["achieved_gbs"] / peak},
         "device_status": tq.tq_status_string(status),
     }
     print(json.dumps(line), flush=True)

@@ -165,6 +165,23 @@ TQ_API tq_status tq_attend_decode(const tq_handle* h, const void* q, tq_dtype qd
                            const int32_t* seq_lens, int64_t T, float scale, float* out, void* ws,
                            size_t ws_bytes, void* stream);
 
+/* ---- PolarQuant-only K (no QJL bit) --------------------------------------- */
+
+/* Attention over a PolarQuant-only K cache: K stored like V, with 3-bit codes
+ * and the fp16 norm but no QJL sign bits and no gamma (3.125 bits/dim at
+ * d = 128 instead of 4.25).  Encode such a K cache with tq_encode_v into a
+ * V-layout buffer (tq_cache_bytes(d, 0, ...)).  Scores drop the QJL term:
+ *   s_t = scale * n_t * <q', c[idx_t]>,
+ * the rest as tq_attend_decode (same arguments, workspace and errors).  The
+ * page weighs the two K flows against each other: its K section adds the
+ * 1-bit QJL residual to correct the inner-product bias of the 3-bit codes,
+ * and its hybrid V2+V3 section trades that accuracy against the faster
+ * PolarQuant-only path. */
+TQ_API tq_status tq_attend_decode_polar(const tq_handle* h, const void* q, tq_dtype qdtype, int64_t B,
+                                        int64_t Hq, const tq_cache* kc, const tq_cache* vc,
+                                        const int32_t* seq_lens, int64_t T, float scale, float* out, void* ws,
+                                        size_t ws_bytes, void* stream);
+
 /* ---- fused append-and-attend step ---------------------------------------- */
 
 /* One decode step of a serving loop: encode Tnew new K and V vectors per

@@ -170,12 +170,12 @@ tq_status prepare_attend(const tq_handle* h, const void* q, tq_dtype qdt, int64_
 // Prologue, split-K attention, combine.  chained: the prologue is a
 // programmatic dependent of the kernel before it (the fused step's encodes).
 cudaError_t launch_attend(const tq_handle* h, const void* q, tq_dtype qdt, const DecodePlan& p, const DecArgs& a,
-                          float* out, bool chained, cudaStream_t s) {
+                          float* out, bool chained, cudaStream_t s, bool qjl = true) {
     const int64_t BHq = a.B * a.Hq;
     cudaError_t e = launch_prologue(h->d, q, qdt, BHq, h->dsign, h->dST, const_cast<float*>(a.qp),
                                     const_cast<float*>(a.up), chained, s);
     if (e == cudaSuccess && h->ev_start) e = cudaEventRecord(h->ev_start, s);
-    if (e == cudaSuccess) e = launch_decode(h->d, p.G, p.use_mma, a, s);
+    if (e == cudaSuccess) e = launch_decode(h->d, p.G, p.use_mma, qjl, a, s);
     if (e == cudaSuccess && h->ev_stop) e = cudaEventRecord(h->ev_stop, s);
     if (e == cudaSuccess) e = launch_combine(h->d, BHq, p.nsplit, a.part_ml, a.part_acc, h->dsign, out, s);
     return e;
@@ -335,6 +335,16 @@ tq_status tq_attend_decode(const tq_handle* h, const void* q, tq_dtype qdt, int6
     const tq_status r = prepare_attend(h, q, qdt, B, Hq, kc, vc, seq_lens, T, scale, out, ws, ws_bytes, &p, &a);
     if (r != TQ_OK || B == 0) return r;
     return cuda_status(launch_attend(h, q, qdt, p, a, out, false, static_cast<cudaStream_t>(stream)));
+}
+
+tq_status tq_attend_decode_polar(const tq_handle* h, const void* q, tq_dtype qdt, int64_t B, int64_t Hq,
+                                 const tq_cache* kc, const tq_cache* vc, const int32_t* seq_lens, int64_t T,
+                                 float scale, float* out, void* ws, size_t ws_bytes, void* stream) {
+    DecodePlan p;
+    DecArgs a;
+    const tq_status r = prepare_attend(h, q, qdt, B, Hq, kc, vc, seq_lens, T, scale, out, ws, ws_bytes, &p, &a);
+    if (r != TQ_OK || B == 0) return r;
+    return cuda_status(launch_attend(h, q, qdt, p, a, out, false, static_cast<cudaStream_t>(stream), false));
 }
 
 tq_status tq_append_attend(const tq_handle* h, const void* k_new, const void* v_new, tq_dtype kv_dtype,

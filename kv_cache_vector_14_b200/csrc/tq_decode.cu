@@ -116,7 +116,7 @@ __device__ __forceinline__ int sign_from_words(const uint32_t* w, int j) {
     return (int)((w[4 * s + t] >> bit) & 1u);
 }
 
-template <int D, int G>
+template <int D, int G, bool QJL>
 __global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
     constexpr int R = D / 32;
     __shared__ float sC[8];
@@ -136,7 +136,8 @@ __global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
     const int64_t w1 = (w0 + per < s1) ? w0 + per : s1;
 
     const int64_t seq = (int64_t)b * a.Hkv + hkv;
-    const int64_t kbb = block_bytes(D, true), vbb = block_bytes(D, false);
+    const int64_t kbb = block_bytes(D, QJL), vbb = block_bytes(D, false);
+    const int64_t knorm = kBlockT * (code_bytes(D) + (QJL ? sign_bytes(D) : 0));
     pdl_wait();                                           // q' and u' from the prologue
     float q[G][R], u[G][R], acc[G][R], mrun[G], lrun[G];
 #pragma unroll
@@ -160,8 +161,8 @@ __global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
         const uint32_t* kw = reinterpret_cast<const uint32_t*>(kb + tau * code_bytes(D));
         const uint32_t* sw = reinterpret_cast<const uint32_t*>(kb + kBlockT * code_bytes(D) + tau * sign_bytes(D));
         const uint32_t* vw = reinterpret_cast<const uint32_t*>(vb + tau * code_bytes(D));
-        const float nk = __half2float(reinterpret_cast<const __half*>(kb + kBlockT * (code_bytes(D) + sign_bytes(D)))[tau]);
-        const float gk = __half2float(reinterpret_cast<const __half*>(kb + kBlockT * (code_bytes(D) + sign_bytes(D)) + 2 * kBlockT)[tau]);
+        const float nk = __half2float(reinterpret_cast<const __half*>(kb + knorm)[tau]);
+        const float gk = QJL ? __half2float(reinterpret_cast<const __half*>(kb + knorm + 2 * kBlockT)[tau]) : 0.f;
         const float nv = __half2float(reinterpret_cast<const __half*>(vb + kBlockT * code_bytes(D))[tau]);
         float part[G];
 #pragma unroll
@@ -171,10 +172,15 @@ __global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
         for (int r = 0; r < R; ++r) {
             const int j = lane + 32 * r;
             const float ck = sC[code_from_words(kw, j)];
-            const float sg = sign_from_words(sw, j) ? gk : -gk;
             cv[r] = sC[code_from_words(vw, j)];
+            if constexpr (QJL) {
+                const float sg = sign_from_words(sw, j) ? gk : -gk;
 #pragma unroll
-            for (int g = 0; g < G; ++g) part[g] = fmaf(q[g][r], ck, fmaf(u[g][r], sg, part[g]));
+                for (int g = 0; g < G; ++g) part[g] = fmaf(q[g][r], ck, fmaf(u[g][r], sg, part[g]));
+            } else {
+#pragma unroll
+                for (int g = 0; g < G; ++g) part[g] = fmaf(q[g][r], ck, part[g]);
+            }
         }
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -307,19 +313,19 @@ cudaError_t launch_prologue_d(const void* q, tq_dtype dt, int64_t BHq, const flo
     return cudaErrorInvalidValue;
 }
 
-template <int D, int G>
+template <int D, int G, bool QJL>
 cudaError_t launch_simt(const DecArgs& a, cudaStream_t s) {
     dim3 grid(a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
-    return launch_pdl(tq_decode_simt_kernel<D, G>, grid, dim3(128), 0, s, a);
+    return launch_pdl(tq_decode_simt_kernel<D, G, QJL>, grid, dim3(128), 0, s, a);
 }
 
-template <int D>
+template <int D, bool QJL>
 cudaError_t launch_simt_g(int G, const DecArgs& a, cudaStream_t s) {
     switch (G) {
-        case 1: return launch_simt<D, 1>(a, s);
-        case 2: return launch_simt<D, 2>(a, s);
-        case 4: return launch_simt<D, 4>(a, s);
-        case 8: return launch_simt<D, 8>(a, s);
+        case 1: return launch_simt<D, 1, QJL>(a, s);
+        case 2: return launch_simt<D, 2, QJL>(a, s);
+        case 4: return launch_simt<D, 4, QJL>(a, s);
+        case 8: return launch_simt<D, 8, QJL>(a, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -333,10 +339,10 @@ cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, cons
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_decode_simt(int d, int G, const DecArgs& a, cudaStream_t s) {
+cudaError_t launch_decode_simt(int d, int G, bool qjl, const DecArgs& a, cudaStream_t s) {
     if (a.B * a.Hkv == 0) return cudaSuccess;
-    if (d == 128) return launch_simt_g<128>(G, a, s);
-    if (d == 256) return launch_simt_g<256>(G, a, s);
+    if (d == 128) return qjl ? launch_simt_g<128, true>(G, a, s) : launch_simt_g<128, false>(G, a, s);
+    if (d == 256) return qjl ? launch_simt_g<256, true>(G, a, s) : launch_simt_g<256, false>(G, a, s);
     return cudaErrorInvalidValue;
 }
 
@@ -354,8 +360,8 @@ cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml,
 
 namespace tqi {
 
-cudaError_t launch_decode_simt(int d, int G, const DecArgs& a, cudaStream_t s);
-cudaError_t launch_decode_mma(int d, int G, const DecArgs& a, cudaStream_t s);
+cudaError_t launch_decode_simt(int d, int G, bool qjl, const DecArgs& a, cudaStream_t s);
+cudaError_t launch_decode_mma(int d, int G, bool qjl, const DecArgs& a, cudaStream_t s);
 int decode_mma_chunk_tokens(int d);
 int decode_mma_warps(int G);
 
@@ -367,8 +373,8 @@ int decode_ctas_per_sm(bool use_mma) { return use_mma ? 1 : 4; }
 int decode_chunk_tokens(int d, bool use_mma) { return use_mma ? decode_mma_chunk_tokens(d) : kBlockT; }
 int decode_warps(bool use_mma, int G) { return use_mma ? decode_mma_warps(G) : 4; }
 
-cudaError_t launch_decode(int d, int G, bool use_mma, const DecArgs& a, cudaStream_t s) {
-    return use_mma ? launch_decode_mma(d, G, a, s) : launch_decode_simt(d, G, a, s);
+cudaError_t launch_decode(int d, int G, bool use_mma, bool qjl, const DecArgs& a, cudaStream_t s) {
+    return use_mma ? launch_decode_mma(d, G, qjl, a, s) : launch_decode_simt(d, G, qjl, a, s);
 }
 
 }  // namespace tqi

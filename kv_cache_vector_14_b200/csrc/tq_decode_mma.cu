@@ -48,20 +48,21 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kStages = 3;             // ring depth per warp
 constexpr int kWaitLimit = 1 << 20;
 
-// Per-head-dim shape of a ring stage (bytes).
-template <int D>
+// Per-head-dim shape of a ring stage (bytes).  QJL = false: the K cache is a
+// PolarQuant-only cache in the V layout (codes and norms, no signs, no gamma).
+template <int D, bool QJL = true>
 struct Cfg {
     static constexpr int kS = D / 128;                        // 128-coordinate slices
     static constexpr int kKC = D / 16;                        // coordinate chunks (mma k-steps)
     static constexpr int kCodeB = 3 * D / 8;                  // code bytes per token
-    static constexpr int kSignB = D / 8;                      // sign bytes per token
+    static constexpr int kSignB = D / 8;                      // sign bytes per token (QJL)
     static constexpr int kChunk = D == 128 ? 32 : 16;         // tokens per stage
     static constexpr int kTiles = kChunk / 16;
     static constexpr int kOffKc = 0;
     static constexpr int kOffKs = kOffKc + kChunk * kCodeB;
-    static constexpr int kOffKn = kOffKs + kChunk * kSignB;
+    static constexpr int kOffKn = kOffKs + (QJL ? kChunk * kSignB : 0);
     static constexpr int kOffKg = kOffKn + 2 * kChunk;
-    static constexpr int kOffVc = kOffKg + 2 * kChunk;
+    static constexpr int kOffVc = kOffKg + (QJL ? 2 * kChunk : 0);
     static constexpr int kOffVn = kOffVc + kChunk * kCodeB;
     static constexpr int kStageB = kOffVn + 2 * kChunk;
     static constexpr bool kBRegs = D == 128;                   // q'/u' fragments in registers
@@ -179,9 +180,9 @@ __device__ __forceinline__ uint32_t sel_for(const uint32_t (&sel)[4], const uint
 // Lane (g, t) = (lane / 4, lane % 4) dequantises tokens g and g + 8 of each
 // 16-token tile; its score columns are head t (hi, lo), so its softmax state
 // and output rows belong to head t (and head 4 + t when NT = 2).
-template <int D, int NT, int NW>
+template <int D, int NT, int NW, bool QJL>
 __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs a, int G) {
-    using C = Cfg<D>;
+    using C = Cfg<D, QJL>;
     constexpr int kKC = C::kKC;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)NW * kStages * C::kStageB);
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     const int nchunk = s1 > s0 ? (int)((s1 - s0 + C::kChunk - 1) / C::kChunk) : 0;
     const int nmine = nchunk > warp ? (nchunk - warp + NW - 1) / NW : 0;
     const int64_t seq = (int64_t)b * a.Hkv + hkv;
-    const int64_t kbb = block_bytes(D, true), vbb = block_bytes(D, false);
+    const int64_t kbb = block_bytes(D, QJL), vbb = block_bytes(D, false);
 
     if (lane == 0)
         for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&bars[warp * kStages + s]), 1);
@@ -217,9 +218,13 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         constexpr int cb = C::kCodeB, sb = C::kSignB, ch = C::kChunk;
         mbar_expect_tx(bar, C::kStageB);
         bulk_g2s(smem_u32(st + C::kOffKc), kb + sub * ch * cb, ch * cb, bar);
-        bulk_g2s(smem_u32(st + C::kOffKs), kb + 64 * cb + sub * ch * sb, ch * sb, bar);
-        bulk_g2s(smem_u32(st + C::kOffKn), kb + 64 * (cb + sb) + sub * 2 * ch, 2 * ch, bar);
-        bulk_g2s(smem_u32(st + C::kOffKg), kb + 64 * (cb + sb) + 128 + sub * 2 * ch, 2 * ch, bar);
+        if constexpr (QJL) {
+            bulk_g2s(smem_u32(st + C::kOffKs), kb + 64 * cb + sub * ch * sb, ch * sb, bar);
+            bulk_g2s(smem_u32(st + C::kOffKn), kb + 64 * (cb + sb) + sub * 2 * ch, 2 * ch, bar);
+            bulk_g2s(smem_u32(st + C::kOffKg), kb + 64 * (cb + sb) + 128 + sub * 2 * ch, 2 * ch, bar);
+        } else {
+            bulk_g2s(smem_u32(st + C::kOffKn), kb + 64 * cb + sub * 2 * ch, 2 * ch, bar);
+        }
         bulk_g2s(smem_u32(st + C::kOffVc), vb + sub * ch * cb, ch * cb, bar);
         bulk_g2s(smem_u32(st + C::kOffVn), vb + 64 * cb + sub * 2 * ch, 2 * ch, bar);
     };
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
 #pragma unroll
             for (int kc = 0; kc < kKC; ++kc) {
                 b_frag(a.qp, nt, kc, bq[nt][kc][0], bq[nt][kc][1]);
-                b_frag(a.up, nt, kc, bu[nt][kc][0], bu[nt][kc][1]);
+                if constexpr (QJL) b_frag(a.up, nt, kc, bu[nt][kc][0], bu[nt][kc][1]);
             }
     } else {
         for (int kc = warp; kc < kKC; kc += NW)
@@ -274,8 +279,10 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                 uint32_t r0, r1;
                 b_frag(a.qp, nt, kc, r0, r1);
                 sB[((0 * NT + nt) * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
-                b_frag(a.up, nt, kc, r0, r1);
-                sB[((1 * NT + nt) * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
+                if constexpr (QJL) {
+                    b_frag(a.up, nt, kc, r0, r1);
+                    sB[((1 * NT + nt) * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
+                }
             }
         __syncthreads();
     }
@@ -315,17 +322,24 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
             constexpr bool PARTIAL = decltype(partial_tag)::value;
             const int tA = kt * 16 + gr, tB = tA + 8;            // this lane's two tokens
             // ---------------- scores
-            uint32_t selA[C::kS][4], selB[C::kS][4], sgA[C::kS], sgB[C::kS];
+            uint32_t selA[C::kS][4], selB[C::kS][4];
+            [[maybe_unused]] uint32_t sgA[C::kS], sgB[C::kS];
 #pragma unroll
             for (int sl = 0; sl < C::kS; ++sl) {
                 code_selectors(st + C::kOffKc + tA * C::kCodeB + sl * 48 + tq4 * 12, pw, selA[sl]);
                 code_selectors(st + C::kOffKc + tB * C::kCodeB + sl * 48 + tq4 * 12, pw, selB[sl]);
-                sgA[sl] = *reinterpret_cast<const uint32_t*>(st + C::kOffKs + tA * C::kSignB + sl * 16 + tq4 * 4);
-                sgB[sl] = *reinterpret_cast<const uint32_t*>(st + C::kOffKs + tB * C::kSignB + sl * 16 + tq4 * 4);
+                if constexpr (QJL) {
+                    sgA[sl] = *reinterpret_cast<const uint32_t*>(st + C::kOffKs + tA * C::kSignB + sl * 16 + tq4 * 4);
+                    sgB[sl] = *reinterpret_cast<const uint32_t*>(st + C::kOffKs + tB * C::kSignB + sl * 16 + tq4 * 4);
+                }
             }
-            const uint32_t gA = *reinterpret_cast<const uint16_t*>(st + C::kOffKg + 2 * tA);
-            const uint32_t gB = *reinterpret_cast<const uint16_t*>(st + C::kOffKg + 2 * tB);
-            const uint32_t ggA = gA | (gA << 16), ggB = gB | (gB << 16);
+            [[maybe_unused]] uint32_t ggA = 0, ggB = 0;
+            if constexpr (QJL) {
+                const uint32_t gA = *reinterpret_cast<const uint16_t*>(st + C::kOffKg + 2 * tA);
+                const uint32_t gB = *reinterpret_cast<const uint16_t*>(st + C::kOffKg + 2 * tB);
+                ggA = gA | (gA << 16);
+                ggB = gB | (gB << 16);
+            }
             float acc[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
@@ -335,22 +349,26 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                 uint32_t ka[4];
                 dequant4(sel_for(selA[sl], pw, kk), lut, ka[0], ka[2]);
                 dequant4(sel_for(selB[sl], pw, kk), lut, ka[1], ka[3]);
-                uint32_t sa[4];
-                // sign bit 1 -> +gamma: the pair (2kk | 2kk+1) of a slot sits at bits (q, 16 + q)
-                sa[0] = ggA ^ (~shl_m(sgA[sl], pw, 15 - 2 * kk) & 0x80008000u);
-                sa[1] = ggB ^ (~shl_m(sgB[sl], pw, 15 - 2 * kk) & 0x80008000u);
-                sa[2] = ggA ^ (~shl_m(sgA[sl], pw, 14 - 2 * kk) & 0x80008000u);
-                sa[3] = ggB ^ (~shl_m(sgB[sl], pw, 14 - 2 * kk) & 0x80008000u);
+                [[maybe_unused]] uint32_t sa[4] = {0u, 0u, 0u, 0u};
+                if constexpr (QJL) {
+                    // sign bit 1 -> +gamma: the pair (2kk | 2kk+1) of a slot sits at bits (q, 16 + q)
+                    sa[0] = ggA ^ (~shl_m(sgA[sl], pw, 15 - 2 * kk) & 0x80008000u);
+                    sa[1] = ggB ^ (~shl_m(sgB[sl], pw, 15 - 2 * kk) & 0x80008000u);
+                    sa[2] = ggA ^ (~shl_m(sgA[sl], pw, 14 - 2 * kk) & 0x80008000u);
+                    sa[3] = ggB ^ (~shl_m(sgB[sl], pw, 14 - 2 * kk) & 0x80008000u);
+                }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     if constexpr (C::kBRegs) {
                         mma16816(acc[nt], ka, bq[nt][kc][0], bq[nt][kc][1]);
-                        mma16816(acc[nt], sa, bu[nt][kc][0], bu[nt][kc][1]);
+                        if constexpr (QJL) mma16816(acc[nt], sa, bu[nt][kc][0], bu[nt][kc][1]);
                     } else {
                         const uint2 fq = sB[((0 * NT + nt) * kKC + kc) * 32 + lane];
-                        const uint2 fu = sB[((1 * NT + nt) * kKC + kc) * 32 + lane];
                         mma16816(acc[nt], ka, fq.x, fq.y);
-                        mma16816(acc[nt], sa, fu.x, fu.y);
+                        if constexpr (QJL) {
+                            const uint2 fu = sB[((1 * NT + nt) * kKC + kc) * 32 + lane];
+                            mma16816(acc[nt], sa, fu.x, fu.y);
+                        }
                     }
                 }
             }
@@ -488,23 +506,29 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
 constexpr int kNW1 = 16;   // warps per CTA, up to 4 heads per kv head (one n-tile)
 constexpr int kNW2 = 8;    // warps per CTA, 8 heads per kv head (two n-tiles, more registers)
 
-template <int D, int NT, int NW>
+template <int D, int NT, int NW, bool QJL>
 cudaError_t launch_mma_t(const DecArgs& a, int G, cudaStream_t s) {
-    using C = Cfg<D>;
+    using C = Cfg<D, QJL>;
     const size_t smem = (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
                         (C::kBRegs ? 0 : (size_t)2 * NT * C::kKC * 32 * sizeof(uint2));
-    auto kern = tq_decode_mma_kernel<D, NT, NW>;
-    cudaError_t e = set_smem_once<tq_decode_mma_kernel<D, NT, NW>>((int)smem);
+    auto kern = tq_decode_mma_kernel<D, NT, NW, QJL>;
+    cudaError_t e = set_smem_once<tq_decode_mma_kernel<D, NT, NW, QJL>>((int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
     return launch_pdl(kern, grid, dim3(NW * 32), smem, s, a, G);
 }
 
-cudaError_t launch_decode_mma(int d, int G, const DecArgs& a, cudaStream_t s) {
+template <bool QJL>
+cudaError_t launch_mma_q(int d, int G, const DecArgs& a, cudaStream_t s) {
+    if (d == 128)
+        return G <= 4 ? launch_mma_t<128, 1, kNW1, QJL>(a, G, s) : launch_mma_t<128, 2, kNW2, QJL>(a, G, s);
+    return G <= 4 ? launch_mma_t<256, 1, kNW1, QJL>(a, G, s) : launch_mma_t<256, 2, kNW2, QJL>(a, G, s);
+}
+
+cudaError_t launch_decode_mma(int d, int G, bool qjl, const DecArgs& a, cudaStream_t s) {
     if ((d != 128 && d != 256) || G < 1 || G > 8) return cudaErrorInvalidValue;
     if (a.B * a.Hkv == 0) return cudaSuccess;
-    if (d == 128) return G <= 4 ? launch_mma_t<128, 1, kNW1>(a, G, s) : launch_mma_t<128, 2, kNW2>(a, G, s);
-    return G <= 4 ? launch_mma_t<256, 1, kNW1>(a, G, s) : launch_mma_t<256, 2, kNW2>(a, G, s);
+    return qjl ? launch_mma_q<true>(d, G, a, s) : launch_mma_q<false>(d, G, a, s);
 }
 
 int decode_mma_chunk_tokens(int d) { return d == 128 ? Cfg<128>::kChunk : Cfg<256>::kChunk; }

@@ -164,7 +164,8 @@ cudaError_t launch_encode128(bool is_k, tq_dtype dt, const EncArgs& a, int num_s
 // append-and-attend step); the kernels then complete only after it.
 cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, const float* dsign,
                             const float* st, float* qp, float* up, bool pdl, cudaStream_t s);
-cudaError_t launch_decode(int d, int G, bool use_mma, const DecArgs& a, cudaStream_t s);
+// qjl = false: PolarQuant-only K cache (V layout), scores without the QJL term.
+cudaError_t launch_decode(int d, int G, bool use_mma, bool qjl, const DecArgs& a, cudaStream_t s);
 cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml,
                            const float* part_acc, const float* dsign, float* out, cudaStream_t s);
 bool mma_supported(int d, int G);

@@ -22,7 +22,7 @@ TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 
 EXPORTED = ("tq_params_host", "tq_init", "tq_destroy", "tq_get_params", "tq_head_dim", "tq_block_bytes",
             "tq_cache_bytes", "tq_encode_k", "tq_encode_v", "tq_attend_workspace_bytes", "tq_attend_decode",
-            "tq_append_attend",
+            "tq_append_attend", "tq_attend_decode_polar",
             "tq_attend_decode_static", "tq_device_status", "tq_set_decode_events", "tq_set_decode_path", "tq_attend_path", "tq_status_string")
 
 
@@ -75,6 +75,8 @@ def lib() -> C.CDLL:
             L.tq_attend_decode_static.argtypes = [P, P, i32, i64, i64, C.POINTER(tq_cache), C.POINTER(tq_cache), P,
                                                   i64, C.c_float, P, P]
             L.tq_attend_decode_static.restype = st
+            L.tq_attend_decode_polar.argtypes = L.tq_attend_decode.argtypes
+            L.tq_attend_decode_polar.restype = st
             L.tq_append_attend.argtypes = [P, P, P, i32, i64, i64, i64, i64, C.POINTER(tq_cache),
                                            C.POINTER(tq_cache), i64, P, i32, i64, C.c_float, P, P, C.c_size_t, P]
             L.tq_append_attend.restype = st
@@ -217,6 +219,22 @@ def tq_attend_decode(h, q, kc: Cache, vc: Cache, out, ws, T: int = 0, seq_lens=N
                                   C.byref(vc.struct), sl, T, float(scale), C.c_void_p(out.data_ptr()),
                                   C.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(), _stream(stream)),
            "tq_attend_decode")
+
+
+def tq_attend_decode_polar(h, q, kc: Cache, vc: Cache, out, ws, T: int = 0, seq_lens=None, scale: float = 1.0,
+                           stream=None) -> None:
+    """Attention with a PolarQuant-only K cache (a V-layout cache written by
+    tq_encode_v): scores without the QJL term."""
+    if q.dim() != 3 or not q.is_contiguous():
+        raise ValueError("tq_attend_decode_polar: q must be contiguous [B, Hq, d]")
+    if kc.is_k:
+        raise ValueError("tq_attend_decode_polar: kc must be a V-layout cache (encoded with tq_encode_v)")
+    B, Hq, _ = q.shape
+    sl = C.c_void_p(seq_lens.data_ptr()) if seq_lens is not None else None
+    _check(lib().tq_attend_decode_polar(h, C.c_void_p(q.data_ptr()), _dtype_code(q), B, Hq, C.byref(kc.struct),
+                                        C.byref(vc.struct), sl, T, float(scale), C.c_void_p(out.data_ptr()),
+                                        C.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(),
+                                        _stream(stream)), "tq_attend_decode_polar")
 
 
 def tq_append_attend(h, k_new, v_new, kc: Cache, vc: Cache, t0: int, q, out, ws, scale: float = 1.0,

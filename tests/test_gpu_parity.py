@@ -319,6 +319,36 @@ def test_attend_group_sizes_and_ragged_lengths(decode_path, handles, prms, d, G)
     assert err.max() <= ATT_TOL
 
 
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_attend_polar_only_k(decode_path, handles, prms, d, G):
+    """PolarQuant-only K (a V-layout K cache from tq_encode_v): the kernels'
+    attention equals the oracle's with gamma = 0 (no QJL term), ragged lengths."""
+    Hkv, B, Tcap = 2, 3, 320
+    Hq = Hkv * G
+    h = handles[d]
+    xk = torch_input(synthetic.gaussian((B, Hkv, Tcap, d), seed=31 + G), "f32")
+    xv = torch_input(synthetic.gaussian((B, Hkv, Tcap, d), seed=41 + G), "f32")
+    kc, vc = tq.Cache(d, False, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
+    tq.tq_encode_v(h, xk, kc, 0)
+    tq.tq_encode_v(h, xv, vc, 0)
+    q = synthetic.gaussian((B, Hq, d), seed=51)
+    lens = [0, 129, 301]
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    ws = torch.empty(tq.tq_attend_workspace_bytes(h, B, Hq, Hkv, Tcap), dtype=torch.uint8, device="cuda")
+    out = torch.full((B, Hq, d), float("nan"), dtype=torch.float32, device="cuda")
+    scale = 1.0 / np.sqrt(d)
+    tq.tq_attend_decode_polar(h, torch_input(q, "f32"), kc, vc, out, ws, seq_lens=sl, scale=scale)
+    ku, vu = unpack_cache(kc, 0, Tcap), unpack_cache(vc, 0, Tcap)
+    ku = {"idx": ku["idx"], "nh": ku["nh"], "sig": np.ones(ku["idx"].shape, np.uint8),
+          "gh": np.zeros_like(ku["nh"])}
+    ref = oracle_attend(prms[d], q.astype(np.float64), ku, vu, Hkv, lens, scale)
+    err = rel_err_rows(out.cpu().numpy(), ref)
+    print("polar-only K max rel err", err.max())
+    assert err.max() <= ATT_TOL
+    assert tq.tq_device_status(h) == tq.TQ_OK
+
+
 @pytest.mark.parametrize("qdt", ["f32", "bf16", "f16"])
 def test_attend_query_dtypes(decode_path, handles, prms, qdt):
     w = synthetic.Workload("t", "qdt", B=1, Hq=8, Hkv=2, d=128, T=500, kv_dtype="bf16", q_dtype=qdt,

@@ -205,6 +205,36 @@ def test_qjl_estimator_unbiased():
     assert np.mean(trues) > 20 * tol      # the test has power against a wrong constant or sign
 
 
+def test_polar_only_scores_shrink_qjl_scores_unbiased():
+    """PolarQuant-only versus QJL-corrected K scores (the page's two K flows).
+    Over random sign diagonals and JL matrices (parameter seeds), the score
+    without the QJL term, n <q', c[idx]>, regresses on the exact <q, x> with
+    slope E<y_hat, y> = 1 - D_mse: the centroid condition makes the residual
+    r = y - y_hat average to zero in each cell, so E<y_hat, r> = 0 and
+    E<y_hat, y> = E||y_hat||^2 = 1 - E||r||^2.  Adding the QJL term (an
+    unbiased estimate of <q', r>) restores slope 1.  D_mse = 0.03454 is the
+    8-level Gaussian quantiser's MSE (pinned above); the tolerance 0.01 is
+    about five standard errors for 12800 samples."""
+    d, nseeds, T = 128, 200, 64
+    x = synthetic.gaussian((T, d), seed=21).astype(np.float64)
+    q = synthetic.gaussian((d,), seed=22).astype(np.float64)
+    exact = x @ q
+    sp, sq = [], []
+    for s in range(nseeds):
+        p = O.params(d, 5000 + s)
+        e = O.encode(x, p, with_qjl=True)
+        kc = {"idx": e["idx"], "sig": e["sig"], "nh": e["nh"], "gh": e["gh"]}
+        sq.append(O.scores(p, q, kc, 1.0))
+        sp.append(O.scores(p, q, dict(kc, gh=np.zeros_like(e["gh"])), 1.0))
+    sp, sq = np.concatenate(sp), np.concatenate(sq)
+    ex = np.tile(exact, nseeds)
+    slope_polar = (sp @ ex) / (ex @ ex)
+    slope_qjl = (sq @ ex) / (ex @ ex)
+    assert abs(slope_qjl - 1.0) < 0.01
+    assert abs(slope_polar - (1.0 - 0.03454)) < 0.01
+    assert slope_qjl - slope_polar > 0.02          # the two estimators are told apart
+
+
 # ---------------------------------------------------------------- layout
 
 @pytest.mark.parametrize("d", [128, 256])
