@@ -44,24 +44,25 @@ __device__ void smem_fwht(float* v) {
 }
 
 // ---------------------------------------------------------------- prologue
-// q' = H D q / sqrt(d) and up = sqrt(pi/2)/m * S q'.  A CTA takes kPQH(D) =
-// D / kRC query heads and one chunk of kRC rows of S: it transforms its heads
-// in shared memory, stages the kRC columns of S^T it needs (one L2 read of S
-// per head group, not per head), and thread t computes row t % kRC of head
-// t / kRC.  The CTAs of row chunk 0 also store q'.
+// q' = H D q / sqrt(d) and up = sqrt(pi/2)/m * S q'.  A CTA takes QH = D / kRC
+// query heads and one chunk of kRC rows of S: it transforms its heads in
+// shared memory and stages the kRC columns of S^T it needs (one L2 read of S
+// per head group).  Warp w then sums coordinates [32 w, 32 w + 32) for row
+// `lane` of the chunk and all QH heads at once (each staged S value is read
+// once per CTA), and the QH partial sums of every output are added in warp
+// order.  The CTAs of row chunk 0 also store q'.
 constexpr int kRC = 32;
 
 template <int D, int DT>
 __global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t BHq, const float* dsign,
                                                         const float* ST, float* qp, float* up) {
-    constexpr int QH = D / kRC;
-    __shared__ float v[QH * D];
-    __shared__ __align__(16) float sst[D * kRC];           // sst[j][i] = S[rc*kRC + i][j]
+    constexpr int QH = D / kRC;                           // heads per CTA = warps per CTA
+    __shared__ __align__(16) float v[QH * D];
+    __shared__ __align__(16) float sst[D * kRC];          // sst[j][i] = S[rc*kRC + i][j]; then partial sums
     pdl_trigger();                                        // the split-K kernel may start its prefetch
-    const int t = threadIdx.x;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int64_t h0 = (int64_t)blockIdx.x * QH;
     const int rc = blockIdx.y;
-    // S^T columns of this row chunk: D rows of kRC floats
     for (int i = t; i < D * kRC / 4; i += D) {
         const int jr = i / (kRC / 4), c4 = i % (kRC / 4);
         reinterpret_cast<float4*>(sst)[i] = __ldg(reinterpret_cast<const float4*>(ST + (size_t)jr * D + rc * kRC) + c4);
@@ -78,16 +79,30 @@ __global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t B
 #pragma unroll
     for (int k = 0; k < QH; ++k) v[k * D + t] *= inv;
     __syncthreads();
-    const int i = t % kRC, k = t / kRC;
-    float u0 = 0.f, u1 = 0.f;
-#pragma unroll 8
-    for (int jj = 0; jj < D; jj += 2) {
-        u0 = fmaf(sst[jj * kRC + i], v[k * D + jj], u0);
-        u1 = fmaf(sst[(jj + 1) * kRC + i], v[k * D + jj + 1], u1);
+    float acc[QH];
+#pragma unroll
+    for (int k = 0; k < QH; ++k) acc[k] = 0.f;
+#pragma unroll 2
+    for (int jj = 32 * warp; jj < 32 * warp + 32; jj += 4) {
+        const float s0 = sst[jj * kRC + lane], s1 = sst[(jj + 1) * kRC + lane];
+        const float s2 = sst[(jj + 2) * kRC + lane], s3 = sst[(jj + 3) * kRC + lane];
+#pragma unroll
+        for (int k = 0; k < QH; ++k) {
+            const float4 vv = *reinterpret_cast<const float4*>(&v[k * D + jj]);
+            acc[k] = fmaf(s3, vv.w, fmaf(s2, vv.z, fmaf(s1, vv.y, fmaf(s0, vv.x, acc[k]))));
+        }
     }
+    __syncthreads();                                      // sst is reused for the partial sums
+#pragma unroll
+    for (int k = 0; k < QH; ++k) sst[(warp * QH + k) * 32 + lane] = acc[k];
+    __syncthreads();
+    const int i = t % kRC, k = t / kRC;
+    float u = 0.f;
+#pragma unroll
+    for (int w = 0; w < QH; ++w) u += sst[(w * QH + k) * 32 + i];
     const float cq = 1.2533141373155003f / (float)D;       // sqrt(pi/2) / m
     const int64_t h = h0 + k;
-    if (h < BHq) up[h * D + rc * kRC + i] = cq * (u0 + u1);
+    if (h < BHq) up[h * D + rc * kRC + i] = cq * u;
     if (rc == 0) {
 #pragma unroll
         for (int kk = 0; kk < QH; ++kk)

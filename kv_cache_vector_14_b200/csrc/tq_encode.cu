@@ -260,27 +260,39 @@ __global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
 
 // ---------------------------------------------------------------- small batches (K)
 // Appends of a few vectors per head: one warp per vector and four warps per
-// CTA, so a 32-vector append runs on 8 SMs at once instead of one.  S is
-// staged through shared memory (all of it at d = 128, 64-column chunks at
-// d = 256) and the projection accumulates over columns in the same order as
-// the tiled kernel, so both give bit-identical sign words.
+// CTA, so a 32-vector append runs on 8 SMs at once instead of one.  The JL
+// rows are split over gridDim.y CTAs (kSmallRowGroups groups of 32 rows each),
+// each staging only its rows of S (64 KB at d = 256) and writing only their
+// sign words; every CTA repeats steps 1-4 for its vectors and the row-chunk-0
+// CTA stores the codes and norms.  Each z_i accumulates over the columns in
+// the same order as the tiled kernel, so both give bit-identical sign words.
 constexpr int kSmallWarps = 4;
+constexpr int kSmallRowGroups = 2;
 
 template <int D, int DT>
 __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(const EncArgs a) {
     constexpr int R = D / 32;
-    constexpr int JC = (D == 128) ? 128 : 64;      // columns of S resident at once
-    extern __shared__ __align__(16) float sS[];     // [JC][R][32]
+    constexpr int RG = kSmallRowGroups;             // row groups of 32 JL rows per CTA
+    extern __shared__ __align__(16) float sS[];     // [D][RG][32]
     __shared__ __align__(16) float sr[kSmallWarps][D];
     __shared__ __align__(16) uint8_t scode[kSmallWarps][D];
     __shared__ float sC[8];
     pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rg0 = blockIdx.y * RG;                // first row group of this CTA
     if (threadIdx.x < 8) sC[threadIdx.x] = a.cb.c[threadIdx.x];
+    {
+        // this CTA's rows of the lane-ordered JL matrix: RG*32 floats per column
+        const float4* src = reinterpret_cast<const float4*>(a.sthr);
+        for (int i = threadIdx.x; i < D * RG * 8; i += kSmallWarps * 32) {
+            const int j = i / (RG * 8), c = i % (RG * 8);
+            reinterpret_cast<float4*>(sS)[i] = __ldg(src + ((size_t)j * R + rg0) * 8 + c);
+        }
+    }
     __syncthreads();
     const int64_t N = a.B * a.Hkv * a.Tnew;
     const int64_t gv0 = (int64_t)blockIdx.x * kSmallWarps + warp;
-    const bool valid = gv0 < N;                     // idle warps still take part in the staging
+    const bool valid = gv0 < N;
     const int64_t gv = valid ? gv0 : N - 1;
     const int64_t tt = gv % a.Tnew, bh = gv / a.Tnew;
     const int64_t t = a.t0 + tt;
@@ -328,26 +340,21 @@ __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(con
         scode[warp][(j >> 7) * 128 + slot_of(j) * 32 + slot_pos(j)] = (uint8_t)code;
     }
     g2 = warp_sum(g2);
-    if (valid && lane == 0) {
+    const bool writer = valid && blockIdx.y == 0;
+    if (writer && lane == 0) {
         const int64_t norm_off = kBlockT * code_bytes(D) + kBlockT * sign_bytes(D);
         reinterpret_cast<__half*>(blk + norm_off)[t & 63] = __float2half_rn(n);
         reinterpret_cast<__half*>(blk + norm_off + 2 * kBlockT)[t & 63] = __float2half_rn(sqrtf(g2));
     }
-    float z[R];
+    __syncwarp();
+    float z[RG];
 #pragma unroll
-    for (int r = 0; r < R; ++r) z[r] = 0.f;
-    for (int j0 = 0; j0 < D; j0 += JC) {
-        __syncthreads();
-        const float4* src = reinterpret_cast<const float4*>(a.sthr + (size_t)j0 * D);
-#pragma unroll 8
-        for (int i = threadIdx.x; i < JC * D / 4; i += kSmallWarps * 32) reinterpret_cast<float4*>(sS)[i] = __ldg(src + i);
-        __syncthreads();
+    for (int k = 0; k < RG; ++k) z[k] = 0.f;
 #pragma unroll 4
-        for (int jj = 0; jj < JC; ++jj) {
-            const float rj = sr[warp][j0 + jj];
+    for (int j = 0; j < D; ++j) {
+        const float rj = sr[warp][j];
 #pragma unroll
-            for (int r = 0; r < R; ++r) z[r] = fmaf(rj, sS[(jj * R + r) * 32 + lane], z[r]);
-        }
+        for (int k = 0; k < RG; ++k) z[k] = fmaf(rj, sS[(j * RG + k) * 32 + lane], z[k]);
     }
     if (!valid) {
         pdl_wait();
@@ -355,13 +362,14 @@ __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(con
     }
     uint32_t mine = 0;
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-        const uint32_t word = __ballot_sync(kFull, z[r] >= 0.f);
-        if (lane == r) mine = word;
+    for (int k = 0; k < RG; ++k) {
+        const uint32_t word = __ballot_sync(kFull, z[k] >= 0.f);
+        if (lane == k) mine = word;
     }
-    if (lane < R) reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(D) + (t & 63) * sign_bytes(D))[lane] = mine;
+    if (lane < RG)
+        reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(D) + (t & 63) * sign_bytes(D))[rg0 + lane] = mine;
     constexpr int W = 3 * D / 32;
-    if (lane < W) {
+    if (blockIdx.y == 0 && lane < W) {
         const int sl = lane / 12, st = (lane % 12) / 3, g = lane % 3;
         const uint32_t* sw = reinterpret_cast<const uint32_t*>(&scode[warp][sl * 128 + st * 32]);
         const uint32_t main = nibbles8(sw[2 * g], sw[2 * g + 1]);
@@ -394,12 +402,12 @@ cudaError_t launch_enc_t(const EncArgs& a, int num_sms, bool pdl, cudaStream_t s
     const int64_t N = a.B * a.Hkv * a.Tnew;
     if constexpr (IS_K) {
         if (N <= (int64_t)4 * num_sms) {        // appends: one warp per vector
-            const unsigned grid = (unsigned)((N + kSmallWarps - 1) / kSmallWarps);
-            const size_t smem = (size_t)((D == 128) ? 128 : 64) * D * sizeof(float);
+            const dim3 grid((unsigned)((N + kSmallWarps - 1) / kSmallWarps), D / 32 / kSmallRowGroups);
+            const size_t smem = (size_t)D * kSmallRowGroups * 32 * sizeof(float);
             auto kern = tq_encode_k_small_kernel<D, DT>;
             cudaError_t e = set_smem_once<tq_encode_k_small_kernel<D, DT>>((int)smem);
             if (e != cudaSuccess) return e;
-            if (pdl) return launch_pdl(kern, dim3(grid), dim3(kSmallWarps * 32), smem, s, a);
+            if (pdl) return launch_pdl(kern, grid, dim3(kSmallWarps * 32), smem, s, a);
             kern<<<grid, kSmallWarps * 32, smem, s>>>(a);
             return cudaGetLastError();
         }
