@@ -42,9 +42,9 @@ ENCODE_BYTES_PER_VECTOR = {("k", 128): 68, ("v", 128): 50}
 
 # DRAM traffic of the split-K kernel from one ncu capture, valid only while the
 # kernel source is unchanged (sha256 of csrc/tq_decode_mma.cu at capture time).
-NCU_TRAFFIC = {"source_sha256": "376492f8052cd60f6a3cdf698519890fad13557c45bc940f971ee97d98da8081",
-               "bytes_per_launch": 390568192,
-               "capture": "profiles/tq_decode_mma128_long_context_b4_hq16_hkv8_t102400.md"}
+NCU_TRAFFIC = {"source_sha256": "1b9a3e166a557864f97fc4810d90c4a6fb92c0057c1f94fa6335c3b8b027aede",
+               "bytes_per_launch": 391289088,
+               "capture": "profiles/tq_decode_mma_d128_long_context_b4_hq16_hkv8_t102400.md"}
 
 
 def peaks():
