@@ -42,8 +42,8 @@ ENCODE_BYTES_PER_VECTOR = {("k", 128): 68, ("v", 128): 50}
 
 # DRAM traffic of the split-K kernel from one ncu capture, valid only while the
 # kernel source is unchanged (sha256 of csrc/tq_decode_mma.cu at capture time).
-NCU_TRAFFIC = {"source_sha256": "1b9a3e166a557864f97fc4810d90c4a6fb92c0057c1f94fa6335c3b8b027aede",
-               "bytes_per_launch": 391289088,
+NCU_TRAFFIC = {"source_sha256": "31c9db5f08a8daeafe93be7d0032b7e17a1b65bf2304b55d178f7ca209d8b8a3",
+               "bytes_per_launch": 390108160,
                "capture": "profiles/tq_decode_mma_d128_long_context_b4_hq16_hkv8_t102400.md"}
 
 
@@ -418,6 +418,48 @@ def measure_polar(h, dev, w, vc, q, out_qjl, ws, n_calls: int) -> dict:
                 "polar_k": rel(out[0, :G].cpu().numpy().astype(np.float64))}}
 
 
+def measure_paged(h, dev, w, kc, vc, q, out_ref, ws, n_calls: int) -> dict:
+    """Paged caches on the long-context workload: the same K and V blocks
+    scattered over two pools by a random permutation (block tables
+    [B*Hkv][T/64]), attention timed on its own (split-K kernel by events)
+    and its output compared with the contiguous caches' bit for bit."""
+    import torch
+    from kv_cache_vector_14_b200 import tq
+    d, B, Hq, Hkv, T = w.d, w.B, w.Hq, w.Hkv, w.T
+    nblk = B * Hkv * (T // 64)
+    gen = torch.Generator().manual_seed(1234)
+    caches = []
+    for src, is_k in ((kc, True), (vc, False)):
+        perm = torch.randperm(nblk, generator=gen).to(torch.int32)
+        table = perm.view(B * Hkv, T // 64).to(dev)
+        pc = tq.Cache(d, is_k, B, Hkv, T, block_table=table, pool_blocks=nblk)
+        bb = tq.tq_block_bytes(d, is_k)
+        pc.buf[:nblk * bb].view(nblk, bb).index_copy_(0, perm.to(dev).long(), src.buf[:nblk * bb].view(nblk, bb))
+        caches.append(pc)
+    kp, vp = caches
+    out = torch.empty_like(out_ref)
+    for _ in range(5):
+        tq.tq_attend_decode(h, q, kp, vp, out, ws, T=T, scale=w.scale)
+    torch.cuda.synchronize()
+    same = bool(torch.equal(out, out_ref))
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_calls)]
+    for a_, b_ in kev:
+        a_.record()
+        b_.record()
+    torch.cuda.synchronize()
+    for i in range(n_calls):
+        tq.tq_set_decode_events(h, kev[i][0], kev[i][1])
+        tq.tq_attend_decode(h, q, kp, vp, out, ws, T=T, scale=w.scale)
+    torch.cuda.synchronize()
+    tq.tq_set_decode_events(h, None, None)
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    del kp, vp, caches
+    nbytes = B * Hkv * T * BYTES_PER_TOKEN_HEAD[d]
+    return {"workload": w.title + ", K and V blocks scattered over pools by random block tables",
+            "kernel_ms": kern_ms, "achieved_gbs": nbytes / (kern_ms * 1e-3) / 1e9,
+            "output_equals_contiguous": same}
+
+
 def run_ours(args, rank: int, world: int, dist):
     import torch
     from kv_cache_vector_14_b200 import build, tq
@@ -555,6 +597,7 @@ def run_ours(args, rank: int, world: int, dist):
     tq.tq_attend_decode(h, q, kc, vc, out, ws, T=T, scale=w.scale)     # QJL output for the quality check
     torch.cuda.synchronize()
     polar = measure_polar(h, dev, w, vc, q, out.clone(), ws, n_kern)
+    paged = measure_paged(h, dev, w, kc, vc, q, out.clone(), ws, n_kern)
     enc = measure_encode(h, dev, world, dist)
     loop = measure_loop(dev, world, dist)
 
@@ -598,6 +641,7 @@ def run_ours(args, rank: int, world: int, dist):
         "encode": {**enc, "frac": enc["achieved_gbs"] / peak, "cpu_baseline": enc_cpu},
         "loop": {**loop, "frac": loop["achieved_gbs"] / peak},
         "polar_k": {**polar, "frac": polar["achieved_gbs"] / peak},
+        "paged": {**paged, "frac": paged["achieved_gbs"] / peak},
         "device_status": tq.tq_status_string(status),
     }
     print(json.dumps(line), flush=True)

@@ -62,6 +62,15 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
 
 /* A compressed cache: caller-owned device buffer of tq_cache_bytes() bytes,
  * 16-byte aligned, laid out as [B][Hkv][Tcap/64] blocks (Tcap a multiple of 64).
+ * Paged form (block_table != NULL): base is a pool of pool_blocks blocks of
+ * tq_block_bytes(d, is_k) bytes, and block_table (device int32
+ * [B*Hkv][Tcap/64], row b*Hkv + h) gives the pool block that holds tokens
+ * [64 lb, 64 lb + 64) of (batch b, kv head h).  Blocks of different sequences
+ * may be anywhere in the pool; a block must not be shared by two live
+ * (sequence, logical block) pairs that are written.  A table entry outside
+ * [0, pool_blocks) is a device-side check failure (reported by
+ * tq_device_status): nothing is written through it and reads go to block 0.
+ * With block_table == NULL pool_blocks is ignored.
  * K block (64 tokens): codes 64 x 3d/8 B | signs 64 x d/8 B | ||k|| fp16 x 64 |
  *                      gamma = ||residual|| fp16 x 64
  * V block (64 tokens): codes 64 x 3d/8 B | ||v|| fp16 x 64
@@ -81,6 +90,8 @@ typedef struct {
     int64_t B;
     int64_t Hkv;
     int64_t Tcap;
+    const int32_t* block_table;   /* NULL: contiguous cache */
+    int64_t pool_blocks;
 } tq_cache;
 
 /* ---- constants -------------------------------------------------------- */

@@ -84,7 +84,8 @@ tq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_
 
 bool cache_ok(const tq_handle* h, const tq_cache* c) {
     return c && c->base && aligned(c->base, 16) && c->B >= 0 && c->Hkv > 0 && c->Tcap > 0 &&
-           c->Tcap % kBlockT == 0 && h;
+           c->Tcap % kBlockT == 0 && h &&
+           (!c->block_table || (aligned(c->block_table, 4) && c->pool_blocks > 0 && c->pool_blocks < (1LL << 31)));
 }
 
 tq_status prepare_encode(const tq_handle* h, const void* x, tq_dtype dt, int64_t B, int64_t Hkv, int64_t Tnew,
@@ -107,6 +108,8 @@ tq_status prepare_encode(const tq_handle* h, const void* x, tq_dtype dt, int64_t
     a->B = B; a->Hkv = Hkv; a->Tnew = Tnew; a->t0 = t0;
     a->NB = c->Tcap / kBlockT;
     a->cache = static_cast<uint8_t*>(c->base);
+    a->table = c->block_table;
+    a->pool = c->pool_blocks;
     a->dsign = h->dsign; a->sthr = h->dSThr; a->bimg = h->dSB; a->err = h->derr; a->cb = h->cb;
     const int64_t es = (int64_t)dtype_size(dt);
     a->vec16 = (aligned(x, 16) && (sb * es) % 16 == 0 && (sh * es) % 16 == 0 && (st * es) % 16 == 0) ? 1 : 0;
@@ -152,6 +155,10 @@ tq_status prepare_attend(const tq_handle* h, const void* q, tq_dtype qdt, int64_
     a->up = reinterpret_cast<float*>(w + p->off_up);
     a->kc = static_cast<const uint8_t*>(kc->base);
     a->vc = static_cast<const uint8_t*>(vc->base);
+    a->ktable = kc->block_table;
+    a->vtable = vc->block_table;
+    a->kpool = kc->pool_blocks;
+    a->vpool = vc->pool_blocks;
     a->NB = kc->Tcap / kBlockT;
     a->seq_lens = seq_lens;
     a->T = T;

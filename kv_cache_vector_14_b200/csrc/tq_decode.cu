@@ -170,8 +170,10 @@ __global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
     __syncthreads();
 
     for (int64_t t = w0; t < w1; ++t) {
-        const uint8_t* kb = a.kc + (seq * a.NB + (t >> 6)) * kbb;
-        const uint8_t* vb = a.vc + (seq * a.NB + (t >> 6)) * vbb;
+        const int64_t kblk = cache_block(a.ktable, a.kpool, a.NB, seq, t >> 6, a.err);
+        const int64_t vblk = cache_block(a.vtable, a.vpool, a.NB, seq, t >> 6, a.err);
+        const uint8_t* kb = a.kc + (kblk >= 0 ? kblk : 0) * kbb;    // a bad table entry reads block 0
+        const uint8_t* vb = a.vc + (vblk >= 0 ? vblk : 0) * vbb;
         const int tau = (int)(t & 63);
         const uint32_t* kw = reinterpret_cast<const uint32_t*>(kb + tau * code_bytes(D));
         const uint32_t* sw = reinterpret_cast<const uint32_t*>(kb + kBlockT * code_bytes(D) + tau * sign_bytes(D));

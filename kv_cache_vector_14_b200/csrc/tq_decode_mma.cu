@@ -209,10 +209,11 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
 
     auto issue = [&](int i) {
         const int64_t t0 = s0 + (int64_t)(warp + i * NW) * C::kChunk;     // multiple of the chunk
-        const int64_t blk = seq * a.NB + (t0 >> 6);
+        const int64_t kblk = cache_block(a.ktable, a.kpool, a.NB, seq, t0 >> 6, a.err);
+        const int64_t vblk = cache_block(a.vtable, a.vpool, a.NB, seq, t0 >> 6, a.err);
         const int sub = (int)((t0 & 63) / C::kChunk);
-        const uint8_t* kb = a.kc + blk * kbb;
-        const uint8_t* vb = a.vc + blk * vbb;
+        const uint8_t* kb = a.kc + (kblk >= 0 ? kblk : 0) * kbb;    // a bad table entry reads block 0
+        const uint8_t* vb = a.vc + (vblk >= 0 ? vblk : 0) * vbb;
         uint8_t* st = ring + (i % kStages) * C::kStageB;
         const uint32_t bar = smem_u32(&bars[warp * kStages + (i % kStages)]);
         constexpr int cb = C::kCodeB, sb = C::kSignB, ch = C::kChunk;

@@ -171,12 +171,15 @@ __global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
         for (int vv = 0; vv < kVecPerWarp; ++vv) {
             if (valid[vv] && lane == 0) {
                 const int64_t t = a.t0 + tt[vv];
-                uint8_t* blk = a.cache + (bh[vv] * a.NB + (t >> 6)) * bb;
+                const int64_t pb = cache_block(a.table, a.pool, a.NB, bh[vv], t >> 6, a.err);
+                uint8_t* blk = a.cache + pb * bb;
                 const int tau = (int)(t & 63);
                 const int64_t norm_off = kBlockT * code_bytes(D) + (IS_K ? kBlockT * sign_bytes(D) : 0);
-                reinterpret_cast<__half*>(blk + norm_off)[tau] = __float2half_rn(sqrtf(ss[vv]));
-                if constexpr (IS_K)
-                    reinterpret_cast<__half*>(blk + norm_off + 2 * kBlockT)[tau] = __float2half_rn(sqrtf(g2[vv]));
+                if (pb >= 0) {
+                    reinterpret_cast<__half*>(blk + norm_off)[tau] = __float2half_rn(sqrtf(ss[vv]));
+                    if constexpr (IS_K)
+                        reinterpret_cast<__half*>(blk + norm_off + 2 * kBlockT)[tau] = __float2half_rn(sqrtf(g2[vv]));
+                }
             }
         }
         __syncthreads();
@@ -227,10 +230,10 @@ __global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
                 }
                 if (gv < N && lane < R) {
                     const int64_t tt = gv % a.Tnew, bh = gv / a.Tnew, t = a.t0 + tt;
-                    uint8_t* blk = a.cache + (bh * a.NB + (t >> 6)) * bb;
-                    uint32_t* sw = reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(D) +
+                    const int64_t pb = cache_block(a.table, a.pool, a.NB, bh, t >> 6, a.err);
+                    uint32_t* sw = reinterpret_cast<uint32_t*>(a.cache + pb * bb + kBlockT * code_bytes(D) +
                                                                (t & 63) * sign_bytes(D));
-                    sw[lane] = mine;
+                    if (pb >= 0) sw[lane] = mine;
                 }
             }
         }
@@ -249,8 +252,8 @@ __global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
                 const uint32_t tail = nibbles8(sw[6], sw[7]);
                 const uint32_t word = main | (((tail >> g) & 0x11111111u) << 3);
                 const int64_t tt = gv % a.Tnew, bh = gv / a.Tnew, tok = a.t0 + tt;
-                uint8_t* blk = a.cache + (bh * a.NB + (tok >> 6)) * bb;
-                reinterpret_cast<uint32_t*>(blk + (tok & 63) * code_bytes(D))[lane] = word;
+                const int64_t pb = cache_block(a.table, a.pool, a.NB, bh, tok >> 6, a.err);
+                if (pb >= 0) reinterpret_cast<uint32_t*>(a.cache + pb * bb + (tok & 63) * code_bytes(D))[lane] = word;
             }
         }
         __syncthreads();
@@ -296,7 +299,9 @@ __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(con
     const int64_t gv = valid ? gv0 : N - 1;
     const int64_t tt = gv % a.Tnew, bh = gv / a.Tnew;
     const int64_t t = a.t0 + tt;
-    uint8_t* blk = a.cache + (bh * a.NB + (t >> 6)) * block_bytes(D, true);
+    const int64_t pb = valid ? cache_block(a.table, a.pool, a.NB, bh, t >> 6, a.err) : 0;
+    uint8_t* blk = a.cache + (pb >= 0 ? pb : 0) * block_bytes(D, true);
+    const bool wr = valid && pb >= 0;                 // this warp stores its vector
     const int64_t h = bh % a.Hkv, b = bh / a.Hkv;
     const int64_t base = b * a.sb + h * a.sh + tt * a.st;
     float x[R];
@@ -340,7 +345,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(con
         scode[warp][(j >> 7) * 128 + slot_of(j) * 32 + slot_pos(j)] = (uint8_t)code;
     }
     g2 = warp_sum(g2);
-    const bool writer = valid && blockIdx.y == 0;
+    const bool writer = wr && blockIdx.y == 0;
     if (writer && lane == 0) {
         const int64_t norm_off = kBlockT * code_bytes(D) + kBlockT * sign_bytes(D);
         reinterpret_cast<__half*>(blk + norm_off)[t & 63] = __float2half_rn(n);
@@ -366,10 +371,10 @@ __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(con
         const uint32_t word = __ballot_sync(kFull, z[k] >= 0.f);
         if (lane == k) mine = word;
     }
-    if (lane < RG)
+    if (wr && lane < RG)
         reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(D) + (t & 63) * sign_bytes(D))[rg0 + lane] = mine;
     constexpr int W = 3 * D / 32;
-    if (blockIdx.y == 0 && lane < W) {
+    if (wr && blockIdx.y == 0 && lane < W) {
         const int sl = lane / 12, st = (lane % 12) / 3, g = lane % 3;
         const uint32_t* sw = reinterpret_cast<const uint32_t*>(&scode[warp][sl * 128 + st * 32]);
         const uint32_t main = nibbles8(sw[2 * g], sw[2 * g + 1]);

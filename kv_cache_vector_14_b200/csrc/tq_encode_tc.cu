@@ -296,7 +296,8 @@ __device__ __forceinline__ uint32_t pack_code_word(const uint8_t* rec, int w) {
     return main | (((tail >> g) & 0x11111111u) << 3);
 }
 
-// Input offset and cache block of vector gv (b, h, token order).
+// Input offset and cache block of vector gv (b, h, token order); blk is null
+// when a paged cache's table entry lies outside its pool.
 __device__ __forceinline__ void locate(const EncArgs& a, uint32_t gv, int64_t bb, int64_t& xoff, uint8_t*& blk,
                                        int& tau) {
     const uint32_t bh = fdiv(gv, a.fdT);
@@ -306,11 +307,13 @@ __device__ __forceinline__ void locate(const EncArgs& a, uint32_t gv, int64_t bb
     xoff = (int64_t)b * a.sb + (int64_t)hh * a.sh + (int64_t)tt * a.st;
     const int64_t t = a.t0 + tt;
     tau = (int)(t & 63);
-    blk = a.cache + ((int64_t)bh * a.NB + (t >> 6)) * bb;
+    const int64_t pb = cache_block(a.table, a.pool, a.NB, bh, t >> 6, a.err);
+    blk = pb >= 0 ? a.cache + pb * bb : nullptr;                   // null: nothing is written
 }
 
 // The 12 code words of each of the warp's four vectors (group g holds vector
-// g; my_rec is the code record of this lane's vector) from the staged bytes.
+// g; my_rec is the code record of this lane's vector, null to skip) from the
+// staged bytes.
 __device__ __forceinline__ void store_code_words(const uint8_t* stage, uint8_t* my_rec, int nvalid, int lane) {
     const unsigned long long mine = reinterpret_cast<unsigned long long>(my_rec);
 #pragma unroll
@@ -318,7 +321,7 @@ __device__ __forceinline__ void store_code_words(const uint8_t* stage, uint8_t* 
         const int idx = lane + 32 * k;                 // 4 vectors x 12 words
         const int vv = idx / 12, w = idx % 12;
         const unsigned long long rec = __shfl_sync(kFull, mine, 8 * (vv < 4 ? vv : 3));
-        if (idx < 48 && vv < nvalid)
+        if (idx < 48 && vv < nvalid && rec != 0ull)
             reinterpret_cast<uint32_t*>(rec)[w] = pack_code_word(stage + vv * 128, w);
     }
 }
@@ -399,7 +402,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
             uint8_t* blk;
             int tau;
             locate(a, (uint32_t)(r0 + v), bb, xoff, blk, tau);
-            reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(kD) + tau * sign_bytes(kD))[warp >> 2] = word;
+            if (blk)
+                reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(kD) + tau * sign_bytes(kD))[warp >> 2] = word;
         }
         tc_fence_before();
         return true;
@@ -432,13 +436,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
                 make_uint4(o.rl[4], o.rl[5], o.rl[6], o.rl[7]);
 #pragma unroll
             for (int t = 0; t < 4; ++t) *reinterpret_cast<uint32_t*>(stage + g * 128 + t * 32 + 4 * l) = o.cw[t];
-            if (valid && l == 0) {
+            if (valid && l == 0 && blk) {
                 __half* nf = reinterpret_cast<__half*>(blk + kBlockT * (code_bytes(kD) + sign_bytes(kD)));
                 nf[tau] = __float2half_rn(o.n);
                 nf[kBlockT + tau] = __float2half_rn(sqrtf(o.g2));
             }
             __syncwarp();
-            store_code_words(stage, blk + tau * code_bytes(kD), nrows - r0, lane);
+            store_code_words(stage, blk ? blk + tau * code_bytes(kD) : nullptr, nrows - r0, lane);
             __syncwarp();
         }
         // ---- step 5 on the tensor core: Z = R_hi S_hi^T + R_hi S_lo^T + R_lo S_hi^T
@@ -510,9 +514,10 @@ __global__ void __launch_bounds__(kVWarps * 32, 3) tq_encode_v128_kernel(const E
         encode_group<DT, false>(a.x, xoff, valid, vec, l, dsg, a.cb, nullptr, o);
 #pragma unroll
         for (int t = 0; t < 4; ++t) *reinterpret_cast<uint32_t*>(&scode[warp][g][t * 32 + 4 * l]) = o.cw[t];
-        if (valid && l == 0) reinterpret_cast<__half*>(blk + kBlockT * code_bytes(kD))[tau] = __float2half_rn(o.n);
+        if (valid && l == 0 && blk) reinterpret_cast<__half*>(blk + kBlockT * code_bytes(kD))[tau] = __float2half_rn(o.n);
         __syncwarp();
-        store_code_words(&scode[warp][0][0], blk + tau * code_bytes(kD), (int)(N - gv0 < 4 ? N - gv0 : 4), lane);
+        store_code_words(&scode[warp][0][0], blk ? blk + tau * code_bytes(kD) : nullptr, (int)(N - gv0 < 4 ? N - gv0 : 4),
+                         lane);
         __syncwarp();
     }
     pdl_wait();

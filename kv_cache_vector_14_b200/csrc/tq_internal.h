@@ -89,6 +89,8 @@ struct EncArgs {
     int64_t B, Hkv, Tnew, t0;
     int64_t NB;               // blocks per sequence (Tcap / 64)
     uint8_t* cache;
+    const int32_t* table;     // paged cache: [B*Hkv][NB] pool blocks, or null
+    int64_t pool;             // pool blocks of a paged cache
     const float* dsign;       // [d] +-1
     const float* sthr;        // [d][d/32][32] JL matrix, encode lane order
     const uint8_t* bimg;      // d = 128: JL matrix as tensor-core operand (hi, lo fp16 limbs)
@@ -103,6 +105,9 @@ struct DecArgs {
     const float* up;          // [B*Hq][d] sqrt(pi/2)/m * S q'
     const uint8_t* kc;
     const uint8_t* vc;
+    const int32_t* ktable;    // paged caches: block tables, or null
+    const int32_t* vtable;
+    int64_t kpool, vpool;
     int64_t NB;               // blocks per sequence
     const int32_t* seq_lens;  // device or null
     int64_t T;                // used when seq_lens is null
@@ -117,6 +122,22 @@ struct DecArgs {
     int64_t fresh_lo, fresh_hi;   // tokens written by a chained encode: read only after pdl_wait
     Codebook cb;
 };
+
+#ifdef __CUDACC__
+// Block index of logical block lb of sequence bh (= b * Hkv + h): bh * NB + lb
+// for a contiguous cache, the block table's entry for a paged one.  An entry
+// outside the pool sets the check word and gives -1.
+__device__ __forceinline__ int64_t cache_block(const int32_t* table, int64_t pool, int64_t NB, int64_t bh,
+                                               int64_t lb, int* err) {
+    if (!table) return bh * NB + lb;
+    const int32_t p = __ldg(table + bh * NB + lb);
+    if (p < 0 || (int64_t)p >= pool) {
+        atomicExch(err, 1);
+        return -1;
+    }
+    return p;
+}
+#endif
 
 // Programmatic dependent launch: a kernel launched with launch_pdl may start
 // while the previous kernel on the stream is still running; it must execute

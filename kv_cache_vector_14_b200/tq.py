@@ -33,7 +33,8 @@ class TQError(RuntimeError):
 
 
 class tq_cache(C.Structure):
-    _fields_ = [("base", C.c_void_p), ("B", C.c_int64), ("Hkv", C.c_int64), ("Tcap", C.c_int64)]
+    _fields_ = [("base", C.c_void_p), ("B", C.c_int64), ("Hkv", C.c_int64), ("Tcap", C.c_int64),
+                ("block_table", C.c_void_p), ("pool_blocks", C.c_int64)]
 
 
 _lock = threading.Lock()
@@ -172,17 +173,30 @@ def tq_cache_bytes(head_dim: int, is_k: bool, B: int, Hkv: int, Tcap: int) -> in
 class Cache:
     """A compressed K or V cache in a PyTorch-owned uint8 device buffer."""
 
-    def __init__(self, head_dim: int, is_k: bool, B: int, Hkv: int, Tcap: int, device="cuda", buf=None):
+    def __init__(self, head_dim: int, is_k: bool, B: int, Hkv: int, Tcap: int, device="cuda", buf=None,
+                 block_table=None, pool_blocks: int = 0):
+        """Contiguous cache, or (block_table: device int32 [B*Hkv, Tcap/64]) a
+        paged cache whose buffer is a pool of pool_blocks blocks."""
         import torch
-        nbytes = tq_cache_bytes(head_dim, is_k, B, Hkv, Tcap)
+        if block_table is not None:
+            if block_table.dtype != torch.int32 or tuple(block_table.shape) != (B * Hkv, Tcap // 64) or \
+                    not block_table.is_contiguous():
+                raise ValueError("block_table must be contiguous int32 [B*Hkv, Tcap/64]")
+            nbytes = pool_blocks * tq_block_bytes(head_dim, is_k)
+        else:
+            nbytes = tq_cache_bytes(head_dim, is_k, B, Hkv, Tcap)
         if nbytes == 0 and B * Hkv > 0:
             raise ValueError("Tcap must be a positive multiple of 64 and head_dim 128 or 256")
         self.head_dim, self.is_k, self.B, self.Hkv, self.Tcap = head_dim, is_k, B, Hkv, Tcap
+        self.block_table, self.pool_blocks = block_table, pool_blocks
         self.buf = buf if buf is not None else torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=device)
-        self.struct = tq_cache(C.c_void_p(self.buf.data_ptr()), B, Hkv, Tcap)
+        table = C.c_void_p(block_table.data_ptr()) if block_table is not None else None
+        self.struct = tq_cache(C.c_void_p(self.buf.data_ptr()), B, Hkv, Tcap, table, pool_blocks)
 
     @property
     def nbytes(self) -> int:
+        if self.block_table is not None:
+            return self.pool_blocks * tq_block_bytes(self.head_dim, self.is_k)
         return tq_cache_bytes(self.head_dim, self.is_k, self.B, self.Hkv, self.Tcap)
 
 

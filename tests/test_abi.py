@@ -50,6 +50,14 @@ def test_sizes_and_bits_per_dim(libtq, golden):
     assert tq.tq_cache_bytes(128, True, 1, 1, 0) == 0
 
 
+def test_cache_struct_layout():
+    """tq_cache as declared in include/tq.h: base, B, Hkv, Tcap, block_table,
+    pool_blocks, 8 bytes each."""
+    import ctypes as C
+    assert C.sizeof(tq.tq_cache) == 48
+    assert [getattr(tq.tq_cache, f).offset for f, _ in tq.tq_cache._fields_] == [0, 8, 16, 24, 32, 40]
+
+
 def test_host_argument_errors(libtq):
     with pytest.raises(tq.TQError) as e:
         tq.tq_params_host(64, 0)

@@ -216,6 +216,80 @@ def test_append_and_attend_loop_d256(handles, prms):
     assert torch.equal(kb.buf, kc.buf) and torch.equal(vb.buf, vc.buf)
 
 
+def _gather_blocks(cache: tq.Cache, table: torch.Tensor) -> torch.Tensor:
+    """The pool blocks of a paged cache in logical order ([B][Hkv][Tcap/64])."""
+    bb = O.block_bytes(cache.head_dim, cache.is_k)
+    pool = cache.buf[:cache.pool_blocks * bb].view(cache.pool_blocks, bb)
+    return pool.index_select(0, table.flatten().long()).flatten()
+
+
+@pytest.mark.parametrize("d", [128, 256])
+def test_paged_cache_matches_contiguous(handles, prms, d):
+    """Paged caches (blocks scattered over a pool by a random table) hold the
+    same bytes per logical block as contiguous caches after bulk encodes and
+    one-token appends; attention over them (the fused step) gives the same
+    output bit for bit as the separate calls on contiguous caches, and the
+    oracle's within the tolerance."""
+    h = handles[d]
+    B, Hkv, G, T0, S, Tcap = 2, 3, 4, 150, 3, 256
+    Hq, NB = Hkv * G, Tcap // 64
+    pool = 2 * B * Hkv * NB + 5
+    perm = np.random.default_rng(7).permutation(pool).astype(np.int32)
+    kt = torch.from_numpy(perm[:B * Hkv * NB].reshape(B * Hkv, NB).copy()).cuda()
+    vt = torch.from_numpy(perm[B * Hkv * NB:2 * B * Hkv * NB].reshape(B * Hkv, NB).copy()).cuda()
+    kp = tq.Cache(d, True, B, Hkv, Tcap, block_table=kt, pool_blocks=pool)
+    vp = tq.Cache(d, False, B, Hkv, Tcap, block_table=vt, pool_blocks=pool)
+    kc, vc = tq.Cache(d, True, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
+    x = torch_input(synthetic.gaussian((2, B, Hkv, T0 + S, d), seed=61), "bf16")
+    q = torch_input(synthetic.gaussian((S, B, Hq, d), seed=62), "f32")
+    for k_, v_ in ((kc, vc), (kp, vp)):
+        tq.tq_encode_k(h, x[0, :, :, :T0], k_, 0)
+        tq.tq_encode_v(h, x[1, :, :, :T0], v_, 0)
+    ws = torch.empty(tq.tq_attend_workspace_bytes(h, B, Hq, Hkv, Tcap), dtype=torch.uint8, device="cuda")
+    scale = 1.0 / np.sqrt(d)
+    for s in range(S):
+        t0 = T0 + s
+        ref = torch.empty((B, Hq, d), dtype=torch.float32, device="cuda")
+        out = torch.full((B, Hq, d), float("nan"), dtype=torch.float32, device="cuda")
+        tq.tq_encode_k(h, x[0, :, :, t0:t0 + 1], kc, t0)
+        tq.tq_encode_v(h, x[1, :, :, t0:t0 + 1], vc, t0)
+        tq.tq_attend_decode(h, q[s], kc, vc, ref, ws, T=t0 + 1, scale=scale)
+        tq.tq_append_attend(h, x[0, :, :, t0:t0 + 1], x[1, :, :, t0:t0 + 1], kp, vp, t0, q[s], out, ws,
+                            scale=scale)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref), f"step {s}"
+    assert torch.equal(_gather_blocks(kp, kt), kc.buf) and torch.equal(_gather_blocks(vp, vt), vc.buf)
+    T = T0 + S
+    oref = oracle_attend(prms[d], q[S - 1].double().cpu().numpy(), unpack_cache(kc, 0, T), unpack_cache(vc, 0, T),
+                         Hkv, [T] * B, scale)
+    assert rel_err_rows(out.cpu().numpy(), oref).max() <= ATT_TOL
+    assert tq.tq_device_status(h) == tq.TQ_OK
+
+
+def test_paged_cache_bad_table_entry_is_a_device_check(handles):
+    """A block-table entry outside the pool is caught by the kernels' own
+    check: nothing is written through it, reads go to block 0 (valid memory),
+    and tq_device_status reports the failed check once."""
+    d, h = 128, handles[128]
+    table = torch.tensor([[0, 2]], dtype=torch.int32, device="cuda")     # block 2 is outside a 2-block pool
+    kp = tq.Cache(d, True, 1, 1, 128, block_table=table, pool_blocks=2)
+    vp = tq.Cache(d, False, 1, 1, 128, block_table=table, pool_blocks=2)
+    x = torch_input(synthetic.gaussian((1, 1, 128, d), seed=71), "f32")
+    tq.tq_encode_k(h, x, kp, 0)
+    tq.tq_encode_v(h, x, vp, 0)
+    assert tq.tq_device_status(h) == tq.TQ_ERR_DEVICE_CHECK
+    assert tq.tq_device_status(h) == tq.TQ_OK                                 # the check word was cleared
+    for c in (kp, vp):
+        bb = O.block_bytes(d, c.is_k)
+        assert torch.any(c.buf[:bb] != 0) and not torch.any(c.buf[bb:2 * bb] != 0)
+    q = torch_input(synthetic.gaussian((1, 4, d), seed=72), "f32")
+    ws = torch.empty(tq.tq_attend_workspace_bytes(h, 1, 4, 1, 128), dtype=torch.uint8, device="cuda")
+    out = torch.empty((1, 4, d), dtype=torch.float32, device="cuda")
+    tq.tq_attend_decode(h, q, kp, vp, out, ws, T=128, scale=1.0 / np.sqrt(d))
+    assert tq.tq_device_status(h) == tq.TQ_ERR_DEVICE_CHECK
+    assert torch.isfinite(out).all()
+
+
 @pytest.mark.parametrize("d", [128, 256])
 @pytest.mark.parametrize("G,T0,Tnew", [(2, 0, 1), (4, 63, 1), (1, 64, 3), (8, 200, 2), (4, 1000, 1)])
 def test_fused_append_attend_equals_separate_calls(handles, d, G, T0, Tnew):
