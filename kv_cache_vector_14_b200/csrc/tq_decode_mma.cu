@@ -12,19 +12,18 @@
 // per token, about twice the HBM time.  The contraction maps onto
 // mma.sync.m16n8k16 (f16 inputs, f32 accumulation) with every operand exact:
 //   * dequantised keys/values c[idx] are fp16 numbers (the codebook is fp16);
-//   * sign terms are +-gamma_t with gamma_t the stored fp16 value;
-//   * q', u' and the softmax weights p * nv are fp32, split into fp16 hi + lo
-//     rows (rows 0..7 hi, 8..15 lo of the 16-row A operand), so the products
-//     carry ~22 significant bits and the sums are fp32.
-// Score tile:  D[16 rows = (head, hi|lo)][8 tokens] = sum over 8 coordinate
-//   chunks (B = c[idx]) and 8 sign chunks (B = +-gamma) of A(q'|u') B.
-// Value tile:  O[16 rows][8 coords] += P[16 rows][16 tokens] * V[16 tokens][8 coords],
-//   P taken straight from the score accumulators' register layout.
+//   * sign terms run on int8 mma (m16n8k32): each sign bit becomes an operand
+//     byte -128 sigma, u' is 16-bit fixed point per head in two byte limbs, the
+//     products accumulate exactly in int32 and gamma_t scales the sum;
+//   * q' and the softmax weights p * nv are fp32, split into fp16 hi + lo
+//     columns, so the products carry ~22 significant bits and the sums are
+//     fp32.
 // The packed layout is built for these fragments: a lane's codes for one
 // token come as three words whose nibbles are prmt selectors into byte
 // look-up tables of the fp16 centroids (lo bytes, hi bytes), and its sign
-// bits come as one word shifted into the fp16 sign positions.  Value
-// fragments are produced key-style and transposed in registers (movmatrix).
+// bits come as one word of which a shift and a mask keep four signs, one per
+// operand byte.  Value fragments are produced key-style and transposed in
+// registers (movmatrix).
 //
 // Data movement: each warp owns a ring of STAGES shared-memory buffers of a
 // chunk of tokens (32 at d = 128, 16 at d = 256; K codes, signs, norms,
@@ -34,7 +33,7 @@
 // contributes an empty partial.
 //
 // head_dim 256 is two 128-coordinate slices of the same record layout: the
-// k-loop runs over 16 coordinate chunks and 16 sign chunks, the value tile
+// k-loop runs over 16 coordinate chunks and 8 sign blocks, the value tile
 // over 16 coordinate tiles.  Its q'/u' fragments are read from shared memory
 // (filled once per CTA) instead of being held in registers.
 #include <type_traits>
@@ -116,6 +115,13 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// D += A B with signed 8-bit operands and exact 32-bit integer accumulation
+__device__ __forceinline__ void imma16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
     uint32_t y;
     asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
@@ -174,8 +180,8 @@ __device__ __forceinline__ uint32_t sel_for(const uint32_t (&sel)[4], const uint
 // ---------------------------------------------------------------- kernel
 // Token-row orientation: each mma tile has 16 tokens on M and the (head,
 // hi|lo) columns on N (NT n-tiles of 4 heads), so no M rows are wasted:
-//   scores  S[16 tok][8] += Kdeq[16 tok][16 coords] * Q'[16 coords][8]   (D/16 coordinate chunks)
-//                         + Sgn[16 tok][16 signs] * U'[16 signs][8]       (D/16 sign chunks)
+//   scores  S[16 tok][8] += Kdeq[16 tok][16 coords] * Q'[16 coords][8]   (D/16 coordinate chunks, fp16)
+//           Z[16 tok][8]  += Sgn[16 tok][32 signs] * U'[32 signs][8]      (D/32 sign blocks, int8)
 //   values  O^T[16 coords][8] += Vdeq^T[16 coords][16 tok] * P[16 tok][8] (D/16 coordinate tiles)
 // Lane (g, t) = (lane / 4, lane % 4) dequantises tokens g and g + 8 of each
 // 16-token tile; its score columns are head t (hi, lo), so its softmax state
@@ -207,10 +213,14 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     fence_mbar_init();
     __syncwarp();
 
-    auto issue = [&](int i) {
+    // cache blocks (K, V) of this warp's chunk i; a paged cache reads its block table
+    auto blocks_of = [&](int i, int64_t& kblk, int64_t& vblk) {
+        const int64_t t0 = s0 + (int64_t)(warp + i * NW) * C::kChunk;
+        kblk = cache_block(a.ktable, a.kpool, a.NB, seq, t0 >> 6, a.err);
+        vblk = cache_block(a.vtable, a.vpool, a.NB, seq, t0 >> 6, a.err);
+    };
+    auto issue = [&](int i, int64_t kblk, int64_t vblk) {
         const int64_t t0 = s0 + (int64_t)(warp + i * NW) * C::kChunk;     // multiple of the chunk
-        const int64_t kblk = cache_block(a.ktable, a.kpool, a.NB, seq, t0 >> 6, a.err);
-        const int64_t vblk = cache_block(a.vtable, a.vpool, a.NB, seq, t0 >> 6, a.err);
         const int sub = (int)((t0 & 63) / C::kChunk);
         const uint8_t* kb = a.kc + (kblk >= 0 ? kblk : 0) * kbb;    // a bad table entry reads block 0
         const uint8_t* vb = a.vc + (vblk >= 0 ? vblk : 0) * vbb;
@@ -236,7 +246,11 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     };
     if (lane == 0) {
         for (int i = 0; i < kStages && i < nmine; ++i)
-            if (!fresh(i)) issue(i);
+            if (!fresh(i)) {
+                int64_t kb_, vb_;
+                blocks_of(i, kb_, vb_);
+                issue(i, kb_, vb_);
+            }
     }
     pdl_wait();                           // q' and u' come from the prologue kernel
     if (lane == 0) {
@@ -245,9 +259,17 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         if (any) {
             asm volatile("fence.proxy.async;" ::: "memory");
             for (int i = 0; i < kStages && i < nmine; ++i)
-                if (fresh(i)) issue(i);
+                if (fresh(i)) {
+                    int64_t kb_, vb_;
+                    blocks_of(i, kb_, vb_);
+                    issue(i, kb_, vb_);
+                }
         }
     }
+    // blocks of the next chunk to issue, looked up one chunk ahead so that a
+    // block-table load overlaps a chunk of work
+    int64_t next_k = 0, next_v = 0;
+    if (lane == 0 && kStages < nmine) blocks_of(kStages, next_k, next_v);
 
     // B-operand fragment of k-step kc: column n = gr of n-tile nt is head
     // 4 nt + gr / 2, limb gr % 2; rows 16 kc + 2 tq4 (+1), +8 (+9)
@@ -264,29 +286,82 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         r0 = (gr & 1) ? l0 : h0;
         r1 = (gr & 1) ? l1 : h1;
     };
-    uint32_t bq[C::kBRegs ? NT : 1][C::kBRegs ? kKC : 1][2], bu[C::kBRegs ? NT : 1][C::kBRegs ? kKC : 1][2];
+    uint32_t bq[C::kBRegs ? NT : 1][C::kBRegs ? kKC : 1][2];
     if constexpr (C::kBRegs) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int kc = 0; kc < kKC; ++kc) {
-                b_frag(a.qp, nt, kc, bq[nt][kc][0], bq[nt][kc][1]);
-                if constexpr (QJL) b_frag(a.up, nt, kc, bu[nt][kc][0], bu[nt][kc][1]);
-            }
+            for (int kc = 0; kc < kKC; ++kc) b_frag(a.qp, nt, kc, bq[nt][kc][0], bq[nt][kc][1]);
     } else {
         for (int kc = warp; kc < kKC; kc += NW)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 uint32_t r0, r1;
                 b_frag(a.qp, nt, kc, r0, r1);
-                sB[((0 * NT + nt) * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
-                if constexpr (QJL) {
-                    b_frag(a.up, nt, kc, r0, r1);
-                    sB[((1 * NT + nt) * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
+                sB[(nt * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
+            }
+    }
+    // QJL term on int8 operands.  u' of each head is taken to 16-bit fixed point,
+    // u_int = rint(u' kQ / max|u'|), as two signed byte limbs (256 hi + lo): B column
+    // n = gr of n-tile nt is head 4 nt + gr / 2, limb gr % 2.  The A operand byte e
+    // of a0/a1 (a2/a3) in k-block kb is -128 times bit 8 e + 7 - 2 (kb % 4)
+    // (8 e + 6 - 2 (kb % 4)) of lane tq4's sign word of slice kb / 4, so b0 (b1)
+    // byte e holds u_int of that bit's JL row.  With acc = sum of the products,
+    // sum_i u'_i (2 sigma_i - 1) = (max|u'| / kQ) (-acc / 64 - sum_i u_int_i), exact
+    // up to the fixed point of u' (the term is scaled by gamma ~ 0.18 of the score).
+    constexpr int kKB = D / 32;
+    constexpr float kQ = 32000.f;
+    [[maybe_unused]] uint32_t iu[QJL && C::kBRegs ? NT : 1][QJL && C::kBRegs ? kKB : 1][2];
+    [[maybe_unused]] float fS[NT], uS[NT];   // factors of this lane's own head 4 nt + tq4
+    if constexpr (QJL) {
+        auto row_of = [&](int kb, int half, int e) {
+            const int bit = 8 * e + 7 - 2 * (kb & 3) - half;
+            return slot_coord(kb >> 2, tq4, bit < 16 ? 2 * bit : 2 * (bit - 16) + 1);
+        };
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int hcol = 4 * nt + (gr >> 1);
+            const bool live = hcol < G;
+            const float* up = a.up + ((int64_t)b * a.Hq + (int64_t)hkv * G + (live ? hcol : 0)) * D;
+            float um = 0.f;
+#pragma unroll
+            for (int kb = 0; kb < kKB; ++kb)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) um = fmaxf(um, fabsf(up[row_of(kb, hf, e)]));
+            um = fmaxf(um, __shfl_xor_sync(kFull, um, 1));
+            um = fmaxf(um, __shfl_xor_sync(kFull, um, 2));
+            if (!live) um = 0.f;
+            const float fu = um > 0.f ? kQ / um : 0.f;
+            int usum = 0;
+#pragma unroll
+            for (int kb = 0; kb < kKB; ++kb) {
+                uint32_t w[2] = {0u, 0u};
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int ui = __float2int_rn(up[row_of(kb, hf, e)] * fu);
+                        const int lo = ((ui + 128) & 255) - 128;
+                        w[hf] |= (uint32_t)(uint8_t)(int8_t)((gr & 1) ? lo : (ui - lo) >> 8) << (8 * e);
+                        usum += ui;
+                    }
+                if constexpr (C::kBRegs) {
+                    iu[nt][kb][0] = w[0];
+                    iu[nt][kb][1] = w[1];
+                } else if (warp == 0) {
+                    sB[((NT + nt) * kKC + kb) * 32 + lane] = make_uint2(w[0], w[1]);
                 }
             }
-        __syncthreads();
+            usum += __shfl_xor_sync(kFull, usum, 1);
+            usum += __shfl_xor_sync(kFull, usum, 2);
+            // this lane's score columns are head 4 nt + tq4, whose factors sit in lane 8 tq4
+            fS[nt] = a.scale_log2 * (__shfl_sync(kFull, um, 8 * tq4) / kQ) * (1.f / 64.f);
+            uS[nt] = 64.f * (float)__shfl_sync(kFull, usum, 8 * tq4);
+        }
     }
+    if constexpr (!C::kBRegs) __syncthreads();
     const uint32_t lut[4] = {a.cb.lut_lo[0], a.cb.lut_lo[1], a.cb.lut_hi[0], a.cb.lut_hi[1]};
     const uint32_t* pw = a.cb.pow2;
 
@@ -334,44 +409,51 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                     sgB[sl] = *reinterpret_cast<const uint32_t*>(st + C::kOffKs + tB * C::kSignB + sl * 16 + tq4 * 4);
                 }
             }
-            [[maybe_unused]] uint32_t ggA = 0, ggB = 0;
-            if constexpr (QJL) {
-                const uint32_t gA = *reinterpret_cast<const uint16_t*>(st + C::kOffKg + 2 * tA);
-                const uint32_t gB = *reinterpret_cast<const uint16_t*>(st + C::kOffKg + 2 * tB);
-                ggA = gA | (gA << 16);
-                ggB = gB | (gB << 16);
-            }
             float acc[NT][4];
+            [[maybe_unused]] int accS[NT][4];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+            for (int nt = 0; nt < NT; ++nt) {
+                acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+                accS[nt][0] = accS[nt][1] = accS[nt][2] = accS[nt][3] = 0;
+            }
 #pragma unroll
             for (int kc = 0; kc < kKC; ++kc) {
                 const int sl = kc >> 3, kk = kc & 7;
                 uint32_t ka[4];
                 dequant4(sel_for(selA[sl], pw, kk), lut, ka[0], ka[2]);
                 dequant4(sel_for(selB[sl], pw, kk), lut, ka[1], ka[3]);
-                [[maybe_unused]] uint32_t sa[4] = {0u, 0u, 0u, 0u};
-                if constexpr (QJL) {
-                    // sign bit 1 -> +gamma: the pair (2kk | 2kk+1) of a slot sits at bits (q, 16 + q)
-                    sa[0] = ggA ^ (~shl_m(sgA[sl], pw, 15 - 2 * kk) & 0x80008000u);
-                    sa[1] = ggB ^ (~shl_m(sgB[sl], pw, 15 - 2 * kk) & 0x80008000u);
-                    sa[2] = ggA ^ (~shl_m(sgA[sl], pw, 14 - 2 * kk) & 0x80008000u);
-                    sa[3] = ggB ^ (~shl_m(sgB[sl], pw, 14 - 2 * kk) & 0x80008000u);
-                }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     if constexpr (C::kBRegs) {
                         mma16816(acc[nt], ka, bq[nt][kc][0], bq[nt][kc][1]);
-                        if constexpr (QJL) mma16816(acc[nt], sa, bu[nt][kc][0], bu[nt][kc][1]);
                     } else {
-                        const uint2 fq = sB[((0 * NT + nt) * kKC + kc) * 32 + lane];
+                        const uint2 fq = sB[(nt * kKC + kc) * 32 + lane];
                         mma16816(acc[nt], ka, fq.x, fq.y);
-                        if constexpr (QJL) {
-                            const uint2 fu = sB[((1 * NT + nt) * kKC + kc) * 32 + lane];
-                            mma16816(acc[nt], sa, fu.x, fu.y);
+                    }
+                }
+                if constexpr (QJL) {
+                    if ((kc & 1) == 0) {                        // one k32 block of signs per two k-steps
+                        const int kb = kc >> 1, k4 = kb & 3;
+                        const uint32_t sg[4] = {shl_m(sgA[sl], pw, 2 * k4) & 0x80808080u,
+                                                shl_m(sgB[sl], pw, 2 * k4) & 0x80808080u,
+                                                shl_m(sgA[sl], pw, 2 * k4 + 1) & 0x80808080u,
+                                                shl_m(sgB[sl], pw, 2 * k4 + 1) & 0x80808080u};
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            if constexpr (C::kBRegs) {
+                                imma16832(accS[nt], sg, iu[nt][kb][0], iu[nt][kb][1]);
+                            } else {
+                                const uint2 fu = sB[((NT + nt) * kKC + kb) * 32 + lane];
+                                imma16832(accS[nt], sg, fu.x, fu.y);
+                            }
                         }
                     }
                 }
+            }
+            [[maybe_unused]] float gAf = 0.f, gBf = 0.f;
+            if constexpr (QJL) {
+                gAf = __half2float(*reinterpret_cast<const __half*>(st + C::kOffKg + 2 * tA));
+                gBf = __half2float(*reinterpret_cast<const __half*>(st + C::kOffKg + 2 * tB));
             }
             // ---------------- online softmax per head (this lane: head 4 nt + tq4)
             const float2 nkA = __half22float2(__halves2half2(*reinterpret_cast<const __half*>(st + C::kOffKn + 2 * tA),
@@ -386,8 +468,15 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
             uint32_t pb[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                float sA = a.scale_log2 * nkA.x * (acc[nt][0] + acc[nt][1]);
-                float sB_ = a.scale_log2 * nkA.y * (acc[nt][2] + acc[nt][3]);
+                float sA = a.scale_log2 * (acc[nt][0] + acc[nt][1]);
+                float sB_ = a.scale_log2 * (acc[nt][2] + acc[nt][3]);
+                if constexpr (QJL) {
+                    // + gamma (max|u'| / kQ) (-acc / 64 - sum u_int), acc = 256 hi-limb + lo-limb column
+                    sA = fmaf(-gAf * fS[nt], (float)(accS[nt][0] * 256 + accS[nt][1]) + uS[nt], sA);
+                    sB_ = fmaf(-gBf * fS[nt], (float)(accS[nt][2] * 256 + accS[nt][3]) + uS[nt], sB_);
+                }
+                sA *= nkA.x;
+                sB_ *= nkA.y;
                 if constexpr (PARTIAL) {
                     if (!okA) sA = -INFINITY;
                     if (!okB) sB_ = -INFINITY;
@@ -445,7 +534,8 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         __syncwarp();
         if (lane == 0 && i + kStages < nmine) {
             fence_proxy_async();
-            issue(i + kStages);
+            issue(i + kStages, next_k, next_v);
+            if (i + kStages + 1 < nmine) blocks_of(i + kStages + 1, next_k, next_v);
         }
     }
 #pragma unroll

@@ -11,8 +11,8 @@
 // four vectors per warp at a time): ||x|| by three shuffle steps, the random
 // sign flip, the Walsh-Hadamard butterflies (4 register stages over coordinate
 // bits 0..3, 3 shuffle stages over bits 4..6), the scale 1 / (||x|| sqrt(d)),
-// the bucket index by binary search over the 7 boundaries, and for K the
-// residual r = y - c[idx] and gamma = ||r||.
+// the bucket index and centroid by saturating compares on the FMA pipe, and for
+// K the residual r = y - c[idx] and gamma = ||r||.
 //
 // K, step 5 (z = S r, sign bits): the tile's residuals (up to 128 vectors) are
 // written to shared memory as two fp16 limbs of r * 2^12 (hi = fp16(r 2^12),
@@ -197,8 +197,7 @@ struct GroupOut {
 // Steps 1-4 for the vector of this lane's group of 8 lanes (lane l = lane & 7).
 template <int DT, bool IS_K>
 __device__ __forceinline__ void encode_group(const void* x, int64_t off, bool valid, bool vec, int l,
-                                             const float (&dsg)[16], const Codebook& cb, const float* sC,
-                                             GroupOut& o) {
+                                             const float (&dsg)[16], const Codebook& cb, GroupOut& o) {
     float v[16];
     if (valid) {
         load16<DT>(x, off + 16 * l, vec, v);
@@ -237,7 +236,19 @@ __device__ __forceinline__ void encode_group(const void* x, int64_t off, bool va
     const float n = sqrtf(ss);
     const bool nz = n > 0.f;
     const float rcp = nz ? __frcp_rn(n * 11.3137084989847604f) : 0.f;   // 1 / (||x|| sqrt(128))
-    uint32_t code[16];
+    // Bucket index and centroid on the FMA pipe.  The codebook is antisymmetric
+    // (b3 = 0, b[6-k] = -b[k], c[7-k] = -c[k]), so with a = |y| and
+    // t_k = sat((b_k - a) 2^60) = [a < b_k] for k = 4, 5, 6 (the product is exact,
+    // its sign decides, and any nonzero difference of two such floats
+    // saturates), T = t4 + t5 + t6 boundaries lie above a: the code is 7 - T for
+    // y >= 0 and T below (a tie at a positive boundary goes up; at a negative
+    // one it goes down, which is inside the 1e-6 window), and
+    // |c| = c7 - t6 (c7 - c6) - t5 (c6 - c5) - t4 (c5 - c4), every partial sum an
+    // exact centroid.
+    constexpr float kBig = 1152921504606846976.f;        // 2^60
+    const float bb4 = cb.b[4] * kBig, bb5 = cb.b[5] * kBig, bb6 = cb.b[6] * kBig;
+    [[maybe_unused]] const float d3 = cb.c[7] - cb.c[6], d2 = cb.c[6] - cb.c[5], d1 = cb.c[5] - cb.c[4];
+    float codef[16];
     float g2 = 0.f;
 #pragma unroll
     for (int i = 0; i < 16; i += 2) {
@@ -245,14 +256,18 @@ __device__ __forceinline__ void encode_group(const void* x, int64_t off, bool va
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const float y = v[i + e] * rcp;
-            // number of boundaries <= y, by binary search over the sorted b[0..6]
-            const bool p2 = y >= cb.b[3];
-            const bool p1 = y >= (p2 ? cb.b[5] : cb.b[1]);
-            const bool p0 = y >= (p2 ? (p1 ? cb.b[6] : cb.b[4]) : (p1 ? cb.b[2] : cb.b[0]));
-            const int c = (p2 ? 4 : 0) | (p1 ? 2 : 0) | (p0 ? 1 : 0);
-            code[i + e] = (uint32_t)c;
+            const float a = fabsf(y);
+            const float t4 = __saturatef(fmaf(a, -kBig, bb4));
+            const float t5 = __saturatef(fmaf(a, -kBig, bb5));
+            const float t6 = __saturatef(fmaf(a, -kBig, bb6));
+            const float T = (t4 + t5) + t6;
+            const float pos = (y >= 0.f) ? 1.f : 0.f;
+            codef[i + e] = fmaf(pos, fmaf(T, -2.f, 7.f), T);
             if constexpr (IS_K) {
-                const float r = nz ? y - sC[c] : 0.f;
+                float m = fmaf(-t6, d3, cb.c[7]);
+                m = fmaf(-t5, d2, m);
+                m = fmaf(-t4, d1, m);
+                const float r = nz ? y - m * fmaf(pos, 2.f, -1.f) : 0.f;
                 g2 = fmaf(r, r, g2);
                 rr[e] = r * kRScale;
             }
@@ -270,10 +285,14 @@ __device__ __forceinline__ void encode_group(const void* x, int64_t off, bool va
         g2 += __shfl_xor_sync(kFull, g2, 2);
         g2 += __shfl_xor_sync(kFull, g2, 4);
     }
-    // slot t holds positions 4l + {0,1,2,3} = coordinates 16l + {2t, 2t+1, 2t+8, 2t+9}
+    // slot t holds positions 4l + {0,1,2,3} = coordinates 16l + {2t, 2t+1, 2t+8, 2t+9}; the
+    // byte pairs are formed as exact float sums and read out of the mantissa (x + 2^23)
 #pragma unroll
-    for (int t = 0; t < 4; ++t)
-        o.cw[t] = code[2 * t] | (code[2 * t + 1] << 8) | (code[2 * t + 8] << 16) | (code[2 * t + 9] << 24);
+    for (int t = 0; t < 4; ++t) {
+        const float lo = fmaf(codef[2 * t + 1], 256.f, codef[2 * t]) + 8388608.f;
+        const float hi = fmaf(codef[2 * t + 9], 256.f, codef[2 * t + 8]) + 8388608.f;
+        o.cw[t] = __byte_perm(__float_as_uint(lo), __float_as_uint(hi), 0x5410);
+    }
     o.n = n;
     o.g2 = g2;
 }
@@ -336,7 +355,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);     // [0] JL image copy, [1..2] mma done
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffBar + 32);
     uint8_t* scode = sm + kOffCode;
-    __shared__ float sC[8];
     pdl_trigger();                 // a chained kernel may start (it waits for this one's writes)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 3, l = lane & 7;
@@ -345,7 +363,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
     const int64_t bb = block_bytes(kD, true);
     const uint32_t bar_b = smem_u32(&bars[0]);
 
-    if (threadIdx.x < 8) sC[threadIdx.x] = a.cb.c[threadIdx.x];
     if (threadIdx.x == 0) {
         mbar_init(bar_b, 1);
         mbar_init(smem_u32(&bars[1]), 1);
@@ -426,7 +443,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
             int tau;
             locate(a, (uint32_t)(row0 + (valid ? v : r0)), bb, xoff, blk, tau);
             GroupOut o;
-            encode_group<DT, true>(a.x, xoff, valid, vec, l, dsg, a.cb, sC, o);
+            encode_group<DT, true>(a.x, xoff, valid, vec, l, dsg, a.cb, o);
             *reinterpret_cast<uint4*>(A + sw128_k_offset(v, 16 * l)) = make_uint4(o.rh[0], o.rh[1], o.rh[2], o.rh[3]);
             *reinterpret_cast<uint4*>(A + sw128_k_offset(v, 16 * l + 8)) =
                 make_uint4(o.rh[4], o.rh[5], o.rh[6], o.rh[7]);
@@ -511,7 +528,7 @@ __global__ void __launch_bounds__(kVWarps * 32, 3) tq_encode_v128_kernel(const E
         int tau;
         locate(a, (uint32_t)(valid ? gv0 + g : gv0), bb, xoff, blk, tau);
         GroupOut o;
-        encode_group<DT, false>(a.x, xoff, valid, vec, l, dsg, a.cb, nullptr, o);
+        encode_group<DT, false>(a.x, xoff, valid, vec, l, dsg, a.cb, o);
 #pragma unroll
         for (int t = 0; t < 4; ++t) *reinterpret_cast<uint32_t*>(&scode[warp][g][t * 32 + 4 * l]) = o.cw[t];
         if (valid && l == 0 && blk) reinterpret_cast<__half*>(blk + kBlockT * code_bytes(kD))[tau] = __float2half_rn(o.n);

@@ -50,6 +50,19 @@ def test_sizes_and_bits_per_dim(libtq, golden):
     assert tq.tq_cache_bytes(128, True, 1, 1, 0) == 0
 
 
+@pytest.mark.parametrize("d", [128, 256])
+def test_codebook_is_exactly_antisymmetric(libtq, d):
+    """The encode kernels find the cell and the centroid from |y| alone; that
+    needs c[7-k] = -c[k], b[6-k] = -b[k] and b[3] = 0 exactly in fp32, and exact
+    differences of adjacent centroids (all checked on the library's constants)."""
+    p = tq.tq_params_host(d, 0)
+    c, b = np.asarray(p["c8"], np.float32), np.asarray(p["b7"], np.float32)
+    assert b[3] == 0.0
+    assert all(c[7 - k] == -c[k] for k in range(8)) and all(b[6 - k] == -b[k] for k in range(7))
+    for k in (4, 5, 6):
+        assert np.float64(c[k + 1]) - np.float64(c[k]) == np.float64(np.float32(c[k + 1] - c[k]))
+
+
 def test_cache_struct_layout():
     """tq_cache as declared in include/tq.h: base, B, Hkv, Tcap, block_table,
     pool_blocks, 8 bytes each."""
