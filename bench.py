@@ -57,6 +57,14 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def bf16_peak_tflops() -> float:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
+
+
 def source_sha(rel: str) -> str:
     with open(os.path.join(ROOT, rel), "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()
@@ -460,6 +468,48 @@ def measure_paged(h, dev, w, kc, vc, q, out_ref, ws, n_calls: int) -> dict:
             "output_equals_contiguous": same}
 
 
+def measure_prefill(dev, world: int, dist, reps: int = 20, Lq: int = 512) -> dict:
+    """Chunked prefill on the GQA workload's cache (B=1, Hq=32/Hkv=8, d=128,
+    40960 tokens): the last Lq tokens' queries as one chunk, query i attending
+    causally over tokens [0, T - Lq + i].  Timed per call (prologue, prefill
+    kernel, combine).  Work: 3 contractions of d multiply-adds per (query row,
+    visible token) pair: 6 d flops."""
+    import torch
+    from kv_cache_vector_14_b200 import tq
+    w = synthetic.WORKLOADS["c3"]
+    d, B, Hq, Hkv, T = w.d, w.B, w.Hq, w.Hkv, w.T
+    T0 = T - Lq
+    h = tq.tq_init(d, 0)
+    kc, vc = tq.Cache(d, True, B, Hkv, T), tq.Cache(d, False, B, Hkv, T)
+    for which, cache in (("k", kc), ("v", vc)):
+        x = torch.from_numpy(synthetic.kv(w, which)).to(dev).to(torch.bfloat16)
+        (tq.tq_encode_k if which == "k" else tq.tq_encode_v)(h, x, cache, 0)
+        del x
+    q = torch.from_numpy(synthetic.gaussian((B, Lq, Hq, d), seed=11)).to(dev).to(torch.bfloat16)
+    out = torch.empty((B, Lq, Hq, d), dtype=torch.float32, device=dev)
+    ws = torch.empty(tq.tq_prefill_workspace_bytes(h, B, Lq, Hq), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        tq.tq_attend_prefill(h, q, kc, vc, T0, out, ws, scale=w.scale)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        tq.tq_attend_prefill(h, q, kc, vc, T0, out, ws, scale=w.scale)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    status = tq.tq_status_string(tq.tq_device_status(h))
+    tq.tq_destroy(h)
+    pairs = B * Hq * (Lq * T0 + Lq * (Lq + 1) // 2)
+    flops = 6 * d * pairs
+    return {"workload": f"chunked prefill: B=1, Hq=32/Hkv=8, d=128, {Lq} queries after {T0} cached tokens",
+            "ms_per_call": ms, "query_token_pairs": pairs, "algorithmic_flops": flops,
+            "tflops": world * flops / (max_over_ranks(ms, dist, dev) * 1e-3) / 1e12,
+            "device_status": status}
+
+
 def run_ours(args, rank: int, world: int, dist):
     import torch
     from kv_cache_vector_14_b200 import build, tq
@@ -475,6 +525,12 @@ def run_ours(args, rank: int, world: int, dist):
         tq.tq_destroy(h)
         if rank == 0:
             print(json.dumps({"encode": enc}), flush=True)
+        return
+    if args.only == "prefill":         # profiling aid: the chunked-prefill workload alone
+        tq.tq_destroy(h)
+        pf = measure_prefill(dev, world, dist, reps=args.steps)
+        if rank == 0:
+            print(json.dumps({"prefill": pf}), flush=True)
         return
     if args.only == "loop":            # profiling aid: the append-and-attend workload alone
         tq.tq_destroy(h)
@@ -600,8 +656,10 @@ def run_ours(args, rank: int, world: int, dist):
     paged = measure_paged(h, dev, w, kc, vc, q, out.clone(), ws, n_kern)
     enc = measure_encode(h, dev, world, dist)
     loop = measure_loop(dev, world, dist)
+    prefill = measure_prefill(dev, world, dist)
 
     peak, peak_kind = peaks()
+    bf16_peak = bf16_peak_tflops()
     achieved = bytes_step / (kern_ms * 1e-3) / 1e9
     traffic = NCU_TRAFFIC["bytes_per_launch"] if (path == "mma" and NCU_TRAFFIC["source_sha256"] == source_sha(
         "kv_cache_vector_14_b200/csrc/tq_decode_mma.cu")) else None
@@ -642,6 +700,8 @@ def run_ours(args, rank: int, world: int, dist):
         "loop": {**loop, "frac": loop["achieved_gbs"] / peak},
         "polar_k": {**polar, "frac": polar["achieved_gbs"] / peak},
         "paged": {**paged, "frac": paged["achieved_gbs"] / peak},
+        "prefill": {**prefill, "peak_tflops": bf16_peak, "frac": prefill["tflops"] / bf16_peak,
+                    "peak_kind": "measured bf16 dense GEMM (burst); the kernel uses mma.sync fp16/int8"},
         "device_status": tq.tq_status_string(status),
     }
     print(json.dumps(line), flush=True)
@@ -655,9 +715,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["step", "encode", "loop"], default=None,
+    ap.add_argument("--only", choices=["step", "encode", "loop", "prefill"], default=None,
                     help="run only the decode step (--steps steps), the encode-only workload (--steps "
-                         "passes) or the append-and-attend workload (--steps graph replays); for profiling")
+                         "passes), the append-and-attend workload (--steps graph replays) or the chunked "
+                         "prefill (--steps calls); for profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

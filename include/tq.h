@@ -193,6 +193,27 @@ TQ_API tq_status tq_attend_decode_polar(const tq_handle* h, const void* q, tq_dt
                                         const int32_t* seq_lens, int64_t T, float scale, float* out, void* ws,
                                         size_t ws_bytes, void* stream);
 
+/* ---- chunked prefill ------------------------------------------------------ */
+
+/* Workspace bytes tq_attend_prefill needs (rotated queries and the per-row
+ * softmax partials of B * Lq * Hq query rows).  0 on bad arguments. */
+TQ_API size_t tq_prefill_workspace_bytes(const tq_handle* h, int64_t B, int64_t Lq, int64_t Hq);
+
+/* Attention for a chunk of Lq new queries per sequence (q [B][Lq][Hq][d]
+ * contiguous, `qdtype`) over the compressed caches, causal: query i of the
+ * chunk attends over tokens [0, T0 + i] of its sequence, so the chunk's own K
+ * and V must already be encoded at positions T0 .. T0 + Lq - 1.  Scores and
+ * output as tq_attend_decode (the same estimator, in the page's K section and
+ * hybrid V2+V3 section, with the QJL term evaluated on 16-bit fixed-point u');
+ * out is fp32 [B][Lq][Hq][d].  With many queries per kv head the score and
+ * value contractions are dense and run on tensor cores with the keys
+ * dequantised once per 16 query rows.  Supported: d = 128, Hq/Hkv in
+ * {1, 2, 4, 8}, T0 + Lq <= Tcap; contiguous or paged caches.
+ * Errors: INVALID_ARG, UNSUPPORTED (d != 128, group size), WORKSPACE, CUDA. */
+TQ_API tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype qdtype, int64_t B, int64_t Lq,
+                                   int64_t Hq, const tq_cache* kc, const tq_cache* vc, int64_t T0, float scale,
+                                   float* out, void* ws, size_t ws_bytes, void* stream);
+
 /* ---- fused append-and-attend step ---------------------------------------- */
 
 /* One decode step of a serving loop: encode Tnew new K and V vectors per

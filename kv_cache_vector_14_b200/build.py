@@ -31,7 +31,8 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = sources() + glob.glob(os.path.join(PKG, "csrc", "*.h")) + [os.path.join(ROOT, "include", "tq.h")]
+    deps = (sources() + glob.glob(os.path.join(PKG, "csrc", "*.h")) + glob.glob(os.path.join(PKG, "csrc", "*.cuh")) +
+            [os.path.join(ROOT, "include", "tq.h")])
     return any(os.path.getmtime(p) > t for p in deps)
 
 

@@ -329,6 +329,63 @@ size_t tq_attend_workspace_bytes(const tq_handle* h, int64_t B, int64_t Hq, int6
     return p.bytes;
 }
 
+size_t tq_prefill_workspace_bytes(const tq_handle* h, int64_t B, int64_t Lq, int64_t Hq) {
+    if (!h || B < 0 || Lq < 0 || Hq <= 0) return 0;
+    DecodePlan p;
+    layout_ws(h->d, (size_t)(B * Lq * Hq), 1, &p);
+    return p.bytes;
+}
+
+tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype qdt, int64_t B, int64_t Lq, int64_t Hq,
+                            const tq_cache* kc, const tq_cache* vc, int64_t T0, float scale, float* out, void* ws,
+                            size_t ws_bytes, void* stream) {
+    if (!h || !dtype_ok(qdt) || !cache_ok(h, kc) || !cache_ok(h, vc)) return TQ_ERR_INVALID_ARG;
+    if (B < 0 || Lq < 0 || Hq <= 0 || T0 < 0 || kc->B != B || vc->B != B || kc->Hkv != vc->Hkv ||
+        kc->Tcap != vc->Tcap || T0 + Lq > kc->Tcap || !std::isfinite(scale))
+        return TQ_ERR_INVALID_ARG;
+    const int64_t Hkv = kc->Hkv;
+    if (Hq % Hkv) return TQ_ERR_INVALID_ARG;
+    const int G = (int)(Hq / Hkv);
+    if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_ERR_UNSUPPORTED;
+    if (h->d != 128) return TQ_ERR_UNSUPPORTED;
+    if (B == 0 || Lq == 0) return TQ_OK;
+    if (!q || !out || !ws || !aligned(q, dtype_size(qdt)) || !aligned(out, 16) || !aligned(ws, 256))
+        return TQ_ERR_INVALID_ARG;
+    if (B * Lq * Hq >= ((int64_t)1 << 31)) return TQ_ERR_UNSUPPORTED;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
+    if (dev != h->device) return TQ_ERR_INVALID_ARG;
+    const int64_t rows = B * Lq * Hq;
+    DecodePlan p;
+    layout_ws(h->d, (size_t)rows, 1, &p);
+    if (ws_bytes < p.bytes) return TQ_ERR_WORKSPACE;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    DecArgs a{};
+    a.qp = reinterpret_cast<float*>(w + p.off_qp);
+    a.up = reinterpret_cast<float*>(w + p.off_up);
+    a.kc = static_cast<const uint8_t*>(kc->base);
+    a.vc = static_cast<const uint8_t*>(vc->base);
+    a.ktable = kc->block_table;
+    a.vtable = vc->block_table;
+    a.kpool = kc->pool_blocks;
+    a.vpool = vc->pool_blocks;
+    a.NB = kc->Tcap / kBlockT;
+    a.Tcap = kc->Tcap;
+    a.B = B; a.Hq = Hq; a.Hkv = Hkv;
+    a.nsplit = 1;
+    a.scale_log2 = scale * kLog2e;
+    a.part_ml = reinterpret_cast<float*>(w + p.off_ml);
+    a.part_acc = reinterpret_cast<float*>(w + p.off_acc);
+    a.err = h->derr;
+    a.cb = h->cb;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_prologue(h->d, q, qdt, rows, h->dsign, h->dST, const_cast<float*>(a.qp),
+                                    const_cast<float*>(a.up), false, s);
+    if (e == cudaSuccess) e = launch_prefill(h->d, G, a, Lq, T0, s);
+    if (e == cudaSuccess) e = launch_combine(h->d, rows, 1, a.part_ml, a.part_acc, h->dsign, out, s);
+    return cuda_status(e);
+}
+
 const char* tq_attend_path(const tq_handle* h, int64_t Hq, int64_t Hkv) {
     if (!h || Hq <= 0 || Hkv <= 0 || Hq % Hkv) return "invalid";
     return (!h->force_simt && mma_supported(h->d, (int)(Hq / Hkv))) ? "mma" : "simt";

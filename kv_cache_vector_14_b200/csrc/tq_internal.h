@@ -185,6 +185,9 @@ cudaError_t launch_encode128(bool is_k, tq_dtype dt, const EncArgs& a, int num_s
 // append-and-attend step); the kernels then complete only after it.
 cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, const float* dsign,
                             const float* st, float* qp, float* up, bool pdl, cudaStream_t s);
+// Chunked prefill (head_dim 128): rows (b, i, head) of Lq queries per sequence,
+// query i over tokens [0, T0 + i]; partials as one split of a.part_ml/part_acc.
+cudaError_t launch_prefill(int d, int G, const DecArgs& a, int64_t Lq, int64_t T0, cudaStream_t s);
 // qjl = false: PolarQuant-only K cache (V layout), scores without the QJL term.
 cudaError_t launch_decode(int d, int G, bool use_mma, bool qjl, const DecArgs& a, cudaStream_t s);
 cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml,

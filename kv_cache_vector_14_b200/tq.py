@@ -22,7 +22,7 @@ TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 
 EXPORTED = ("tq_params_host", "tq_init", "tq_destroy", "tq_get_params", "tq_head_dim", "tq_block_bytes",
             "tq_cache_bytes", "tq_encode_k", "tq_encode_v", "tq_attend_workspace_bytes", "tq_attend_decode",
-            "tq_append_attend", "tq_attend_decode_polar",
+            "tq_append_attend", "tq_prefill_workspace_bytes", "tq_attend_prefill", "tq_attend_decode_polar",
             "tq_attend_decode_static", "tq_device_status", "tq_set_decode_events", "tq_set_decode_path", "tq_attend_path", "tq_status_string")
 
 
@@ -81,6 +81,11 @@ def lib() -> C.CDLL:
             L.tq_append_attend.argtypes = [P, P, P, i32, i64, i64, i64, i64, C.POINTER(tq_cache),
                                            C.POINTER(tq_cache), i64, P, i32, i64, C.c_float, P, P, C.c_size_t, P]
             L.tq_append_attend.restype = st
+            L.tq_prefill_workspace_bytes.argtypes = [P, i64, i64, i64]
+            L.tq_prefill_workspace_bytes.restype = C.c_size_t
+            L.tq_attend_prefill.argtypes = [P, P, i32, i64, i64, i64, C.POINTER(tq_cache), C.POINTER(tq_cache), i64,
+                                            C.c_float, P, P, C.c_size_t, P]
+            L.tq_attend_prefill.restype = st
             L.tq_device_status.argtypes = [P, P]
             L.tq_device_status.restype = st
             L.tq_set_decode_events.argtypes = [P, P, P]
@@ -267,6 +272,22 @@ def tq_append_attend(h, k_new, v_new, kc: Cache, vc: Cache, t0: int, q, out, ws,
                                   C.c_void_p(q.data_ptr()), _dtype_code(q), q.shape[1], float(scale),
                                   C.c_void_p(out.data_ptr()), C.c_void_p(ws.data_ptr()),
                                   ws.numel() * ws.element_size(), _stream(stream)), "tq_append_attend")
+
+
+def tq_prefill_workspace_bytes(h, B: int, Lq: int, Hq: int) -> int:
+    return int(lib().tq_prefill_workspace_bytes(h, B, Lq, Hq))
+
+
+def tq_attend_prefill(h, q, kc: Cache, vc: Cache, T0: int, out, ws, scale: float = 1.0, stream=None) -> None:
+    """Causal attention of a chunk of queries q [B, Lq, Hq, d] (query i over
+    tokens [0, T0 + i]) over the compressed caches; out fp32 [B, Lq, Hq, d]."""
+    if q.dim() != 4 or not q.is_contiguous():
+        raise ValueError("tq_attend_prefill: q must be contiguous [B, Lq, Hq, d]")
+    B, Lq, Hq, _ = q.shape
+    _check(lib().tq_attend_prefill(h, C.c_void_p(q.data_ptr()), _dtype_code(q), B, Lq, Hq, C.byref(kc.struct),
+                                   C.byref(vc.struct), T0, float(scale), C.c_void_p(out.data_ptr()),
+                                   C.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(), _stream(stream)),
+           "tq_attend_prefill")
 
 
 def tq_device_status(h, stream=None) -> int:

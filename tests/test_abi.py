@@ -86,6 +86,9 @@ def test_host_argument_errors(libtq):
     assert L.tq_append_attend(None, None, None, 0, 1, 0, 0, 0, None, None, 0, None, 0, 1, 1.0,
                               None, None, 0, None) == tq.TQ_ERR_INVALID_ARG
     assert L.tq_attend_workspace_bytes(None, 1, 1, 1, 64) == 0
+    assert L.tq_attend_prefill(None, None, 0, 1, 1, 1, C.byref(c), C.byref(c), 0, 1.0, None, None, 0,
+                               None) == tq.TQ_ERR_INVALID_ARG
+    assert L.tq_prefill_workspace_bytes(None, 1, 1, 1) == 0
     assert L.tq_destroy(None) == tq.TQ_OK
     assert L.tq_head_dim(None) == 0
     for s in range(6):
