@@ -259,6 +259,14 @@ void orc_sketch_given_codes(int d, const double* S, const double* c8, const doub
  * and bit 2 of code(24+k).
  * Signs are d/32 words per token: word 4s+t has sign(i = 2q) at bit q and
  * sign(i = 2q+1) at bit 16+q (q = 0..15), i mapping to a JL row as above.
+ * d = 64 has one 64-coordinate slice of 16 codes per slot (i = 0..15, same
+ * coordinate formula with s = 0).  Per token, word t (t = 0..3) holds code(k)
+ * in bits 0-2 of nibble k (k = 0..7); halfword t of bytes 16..23 (bits
+ * 16 (t & 1) .. of word 4 + t / 2) holds code(8 + k) in bits 0-2 of nibble k
+ * (k = 0..3); the three bits of code(12 + k) are bit 3 of nibble k of word t,
+ * bit 3 of nibble 4 + k of word t and bit 3 of nibble k of halfword t.  Its
+ * signs are 4 halfwords per token: bit i of halfword t (bits 16 (t & 1) + i
+ * of word t / 2) is the sign of the JL row of slot position i.
  * These functions pack/unpack one (b, kv-head) sequence of Tcap slots.
  * ---------------------------------------------------------------------- */
 int64_t orc_block_bytes(int d, int is_k) {
@@ -277,7 +285,52 @@ static void orc_put_bit(uint32_t* w, int pos, int bit) {
 }
 static int orc_get_bit(uint32_t w, int pos) { return (int)((w >> pos) & 1u); }
 
+/* d = 64: bit `bit` of halfword t of the code record (words 4, 5) */
+static int orc_h64_pos(int t, int bit) { return 16 * (t & 1) + bit; }
+
+static void orc_pack_codes64(const uint8_t* code, uint32_t* words) {
+    for (int w = 0; w < 6; ++w) words[w] = 0;
+    for (int t = 0; t < 4; ++t) {
+        uint32_t* H = &words[4 + t / 2];
+        for (int k = 0; k < 8; ++k) {
+            int c = code[orc_slot_coord(0, t, k)];
+            for (int b = 0; b < 3; ++b) orc_put_bit(&words[t], 4 * k + b, (c >> b) & 1);
+        }
+        for (int k = 0; k < 4; ++k) {
+            int c = code[orc_slot_coord(0, t, 8 + k)];
+            for (int b = 0; b < 3; ++b) orc_put_bit(H, orc_h64_pos(t, 4 * k + b), (c >> b) & 1);
+            int c4 = code[orc_slot_coord(0, t, 12 + k)];
+            orc_put_bit(&words[t], 4 * k + 3, c4 & 1);
+            orc_put_bit(&words[t], 4 * (4 + k) + 3, (c4 >> 1) & 1);
+            orc_put_bit(H, orc_h64_pos(t, 4 * k + 3), (c4 >> 2) & 1);
+        }
+    }
+}
+
+static void orc_unpack_codes64(const uint32_t* words, uint8_t* code) {
+    for (int t = 0; t < 4; ++t) {
+        const uint32_t H = words[4 + t / 2];
+        for (int k = 0; k < 8; ++k) {
+            int c = 0;
+            for (int b = 0; b < 3; ++b) c |= orc_get_bit(words[t], 4 * k + b) << b;
+            code[orc_slot_coord(0, t, k)] = (uint8_t)c;
+        }
+        for (int k = 0; k < 4; ++k) {
+            int c = 0;
+            for (int b = 0; b < 3; ++b) c |= orc_get_bit(H, orc_h64_pos(t, 4 * k + b)) << b;
+            code[orc_slot_coord(0, t, 8 + k)] = (uint8_t)c;
+            int c4 = orc_get_bit(words[t], 4 * k + 3) | (orc_get_bit(words[t], 4 * (4 + k) + 3) << 1) |
+                     (orc_get_bit(H, orc_h64_pos(t, 4 * k + 3)) << 2);
+            code[orc_slot_coord(0, t, 12 + k)] = (uint8_t)c4;
+        }
+    }
+}
+
 static void orc_pack_codes(int d, const uint8_t* code, uint32_t* words) {
+    if (d == 64) {
+        orc_pack_codes64(code, words);
+        return;
+    }
     for (int s = 0; s < d / 128; ++s)
         for (int t = 0; t < 4; ++t) {
             uint32_t* W = words + 12 * s + 3 * t;
@@ -294,6 +347,10 @@ static void orc_pack_codes(int d, const uint8_t* code, uint32_t* words) {
 }
 
 static void orc_unpack_codes(int d, const uint32_t* words, uint8_t* code) {
+    if (d == 64) {
+        orc_unpack_codes64(words, code);
+        return;
+    }
     for (int s = 0; s < d / 128; ++s)
         for (int t = 0; t < 4; ++t) {
             const uint32_t* W = words + 12 * s + 3 * t;
@@ -311,6 +368,12 @@ static void orc_unpack_codes(int d, const uint32_t* words, uint8_t* code) {
 }
 
 static void orc_pack_signs(int d, const uint8_t* sg, uint32_t* words) {
+    if (d == 64) {
+        words[0] = words[1] = 0;
+        for (int t = 0; t < 4; ++t)
+            for (int i = 0; i < 16; ++i) orc_put_bit(&words[t / 2], 16 * (t & 1) + i, sg[orc_slot_coord(0, t, i)]);
+        return;
+    }
     for (int s = 0; s < d / 128; ++s)
         for (int t = 0; t < 4; ++t) {
             uint32_t w = 0;
@@ -323,6 +386,12 @@ static void orc_pack_signs(int d, const uint8_t* sg, uint32_t* words) {
 }
 
 static void orc_unpack_signs(int d, const uint32_t* words, uint8_t* sg) {
+    if (d == 64) {
+        for (int t = 0; t < 4; ++t)
+            for (int i = 0; i < 16; ++i)
+                sg[orc_slot_coord(0, t, i)] = (uint8_t)orc_get_bit(words[t / 2], 16 * (t & 1) + i);
+        return;
+    }
     for (int s = 0; s < d / 128; ++s)
         for (int t = 0; t < 4; ++t)
             for (int q = 0; q < 16; ++q) {

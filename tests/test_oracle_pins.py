@@ -77,7 +77,7 @@ def test_lloyd_max_optimality_conditions():
         assert abs(num / den - c[k]) < 1e-9
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_codebook_scaled_fp16(golden, d):
     lv, th, _ = _levels_from_golden(golden)
     p = O.params(d, 0)
@@ -129,7 +129,7 @@ def _dense_HD(p):
     return (scipy.linalg.hadamard(d).astype(np.float64) / math.sqrt(d)) * p["D"].astype(np.float64)[None, :]
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_encode_steps_against_library_routines(d):
     p = O.params(d, 11)
     x = synthetic.gaussian((300, d), seed=d).astype(np.float64)
@@ -237,7 +237,7 @@ def test_polar_only_scores_shrink_qjl_scores_unbiased():
 
 # ---------------------------------------------------------------- layout
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_bits_per_dim_and_pack_roundtrip(golden, d):
     for cache, hd, bpd in golden("bits_per_dim.txt"):
         if int(hd) == d:
@@ -260,7 +260,7 @@ def test_bits_per_dim_and_pack_roundtrip(golden, d):
             assert np.array_equal(u["sig"], sig) and np.array_equal(u["gh"], gh)
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_layout_is_a_bijection(d):
     """Every (coordinate, code bit) and every sign lands on its own bit of the record."""
     seen = set()
@@ -301,7 +301,7 @@ def _random_cache(d, T, seed, gamma_zero=False):
     return kc, vc
 
 
-@pytest.mark.parametrize("d,T,G", [(128, 1, 1), (128, 7, 2), (128, 16, 4), (256, 9, 3)])
+@pytest.mark.parametrize("d,T,G", [(64, 5, 2), (128, 1, 1), (128, 7, 2), (128, 16, 4), (256, 9, 3)])
 def test_attend_bruteforce(d, T, G):
     """Per-token dequantisation in the original domain, explicit QJL term, library
     softmax, per-token inverse transforms -- against the oracle's rotated-domain
