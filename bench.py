@@ -37,7 +37,7 @@ from kv_cache_vector_14_b200 import synthetic  # noqa: E402
 
 METRIC = "decode-attn achieved HBM GB/s (% of B200 peak); KV encode Mvectors/s"
 UNIT = "GB/s"
-BYTES_PER_TOKEN_HEAD = {128: 68 + 50, 256: 132 + 98}      # packed K + V record per token per kv head
+BYTES_PER_TOKEN_HEAD = {64: 36 + 26, 128: 68 + 50, 256: 132 + 98}   # packed K + V record per token per kv head
 ENCODE_BYTES_PER_VECTOR = {("k", 128): 68, ("v", 128): 50}
 
 # DRAM traffic of the split-K kernel from one ncu capture, valid only while the
@@ -468,6 +468,74 @@ def measure_paged(h, dev, w, kc, vc, q, out_ref, ws, n_calls: int) -> dict:
             "output_equals_contiguous": same}
 
 
+def measure_d64(dev, world: int, dist, n_calls: int = 200) -> dict:
+    """head_dim 64 on the long-context shape (B=4, Hq=16/Hkv=8, T=102400,
+    bf16 K/V with outlier channels and log-normal norms): the bulk encode of
+    the whole cache (K then V, timed by events) and decode attention over it
+    (split-K kernel by events, and the whole call).  62 bytes of packed cache
+    per (token, kv head)."""
+    import torch
+    from kv_cache_vector_14_b200 import tq
+    base = synthetic.WORKLOADS["c4"]
+    w = synthetic.Workload("d64", "head_dim 64, long context: B=4, Hq=16/Hkv=8, T=102400",
+                           B=base.B, Hq=base.Hq, Hkv=base.Hkv, d=64, T=base.T, kv_dtype="bf16", q_dtype="bf16",
+                           lognormal_norms=True, seed=640, scale=0.125)
+    d, B, Hq, Hkv, T = w.d, w.B, w.Hq, w.Hkv, w.T
+    h = tq.tq_init(d, 0)
+    kc, vc = tq.Cache(d, True, B, Hkv, T), tq.Cache(d, False, B, Hkv, T)
+    xk = torch.from_numpy(synthetic.kv(w, "k")).to(dev).to(torch.bfloat16)
+    xv = torch.from_numpy(synthetic.kv(w, "v")).to(dev).to(torch.bfloat16)
+    ek = []
+    for i in range(8):
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        tq.tq_encode_k(h, xk, kc, 0)
+        e1.record()
+        tq.tq_encode_v(h, xv, vc, 0)
+        e2.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            ek.append((e0.elapsed_time(e1), e1.elapsed_time(e2)))
+    k_ms = statistics.median(a for a, _ in ek)
+    v_ms = statistics.median(b for _, b in ek)
+    del xk, xv
+    q = torch.from_numpy(synthetic.queries(w)).to(dev).to(torch.bfloat16)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    ws = torch.empty(tq.tq_attend_workspace_bytes(h, B, Hq, Hkv, T), dtype=torch.uint8, device=dev)
+    for _ in range(10):
+        tq.tq_attend_decode(h, q, kc, vc, out, ws, T=T, scale=w.scale)
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_calls)]
+    for a_, b_ in kev:
+        a_.record()
+        b_.record()
+    torch.cuda.synchronize()
+    for i in range(n_calls):
+        tq.tq_set_decode_events(h, kev[i][0], kev[i][1])
+        tq.tq_attend_decode(h, q, kc, vc, out, ws, T=T, scale=w.scale)
+    torch.cuda.synchronize()
+    tq.tq_set_decode_events(h, None, None)
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record()
+    for _ in range(n_calls):
+        tq.tq_attend_decode(h, q, kc, vc, out, ws, T=T, scale=w.scale)
+    c1.record()
+    torch.cuda.synchronize()
+    call_ms = c0.elapsed_time(c1) / n_calls
+    status = tq.tq_status_string(tq.tq_device_status(h))
+    path = tq.tq_attend_path(h, Hq, Hkv)
+    tq.tq_destroy(h)
+    nbytes = B * Hkv * T * BYTES_PER_TOKEN_HEAD[d]
+    nvec = B * Hkv * T
+    return {"workload": w.title + ", bf16 K/V with outlier channels and log-normal norms",
+            "decode_path": path, "kernel_ms": kern_ms, "call_ms": call_ms,
+            "achieved_gbs": world * nbytes / (max_over_ranks(kern_ms, dist, dev) * 1e-3) / 1e9,
+            "call_gbs": world * nbytes / (max_over_ranks(call_ms, dist, dev) * 1e-3) / 1e9,
+            "encode_k_ms": k_ms, "encode_v_ms": v_ms,
+            "encode_mvec_s": world * 2 * nvec / (max_over_ranks(k_ms + v_ms, dist, dev) * 1e-3) / 1e6,
+            "device_status": status}
+
+
 def measure_prefill(dev, world: int, dist, reps: int = 20, Lq: int = 512) -> dict:
     """Chunked prefill on the GQA workload's cache (B=1, Hq=32/Hkv=8, d=128,
     40960 tokens): the last Lq tokens' queries as one chunk, query i attending
@@ -531,6 +599,12 @@ def run_ours(args, rank: int, world: int, dist):
         pf = measure_prefill(dev, world, dist, reps=args.steps)
         if rank == 0:
             print(json.dumps({"prefill": pf}), flush=True)
+        return
+    if args.only == "d64":             # profiling aid: the head_dim 64 workload alone
+        tq.tq_destroy(h)
+        r = measure_d64(dev, world, dist, n_calls=args.steps)
+        if rank == 0:
+            print(json.dumps({"d64": r}), flush=True)
         return
     if args.only == "loop":            # profiling aid: the append-and-attend workload alone
         tq.tq_destroy(h)
@@ -657,6 +731,7 @@ def run_ours(args, rank: int, world: int, dist):
     enc = measure_encode(h, dev, world, dist)
     loop = measure_loop(dev, world, dist)
     prefill = measure_prefill(dev, world, dist)
+    d64 = measure_d64(dev, world, dist)
 
     peak, peak_kind = peaks()
     bf16_peak = bf16_peak_tflops()
@@ -702,6 +777,7 @@ def run_ours(args, rank: int, world: int, dist):
         "paged": {**paged, "frac": paged["achieved_gbs"] / peak},
         "prefill": {**prefill, "peak_tflops": bf16_peak, "frac": prefill["tflops"] / bf16_peak,
                     "peak_kind": "measured bf16 dense GEMM (burst); the kernel uses mma.sync fp16/int8"},
+        "d64": {**d64, "frac": d64["achieved_gbs"] / peak},
         "device_status": tq.tq_status_string(status),
     }
     print(json.dumps(line), flush=True)
@@ -715,10 +791,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["step", "encode", "loop", "prefill"], default=None,
+    ap.add_argument("--only", choices=["step", "encode", "loop", "prefill", "d64"], default=None,
                     help="run only the decode step (--steps steps), the encode-only workload (--steps "
-                         "passes), the append-and-attend workload (--steps graph replays) or the chunked "
-                         "prefill (--steps calls); for profiling")
+                         "passes), the append-and-attend workload (--steps graph replays), the chunked "
+                         "prefill (--steps calls) or the head_dim 64 workload (--steps decode calls); for "
+                         "profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

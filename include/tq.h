@@ -17,7 +17,7 @@
  *   Attention, section on the hybrid V2+V3 design: dequantisation is fused
  *     into the attention kernel, which reads the packed cache directly.
  *
- * Conventions.  d = head_dim (128 or 256); m = d JL rows; tokens per cache
+ * Conventions.  d = head_dim (64, 128 or 256); m = d JL rows; tokens per cache
  * block = 64.  All data buffers (inputs, caches, outputs, workspace) are
  * device memory owned by the caller; the library owns only the constants
  * created by tq_init.  Hot calls (encode, attend) allocate nothing, do not
@@ -82,8 +82,13 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
  * Wb: code(8 + k) and bit 1 of code(24 + k); Wc: code(16 + k) and bit 2 of
  * code(24 + k).  Signs are d/32 words per token; word 4s+t holds the sign of
  * JL row i = 2q at bit q and of row 2q+1 at bit 16+q (q = 0..15), rows mapped
- * to indices exactly as coordinates above.  A sign bit is 1 when the
- * projection is >= 0.  Storage: (3d + m + 32)/d bits/dim for K (4.25 at
+ * to indices exactly as coordinates above.  d = 64 is one slice of 16 codes
+ * per slot (i = 0..15, s = 0): word t (t = 0..3) holds code(k) in bits 0-2 of
+ * nibble k (k = 0..7); halfword t of bytes 16..23 holds code(8 + k) in bits
+ * 0-2 of nibble k (k = 0..3); bits 0, 1, 2 of code(12 + k) are bit 3 of
+ * nibble k of word t, of nibble 4 + k of word t and of nibble k of halfword t.
+ * Its signs are 4 halfwords per token: bit i of halfword t is the sign of the
+ * JL row of slot position i.  A sign bit is 1 when the projection is >= 0.  Storage: (3d + m + 32)/d bits/dim for K (4.25 at
  * d = 128) and (3d + 16)/d for V (3.125 at d = 128). */
 typedef struct {
     void* base;

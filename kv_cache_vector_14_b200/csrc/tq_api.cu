@@ -209,17 +209,17 @@ tq_status tq_params_host(int head_dim, uint64_t seed, int8_t* D, float* S, float
 }
 
 size_t tq_block_bytes(int head_dim, int is_k) {
-    if (head_dim != 128 && head_dim != 256) return 0;
+    if (!head_dim_ok(head_dim)) return 0;
     return (size_t)block_bytes(head_dim, is_k != 0);
 }
 
 size_t tq_cache_bytes(int head_dim, int is_k, int64_t B, int64_t Hkv, int64_t Tcap) {
-    if ((head_dim != 128 && head_dim != 256) || B < 0 || Hkv < 0 || Tcap <= 0 || Tcap % kBlockT) return 0;
+    if (!head_dim_ok(head_dim) || B < 0 || Hkv < 0 || Tcap <= 0 || Tcap % kBlockT) return 0;
     return (size_t)(B * Hkv * (Tcap / kBlockT)) * (size_t)block_bytes(head_dim, is_k != 0);
 }
 
 tq_status tq_init(int head_dim, uint64_t seed, tq_handle** out) {
-    if (!out || (head_dim != 128 && head_dim != 256)) return TQ_ERR_INVALID_ARG;
+    if (!out || !head_dim_ok(head_dim)) return TQ_ERR_INVALID_ARG;
     *out = nullptr;
     tq_handle* h = new (std::nothrow) tq_handle();
     if (!h) return TQ_ERR_CUDA;
@@ -249,7 +249,7 @@ tq_status tq_init(int head_dim, uint64_t seed, tq_handle** out) {
     for (int j = 0; j < d; ++j)
         for (int r = 0; r < R; ++r)
             for (int l = 0; l < 32; ++l) {
-                const int row = slot_coord(r / 4, r % 4, 2 * (l & 15) + (l >> 4));
+                const int row = sign_row(d, r, l);
                 sthr[((size_t)j * R + r) * 32 + l] = h->hS[(size_t)row * d + j];
             }
     // d = 128: the JL matrix as the B operand of the tensor-core encode, rows

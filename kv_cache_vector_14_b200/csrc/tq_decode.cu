@@ -117,16 +117,27 @@ __global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t B
 // j = l + 32 r.  Partial scores are reduced across the warp, the online
 // softmax runs in log2 units, and the four warps are merged through shared
 // memory into one partial per query head.
+template <int D>
 __device__ __forceinline__ int code_from_words(const uint32_t* w, int j) {
     const int s = j >> 7, t = slot_of(j), i = slot_pos(j);
+    if constexpr (D == 64) {             // word t: codes 0..7; halfword t (words 4, 5): codes 8..11
+        const uint32_t H = w[4 + (t >> 1)] >> (16 * (t & 1));
+        if (i < 8) return (int)((w[t] >> (4 * i)) & 7u);
+        if (i < 12) return (int)((H >> (4 * (i - 8))) & 7u);
+        const int k = i - 12;
+        return (int)(((w[t] >> (4 * k + 3)) & 1u) | (((w[t] >> (4 * k + 19)) & 1u) << 1) |
+                     (((H >> (4 * k + 3)) & 1u) << 2));
+    }
     const uint32_t* W = w + 12 * s + 3 * t;
     if (i < 24) return (int)((W[i >> 3] >> (4 * (i & 7))) & 7u);
     const int k = i - 24;
     return (int)(((W[0] >> (4 * k + 3)) & 1u) | (((W[1] >> (4 * k + 3)) & 1u) << 1) |
                  (((W[2] >> (4 * k + 3)) & 1u) << 2));
 }
+template <int D>
 __device__ __forceinline__ int sign_from_words(const uint32_t* w, int j) {
     const int s = j >> 7, t = slot_of(j), i = slot_pos(j);
+    if constexpr (D == 64) return (int)((w[t >> 1] >> (16 * (t & 1) + i)) & 1u);
     const int bit = (i & 1) ? 16 + (i >> 1) : (i >> 1);
     return (int)((w[4 * s + t] >> bit) & 1u);
 }
@@ -188,10 +199,10 @@ __global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const int j = lane + 32 * r;
-            const float ck = sC[code_from_words(kw, j)];
-            cv[r] = sC[code_from_words(vw, j)];
+            const float ck = sC[code_from_words<D>(kw, j)];
+            cv[r] = sC[code_from_words<D>(vw, j)];
             if constexpr (QJL) {
-                const float sg = sign_from_words(sw, j) ? gk : -gk;
+                const float sg = sign_from_words<D>(sw, j) ? gk : -gk;
 #pragma unroll
                 for (int g = 0; g < G; ++g) part[g] = fmaf(q[g][r], ck, fmaf(u[g][r], sg, part[g]));
             } else {
@@ -351,6 +362,7 @@ cudaError_t launch_simt_g(int G, const DecArgs& a, cudaStream_t s) {
 
 cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, const float* dsign, const float* st,
                             float* qp, float* up, bool pdl, cudaStream_t s) {
+    if (d == 64) return launch_prologue_d<64>(q, dt, BHq, dsign, st, qp, up, pdl, s);
     if (d == 128) return launch_prologue_d<128>(q, dt, BHq, dsign, st, qp, up, pdl, s);
     if (d == 256) return launch_prologue_d<256>(q, dt, BHq, dsign, st, qp, up, pdl, s);
     return cudaErrorInvalidValue;
@@ -358,6 +370,7 @@ cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, cons
 
 cudaError_t launch_decode_simt(int d, int G, bool qjl, const DecArgs& a, cudaStream_t s) {
     if (a.B * a.Hkv == 0) return cudaSuccess;
+    if (d == 64) return qjl ? launch_simt_g<64, true>(G, a, s) : launch_simt_g<64, false>(G, a, s);
     if (d == 128) return qjl ? launch_simt_g<128, true>(G, a, s) : launch_simt_g<128, false>(G, a, s);
     if (d == 256) return qjl ? launch_simt_g<256, true>(G, a, s) : launch_simt_g<256, false>(G, a, s);
     return cudaErrorInvalidValue;
@@ -366,6 +379,8 @@ cudaError_t launch_decode_simt(int d, int G, bool qjl, const DecArgs& a, cudaStr
 cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml, const float* part_acc,
                            const float* dsign, float* out, cudaStream_t s) {
     if (BHq == 0) return cudaSuccess;
+    if (d == 64)
+        return launch_pdl(tq_combine_kernel<64>, dim3((unsigned)BHq), dim3(64), 0, s, part_ml, part_acc, nsplit, dsign, out);
     if (d == 128)
         return launch_pdl(tq_combine_kernel<128>, dim3((unsigned)BHq), dim3(128), 0, s, part_ml, part_acc, nsplit, dsign, out);
     if (d == 256)
@@ -382,9 +397,9 @@ cudaError_t launch_decode_mma(int d, int G, bool qjl, const DecArgs& a, cudaStre
 int decode_mma_chunk_tokens(int d);
 int decode_mma_warps(int G);
 
-// The tensor-core kernel covers head_dim 128 and 256 with up to 8 query heads
-// per kv head; other group sizes take the SIMT kernel.
-bool mma_supported(int d, int G) { return (d == 128 || d == 256) && G >= 1 && G <= 8; }
+// The tensor-core kernel covers head_dim 64, 128 and 256 with up to 8 query
+// heads per kv head; other group sizes take the SIMT kernel.
+bool mma_supported(int d, int G) { return head_dim_ok(d) && G >= 1 && G <= 8; }
 
 int decode_ctas_per_sm(bool use_mma) { return use_mma ? 1 : 4; }
 int decode_chunk_tokens(int d, bool use_mma) { return use_mma ? decode_mma_chunk_tokens(d) : kBlockT; }

@@ -1,5 +1,5 @@
 // Tensor-core split-K decode attention over the packed TurboQuant cache
-// (head_dim 128 or 256, up to 8 query heads per kv head), for sm_100a.
+// (head_dim 64, 128 or 256, up to 8 query heads per kv head), for sm_100a.
 //
 // Page "Apple Silicon向けSwiftLM、TurboQuant KVキャッシュ圧縮とSSD Expert
 // Streamingを実装" (ai-heartland.com), hybrid V2+V3 section: dequantisation is
@@ -35,7 +35,9 @@
 // head_dim 256 is two 128-coordinate slices of the same record layout: the
 // k-loop runs over 16 coordinate chunks and 8 sign blocks, the value tile
 // over 16 coordinate tiles.  Its q'/u' fragments are read from shared memory
-// (filled once per CTA) instead of being held in registers.
+// (filled once per CTA) instead of being held in registers.  head_dim 64 is
+// half a slice: 16 codes and 16 signs per slot (4 k-steps, 2 sign blocks),
+// its sign halfword widened so that the same shifts pick its bits.
 #include <type_traits>
 
 #include "tq_frag.cuh"
@@ -182,6 +184,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     if constexpr (QJL) {
         auto row_of = [&](int kb, int half, int e) {
             const int bit = 8 * e + 7 - 2 * (kb & 3) - half;
+            if constexpr (D == 64) return slot_coord(0, tq4, e < 2 ? bit : bit - 20);   // h | h << 20
             return slot_coord(kb >> 2, tq4, bit < 16 ? 2 * bit : 2 * (bit - 16) + 1);
         };
 #pragma unroll
@@ -230,6 +233,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     if constexpr (!C::kBRegs) __syncthreads();
     const uint32_t lut[4] = {a.cb.lut_lo[0], a.cb.lut_lo[1], a.cb.lut_hi[0], a.cb.lut_hi[1]};
     const uint32_t* pw = a.cb.pow2;
+    [[maybe_unused]] const uint32_t m64 = pw[20] | 1u;    // d = 64 sign widening factor
 
     float o[NT][kKC][4];
 #pragma unroll
@@ -269,11 +273,11 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
             [[maybe_unused]] uint32_t sgA[C::kS], sgB[C::kS];
 #pragma unroll
             for (int sl = 0; sl < C::kS; ++sl) {
-                code_selectors(st + C::kOffKc + tA * C::kCodeB + sl * 48 + tq4 * 12, pw, selA[sl]);
-                code_selectors(st + C::kOffKc + tB * C::kCodeB + sl * 48 + tq4 * 12, pw, selB[sl]);
+                token_selectors<D>(st + C::kOffKc + tA * C::kCodeB, sl, tq4, pw, selA[sl]);
+                token_selectors<D>(st + C::kOffKc + tB * C::kCodeB, sl, tq4, pw, selB[sl]);
                 if constexpr (QJL) {
-                    sgA[sl] = *reinterpret_cast<const uint32_t*>(st + C::kOffKs + tA * C::kSignB + sl * 16 + tq4 * 4);
-                    sgB[sl] = *reinterpret_cast<const uint32_t*>(st + C::kOffKs + tB * C::kSignB + sl * 16 + tq4 * 4);
+                    sgA[sl] = token_signs<D>(st + C::kOffKs + tA * C::kSignB, sl, tq4, m64);
+                    sgB[sl] = token_signs<D>(st + C::kOffKs + tB * C::kSignB, sl, tq4, m64);
                 }
             }
             float acc[NT][4];
@@ -377,8 +381,8 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
             // ---------------- values: O^T += Vdeq^T P
 #pragma unroll
             for (int sl = 0; sl < C::kS; ++sl) {
-                code_selectors(st + C::kOffVc + tA * C::kCodeB + sl * 48 + tq4 * 12, pw, selA[sl]);
-                code_selectors(st + C::kOffVc + tB * C::kCodeB + sl * 48 + tq4 * 12, pw, selB[sl]);
+                token_selectors<D>(st + C::kOffVc + tA * C::kCodeB, sl, tq4, pw, selA[sl]);
+                token_selectors<D>(st + C::kOffVc + tB * C::kCodeB, sl, tq4, pw, selB[sl]);
             }
 #pragma unroll
             for (int kc = 0; kc < kKC; ++kc) {
@@ -478,18 +482,22 @@ cudaError_t launch_mma_t(const DecArgs& a, int G, cudaStream_t s) {
 
 template <bool QJL>
 cudaError_t launch_mma_q(int d, int G, const DecArgs& a, cudaStream_t s) {
+    if (d == 64)
+        return G <= 4 ? launch_mma_t<64, 1, kNW1, QJL>(a, G, s) : launch_mma_t<64, 2, kNW2, QJL>(a, G, s);
     if (d == 128)
         return G <= 4 ? launch_mma_t<128, 1, kNW1, QJL>(a, G, s) : launch_mma_t<128, 2, kNW2, QJL>(a, G, s);
     return G <= 4 ? launch_mma_t<256, 1, kNW1, QJL>(a, G, s) : launch_mma_t<256, 2, kNW2, QJL>(a, G, s);
 }
 
 cudaError_t launch_decode_mma(int d, int G, bool qjl, const DecArgs& a, cudaStream_t s) {
-    if ((d != 128 && d != 256) || G < 1 || G > 8) return cudaErrorInvalidValue;
+    if (!head_dim_ok(d) || G < 1 || G > 8) return cudaErrorInvalidValue;
     if (a.B * a.Hkv == 0) return cudaSuccess;
     return qjl ? launch_mma_q<true>(d, G, a, s) : launch_mma_q<false>(d, G, a, s);
 }
 
-int decode_mma_chunk_tokens(int d) { return d == 128 ? Cfg<128>::kChunk : Cfg<256>::kChunk; }
+int decode_mma_chunk_tokens(int d) {
+    return d == 64 ? Cfg<64>::kChunk : d == 128 ? Cfg<128>::kChunk : Cfg<256>::kChunk;
+}
 int decode_mma_warps(int G) { return G <= 4 ? kNW1 : kNW2; }
 
 }  // namespace tqi

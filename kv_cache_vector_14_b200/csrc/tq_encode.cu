@@ -5,7 +5,8 @@
 // 1-bit QJL = 4.25 bits/dim" (steps 1-5) and section "V-Cache圧縮：3-bit
 // PolarQuant = 3.125 bits/dim" (steps 1-3, no QJL).
 //
-// One CTA of 8 warps handles tiles of 32 vectors (4 per warp):
+// Head dims 64 and 256 (head_dim 128 runs on the tensor-core kernels of
+// tq_encode_tc.cu).  One CTA of 8 warps handles tiles of 32 vectors (4 per warp):
 //   phase 1, one warp per vector: coalesced load, ||x|| by warp reduction,
 //     sign flip + Walsh-Hadamard butterflies (register stages for the lane's
 //     own coordinates j = lane + 32 r, shuffle stages across lanes), scale by
@@ -45,6 +46,41 @@ __device__ __forceinline__ uint32_t nibbles8(uint32_t lo4, uint32_t hi4) {
     uint32_t b = (hi4 | (hi4 >> 4)) & 0x00FF00FFu;
     b = (b | (b >> 8)) & 0x0000FFFFu;
     return a | (b << 16);
+}
+
+// Shared-memory index of coordinate j's staged code: slots of 32 positions
+// per 128-coordinate slice (16 positions per slot at d = 64).
+template <int D>
+__device__ __forceinline__ int stage_at(int j) {
+    if constexpr (D == 64) return slot_of(j) * 16 + slot_pos(j);
+    else return (j >> 7) * 128 + slot_of(j) * 32 + slot_pos(j);
+}
+
+// Code word w (0 .. 3D/32 - 1) of one token, from its codes staged in slot
+// order (one byte per code).
+template <int D>
+__device__ __forceinline__ uint32_t code_word(const uint8_t* sc, int w) {
+    if constexpr (D == 64) {
+        if (w < 4) {                      // word t: codes 0..7 of slot t, bits 0 and 1 of codes 12..15
+            const uint32_t* sw = reinterpret_cast<const uint32_t*>(sc + 16 * w);
+            const uint32_t tl = nibbles8(sw[3], 0u);
+            return nibbles8(sw[0], sw[1]) | ((tl & 0x1111u) << 3) | (((tl >> 1) & 0x1111u) << 19);
+        }
+        uint32_t r = 0;                   // halfwords of slots 2(w-4), 2(w-4)+1: codes 8..11, bit 2 of 12..15
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t* sw = reinterpret_cast<const uint32_t*>(sc + 16 * (2 * (w - 4) + hh));
+            const uint32_t half = nibbles8(sw[2], 0u) | (((nibbles8(sw[3], 0u) >> 2) & 0x1111u) << 3);
+            r |= half << (16 * hh);
+        }
+        return r;
+    } else {
+        const int s = w / 12, t = (w % 12) / 3, g = w % 3;
+        const uint32_t* sw = reinterpret_cast<const uint32_t*>(sc + s * 128 + t * 32);
+        const uint32_t main = nibbles8(sw[2 * g], sw[2 * g + 1]);
+        const uint32_t tail = nibbles8(sw[6], sw[7]);
+        return main | (((tail >> g) & 0x11111111u) << 3);
+    }
 }
 
 template <int D, bool IS_K, int TV>
@@ -158,7 +194,7 @@ __global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
                 const float res = (n > 0.f) ? (y - sC[code]) : 0.f;
                 g2[vv] = fmaf(res, res, g2[vv]);
                 if constexpr (IS_K) sR[v * D + j] = res;
-                sCode[v * D + (j >> 7) * 128 + slot_of(j) * 32 + slot_pos(j)] = (uint8_t)code;
+                sCode[v * D + stage_at<D>(j)] = (uint8_t)code;
             }
         }
         if constexpr (IS_K) {
@@ -245,12 +281,7 @@ __global__ void __launch_bounds__(kThreads) tq_encode_kernel(const EncArgs a) {
             const int v = warp * kVecPerWarp + vv;
             const int64_t gv = tile * kTileV + v;
             if (gv < N && lane < W) {
-                const int s = lane / 12, t = (lane % 12) / 3, g = lane % 3;
-                const uint8_t* slot = sCode + v * D + s * 128 + t * 32;
-                const uint32_t* sw = reinterpret_cast<const uint32_t*>(slot);
-                const uint32_t main = nibbles8(sw[2 * g], sw[2 * g + 1]);
-                const uint32_t tail = nibbles8(sw[6], sw[7]);
-                const uint32_t word = main | (((tail >> g) & 0x11111111u) << 3);
+                const uint32_t word = code_word<D>(sCode + v * D, lane);
                 const int64_t tt = gv % a.Tnew, bh = gv / a.Tnew, tok = a.t0 + tt;
                 const int64_t pb = cache_block(a.table, a.pool, a.NB, bh, tok >> 6, a.err);
                 if (pb >= 0) reinterpret_cast<uint32_t*>(a.cache + pb * bb + (tok & 63) * code_bytes(D))[lane] = word;
@@ -342,7 +373,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(con
         const float res = (n > 0.f) ? (y - sC[code]) : 0.f;
         g2 = fmaf(res, res, g2);
         sr[warp][j] = res;
-        scode[warp][(j >> 7) * 128 + slot_of(j) * 32 + slot_pos(j)] = (uint8_t)code;
+        scode[warp][stage_at<D>(j)] = (uint8_t)code;
     }
     g2 = warp_sum(g2);
     const bool writer = wr && blockIdx.y == 0;
@@ -374,13 +405,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(con
     if (wr && lane < RG)
         reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(D) + (t & 63) * sign_bytes(D))[rg0 + lane] = mine;
     constexpr int W = 3 * D / 32;
-    if (wr && blockIdx.y == 0 && lane < W) {
-        const int sl = lane / 12, st = (lane % 12) / 3, g = lane % 3;
-        const uint32_t* sw = reinterpret_cast<const uint32_t*>(&scode[warp][sl * 128 + st * 32]);
-        const uint32_t main = nibbles8(sw[2 * g], sw[2 * g + 1]);
-        const uint32_t tail = nibbles8(sw[6], sw[7]);
-        reinterpret_cast<uint32_t*>(blk + (t & 63) * code_bytes(D))[lane] = main | (((tail >> g) & 0x11111111u) << 3);
-    }
+    if (wr && blockIdx.y == 0 && lane < W)
+        reinterpret_cast<uint32_t*>(blk + (t & 63) * code_bytes(D))[lane] = code_word<D>(scode[warp], lane);
     pdl_wait();
 }
 
@@ -435,6 +461,8 @@ cudaError_t launch_enc_dt(tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, 
 
 cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
     if (d == 128) return launch_encode128(is_k, dt, a, num_sms, pdl, s);
+    if (d == 64)
+        return is_k ? launch_enc_dt<64, true>(dt, a, num_sms, pdl, s) : launch_enc_dt<64, false>(dt, a, num_sms, pdl, s);
     if (d == 256)
         return is_k ? launch_enc_dt<256, true>(dt, a, num_sms, pdl, s) : launch_enc_dt<256, false>(dt, a, num_sms, pdl, s);
     return cudaErrorInvalidValue;

@@ -19,11 +19,11 @@ constexpr int kWaitLimit = 1 << 20;
 // PolarQuant-only cache in the V layout (codes and norms, no signs, no gamma).
 template <int D, bool QJL = true>
 struct Cfg {
-    static constexpr int kS = D / 128;                        // 128-coordinate slices
+    static constexpr int kS = D >= 128 ? D / 128 : 1;         // 128-coordinate slices (d = 64: one half slice)
     static constexpr int kKC = D / 16;                        // coordinate chunks (mma k-steps)
     static constexpr int kCodeB = 3 * D / 8;                  // code bytes per token
     static constexpr int kSignB = D / 8;                      // sign bytes per token (QJL)
-    static constexpr int kChunk = D == 128 ? 32 : 16;         // tokens per stage
+    static constexpr int kChunk = D <= 128 ? 32 : 16;         // tokens per stage
     static constexpr int kTiles = kChunk / 16;
     static constexpr int kOffKc = 0;
     static constexpr int kOffKs = kOffKc + kChunk * kCodeB;
@@ -32,7 +32,7 @@ struct Cfg {
     static constexpr int kOffVc = kOffKg + (QJL ? 2 * kChunk : 0);
     static constexpr int kOffVn = kOffVc + kChunk * kCodeB;
     static constexpr int kStageB = kOffVn + 2 * kChunk;
-    static constexpr bool kBRegs = D == 128;                   // q'/u' fragments in registers
+    static constexpr bool kBRegs = D <= 128;                   // q'/u' fragments in registers
     static_assert(kStageB % 16 == 0 && kOffKn % 16 == 0 && kOffKg % 16 == 0 && kOffVc % 16 == 0 &&
                       kOffVn % 16 == 0,
                   "stage fields must keep 16-byte alignment");
@@ -143,6 +143,35 @@ __device__ __forceinline__ void dequant4(uint32_t sel16, const uint32_t (&lut)[4
 
 __device__ __forceinline__ uint32_t sel_for(const uint32_t (&sel)[4], const uint32_t* pw, int kc) {
     return (kc & 1) ? shr_m(sel[kc >> 1], pw, 16) : sel[kc >> 1];
+}
+
+// Selector words of slot t of slice sl of one token record (tok), in the
+// sel_for order.  d = 64 (16 codes per slot): word t gives positions 0..7
+// (sel[0]); halfword t gives positions 8..11 and, with the bit-3 planes of
+// both, positions 12..15 (sel[1]).
+template <int D>
+__device__ __forceinline__ void token_selectors(const uint8_t* tok, int sl, int t, const uint32_t* pw,
+                                                uint32_t (&sel)[4]) {
+    if constexpr (D == 64) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(tok + 4 * t);
+        const uint32_t h = *reinterpret_cast<const uint16_t*>(tok + 16 + 2 * t);
+        sel[0] = w & 0x77777777u;
+        const uint32_t plane = (shr_m(w, pw, 3) & 0x1111u) | (shr_m(w, pw, 18) & 0x2222u) | (shr_m(h, pw, 1) & 0x4444u);
+        sel[1] = (h & 0x7777u) | shl_m(plane, pw, 16);
+        sel[2] = sel[3] = 0u;
+    } else {
+        code_selectors(tok + sl * 48 + t * 12, pw, sel);
+    }
+}
+
+// Sign word of slot t of slice sl of one token's sign record.  d = 64: the
+// 16-bit halfword h of slot t as h | h << 20 (m64 = 2^20 + 1), so that byte e
+// of the word has h's bits 4e' .. 4e'+3 in its bits 4..7 (e' = 1, 3, 0, 2 for
+// e = 0..3) and the shifts of the d >= 128 extraction pick every bit once.
+template <int D>
+__device__ __forceinline__ uint32_t token_signs(const uint8_t* tok, int sl, int t, uint32_t m64) {
+    if constexpr (D == 64) return (uint32_t)*reinterpret_cast<const uint16_t*>(tok + 2 * t) * m64;
+    else return *reinterpret_cast<const uint32_t*>(tok + sl * 16 + t * 4);
 }
 
 }  // namespace

@@ -40,7 +40,8 @@ __host__ __device__ inline int64_t block_bytes(int d, bool is_k) {
 }
 
 // Slot order of coordinate j inside a token record: slot t (0..3) of slice
-// j >> 7 owns 32 coordinates; position i inside the slot.
+// j >> 7 owns 32 coordinates (16 at d = 64, one slice); position i inside the
+// slot.
 __host__ __device__ inline int slot_of(int j) { return (j >> 1) & 3; }
 __host__ __device__ inline int slot_pos(int j) {
     int jj = j & 127;
@@ -66,6 +67,15 @@ __host__ __device__ inline int qjl_row_of_column(int n) {
     const int b = n & 31;
     return slot_coord(0, n >> 5, b < 16 ? 2 * b : 2 * (b - 16) + 1);
 }
+// JL row whose sign is bit l of stored sign word r.  d >= 128: word 4s+t is
+// slot t of slice s, bit q -> position 2q, bit 16+q -> position 2q+1.  d = 64:
+// word r holds the 16-bit sign halfwords of slots 2r (bits 0-15) and 2r+1,
+// bit i of a halfword -> position i.
+__host__ __device__ inline int sign_row(int d, int r, int l) {
+    if (d == 64) return slot_coord(0, 2 * r + (l >> 4), l & 15);
+    return slot_coord(r >> 2, r & 3, l < 16 ? 2 * l : 2 * (l - 16) + 1);
+}
+__host__ __device__ inline bool head_dim_ok(int d) { return d == 64 || d == 128 || d == 256; }
 
 // Division by a fixed divisor d >= 1 for dividends below 2^31:
 // q = umulhi(n, m) >> s with m = ceil(2^(31 + ceil(log2 d)) / d); m = 0 marks d = 1.

@@ -88,7 +88,7 @@ double half_bits_to_double(uint16_t h) {
 }
 
 bool make_params(int d, uint64_t seed, int8_t* D, float* S, float* c8, float* b7) {
-    if (d != 128 && d != 256) return false;
+    if (!head_dim_ok(d)) return false;
     if (D)
         for (int j = 0; j < d; ++j) D[j] = (splitmix_draw(seed, (uint64_t)j) & (1ull << 63)) ? -1 : 1;
     if (S) {

@@ -191,7 +191,7 @@ class Cache:
         else:
             nbytes = tq_cache_bytes(head_dim, is_k, B, Hkv, Tcap)
         if nbytes == 0 and B * Hkv > 0:
-            raise ValueError("Tcap must be a positive multiple of 64 and head_dim 128 or 256")
+            raise ValueError("Tcap must be a positive multiple of 64 and head_dim 64, 128 or 256")
         self.head_dim, self.is_k, self.B, self.Hkv, self.Tcap = head_dim, is_k, B, Hkv, Tcap
         self.block_table, self.pool_blocks = block_table, pool_blocks
         self.buf = buf if buf is not None else torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=device)

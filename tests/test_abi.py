@@ -25,7 +25,7 @@ def test_exports_every_declared_symbol(libtq):
         assert hasattr(libtq, n), n
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("seed", [0, 1, 12345, 2**63 + 7])
 def test_params_host_bit_identical_to_oracle(libtq, d, seed):
     p = tq.tq_params_host(d, seed)
@@ -41,16 +41,16 @@ def test_sizes_and_bits_per_dim(libtq, golden):
         is_k = cache == "K"
         assert tq.tq_block_bytes(int(hd), is_k) == O.block_bytes(int(hd), is_k)
         assert 8 * tq.tq_cache_bytes(int(hd), is_k, 3, 5, 640) / (3 * 5 * 640 * int(hd)) == float(bpd)
-    for d in (128, 256):
+    for d in (64, 128, 256):
         for is_k in (True, False):
             assert tq.tq_block_bytes(d, is_k) == O.block_bytes(d, is_k)
             assert tq.tq_block_bytes(d, is_k) % 16 == 0
-    assert tq.tq_block_bytes(64, True) == 0
+    assert tq.tq_block_bytes(32, True) == 0 and tq.tq_block_bytes(512, False) == 0
     assert tq.tq_cache_bytes(128, True, 1, 1, 100) == 0      # Tcap not a multiple of 64
     assert tq.tq_cache_bytes(128, True, 1, 1, 0) == 0
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_codebook_is_exactly_antisymmetric(libtq, d):
     """The encode kernels find the cell and the centroid from |y| alone; that
     needs c[7-k] = -c[k], b[6-k] = -b[k] and b[3] = 0 exactly in fp32, and exact
@@ -72,9 +72,10 @@ def test_cache_struct_layout():
 
 
 def test_host_argument_errors(libtq):
-    with pytest.raises(tq.TQError) as e:
-        tq.tq_params_host(64, 0)
-    assert e.value.status == tq.TQ_ERR_INVALID_ARG
+    for bad_d in (32, 96, 512):
+        with pytest.raises(tq.TQError) as e:
+            tq.tq_params_host(bad_d, 0)
+        assert e.value.status == tq.TQ_ERR_INVALID_ARG
     L = libtq
     c = tq.tq_cache(None, 1, 1, 64)
     import ctypes as C

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 def handles(libtq):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    hs = {d: tq.tq_init(d, 0) for d in (128, 256)}
+    hs = {d: tq.tq_init(d, 0) for d in (64, 128, 256)}
     yield hs
     torch.cuda.synchronize()
     for h in hs.values():
@@ -38,7 +38,7 @@ def decode_path(request, handles):
 
 @pytest.fixture(scope="module")
 def prms():
-    return {d: O.params(d, 0) for d in (128, 256)}
+    return {d: O.params(d, 0) for d in (64, 128, 256)}
 
 
 def _flat(u: dict) -> dict:
@@ -49,7 +49,7 @@ def _x64(x: np.ndarray) -> np.ndarray:
     return x.astype(np.float64).reshape(-1, x.shape[-1])
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_params_on_device(handles, d):
     p, hp = tq.tq_get_params(handles[d]), tq.tq_params_host(d, 0)
     for k in ("D", "S", "c8", "b7"):
@@ -89,7 +89,7 @@ def test_encode_d256_sampled(handles, prms):
     print(check_encode(prms[256], _x64(xs), _flat(gk), _flat(gv)))
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 def test_encode_ragged_offsets_strides(handles, prms, d, dtype):
     B, Hkv, T, t0, Tcap = 2, 3, 77, 50, 192
@@ -125,7 +125,7 @@ def test_encode_zero_and_special_vectors(handles, prms):
     print(check_encode(prms[d], _x64(x), gk, gv))
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_append_one_token_at_a_time_equals_bulk(handles, d):
     """Bulk encodes (over 4 vectors per SM: the tiled kernel) and one-token
     appends (the small-batch kernel) write identical bytes."""
@@ -283,7 +283,7 @@ def _gather_blocks(cache: tq.Cache, table: torch.Tensor) -> torch.Tensor:
     return pool.index_select(0, table.flatten().long()).flatten()
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_paged_cache_matches_contiguous(handles, prms, d):
     """Paged caches (blocks scattered over a pool by a random table) hold the
     same bytes per logical block as contiguous caches after bulk encodes and
@@ -350,7 +350,7 @@ def test_paged_cache_bad_table_entry_is_a_device_check(handles):
     assert torch.isfinite(out).all()
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("G,T0,Tnew", [(2, 0, 1), (4, 63, 1), (1, 64, 3), (8, 200, 2), (4, 1000, 1)])
 def test_fused_append_attend_equals_separate_calls(handles, d, G, T0, Tnew):
     """tq_append_attend writes the same cache bytes and outputs, bit for bit, as
@@ -387,7 +387,7 @@ def test_fused_append_attend_equals_separate_calls(handles, d, G, T0, Tnew):
     assert tq.tq_device_status(h) == tq.TQ_OK
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("fused", [False, True])
 def test_append_and_attend_graph_replay_equals_eager(handles, d, fused):
     """The append-and-attend step sequence (separate calls, or the fused
@@ -436,7 +436,7 @@ def test_append_and_attend_graph_replay_equals_eager(handles, d, fused):
     del g
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_attend_group_sizes_and_ragged_lengths(decode_path, handles, prms, d, G):
     Hkv, B, Tcap = 2, 3, 320
@@ -453,7 +453,7 @@ def test_attend_group_sizes_and_ragged_lengths(decode_path, handles, prms, d, G)
     assert err.max() <= ATT_TOL
 
 
-@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_attend_polar_only_k(decode_path, handles, prms, d, G):
     """PolarQuant-only K (a V-layout K cache from tq_encode_v): the kernels'
@@ -481,6 +481,19 @@ def test_attend_polar_only_k(decode_path, handles, prms, d, G):
     print("polar-only K max rel err", err.max())
     assert err.max() <= ATT_TOL
     assert tq.tq_device_status(h) == tq.TQ_OK
+
+
+def test_attend_d64_many_splits(decode_path, handles, prms):
+    """head_dim 64 over 20000 tokens (many splits and chunks, a ragged tail) with
+    outlier channels and log-normal norms: every output row against the
+    oracle, both decode kernels."""
+    w = synthetic.Workload("t", "d64", B=2, Hq=16, Hkv=4, d=64, T=20000, kv_dtype="bf16", q_dtype="bf16",
+                           lognormal_norms=True, seed=64, scale=0.125)
+    out, ref, err = _attend_case(handles[64], prms[64], w, synthetic.kv(w, "k"), synthetic.kv(w, "v"),
+                                 synthetic.queries(w), w.T, 20032)
+    print("d64 max rel err", err.max(), "path", tq.tq_attend_path(handles[64], w.Hq, w.Hkv), decode_path)
+    assert err.max() <= ATT_TOL
+    assert tq.tq_device_status(handles[64]) == tq.TQ_OK
 
 
 @pytest.mark.parametrize("qdt", ["f32", "bf16", "f16"])
