@@ -41,7 +41,8 @@ BYTES_PER_TOKEN_HEAD = {64: 36 + 26, 128: 68 + 50, 256: 132 + 98}   # packed K +
 ENCODE_BYTES_PER_VECTOR = {("k", 128): 68, ("v", 128): 50}
 
 # DRAM traffic of the split-K kernel from one ncu capture, valid only while the
-# kernel source is unchanged (sha256 of csrc/tq_decode_mma.cu at capture time).
+# kernel source is unchanged (sha256 over csrc/tq_decode_mma.cu, csrc/tq_frag.cuh
+# and csrc/tq_internal.h at capture time).
 NCU_TRAFFIC = {"source_sha256": "31c9db5f08a8daeafe93be7d0032b7e17a1b65bf2304b55d178f7ca209d8b8a3",
                "bytes_per_launch": 390108160,
                "capture": "profiles/tq_decode_mma_d128_long_context_b4_hq16_hkv8_t102400.md"}
@@ -65,9 +66,16 @@ def bf16_peak_tflops() -> float:
         return 1590.0
 
 
-def source_sha(rel: str) -> str:
-    with open(os.path.join(ROOT, rel), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+DECODE_SOURCES = ("kv_cache_vector_14_b200/csrc/tq_decode_mma.cu", "kv_cache_vector_14_b200/csrc/tq_frag.cuh",
+                  "kv_cache_vector_14_b200/csrc/tq_internal.h")
+
+
+def source_sha(rels) -> str:
+    h = hashlib.sha256()
+    for rel in rels:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 class ClockSampler:
@@ -736,8 +744,8 @@ def run_ours(args, rank: int, world: int, dist):
     peak, peak_kind = peaks()
     bf16_peak = bf16_peak_tflops()
     achieved = bytes_step / (kern_ms * 1e-3) / 1e9
-    traffic = NCU_TRAFFIC["bytes_per_launch"] if (path == "mma" and NCU_TRAFFIC["source_sha256"] == source_sha(
-        "kv_cache_vector_14_b200/csrc/tq_decode_mma.cu")) else None
+    traffic = NCU_TRAFFIC["bytes_per_launch"] if (path == "mma" and
+                                                  NCU_TRAFFIC["source_sha256"] == source_sha(DECODE_SOURCES)) else None
 
     cpu = None
     enc_cpu = None
