@@ -172,8 +172,10 @@ TQ_API size_t tq_attend_workspace_bytes(const tq_handle* h, int64_t B, int64_t H
  *   out = D H sum_t softmax(s)_t * nv_t * c[idxv_t],
  * with n_t, gamma_t, nv_t the stored fp16 values, in fp32 with split-K
  * (flash-decoding) partials in `ws` merged by a final kernel.  out is fp32
- * [B][Hq][d]; an empty sequence gives zeros.  Supported: d in {128, 256},
- * Hq/Hkv in {1, 2, 4, 8}.  ws must be 256-byte aligned with at least
+ * [B][Hq][d]; an empty sequence gives zeros.  Supported: d in {64, 128, 256},
+ * any Hq/Hkv (kv heads with more than 8 query heads are served in groups of
+ * up to 8), B <= 65535, Hkv * ceil(Hq/Hkv / 8) <= 65535.  ws must be 256-byte
+ * aligned with at least
  * tq_attend_workspace_bytes(h, B, Hq, Hkv, T or max seq_len) bytes.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 TQ_API tq_status tq_attend_decode(const tq_handle* h, const void* q, tq_dtype qdtype, int64_t B,
@@ -212,9 +214,9 @@ TQ_API size_t tq_prefill_workspace_bytes(const tq_handle* h, int64_t B, int64_t 
  * hybrid V2+V3 section, with the QJL term evaluated on 16-bit fixed-point u');
  * out is fp32 [B][Lq][Hq][d].  With many queries per kv head the score and
  * value contractions are dense and run on tensor cores with the keys
- * dequantised once per 16 query rows.  Supported: d = 128, Hq/Hkv in
- * {1, 2, 4, 8}, T0 + Lq <= Tcap; contiguous or paged caches.
- * Errors: INVALID_ARG, UNSUPPORTED (d != 128, group size), WORKSPACE, CUDA. */
+ * dequantised once per 16 query rows.  Supported: d = 128, any Hq/Hkv,
+ * B <= 65535, T0 + Lq <= Tcap; contiguous or paged caches.
+ * Errors: INVALID_ARG, UNSUPPORTED (d != 128, grid limits), WORKSPACE, CUDA. */
 TQ_API tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype qdtype, int64_t B, int64_t Lq,
                                    int64_t Hq, const tq_cache* kc, const tq_cache* vc, int64_t T0, float scale,
                                    float* out, void* ws, size_t ws_bytes, void* stream);

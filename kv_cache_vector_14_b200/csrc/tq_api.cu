@@ -69,7 +69,7 @@ bool make_plan(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t T
     const int d = h->d;
     p->G = (int)(Hq / Hkv);
     p->use_mma = !h->force_simt && mma_supported(d, p->G);
-    const int64_t pairs = B * Hkv > 0 ? B * Hkv : 1;
+    const int64_t pairs = B * Hkv > 0 ? B * Hkv * decode_head_groups(p->use_mma, p->G) : 1;
     const int64_t cap = (int64_t)h->num_sms * decode_ctas_per_sm(p->use_mma);
     const int chunk = decode_chunk_tokens(d, p->use_mma);
     const int64_t nchunk = Tmax > 0 ? (Tmax + chunk - 1) / chunk : 1;
@@ -136,8 +136,9 @@ tq_status prepare_attend(const tq_handle* h, const void* q, tq_dtype qdt, int64_
         return TQ_ERR_INVALID_ARG;
     const int64_t Hkv = kc->Hkv;
     if (Hq % Hkv) return TQ_ERR_INVALID_ARG;
-    const int G = (int)(Hq / Hkv);
-    if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_ERR_UNSUPPORTED;
+    const int64_t G = Hq / Hkv;
+    // grid limits: y = kv heads x query-head groups, z = batch
+    if (B > 65535 || Hkv * ((G + 7) / 8) > 65535) return TQ_ERR_UNSUPPORTED;
     if (!seq_lens && (T < 0 || T > kc->Tcap)) return TQ_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
     if (B == 0) return TQ_OK;
@@ -346,7 +347,7 @@ tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype qdt, int
     const int64_t Hkv = kc->Hkv;
     if (Hq % Hkv) return TQ_ERR_INVALID_ARG;
     const int G = (int)(Hq / Hkv);
-    if (G != 1 && G != 2 && G != 4 && G != 8) return TQ_ERR_UNSUPPORTED;
+    if (B > 65535 || Hkv > 65535) return TQ_ERR_UNSUPPORTED;          // grid limits
     if (h->d != 128) return TQ_ERR_UNSUPPORTED;
     if (B == 0 || Lq == 0) return TQ_OK;
     if (!q || !out || !ws || !aligned(q, dtype_size(qdt)) || !aligned(out, 16) || !aligned(ws, 256))

@@ -111,8 +111,12 @@ __global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t B
     pdl_wait();          // chained after an encode (fused step): complete only after it
 }
 
+// Query heads per SIMT CTA: G itself for 1, 2 and 4, else groups of up to 8.
+int simt_heads_per_cta(int G) { return G <= 2 ? G : (G <= 4 ? 4 : 8); }
+
 // ---------------------------------------------------------------- SIMT decode
-// One CTA (4 warps) per (split, kv head, batch).  Each warp walks a quarter of
+// One CTA (4 warps) per (split, kv head, batch) and group of up to GT of the
+// kv head's G query heads (grid.y = Hkv x head groups).  Each warp walks a quarter of
 // the split's token range one token at a time; lane l owns coordinates
 // j = l + 32 r.  Partial scores are reduced across the warp, the online
 // softmax runs in log2 units, and the four warps are merged through shared
@@ -142,14 +146,20 @@ __device__ __forceinline__ int sign_from_words(const uint32_t* w, int j) {
     return (int)((w[4 * s + t] >> bit) & 1u);
 }
 
-template <int D, int G, bool QJL>
-__global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
+template <int D, int GT, bool QJL>
+__global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a, int Gq) {
     constexpr int R = D / 32;
+    constexpr int G = GT;                                  // query heads per CTA (slots; Gl of them live)
     __shared__ float sC[8];
     __shared__ float sm[4][G][2];
     __shared__ float sacc[4][G][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int split = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
+    const int split = blockIdx.x, b = blockIdx.z;
+    const int hgroups = (Gq + GT - 1) / GT;
+    const int hkv = blockIdx.y / hgroups;
+    const int g0 = (blockIdx.y - hkv * hgroups) * GT;
+    const int Gl = Gq - g0 < GT ? Gq - g0 : GT;
+    const int64_t hbase = (int64_t)b * a.Hq + (int64_t)hkv * Gq + g0;
     if (threadIdx.x < 8) sC[threadIdx.x] = a.cb.c[threadIdx.x];
 
     int64_t Tb = a.seq_lens ? (int64_t)a.seq_lens[b] : a.T;
@@ -168,11 +178,11 @@ __global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
     float q[G][R], u[G][R], acc[G][R], mrun[G], lrun[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        const int64_t bh = (int64_t)b * a.Hq + (int64_t)hkv * G + g;
+        const int64_t bh = hbase + (g < Gl ? g : 0);
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            q[g][r] = a.qp[bh * D + lane + 32 * r];
-            u[g][r] = a.up[bh * D + lane + 32 * r];
+            q[g][r] = g < Gl ? a.qp[bh * D + lane + 32 * r] : 0.f;
+            u[g][r] = g < Gl ? a.up[bh * D + lane + 32 * r] : 0.f;
             acc[g][r] = 0.f;
         }
         mrun[g] = -INFINITY;
@@ -232,7 +242,7 @@ __global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
         for (int r = 0; r < R; ++r) sacc[warp][g][lane + 32 * r] = acc[g][r];
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * D; idx += 128) {
+    for (int idx = threadIdx.x; idx < Gl * D; idx += 128) {
         const int g = idx / D, j = idx % D;
         float M = -INFINITY;
 #pragma unroll
@@ -246,7 +256,7 @@ __global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a) {
                 A = fmaf(f, sacc[w][g][j], A);
             }
         }
-        const int64_t bh = (int64_t)b * a.Hq + (int64_t)hkv * G + g;
+        const int64_t bh = hbase + g;
         const int64_t pidx = bh * a.nsplit + split;
         a.part_acc[pidx * D + j] = A;
         if (j == 0) { a.part_ml[2 * pidx] = M; a.part_ml[2 * pidx + 1] = L; }
@@ -341,19 +351,19 @@ cudaError_t launch_prologue_d(const void* q, tq_dtype dt, int64_t BHq, const flo
     return cudaErrorInvalidValue;
 }
 
-template <int D, int G, bool QJL>
-cudaError_t launch_simt(const DecArgs& a, cudaStream_t s) {
-    dim3 grid(a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
-    return launch_pdl(tq_decode_simt_kernel<D, G, QJL>, grid, dim3(128), 0, s, a);
+template <int D, int GT, bool QJL>
+cudaError_t launch_simt(int G, const DecArgs& a, cudaStream_t s) {
+    dim3 grid(a.nsplit, (unsigned)(a.Hkv * ((G + GT - 1) / GT)), (unsigned)a.B);
+    return launch_pdl(tq_decode_simt_kernel<D, GT, QJL>, grid, dim3(128), 0, s, a, G);
 }
 
 template <int D, bool QJL>
 cudaError_t launch_simt_g(int G, const DecArgs& a, cudaStream_t s) {
-    switch (G) {
-        case 1: return launch_simt<D, 1, QJL>(a, s);
-        case 2: return launch_simt<D, 2, QJL>(a, s);
-        case 4: return launch_simt<D, 4, QJL>(a, s);
-        case 8: return launch_simt<D, 8, QJL>(a, s);
+    switch (simt_heads_per_cta(G)) {
+        case 1: return launch_simt<D, 1, QJL>(G, a, s);
+        case 2: return launch_simt<D, 2, QJL>(G, a, s);
+        case 4: return launch_simt<D, 4, QJL>(G, a, s);
+        case 8: return launch_simt<D, 8, QJL>(G, a, s);
     }
     return cudaErrorInvalidValue;
 }
@@ -397,9 +407,15 @@ cudaError_t launch_decode_mma(int d, int G, bool qjl, const DecArgs& a, cudaStre
 int decode_mma_chunk_tokens(int d);
 int decode_mma_warps(int G);
 
-// The tensor-core kernel covers head_dim 64, 128 and 256 with up to 8 query
-// heads per kv head; other group sizes take the SIMT kernel.
-bool mma_supported(int d, int G) { return head_dim_ok(d) && G >= 1 && G <= 8; }
+// The tensor-core kernel covers head_dim 64, 128 and 256 and any group size
+// (query heads in CTAs of up to 8 per kv head).
+bool mma_supported(int d, int G) { return head_dim_ok(d) && G >= 1; }
+
+// CTAs per (split, kv head, batch): query-head groups of the kernel that runs.
+int decode_head_groups(bool use_mma, int G) {
+    const int per = use_mma ? 8 : simt_heads_per_cta(G);
+    return (G + per - 1) / per;
+}
 
 int decode_ctas_per_sm(bool use_mma) { return use_mma ? 1 : 4; }
 int decode_chunk_tokens(int d, bool use_mma) { return use_mma ? decode_mma_chunk_tokens(d) : kBlockT; }

@@ -53,7 +53,9 @@ namespace {
 //   values  O^T[16 coords][8] += Vdeq^T[16 coords][16 tok] * P[16 tok][8] (D/16 coordinate tiles)
 // Lane (g, t) = (lane / 4, lane % 4) dequantises tokens g and g + 8 of each
 // 16-token tile; its score columns are head t (hi, lo), so its softmax state
-// and output rows belong to head t (and head 4 + t when NT = 2).
+// and output rows belong to head t (and head 4 + t when NT = 2).  A kv head
+// with more than 8 query heads is served by ceil(G / 8) CTAs (grid.y = Hkv x
+// head groups), each taking up to 8 of its query heads.
 template <int D, int NT, int NW, bool QJL>
 __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs a, int G) {
     using C = Cfg<D, QJL>;
@@ -65,7 +67,12 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gr = lane >> 2, tq4 = lane & 3;
     uint8_t* ring = smem + (size_t)warp * kStages * C::kStageB;
-    const int split = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
+    const int split = blockIdx.x, b = blockIdx.z;
+    const int hgroups = (G + 7) >> 3;
+    const int hkv = blockIdx.y / hgroups;
+    const int g0 = (blockIdx.y - hkv * hgroups) * 8;          // first query head of this CTA's group
+    const int Gl = G - g0 < 8 ? G - g0 : 8;                    // query heads in the group
+    const int64_t hbase = (int64_t)b * a.Hq + (int64_t)hkv * G + g0;
 
     int64_t Tb = a.seq_lens ? (int64_t)a.seq_lens[b] : a.T;
     Tb = Tb < 0 ? 0 : (Tb > a.Tcap ? a.Tcap : Tb);
@@ -144,8 +151,8 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     auto b_frag = [&](const float* base, int nt, int kc, uint32_t& r0, uint32_t& r1) {
         const int hcol = 4 * nt + (gr >> 1);
         float x[4] = {0.f, 0.f, 0.f, 0.f};
-        if (hcol < G) {
-            const float* p = base + ((int64_t)b * a.Hq + (int64_t)hkv * G + hcol) * D + 16 * kc + 2 * tq4;
+        if (hcol < Gl) {
+            const float* p = base + (hbase + hcol) * D + 16 * kc + 2 * tq4;
             x[0] = p[0]; x[1] = p[1]; x[2] = p[8]; x[3] = p[9];
         }
         uint32_t h0, l0, h1, l1;
@@ -190,8 +197,8 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int hcol = 4 * nt + (gr >> 1);
-            const bool live = hcol < G;
-            const float* up = a.up + ((int64_t)b * a.Hq + (int64_t)hkv * G + (live ? hcol : 0)) * D;
+            const bool live = hcol < Gl;
+            const float* up = a.up + (hbase + (live ? hcol : 0)) * D;
             float um = 0.f;
 #pragma unroll
             for (int kb = 0; kb < kKB; ++kb)
@@ -245,7 +252,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     for (int nt = 0; nt < NT; ++nt) {
         mrun[nt] = -INFINITY;
         lrun[nt] = 0.f;
-        live[nt] = (4 * nt + tq4 < G) ? 1.f : 0.f;   // this lane's head exists
+        live[nt] = (4 * nt + tq4 < Gl) ? 1.f : 0.f;   // this lane's head exists
     }
     bool failed = false;
 
@@ -420,11 +427,11 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     pdl_trigger();                        // the combine kernel may start launching
     // ---------------- merge the warps of the CTA into one partial per head
     __syncwarp();
-    float* wbuf = reinterpret_cast<float*>(ring);             // [G][D + 2], in this warp's own ring
+    float* wbuf = reinterpret_cast<float*>(ring);             // [Gl][D + 2], in this warp's own ring
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         const int h = 4 * nt + tq4;
-        if (h < G) {
+        if (h < Gl) {
 #pragma unroll
             for (int mt = 0; mt < kKC; ++mt) {
                 wbuf[h * (D + 2) + 16 * mt + gr] = o[nt][mt][0] + o[nt][mt][1];
@@ -437,7 +444,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < G * D; idx += NW * 32) {
+    for (int idx = threadIdx.x; idx < Gl * D; idx += NW * 32) {
         const int g = idx / D, j = idx % D;
         float M = -INFINITY;
 #pragma unroll
@@ -453,7 +460,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                 A = fmaf(f, wb[j], A);
             }
         }
-        const int64_t bh = (int64_t)b * a.Hq + (int64_t)hkv * G + g;
+        const int64_t bh = hbase + g;
         const int64_t pidx = bh * a.nsplit + split;
         a.part_acc[pidx * D + j] = A;
         if (j == 0) {
@@ -476,7 +483,7 @@ cudaError_t launch_mma_t(const DecArgs& a, int G, cudaStream_t s) {
     auto kern = tq_decode_mma_kernel<D, NT, NW, QJL>;
     cudaError_t e = set_smem_once<tq_decode_mma_kernel<D, NT, NW, QJL>>((int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
+    dim3 grid(a.nsplit, (unsigned)(a.Hkv * ((G + 7) / 8)), (unsigned)a.B);
     return launch_pdl(kern, grid, dim3(NW * 32), smem, s, a, G);
 }
 
@@ -490,7 +497,7 @@ cudaError_t launch_mma_q(int d, int G, const DecArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_decode_mma(int d, int G, bool qjl, const DecArgs& a, cudaStream_t s) {
-    if (!head_dim_ok(d) || G < 1 || G > 8) return cudaErrorInvalidValue;
+    if (!head_dim_ok(d) || G < 1) return cudaErrorInvalidValue;
     if (a.B * a.Hkv == 0) return cudaSuccess;
     return qjl ? launch_mma_q<true>(d, G, a, s) : launch_mma_q<false>(d, G, a, s);
 }

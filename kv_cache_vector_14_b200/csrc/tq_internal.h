@@ -206,6 +206,7 @@ bool mma_supported(int d, int G);
 int decode_ctas_per_sm(bool use_mma);
 int decode_chunk_tokens(int d, bool use_mma);   // split ranges are multiples of this
 int decode_warps(bool use_mma, int G);   // warps sharing one split
+int decode_head_groups(bool use_mma, int G);   // CTAs per (split, kv head, batch)
 
 }  // namespace tqi
 

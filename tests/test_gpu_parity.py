@@ -216,7 +216,7 @@ def test_append_and_attend_loop_d256(handles, prms):
     assert torch.equal(kb.buf, kc.buf) and torch.equal(vb.buf, vc.buf)
 
 
-@pytest.mark.parametrize("G,T0,Lq", [(4, 0, 20), (2, 100, 37), (1, 64, 5), (8, 300, 17)])
+@pytest.mark.parametrize("G,T0,Lq", [(4, 0, 20), (2, 100, 37), (1, 64, 5), (8, 300, 17), (3, 70, 23), (16, 129, 9)])
 def test_attend_prefill_matches_oracle(handles, prms, G, T0, Lq):
     """Chunked prefill: query i of the chunk attends causally over tokens
     [0, T0 + i]; every query row equals the oracle's attention over T0 + i + 1
@@ -244,6 +244,38 @@ def test_attend_prefill_matches_oracle(handles, prms, G, T0, Lq):
         ref = oracle_attend(prms[d], qb[:, i], ku, vu, Hkv, [T0 + i + 1] * B, scale)
         worst = max(worst, float(rel_err_rows(got[:, i], ref).max()))
     print("prefill max rel err", worst)
+    assert worst <= ATT_TOL
+    assert tq.tq_device_status(h) == tq.TQ_OK
+
+
+def test_attend_prefill_bench_size_sampled_rows(handles, prms):
+    """The benchmark's prefill workload and launch configuration (c3's cache:
+    B=1, Hq=32/Hkv=8, d=128, 40960 tokens; the last 512 tokens' queries as one
+    chunk): sampled query rows of two kv heads (first, middle, last query of the
+    chunk) against the oracle's decode over T0 + i + 1 tokens, and every output
+    finite."""
+    w = synthetic.WORKLOADS["c3"]
+    d, B, Hq, Hkv, T = w.d, w.B, w.Hq, w.Hkv, w.T
+    G, Lq = Hq // Hkv, 512
+    T0 = T - Lq
+    h = handles[d]
+    kc, _ = encode_gpu(h, d, torch_input(synthetic.kv(w, "k"), w.kv_dtype), Tcap=T, which="k")
+    _, vc = encode_gpu(h, d, torch_input(synthetic.kv(w, "v"), w.kv_dtype), Tcap=T, which="v")
+    q = synthetic.bf16_round(synthetic.gaussian((B, Lq, Hq, d), seed=11))
+    ws = torch.empty(tq.tq_prefill_workspace_bytes(h, B, Lq, Hq), dtype=torch.uint8, device="cuda")
+    out = torch.full((B, Lq, Hq, d), float("nan"), dtype=torch.float32, device="cuda")
+    tq.tq_attend_prefill(h, torch_input(q, "bf16"), kc, vc, T0, out, ws, scale=w.scale)
+    got = out.cpu().numpy()
+    assert np.all(np.isfinite(got))
+    worst = 0.0
+    for hk in (0, Hkv - 1):
+        ku, vu = unpack_cache(kc, 0, T, [(0, hk)]), unpack_cache(vc, 0, T, [(0, hk)])
+        for i in (0, Lq // 2, Lq - 1):
+            kcs = {k: v[0, :T0 + i + 1] for k, v in ku.items()}
+            vcs = {k: v[0, :T0 + i + 1] for k, v in vu.items()}
+            ref = O.attend(prms[d], q[0, i, hk * G:(hk + 1) * G].astype(np.float64), kcs, vcs, w.scale)
+            worst = max(worst, float(rel_err_rows(got[0, i, hk * G:(hk + 1) * G], ref).max()))
+    print("prefill bench-size sampled max rel err", worst)
     assert worst <= ATT_TOL
     assert tq.tq_device_status(h) == tq.TQ_OK
 
@@ -351,7 +383,7 @@ def test_paged_cache_bad_table_entry_is_a_device_check(handles):
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
-@pytest.mark.parametrize("G,T0,Tnew", [(2, 0, 1), (4, 63, 1), (1, 64, 3), (8, 200, 2), (4, 1000, 1)])
+@pytest.mark.parametrize("G,T0,Tnew", [(2, 0, 1), (4, 63, 1), (1, 64, 3), (8, 200, 2), (4, 1000, 1), (16, 100, 1)])
 def test_fused_append_attend_equals_separate_calls(handles, d, G, T0, Tnew):
     """tq_append_attend writes the same cache bytes and outputs, bit for bit, as
     tq_encode_k + tq_encode_v + tq_attend_decode, over several steps, with the
@@ -437,7 +469,7 @@ def test_append_and_attend_graph_replay_equals_eager(handles, d, fused):
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
-@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("G", [1, 2, 3, 4, 6, 8, 16])
 def test_attend_group_sizes_and_ragged_lengths(decode_path, handles, prms, d, G):
     Hkv, B, Tcap = 2, 3, 320
     w = synthetic.Workload("t", "edge", B=B, Hq=Hkv * G, Hkv=Hkv, d=d, T=Tcap, kv_dtype="f32", q_dtype="f32",
@@ -454,7 +486,7 @@ def test_attend_group_sizes_and_ragged_lengths(decode_path, handles, prms, d, G)
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
-@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
 def test_attend_polar_only_k(decode_path, handles, prms, d, G):
     """PolarQuant-only K (a V-layout K cache from tq_encode_v): the kernels'
     attention equals the oracle's with gamma = 0 (no QJL term), ragged lengths."""
@@ -539,12 +571,11 @@ def test_group_heads_equal_separate_heads(decode_path, handles):
 def test_attend_argument_errors(handles):
     h = handles[128]
     kc, vc = tq.Cache(128, True, 1, 2, 64), tq.Cache(128, False, 1, 2, 64)
-    q = torch.zeros((1, 6, 128), device="cuda")
-    out = torch.empty((1, 6, 128), device="cuda")
+    out = torch.empty((1, 4, 128), device="cuda")
     ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
     with pytest.raises(tq.TQError) as e:
-        tq.tq_attend_decode(h, q, kc, vc, out, ws, T=10)           # G = 3
-    assert e.value.status == tq.TQ_ERR_UNSUPPORTED
+        tq.tq_attend_decode(h, torch.zeros((1, 5, 128), device="cuda"), kc, vc, out, ws, T=10)   # Hq % Hkv
+    assert e.value.status == tq.TQ_ERR_INVALID_ARG
     q = torch.zeros((1, 4, 128), device="cuda")
     with pytest.raises(tq.TQError) as e:
         tq.tq_attend_decode(h, q, kc, vc, out, ws[:16], T=10)
