@@ -43,8 +43,8 @@ ENCODE_BYTES_PER_VECTOR = {("k", 128): 68, ("v", 128): 50}
 # DRAM traffic of the split-K kernel from one ncu capture, valid only while the
 # kernel source is unchanged (sha256 over csrc/tq_decode_mma.cu, csrc/tq_frag.cuh
 # and csrc/tq_internal.h at capture time).
-NCU_TRAFFIC = {"source_sha256": "0fd6e7a95c8c92a59a819af72948f832749928439b7e4e90b04e41585af7c496",
-               "bytes_per_launch": 390292480,
+NCU_TRAFFIC = {"source_sha256": "aa1d01a010032ee36b51c3c2b94d25f6c58ce3f2dad4135b4ed7498207f10c61",
+               "bytes_per_launch": 390361344,
                "capture": "profiles/tq_decode_mma_d128_long_context_b4_hq16_hkv8_t102400.md"}
 
 
