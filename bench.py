@@ -544,16 +544,20 @@ def measure_d64(dev, world: int, dist, n_calls: int = 200) -> dict:
             "device_status": status}
 
 
-def measure_prefill(dev, world: int, dist, reps: int = 20, Lq: int = 512) -> dict:
-    """Chunked prefill on the GQA workload's cache (B=1, Hq=32/Hkv=8, d=128,
-    40960 tokens): the last Lq tokens' queries as one chunk, query i attending
+def measure_prefill(dev, world: int, dist, reps: int = 20, Lq: int = 512, d: int = 128) -> dict:
+    """Chunked prefill on the GQA workload's cache (B=1, Hq=32/Hkv=8, 40960
+    tokens; head_dim d, 128 as in the workload or 64 with the same data
+    recipe): the last Lq tokens' queries as one chunk, query i attending
     causally over tokens [0, T - Lq + i].  Timed per call (prologue, prefill
     kernel, combine).  Work: 3 contractions of d multiply-adds per (query row,
     visible token) pair: 6 d flops."""
+    import dataclasses
     import torch
     from kv_cache_vector_14_b200 import tq
     w = synthetic.WORKLOADS["c3"]
-    d, B, Hq, Hkv, T = w.d, w.B, w.Hq, w.Hkv, w.T
+    if d != w.d:
+        w = dataclasses.replace(w, d=d, scale=1.0 / math.sqrt(d))
+    B, Hq, Hkv, T = w.B, w.Hq, w.Hkv, w.T
     T0 = T - Lq
     h = tq.tq_init(d, 0)
     kc, vc = tq.Cache(d, True, B, Hkv, T), tq.Cache(d, False, B, Hkv, T)
@@ -580,7 +584,7 @@ def measure_prefill(dev, world: int, dist, reps: int = 20, Lq: int = 512) -> dic
     tq.tq_destroy(h)
     pairs = B * Hq * (Lq * T0 + Lq * (Lq + 1) // 2)
     flops = 6 * d * pairs
-    return {"workload": f"chunked prefill: B=1, Hq=32/Hkv=8, d=128, {Lq} queries after {T0} cached tokens",
+    return {"workload": f"chunked prefill: B=1, Hq=32/Hkv=8, d={d}, {Lq} queries after {T0} cached tokens",
             "ms_per_call": ms, "query_token_pairs": pairs, "algorithmic_flops": flops,
             "tflops": world * flops / (max_over_ranks(ms, dist, dev) * 1e-3) / 1e12,
             "device_status": status}
@@ -611,6 +615,7 @@ def run_ours(args, rank: int, world: int, dist):
     if args.only == "d64":             # profiling aid: the head_dim 64 workload alone
         tq.tq_destroy(h)
         r = measure_d64(dev, world, dist, n_calls=args.steps)
+        r["prefill"] = measure_prefill(dev, world, dist, reps=5, d=64)
         if rank == 0:
             print(json.dumps({"d64": r}), flush=True)
         return
@@ -739,6 +744,7 @@ def run_ours(args, rank: int, world: int, dist):
     enc = measure_encode(h, dev, world, dist)
     loop = measure_loop(dev, world, dist)
     prefill = measure_prefill(dev, world, dist)
+    prefill64 = measure_prefill(dev, world, dist, d=64)
     d64 = measure_d64(dev, world, dist)
 
     peak, peak_kind = peaks()
@@ -785,7 +791,8 @@ def run_ours(args, rank: int, world: int, dist):
         "paged": {**paged, "frac": paged["achieved_gbs"] / peak},
         "prefill": {**prefill, "peak_tflops": bf16_peak, "frac": prefill["tflops"] / bf16_peak,
                     "peak_kind": "measured bf16 dense GEMM (burst); the kernel uses mma.sync fp16/int8"},
-        "d64": {**d64, "frac": d64["achieved_gbs"] / peak},
+        "d64": {**d64, "frac": d64["achieved_gbs"] / peak,
+                "prefill": {**prefill64, "frac": prefill64["tflops"] / bf16_peak}},
         "device_status": tq.tq_status_string(status),
     }
     print(json.dumps(line), flush=True)

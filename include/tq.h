@@ -214,9 +214,9 @@ TQ_API size_t tq_prefill_workspace_bytes(const tq_handle* h, int64_t B, int64_t 
  * hybrid V2+V3 section, with the QJL term evaluated on 16-bit fixed-point u');
  * out is fp32 [B][Lq][Hq][d].  With many queries per kv head the score and
  * value contractions are dense and run on tensor cores with the keys
- * dequantised once per 16 query rows.  Supported: d = 128, any Hq/Hkv,
+ * dequantised once per 16 query rows.  Supported: d in {64, 128}, any Hq/Hkv,
  * B <= 65535, T0 + Lq <= Tcap; contiguous or paged caches.
- * Errors: INVALID_ARG, UNSUPPORTED (d != 128, grid limits), WORKSPACE, CUDA. */
+ * Errors: INVALID_ARG, UNSUPPORTED (d = 256, grid limits), WORKSPACE, CUDA. */
 TQ_API tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype qdtype, int64_t B, int64_t Lq,
                                    int64_t Hq, const tq_cache* kc, const tq_cache* vc, int64_t T0, float scale,
                                    float* out, void* ws, size_t ws_bytes, void* stream);

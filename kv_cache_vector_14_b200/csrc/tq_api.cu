@@ -348,7 +348,7 @@ tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype qdt, int
     if (Hq % Hkv) return TQ_ERR_INVALID_ARG;
     const int G = (int)(Hq / Hkv);
     if (B > 65535 || Hkv > 65535) return TQ_ERR_UNSUPPORTED;          // grid limits
-    if (h->d != 128) return TQ_ERR_UNSUPPORTED;
+    if (h->d != 64 && h->d != 128) return TQ_ERR_UNSUPPORTED;
     if (B == 0 || Lq == 0) return TQ_OK;
     if (!q || !out || !ws || !aligned(q, dtype_size(qdt)) || !aligned(out, 16) || !aligned(ws, 256))
         return TQ_ERR_INVALID_ARG;

@@ -1,5 +1,5 @@
-// Chunked-prefill attention over the packed TurboQuant cache (head_dim 128),
-// for sm_100a: a chunk of Lq new queries per sequence, query i attending
+// Chunked-prefill attention over the packed TurboQuant cache (head_dim 64 and
+// 128), for sm_100a: a chunk of Lq new queries per sequence, query i attending
 // causally over cache tokens [0, T0 + i] (the chunk's own K/V already
 // appended at T0 .. T0 + Lq - 1).
 //
@@ -33,20 +33,22 @@
 namespace tqi {
 namespace {
 
-constexpr int kPD = 128;
 constexpr int kPW = 4;                         // warps per CTA, 16 query rows each
 constexpr int kPRows = 16 * kPW;
 constexpr float kQfix = 32000.f;               // u' fixed-point scale
-using PC = Cfg<kPD, true>;
-constexpr int kPKC = kPD / 16;                 // 16-coordinate k-steps
-constexpr int kPKB = kPD / 32;                 // 32-row sign blocks
 
-// shared memory: per warp a ring of staged chunks, the fp16 q' fragments
-// [k-step][limb][lane] and the int8 u' fragments [block][limb][lane]
-constexpr size_t kPRing = (size_t)kPW * kStages * PC::kStageB;
-constexpr size_t kPQa = (size_t)kPW * kPKC * 2 * 32 * 16;
-constexpr size_t kPUa = (size_t)kPW * kPKB * 2 * 32 * 16;
-constexpr size_t kPSmem = kPRing + kPQa + kPUa + (size_t)kPW * kStages * 8;
+// Shared memory per CTA: per warp a ring of staged chunks, the fp16 q'
+// fragments [k-step][limb][lane] and the int8 u' fragments [block][limb][lane].
+template <int D>
+struct PShape {
+    using PC = Cfg<D, true>;
+    static constexpr int kKC = D / 16;         // 16-coordinate k-steps
+    static constexpr int kKB = D / 32;         // 32-row sign blocks
+    static constexpr size_t kRing = (size_t)kPW * kStages * PC::kStageB;
+    static constexpr size_t kQa = (size_t)kPW * kKC * 2 * 32 * 16;
+    static constexpr size_t kUa = (size_t)kPW * kKB * 2 * 32 * 16;
+    static constexpr size_t kSmem = kRing + kQa + kUa + (size_t)kPW * kStages * 8;
+};
 
 struct PrefillArgs {
     DecArgs a;          // caches, workspace, scale, partials (one split), check word
@@ -54,7 +56,12 @@ struct PrefillArgs {
     int G;              // query heads per kv head
 };
 
-__global__ void __launch_bounds__(kPW * 32) tq_prefill_mma128_kernel(const PrefillArgs pa) {
+template <int D>
+__global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillArgs pa) {
+    using PC = Cfg<D, true>;
+    constexpr int kPD = D;
+    constexpr int kPKC = PShape<D>::kKC, kPKB = PShape<D>::kKB;
+    constexpr size_t kPRing = PShape<D>::kRing, kPQa = PShape<D>::kQa, kPUa = PShape<D>::kUa;
     const DecArgs& a = pa.a;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -118,8 +125,10 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma128_kernel(const Prefi
     // coordinates 16 kc + 2t, +1; a1 = row g + 8, same; a2/a3 = coordinates +8, +9.
     // u' (m16n8k32): byte e of a0/a1 (a2/a3) in block kb is u_int of the JL row whose
     // sign sits at bit 8 e + 7 - 2 (kb % 4) (8 e + 6 - 2 (kb % 4)) of slot word tq4.
+    // (d = 64: the slot's sign halfword h is widened to h | h << 20, see token_signs)
     auto row_of = [&](int kb, int half, int e) {
         const int bit = 8 * e + 7 - 2 * (kb & 3) - half;
+        if constexpr (D == 64) return slot_coord(0, tq4, e < 2 ? bit : bit - 20);
         return slot_coord(kb >> 2, tq4, bit < 16 ? 2 * bit : 2 * (bit - 16) + 1);
     };
     float fS[2], uS[2];
@@ -184,6 +193,7 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma128_kernel(const Prefi
 
     const uint32_t lut[4] = {a.cb.lut_lo[0], a.cb.lut_lo[1], a.cb.lut_hi[0], a.cb.lut_hi[1]};
     const uint32_t* pw = a.cb.pow2;
+    [[maybe_unused]] const uint32_t m64 = pw[20] | 1u;    // d = 64 sign widening factor
     float o[2 * kPKC][4];                 // 16 coordinate n-tiles: rows g (0, 1), g + 8 (2, 3)
 #pragma unroll
     for (int nc = 0; nc < 2 * kPKC; ++nc) o[nc][0] = o[nc][1] = o[nc][2] = o[nc][3] = 0.f;
@@ -207,10 +217,10 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma128_kernel(const Prefi
             // ---------------- scores of 16 rows x 16 tokens (two n-tiles of 8)
             const int tA = kt * 16 + gr, tB = tA + 8;            // B-fragment tokens of n-tiles 0, 1
             uint32_t selA[4], selB[4];
-            code_selectors(st + PC::kOffKc + tA * PC::kCodeB + tq4 * 12, pw, selA);
-            code_selectors(st + PC::kOffKc + tB * PC::kCodeB + tq4 * 12, pw, selB);
-            const uint32_t sgA = *reinterpret_cast<const uint32_t*>(st + PC::kOffKs + tA * PC::kSignB + tq4 * 4);
-            const uint32_t sgB = *reinterpret_cast<const uint32_t*>(st + PC::kOffKs + tB * PC::kSignB + tq4 * 4);
+            token_selectors<D>(st + PC::kOffKc + tA * PC::kCodeB, 0, tq4, pw, selA);
+            token_selectors<D>(st + PC::kOffKc + tB * PC::kCodeB, 0, tq4, pw, selB);
+            const uint32_t sgA = token_signs<D>(st + PC::kOffKs + tA * PC::kSignB, 0, tq4, m64);
+            const uint32_t sgB = token_signs<D>(st + PC::kOffKs + tB * PC::kSignB, 0, tq4, m64);
             float sacc[2][4];
             int iacc[2][2][4];                                  // [n-tile][u' limb]
 #pragma unroll
@@ -298,8 +308,8 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma128_kernel(const Prefi
             split_hilo(pv[1][0], pv[1][1], pH[2], pL[2]);
             split_hilo(pv[1][2], pv[1][3], pH[3], pL[3]);
             // ---------------- values: O[16 rows][8 coords] += P Vdeq, Vdeq^T by movmatrix
-            code_selectors(st + PC::kOffVc + tA * PC::kCodeB + tq4 * 12, pw, selA);
-            code_selectors(st + PC::kOffVc + tB * PC::kCodeB + tq4 * 12, pw, selB);
+            token_selectors<D>(st + PC::kOffVc + tA * PC::kCodeB, 0, tq4, pw, selA);
+            token_selectors<D>(st + PC::kOffVc + tB * PC::kCodeB, 0, tq4, pw, selB);
 #pragma unroll
             for (int kc = 0; kc < kPKC; ++kc) {
                 uint32_t x0, x1, y0, y1;
@@ -337,17 +347,23 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma128_kernel(const Prefi
     }
 }
 
+template <int D>
+cudaError_t launch_prefill_d(int G, const DecArgs& a, int64_t Lq, int64_t T0, cudaStream_t s) {
+    constexpr size_t smem = PShape<D>::kSmem;
+    PrefillArgs pa{a, Lq, T0, G};
+    const int64_t tiles = (Lq * G + kPRows - 1) / kPRows;
+    cudaError_t e = set_smem_once<tq_prefill_mma_kernel<D>>((int)smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)tiles, (unsigned)a.Hkv, (unsigned)a.B);
+    return launch_pdl(tq_prefill_mma_kernel<D>, grid, dim3(kPW * 32), smem, s, pa);
+}
+
 }  // namespace
 
 cudaError_t launch_prefill(int d, int G, const DecArgs& a, int64_t Lq, int64_t T0, cudaStream_t s) {
-    if (d != kPD || G < 1) return cudaErrorInvalidValue;
+    if ((d != 64 && d != 128) || G < 1) return cudaErrorInvalidValue;
     if (a.B * a.Hkv == 0 || Lq == 0) return cudaSuccess;
-    PrefillArgs pa{a, Lq, T0, G};
-    const int64_t tiles = (Lq * G + kPRows - 1) / kPRows;
-    cudaError_t e = set_smem_once<tq_prefill_mma128_kernel>((int)kPSmem);
-    if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)tiles, (unsigned)a.Hkv, (unsigned)a.B);
-    return launch_pdl(tq_prefill_mma128_kernel, grid, dim3(kPW * 32), kPSmem, s, pa);
+    return d == 64 ? launch_prefill_d<64>(G, a, Lq, T0, s) : launch_prefill_d<128>(G, a, Lq, T0, s);
 }
 
 }  // namespace tqi

@@ -216,13 +216,14 @@ def test_append_and_attend_loop_d256(handles, prms):
     assert torch.equal(kb.buf, kc.buf) and torch.equal(vb.buf, vc.buf)
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("G,T0,Lq", [(4, 0, 20), (2, 100, 37), (1, 64, 5), (8, 300, 17), (3, 70, 23), (16, 129, 9)])
-def test_attend_prefill_matches_oracle(handles, prms, G, T0, Lq):
+def test_attend_prefill_matches_oracle(handles, prms, d, G, T0, Lq):
     """Chunked prefill: query i of the chunk attends causally over tokens
     [0, T0 + i]; every query row equals the oracle's attention over T0 + i + 1
     tokens within the tolerance (ragged row tiles, queries at the cache start,
     all group sizes)."""
-    d, h = 128, handles[128]
+    h = handles[d]
     B, Hkv = 2, 2
     Hq, T = Hkv * G, T0 + Lq
     Tcap = (T + 63) // 64 * 64
@@ -280,10 +281,11 @@ def test_attend_prefill_bench_size_sampled_rows(handles, prms):
     assert tq.tq_device_status(h) == tq.TQ_OK
 
 
-def test_attend_prefill_paged_equals_contiguous(handles):
+@pytest.mark.parametrize("d", [64, 128])
+def test_attend_prefill_paged_equals_contiguous(handles, d):
     """Prefill over paged caches (random block tables) gives the same output,
     bit for bit, as over contiguous caches holding the same blocks."""
-    d, h = 128, handles[128]
+    h = handles[d]
     B, Hkv, G, T0, Lq, Tcap = 2, 2, 4, 150, 40, 192
     Hq, NB = Hkv * G, Tcap // 64
     x = torch_input(synthetic.gaussian((2, B, Hkv, T0 + Lq, d), seed=91), "f32")
@@ -590,4 +592,10 @@ def test_attend_argument_errors(handles):
     with pytest.raises(tq.TQError) as e:
         tq.tq_encode_k(h, x, kc, t0=60)                            # past Tcap
     assert e.value.status == tq.TQ_ERR_INVALID_ARG
+    h2 = handles[256]                                              # prefill: head_dim 64 and 128 only
+    k2, v2 = tq.Cache(256, True, 1, 2, 64), tq.Cache(256, False, 1, 2, 64)
+    with pytest.raises(tq.TQError) as e:
+        tq.tq_attend_prefill(h2, torch.zeros((1, 3, 4, 256), device="cuda"), k2, v2, 0,
+                             torch.empty((1, 3, 4, 256), device="cuda"), ws)
+    assert e.value.status == tq.TQ_ERR_UNSUPPORTED
     assert tq.tq_device_status(h) == tq.TQ_OK
