@@ -142,6 +142,20 @@ def whole_job_rate(units_per_rank: float, seconds_local: float, world: int, dist
 
 # ----------------------------------------------------------------------------- CPU oracle (baseline)
 
+def host_cpu() -> dict:
+    """Model name and logical CPU count of the host the oracle runs on."""
+    name = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    name = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": name, "nproc": os.cpu_count()}
+
+
 def oracle_decode_rate(w, seconds: float, tokens: int | None = None):
     """Time the float64 oracle's decode attention on host cores over a bounded
     sample: the G query heads of kv head 0 of sequence 0, over its first
@@ -222,7 +236,7 @@ def run_reference(args, rank: int, world: int):
         "data": "synthetic",
         "config": {"workload": w.title, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.d, "T": w.T,
                    "l2": "n/a (host)"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", **host_cpu(),
                          "sample": f"per step: oracle attention of {G} query heads over {tok} tokens of one kv head"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -757,7 +771,7 @@ def run_ours(args, rank: int, world: int, dist):
     enc_cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample, _ = oracle_decode_rate(w, args.cpu_seconds)
-        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample, **host_cpu()}
         ev_, ecores, esample = oracle_encode_rate(synthetic.WORKLOADS["c2"], min(10.0, args.cpu_seconds))
         enc_cpu = {"value": ev_, "unit": "Mvectors/s", "cores": ecores, "kind": "oracle", "sample": esample}
 
