@@ -79,8 +79,9 @@ double orc_from_fp16(uint16_t h) {
 }
 
 /* ------------------------------------------------------------------------
- * Lloyd-Max quantiser for the standard normal [P4, "3-bit非線形Lloyd-Max符号帳";
- * "V3のLloyd-Max符号帳" in the hybrid V2+V3 section].  Lloyd's two optimality
+ * Lloyd-Max quantiser for the standard normal [P4, K-Cache section, step 3: the
+ * 3-bit non-linear Lloyd-Max codebook; the hybrid V2+V3 section: the codebook
+ * taken from V3].  Lloyd's two optimality
  * conditions are applied alternately: decision edges at midpoints of adjacent
  * levels; each level at the conditional mean of N(0,1) on its cell,
  * (phi(a) - phi(b)) / (Phi(b) - Phi(a)).  Iterates until the largest level
