@@ -174,7 +174,7 @@ TQ_API size_t tq_attend_workspace_bytes(const tq_handle* h, int64_t B, int64_t H
  * (flash-decoding) partials in `ws` merged by a final kernel.  out is fp32
  * [B][Hq][d]; an empty sequence gives zeros.  Supported: d in {64, 128, 256},
  * any Hq/Hkv (kv heads with more than 8 query heads are served in groups of
- * up to 8), B <= 65535, Hkv * ceil(Hq/Hkv / 8) <= 65535.  ws must be 256-byte
+ * up to 8), B <= 65535, Hkv * ceil(Hq/Hkv / 8) <= 65535, B * Hq < 2^31.  ws must be 256-byte
  * aligned with at least
  * tq_attend_workspace_bytes(h, B, Hq, Hkv, T or max seq_len) bytes.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */

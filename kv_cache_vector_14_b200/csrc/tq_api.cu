@@ -137,8 +137,8 @@ tq_status prepare_attend(const tq_handle* h, const void* q, tq_dtype qdt, int64_
     const int64_t Hkv = kc->Hkv;
     if (Hq % Hkv) return TQ_ERR_INVALID_ARG;
     const int64_t G = Hq / Hkv;
-    // grid limits: y = kv heads x query-head groups, z = batch
-    if (B > 65535 || Hkv * ((G + 7) / 8) > 65535) return TQ_ERR_UNSUPPORTED;
+    // grid limits: y = kv heads x query-head groups, z = batch; one combine CTA per query head
+    if (B > 65535 || Hkv * ((G + 7) / 8) > 65535 || B * Hq >= ((int64_t)1 << 31)) return TQ_ERR_UNSUPPORTED;
     if (!seq_lens && (T < 0 || T > kc->Tcap)) return TQ_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
     if (B == 0) return TQ_OK;
