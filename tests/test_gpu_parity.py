@@ -1,5 +1,6 @@
 """GPU parity: the CUDA library (through its C ABI) against the float64 oracle on
 the same seeded inputs, for the five workloads and their edge cases."""
+import dataclasses
 import math
 
 import numpy as np
@@ -249,14 +250,17 @@ def test_attend_prefill_matches_oracle(handles, prms, d, G, T0, Lq):
     assert tq.tq_device_status(h) == tq.TQ_OK
 
 
-def test_attend_prefill_bench_size_sampled_rows(handles, prms):
-    """The benchmark's prefill workload and launch configuration (c3's cache:
-    B=1, Hq=32/Hkv=8, d=128, 40960 tokens; the last 512 tokens' queries as one
-    chunk): sampled query rows of two kv heads (first, middle, last query of the
-    chunk) against the oracle's decode over T0 + i + 1 tokens, and every output
-    finite."""
+@pytest.mark.parametrize("d", [64, 128])
+def test_attend_prefill_bench_size_sampled_rows(handles, prms, d):
+    """The benchmark's prefill workloads and launch configuration (c3's cache:
+    B=1, Hq=32/Hkv=8, 40960 tokens, at d = 128 and with the same recipe at
+    d = 64; the last 512 tokens' queries as one chunk): sampled query rows of
+    two kv heads (first, middle, last query of the chunk) against the oracle's
+    decode over T0 + i + 1 tokens, and every output finite."""
     w = synthetic.WORKLOADS["c3"]
-    d, B, Hq, Hkv, T = w.d, w.B, w.Hq, w.Hkv, w.T
+    if d != w.d:
+        w = dataclasses.replace(w, d=d, scale=1.0 / math.sqrt(d))
+    B, Hq, Hkv, T = w.B, w.Hq, w.Hkv, w.T
     G, Lq = Hq // Hkv, 512
     T0 = T - Lq
     h = handles[d]
@@ -514,6 +518,31 @@ def test_attend_polar_only_k(decode_path, handles, prms, d, G):
     err = rel_err_rows(out.cpu().numpy(), ref)
     print("polar-only K max rel err", err.max())
     assert err.max() <= ATT_TOL
+    assert tq.tq_device_status(h) == tq.TQ_OK
+
+
+def test_attend_d64_bench_size_sampled(handles, prms):
+    """The benchmark's head_dim 64 workload in its launch configuration (B=4,
+    Hq=16/Hkv=8, T=102400, bf16 K/V with outliers and log-normal norms, bf16
+    queries): encode and decode on the GPU, two sampled sequences' outputs
+    against the oracle over all 102400 tokens, every output finite."""
+    w = synthetic.Workload("d64", "d64 bench", B=4, Hq=16, Hkv=8, d=64, T=102400, kv_dtype="bf16",
+                           q_dtype="bf16", lognormal_norms=True, seed=640, scale=0.125)
+    h, d = handles[64], 64
+    kc, _ = encode_gpu(h, d, torch_input(synthetic.kv(w, "k"), w.kv_dtype), Tcap=w.T, which="k")
+    _, vc = encode_gpu(h, d, torch_input(synthetic.kv(w, "v"), w.kv_dtype), Tcap=w.T, which="v")
+    q = synthetic.queries(w)
+    out = attend_gpu(h, torch_input(q, w.q_dtype), kc, vc, T=w.T, scale=w.scale).cpu().numpy()
+    assert np.all(np.isfinite(out))
+    G = w.Hq // w.Hkv
+    worst = 0.0
+    for b, hk in ((0, 0), (3, 7)):
+        ku, vu = unpack_cache(kc, 0, w.T, [(b, hk)]), unpack_cache(vc, 0, w.T, [(b, hk)])
+        ref = O.attend(prms[d], q[b, hk * G:(hk + 1) * G].astype(np.float64),
+                       {k: v[0] for k, v in ku.items()}, {k: v[0] for k, v in vu.items()}, w.scale)
+        worst = max(worst, float(rel_err_rows(out[b, hk * G:(hk + 1) * G], ref).max()))
+    print("d64 bench-size sampled max rel err", worst)
+    assert worst <= ATT_TOL
     assert tq.tq_device_status(h) == tq.TQ_OK
 
 
