@@ -37,14 +37,36 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every source to an object (in parallel, under _build/), then link."""
     if not force and not _stale():
         return LIB
+    from concurrent.futures import ThreadPoolExecutor
+    objdir = os.path.join(ROOT, "_build", f"obj{os.getpid()}")
+    os.makedirs(objdir, exist_ok=True)
+    compile_flags = [f for f in FLAGS if f not in ("-shared", "-cudart", "static")]
+    jobs = []
+    for src in sources():
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        jobs.append((obj, [NVCC, *compile_flags, "-c", "-o", obj, src]))
+
+    def run(job):
+        if verbose:
+            print(" ".join(job[1]), flush=True)
+        subprocess.check_call(job[1])
+        return job[0]
+
+    with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 4)) as ex:
+        objs = list(ex.map(run, jobs))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *FLAGS, "-o", tmp, *sources()]
+    link = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static",
+            "-Xcompiler", "-fPIC", "-o", tmp, *objs]
     if verbose:
-        print(" ".join(cmd), flush=True)
-    subprocess.check_call(cmd)
+        print(" ".join(link), flush=True)
+    subprocess.check_call(link)
     os.replace(tmp, LIB)
+    for o in objs:
+        os.remove(o)
+    os.rmdir(objdir)
     return LIB
 
 

@@ -62,8 +62,11 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     constexpr int kKC = C::kKC;
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)NW * kStages * C::kStageB);
+    // per-warp (max, sum) of each head for the merge: [NW][8][2]
+    float* sML = reinterpret_cast<float*>(smem + (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8);
     // d = 256: q'/u' fragments per (operand, n-tile, k-step, lane), filled once per CTA
-    uint2* sB = reinterpret_cast<uint2*>(smem + (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8);
+    uint2* sB = reinterpret_cast<uint2*>(smem + (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
+                                         (size_t)NW * 8 * 2 * sizeof(float));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gr = lane >> 2, tq4 = lane & 3;
     uint8_t* ring = smem + (size_t)warp * kStages * C::kStageB;
@@ -254,16 +257,19 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         lrun[nt] = 0.f;
         live[nt] = (4 * nt + tq4 < Gl) ? 1.f : 0.f;   // this lane's head exists
     }
-    bool failed = false;
+    bool failed = false, drained = true;
 
     for (int i = 0; i < nmine; ++i) {
         const uint32_t bar = smem_u32(&bars[warp * kStages + (i % kStages)]);
-        const bool ok = mbar_wait_bounded(bar, (uint32_t)((i / kStages) & 1));
+        const bool ok = mbar_wait_bounded(bar, (uint32_t)((i / kStages) & 1), i == 0 ? a.first_wait : kWaitLimit);
         if (__any_sync(kFull, !ok)) {         // warp-uniform: no lane may run on alone into mma.sync
             failed = true;
             if (lane == 0) atomicExch(a.err, 1);
+            // wait (bounded) for this warp's copies still in flight before its ring is reused
+            bool all = true;
             for (int j = i; j < nmine && j < i + kStages; ++j)
-                mbar_wait_bounded(smem_u32(&bars[warp * kStages + (j % kStages)]), (uint32_t)((j / kStages) & 1));
+                all &= mbar_wait_bounded(smem_u32(&bars[warp * kStages + (j % kStages)]), (uint32_t)((j / kStages) & 1));
+            drained = __all_sync(kFull, all);
             break;
         }
         const uint8_t* st = ring + (i % kStages) * C::kStageB;
@@ -425,21 +431,26 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     }
 
     pdl_trigger();                        // the combine kernel may start launching
-    // ---------------- merge the warps of the CTA into one partial per head
+    // ---------------- merge the warps of the CTA into one partial per head.  Each
+    // warp's (max, sum) go to sML; its accumulators to its own ring, unless a
+    // failed wait left copies of unknown state there (then the warp is skipped:
+    // its max is -inf and its accumulators are never read).
     __syncwarp();
-    float* wbuf = reinterpret_cast<float*>(ring);             // [Gl][D + 2], in this warp's own ring
+    float* wbuf = reinterpret_cast<float*>(ring);             // [Gl][D], in this warp's own ring
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         const int h = 4 * nt + tq4;
         if (h < Gl) {
+            if (drained) {
 #pragma unroll
-            for (int mt = 0; mt < kKC; ++mt) {
-                wbuf[h * (D + 2) + 16 * mt + gr] = o[nt][mt][0] + o[nt][mt][1];
-                wbuf[h * (D + 2) + 16 * mt + 8 + gr] = o[nt][mt][2] + o[nt][mt][3];
+                for (int mt = 0; mt < kKC; ++mt) {
+                    wbuf[h * D + 16 * mt + gr] = o[nt][mt][0] + o[nt][mt][1];
+                    wbuf[h * D + 16 * mt + 8 + gr] = o[nt][mt][2] + o[nt][mt][3];
+                }
             }
             if (gr == 0) {
-                wbuf[h * (D + 2) + D] = mrun[nt];
-                wbuf[h * (D + 2) + D + 1] = lrun[nt];
+                sML[(warp * 8 + h) * 2] = mrun[nt];
+                sML[(warp * 8 + h) * 2 + 1] = lrun[nt];
             }
         }
     }
@@ -448,15 +459,16 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         const int g = idx / D, j = idx % D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < NW; ++w)
-            M = fmaxf(M, reinterpret_cast<const float*>(smem + (size_t)w * kStages * C::kStageB)[g * (D + 2) + D]);
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, sML[(w * 8 + g) * 2]);
         float L = 0.f, A = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
             for (int w = 0; w < NW; ++w) {
-                const float* wb = reinterpret_cast<const float*>(smem + (size_t)w * kStages * C::kStageB) + g * (D + 2);
-                const float f = exp2f(wb[D] - M);
-                L = fmaf(f, wb[D + 1], L);
+                const float mw = sML[(w * 8 + g) * 2];
+                if (mw == -INFINITY) continue;                    // empty or failed warp
+                const float* wb = reinterpret_cast<const float*>(smem + (size_t)w * kStages * C::kStageB) + g * D;
+                const float f = exp2f(mw - M);
+                L = fmaf(f, sML[(w * 8 + g) * 2 + 1], L);
                 A = fmaf(f, wb[j], A);
             }
         }
@@ -479,6 +491,7 @@ template <int D, int NT, int NW, bool QJL>
 cudaError_t launch_mma_t(const DecArgs& a, int G, cudaStream_t s) {
     using C = Cfg<D, QJL>;
     const size_t smem = (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
+                        (size_t)NW * 8 * 2 * sizeof(float) +
                         (C::kBRegs ? 0 : (size_t)2 * NT * C::kKC * 32 * sizeof(uint2));
     auto kern = tq_decode_mma_kernel<D, NT, NW, QJL>;
     cudaError_t e = set_smem_once<tq_decode_mma_kernel<D, NT, NW, QJL>>((int)smem);
@@ -491,9 +504,9 @@ template <bool QJL>
 cudaError_t launch_mma_q(int d, int G, const DecArgs& a, cudaStream_t s) {
     if (d == 64)
         return G <= 4 ? launch_mma_t<64, 1, kNW1, QJL>(a, G, s) : launch_mma_t<64, 2, kNW2, QJL>(a, G, s);
-    if (d == 128)
-        return G <= 4 ? launch_mma_t<128, 1, kNW1, QJL>(a, G, s) : launch_mma_t<128, 2, kNW2, QJL>(a, G, s);
-    return G <= 4 ? launch_mma_t<256, 1, kNW1, QJL>(a, G, s) : launch_mma_t<256, 2, kNW2, QJL>(a, G, s);
+    if (d == 256)
+        return G <= 4 ? launch_mma_t<256, 1, kNW1, QJL>(a, G, s) : launch_mma_t<256, 2, kNW2, QJL>(a, G, s);
+    return cudaErrorInvalidValue;         // head_dim 128 (V code rows) runs on the tcgen05 kernel
 }
 
 cudaError_t launch_decode_mma(int d, int G, bool qjl, const DecArgs& a, cudaStream_t s) {
@@ -502,9 +515,7 @@ cudaError_t launch_decode_mma(int d, int G, bool qjl, const DecArgs& a, cudaStre
     return qjl ? launch_mma_q<true>(d, G, a, s) : launch_mma_q<false>(d, G, a, s);
 }
 
-int decode_mma_chunk_tokens(int d) {
-    return d == 64 ? Cfg<64>::kChunk : d == 128 ? Cfg<128>::kChunk : Cfg<256>::kChunk;
-}
+int decode_mma_chunk_tokens(int d) { return d == 64 ? Cfg<64>::kChunk : Cfg<256>::kChunk; }
 int decode_mma_warps(int G) { return G <= 4 ? kNW1 : kNW2; }
 
 }  // namespace tqi

@@ -1,5 +1,5 @@
-// Chunked-prefill attention over the packed TurboQuant cache (head_dim 64 and
-// 128), for sm_100a: a chunk of Lq new queries per sequence, query i attending
+// Chunked-prefill attention over the packed TurboQuant cache (head_dim 64, 128
+// and 256), for sm_100a: a chunk of Lq new queries per sequence, query i attending
 // causally over cache tokens [0, T0 + i] (the chunk's own K/V already
 // appended at T0 .. T0 + Lq - 1).
 //
@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillA
     using PC = Cfg<D, true>;
     constexpr int kPD = D;
     constexpr int kPKC = PShape<D>::kKC, kPKB = PShape<D>::kKB;
+    constexpr int kVKC = D == 256 ? 8 : kPKC;            // 16-coordinate value tiles of this CTA
     constexpr size_t kPRing = PShape<D>::kRing, kPQa = PShape<D>::kQa, kPUa = PShape<D>::kUa;
     const DecArgs& a = pa.a;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -73,7 +74,10 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillA
     const int hkv = blockIdx.y, b = blockIdx.z;
     const int G = pa.G;
     const int64_t nrows = pa.Lq * G;
-    const int64_t row0 = (int64_t)blockIdx.x * kPRows + 16 * warp;   // this warp's first row
+    // head_dim 256: CTA pairs share their rows, each accumulating one half of the
+    // value coordinates (both compute the scores)
+    const int vh = D == 256 ? (int)(blockIdx.x & 1) : 0;
+    const int64_t row0 = (int64_t)(D == 256 ? blockIdx.x >> 1 : blockIdx.x) * kPRows + 16 * warp;   // this warp's first row
     const int64_t seq = (int64_t)b * a.Hkv + hkv;
     const int64_t kbb = block_bytes(kPD, true), vbb = block_bytes(kPD, false);
 
@@ -114,7 +118,8 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillA
         bulk_g2s(smem_u32(st + PC::kOffKs), kb + 64 * cb + sub * ch * sb, ch * sb, bar);
         bulk_g2s(smem_u32(st + PC::kOffKn), kb + 64 * (cb + sb) + sub * 2 * ch, 2 * ch, bar);
         bulk_g2s(smem_u32(st + PC::kOffKg), kb + 64 * (cb + sb) + 128 + sub * 2 * ch, 2 * ch, bar);
-        bulk_g2s(smem_u32(st + PC::kOffVc), vb + sub * ch * cb, ch * cb, bar);
+        if constexpr (PC::kVRows) bulk_g2s(smem_u32(st + PC::kOffVc), vb, PC::kVcB, bar);
+        else bulk_g2s(smem_u32(st + PC::kOffVc), vb + sub * ch * cb, ch * cb, bar);
         bulk_g2s(smem_u32(st + PC::kOffVn), vb + 64 * cb + sub * 2 * ch, 2 * ch, bar);
     };
     if (lane == 0)
@@ -194,9 +199,9 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillA
     const uint32_t lut[4] = {a.cb.lut_lo[0], a.cb.lut_lo[1], a.cb.lut_hi[0], a.cb.lut_hi[1]};
     const uint32_t* pw = a.cb.pow2;
     [[maybe_unused]] const uint32_t m64 = pw[20] | 1u;    // d = 64 sign widening factor
-    float o[2 * kPKC][4];                 // 16 coordinate n-tiles: rows g (0, 1), g + 8 (2, 3)
+    float o[2 * kVKC][4];                 // coordinate n-tiles of 8: rows g (0, 1), g + 8 (2, 3)
 #pragma unroll
-    for (int nc = 0; nc < 2 * kPKC; ++nc) o[nc][0] = o[nc][1] = o[nc][2] = o[nc][3] = 0.f;
+    for (int nc = 0; nc < 2 * kVKC; ++nc) o[nc][0] = o[nc][1] = o[nc][2] = o[nc][3] = 0.f;
     float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};
     bool failed = false;
 
@@ -216,11 +221,14 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillA
         for (int kt = 0; kt < PC::kTiles; ++kt) {
             // ---------------- scores of 16 rows x 16 tokens (two n-tiles of 8)
             const int tA = kt * 16 + gr, tB = tA + 8;            // B-fragment tokens of n-tiles 0, 1
-            uint32_t selA[4], selB[4];
-            token_selectors<D>(st + PC::kOffKc + tA * PC::kCodeB, 0, tq4, pw, selA);
-            token_selectors<D>(st + PC::kOffKc + tB * PC::kCodeB, 0, tq4, pw, selB);
-            const uint32_t sgA = token_signs<D>(st + PC::kOffKs + tA * PC::kSignB, 0, tq4, m64);
-            const uint32_t sgB = token_signs<D>(st + PC::kOffKs + tB * PC::kSignB, 0, tq4, m64);
+            uint32_t selA[PC::kS][4], selB[PC::kS][4], sgA[PC::kS], sgB[PC::kS];
+#pragma unroll
+            for (int sl = 0; sl < PC::kS; ++sl) {                // 128-coordinate slices
+                token_selectors<D>(st + PC::kOffKc + tA * PC::kCodeB, sl, tq4, pw, selA[sl]);
+                token_selectors<D>(st + PC::kOffKc + tB * PC::kCodeB, sl, tq4, pw, selB[sl]);
+                sgA[sl] = token_signs<D>(st + PC::kOffKs + tA * PC::kSignB, sl, tq4, m64);
+                sgB[sl] = token_signs<D>(st + PC::kOffKs + tB * PC::kSignB, sl, tq4, m64);
+            }
             float sacc[2][4];
             int iacc[2][2][4];                                  // [n-tile][u' limb]
 #pragma unroll
@@ -233,8 +241,8 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillA
 #pragma unroll
             for (int kc = 0; kc < kPKC; ++kc) {
                 uint32_t kA0, kA1, kB0, kB1;
-                dequant4(sel_for(selA, pw, kc), lut, kA0, kA1);
-                dequant4(sel_for(selB, pw, kc), lut, kB0, kB1);
+                dequant4(sel_for(selA[kc >> 3], pw, kc & 7), lut, kA0, kA1);
+                dequant4(sel_for(selB[kc >> 3], pw, kc & 7), lut, kB0, kB1);
                 const uint4 ah = qa[(kc * 2 + 0) * 32 + lane], al = qa[(kc * 2 + 1) * 32 + lane];
                 const uint32_t aH[4] = {ah.x, ah.y, ah.z, ah.w}, aL[4] = {al.x, al.y, al.z, al.w};
                 mma16816(sacc[0], aH, kA0, kA1);
@@ -242,11 +250,11 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillA
                 mma16816(sacc[1], aH, kB0, kB1);
                 mma16816(sacc[1], aL, kB0, kB1);
                 if ((kc & 1) == 0) {                            // one 32-row sign block per two k-steps
-                    const int kb = kc >> 1;
-                    const uint32_t bA0 = shl_m(sgA, pw, 2 * kb) & 0x80808080u;
-                    const uint32_t bA1 = shl_m(sgA, pw, 2 * kb + 1) & 0x80808080u;
-                    const uint32_t bB0 = shl_m(sgB, pw, 2 * kb) & 0x80808080u;
-                    const uint32_t bB1 = shl_m(sgB, pw, 2 * kb + 1) & 0x80808080u;
+                    const int kb = kc >> 1, k4 = kb & 3;
+                    const uint32_t bA0 = shl_m(sgA[kb >> 2], pw, 2 * k4) & 0x80808080u;
+                    const uint32_t bA1 = shl_m(sgA[kb >> 2], pw, 2 * k4 + 1) & 0x80808080u;
+                    const uint32_t bB0 = shl_m(sgB[kb >> 2], pw, 2 * k4) & 0x80808080u;
+                    const uint32_t bB1 = shl_m(sgB[kb >> 2], pw, 2 * k4 + 1) & 0x80808080u;
                     const uint4 uh = ua[(kb * 2 + 0) * 32 + lane], ul = ua[(kb * 2 + 1) * 32 + lane];
                     const uint32_t uH[4] = {uh.x, uh.y, uh.z, uh.w}, uL[4] = {ul.x, ul.y, ul.z, ul.w};
                     imma16832(iacc[0][0], uH, bA0, bA1);
@@ -282,7 +290,7 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillA
                     const float corr = (mnew == -INFINITY) ? 1.f : fast_exp2(mrun[h] - mnew);
                     lrun[h] *= corr;
 #pragma unroll
-                    for (int nc = 0; nc < 2 * kPKC; ++nc) {
+                    for (int nc = 0; nc < 2 * kVKC; ++nc) {
                         o[nc][2 * h] *= corr;
                         o[nc][2 * h + 1] *= corr;
                     }
@@ -307,20 +315,35 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillA
             split_hilo(pv[0][2], pv[0][3], pH[1], pL[1]);
             split_hilo(pv[1][0], pv[1][1], pH[2], pL[2]);
             split_hilo(pv[1][2], pv[1][3], pH[3], pL[3]);
-            // ---------------- values: O[16 rows][8 coords] += P Vdeq, Vdeq^T by movmatrix
-            token_selectors<D>(st + PC::kOffVc + tA * PC::kCodeB, 0, tq4, pw, selA);
-            token_selectors<D>(st + PC::kOffVc + tB * PC::kCodeB, 0, tq4, pw, selB);
+            // ---------------- values: O[16 rows][8 coords] += P Vdeq
+            if constexpr (PC::kVRows) {
+                // B fragment of coordinate n-tile nc straight from V code rows: lane (g, t)
+                // takes row 8 nc + g, tokens 2t, 2t + 1 (b0) and 2t + 8, 2t + 9 (b1) of the
+                // tile's 16-token group of the block
+                const int q = (int)((tok0 & 63) >> 4) + kt;
 #pragma unroll
-            for (int kc = 0; kc < kPKC; ++kc) {
-                uint32_t x0, x1, y0, y1;
-                dequant4(sel_for(selA, pw, kc), lut, x0, x1);   // tokens 0..7 of the tile
-                dequant4(sel_for(selB, pw, kc), lut, y0, y1);   // tokens 8..15
-                const uint32_t mx0 = movmatrix_t(x0), mx1 = movmatrix_t(x1);
-                const uint32_t my0 = movmatrix_t(y0), my1 = movmatrix_t(y1);
-                mma16816(o[2 * kc], pH, mx0, my0);
-                mma16816(o[2 * kc], pL, mx0, my0);
-                mma16816(o[2 * kc + 1], pH, mx1, my1);
-                mma16816(o[2 * kc + 1], pL, mx1, my1);
+                for (int nc = 0; nc < 2 * kVKC; ++nc) {
+                    uint32_t b0, b1;
+                    dequant4(vrow_selector(st + PC::kOffVc + (8 * nc + gr) * kVRowB, tq4, q), lut, b0, b1);
+                    mma16816(o[nc], pH, b0, b1);
+                    mma16816(o[nc], pL, b0, b1);
+                }
+            } else {
+                // Vdeq^T by movmatrix from token-record fragments
+                token_selectors<D>(st + PC::kOffVc + tA * PC::kCodeB, vh, tq4, pw, selA[0]);
+                token_selectors<D>(st + PC::kOffVc + tB * PC::kCodeB, vh, tq4, pw, selB[0]);
+#pragma unroll
+                for (int kc = 0; kc < kVKC; ++kc) {
+                    uint32_t x0, x1, y0, y1;
+                    dequant4(sel_for(selA[0], pw, kc), lut, x0, x1);   // tokens 0..7 of the tile
+                    dequant4(sel_for(selB[0], pw, kc), lut, y0, y1);   // tokens 8..15
+                    const uint32_t mx0 = movmatrix_t(x0), mx1 = movmatrix_t(x1);
+                    const uint32_t my0 = movmatrix_t(y0), my1 = movmatrix_t(y1);
+                    mma16816(o[2 * kc], pH, mx0, my0);
+                    mma16816(o[2 * kc], pL, mx0, my0);
+                    mma16816(o[2 * kc + 1], pH, mx1, my1);
+                    mma16816(o[2 * kc + 1], pL, mx1, my1);
+                }
             }
         }
         __syncwarp();
@@ -336,11 +359,11 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillA
         lrun[h] += __shfl_xor_sync(kFull, lrun[h], 1);
         lrun[h] += __shfl_xor_sync(kFull, lrun[h], 2);
         if (!rvalid[h]) continue;
-        float* acc = a.part_acc + qrow[h] * kPD;          // one split per row
+        float* acc = a.part_acc + qrow[h] * kPD + 128 * vh;   // one split per row
 #pragma unroll
-        for (int nc = 0; nc < 2 * kPKC; ++nc)
+        for (int nc = 0; nc < 2 * kVKC; ++nc)
             *reinterpret_cast<float2*>(acc + 8 * nc + 2 * tq4) = make_float2(o[nc][2 * h], o[nc][2 * h + 1]);
-        if (tq4 == 0) {
+        if (tq4 == 0 && vh == 0) {
             a.part_ml[2 * qrow[h]] = mrun[h];
             a.part_ml[2 * qrow[h] + 1] = lrun[h];
         }
@@ -354,16 +377,17 @@ cudaError_t launch_prefill_d(int G, const DecArgs& a, int64_t Lq, int64_t T0, cu
     const int64_t tiles = (Lq * G + kPRows - 1) / kPRows;
     cudaError_t e = set_smem_once<tq_prefill_mma_kernel<D>>((int)smem);
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)tiles, (unsigned)a.Hkv, (unsigned)a.B);
+    const dim3 grid((unsigned)(tiles * (D == 256 ? 2 : 1)), (unsigned)a.Hkv, (unsigned)a.B);
     return launch_pdl(tq_prefill_mma_kernel<D>, grid, dim3(kPW * 32), smem, s, pa);
 }
 
 }  // namespace
 
 cudaError_t launch_prefill(int d, int G, const DecArgs& a, int64_t Lq, int64_t T0, cudaStream_t s) {
-    if ((d != 64 && d != 128) || G < 1) return cudaErrorInvalidValue;
+    if (!head_dim_ok(d) || G < 1) return cudaErrorInvalidValue;
     if (a.B * a.Hkv == 0 || Lq == 0) return cudaSuccess;
-    return d == 64 ? launch_prefill_d<64>(G, a, Lq, T0, s) : launch_prefill_d<128>(G, a, Lq, T0, s);
+    if (d == 64) return launch_prefill_d<64>(G, a, Lq, T0, s);
+    return d == 128 ? launch_prefill_d<128>(G, a, Lq, T0, s) : launch_prefill_d<256>(G, a, Lq, T0, s);
 }
 
 }  // namespace tqi

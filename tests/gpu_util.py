@@ -9,7 +9,9 @@ Criteria:
     does not count against the signs); the excluded mismatches must also be
     at most 1e-5 of the total;
   * stored fp16 norms within one fp16 unit in the last place;
-  * attention outputs: per (batch, query head) row, ||o - r||_inf / ||r||_inf <= 1e-3.
+  * attention outputs: per (batch, query head) row, ||o - r||_inf / ||r||_inf <= 1e-3
+    (the largest per-element relative error over elements above 1e-3 of their
+    row's largest magnitude is printed beside it).
 """
 from __future__ import annotations
 
@@ -49,7 +51,7 @@ def unpack_cache(cache: tq.Cache, t0: int, T: int, seqs=None) -> dict:
     d, is_k = cache.head_dim, cache.is_k
     raw = cache.buf.cpu().numpy()
     nb = cache.Tcap // 64
-    bb = O.block_bytes(d, is_k)
+    bb = O.block_bytes(d, cache.kind)
     seqs = seqs if seqs is not None else [(b, h) for b in range(cache.B) for h in range(cache.Hkv)]
     out = {"idx": np.zeros((len(seqs), T, d), np.uint8), "nh": np.zeros((len(seqs), T), np.uint16)}
     if is_k:
@@ -57,7 +59,7 @@ def unpack_cache(cache: tq.Cache, t0: int, T: int, seqs=None) -> dict:
         out["gh"] = np.zeros((len(seqs), T), np.uint16)
     for n, (b, h) in enumerate(seqs):
         s = (b * cache.Hkv + h) * nb
-        u = O.unpack(d, is_k, t0, T, raw[s * bb:(s + nb) * bb])
+        u = O.unpack(d, cache.kind, t0, T, raw[s * bb:(s + nb) * bb])
         for k in out:
             out[k][n] = u[k]
     return out
@@ -72,7 +74,9 @@ def check_encode(prm: dict, x: np.ndarray, gk: dict | None, gv: dict | None) -> 
     d = prm["d"]
     x = np.asarray(x, np.float64).reshape(-1, d)
     e = O.encode(x, prm, with_qjl=gk is not None)
-    near = np.min(np.abs(e["y"][..., None] - prm["b7"]), axis=-1) < EPS_WINDOW
+    near = np.zeros(e["y"].shape, dtype=bool)
+    for b in prm["b7"]:                       # one boundary at a time (bounded host memory)
+        near |= np.abs(e["y"] - b) < EPS_WINDOW
     stats = {"vectors": x.shape[0], "near_boundary": int(near.sum())}
     for name, g in (("k", gk), ("v", gv)):
         if g is None:
@@ -121,6 +125,20 @@ def rel_err_rows(out: np.ndarray, ref: np.ndarray) -> np.ndarray:
     den = np.abs(r).max(axis=1)
     num = np.abs(o - r).max(axis=1)
     return np.where(den > 0, num / np.where(den > 0, den, 1), num)
+
+
+def rel_err_elements(out: np.ndarray, ref: np.ndarray, floor: float = 1e-3) -> float:
+    """Largest per-element relative error |o - r| / |r| over the elements whose
+    |r| is at least `floor` times their row's ||r||_inf (reported beside the
+    per-row criterion; elements near zero are left out since their relative
+    error is unbounded)."""
+    o = out.reshape(-1, out.shape[-1])
+    r = ref.reshape(-1, ref.shape[-1])
+    big = np.abs(r) >= floor * np.abs(r).max(axis=1, keepdims=True)
+    big &= np.abs(r) > 0
+    if not big.any():
+        return 0.0
+    return float((np.abs(o - r)[big] / np.abs(r)[big]).max())
 
 
 def attend_gpu(h, q: torch.Tensor, kc, vc, T: int = 0, seq_lens=None, scale=1.0):

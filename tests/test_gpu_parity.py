@@ -9,7 +9,7 @@ import torch
 
 import oracle as O
 from kv_cache_vector_14_b200 import synthetic, tq
-from gpu_util import (ATT_TOL, attend_gpu, check_encode, encode_gpu, oracle_attend, rel_err_rows,
+from gpu_util import (ATT_TOL, attend_gpu, check_encode, encode_gpu, oracle_attend, rel_err_elements, rel_err_rows,
                       torch_input, unpack_cache)
 
 pytestmark = pytest.mark.gpu
@@ -90,6 +90,52 @@ def test_encode_d256_sampled(handles, prms):
     print(check_encode(prms[256], _x64(xs), _flat(gk), _flat(gv)))
 
 
+def test_encode_gqa_40960_full(handles, prms):
+    """The 40960-token GQA workload's cache (B=1, 8 kv heads, bf16 K and V with
+    outliers and log-normal norms): every K and V vector of every head compared
+    with the oracle's encode."""
+    w = synthetic.WORKLOADS["c3"]
+    xk, xv = synthetic.kv(w, "k"), synthetic.kv(w, "v")
+    kc, _ = encode_gpu(handles[128], 128, torch_input(xk, w.kv_dtype), Tcap=w.T, which="k")
+    _, vc = encode_gpu(handles[128], 128, torch_input(xv, w.kv_dtype), Tcap=w.T, which="v")
+    print("K", check_encode(prms[128], _x64(xk), _flat(unpack_cache(kc, 0, w.T)), None))
+    print("V", check_encode(prms[128], _x64(xv), None, _flat(unpack_cache(vc, 0, w.T))))
+
+
+def test_encode_long_context_b4_102400_sampled(handles, prms):
+    """The long-context workload's cache (B=4, 8 kv heads, 102400 fp32 tokens with
+    outliers: the benchmark's own cache, encoded in the benchmark's launch
+    configuration): four whole sequences, the first and the last among them,
+    compared with the oracle's encode over all 102400 tokens."""
+    w = synthetic.WORKLOADS["c4"]
+    seqs = [(0, 0), (1, 3), (2, 6), (w.B - 1, w.Hkv - 1)]
+    for which in ("k", "v"):
+        x = synthetic.kv(w, which)
+        c = encode_gpu(handles[128], 128, torch_input(x, w.kv_dtype), Tcap=w.T, which=which)[0 if which == "k" else 1]
+        g = _flat(unpack_cache(c, 0, w.T, seqs))
+        xs = np.stack([x[b, hk] for b, hk in seqs])
+        del x, c
+        st = check_encode(prms[128], _x64(xs), g if which == "k" else None, g if which == "v" else None)
+        print(which.upper(), st)
+
+
+def test_encode_d64_bench_sampled(handles, prms):
+    """The head_dim 64 benchmark workload's cache (B=4, 8 kv heads, 102400 bf16
+    tokens, outliers and log-normal norms): two whole sequences, the last among
+    them, against the oracle's encode."""
+    w = synthetic.Workload("d64", "d64 bench", B=4, Hq=16, Hkv=8, d=64, T=102400, kv_dtype="bf16",
+                           q_dtype="bf16", lognormal_norms=True, seed=640, scale=0.125)
+    seqs = [(0, 0), (w.B - 1, w.Hkv - 1)]
+    for which in ("k", "v"):
+        x = synthetic.kv(w, which)
+        c = encode_gpu(handles[64], 64, torch_input(x, w.kv_dtype), Tcap=w.T, which=which)[0 if which == "k" else 1]
+        g = _flat(unpack_cache(c, 0, w.T, seqs))
+        xs = np.stack([x[b, hk] for b, hk in seqs])
+        del x, c
+        st = check_encode(prms[64], _x64(xs), g if which == "k" else None, g if which == "v" else None)
+        print(which.upper(), st)
+
+
 @pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 def test_encode_ragged_offsets_strides(handles, prms, d, dtype):
@@ -160,7 +206,7 @@ def test_attend_single_head(decode_path, handles, prms):
     w = synthetic.WORKLOADS["c1"]
     out, ref, err = _attend_case(handles[128], prms[128], w, synthetic.kv(w, "k"), synthetic.kv(w, "v"),
                                  synthetic.queries(w), w.T, w.T)
-    print("max rel err", err.max())
+    print("max rel err", err.max(), "per element", rel_err_elements(out, ref))
     assert err.max() <= ATT_TOL
 
 
@@ -168,7 +214,7 @@ def test_attend_gqa_32_8_40960_full(decode_path, handles, prms):
     w = synthetic.WORKLOADS["c3"]
     out, ref, err = _attend_case(handles[128], prms[128], w, synthetic.kv(w, "k"), synthetic.kv(w, "v"),
                                  synthetic.queries(w), w.T, w.T)
-    print("max rel err", err.max())
+    print("max rel err", err.max(), "per element", rel_err_elements(out, ref))
     assert err.max() <= ATT_TOL
 
 
@@ -177,7 +223,8 @@ def test_attend_long_context_b4_102400_full(decode_path, handles, prms):
     w = synthetic.WORKLOADS["c4"]
     out, ref, err = _attend_case(handles[128], prms[128], w, synthetic.kv(w, "k"), synthetic.kv(w, "v"),
                                  synthetic.queries(w), w.T, w.T)
-    print("max rel err", err.max(), "path", tq.tq_attend_path(handles[128], w.Hq, w.Hkv), decode_path)
+    print("max rel err", err.max(), "per element", rel_err_elements(out, ref), "path",
+          tq.tq_attend_path(handles[128], w.Hq, w.Hkv), decode_path)
     assert err.max() <= ATT_TOL
 
 
@@ -217,7 +264,7 @@ def test_append_and_attend_loop_d256(handles, prms):
     assert torch.equal(kb.buf, kc.buf) and torch.equal(vb.buf, vc.buf)
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("G,T0,Lq", [(4, 0, 20), (2, 100, 37), (1, 64, 5), (8, 300, 17), (3, 70, 23), (16, 129, 9)])
 def test_attend_prefill_matches_oracle(handles, prms, d, G, T0, Lq):
     """Chunked prefill: query i of the chunk attends causally over tokens
@@ -285,7 +332,7 @@ def test_attend_prefill_bench_size_sampled_rows(handles, prms, d):
     assert tq.tq_device_status(h) == tq.TQ_OK
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_attend_prefill_paged_equals_contiguous(handles, d):
     """Prefill over paged caches (random block tables) gives the same output,
     bit for bit, as over contiguous caches holding the same blocks."""
@@ -494,15 +541,16 @@ def test_attend_group_sizes_and_ragged_lengths(decode_path, handles, prms, d, G)
 @pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
 def test_attend_polar_only_k(decode_path, handles, prms, d, G):
-    """PolarQuant-only K (a V-layout K cache from tq_encode_v): the kernels'
-    attention equals the oracle's with gamma = 0 (no QJL term), ragged lengths."""
+    """PolarQuant-only K (a K cache of codes and norms from tq_encode_k_polar):
+    the kernels' attention equals the oracle's with gamma = 0 (no QJL term),
+    ragged lengths; the K cache holds the oracle's V-flow codes and norms."""
     Hkv, B, Tcap = 2, 3, 320
     Hq = Hkv * G
     h = handles[d]
     xk = torch_input(synthetic.gaussian((B, Hkv, Tcap, d), seed=31 + G), "f32")
     xv = torch_input(synthetic.gaussian((B, Hkv, Tcap, d), seed=41 + G), "f32")
-    kc, vc = tq.Cache(d, False, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
-    tq.tq_encode_v(h, xk, kc, 0)
+    kc, vc = tq.Cache(d, False, B, Hkv, Tcap, polar=True), tq.Cache(d, False, B, Hkv, Tcap)
+    tq.tq_encode_k_polar(h, xk, kc, 0)
     tq.tq_encode_v(h, xv, vc, 0)
     q = synthetic.gaussian((B, Hq, d), seed=51)
     lens = [0, 129, 301]
@@ -512,6 +560,8 @@ def test_attend_polar_only_k(decode_path, handles, prms, d, G):
     scale = 1.0 / np.sqrt(d)
     tq.tq_attend_decode_polar(h, torch_input(q, "f32"), kc, vc, out, ws, seq_lens=sl, scale=scale)
     ku, vu = unpack_cache(kc, 0, Tcap), unpack_cache(vc, 0, Tcap)
+    if G == 1:
+        print(check_encode(prms[d], xk.double().cpu().numpy().reshape(-1, d), None, _flat(ku)))
     ku = {"idx": ku["idx"], "nh": ku["nh"], "sig": np.ones(ku["idx"].shape, np.uint8),
           "gh": np.zeros_like(ku["nh"])}
     ref = oracle_attend(prms[d], q.astype(np.float64), ku, vu, Hkv, lens, scale)
@@ -599,6 +649,37 @@ def test_group_heads_equal_separate_heads(decode_path, handles):
         assert rel_err_rows(one[0, 0], full[0, 4 + g]).max() <= 1e-5
 
 
+@pytest.mark.parametrize("d,G", [(128, 4), (128, 2), (64, 2), (256, 4), (128, 8)])
+def test_bounded_wait_give_up_path(handles, prms, d, G):
+    """Every wait in the attention kernel is bounded.  With the first-wait
+    budget set to zero polls every warp gives up at its first staged chunk: the
+    call completes, the check word reports the failed wait, the outputs are
+    finite (the warps' tokens are left out), and after the budget is restored
+    the same handle computes the attention again and matches the oracle."""
+    h = handles[d]
+    B, Hkv, T = 2, 2, 777
+    Hq, Tcap = Hkv * G, 832
+    x = synthetic.gaussian((2, B, Hkv, Tcap, d), seed=17)
+    kc, vc = tq.Cache(d, True, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
+    tq.tq_encode_k(h, torch_input(x[0], "f32"), kc, 0)
+    tq.tq_encode_v(h, torch_input(x[1], "f32"), vc, 0)
+    q = synthetic.gaussian((B, Hq, d), seed=18)
+    assert tq.tq_device_status(h) == tq.TQ_OK
+    try:
+        tq.tq_set_wait_limit(h, 0)
+        out = attend_gpu(h, torch_input(q, "f32"), kc, vc, T=T, scale=0.1)
+        assert tq.tq_device_status(h) == tq.TQ_ERR_DEVICE_CHECK
+        assert torch.isfinite(out).all()
+    finally:
+        tq.tq_set_wait_limit(h, -1)
+    assert tq.tq_device_status(h) == tq.TQ_OK
+    out = attend_gpu(h, torch_input(q, "f32"), kc, vc, T=T, scale=0.1).cpu().numpy()
+    assert tq.tq_device_status(h) == tq.TQ_OK
+    ref = oracle_attend(prms[d], q.astype(np.float64), unpack_cache(kc, 0, Tcap), unpack_cache(vc, 0, Tcap), Hkv,
+                        [T] * B, 0.1)
+    assert rel_err_rows(out, ref).max() <= ATT_TOL
+
+
 def test_attend_argument_errors(handles):
     h = handles[128]
     kc, vc = tq.Cache(128, True, 1, 2, 64), tq.Cache(128, False, 1, 2, 64)
@@ -621,10 +702,12 @@ def test_attend_argument_errors(handles):
     with pytest.raises(tq.TQError) as e:
         tq.tq_encode_k(h, x, kc, t0=60)                            # past Tcap
     assert e.value.status == tq.TQ_ERR_INVALID_ARG
-    h2 = handles[256]                                              # prefill: head_dim 64 and 128 only
+    h2 = handles[256]
     k2, v2 = tq.Cache(256, True, 1, 2, 64), tq.Cache(256, False, 1, 2, 64)
-    with pytest.raises(tq.TQError) as e:
-        tq.tq_attend_prefill(h2, torch.zeros((1, 3, 4, 256), device="cuda"), k2, v2, 0,
+    with pytest.raises(tq.TQError) as e:                           # prefill past Tcap
+        tq.tq_attend_prefill(h2, torch.zeros((1, 3, 4, 256), device="cuda"), k2, v2, 62,
                              torch.empty((1, 3, 4, 256), device="cuda"), ws)
-    assert e.value.status == tq.TQ_ERR_UNSUPPORTED
+    assert e.value.status == tq.TQ_ERR_INVALID_ARG
+    with pytest.raises(ValueError):                                # a V cache is not a PolarQuant-only K cache
+        tq.tq_attend_decode_polar(h, q, vc, vc, out, ws, T=10)
     assert tq.tq_device_status(h) == tq.TQ_OK
