@@ -40,9 +40,12 @@ UNIT = "GB/s"
 BYTES_PER_TOKEN_HEAD = {64: 36 + 26, 128: 68 + 50, 256: 132 + 98}   # packed K + V record per token per kv head
 ENCODE_BYTES_PER_VECTOR = {("k", 128): 68, ("v", 128): 50}
 
-# DRAM traffic of the split-K kernel from one ncu capture, valid only while the
-# kernel sources are unchanged (sha256 over DECODE_SOURCES at capture time).
-NCU_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None, "capture": None}
+# DRAM traffic of the split-K kernel (read + write bytes per launch) from one
+# ncu capture, valid only while the kernel sources are unchanged (sha256 over
+# DECODE_SOURCES at capture time).
+NCU_TRAFFIC = {"source_sha256": "03f1b57d61869e3c17d52360942f696182b86736a82f9a82d442e1e50e17db93",
+               "bytes_per_launch": 386811136 + 3334656,
+               "capture": "profiles/tq_decode_mma_d128_long_context_b4_hq16_hkv8_t102400.md"}
 
 
 def peaks():
@@ -63,8 +66,7 @@ def bf16_peak_tflops() -> float:
         return 1590.0
 
 
-DECODE_SOURCES = ("kv_cache_vector_14_b200/csrc/tq_decode_tc.cu", "kv_cache_vector_14_b200/csrc/tq_tc.cuh",
-                  "kv_cache_vector_14_b200/csrc/tq_frag.cuh", "kv_cache_vector_14_b200/csrc/tq_internal.h")
+DECODE_SOURCES = ("kv_cache_vector_14_b200/csrc/tq_decode_mma.cu", "kv_cache_vector_14_b200/csrc/tq_frag.cuh")
 
 
 def source_sha(rels) -> str:
@@ -408,9 +410,9 @@ def measure_polar(h, dev, w, vc, q, out_qjl, ws, n_calls: int) -> dict:
     import torch
     from kv_cache_vector_14_b200 import tq
     d, B, Hq, Hkv, T = w.d, w.B, w.Hq, w.Hkv, w.T
-    kp = tq.Cache(d, False, B, Hkv, T, polar=True)
+    kp = tq.Cache(d, False, B, Hkv, T)
     x = torch.from_numpy(synthetic.kv(w, "k")).to(dev)
-    tq.tq_encode_k_polar(h, x, kp, 0)
+    tq.tq_encode_v(h, x, kp, 0)
     del x
     out = torch.empty_like(out_qjl)
     for _ in range(5):
@@ -743,6 +745,7 @@ def run_ours(args, rank: int, world: int, dist):
         tq.tq_destroy(h)
         r = measure_d64(dev, world, dist, n_calls=args.steps)
         r["prefill"] = measure_prefill(dev, world, dist, reps=5, d=64)
+        r["prefill_d256"] = measure_prefill(dev, world, dist, reps=5, d=256)
         if rank == 0:
             print(json.dumps({"d64": r}), flush=True)
         return
@@ -880,12 +883,13 @@ def run_ours(args, rank: int, world: int, dist):
     single = measure_single_head(dev, world, dist)
     prefill = measure_prefill(dev, world, dist)
     prefill64 = measure_prefill(dev, world, dist, d=64)
+    prefill256 = measure_prefill(dev, world, dist, reps=10, d=256)
     d64 = measure_d64(dev, world, dist)
 
     peak, peak_kind = peaks()
     bf16_peak = bf16_peak_tflops()
     achieved = bytes_step / (kern_ms * 1e-3) / 1e9
-    traffic = NCU_TRAFFIC["bytes_per_launch"] if (path == "tc" and
+    traffic = NCU_TRAFFIC["bytes_per_launch"] if (path == "mma" and
                                                   NCU_TRAFFIC["source_sha256"] == source_sha(DECODE_SOURCES)) else None
 
     cpu = None
@@ -936,6 +940,7 @@ def run_ours(args, rank: int, world: int, dist):
                     "peak_kind": "measured bf16 dense GEMM (burst); the kernel uses mma.sync fp16/int8"},
         "d64": {**d64, "frac": d64["achieved_gbs"] / peak,
                 "prefill": {**prefill64, "frac": prefill64["tflops"] / bf16_peak}},
+        "prefill_d256": {**prefill256, "frac": prefill256["tflops"] / bf16_peak},
         "device_status": tq.tq_status_string(status),
     }
     print(json.dumps(line), flush=True)

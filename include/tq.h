@@ -73,18 +73,8 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1, TQ_F16 = 2 } tq_dtype;
  * With block_table == NULL pool_blocks is ignored.
  * K block (64 tokens): codes 64 x 3d/8 B | signs 64 x d/8 B | ||k|| fp16 x 64 |
  *                      gamma = ||residual|| fp16 x 64
- * V block (64 tokens), d = 128: code rows d x 24 B | ||v|| fp16 x 64
- * V block, d = 64 and 256, and PolarQuant-only K block (tq_encode_k_polar),
- * every d: codes 64 x 3d/8 B | norm fp16 x 64 (the K block without signs and
- * gamma)
- * d = 128 V code rows: row j (bytes 24 j .. 24 j + 23) holds the codes of
- * coordinate j for the block's 64 tokens, six little-endian uint32 words laid
- * out like the d = 64 token record below with token tau in the place of
- * coordinate tau: token tau has slot (tau >> 1) & 3 and slot position
- * i = 4 (tau >> 4) + 2 ((tau >> 3) & 1) + (tau & 1).  A row gives the value
- * contraction its operand along tokens without a transpose.
- * Token records: per token the 3-bit codes are 3d/32 little-endian uint32
- * words (codes 64 x 3d/8 B above, token after token).  Slice s
+ * V block (64 tokens): codes 64 x 3d/8 B | ||v|| fp16 x 64
+ * Per token the 3-bit codes are 3d/32 little-endian uint32 words.  Slice s
  * (128 coordinates) and slot t (0..3) own words 12s+3t+{0,1,2} (Wa, Wb, Wc)
  * holding slot codes i = 0..31, where slot code i is coordinate
  *     j = 128 s + 16 (i >> 2) + 2 t + (i & 1) + 8 ((i >> 1) & 1).
@@ -166,16 +156,6 @@ TQ_API tq_status tq_encode_v(const tq_handle* h, const void* x, tq_dtype dtype, 
                       int64_t Tnew, int64_t sb, int64_t sh, int64_t st, const tq_cache* vc,
                       int64_t t0, void* stream);
 
-/* The V flow (K section steps 1-3 without the QJL bit, as the page's V
- * section encodes V) into a PolarQuant-only K cache of tq_cache_bytes(d, 0,
- * ...) bytes: codes in token records and the fp16 norm, 3.125 bits/dim at
- * d = 128, for tq_attend_decode_polar (the page's hybrid V2+V3 section keeps
- * K at 3 bits without QJL on its faster path).  At d = 64 and 256 the bytes
- * equal those tq_encode_v writes.  Arguments and errors as tq_encode_k. */
-TQ_API tq_status tq_encode_k_polar(const tq_handle* h, const void* x, tq_dtype dtype, int64_t B, int64_t Hkv,
-                                   int64_t Tnew, int64_t sb, int64_t sh, int64_t st, const tq_cache* kc,
-                                   int64_t t0, void* stream);
-
 /* ---- decode attention --------------------------------------------------- */
 
 /* Workspace bytes tq_attend_decode needs for these sizes on this handle's
@@ -197,9 +177,8 @@ TQ_API size_t tq_attend_workspace_bytes(const tq_handle* h, int64_t B, int64_t H
  * with n_t, gamma_t, nv_t the stored fp16 values, in fp32 with split-K
  * (flash-decoding) partials in `ws` merged by a final kernel.  out is fp32
  * [B][Hq][d]; an empty sequence gives zeros.  Supported: d in {64, 128, 256},
- * any Hq/Hkv (kv heads with many query heads are served in groups of up to 4
- * at d = 128 and 8 otherwise), B <= 65535, Hkv * ceil(Hq/Hkv / 4) <= 65535,
- * B * Hq < 2^31.  ws must be 256-byte
+ * any Hq/Hkv (kv heads with more than 8 query heads are served in groups of
+ * up to 8), B <= 65535, Hkv * ceil(Hq/Hkv / 8) <= 65535, B * Hq < 2^31.  ws must be 256-byte
  * aligned with at least
  * tq_attend_workspace_bytes(h, B, Hq, Hkv, T or max seq_len) bytes.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
@@ -210,10 +189,10 @@ TQ_API tq_status tq_attend_decode(const tq_handle* h, const void* q, tq_dtype qd
 
 /* ---- PolarQuant-only K (no QJL bit) --------------------------------------- */
 
-/* Attention over a PolarQuant-only K cache: 3-bit codes and the fp16 norm but
- * no QJL sign bits and no gamma (3.125 bits/dim at d = 128 instead of 4.25),
- * written by tq_encode_k_polar into a buffer of tq_cache_bytes(d, 0, ...)
- * bytes.  Scores drop the QJL term:
+/* Attention over a PolarQuant-only K cache: K stored like V, with 3-bit codes
+ * and the fp16 norm but no QJL sign bits and no gamma (3.125 bits/dim at
+ * d = 128 instead of 4.25).  Encode such a K cache with tq_encode_v into a
+ * V-layout buffer (tq_cache_bytes(d, 0, ...)).  Scores drop the QJL term:
  *   s_t = scale * n_t * <q', c[idx_t]>,
  * the rest as tq_attend_decode (same arguments, workspace and errors).  The
  * page weighs the two K flows against each other: its K section adds the
@@ -329,13 +308,12 @@ TQ_API tq_status tq_set_decode_events(tq_handle* h, void* ev_start, void* ev_sto
 TQ_API tq_status tq_set_wait_limit(tq_handle* h, int first_wait);
 
 /* Diagnostics: choose the decode kernel of later tq_attend_decode calls on this
- * handle: 0 = automatic (the tensor-core kernel of the head_dim), 1 = the SIMT
+ * handle: 0 = automatic (tensor-core kernel where supported), 1 = the SIMT
  * kernel.  Changes the workspace size tq_attend_workspace_bytes reports. */
 TQ_API tq_status tq_set_decode_path(tq_handle* h, int path);
 
 /* Name of the kernel path tq_attend_decode uses for these sizes on this handle
- * ("tc": tcgen05 kernel, head_dim 128; "mma": mma.sync kernel, head_dim 64 and
- * 256; "simt": the SIMT kernel); static string. */
+ * ("mma" or "simt"); static string. */
 TQ_API const char* tq_attend_path(const tq_handle* h, int64_t Hq, int64_t Hkv);
 
 TQ_API const char* tq_status_string(tq_status s);

@@ -48,7 +48,7 @@ int choose_nsplit(int64_t cap, int warps, int64_t pairs, int64_t nchunk) {
 
 struct DecodePlan {
     int G = 0;
-    DecPath path = DecPath::SIMT;
+    bool use_mma = false;
     int nsplit = 0;
     int64_t split_tokens = 0;
     size_t off_qp = 0, off_up = 0, off_ml = 0, off_acc = 0, bytes = 0;
@@ -68,13 +68,13 @@ bool make_plan(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t T
     if (!h || B < 0 || Hq <= 0 || Hkv <= 0 || Tmax < 0 || Hq % Hkv) return false;
     const int d = h->d;
     p->G = (int)(Hq / Hkv);
-    p->path = decode_path(d, p->G, h->force_simt != 0);
-    const int64_t pairs = B * Hkv > 0 ? B * Hkv * decode_head_groups(p->path, p->G) : 1;
-    const int64_t cap = (int64_t)h->num_sms * decode_ctas_per_sm(p->path);
-    const int chunk = decode_chunk_tokens(d, p->path);
+    p->use_mma = !h->force_simt && mma_supported(d, p->G);
+    const int64_t pairs = B * Hkv > 0 ? B * Hkv * decode_head_groups(p->use_mma, p->G) : 1;
+    const int64_t cap = (int64_t)h->num_sms * decode_ctas_per_sm(p->use_mma);
+    const int chunk = decode_chunk_tokens(d, p->use_mma);
     const int64_t nchunk = Tmax > 0 ? (Tmax + chunk - 1) / chunk : 1;
     p->nsplit = upper_bound ? (int)split_loop_bound(cap, pairs, nchunk)
-                            : choose_nsplit(cap, decode_warps(p->path, p->G), pairs, nchunk);
+                            : choose_nsplit(cap, decode_warps(p->use_mma, p->G), pairs, nchunk);
     p->split_tokens = ((nchunk + p->nsplit - 1) / p->nsplit) * chunk;
     layout_ws(d, (size_t)(B * Hq), p->nsplit, p);
     return true;
@@ -119,13 +119,12 @@ tq_status prepare_encode(const tq_handle* h, const void* x, tq_dtype dt, int64_t
 }
 
 tq_status encode_common(const tq_handle* h, const void* x, tq_dtype dt, int64_t B, int64_t Hkv, int64_t Tnew,
-                        int64_t sb, int64_t sh, int64_t st, const tq_cache* c, int64_t t0, void* stream,
-                        EncKind kind) {
+                        int64_t sb, int64_t sh, int64_t st, const tq_cache* c, int64_t t0, void* stream, bool is_k) {
     EncArgs a;
     bool empty;
     const tq_status r = prepare_encode(h, x, dt, B, Hkv, Tnew, sb, sh, st, c, t0, &a, &empty);
     if (r != TQ_OK || empty) return r;
-    return cuda_status(launch_encode(h->d, kind, dt, a, h->num_sms, false, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_encode(h->d, is_k, dt, a, h->num_sms, false, static_cast<cudaStream_t>(stream)));
 }
 
 // Checks of an attention call and its kernel arguments; *G receives the group size.
@@ -138,9 +137,8 @@ tq_status prepare_attend(const tq_handle* h, const void* q, tq_dtype qdt, int64_
     const int64_t Hkv = kc->Hkv;
     if (Hq % Hkv) return TQ_ERR_INVALID_ARG;
     const int64_t G = Hq / Hkv;
-    // grid limits: y = kv heads x query-head groups (groups of 4 or more), z = batch;
-    // one combine CTA per query head
-    if (B > 65535 || Hkv * ((G + 3) / 4) > 65535 || B * Hq >= ((int64_t)1 << 31)) return TQ_ERR_UNSUPPORTED;
+    // grid limits: y = kv heads x query-head groups, z = batch; one combine CTA per query head
+    if (B > 65535 || Hkv * ((G + 7) / 8) > 65535 || B * Hq >= ((int64_t)1 << 31)) return TQ_ERR_UNSUPPORTED;
     if (!seq_lens && (T < 0 || T > kc->Tcap)) return TQ_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return TQ_ERR_INVALID_ARG;
     if (B == 0) return TQ_OK;
@@ -186,7 +184,7 @@ cudaError_t launch_attend(const tq_handle* h, const void* q, tq_dtype qdt, const
     cudaError_t e = launch_prologue(h->d, q, qdt, BHq, h->dsign, h->dST, const_cast<float*>(a.qp),
                                     const_cast<float*>(a.up), chained, s);
     if (e == cudaSuccess && h->ev_start) e = cudaEventRecord(h->ev_start, s);
-    if (e == cudaSuccess) e = launch_decode(h->d, p.G, p.path, qjl, a, s);
+    if (e == cudaSuccess) e = launch_decode(h->d, p.G, p.use_mma, qjl, a, s);
     if (e == cudaSuccess && h->ev_stop) e = cudaEventRecord(h->ev_stop, s);
     if (e == cudaSuccess) e = launch_combine(h->d, BHq, p.nsplit, a.part_ml, a.part_acc, h->dsign, out, s);
     return e;
@@ -243,29 +241,6 @@ tq_status tq_init(int head_dim, uint64_t seed, tq_handle** out) {
     }
     h->cb.lut_lo[0] = lo[0]; h->cb.lut_lo[1] = lo[1];
     h->cb.lut_hi[0] = hi[0]; h->cb.lut_hi[1] = hi[1];
-    // the centroids as exact integers times 2^-s (smallest such s), split into
-    // signed byte limbs c = 2^-s (256 hi + lo)
-    {
-        int sc = 0;
-        for (; sc < 24; ++sc) {
-            bool whole = true;
-            for (int k = 0; k < 8; ++k) {
-                const double v = std::ldexp((double)h->hc[k], sc);
-                whole &= v == std::nearbyint(v);
-            }
-            if (whole) break;
-        }
-        uint32_t ilo[2] = {0, 0}, ihi[2] = {0, 0};
-        for (int k = 0; k < 8; ++k) {
-            const int v = (int)std::nearbyint(std::ldexp((double)h->hc[k], sc));
-            const int l8 = ((v + 128) & 255) - 128, h8 = (v - l8) / 256;
-            ilo[k >> 2] |= (uint32_t)(uint8_t)(int8_t)l8 << (8 * (k & 3));
-            ihi[k >> 2] |= (uint32_t)(uint8_t)(int8_t)h8 << (8 * (k & 3));
-        }
-        h->cb.ilut_lo[0] = ilo[0]; h->cb.ilut_lo[1] = ilo[1];
-        h->cb.ilut_hi[0] = ihi[0]; h->cb.ilut_hi[1] = ihi[1];
-        h->cb.iscale = (float)std::ldexp(1.0, -sc);
-    }
     for (int k = 0; k < 32; ++k) h->cb.pow2[k] = 1u << k;
 
     std::vector<float> sign(d), st((size_t)d * d), sthr((size_t)d * d);
@@ -342,17 +317,12 @@ int tq_head_dim(const tq_handle* h) { return h ? h->d : 0; }
 
 tq_status tq_encode_k(const tq_handle* h, const void* x, tq_dtype dt, int64_t B, int64_t Hkv, int64_t Tnew,
                       int64_t sb, int64_t sh, int64_t st, const tq_cache* kc, int64_t t0, void* stream) {
-    return encode_common(h, x, dt, B, Hkv, Tnew, sb, sh, st, kc, t0, stream, EncKind::K);
-}
-
-tq_status tq_encode_k_polar(const tq_handle* h, const void* x, tq_dtype dt, int64_t B, int64_t Hkv, int64_t Tnew,
-                            int64_t sb, int64_t sh, int64_t st, const tq_cache* kc, int64_t t0, void* stream) {
-    return encode_common(h, x, dt, B, Hkv, Tnew, sb, sh, st, kc, t0, stream, EncKind::PolarK);
+    return encode_common(h, x, dt, B, Hkv, Tnew, sb, sh, st, kc, t0, stream, true);
 }
 
 tq_status tq_encode_v(const tq_handle* h, const void* x, tq_dtype dt, int64_t B, int64_t Hkv, int64_t Tnew,
                       int64_t sb, int64_t sh, int64_t st, const tq_cache* vc, int64_t t0, void* stream) {
-    return encode_common(h, x, dt, B, Hkv, Tnew, sb, sh, st, vc, t0, stream, EncKind::V);
+    return encode_common(h, x, dt, B, Hkv, Tnew, sb, sh, st, vc, t0, stream, false);
 }
 
 size_t tq_attend_workspace_bytes(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t Tmax) {
@@ -421,7 +391,7 @@ tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype qdt, int
 
 const char* tq_attend_path(const tq_handle* h, int64_t Hq, int64_t Hkv) {
     if (!h || Hq <= 0 || Hkv <= 0 || Hq % Hkv) return "invalid";
-    return decode_path_name(decode_path(h->d, (int)(Hq / Hkv), h->force_simt != 0));
+    return (!h->force_simt && mma_supported(h->d, (int)(Hq / Hkv))) ? "mma" : "simt";
 }
 
 tq_status tq_attend_decode(const tq_handle* h, const void* q, tq_dtype qdt, int64_t B, int64_t Hq,
@@ -467,8 +437,8 @@ tq_status tq_append_attend(const tq_handle* h, const void* k_new, const void* v_
         // programmatic dependents (each completes only after its predecessor);
         // the split-K kernel prefetches every chunk but the appended tokens'
         // before it waits.
-        e = launch_encode(h->d, EncKind::K, kv_dtype, ek, h->num_sms, false, s);
-        if (e == cudaSuccess) e = launch_encode(h->d, EncKind::V, kv_dtype, ev, h->num_sms, true, s);
+        e = launch_encode(h->d, true, kv_dtype, ek, h->num_sms, false, s);
+        if (e == cudaSuccess) e = launch_encode(h->d, false, kv_dtype, ev, h->num_sms, true, s);
         a.fresh_lo = t0;
         a.fresh_hi = t0 + Tnew;
     }

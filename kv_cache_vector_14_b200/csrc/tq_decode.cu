@@ -210,10 +210,7 @@ __global__ void __launch_bounds__(128) tq_decode_simt_kernel(const DecArgs a, in
         for (int r = 0; r < R; ++r) {
             const int j = lane + 32 * r;
             const float ck = sC[code_from_words<D>(kw, j)];
-            if constexpr (v_rows(D))        // V code rows: row j holds coordinate j's token codes
-                cv[r] = sC[code_from_words<64>(reinterpret_cast<const uint32_t*>(vb + (int64_t)j * kVRowB), tau)];
-            else
-                cv[r] = sC[code_from_words<D>(vw, j)];
+            cv[r] = sC[code_from_words<D>(vw, j)];
             if constexpr (QJL) {
                 const float sg = sign_from_words<D>(sw, j) ? gk : -gk;
 #pragma unroll
@@ -410,37 +407,22 @@ cudaError_t launch_decode_mma(int d, int G, bool qjl, const DecArgs& a, cudaStre
 int decode_mma_chunk_tokens(int d);
 int decode_mma_warps(int G);
 
-// The mma.sync kernel covers head_dim 64 and 256 (token-record V blocks) and
-// any group size (query heads in CTAs of up to 8 per kv head).
-bool mma_supported(int d, int G) { return (d == 64 || d == 256) && G >= 1; }
-
-DecPath decode_path(int d, int G, bool force_simt) {
-    if (force_simt || G < 1) return DecPath::SIMT;
-    if (d == 128) return DecPath::TC;
-    return mma_supported(d, G) ? DecPath::MMA : DecPath::SIMT;
-}
-
-const char* decode_path_name(DecPath p) {
-    return p == DecPath::TC ? "tc" : (p == DecPath::MMA ? "mma" : "simt");
-}
+// The tensor-core kernel covers head_dim 64, 128 and 256 and any group size
+// (query heads in CTAs of up to 8 per kv head).
+bool mma_supported(int d, int G) { return head_dim_ok(d) && G >= 1; }
 
 // CTAs per (split, kv head, batch): query-head groups of the kernel that runs.
-int decode_head_groups(DecPath p, int G) {
-    const int per = p == DecPath::TC ? decode_tc_heads() : (p == DecPath::MMA ? 8 : simt_heads_per_cta(G));
+int decode_head_groups(bool use_mma, int G) {
+    const int per = use_mma ? 8 : simt_heads_per_cta(G);
     return (G + per - 1) / per;
 }
 
-int decode_ctas_per_sm(DecPath p) { return p == DecPath::TC ? 2 : (p == DecPath::MMA ? 1 : 4); }
-int decode_chunk_tokens(int d, DecPath p) {
-    return p == DecPath::TC ? decode_tc_tile_tokens() : (p == DecPath::MMA ? decode_mma_chunk_tokens(d) : kBlockT);
-}
-// a tcgen05 CTA walks its tiles one after another; an mma.sync CTA's warps and
-// a SIMT CTA's four warps walk theirs side by side
-int decode_warps(DecPath p, int G) { return p == DecPath::TC ? 1 : (p == DecPath::MMA ? decode_mma_warps(G) : 4); }
+int decode_ctas_per_sm(bool use_mma) { return use_mma ? 1 : 4; }
+int decode_chunk_tokens(int d, bool use_mma) { return use_mma ? decode_mma_chunk_tokens(d) : kBlockT; }
+int decode_warps(bool use_mma, int G) { return use_mma ? decode_mma_warps(G) : 4; }
 
-cudaError_t launch_decode(int d, int G, DecPath path, bool qjl, const DecArgs& a, cudaStream_t s) {
-    if (path == DecPath::TC) return launch_decode_tc(d, G, qjl, a, s);
-    return path == DecPath::MMA ? launch_decode_mma(d, G, qjl, a, s) : launch_decode_simt(d, G, qjl, a, s);
+cudaError_t launch_decode(int d, int G, bool use_mma, bool qjl, const DecArgs& a, cudaStream_t s) {
+    return use_mma ? launch_decode_mma(d, G, qjl, a, s) : launch_decode_simt(d, G, qjl, a, s);
 }
 
 }  // namespace tqi

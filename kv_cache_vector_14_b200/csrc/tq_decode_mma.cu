@@ -504,9 +504,9 @@ template <bool QJL>
 cudaError_t launch_mma_q(int d, int G, const DecArgs& a, cudaStream_t s) {
     if (d == 64)
         return G <= 4 ? launch_mma_t<64, 1, kNW1, QJL>(a, G, s) : launch_mma_t<64, 2, kNW2, QJL>(a, G, s);
-    if (d == 256)
-        return G <= 4 ? launch_mma_t<256, 1, kNW1, QJL>(a, G, s) : launch_mma_t<256, 2, kNW2, QJL>(a, G, s);
-    return cudaErrorInvalidValue;         // head_dim 128 (V code rows) runs on the tcgen05 kernel
+    if (d == 128)
+        return G <= 4 ? launch_mma_t<128, 1, kNW1, QJL>(a, G, s) : launch_mma_t<128, 2, kNW2, QJL>(a, G, s);
+    return G <= 4 ? launch_mma_t<256, 1, kNW1, QJL>(a, G, s) : launch_mma_t<256, 2, kNW2, QJL>(a, G, s);
 }
 
 cudaError_t launch_decode_mma(int d, int G, bool qjl, const DecArgs& a, cudaStream_t s) {
@@ -515,7 +515,9 @@ cudaError_t launch_decode_mma(int d, int G, bool qjl, const DecArgs& a, cudaStre
     return qjl ? launch_mma_q<true>(d, G, a, s) : launch_mma_q<false>(d, G, a, s);
 }
 
-int decode_mma_chunk_tokens(int d) { return d == 64 ? Cfg<64>::kChunk : Cfg<256>::kChunk; }
+int decode_mma_chunk_tokens(int d) {
+    return d == 64 ? Cfg<64>::kChunk : d == 128 ? Cfg<128>::kChunk : Cfg<256>::kChunk;
+}
 int decode_mma_warps(int G) { return G <= 4 ? kNW1 : kNW2; }
 
 }  // namespace tqi

@@ -459,10 +459,8 @@ cudaError_t launch_enc_dt(tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, 
 
 }  // namespace
 
-cudaError_t launch_encode(int d, EncKind kind, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl,
-                          cudaStream_t s) {
-    if (d == 128) return launch_encode128(kind, dt, a, num_sms, pdl, s);
-    const bool is_k = kind == EncKind::K;     // head_dim 64 and 256: V and PolarQuant-only K blocks are alike
+cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
+    if (d == 128) return launch_encode128(is_k, dt, a, num_sms, pdl, s);
     if (d == 64)
         return is_k ? launch_enc_dt<64, true>(dt, a, num_sms, pdl, s) : launch_enc_dt<64, false>(dt, a, num_sms, pdl, s);
     if (d == 256)

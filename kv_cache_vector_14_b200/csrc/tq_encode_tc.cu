@@ -505,8 +505,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
     pdl_wait();                    // when chained: complete only after the previous kernel
 }
 
-// ---------------------------------------------------------------- V flow into token records
-// (PolarQuant-only K blocks): four vectors per warp, codes packed per token.
+// ---------------------------------------------------------------- V kernel
 constexpr int kVWarps = 8;
 
 template <int DT>
@@ -541,112 +540,11 @@ __global__ void __launch_bounds__(kVWarps * 32, 3) tq_encode_v128_kernel(const E
     pdl_wait();
 }
 
-// ---------------------------------------------------------------- V kernel, coordinate rows
-// head_dim 128 V blocks hold one 24-byte row per coordinate (the codes of the
-// block's 64 tokens).  One CTA of 8 warps per unit = (sequence, cache block):
-// steps 1-3 for the unit's tokens (at most 64; group gi = 4 warp + g takes the
-// unit's tokens gi and gi + 32) with the codes staged in shared memory, one
-// 128-byte slot-order record per token; the norms are stored directly.  Then
-// thread j builds row j from the staged codes of coordinate j and stores its
-// six words.  A block that the encode covers only in part keeps the bits of
-// its other tokens: the row is read, those bits are kept under a mask and the
-// new tokens' bits merged in.  One CTA owns a block for the whole launch.
-constexpr int kVRowWarps = 8;
-
-// Put 3-bit value c of token tau into the six words of a row (the head_dim-64
-// record rule with token tau as coordinate tau).
-__device__ __forceinline__ void vrow_put(uint32_t (&w)[6], int tau, uint32_t c) {
-    const int t = slot_of(tau), i = slot_pos(tau);
-    const int hw = 4 + (t >> 1), hs = 16 * (t & 1);
-    if (i < 8) {
-        w[t] |= c << (4 * i);
-    } else if (i < 12) {
-        w[hw] |= c << (hs + 4 * (i - 8));
-    } else {
-        const int k = i - 12;
-        w[t] |= (c & 1u) << (4 * k + 3);
-        w[t] |= ((c >> 1) & 1u) << (4 * (4 + k) + 3);
-        w[hw] |= ((c >> 2) & 1u) << (hs + 4 * k + 3);
-    }
-}
-
 template <int DT>
-__global__ void __launch_bounds__(kVRowWarps * 32) tq_encode_v128_rows_kernel(const EncArgs a, int64_t nblk) {
-    __shared__ __align__(16) uint8_t scode[kBlockT][128];     // [token of the block][slot order]
-    pdl_trigger();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 3, l = lane & 7;
-    const int64_t units = a.B * a.Hkv * nblk;
-    const int64_t bb = block_bytes(kD, false);
-    const int64_t blk0 = a.t0 >> 6;
-    float dsg[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) dsg[i] = __ldg(a.dsign + 16 * l + i);
-    const bool vec = a.vec16 != 0;
-    for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
-        const int64_t bh = u / nblk, blk = blk0 + (u - bh * nblk);
-        const int64_t lo = a.t0 > blk * kBlockT ? a.t0 : blk * kBlockT;
-        const int64_t hi = (a.t0 + a.Tnew < (blk + 1) * kBlockT) ? a.t0 + a.Tnew : (blk + 1) * kBlockT;
-        const int n = (int)(hi - lo), tau0 = (int)(lo - blk * kBlockT);
-        const int64_t pb = cache_block(a.table, a.pool, a.NB, bh, blk, a.err);
-        uint8_t* base = pb >= 0 ? a.cache + pb * bb : nullptr;      // null: nothing is written
-        const int64_t b = bh / a.Hkv, hh = bh - b * a.Hkv;
-#pragma unroll
-        for (int pass = 0; pass < 2; ++pass) {
-            const int k0 = 32 * pass + 4 * warp;
-            if (k0 >= n) break;                               // warp-uniform
-            const int k = k0 + g;
-            const bool valid = k < n;
-            const int64_t tt = lo - a.t0 + (valid ? k : k0);
-            GroupOut o;
-            encode_group<DT, false>(a.x, b * a.sb + hh * a.sh + tt * a.st, valid, vec, l, dsg, a.cb, o);
-            if (valid) {
-#pragma unroll
-                for (int t = 0; t < 4; ++t) *reinterpret_cast<uint32_t*>(&scode[tau0 + k][t * 32 + 4 * l]) = o.cw[t];
-                if (l == 0 && base) reinterpret_cast<__half*>(base + kD * kVRowB)[tau0 + k] = __float2half_rn(o.n);
-            }
-        }
-        __syncthreads();
-        if (threadIdx.x < kD && base) {
-            const int j = threadIdx.x;
-            const int off = slot_of(j) * 32 + slot_pos(j);           // coordinate j in a staged record
-            uint32_t w[6] = {0u, 0u, 0u, 0u, 0u, 0u}, m[6] = {0u, 0u, 0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int tau = 0; tau < kBlockT; ++tau) {
-                const bool in = tau >= tau0 && tau < tau0 + n;
-                vrow_put(w, tau, in ? (uint32_t)scode[tau][off] : 0u);
-                vrow_put(m, tau, in ? 7u : 0u);
-            }
-            uint2* row = reinterpret_cast<uint2*>(base + (int64_t)j * kVRowB);
-            if (n < kBlockT) {
-#pragma unroll
-                for (int q = 0; q < 3; ++q) {
-                    const uint2 old = row[q];
-                    w[2 * q] |= old.x & ~m[2 * q];
-                    w[2 * q + 1] |= old.y & ~m[2 * q + 1];
-                }
-            }
-#pragma unroll
-            for (int q = 0; q < 3; ++q) row[q] = make_uint2(w[2 * q], w[2 * q + 1]);
-        }
-        __syncthreads();
-    }
-    pdl_wait();
-}
-
-template <int DT>
-cudaError_t launch_t(EncKind kind, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
+cudaError_t launch_t(bool is_k, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
     const int64_t N = a.B * a.Hkv * a.Tnew;
     if (N <= 0) return cudaSuccess;
-    if (kind == EncKind::V) {
-        const int64_t nblk = ((a.t0 + a.Tnew - 1) >> 6) - (a.t0 >> 6) + 1;
-        const int64_t units = a.B * a.Hkv * nblk;
-        const int64_t cap = (int64_t)num_sms * 8;
-        const unsigned grid = (unsigned)(units < cap ? units : cap);
-        if (pdl) return launch_pdl(tq_encode_v128_rows_kernel<DT>, dim3(grid), dim3(kVRowWarps * 32), 0, s, a, nblk);
-        tq_encode_v128_rows_kernel<DT><<<grid, kVRowWarps * 32, 0, s>>>(a, nblk);
-        return cudaGetLastError();
-    }
-    if (kind == EncKind::K) {
+    if (is_k) {
         // rows per tile: enough tiles to cover the SMs, multiples of 4, at most 128
         int64_t rows = (N + num_sms - 1) / num_sms;
         rows = ((rows + 3) / 4) * 4;
@@ -671,11 +569,11 @@ cudaError_t launch_t(EncKind kind, const EncArgs& a, int num_sms, bool pdl, cuda
 
 }  // namespace
 
-cudaError_t launch_encode128(EncKind kind, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
+cudaError_t launch_encode128(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
     switch (dt) {
-        case TQ_F32: return launch_t<TQ_F32>(kind, a, num_sms, pdl, s);
-        case TQ_BF16: return launch_t<TQ_BF16>(kind, a, num_sms, pdl, s);
-        case TQ_F16: return launch_t<TQ_F16>(kind, a, num_sms, pdl, s);
+        case TQ_F32: return launch_t<TQ_F32>(is_k, a, num_sms, pdl, s);
+        case TQ_BF16: return launch_t<TQ_BF16>(is_k, a, num_sms, pdl, s);
+        case TQ_F16: return launch_t<TQ_F16>(is_k, a, num_sms, pdl, s);
     }
     return cudaErrorInvalidValue;
 }

@@ -30,11 +30,7 @@ struct Cfg {
     static constexpr int kOffKn = kOffKs + (QJL ? kChunk * kSignB : 0);
     static constexpr int kOffKg = kOffKn + 2 * kChunk;
     static constexpr int kOffVc = kOffKg + (QJL ? 2 * kChunk : 0);
-    // V codes: the chunk's token records, or (head_dim 128) the block's whole
-    // coordinate rows (a row mixes the bits of all 64 tokens)
-    static constexpr bool kVRows = v_rows(D);
-    static constexpr int kVcB = kVRows ? D * kVRowB : kChunk * kCodeB;
-    static constexpr int kOffVn = kOffVc + kVcB;
+    static constexpr int kOffVn = kOffVc + kChunk * kCodeB;
     static constexpr int kStageB = kOffVn + 2 * kChunk;
     static constexpr bool kBRegs = D <= 128;                   // q'/u' fragments in registers
     static_assert(kStageB % 16 == 0 && kOffKn % 16 == 0 && kOffKg % 16 == 0 && kOffVc % 16 == 0 &&
@@ -172,17 +168,6 @@ __device__ __forceinline__ void token_selectors(const uint8_t* tok, int sl, int 
 // 16-bit halfword h of slot t as h | h << 20 (m64 = 2^20 + 1), so that byte e
 // of the word has h's bits 4e' .. 4e'+3 in its bits 4..7 (e' = 1, 3, 0, 2 for
 // e = 0..3) and the shifts of the d >= 128 extraction pick every bit once.
-// head_dim 128 V code row (six words): the prmt selector of the 4 codes of
-// 16-token group q (tokens 16 q + 2t, 2t + 1, 2t + 8, 2t + 9) of slot t.
-__device__ __forceinline__ uint32_t vrow_selector(const uint8_t* row, int t, int q) {
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(row + 4 * t);
-    if (q == 0) return w & 0x7777u;
-    if (q == 1) return (w >> 16) & 0x7777u;
-    const uint32_t h = *reinterpret_cast<const uint16_t*>(row + 16 + 2 * t);
-    if (q == 2) return h & 0x7777u;
-    return ((w >> 3) & 0x1111u) | ((w >> 18) & 0x2222u) | ((h >> 1) & 0x4444u);
-}
-
 template <int D>
 __device__ __forceinline__ uint32_t token_signs(const uint8_t* tok, int sl, int t, uint32_t m64) {
     if constexpr (D == 64) return (uint32_t)*reinterpret_cast<const uint16_t*>(tok + 2 * t) * m64;

@@ -26,11 +26,6 @@ struct Codebook {
     uint32_t lut_lo[2]; // low bytes of the fp16 bit patterns of c[0..7]
     uint32_t lut_hi[2]; // high bytes of the fp16 bit patterns of c[0..7]
     uint32_t pow2[32];  // 1 << k: shifts done as integer multiplies (FMA pipe, not ALU)
-    // head_dim 128 tensor-core decode: c[k] = iscale * (256 hi[k] + lo[k]) exactly,
-    // hi and lo signed bytes (lo in [-128, 127]); byte look-up tables as above
-    uint32_t ilut_lo[2];
-    uint32_t ilut_hi[2];
-    float iscale;
 };
 
 // Host-side generation of the constants (tq_params.cpp).
@@ -82,13 +77,6 @@ __host__ __device__ inline int sign_row(int d, int r, int l) {
     return slot_coord(r >> 2, r & 3, l < 16 ? 2 * l : 2 * (l - 16) + 1);
 }
 __host__ __device__ inline bool head_dim_ok(int d) { return d == 64 || d == 128 || d == 256; }
-
-// head_dim 128 V blocks: d code rows of 24 bytes (six words), row j holding
-// the codes of coordinate j for the block's 64 tokens, packed as a head_dim-64
-// token record packs 64 coordinates (token tau in the place of coordinate tau:
-// slot (tau >> 1) & 3, position slot_pos(tau)).
-constexpr int kVRowB = 24;
-__host__ __device__ constexpr bool v_rows(int d) { return d == 128; }
 
 // Division by a fixed divisor d >= 1 for dividends below 2^31:
 // q = umulhi(n, m) >> s with m = ceil(2^(31 + ceil(log2 d)) / d); m = 0 marks d = 1.
@@ -201,15 +189,10 @@ cudaError_t set_smem_once(int bytes) {
     return e;
 }
 
-// What an encode writes: the K flow into K blocks, the V flow into V blocks
-// (coordinate rows at head_dim 128, token records otherwise), or the V flow
-// into PolarQuant-only K blocks (token records).
-enum class EncKind { K, V, PolarK };
-
 // Kernel launchers (tq_encode.cu, tq_decode.cu); return a CUDA error code.
-cudaError_t launch_encode(int d, EncKind kind, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl,
+cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl,
                           cudaStream_t s);
-cudaError_t launch_encode128(EncKind kind, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s);
+cudaError_t launch_encode128(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s);
 // pdl: launched as a programmatic dependent of the previous kernel (fused
 // append-and-attend step); the kernels then complete only after it.
 cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, const float* dsign,
@@ -217,24 +200,15 @@ cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, cons
 // Chunked prefill (head_dim 128): rows (b, i, head) of Lq queries per sequence,
 // query i over tokens [0, T0 + i]; partials as one split of a.part_ml/part_acc.
 cudaError_t launch_prefill(int d, int G, const DecArgs& a, int64_t Lq, int64_t T0, cudaStream_t s);
-// Split-K decode kernels: tcgen05 (head_dim 128), mma.sync (head_dim 64 and
-// 256), SIMT (any head_dim; the cross-check path).
-enum class DecPath { SIMT, MMA, TC };
-DecPath decode_path(int d, int G, bool force_simt);
-const char* decode_path_name(DecPath p);
-// qjl = false: PolarQuant-only K cache (codes and norms), scores without the QJL term.
-cudaError_t launch_decode(int d, int G, DecPath path, bool qjl, const DecArgs& a, cudaStream_t s);
+// qjl = false: PolarQuant-only K cache (V layout), scores without the QJL term.
+cudaError_t launch_decode(int d, int G, bool use_mma, bool qjl, const DecArgs& a, cudaStream_t s);
 cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml,
                            const float* part_acc, const float* dsign, float* out, cudaStream_t s);
 bool mma_supported(int d, int G);
-// head_dim 128: the tcgen05 kernel (tq_decode_tc.cu)
-cudaError_t launch_decode_tc(int d, int G, bool qjl, const DecArgs& a, cudaStream_t s);
-int decode_tc_heads();
-int decode_tc_tile_tokens();
-int decode_ctas_per_sm(DecPath p);
-int decode_chunk_tokens(int d, DecPath p);   // split ranges are multiples of this
-int decode_warps(DecPath p, int G);          // independent token streams sharing one split
-int decode_head_groups(DecPath p, int G);    // CTAs per (split, kv head, batch)
+int decode_ctas_per_sm(bool use_mma);
+int decode_chunk_tokens(int d, bool use_mma);   // split ranges are multiples of this
+int decode_warps(bool use_mma, int G);   // warps sharing one split
+int decode_head_groups(bool use_mma, int G);   // CTAs per (split, kv head, batch)
 
 }  // namespace tqi
 

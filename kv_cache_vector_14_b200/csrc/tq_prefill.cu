@@ -118,8 +118,7 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillA
         bulk_g2s(smem_u32(st + PC::kOffKs), kb + 64 * cb + sub * ch * sb, ch * sb, bar);
         bulk_g2s(smem_u32(st + PC::kOffKn), kb + 64 * (cb + sb) + sub * 2 * ch, 2 * ch, bar);
         bulk_g2s(smem_u32(st + PC::kOffKg), kb + 64 * (cb + sb) + 128 + sub * 2 * ch, 2 * ch, bar);
-        if constexpr (PC::kVRows) bulk_g2s(smem_u32(st + PC::kOffVc), vb, PC::kVcB, bar);
-        else bulk_g2s(smem_u32(st + PC::kOffVc), vb + sub * ch * cb, ch * cb, bar);
+        bulk_g2s(smem_u32(st + PC::kOffVc), vb + sub * ch * cb, ch * cb, bar);
         bulk_g2s(smem_u32(st + PC::kOffVn), vb + 64 * cb + sub * 2 * ch, 2 * ch, bar);
     };
     if (lane == 0)
@@ -315,35 +314,20 @@ __global__ void __launch_bounds__(kPW * 32) tq_prefill_mma_kernel(const PrefillA
             split_hilo(pv[0][2], pv[0][3], pH[1], pL[1]);
             split_hilo(pv[1][0], pv[1][1], pH[2], pL[2]);
             split_hilo(pv[1][2], pv[1][3], pH[3], pL[3]);
-            // ---------------- values: O[16 rows][8 coords] += P Vdeq
-            if constexpr (PC::kVRows) {
-                // B fragment of coordinate n-tile nc straight from V code rows: lane (g, t)
-                // takes row 8 nc + g, tokens 2t, 2t + 1 (b0) and 2t + 8, 2t + 9 (b1) of the
-                // tile's 16-token group of the block
-                const int q = (int)((tok0 & 63) >> 4) + kt;
+            // ---------------- values: O[16 rows][8 coords] += P Vdeq, Vdeq^T by movmatrix
+            token_selectors<D>(st + PC::kOffVc + tA * PC::kCodeB, vh, tq4, pw, selA[0]);
+            token_selectors<D>(st + PC::kOffVc + tB * PC::kCodeB, vh, tq4, pw, selB[0]);
 #pragma unroll
-                for (int nc = 0; nc < 2 * kVKC; ++nc) {
-                    uint32_t b0, b1;
-                    dequant4(vrow_selector(st + PC::kOffVc + (8 * nc + gr) * kVRowB, tq4, q), lut, b0, b1);
-                    mma16816(o[nc], pH, b0, b1);
-                    mma16816(o[nc], pL, b0, b1);
-                }
-            } else {
-                // Vdeq^T by movmatrix from token-record fragments
-                token_selectors<D>(st + PC::kOffVc + tA * PC::kCodeB, vh, tq4, pw, selA[0]);
-                token_selectors<D>(st + PC::kOffVc + tB * PC::kCodeB, vh, tq4, pw, selB[0]);
-#pragma unroll
-                for (int kc = 0; kc < kVKC; ++kc) {
-                    uint32_t x0, x1, y0, y1;
-                    dequant4(sel_for(selA[0], pw, kc), lut, x0, x1);   // tokens 0..7 of the tile
-                    dequant4(sel_for(selB[0], pw, kc), lut, y0, y1);   // tokens 8..15
-                    const uint32_t mx0 = movmatrix_t(x0), mx1 = movmatrix_t(x1);
-                    const uint32_t my0 = movmatrix_t(y0), my1 = movmatrix_t(y1);
-                    mma16816(o[2 * kc], pH, mx0, my0);
-                    mma16816(o[2 * kc], pL, mx0, my0);
-                    mma16816(o[2 * kc + 1], pH, mx1, my1);
-                    mma16816(o[2 * kc + 1], pL, mx1, my1);
-                }
+            for (int kc = 0; kc < kVKC; ++kc) {
+                uint32_t x0, x1, y0, y1;
+                dequant4(sel_for(selA[0], pw, kc), lut, x0, x1);   // tokens 0..7 of the tile
+                dequant4(sel_for(selB[0], pw, kc), lut, y0, y1);   // tokens 8..15
+                const uint32_t mx0 = movmatrix_t(x0), mx1 = movmatrix_t(x1);
+                const uint32_t my0 = movmatrix_t(y0), my1 = movmatrix_t(y1);
+                mma16816(o[2 * kc], pH, mx0, my0);
+                mma16816(o[2 * kc], pL, mx0, my0);
+                mma16816(o[2 * kc + 1], pH, mx1, my1);
+                mma16816(o[2 * kc + 1], pL, mx1, my1);
             }
         }
         __syncwarp();

@@ -21,7 +21,7 @@ TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA, TQ_ERR_WORKSPACE, TQ
 TQ_F32, TQ_BF16, TQ_F16 = 0, 1, 2
 
 EXPORTED = ("tq_params_host", "tq_init", "tq_destroy", "tq_get_params", "tq_head_dim", "tq_block_bytes",
-            "tq_cache_bytes", "tq_encode_k", "tq_encode_v", "tq_encode_k_polar", "tq_attend_workspace_bytes", "tq_attend_decode",
+            "tq_cache_bytes", "tq_encode_k", "tq_encode_v", "tq_attend_workspace_bytes", "tq_attend_decode",
             "tq_append_attend", "tq_prefill_workspace_bytes", "tq_attend_prefill", "tq_attend_decode_polar",
             "tq_attend_decode_static", "tq_device_status", "tq_set_decode_events", "tq_set_decode_path", "tq_set_wait_limit", "tq_attend_path",
             "tq_status_string")
@@ -65,7 +65,7 @@ def lib() -> C.CDLL:
             L.tq_block_bytes.restype = C.c_size_t
             L.tq_cache_bytes.argtypes = [i32, i32, i64, i64, i64]
             L.tq_cache_bytes.restype = C.c_size_t
-            for name in ("tq_encode_k", "tq_encode_v", "tq_encode_k_polar"):
+            for name in ("tq_encode_k", "tq_encode_v"):
                 f = getattr(L, name)
                 f.argtypes = [P, P, i32, i64, i64, i64, i64, i64, i64, C.POINTER(tq_cache), i64, P]
                 f.restype = st
@@ -182,12 +182,9 @@ class Cache:
     """A compressed K or V cache in a PyTorch-owned uint8 device buffer."""
 
     def __init__(self, head_dim: int, is_k: bool, B: int, Hkv: int, Tcap: int, device="cuda", buf=None,
-                 block_table=None, pool_blocks: int = 0, polar: bool = False):
+                 block_table=None, pool_blocks: int = 0):
         """Contiguous cache, or (block_table: device int32 [B*Hkv, Tcap/64]) a
-        paged cache whose buffer is a pool of pool_blocks blocks.  polar: a
-        PolarQuant-only K cache (is_k False; written by tq_encode_k_polar)."""
-        if polar and is_k:
-            raise ValueError("a PolarQuant-only K cache has the size of a V cache: pass is_k=False, polar=True")
+        paged cache whose buffer is a pool of pool_blocks blocks."""
         import torch
         if block_table is not None:
             if block_table.dtype != torch.int32 or tuple(block_table.shape) != (B * Hkv, Tcap // 64) or \
@@ -199,7 +196,6 @@ class Cache:
         if nbytes == 0 and B * Hkv > 0:
             raise ValueError("Tcap must be a positive multiple of 64 and head_dim 64, 128 or 256")
         self.head_dim, self.is_k, self.B, self.Hkv, self.Tcap = head_dim, is_k, B, Hkv, Tcap
-        self.kind = "k" if is_k else ("polar" if polar else "v")
         self.block_table, self.pool_blocks = block_table, pool_blocks
         self.buf = buf if buf is not None else torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=device)
         table = C.c_void_p(block_table.data_ptr()) if block_table is not None else None
@@ -228,15 +224,7 @@ def tq_encode_k(h, x, kc: Cache, t0: int = 0, stream=None) -> None:
 
 
 def tq_encode_v(h, x, vc: Cache, t0: int = 0, stream=None) -> None:
-    if vc.kind != "v":
-        raise ValueError("tq_encode_v: vc must be a V cache")
     _encode(lib().tq_encode_v, "tq_encode_v", h, x, vc, t0, stream)
-
-
-def tq_encode_k_polar(h, x, kc: Cache, t0: int = 0, stream=None) -> None:
-    if kc.kind != "polar":
-        raise ValueError("tq_encode_k_polar: kc must be a PolarQuant-only K cache (Cache(..., polar=True))")
-    _encode(lib().tq_encode_k_polar, "tq_encode_k_polar", h, x, kc, t0, stream)
 
 
 def tq_attend_workspace_bytes(h, B: int, Hq: int, Hkv: int, Tmax: int) -> int:
@@ -257,12 +245,12 @@ def tq_attend_decode(h, q, kc: Cache, vc: Cache, out, ws, T: int = 0, seq_lens=N
 
 def tq_attend_decode_polar(h, q, kc: Cache, vc: Cache, out, ws, T: int = 0, seq_lens=None, scale: float = 1.0,
                            stream=None) -> None:
-    """Attention with a PolarQuant-only K cache (written by tq_encode_k_polar):
-    scores without the QJL term."""
+    """Attention with a PolarQuant-only K cache (a V-layout cache written by
+    tq_encode_v): scores without the QJL term."""
     if q.dim() != 3 or not q.is_contiguous():
         raise ValueError("tq_attend_decode_polar: q must be contiguous [B, Hq, d]")
-    if kc.kind != "polar":
-        raise ValueError("tq_attend_decode_polar: kc must be a PolarQuant-only K cache (tq_encode_k_polar)")
+    if kc.is_k:
+        raise ValueError("tq_attend_decode_polar: kc must be a V-layout cache (encoded with tq_encode_v)")
     B, Hq, _ = q.shape
     sl = C.c_void_p(seq_lens.data_ptr()) if seq_lens is not None else None
     _check(lib().tq_attend_decode_polar(h, C.c_void_p(q.data_ptr()), _dtype_code(q), B, Hq, C.byref(kc.struct),

@@ -175,42 +175,31 @@ def sketch_given_codes(prm: dict, y, idx, nonzero) -> dict:
     return {"sig": sig, "gamma": g, "gh": to_fp16_bits(g), "z": z}
 
 
-KIND_V, KIND_K, KIND_POLAR_K = 0, 1, 2
+def block_bytes(d: int, is_k: bool) -> int:
+    return int(_L().orc_block_bytes(d, 1 if is_k else 0))
 
 
-def _kind(k) -> int:
-    """Block kind: True / 1 -> K, False / 0 -> V, "polar" / 2 -> PolarQuant-only K."""
-    if isinstance(k, str):
-        return {"k": KIND_K, "v": KIND_V, "polar": KIND_POLAR_K, "polar_k": KIND_POLAR_K}[k]
-    return int(k)
-
-
-def block_bytes(d: int, is_k) -> int:
-    return int(_L().orc_block_bytes(d, _kind(is_k)))
-
-
-def pack(d: int, is_k, t0: int, idx, sig, nh, gh, blocks: np.ndarray) -> None:
-    """Write tokens [t0, t0+T) of one sequence into its block array (uint8, in
-    place).  is_k: the block kind (True K, False V, "polar" PolarQuant-only K)."""
+def pack(d: int, is_k: bool, t0: int, idx, sig, nh, gh, blocks: np.ndarray) -> None:
+    """Write tokens [t0, t0+T) of one sequence into its block array (uint8, in place)."""
     idx = np.ascontiguousarray(idx, dtype=np.uint8)
     T = idx.shape[0]
     sig = np.ascontiguousarray(sig if sig is not None else np.zeros((T, d)), dtype=np.uint8)
     nh = np.ascontiguousarray(nh, dtype=np.uint16)
     gh = np.ascontiguousarray(gh if gh is not None else np.zeros(T), dtype=np.uint16)
     assert blocks.dtype == np.uint8 and blocks.flags["C_CONTIGUOUS"]
-    _L().orc_pack(d, _kind(is_k), t0, T, _p(idx), _p(sig), _p(nh), _p(gh), _p(blocks))
+    _L().orc_pack(d, 1 if is_k else 0, t0, T, _p(idx), _p(sig), _p(nh), _p(gh), _p(blocks))
 
 
-def unpack(d: int, is_k, t0: int, T: int, blocks: np.ndarray) -> dict:
-    """Read tokens [t0, t0+T) of one sequence from its block array (kind as in pack)."""
+def unpack(d: int, is_k: bool, t0: int, T: int, blocks: np.ndarray) -> dict:
+    """Read tokens [t0, t0+T) of one sequence from its block array."""
     blocks = np.ascontiguousarray(blocks, dtype=np.uint8)
     idx = np.zeros((T, d), dtype=np.uint8)
     sig = np.zeros((T, d), dtype=np.uint8)
     nh = np.zeros(T, dtype=np.uint16)
     gh = np.zeros(T, dtype=np.uint16)
-    _L().orc_unpack(d, _kind(is_k), t0, T, _p(blocks), _p(idx), _p(sig), _p(nh), _p(gh))
+    _L().orc_unpack(d, 1 if is_k else 0, t0, T, _p(blocks), _p(idx), _p(sig), _p(nh), _p(gh))
     out = {"idx": idx, "nh": nh}
-    if _kind(is_k) == KIND_K:
+    if is_k:
         out.update(sig=sig, gh=gh)
     return out
 

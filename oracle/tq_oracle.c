@@ -248,19 +248,9 @@ void orc_sketch_given_codes(int d, const double* S, const double* c8, const doub
  * Packed cache layout (this library's own contract; the pages give none
  * beyond the bit budget of 4.25 b/dim for K and 3.125 b/dim for V).
  *
- * A cache is [B][Hkv][Tcap/64 blocks]; one block holds 64 tokens.  Three
- * block kinds:
- *   K block (kind 1): codes 64 x 3d/8 B | signs 64 x d/8 B | n fp16 x 64 |
- *                     gamma fp16 x 64, codes and signs one record per token;
- *   V block (kind 0), head_dim 128: code rows d x 24 B | n fp16 x 64, one row
- *                     per coordinate holding that coordinate's 64 token codes;
- *   V block (kind 0), head_dim 64 and 256, and PolarQuant-only K block
- *                     (kind 2), every head_dim: codes 64 x 3d/8 B | n fp16 x 64,
- *                     the K block without signs and gamma.
- * A V code row packs the codes of tokens tau = 0..63 of one coordinate exactly
- * as a head_dim-64 token record (below) packs the codes of coordinates 0..63:
- * token tau takes the place of coordinate tau (slot t = (tau >> 1) & 3,
- * position i = 4 (tau >> 4) + 2 ((tau >> 3) & 1) + (tau & 1)).
+ * A cache is [B][Hkv][Tcap/64 blocks]; one block holds 64 tokens:
+ *   K block: codes 64 x 3d/8 B | signs 64 x d/8 B | n fp16 x 64 | gamma fp16 x 64
+ *   V block: codes 64 x 3d/8 B | n fp16 x 64
  * Per token, codes are 3d/32 little-endian uint32 words: for slice s (128
  * coordinates) and slot t (0..3) words 12s+3t+{0,1,2} = Wa, Wb, Wc hold slot
  * codes i = 0..31, slot code i meaning coordinate
@@ -280,13 +270,9 @@ void orc_sketch_given_codes(int d, const double* S, const double* c8, const doub
  * of word t / 2) is the sign of the JL row of slot position i.
  * These functions pack/unpack one (b, kv-head) sequence of Tcap slots.
  * ---------------------------------------------------------------------- */
-#define ORC_KIND_V 0
-#define ORC_KIND_K 1
-#define ORC_KIND_POLAR_K 2
-
-int64_t orc_block_bytes(int d, int kind) {
+int64_t orc_block_bytes(int d, int is_k) {
     int64_t codes = (int64_t)ORC_BLOCK_T * 3 * d / 8;
-    if (kind == ORC_KIND_K) return codes + (int64_t)ORC_BLOCK_T * d / 8 + 4 * ORC_BLOCK_T;
+    if (is_k) return codes + (int64_t)ORC_BLOCK_T * d / 8 + 4 * ORC_BLOCK_T;
     return codes + 2 * ORC_BLOCK_T;
 }
 
@@ -415,76 +401,23 @@ static void orc_unpack_signs(int d, const uint32_t* words, uint8_t* sg) {
             }
 }
 
-/* byte offsets of the fields of token tau inside its block (token records) */
+/* byte offsets of the fields of token tau inside its block */
 static int64_t orc_off_codes(int d, int tau) { return (int64_t)tau * 3 * d / 8; }
 static int64_t orc_off_signs(int d, int tau) {
     return (int64_t)ORC_BLOCK_T * 3 * d / 8 + (int64_t)tau * d / 8;
 }
-static int64_t orc_off_norm(int d, int kind, int tau) {
-    int64_t base = (int64_t)ORC_BLOCK_T * 3 * d / 8 + (kind == ORC_KIND_K ? (int64_t)ORC_BLOCK_T * d / 8 : 0);
+static int64_t orc_off_norm(int d, int is_k, int tau) {
+    int64_t base = (int64_t)ORC_BLOCK_T * 3 * d / 8 + (is_k ? (int64_t)ORC_BLOCK_T * d / 8 : 0);
     return base + 2 * tau;
-}
-/* byte offset of the code row of coordinate j inside a V block (6 words each) */
-static int64_t orc_off_vrow(int j) { return (int64_t)j * 24; }
-
-/* V blocks: tokens [t0, t0 + T) of one sequence, one block at a time; each
- * coordinate row is unpacked to its 64 token codes, the tokens in range are
- * replaced, and the row is packed again (the head_dim-64 record packer with
- * token tau in place of coordinate tau). */
-static void orc_pack_v(int d, int64_t t0, int64_t T, const uint8_t* idx, const uint16_t* nh,
-                       uint8_t* blocks) {
-    const int64_t bb = orc_block_bytes(d, ORC_KIND_V);
-    for (int64_t blk = t0 / ORC_BLOCK_T; blk * ORC_BLOCK_T < t0 + T; ++blk) {
-        uint8_t* b = blocks + blk * bb;
-        const int64_t lo = blk * ORC_BLOCK_T > t0 ? blk * ORC_BLOCK_T : t0;
-        const int64_t hi = (blk + 1) * ORC_BLOCK_T < t0 + T ? (blk + 1) * ORC_BLOCK_T : t0 + T;
-        for (int j = 0; j < d; ++j) {
-            uint32_t w[6];
-            uint8_t tok[ORC_BLOCK_T];
-            memcpy(w, b + orc_off_vrow(j), 24);
-            orc_unpack_codes64(w, tok);
-            for (int64_t t = lo; t < hi; ++t) tok[t - blk * ORC_BLOCK_T] = idx[(t - t0) * d + j];
-            orc_pack_codes64(tok, w);
-            memcpy(b + orc_off_vrow(j), w, 24);
-        }
-        for (int64_t t = lo; t < hi; ++t)
-            memcpy(b + (int64_t)d * 24 + 2 * (t - blk * ORC_BLOCK_T), &nh[t - t0], 2);
-    }
-}
-
-static void orc_unpack_v(int d, int64_t t0, int64_t T, const uint8_t* blocks, uint8_t* idx, uint16_t* nh) {
-    const int64_t bb = orc_block_bytes(d, ORC_KIND_V);
-    const int64_t b0 = t0 / ORC_BLOCK_T, b1 = (t0 + T + ORC_BLOCK_T - 1) / ORC_BLOCK_T;
-#pragma omp parallel for schedule(static)
-    for (int64_t blk = b0; blk < b1; ++blk) {
-        const uint8_t* b = blocks + blk * bb;
-        const int64_t lo = blk * ORC_BLOCK_T > t0 ? blk * ORC_BLOCK_T : t0;
-        const int64_t hi = (blk + 1) * ORC_BLOCK_T < t0 + T ? (blk + 1) * ORC_BLOCK_T : t0 + T;
-        for (int j = 0; j < d; ++j) {
-            uint32_t w[6];
-            uint8_t tok[ORC_BLOCK_T];
-            memcpy(w, b + orc_off_vrow(j), 24);
-            orc_unpack_codes64(w, tok);
-            for (int64_t t = lo; t < hi; ++t) idx[(t - t0) * d + j] = tok[t - blk * ORC_BLOCK_T];
-        }
-        for (int64_t t = lo; t < hi; ++t)
-            memcpy(&nh[t - t0], b + (int64_t)d * 24 + 2 * (t - blk * ORC_BLOCK_T), 2);
-    }
 }
 static int64_t orc_off_gamma(int d, int tau) {
     return (int64_t)ORC_BLOCK_T * 3 * d / 8 + (int64_t)ORC_BLOCK_T * d / 8 + 2 * ORC_BLOCK_T + 2 * tau;
 }
 
-/* tokens [t0, t0 + T) of one sequence; blocks points at the sequence's first
- * block; kind: 0 V, 1 K, 2 PolarQuant-only K */
-void orc_pack(int d, int kind, int64_t t0, int64_t T, const uint8_t* idx, const uint8_t* sig,
+/* tokens [t0, t0 + T) of one sequence; blocks points at the sequence's first block */
+void orc_pack(int d, int is_k, int64_t t0, int64_t T, const uint8_t* idx, const uint8_t* sig,
               const uint16_t* nh, const uint16_t* gh, uint8_t* blocks) {
-    if (kind == ORC_KIND_V && d == 128) {
-        orc_pack_v(d, t0, T, idx, nh, blocks);
-        return;
-    }
-    const int is_k = kind == ORC_KIND_K;
-    const int64_t bb = orc_block_bytes(d, kind);
+    const int64_t bb = orc_block_bytes(d, is_k);
     for (int64_t tt = 0; tt < T; ++tt) {
         int64_t t = t0 + tt;
         uint8_t* blk = blocks + (t / ORC_BLOCK_T) * bb;
@@ -492,7 +425,7 @@ void orc_pack(int d, int kind, int64_t t0, int64_t T, const uint8_t* idx, const 
         uint32_t cw[24], sw[8];
         orc_pack_codes(d, idx + tt * d, cw);
         memcpy(blk + orc_off_codes(d, tau), cw, (size_t)3 * d / 8);
-        memcpy(blk + orc_off_norm(d, kind, tau), &nh[tt], 2);
+        memcpy(blk + orc_off_norm(d, is_k, tau), &nh[tt], 2);
         if (is_k) {
             orc_pack_signs(d, sig + tt * d, sw);
             memcpy(blk + orc_off_signs(d, tau), sw, (size_t)d / 8);
@@ -501,14 +434,9 @@ void orc_pack(int d, int kind, int64_t t0, int64_t T, const uint8_t* idx, const 
     }
 }
 
-void orc_unpack(int d, int kind, int64_t t0, int64_t T, const uint8_t* blocks,
+void orc_unpack(int d, int is_k, int64_t t0, int64_t T, const uint8_t* blocks,
                 uint8_t* idx, uint8_t* sig, uint16_t* nh, uint16_t* gh) {
-    if (kind == ORC_KIND_V && d == 128) {
-        orc_unpack_v(d, t0, T, blocks, idx, nh);
-        return;
-    }
-    const int is_k = kind == ORC_KIND_K;
-    const int64_t bb = orc_block_bytes(d, kind);
+    const int64_t bb = orc_block_bytes(d, is_k);
 #pragma omp parallel for schedule(static)
     for (int64_t tt = 0; tt < T; ++tt) {
         int64_t t = t0 + tt;
@@ -517,7 +445,7 @@ void orc_unpack(int d, int kind, int64_t t0, int64_t T, const uint8_t* blocks,
         uint32_t cw[24], sw[8];
         memcpy(cw, blk + orc_off_codes(d, tau), (size_t)3 * d / 8);
         orc_unpack_codes(d, cw, idx + tt * d);
-        memcpy(&nh[tt], blk + orc_off_norm(d, kind, tau), 2);
+        memcpy(&nh[tt], blk + orc_off_norm(d, is_k, tau), 2);
         if (is_k) {
             memcpy(sw, blk + orc_off_signs(d, tau), (size_t)d / 8);
             orc_unpack_signs(d, sw, sig + tt * d);

@@ -51,7 +51,7 @@ def unpack_cache(cache: tq.Cache, t0: int, T: int, seqs=None) -> dict:
     d, is_k = cache.head_dim, cache.is_k
     raw = cache.buf.cpu().numpy()
     nb = cache.Tcap // 64
-    bb = O.block_bytes(d, cache.kind)
+    bb = O.block_bytes(d, is_k)
     seqs = seqs if seqs is not None else [(b, h) for b in range(cache.B) for h in range(cache.Hkv)]
     out = {"idx": np.zeros((len(seqs), T, d), np.uint8), "nh": np.zeros((len(seqs), T), np.uint16)}
     if is_k:
@@ -59,7 +59,7 @@ def unpack_cache(cache: tq.Cache, t0: int, T: int, seqs=None) -> dict:
         out["gh"] = np.zeros((len(seqs), T), np.uint16)
     for n, (b, h) in enumerate(seqs):
         s = (b * cache.Hkv + h) * nb
-        u = O.unpack(d, cache.kind, t0, T, raw[s * bb:(s + nb) * bb])
+        u = O.unpack(d, is_k, t0, T, raw[s * bb:(s + nb) * bb])
         for k in out:
             out[k][n] = u[k]
     return out

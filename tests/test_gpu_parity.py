@@ -541,16 +541,16 @@ def test_attend_group_sizes_and_ragged_lengths(decode_path, handles, prms, d, G)
 @pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
 def test_attend_polar_only_k(decode_path, handles, prms, d, G):
-    """PolarQuant-only K (a K cache of codes and norms from tq_encode_k_polar):
-    the kernels' attention equals the oracle's with gamma = 0 (no QJL term),
-    ragged lengths; the K cache holds the oracle's V-flow codes and norms."""
+    """PolarQuant-only K (a V-layout K cache from tq_encode_v): the kernels'
+    attention equals the oracle's with gamma = 0 (no QJL term), ragged lengths;
+    the K cache holds the oracle's V-flow codes and norms."""
     Hkv, B, Tcap = 2, 3, 320
     Hq = Hkv * G
     h = handles[d]
     xk = torch_input(synthetic.gaussian((B, Hkv, Tcap, d), seed=31 + G), "f32")
     xv = torch_input(synthetic.gaussian((B, Hkv, Tcap, d), seed=41 + G), "f32")
-    kc, vc = tq.Cache(d, False, B, Hkv, Tcap, polar=True), tq.Cache(d, False, B, Hkv, Tcap)
-    tq.tq_encode_k_polar(h, xk, kc, 0)
+    kc, vc = tq.Cache(d, False, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
+    tq.tq_encode_v(h, xk, kc, 0)
     tq.tq_encode_v(h, xv, vc, 0)
     q = synthetic.gaussian((B, Hq, d), seed=51)
     lens = [0, 129, 301]
@@ -708,6 +708,6 @@ def test_attend_argument_errors(handles):
         tq.tq_attend_prefill(h2, torch.zeros((1, 3, 4, 256), device="cuda"), k2, v2, 62,
                              torch.empty((1, 3, 4, 256), device="cuda"), ws)
     assert e.value.status == tq.TQ_ERR_INVALID_ARG
-    with pytest.raises(ValueError):                                # a V cache is not a PolarQuant-only K cache
-        tq.tq_attend_decode_polar(h, q, vc, vc, out, ws, T=10)
+    with pytest.raises(ValueError):                                # a K cache is not a PolarQuant-only K cache
+        tq.tq_attend_decode_polar(h, q, kc, vc, out, ws, T=10)
     assert tq.tq_device_status(h) == tq.TQ_OK

@@ -277,51 +277,38 @@ def test_bits_per_dim_and_pack_roundtrip(golden, d):
     sig = g.integers(0, 2, (T, d), dtype=np.uint8)
     nh = g.integers(0, 2 ** 16, T, dtype=np.uint16)
     gh = g.integers(0, 2 ** 16, T, dtype=np.uint16)
-    assert O.block_bytes(d, "polar") == O.block_bytes(d, False)
-    for kind in (True, False, "polar"):
-        is_k = kind is True
-        blocks = np.zeros(Tcap // 64 * O.block_bytes(d, kind), dtype=np.uint8)
-        O.pack(d, kind, t0, idx, sig if is_k else None, nh, gh if is_k else None, blocks)
-        u = O.unpack(d, kind, t0, T, blocks)
+    for is_k in (True, False):
+        blocks = np.zeros(Tcap // 64 * O.block_bytes(d, is_k), dtype=np.uint8)
+        O.pack(d, is_k, t0, idx, sig if is_k else None, nh, gh if is_k else None, blocks)
+        u = O.unpack(d, is_k, t0, T, blocks)
         assert np.array_equal(u["idx"], idx) and np.array_equal(u["nh"], nh)
         if is_k:
             assert np.array_equal(u["sig"], sig) and np.array_equal(u["gh"], gh)
         # tokens outside [t0, t0 + T) stay zero
-        full = O.unpack(d, kind, 0, Tcap, blocks)
+        full = O.unpack(d, is_k, 0, Tcap, blocks)
         assert not full["idx"][:t0].any() and not full["idx"][t0 + T:].any()
         assert not full["nh"][:t0].any() and not full["nh"][t0 + T:].any()
-    # packing in pieces (appends) gives the same blocks as one bulk pack
-    for kind in (True, False, "polar"):
-        is_k = kind is True
-        bulk = np.zeros(Tcap // 64 * O.block_bytes(d, kind), dtype=np.uint8)
-        O.pack(d, kind, t0, idx, sig if is_k else None, nh, gh if is_k else None, bulk)
-        part = np.zeros_like(bulk)
+        # packing in pieces (appends) gives the same blocks as one bulk pack
+        part = np.zeros_like(blocks)
         for a, b in ((0, 1), (1, 30), (30, 31), (31, T)):
-            O.pack(d, kind, t0 + a, idx[a:b], sig[a:b] if is_k else None, nh[a:b], gh[a:b] if is_k else None, part)
-        assert np.array_equal(part, bulk)
+            O.pack(d, is_k, t0 + a, idx[a:b], sig[a:b] if is_k else None, nh[a:b], gh[a:b] if is_k else None, part)
+        assert np.array_equal(part, blocks)
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
 def test_layout_is_a_bijection(d):
-    """Every (token, coordinate, code bit) of a block and every sign lands on its
-    own bit: token records of the K and PolarQuant-only K blocks, coordinate
-    rows of the V block."""
-    ncode = 64 * 3 * d // 8
-    for kind, tokens in (("polar", [0, 37]), (True, [5]), (False, range(64) if d == 128 else [9])):
-        seen = set()
-        for tau in tokens:
-            for j in range(d):
-                for b in range(3):
-                    idx = np.zeros((1, d), dtype=np.uint8)
-                    idx[0, j] = 1 << b
-                    blocks = np.zeros(O.block_bytes(d, kind), dtype=np.uint8)
-                    O.pack(d, kind, tau, idx, None, np.zeros(1, np.uint16), None, blocks)
-                    bits = np.flatnonzero(np.unpackbits(blocks[:ncode], bitorder="little"))
-                    assert len(bits) == 1
-                    seen.add(int(bits[0]))
-        assert len(seen) == 3 * d * len(tokens)
-        if kind is not False or d != 128:  # token records: token tau's codes fill record tau
-            assert min(seen) >= 8 * (3 * d // 8) * tokens[0]
+    """Every (coordinate, code bit) and every sign lands on its own bit of the record."""
+    seen = set()
+    for j in range(d):
+        for b in range(3):
+            idx = np.zeros((1, d), dtype=np.uint8)
+            idx[0, j] = 1 << b
+            blocks = np.zeros(O.block_bytes(d, False), dtype=np.uint8)
+            O.pack(d, False, 0, idx, None, np.zeros(1, np.uint16), None, blocks)
+            bits = np.flatnonzero(np.unpackbits(blocks[: 3 * d // 8], bitorder="little"))
+            assert len(bits) == 1
+            seen.add(int(bits[0]))
+    assert len(seen) == 3 * d
     seen = set()
     for j in range(d):
         sig = np.zeros((1, d), dtype=np.uint8)
@@ -405,26 +392,6 @@ def test_attend_empty_and_gqa_independence():
     allh = O.attend(p, q, kc, vc, 0.2)
     for g in range(4):
         assert np.array_equal(allh[g], O.attend(p, q[g:g + 1], kc, vc, 0.2)[0])
-
-
-def test_v_layout_hand_worked_entries(golden):
-    """Single-entry head_dim-128 V blocks (one token's code at one coordinate)
-    against words worked out by hand from the written V layout (coordinate rows)."""
-    rows = golden("v_layout_single_entries.txt")
-    cases = {}
-    for d, tau, j, val, widx, whex in rows:
-        cases.setdefault((int(d), int(tau), int(j), int(val)), {})[int(widx)] = int(whex, 16)
-    assert len(cases) >= 10
-    for (d, tau, j, val), words in cases.items():
-        idx = np.zeros((1, d), np.uint8)
-        idx[0, j] = val
-        blocks = np.zeros(O.block_bytes(d, False), dtype=np.uint8)
-        O.pack(d, False, tau, idx, None, np.zeros(1, np.uint16), None, blocks)
-        rec = blocks[: 64 * 3 * d // 8].view(np.uint32)
-        expect = np.zeros_like(rec)
-        for w, v in words.items():
-            expect[w] = v
-        assert np.array_equal(rec, expect), (d, tau, j, val, [(i, hex(x)) for i, x in enumerate(rec) if x])
 
 
 def test_layout_hand_worked_entries(golden):
