@@ -46,6 +46,21 @@ namespace tqi {
 namespace {
 
 // ---------------------------------------------------------------- kernel
+constexpr int kTabMax = 512;   // block-table entries of a split staged in shared memory (32768 tokens)
+
+// Pool block of a paged cache from the staged table slice (contiguous cache:
+// the logical block index); an entry outside the pool sets the check word and
+// gives -1, as cache_block does.
+__device__ __forceinline__ int64_t staged_block(const int32_t* table, const int32_t* st, int64_t pool,
+                                                int64_t contiguous, int i, int* err) {
+    if (!table) return contiguous;
+    const int32_t p = st[i];
+    if (p < 0 || (int64_t)p >= pool) {
+        atomicExch(err, 1);
+        return -1;
+    }
+    return p;
+}
 // Token-row orientation: each mma tile has 16 tokens on M and the (head,
 // hi|lo) columns on N (NT n-tiles of 4 heads), so no M rows are wasted:
 //   scores  S[16 tok][8] += Kdeq[16 tok][16 coords] * Q'[16 coords][8]   (D/16 coordinate chunks, fp16)
@@ -65,8 +80,11 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     // per-warp (max, sum) of each head for the merge: [NW][8][2]
     float* sML = reinterpret_cast<float*>(smem + (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8);
     // d = 256: q'/u' fragments per (operand, n-tile, k-step, lane), filled once per CTA
+    // paged caches: the split's slice of the K and V block tables, [2][kTabMax]
+    int32_t* sTab = reinterpret_cast<int32_t*>(smem + (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
+                                               (size_t)NW * 8 * 2 * sizeof(float));
     uint2* sB = reinterpret_cast<uint2*>(smem + (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
-                                         (size_t)NW * 8 * 2 * sizeof(float));
+                                         (size_t)NW * 8 * 2 * sizeof(float) + 2 * kTabMax * sizeof(int32_t));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gr = lane >> 2, tq4 = lane & 3;
     uint8_t* ring = smem + (size_t)warp * kStages * C::kStageB;
@@ -84,6 +102,19 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     const int nchunk = s1 > s0 ? (int)((s1 - s0 + C::kChunk - 1) / C::kChunk) : 0;
     const int nmine = nchunk > warp ? (nchunk - warp + NW - 1) / NW : 0;
     const int64_t seq = (int64_t)b * a.Hkv + hkv;
+    // A paged cache's table entries for this split go to shared memory first (one
+    // coalesced load per CTA), so the per-chunk lookups that feed the bulk copies
+    // do not wait on global memory; longer splits keep the direct lookups.
+    const int64_t lb0 = s0 >> 6;
+    const int ntab = s1 > s0 ? (int)(((s1 + 63) >> 6) - lb0) : 0;
+    const bool staged = (a.ktable || a.vtable) && ntab <= kTabMax;
+    if (staged) {
+        for (int i = threadIdx.x; i < ntab; i += NW * 32) {
+            sTab[i] = a.ktable ? __ldg(a.ktable + seq * a.NB + lb0 + i) : 0;
+            sTab[kTabMax + i] = a.vtable ? __ldg(a.vtable + seq * a.NB + lb0 + i) : 0;
+        }
+        __syncthreads();
+    }
     const int64_t kbb = block_bytes(D, QJL), vbb = block_bytes(D, false);
 
     if (lane == 0)
@@ -94,8 +125,14 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     // cache blocks (K, V) of this warp's chunk i; a paged cache reads its block table
     auto blocks_of = [&](int i, int64_t& kblk, int64_t& vblk) {
         const int64_t t0 = s0 + (int64_t)(warp + i * NW) * C::kChunk;
-        kblk = cache_block(a.ktable, a.kpool, a.NB, seq, t0 >> 6, a.err);
-        vblk = cache_block(a.vtable, a.vpool, a.NB, seq, t0 >> 6, a.err);
+        if (staged) {
+            kblk = staged_block(a.ktable, sTab, a.kpool, seq * a.NB + (t0 >> 6), (int)((t0 >> 6) - lb0), a.err);
+            vblk = staged_block(a.vtable, sTab + kTabMax, a.vpool, seq * a.NB + (t0 >> 6), (int)((t0 >> 6) - lb0),
+                                a.err);
+        } else {
+            kblk = cache_block(a.ktable, a.kpool, a.NB, seq, t0 >> 6, a.err);
+            vblk = cache_block(a.vtable, a.vpool, a.NB, seq, t0 >> 6, a.err);
+        }
     };
     auto issue = [&](int i, int64_t kblk, int64_t vblk) {
         const int64_t t0 = s0 + (int64_t)(warp + i * NW) * C::kChunk;     // multiple of the chunk
@@ -491,7 +528,7 @@ template <int D, int NT, int NW, bool QJL>
 cudaError_t launch_mma_t(const DecArgs& a, int G, cudaStream_t s) {
     using C = Cfg<D, QJL>;
     const size_t smem = (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
-                        (size_t)NW * 8 * 2 * sizeof(float) +
+                        (size_t)NW * 8 * 2 * sizeof(float) + 2 * kTabMax * sizeof(int32_t) +
                         (C::kBRegs ? 0 : (size_t)2 * NT * C::kKC * 32 * sizeof(uint2));
     auto kern = tq_decode_mma_kernel<D, NT, NW, QJL>;
     cudaError_t e = set_smem_once<tq_decode_mma_kernel<D, NT, NW, QJL>>((int)smem);

@@ -83,9 +83,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// give up after kWaitLimit polls or about one second, whichever comes first
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
-    for (int i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (int i = 1; i < kWaitLimit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63) == 0 && global_ns() - t0 > kWaitNs) return false;
+    }
     return false;
 }
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

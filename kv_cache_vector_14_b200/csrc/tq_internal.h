@@ -17,7 +17,17 @@ namespace tqi {
 constexpr int kBlockT = 64;      // tokens per cache block
 constexpr int kMaxSplits = 2048; // split-K partials per query head (combine keeps their weights in smem)
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kDefaultWaitLimit = 1 << 20;   // try count of a bounded mbarrier wait
+constexpr int kDefaultWaitLimit = 1 << 20;   // poll count of a bounded mbarrier wait
+constexpr uint64_t kWaitNs = 1000000000ull;   // and its time bound (1 s)
+
+#ifdef __CUDACC__
+// global nanosecond timer of the GPU
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+#endif
 
 // Codebook passed by value to every kernel (it lands in the constant bank).
 struct Codebook {
@@ -200,6 +210,8 @@ cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, cons
 // Chunked prefill (head_dim 128): rows (b, i, head) of Lq queries per sequence,
 // query i over tokens [0, T0 + i]; partials as one split of a.part_ml/part_acc.
 cudaError_t launch_prefill(int d, int G, const DecArgs& a, int64_t Lq, int64_t T0, cudaStream_t s);
+// head_dim 128: the tcgen05 form (tq_prefill_tc.cu)
+cudaError_t launch_prefill_tc(int G, const DecArgs& a, int64_t Lq, int64_t T0, cudaStream_t s);
 // qjl = false: PolarQuant-only K cache (V layout), scores without the QJL term.
 cudaError_t launch_decode(int d, int G, bool use_mma, bool qjl, const DecArgs& a, cudaStream_t s);
 cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml,

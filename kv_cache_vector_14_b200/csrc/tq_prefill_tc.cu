@@ -1,0 +1,460 @@
+// Chunked-prefill attention over the packed TurboQuant cache for head_dim 128
+// on the 5th-generation tensor cores (tcgen05, accumulators and the query
+// operand in tensor memory), for sm_100a.
+//
+// Page "Apple Silicon向けSwiftLM、TurboQuant KVキャッシュ圧縮とSSD Expert
+// Streamingを実装" (ai-heartland.com): the decode estimator (K section: 3-bit
+// codes plus the 1-bit QJL residual correction; V section; hybrid V2+V3
+// section: dequantisation fused into attention) for a chunk of Lq new queries
+// per sequence, query i attending causally over cache tokens [0, T0 + i].
+//
+// A CTA owns 128 query rows (query i, head g of one kv head: row i G + g) and
+// walks the cache in tiles of 64 tokens (one cache block).  With 128 rows per
+// tile the contraction is dense, so the dequantised tile is built once in
+// shared memory and consumed by the tensor core for all rows:
+//   S[128 rows][64 tok] = [Q'hi | Q'lo | U'hi | U'lo] [Kdeq ; Kdeq ; Sgn ; Sgn]^T
+//       (A in tensor memory: q' and u' of each row as fp16 hi and lo limbs,
+//        K = 4 x 128; B in shared memory: the keys' fp16 centroids and the
+//        sign operand +-gamma_t, both exact in fp16, so one fp32 accumulator
+//        holds <q', c[idx]> + gamma <u', 2 sigma - 1>)
+//   O[128 rows][128 coords] += [Phi | Plo] [Vdeq ; Vdeq]
+//       (A in tensor memory: the softmax weights p * nv, scaled by 2^-6, as
+//        fp16 hi and lo limbs; B in shared memory: the values' centroids, one row per
+//        coordinate along tokens)
+// Warp roles: warps 4-7 stage the cache blocks (bulk copies into a ring),
+// expand the codes into the B operands of the next tile (two buffers) and
+// issue the mma (one thread); warps 0-3 own one row each per thread (tensor-
+// memory lane = row): they load S, apply the norms, the causal mask and the
+// online softmax, and write P.  The running maximum used for P is moved only
+// when it grows by more than 2^8, and then O in tensor memory is rescaled.
+// mbarriers order the two roles and the tensor core; every wait is bounded.
+#include "tq_frag.cuh"
+#include "tq_tc.cuh"
+
+namespace tqi {
+namespace {
+
+constexpr int kPD = 128;                 // head_dim
+constexpr int kPT = 64;                  // tokens per tile (one cache block)
+constexpr int kPRows = 128;              // query rows per CTA
+constexpr int kPRing = 3;                // raw block stages
+constexpr float kRescaleLog2 = 8.f;      // move the maximum used for P only when it grows by more than this
+constexpr float kPScale = 1.f / 64.f;    // P holds p nv 2^-6 (p <= 2^8, so fp16 holds it unless nv > 2^14)
+
+struct PtcShape {
+    static constexpr int kKB = 64 * 48 + 64 * 16 + 256;     // K block bytes
+    static constexpr int kVB = 64 * 48 + 128;                // V block bytes
+    // B buffers (x2): keys [64 tok][128 coords] fp16, signs [64 tok][128 rows] fp16,
+    // values [128 coords][64 tok] fp16; 128-byte swizzled, K-major
+    static constexpr int kOffK = 0;
+    static constexpr int kOffS = 16384;
+    static constexpr int kOffV = 32768;
+    static constexpr int kBuf = 49152;
+    static constexpr int kOffScal = 2 * kBuf;                // [2][64] n, [2][64] nv (floats)
+    static constexpr int kOffRing = kOffScal + 1024;
+    static constexpr int kStage = kKB + kVB;
+    static constexpr int kOffBar = kOffRing + kPRing * kStage;
+    static constexpr int kOffMisc = kOffBar + 8 * 16;
+    static constexpr int kSmem = kOffMisc + 64 + 1024;       // + slack to align the base
+    // tensor memory: the query operand (4 x 64 columns), S, P, O
+    static constexpr int kColA = 0;
+    static constexpr int kColS = 256;
+    static constexpr int kColP = 320;
+    static constexpr int kColO = 384;
+    static constexpr int kAlloc = 512;
+};
+
+struct PrefillTcArgs {
+    DecArgs a;          // caches, workspace, scale, partials (one split), check word
+    int64_t Lq, T0;     // queries per sequence in the chunk; tokens cached before it
+    int G;              // query heads per kv head
+};
+
+__device__ __forceinline__ void named_bar(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// barrier id over n threads that also ORs v across them (every thread gets the result)
+__device__ __forceinline__ bool bar_or(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__global__ void __launch_bounds__(256, 1) tq_prefill_tc_kernel(const PrefillTcArgs pa) {
+    using S = PtcShape;
+    const DecArgs& a = pa.a;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + S::kOffBar);
+    // bars: ring full [0..2], B ready [3..4] (128 producer arrivals), S full [5]
+    // (commit), S free [6] (128 softmax arrivals), O done [7] (commit)
+    const uint32_t bar_sfull = smem_u32(&bars[5]), bar_sfree = smem_u32(&bars[6]), bar_odone = smem_u32(&bars[7]);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + S::kOffMisc);
+    float* scal = reinterpret_cast<float*>(sm + S::kOffScal);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int hkv = blockIdx.y, b = blockIdx.z, G = pa.G;
+    const int64_t nrows = pa.Lq * G;
+    const int64_t row0 = (int64_t)blockIdx.x * kPRows;
+    const int64_t rlast = (row0 + kPRows - 1 < nrows ? row0 + kPRows - 1 : nrows - 1);
+    const int64_t tend = pa.T0 + rlast / G + 1;                  // tokens any row of the CTA sees
+    const int ntile = (int)((tend + kPT - 1) / kPT);
+    const int64_t seq = (int64_t)b * a.Hkv + hkv;
+
+    if (tid == 0) {
+        for (int s = 0; s < kPRing; ++s) mbar_init(smem_u32(&bars[s]), 1);
+        mbar_init(smem_u32(&bars[3]), 128);
+        mbar_init(smem_u32(&bars[4]), 128);
+        mbar_init(bar_sfull, 1);
+        mbar_init(bar_sfree, 128);
+        mbar_init(bar_odone, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc_alloc(smem_u32(tmem_slot), S::kAlloc);
+        tc_relinquish();
+    }
+    auto issue = [&](int k) {              // raw K and V blocks of tile k -> ring stage k % kPRing
+        uint8_t* st = sm + S::kOffRing + (k % kPRing) * S::kStage;
+        const uint32_t bar = smem_u32(&bars[k % kPRing]);
+        const int64_t kblk = cache_block(a.ktable, a.kpool, a.NB, seq, k, a.err);
+        const int64_t vblk = cache_block(a.vtable, a.vpool, a.NB, seq, k, a.err);
+        mbar_expect_tx(bar, (uint32_t)S::kStage);
+        bulk_g2s(smem_u32(st), a.kc + (kblk >= 0 ? kblk : 0) * S::kKB, S::kKB, bar);
+        bulk_g2s(smem_u32(st + S::kKB), a.vc + (vblk >= 0 ? vblk : 0) * S::kVB, S::kVB, bar);
+    };
+    tc_fence_before();
+    __syncthreads();                       // the mbarriers are initialised before anyone uses them
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 128)
+        for (int k = 0; k < kPRing && k < ntile; ++k) issue(k);
+    pdl_wait();                            // q' and u' come from the prologue kernel
+
+    bool failed = false;
+    if (warp < 4) {
+        // ======================================== softmax warps: thread r = row r
+        const int r = tid;
+        const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+        const int64_t grow = row0 + r;
+        const bool rvalid = grow < nrows;
+        const int64_t qi = rvalid ? grow / G : 0, qg = rvalid ? grow % G : 0;
+        const int64_t qrow = ((int64_t)b * pa.Lq + qi) * a.Hq + (int64_t)hkv * G + qg;
+        const int64_t lim = rvalid ? pa.T0 + qi + 1 : 0;          // tokens [0, lim) visible
+        // query operand: column c of each 64-column part holds K positions 2c, 2c + 1;
+        // K position kappa = 32 t + p is coordinate (JL row) slot_coord(0, t, p)
+        {
+            const float* qp = a.qp + qrow * kPD;
+            const float* up = a.up + qrow * kPD;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {           // q', u'
+                const float* src = part == 0 ? qp : up;
+#pragma unroll
+                for (int c0 = 0; c0 < 64; c0 += 16) {
+                    uint32_t hi[16], lo[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int kap = 2 * (c0 + c), t = kap >> 5, p = kap & 31;
+                        const float x0 = rvalid ? src[slot_coord(0, t, p)] : 0.f;
+                        const float x1 = rvalid ? src[slot_coord(0, t, p + 1)] : 0.f;
+                        split_hilo(x0, x1, hi[c], lo[c]);
+                    }
+                    tc_st16(tl + S::kColA + 128 * part + c0, hi);
+                    tc_st16(tl + S::kColA + 128 * part + 64 + c0, lo);
+                }
+            }
+            tc_wait_st();
+            tc_fence_before();
+        }
+        named_bar(2, 256);                 // the query operand is in place (both roles)
+        float m_run = -INFINITY, m_used = -INFINITY, l = 0.f;
+        for (int k = 0; k < ntile; ++k) {
+            // (failures are made warp-uniform: the tensor-memory loads and stores are warp-collective)
+            if (!__all_sync(kFull, mbar_wait_bounded(bar_sfull, (uint32_t)(k & 1)))) { failed = true; break; }
+            tc_fence_after();
+            uint32_t sv[64];
+            {
+                uint32_t t32[32];
+                tc_ld32(tl + S::kColS, t32);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) sv[c] = t32[c];
+                tc_ld32(tl + S::kColS + 32, t32);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) sv[32 + c] = t32[c];
+            }
+            if (!__all_sync(kFull, mbar_wait_bounded(smem_u32(&bars[3 + (k & 1)]), (uint32_t)((k >> 1) & 1)))) {
+                failed = true;
+                break;
+            }
+            const float* sn = scal + (k & 1) * 128;          // n[64], nv[64] of this tile
+            const int64_t tok0 = (int64_t)k * kPT;
+            const int vis = lim - tok0 >= kPT ? kPT : (int)(lim > tok0 ? lim - tok0 : 0);
+            float s[64];
+            float mt = -INFINITY;
+#pragma unroll
+            for (int t = 0; t < 64; ++t) {
+                s[t] = t < vis ? __uint_as_float(sv[t]) * a.scale_log2 * sn[t] : -INFINITY;
+                mt = fmaxf(mt, s[t]);
+            }
+            const float m_new = fmaxf(m_run, mt);
+            m_run = m_new;
+            // the previous tile's P . V must be done before P and O are touched
+            if (k > 0 && !__all_sync(kFull, mbar_wait_bounded(bar_odone, (uint32_t)((k - 1) & 1)))) {
+                failed = true;
+                break;
+            }
+            tc_fence_after();
+            // Move this row's reference maximum when it grew by more than 2^8; O is rescaled
+            // by the warp as a whole (tensor-memory loads and stores are warp-collective),
+            // with factor 1 on the rows that keep theirs.
+            float f = 1.f;
+            if (m_new != -INFINITY && (m_used == -INFINITY || m_new > m_used + kRescaleLog2)) {
+                if (m_used != -INFINITY) {                    // O and l were built on m_used
+                    f = fast_exp2(m_used - m_new);
+                    l *= f;
+                }
+                m_used = m_new;
+            }
+            if (__any_sync(kFull, f != 1.f)) {
+#pragma unroll
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    uint32_t ov[32];
+                    tc_ld32(tl + S::kColO + c0, ov);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * f);
+                    tc_st32(tl + S::kColO + c0, ov);
+                }
+            }
+            // P = 2^(s - m_used) nv: hi limbs in columns 0-31, lo limbs in 32-63 (tokens 2c, 2c + 1)
+            uint32_t ph[32], plo[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                float pv[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int t = 2 * c + e;
+                    const float p = s[t] == -INFINITY ? 0.f : fast_exp2(s[t] - m_used);
+                    l += p;
+                    pv[e] = p == 0.f ? 0.f : p * sn[64 + t] * kPScale;
+                }
+                split_hilo(pv[0], pv[1], ph[c], plo[c]);
+            }
+            uint32_t h16[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) h16[c] = ph[c];
+            tc_st16(tl + S::kColP, h16);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) h16[c] = ph[16 + c];
+            tc_st16(tl + S::kColP + 16, h16);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) h16[c] = plo[c];
+            tc_st16(tl + S::kColP + 32, h16);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) h16[c] = plo[16 + c];
+            tc_st16(tl + S::kColP + 48, h16);
+            tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar_sfree);
+        }
+        // ---- the last tile's P . V, then this row's partial
+        if (!failed && ntile > 0 && !__all_sync(kFull, mbar_wait_bounded(bar_odone, (uint32_t)((ntile - 1) & 1))))
+            failed = true;
+        tc_fence_after();
+        pdl_trigger();
+        if (failed) atomicExch(a.err, 1);
+        // (the loads are warp-collective: every lane loads, valid rows store)
+        float* acc = a.part_acc + qrow * kPD;
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t ov[32];
+            tc_ld32(tl + S::kColO + c0, ov);
+            if (rvalid) {
+#pragma unroll
+                for (int c = 0; c < 32; c += 4)
+                    *reinterpret_cast<float4*>(acc + c0 + c) =
+                        failed ? make_float4(0.f, 0.f, 0.f, 0.f)
+                               : make_float4(__uint_as_float(ov[c]) * (1.f / kPScale),
+                                             __uint_as_float(ov[c + 1]) * (1.f / kPScale),
+                                             __uint_as_float(ov[c + 2]) * (1.f / kPScale),
+                                             __uint_as_float(ov[c + 3]) * (1.f / kPScale));
+            }
+        }
+        if (rvalid) {
+            a.part_ml[2 * qrow] = failed ? -INFINITY : m_used;
+            a.part_ml[2 * qrow + 1] = failed ? 0.f : l;
+        }
+    } else {
+        // ======================================== producer warps: thread pt of 128
+        const int pt = tid - 128;
+        const int tau = pt >> 1, hf = pt & 1;                   // token of the tile, half of its slots
+        const uint32_t lut[4] = {a.cb.lut_lo[0], a.cb.lut_lo[1], a.cb.lut_hi[0], a.cb.lut_hi[1]};
+        const uint32_t* pw = a.cb.pow2;
+        constexpr uint32_t kIdS = idesc_f16(128, kPT), kIdO = idesc_f16(128, kPD);
+        int n_s = 0, n_o = 0, n_ring = ntile < kPRing ? ntile : kPRing;
+        bool fail_mma = false;             // thread pt 0: a wait of the mma phase gave up
+        named_bar(2, 256);                 // the query operand is in place
+        tc_fence_after();
+        for (int k = 0; k < ntile; ++k) {
+            const int buf = k & 1;
+            const uint8_t* st = sm + S::kOffRing + (k % kPRing) * S::kStage;
+            // every producer thread reaches the barrier below whatever happens, so that
+            // the decision to stop is the same for all of them
+            bool f = fail_mma || !mbar_wait_bounded(smem_u32(&bars[k % kPRing]), (uint32_t)((k / kPRing) & 1));
+            // buffer buf was last read by tile k - 2's mma
+            if (!f && k >= 2) f = !mbar_wait_bounded(bar_odone, (uint32_t)((k - 2) & 1));
+            if (!f) {
+            uint8_t* Kt = sm + buf * S::kBuf + S::kOffK;
+            uint8_t* Sg = sm + buf * S::kBuf + S::kOffS;
+            uint8_t* Vt = sm + buf * S::kBuf + S::kOffV;
+            const uint8_t* kb = st;
+            const uint8_t* vb = st + S::kKB;
+            const uint32_t gam = *reinterpret_cast<const uint16_t*>(kb + 64 * 64 + 128 + 2 * tau);
+            const uint32_t g2 = gam | (gam << 16);
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                const int t = 2 * hf + tt;
+                uint32_t sel[4], vsel[4];
+                code_selectors(kb + tau * 48 + 12 * t, pw, sel);
+                code_selectors(vb + tau * 48 + 12 * t, pw, vsel);
+                // keys: K positions 32 t .. 32 t + 31 of row tau (four 16-byte chunks)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t x[4];
+                    dequant4(sel_for(sel, pw, 2 * c), lut, x[0], x[1]);
+                    dequant4(sel_for(sel, pw, 2 * c + 1), lut, x[2], x[3]);
+                    *reinterpret_cast<uint4*>(Kt + sw128_byte(tau, 2 * (32 * t + 8 * c), kPT)) =
+                        make_uint4(x[0], x[1], x[2], x[3]);
+                }
+                // signs: +-gamma for JL rows at positions 2q, 2q + 1 (sign bits q, 16 + q)
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(kb + 64 * 48 + tau * 16 + 4 * t);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t x[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int q = 4 * c + e;
+                        const uint32_t sh = shl_m(w, pw, 15 - q);         // bits q, 16 + q -> 15, 31
+                        x[e] = g2 ^ (~sh & 0x80008000u);                  // sigma = 0: -gamma
+                    }
+                    *reinterpret_cast<uint4*>(Sg + sw128_byte(tau, 2 * (32 * t + 8 * c), kPT)) =
+                        make_uint4(x[0], x[1], x[2], x[3]);
+                }
+                // values: row = coordinate, K position = token tau
+#pragma unroll
+                for (int kc = 0; kc < 8; ++kc) {
+                    uint32_t x0, x1;
+                    dequant4(sel_for(vsel, pw, kc), lut, x0, x1);
+                    const int p = 4 * kc;
+                    const uint32_t v4[4] = {x0 & 0xFFFFu, x0 >> 16, x1 & 0xFFFFu, x1 >> 16};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        *reinterpret_cast<uint16_t*>(Vt + sw128_byte(slot_coord(0, t, p + e), 2 * tau, kPD)) =
+                            (uint16_t)v4[e];
+                }
+            }
+            if (hf == 0) {
+                scal[buf * 128 + tau] = __half2float(*reinterpret_cast<const __half*>(kb + 64 * 64 + 2 * tau));
+                scal[buf * 128 + 64 + tau] = __half2float(*reinterpret_cast<const __half*>(vb + 64 * 48 + 2 * tau));
+            }
+            fence_proxy_async();           // B operands written by threads, read by the tensor core
+            mbar_arrive(smem_u32(&bars[3 + buf]));
+            }
+            // every producer thread is done with stage k and buffer buf (or one gave up)
+            if (bar_or(1, 128, f)) { failed = true; break; }
+            if (pt == 0) {
+                if (k >= 1) {              // P of tile k - 1 is written: O += P V
+                    if (!mbar_wait_bounded(bar_sfree, (uint32_t)((k - 1) & 1))) {
+                        fail_mma = true;
+                    } else {
+                        tc_fence_after();
+                        const uint32_t vd = sbase + (uint32_t)(((k - 1) & 1) * S::kBuf + S::kOffV);
+#pragma unroll
+                        for (int s = 0; s < 8; ++s)
+                            tc_mma_f16_ts(tmem + S::kColO, tmem + S::kColP + 8 * s, sw128_desc(vd + 32 * (s & 3)),
+                                          kIdO, (k - 1 > 0 || s > 0) ? 1u : 0u);
+                        tc_commit(bar_odone);
+                        ++n_o;
+                    }
+                }
+                if (!fail_mma) {           // S = [Q' | U'] [K ; K ; Sg ; Sg]^T
+                    const uint32_t kd = sbase + (uint32_t)(buf * S::kBuf + S::kOffK);
+                    const uint32_t sd = sbase + (uint32_t)(buf * S::kBuf + S::kOffS);
+#pragma unroll
+                    for (int s = 0; s < 32; ++s) {
+                        const int ss = s & 7;
+                        const uint32_t base = s < 16 ? kd : sd;
+                        const uint32_t addr = base + (uint32_t)((ss >> 2) * (kPT * 128) + (ss & 3) * 32);
+                        tc_mma_f16_ts(tmem + S::kColS, tmem + S::kColA + 8 * s, sw128_desc(addr), kIdS,
+                                      s > 0 ? 1u : 0u);
+                    }
+                    tc_commit(bar_sfull);
+                    ++n_s;
+                    if (k + kPRing < ntile) {
+                        fence_proxy_async();
+                        issue(k + kPRing);
+                        ++n_ring;
+                    }
+                }
+            }
+        }
+        if (fail_mma) failed = true;
+        // the last tile's O += P V
+        if (pt == 0 && !failed && ntile > 0) {
+            if (!mbar_wait_bounded(bar_sfree, (uint32_t)((ntile - 1) & 1))) {
+                failed = true;
+            } else {
+                tc_fence_after();
+                const uint32_t vd = sbase + (uint32_t)(((ntile - 1) & 1) * S::kBuf + S::kOffV);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    tc_mma_f16_ts(tmem + S::kColO, tmem + S::kColP + 8 * s, sw128_desc(vd + 32 * (s & 3)), kIdO,
+                                  (ntile - 1 > 0 || s > 0) ? 1u : 0u);
+                tc_commit(bar_odone);
+                ++n_o;
+            }
+        }
+        if (pt == 0) {
+            // wait (bounded) for the mma and copies this thread issued
+            if (n_s > 0) mbar_wait_bounded(bar_sfull, (uint32_t)((n_s - 1) & 1));
+            if (n_o > 0) mbar_wait_bounded(bar_odone, (uint32_t)((n_o - 1) & 1));
+            // only the last copy into each stage can still be in flight: an earlier one was
+            // waited for before its stage was refilled (and a wait on an older phase of the
+            // same parity as the current one would not return)
+            for (int k = n_ring > kPRing ? n_ring - kPRing : 0; k < n_ring; ++k)
+                mbar_wait_bounded(smem_u32(&bars[k % kPRing]), (uint32_t)((k / kPRing) & 1));
+            if (failed) atomicExch(a.err, 1);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tc_dealloc(tmem, S::kAlloc);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_tc(int G, const DecArgs& a, int64_t Lq, int64_t T0, cudaStream_t s) {
+    constexpr int smem = PtcShape::kSmem;
+    PrefillTcArgs pa{a, Lq, T0, G};
+    const int64_t tiles = (Lq * G + kPRows - 1) / kPRows;
+    cudaError_t e = set_smem_once<tq_prefill_tc_kernel>(smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)tiles, (unsigned)a.Hkv, (unsigned)a.B);
+    return launch_pdl(tq_prefill_tc_kernel, grid, dim3(256), smem, s, pa);
+}
+
+}  // namespace tqi
