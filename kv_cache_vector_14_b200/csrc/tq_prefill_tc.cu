@@ -21,13 +21,18 @@
 //       (A in tensor memory: the softmax weights p * nv, scaled by 2^-6, as
 //        fp16 hi and lo limbs; B in shared memory: the values' centroids, one row per
 //        coordinate along tokens)
-// Warp roles: warps 4-7 stage the cache blocks (bulk copies into a ring),
-// expand the codes into the B operands of the next tile (two buffers) and
-// issue the mma (one thread); warps 0-3 own one row each per thread (tensor-
-// memory lane = row): they load S, apply the norms, the causal mask and the
-// online softmax, and write P.  The running maximum used for P is moved only
-// when it grows by more than 2^8, and then O in tensor memory is rescaled.
-// mbarriers order the two roles and the tensor core; every wait is bounded.
+// Warp roles: warps 4-7 stage the cache blocks (bulk copies into a ring)
+// and expand the codes into the B operands (three buffers, so they run up to
+// two tiles ahead); warp 8 issues the mma (one thread); warps 0-3 own one row
+// each per thread (tensor-memory lane = row): they load S, apply the norms,
+// the causal mask and the online softmax, and write P over S in tensor memory.
+// S and P have two tensor-memory buffers, so the tensor core computes the
+// scores of tile k + 1 while the softmax works on tile k; the mma of one
+// thread run in issue order, so S(k + 2) cannot overwrite P(k) before O += P(k)
+// V(k), issued earlier, has read it.  The running maximum used for P is moved
+// only when it grows by more than 2^8, and then O in tensor memory is
+// rescaled.  mbarriers order the roles and the tensor core; every wait is
+// bounded.
 #include "tq_frag.cuh"
 #include "tq_tc.cuh"
 
@@ -38,30 +43,47 @@ constexpr int kPD = 128;                 // head_dim
 constexpr int kPT = 64;                  // tokens per tile (one cache block)
 constexpr int kPRows = 128;              // query rows per CTA
 constexpr int kPRing = 3;                // raw block stages
+constexpr int kPBuf = 3;                 // B operand buffers
+constexpr int kSoftmaxThreads = 128, kProducerThreads = 128;
+constexpr int kThreads = kSoftmaxThreads + kProducerThreads + 32;   // + the mma warp
 constexpr float kRescaleLog2 = 8.f;      // move the maximum used for P only when it grows by more than this
 constexpr float kPScale = 1.f / 64.f;    // P holds p nv 2^-6 (p <= 2^8, so fp16 holds it unless nv > 2^14)
 
 struct PtcShape {
     static constexpr int kKB = 64 * 48 + 64 * 16 + 256;     // K block bytes
     static constexpr int kVB = 64 * 48 + 128;                // V block bytes
-    // B buffers (x2): keys [64 tok][128 coords] fp16, signs [64 tok][128 rows] fp16,
+    // B buffers: keys [64 tok][128 coords] fp16, signs [64 tok][128 rows] fp16,
     // values [128 coords][64 tok] fp16; 128-byte swizzled, K-major
     static constexpr int kOffK = 0;
     static constexpr int kOffS = 16384;
     static constexpr int kOffV = 32768;
     static constexpr int kBuf = 49152;
-    static constexpr int kOffScal = 2 * kBuf;                // [2][64] n, [2][64] nv (floats)
-    static constexpr int kOffRing = kOffScal + 1024;
+    static constexpr int kOffScal = kPBuf * kBuf;            // per buffer: n scale log2(e) [64], nv 2^-6 [64]
+    static constexpr int kOffRing = kOffScal + kPBuf * 512;
     static constexpr int kStage = kKB + kVB;
     static constexpr int kOffBar = kOffRing + kPRing * kStage;
-    static constexpr int kOffMisc = kOffBar + 8 * 16;
+    static constexpr int kNumBars = 16;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmem = kOffMisc + 64 + 1024;       // + slack to align the base
-    // tensor memory: the query operand (4 x 64 columns), S, P, O
+    // tensor memory: the query operand (4 x 64 columns), S / P (two buffers), O
     static constexpr int kColA = 0;
-    static constexpr int kColS = 256;
-    static constexpr int kColP = 320;
+    static constexpr int kColX = 256;                        // buffer x at kColX + 64 x
     static constexpr int kColO = 384;
     static constexpr int kAlloc = 512;
+};
+static_assert(PtcShape::kOffRing % 16 == 0 && PtcShape::kStage % 16 == 0, "bulk copy alignment");
+static_assert(PtcShape::kSmem <= 227 * 1024, "shared memory per CTA");
+
+// mbarriers (index into the barrier array)
+enum : int {
+    kBarRing = 0,     // [3] raw stage filled (bulk copy bytes)
+    kBarBReady = 3,   // [3] B buffer built (128 producer arrivals)
+    kBarBFree = 6,    // [3] B buffer read by S and O of its tile (commit)
+    kBarSFull = 9,    // [2] S computed into buffer x (commit)
+    kBarPReady = 11,  // [2] P written into buffer x (128 softmax arrivals)
+    kBarODone = 13,   // O += P V of a tile done (commit)
+    kBarAReady = 14,  // query operand in tensor memory (128 softmax arrivals)
+    kBarDrain = 15,   // every mma issued by the mma thread done (commit, at exit)
 };
 
 struct PrefillTcArgs {
@@ -70,9 +92,6 @@ struct PrefillTcArgs {
     int G;              // query heads per kv head
 };
 
-__device__ __forceinline__ void named_bar(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 // barrier id over n threads that also ORs v across them (every thread gets the result)
 __device__ __forceinline__ bool bar_or(int id, int n, bool v) {
     uint32_t r;
@@ -89,8 +108,12 @@ __device__ __forceinline__ bool bar_or(int id, int n, bool v) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// warp-uniform bounded wait (the warp then runs warp-collective tensor-memory instructions)
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
+    return __all_sync(kFull, mbar_wait_bounded(bar, parity));
+}
 
-__global__ void __launch_bounds__(256, 1) tq_prefill_tc_kernel(const PrefillTcArgs pa) {
+__global__ void __launch_bounds__(kThreads, 1) tq_prefill_tc_kernel(const PrefillTcArgs pa) {
     using S = PtcShape;
     const DecArgs& a = pa.a;
     extern __shared__ uint8_t smem_raw[];
@@ -98,9 +121,7 @@ __global__ void __launch_bounds__(256, 1) tq_prefill_tc_kernel(const PrefillTcAr
     uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     const uint32_t sbase = smem_u32(sm);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + S::kOffBar);
-    // bars: ring full [0..2], B ready [3..4] (128 producer arrivals), S full [5]
-    // (commit), S free [6] (128 softmax arrivals), O done [7] (commit)
-    const uint32_t bar_sfull = smem_u32(&bars[5]), bar_sfree = smem_u32(&bars[6]), bar_odone = smem_u32(&bars[7]);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + S::kOffMisc);
     float* scal = reinterpret_cast<float*>(sm + S::kOffScal);
 
@@ -114,12 +135,18 @@ __global__ void __launch_bounds__(256, 1) tq_prefill_tc_kernel(const PrefillTcAr
     const int64_t seq = (int64_t)b * a.Hkv + hkv;
 
     if (tid == 0) {
-        for (int s = 0; s < kPRing; ++s) mbar_init(smem_u32(&bars[s]), 1);
-        mbar_init(smem_u32(&bars[3]), 128);
-        mbar_init(smem_u32(&bars[4]), 128);
-        mbar_init(bar_sfull, 1);
-        mbar_init(bar_sfree, 128);
-        mbar_init(bar_odone, 1);
+        for (int i = 0; i < kPRing; ++i) mbar_init(bar(kBarRing + i), 1);
+        for (int i = 0; i < kPBuf; ++i) {
+            mbar_init(bar(kBarBReady + i), kProducerThreads);
+            mbar_init(bar(kBarBFree + i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(kBarSFull + i), 1);
+            mbar_init(bar(kBarPReady + i), kSoftmaxThreads);
+        }
+        mbar_init(bar(kBarODone), 1);
+        mbar_init(bar(kBarAReady), kSoftmaxThreads);
+        mbar_init(bar(kBarDrain), 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -128,18 +155,18 @@ __global__ void __launch_bounds__(256, 1) tq_prefill_tc_kernel(const PrefillTcAr
     }
     auto issue = [&](int k) {              // raw K and V blocks of tile k -> ring stage k % kPRing
         uint8_t* st = sm + S::kOffRing + (k % kPRing) * S::kStage;
-        const uint32_t bar = smem_u32(&bars[k % kPRing]);
+        const uint32_t br = bar(kBarRing + k % kPRing);
         const int64_t kblk = cache_block(a.ktable, a.kpool, a.NB, seq, k, a.err);
         const int64_t vblk = cache_block(a.vtable, a.vpool, a.NB, seq, k, a.err);
-        mbar_expect_tx(bar, (uint32_t)S::kStage);
-        bulk_g2s(smem_u32(st), a.kc + (kblk >= 0 ? kblk : 0) * S::kKB, S::kKB, bar);
-        bulk_g2s(smem_u32(st + S::kKB), a.vc + (vblk >= 0 ? vblk : 0) * S::kVB, S::kVB, bar);
+        mbar_expect_tx(br, (uint32_t)S::kStage);
+        bulk_g2s(smem_u32(st), a.kc + (kblk >= 0 ? kblk : 0) * S::kKB, S::kKB, br);
+        bulk_g2s(smem_u32(st + S::kKB), a.vc + (vblk >= 0 ? vblk : 0) * S::kVB, S::kVB, br);
     };
     tc_fence_before();
     __syncthreads();                       // the mbarriers are initialised before anyone uses them
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    if (tid == 128)
+    if (tid == kSoftmaxThreads)
         for (int k = 0; k < kPRing && k < ntile; ++k) issue(k);
     pdl_wait();                            // q' and u' come from the prologue kernel
 
@@ -177,48 +204,56 @@ __global__ void __launch_bounds__(256, 1) tq_prefill_tc_kernel(const PrefillTcAr
             }
             tc_wait_st();
             tc_fence_before();
+            mbar_arrive(bar(kBarAReady));
         }
-        named_bar(2, 256);                 // the query operand is in place (both roles)
         float m_run = -INFINITY, m_used = -INFINITY, l = 0.f;
+        int b3 = 0, ph3 = 0;                                  // k % 3, (k / 3) & 1
         for (int k = 0; k < ntile; ++k) {
+            const int x = k & 1;
+            const uint32_t tx = tl + S::kColX + 64 * x;
             // (failures are made warp-uniform: the tensor-memory loads and stores are warp-collective)
-            if (!__all_sync(kFull, mbar_wait_bounded(bar_sfull, (uint32_t)(k & 1)))) { failed = true; break; }
+            if (!warp_wait(bar(kBarSFull + x), (uint32_t)((k >> 1) & 1))) { failed = true; break; }
             tc_fence_after();
             uint32_t sv[64];
             {
                 uint32_t t32[32];
-                tc_ld32(tl + S::kColS, t32);
+                tc_ld32(tx, t32);
 #pragma unroll
                 for (int c = 0; c < 32; ++c) sv[c] = t32[c];
-                tc_ld32(tl + S::kColS + 32, t32);
+                tc_ld32(tx + 32, t32);
 #pragma unroll
                 for (int c = 0; c < 32; ++c) sv[32 + c] = t32[c];
             }
-            if (!__all_sync(kFull, mbar_wait_bounded(smem_u32(&bars[3 + (k & 1)]), (uint32_t)((k >> 1) & 1)))) {
-                failed = true;
-                break;
-            }
-            const float* sn = scal + (k & 1) * 128;          // n[64], nv[64] of this tile
+            // the tile's norms (written with its B operands)
+            if (!warp_wait(bar(kBarBReady + b3), (uint32_t)ph3)) { failed = true; break; }
+            const float4* sn4 = reinterpret_cast<const float4*>(scal + b3 * 128);
             const int64_t tok0 = (int64_t)k * kPT;
             const int vis = lim - tok0 >= kPT ? kPT : (int)(lim > tok0 ? lim - tok0 : 0);
             float s[64];
+#pragma unroll
+            for (int t4 = 0; t4 < 16; ++t4) {
+                const float4 n4 = sn4[t4];
+                s[4 * t4 + 0] = __uint_as_float(sv[4 * t4 + 0]) * n4.x;
+                s[4 * t4 + 1] = __uint_as_float(sv[4 * t4 + 1]) * n4.y;
+                s[4 * t4 + 2] = __uint_as_float(sv[4 * t4 + 2]) * n4.z;
+                s[4 * t4 + 3] = __uint_as_float(sv[4 * t4 + 3]) * n4.w;
+            }
+            if (vis < kPT) {
+#pragma unroll
+                for (int t = 0; t < 64; ++t)
+                    if (t >= vis) s[t] = -INFINITY;
+            }
             float mt = -INFINITY;
 #pragma unroll
-            for (int t = 0; t < 64; ++t) {
-                s[t] = t < vis ? __uint_as_float(sv[t]) * a.scale_log2 * sn[t] : -INFINITY;
-                mt = fmaxf(mt, s[t]);
-            }
+            for (int t = 0; t < 64; ++t) mt = fmaxf(mt, s[t]);
             const float m_new = fmaxf(m_run, mt);
             m_run = m_new;
-            // the previous tile's P . V must be done before P and O are touched
-            if (k > 0 && !__all_sync(kFull, mbar_wait_bounded(bar_odone, (uint32_t)((k - 1) & 1)))) {
-                failed = true;
-                break;
-            }
+            // O += P(k-1) V(k-1) must be done before O is rescaled (and, for the
+            // barrier's phase tracking, every tile waits for it)
+            if (k > 0 && !warp_wait(bar(kBarODone), (uint32_t)((k - 1) & 1))) { failed = true; break; }
             tc_fence_after();
             // Move this row's reference maximum when it grew by more than 2^8; O is rescaled
-            // by the warp as a whole (tensor-memory loads and stores are warp-collective),
-            // with factor 1 on the rows that keep theirs.
+            // by the warp as a whole, with factor 1 on the rows that keep theirs.
             float f = 1.f;
             if (m_new != -INFINITY && (m_used == -INFINITY || m_new > m_used + kRescaleLog2)) {
                 if (m_used != -INFINITY) {                    // O and l were built on m_used
@@ -237,40 +272,29 @@ __global__ void __launch_bounds__(256, 1) tq_prefill_tc_kernel(const PrefillTcAr
                     tc_st32(tl + S::kColO + c0, ov);
                 }
             }
-            // P = 2^(s - m_used) nv: hi limbs in columns 0-31, lo limbs in 32-63 (tokens 2c, 2c + 1)
+            // P = 2^(s - m_used) nv 2^-6 over S: hi limbs in columns 0-31, lo limbs in
+            // 32-63 (tokens 2c, 2c + 1).  A row that has seen nothing yet (an absent
+            // row) keeps P = 0.
+            const float mu = m_used == -INFINITY ? 0.f : m_used;
             uint32_t ph[32], plo[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                float pv[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int t = 2 * c + e;
-                    const float p = s[t] == -INFINITY ? 0.f : fast_exp2(s[t] - m_used);
-                    l += p;
-                    pv[e] = p == 0.f ? 0.f : p * sn[64 + t] * kPScale;
-                }
-                split_hilo(pv[0], pv[1], ph[c], plo[c]);
+            for (int c4 = 0; c4 < 16; ++c4) {
+                const float4 v4 = sn4[16 + c4];
+                const float p0 = fast_exp2(s[4 * c4 + 0] - mu), p1 = fast_exp2(s[4 * c4 + 1] - mu);
+                const float p2 = fast_exp2(s[4 * c4 + 2] - mu), p3 = fast_exp2(s[4 * c4 + 3] - mu);
+                l += (p0 + p1) + (p2 + p3);
+                split_hilo(p0 * v4.x, p1 * v4.y, ph[2 * c4], plo[2 * c4]);
+                split_hilo(p2 * v4.z, p3 * v4.w, ph[2 * c4 + 1], plo[2 * c4 + 1]);
             }
-            uint32_t h16[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) h16[c] = ph[c];
-            tc_st16(tl + S::kColP, h16);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) h16[c] = ph[16 + c];
-            tc_st16(tl + S::kColP + 16, h16);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) h16[c] = plo[c];
-            tc_st16(tl + S::kColP + 32, h16);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) h16[c] = plo[16 + c];
-            tc_st16(tl + S::kColP + 48, h16);
+            tc_st32(tx, ph);
+            tc_st32(tx + 32, plo);
             tc_wait_st();
             tc_fence_before();
-            mbar_arrive(bar_sfree);
+            mbar_arrive(bar(kBarPReady + x));
+            if (++b3 == kPBuf) { b3 = 0; ph3 ^= 1; }
         }
-        // ---- the last tile's P . V, then this row's partial
-        if (!failed && ntile > 0 && !__all_sync(kFull, mbar_wait_bounded(bar_odone, (uint32_t)((ntile - 1) & 1))))
-            failed = true;
+        // ---- the last tile's P V, then this row's partial
+        if (!failed && !warp_wait(bar(kBarODone), (uint32_t)((ntile - 1) & 1))) failed = true;
         tc_fence_after();
         pdl_trigger();
         if (failed) atomicExch(a.err, 1);
@@ -295,147 +319,144 @@ __global__ void __launch_bounds__(256, 1) tq_prefill_tc_kernel(const PrefillTcAr
             a.part_ml[2 * qrow] = failed ? -INFINITY : m_used;
             a.part_ml[2 * qrow + 1] = failed ? 0.f : l;
         }
-    } else {
+    } else if (warp < 8) {
         // ======================================== producer warps: thread pt of 128
-        const int pt = tid - 128;
+        const int pt = tid - kSoftmaxThreads;
         const int tau = pt >> 1, hf = pt & 1;                   // token of the tile, half of its slots
         const uint32_t lut[4] = {a.cb.lut_lo[0], a.cb.lut_lo[1], a.cb.lut_hi[0], a.cb.lut_hi[1]};
         const uint32_t* pw = a.cb.pow2;
-        constexpr uint32_t kIdS = idesc_f16(128, kPT), kIdO = idesc_f16(128, kPD);
-        int n_s = 0, n_o = 0, n_ring = ntile < kPRing ? ntile : kPRing;
-        bool fail_mma = false;             // thread pt 0: a wait of the mma phase gave up
-        named_bar(2, 256);                 // the query operand is in place
-        tc_fence_after();
+        int n_ring = ntile < kPRing ? ntile : kPRing;
+        int b3 = 0, ph3 = 0;                                  // k % 3 (B buffer and ring stage), (k / 3) & 1
         for (int k = 0; k < ntile; ++k) {
-            const int buf = k & 1;
-            const uint8_t* st = sm + S::kOffRing + (k % kPRing) * S::kStage;
+            const uint8_t* st = sm + S::kOffRing + b3 * S::kStage;
             // every producer thread reaches the barrier below whatever happens, so that
             // the decision to stop is the same for all of them
-            bool f = fail_mma || !mbar_wait_bounded(smem_u32(&bars[k % kPRing]), (uint32_t)((k / kPRing) & 1));
-            // buffer buf was last read by tile k - 2's mma
-            if (!f && k >= 2) f = !mbar_wait_bounded(bar_odone, (uint32_t)((k - 2) & 1));
+            bool f = !mbar_wait_bounded(bar(kBarRing + b3), (uint32_t)ph3);
+            // buffer b3 was last read by the mma of tile k - 3
+            if (!f && k >= kPBuf) f = !mbar_wait_bounded(bar(kBarBFree + b3), (uint32_t)(ph3 ^ 1));
             if (!f) {
-            uint8_t* Kt = sm + buf * S::kBuf + S::kOffK;
-            uint8_t* Sg = sm + buf * S::kBuf + S::kOffS;
-            uint8_t* Vt = sm + buf * S::kBuf + S::kOffV;
-            const uint8_t* kb = st;
-            const uint8_t* vb = st + S::kKB;
-            const uint32_t gam = *reinterpret_cast<const uint16_t*>(kb + 64 * 64 + 128 + 2 * tau);
-            const uint32_t g2 = gam | (gam << 16);
+                uint8_t* Kt = sm + b3 * S::kBuf + S::kOffK;
+                uint8_t* Sg = sm + b3 * S::kBuf + S::kOffS;
+                uint8_t* Vt = sm + b3 * S::kBuf + S::kOffV;
+                const uint8_t* kb = st;
+                const uint8_t* vb = st + S::kKB;
+                const uint32_t gam = *reinterpret_cast<const uint16_t*>(kb + 64 * 64 + 128 + 2 * tau);
+                const uint32_t g2 = gam | (gam << 16);
 #pragma unroll
-            for (int tt = 0; tt < 2; ++tt) {
-                const int t = 2 * hf + tt;
-                uint32_t sel[4], vsel[4];
-                code_selectors(kb + tau * 48 + 12 * t, pw, sel);
-                code_selectors(vb + tau * 48 + 12 * t, pw, vsel);
-                // keys: K positions 32 t .. 32 t + 31 of row tau (four 16-byte chunks)
+                for (int tt = 0; tt < 2; ++tt) {
+                    const int t = 2 * hf + tt;
+                    uint32_t sel[4], vsel[4];
+                    code_selectors(kb + tau * 48 + 12 * t, pw, sel);
+                    code_selectors(vb + tau * 48 + 12 * t, pw, vsel);
+                    // keys: K positions 32 t .. 32 t + 31 of row tau (four 16-byte chunks)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t x[4];
-                    dequant4(sel_for(sel, pw, 2 * c), lut, x[0], x[1]);
-                    dequant4(sel_for(sel, pw, 2 * c + 1), lut, x[2], x[3]);
-                    *reinterpret_cast<uint4*>(Kt + sw128_byte(tau, 2 * (32 * t + 8 * c), kPT)) =
-                        make_uint4(x[0], x[1], x[2], x[3]);
-                }
-                // signs: +-gamma for JL rows at positions 2q, 2q + 1 (sign bits q, 16 + q)
-                const uint32_t w = *reinterpret_cast<const uint32_t*>(kb + 64 * 48 + tau * 16 + 4 * t);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t x[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int q = 4 * c + e;
-                        const uint32_t sh = shl_m(w, pw, 15 - q);         // bits q, 16 + q -> 15, 31
-                        x[e] = g2 ^ (~sh & 0x80008000u);                  // sigma = 0: -gamma
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t xk[4];
+                        dequant4(sel_for(sel, pw, 2 * c), lut, xk[0], xk[1]);
+                        dequant4(sel_for(sel, pw, 2 * c + 1), lut, xk[2], xk[3]);
+                        *reinterpret_cast<uint4*>(Kt + sw128_byte(tau, 2 * (32 * t + 8 * c), kPT)) =
+                            make_uint4(xk[0], xk[1], xk[2], xk[3]);
                     }
-                    *reinterpret_cast<uint4*>(Sg + sw128_byte(tau, 2 * (32 * t + 8 * c), kPT)) =
-                        make_uint4(x[0], x[1], x[2], x[3]);
-                }
-                // values: row = coordinate, K position = token tau
+                    // signs: +-gamma for JL rows at positions 2q, 2q + 1 (sign bits q, 16 + q)
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(kb + 64 * 48 + tau * 16 + 4 * t);
 #pragma unroll
-                for (int kc = 0; kc < 8; ++kc) {
-                    uint32_t x0, x1;
-                    dequant4(sel_for(vsel, pw, kc), lut, x0, x1);
-                    const int p = 4 * kc;
-                    const uint32_t v4[4] = {x0 & 0xFFFFu, x0 >> 16, x1 & 0xFFFFu, x1 >> 16};
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t xs[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        *reinterpret_cast<uint16_t*>(Vt + sw128_byte(slot_coord(0, t, p + e), 2 * tau, kPD)) =
-                            (uint16_t)v4[e];
-                }
-            }
-            if (hf == 0) {
-                scal[buf * 128 + tau] = __half2float(*reinterpret_cast<const __half*>(kb + 64 * 64 + 2 * tau));
-                scal[buf * 128 + 64 + tau] = __half2float(*reinterpret_cast<const __half*>(vb + 64 * 48 + 2 * tau));
-            }
-            fence_proxy_async();           // B operands written by threads, read by the tensor core
-            mbar_arrive(smem_u32(&bars[3 + buf]));
-            }
-            // every producer thread is done with stage k and buffer buf (or one gave up)
-            if (bar_or(1, 128, f)) { failed = true; break; }
-            if (pt == 0) {
-                if (k >= 1) {              // P of tile k - 1 is written: O += P V
-                    if (!mbar_wait_bounded(bar_sfree, (uint32_t)((k - 1) & 1))) {
-                        fail_mma = true;
-                    } else {
-                        tc_fence_after();
-                        const uint32_t vd = sbase + (uint32_t)(((k - 1) & 1) * S::kBuf + S::kOffV);
+                        for (int e = 0; e < 4; ++e) {
+                            const int q = 4 * c + e;
+                            const uint32_t sh = shl_m(w, pw, 15 - q);         // bits q, 16 + q -> 15, 31
+                            xs[e] = g2 ^ (~sh & 0x80008000u);                 // sigma = 0: -gamma
+                        }
+                        *reinterpret_cast<uint4*>(Sg + sw128_byte(tau, 2 * (32 * t + 8 * c), kPT)) =
+                            make_uint4(xs[0], xs[1], xs[2], xs[3]);
+                    }
+                    // values: row = coordinate, K position = token tau
 #pragma unroll
-                        for (int s = 0; s < 8; ++s)
-                            tc_mma_f16_ts(tmem + S::kColO, tmem + S::kColP + 8 * s, sw128_desc(vd + 32 * (s & 3)),
-                                          kIdO, (k - 1 > 0 || s > 0) ? 1u : 0u);
-                        tc_commit(bar_odone);
-                        ++n_o;
+                    for (int kc = 0; kc < 8; ++kc) {
+                        uint32_t x0, x1;
+                        dequant4(sel_for(vsel, pw, kc), lut, x0, x1);
+                        const int p = 4 * kc;
+                        const uint32_t v4[4] = {x0 & 0xFFFFu, x0 >> 16, x1 & 0xFFFFu, x1 >> 16};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            *reinterpret_cast<uint16_t*>(Vt + sw128_byte(slot_coord(0, t, p + e), 2 * tau, kPD)) =
+                                (uint16_t)v4[e];
                     }
                 }
-                if (!fail_mma) {           // S = [Q' | U'] [K ; K ; Sg ; Sg]^T
-                    const uint32_t kd = sbase + (uint32_t)(buf * S::kBuf + S::kOffK);
-                    const uint32_t sd = sbase + (uint32_t)(buf * S::kBuf + S::kOffS);
-#pragma unroll
-                    for (int s = 0; s < 32; ++s) {
-                        const int ss = s & 7;
-                        const uint32_t base = s < 16 ? kd : sd;
-                        const uint32_t addr = base + (uint32_t)((ss >> 2) * (kPT * 128) + (ss & 3) * 32);
-                        tc_mma_f16_ts(tmem + S::kColS, tmem + S::kColA + 8 * s, sw128_desc(addr), kIdS,
-                                      s > 0 ? 1u : 0u);
-                    }
-                    tc_commit(bar_sfull);
-                    ++n_s;
-                    if (k + kPRing < ntile) {
-                        fence_proxy_async();
-                        issue(k + kPRing);
-                        ++n_ring;
-                    }
+                if (hf == 0) {             // the tile's per-token factors for the softmax
+                    scal[b3 * 128 + tau] =
+                        __half2float(*reinterpret_cast<const __half*>(kb + 64 * 64 + 2 * tau)) * a.scale_log2;
+                    scal[b3 * 128 + 64 + tau] =
+                        __half2float(*reinterpret_cast<const __half*>(vb + 64 * 48 + 2 * tau)) * kPScale;
                 }
+                fence_proxy_async();       // B operands written by threads, read by the tensor core
+                mbar_arrive(bar(kBarBReady + b3));
             }
-        }
-        if (fail_mma) failed = true;
-        // the last tile's O += P V
-        if (pt == 0 && !failed && ntile > 0) {
-            if (!mbar_wait_bounded(bar_sfree, (uint32_t)((ntile - 1) & 1))) {
-                failed = true;
-            } else {
-                tc_fence_after();
-                const uint32_t vd = sbase + (uint32_t)(((ntile - 1) & 1) * S::kBuf + S::kOffV);
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    tc_mma_f16_ts(tmem + S::kColO, tmem + S::kColP + 8 * s, sw128_desc(vd + 32 * (s & 3)), kIdO,
-                                  (ntile - 1 > 0 || s > 0) ? 1u : 0u);
-                tc_commit(bar_odone);
-                ++n_o;
+            // every producer thread is done with stage b3 (or one gave up)
+            if (bar_or(1, kProducerThreads, f)) { failed = true; break; }
+            if (pt == 0 && k + kPRing < ntile) {
+                issue(k + kPRing);
+                ++n_ring;
             }
+            if (++b3 == kPBuf) { b3 = 0; ph3 ^= 1; }
         }
         if (pt == 0) {
-            // wait (bounded) for the mma and copies this thread issued
-            if (n_s > 0) mbar_wait_bounded(bar_sfull, (uint32_t)((n_s - 1) & 1));
-            if (n_o > 0) mbar_wait_bounded(bar_odone, (uint32_t)((n_o - 1) & 1));
             // only the last copy into each stage can still be in flight: an earlier one was
             // waited for before its stage was refilled (and a wait on an older phase of the
             // same parity as the current one would not return)
             for (int k = n_ring > kPRing ? n_ring - kPRing : 0; k < n_ring; ++k)
-                mbar_wait_bounded(smem_u32(&bars[k % kPRing]), (uint32_t)((k / kPRing) & 1));
+                mbar_wait_bounded(bar(kBarRing + k % kPRing), (uint32_t)((k / kPRing) & 1));
             if (failed) atomicExch(a.err, 1);
         }
+    } else if ((tid & 31) == 0) {
+        // ======================================== the mma thread
+        constexpr uint32_t kIdS = idesc_f16(128, kPT), kIdO = idesc_f16(128, kPD);
+        auto mma_o = [&](int k) {          // O += P(k) V(k)
+            const uint32_t vd = sbase + (uint32_t)((k % kPBuf) * S::kBuf + S::kOffV);
+            const uint32_t pa_t = tmem + S::kColX + 64 * (k & 1);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                tc_mma_f16_ts(tmem + S::kColO, pa_t + 8 * s, sw128_desc(vd + 32 * (s & 3)), kIdO,
+                              (k > 0 || s > 0) ? 1u : 0u);
+            tc_commit(bar(kBarODone));
+            tc_commit(bar(kBarBFree + k % kPBuf));
+        };
+        bool ok = mbar_wait_bounded(bar(kBarAReady), 0u);
+        int b3 = 0, ph3 = 0;
+        for (int k = 0; ok && k < ntile; ++k) {
+            // S(k) = [Q' | U'] [K ; K ; Sg ; Sg]^T into buffer k & 1 (its P(k - 2) was read by
+            // the O mma issued before this one)
+            if (!(ok = mbar_wait_bounded(bar(kBarBReady + b3), (uint32_t)ph3))) break;
+            tc_fence_after();
+            const uint32_t kd = sbase + (uint32_t)(b3 * S::kBuf + S::kOffK);
+            const uint32_t sd = sbase + (uint32_t)(b3 * S::kBuf + S::kOffS);
+            const uint32_t xd = tmem + S::kColX + 64 * (k & 1);
+#pragma unroll
+            for (int s = 0; s < 32; ++s) {
+                const int ss = s & 7;
+                const uint32_t base = s < 16 ? kd : sd;
+                const uint32_t addr = base + (uint32_t)((ss >> 2) * (kPT * 128) + (ss & 3) * 32);
+                tc_mma_f16_ts(xd, tmem + S::kColA + 8 * s, sw128_desc(addr), kIdS, s > 0 ? 1u : 0u);
+            }
+            tc_commit(bar(kBarSFull + (k & 1)));
+            if (k >= 1) {                  // P(k - 1) is written: O += P(k - 1) V(k - 1)
+                if (!(ok = mbar_wait_bounded(bar(kBarPReady + ((k - 1) & 1)), (uint32_t)(((k - 1) >> 1) & 1)))) break;
+                tc_fence_after();
+                mma_o(k - 1);
+            }
+            if (++b3 == kPBuf) { b3 = 0; ph3 ^= 1; }
+        }
+        if (ok && ntile > 0) {
+            if ((ok = mbar_wait_bounded(bar(kBarPReady + ((ntile - 1) & 1)), (uint32_t)(((ntile - 1) >> 1) & 1)))) {
+                tc_fence_after();
+                mma_o(ntile - 1);
+            }
+        }
+        // every mma this thread issued is done before tensor memory is released
+        tc_commit(bar(kBarDrain));
+        mbar_wait_bounded(bar(kBarDrain), 0u);
+        if (!ok) atomicExch(a.err, 1);
     }
     tc_fence_before();
     __syncthreads();
@@ -454,7 +475,7 @@ cudaError_t launch_prefill_tc(int G, const DecArgs& a, int64_t Lq, int64_t T0, c
     cudaError_t e = set_smem_once<tq_prefill_tc_kernel>(smem);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)tiles, (unsigned)a.Hkv, (unsigned)a.B);
-    return launch_pdl(tq_prefill_tc_kernel, grid, dim3(256), smem, s, pa);
+    return launch_pdl(tq_prefill_tc_kernel, grid, dim3(kThreads), smem, s, pa);
 }
 
 }  // namespace tqi
