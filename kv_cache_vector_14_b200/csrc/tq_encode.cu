@@ -460,7 +460,10 @@ cudaError_t launch_enc_dt(tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, 
 }  // namespace
 
 cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
-    if (d == 128) return launch_encode128(is_k, dt, a, num_sms, pdl, s);
+    if (d == 128) {
+        const cudaError_t e = launch_encode128_rot(is_k, dt, a, num_sms, pdl, s);
+        return e == cudaErrorNotSupported ? launch_encode128(is_k, dt, a, num_sms, pdl, s) : e;
+    }
     if (d == 64)
         return is_k ? launch_enc_dt<64, true>(dt, a, num_sms, pdl, s) : launch_enc_dt<64, false>(dt, a, num_sms, pdl, s);
     if (d == 256)

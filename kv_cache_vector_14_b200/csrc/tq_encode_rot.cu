@@ -1,0 +1,437 @@
+// TurboQuant K/V encode for head_dim 128 with the random rotation on the
+// 5th-generation tensor cores, for bulk encodes of contiguous bf16 / fp16
+// input on sm_100a.
+//
+// Page "Apple Silicon向けSwiftLM、TurboQuant KVキャッシュ圧縮とSSD Expert
+// Streamingを実装" (ai-heartland.com), section "K-Cache圧縮：3-bit PolarQuant +
+// 1-bit QJL = 4.25 bits/dim" (steps 1-5) and section "V-Cache圧縮：3-bit
+// PolarQuant = 3.125 bits/dim" (steps 1-3, no QJL).
+//
+// One tile is 128 consecutive input vectors (rows of the flattened [B, Hkv,
+// T, 128] input).  A TMA load brings the tile into shared memory in the
+// 128-byte-swizzled K-major layout; the tensor core computes
+//     Y = X (H D)^T          (8 tcgen05.mma, M = N = 128, K = 16)
+// into tensor memory: H D has entries +-1, exact in bf16 and fp16, so every
+// product is exact and only the fp32 accumulation rounds (as the butterflies
+// of the per-lane path do).  Then each of 128 threads owns one vector (its
+// tensor-memory lane): ||Y||^2 = 128 ||x||^2 gives the norm, y = Y / ||Y|| the
+// unit-sphere coordinates, the cell search and the centroid run on the FMA
+// pipe (saturated fused multiply-adds against the boundaries), and the codes
+// are packed into the token record.  For K, the residual r = y - c[idx] goes
+// back into the same tensor-memory columns as fp16 hi and lo limbs of r 2^12
+// (each 32-column chunk is overwritten only after it has been read), and the
+// tensor core computes the QJL projection from there:
+//     Z = R_hi S_hi^T + R_hi S_lo^T + R_lo S_hi^T   (24 tcgen05.mma, A in tensor memory)
+// whose sign bits are read out one tile later.  Warp 4 issues the TMA loads
+// (three tile buffers) and the mma (one thread); Y/R and Z are double-
+// buffered in tensor memory, so the rotation of the next tile and the
+// projection of this one overlap the quantisation.  Every wait is bounded.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "tq_frag.cuh"
+#include "tq_tc.cuh"
+
+namespace tqi {
+namespace {
+
+constexpr int kRD = 128;                  // head_dim
+constexpr int kRRows = 128;               // vectors per tile (tensor-memory lanes)
+constexpr int kRQuant = 128;              // quantiser threads, one vector each
+constexpr int kRThreads = kRQuant + 32;   // + the copy / mma warp
+constexpr int kRXBuf = 3;                 // input tile buffers
+constexpr int kRTile = kRRows * kRD * 2;  // one 16-bit 128 x 128 operand (32 KB)
+constexpr int64_t kRotMinVectors = 16384; // smaller encodes keep the per-lane kernels
+constexpr float kRScale = 4096.f;         // residual scale before the fp16 split
+
+template <bool IS_K>
+struct RotShape {
+    static constexpr int kOffM = 0;                              // rotation operand H D
+    static constexpr int kOffS = kRTile;                         // K: JL operand, hi then lo limb
+    static constexpr int kOffX = IS_K ? 3 * kRTile : kRTile;     // input tiles
+    static constexpr int kOffBar = kOffX + kRXBuf * kRTile;
+    static constexpr int kOffMisc = kOffBar + 16 * 8;
+    static constexpr int kSmem = kOffMisc + 16 + 1024;           // + slack to align the base
+    static constexpr int kCols = IS_K ? 512 : 256;               // Y/R x 2 (+ Z x 2)
+};
+static_assert(RotShape<true>::kSmem <= 227 * 1024, "shared memory per CTA");
+
+// mbarriers
+enum : int {
+    kRBarB = 0,       // JL operand copied (K)
+    kRBarXFull = 1,   // [3] input tile landed (TMA bytes)
+    kRBarXFree = 4,   // [3] input tile read by its rotation (commit)
+    kRBarYFull = 7,   // [2] Y computed (commit)
+    kRBarRFull = 9,   // [2] Y read and, for K, R written (128 quantiser arrivals)
+    kRBarZFull = 11,  // [2] Z computed (commit)
+    kRBarDrain = 13,  // every mma of the mma thread done (commit, at exit)
+};
+
+__device__ __forceinline__ bool warp_wait_r(uint32_t bar, uint32_t parity) {
+    return __all_sync(kFull, mbar_wait_bounded(bar, parity));
+}
+
+template <int DT, bool IS_K>
+__global__ void __launch_bounds__(kRThreads, 1)
+    tq_encode_rot_kernel(const __grid_constant__ CUtensorMap tmap, const EncArgs a) {
+    using S = RotShape<IS_K>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + S::kOffBar);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + S::kOffMisc);
+    pdl_trigger();                 // a chained kernel may start (it waits for this one's writes)
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int64_t N = a.B * a.Hkv * a.Tnew;
+    const int64_t ntiles = (N + kRRows - 1) / kRRows;
+    const int n = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);   // this CTA's tiles
+    auto row0_of = [&](int j) { return ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kRRows; };
+    const int64_t bb = block_bytes(kRD, IS_K);
+
+    if (tid == 0) {
+        mbar_init(bar(kRBarB), 1);
+        for (int i = 0; i < kRXBuf; ++i) {
+            mbar_init(bar(kRBarXFull + i), 1);
+            mbar_init(bar(kRBarXFree + i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(kRBarYFull + i), 1);
+            mbar_init(bar(kRBarRFull + i), kRQuant);
+            mbar_init(bar(kRBarZFull + i), 1);
+        }
+        mbar_init(bar(kRBarDrain), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc_alloc(smem_u32(tmem_slot), S::kCols);
+        tc_relinquish();
+    }
+    // Rotation operand, row j (output coordinate), K index i (input coordinate):
+    // (-1)^popcount(i & j) d_i, the Walsh-Hadamard matrix in natural order times
+    // the random signs, as bf16 / fp16 +-1.
+    if (tid < kRQuant) {
+        const int j = tid;
+        const uint32_t one = DT == TQ_BF16 ? 0x3F80u : 0x3C00u;
+#pragma unroll 1
+        for (int i0 = 0; i0 < kRD; i0 += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                uint32_t h2[2];
+#pragma unroll
+                for (int f = 0; f < 2; ++f) {
+                    const int i = i0 + 2 * e + f;
+                    const uint32_t neg = ((uint32_t)__popc(i & j) & 1u) ^ (__ldg(a.dsign + i) < 0.f ? 1u : 0u);
+                    h2[f] = one | (neg << 15);
+                }
+                w[e] = h2[0] | (h2[1] << 16);
+            }
+            *reinterpret_cast<uint4*>(sm + S::kOffM + sw128_byte(j, 2 * i0, kRD)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async();           // written by threads, read by the tensor core
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (tid == kRQuant) {
+        // ======================================== copy and mma thread
+        constexpr uint32_t kIdY = DT == TQ_BF16 ? idesc_bf16(kRRows, kRD) : idesc_f16(kRRows, kRD);
+        constexpr uint32_t kIdZ = idesc_f16(kRRows, kRD);
+        auto load = [&](int j) {       // input tile j -> buffer j % 3 (two 64-column boxes)
+            const int bx = j % kRXBuf;
+            const uint32_t dst = sbase + (uint32_t)(S::kOffX + bx * kRTile), br = bar(kRBarXFull + bx);
+            mbar_expect_tx(br, (uint32_t)kRTile);
+            const int r0 = (int)row0_of(j);
+            tma_load_2d(dst, &tmap, 0, r0, br);
+            tma_load_2d(dst + kRTile / 2, &tmap, 64, r0, br);
+        };
+        int n_load = n < kRXBuf ? n : kRXBuf;
+        for (int j = 0; j < n_load; ++j) load(j);
+        bool ok = true;
+        if constexpr (IS_K) {
+            mbar_expect_tx(bar(kRBarB), (uint32_t)(2 * kRTile));
+            bulk_g2s(sbase + (uint32_t)S::kOffS, a.bimg, (uint32_t)(2 * kRTile), bar(kRBarB));
+            ok = mbar_wait_bounded(bar(kRBarB), 0u);
+        }
+        // Z(j) = R_hi S_hi^T + R_hi S_lo^T + R_lo S_hi^T.  R(j) lies in Y(j)'s columns:
+        // coordinates 32 c + 2 m, + 1 in column 32 c + m (hi) and 32 c + 16 + m (lo).
+        auto qjl = [&](int j) {
+            const uint32_t rb = tmem + (uint32_t)(128 * (j & 1)), zd = tmem + 256u + (uint32_t)(128 * (j & 1));
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t koff = (uint32_t)((ks >> 2) * (kRRows * 128) + (ks & 3) * 32);
+                const uint32_t ahi = rb + (uint32_t)(32 * (ks >> 1) + 8 * (ks & 1)), alo = ahi + 16u;
+                const uint64_t bhi = sw128_desc(sbase + (uint32_t)S::kOffS + koff);
+                const uint64_t blo = sw128_desc(sbase + (uint32_t)(S::kOffS + kRTile) + koff);
+                tc_mma_f16_ts(zd, ahi, bhi, kIdZ, ks > 0 ? 1u : 0u);
+                tc_mma_f16_ts(zd, ahi, blo, kIdZ, 1u);
+                tc_mma_f16_ts(zd, alo, bhi, kIdZ, 1u);
+            }
+            tc_commit(bar(kRBarZFull + (j & 1)));
+        };
+        for (int j = 0; ok && j < n; ++j) {
+            const int bx = j % kRXBuf;
+            if (!(ok = mbar_wait_bounded(bar(kRBarXFull + bx), (uint32_t)((j / kRXBuf) & 1)))) break;
+            // Y(j) overwrites buffer j % 2: the quantisers are done with tile j - 2 there, and
+            // (K) its R was read by the projection mma, issued before this one
+            if (j >= 2 && !(ok = mbar_wait_bounded(bar(kRBarRFull + (j & 1)), (uint32_t)(((j - 2) >> 1) & 1)))) break;
+            tc_fence_after();
+            const uint32_t xa = sbase + (uint32_t)(S::kOffX + bx * kRTile);
+            const uint32_t yd = tmem + (uint32_t)(128 * (j & 1));
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t koff = (uint32_t)((ks >> 2) * (kRRows * 128) + (ks & 3) * 32);
+                tc_mma_f16_ss(yd, sw128_desc(xa + koff), sw128_desc(sbase + (uint32_t)S::kOffM + koff), kIdY,
+                              ks > 0 ? 1u : 0u);
+            }
+            tc_commit(bar(kRBarYFull + (j & 1)));
+            tc_commit(bar(kRBarXFree + bx));
+            if constexpr (IS_K) {
+                if (j >= 1) {          // R(j - 1) is written: its projection
+                    if (!(ok = mbar_wait_bounded(bar(kRBarRFull + ((j - 1) & 1)), (uint32_t)(((j - 1) >> 1) & 1))))
+                        break;
+                    tc_fence_after();
+                    qjl(j - 1);
+                }
+            }
+            // tile j + 2 goes into tile j - 1's buffer once that tile's rotation is done
+            if (j >= 1 && j + 2 < n) {
+                if (!(ok = mbar_wait_bounded(bar(kRBarXFree + (j - 1) % kRXBuf), (uint32_t)(((j - 1) / kRXBuf) & 1))))
+                    break;
+                load(j + 2);
+                ++n_load;
+            }
+        }
+        if constexpr (IS_K) {
+            if (ok && n > 0) {
+                if ((ok = mbar_wait_bounded(bar(kRBarRFull + ((n - 1) & 1)), (uint32_t)(((n - 1) >> 1) & 1)))) {
+                    tc_fence_after();
+                    qjl(n - 1);
+                }
+            }
+        }
+        // every mma and copy this thread issued is done before shared and tensor memory are
+        // released (only the last load into each buffer can still be in flight)
+        tc_commit(bar(kRBarDrain));
+        mbar_wait_bounded(bar(kRBarDrain), 0u);
+        for (int j = n_load > kRXBuf ? n_load - kRXBuf : 0; j < n_load; ++j)
+            mbar_wait_bounded(bar(kRBarXFull + j % kRXBuf), (uint32_t)((j / kRXBuf) & 1));
+        if (!ok) atomicExch(a.err, 1);
+    } else if (tid < kRQuant) {
+        // ======================================== quantisers: thread r = vector r of the tile
+        const int r = tid;
+        const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+        const Codebook& cb = a.cb;
+        // Bucket index and centroid on the FMA pipe.  The codebook is antisymmetric
+        // (b3 = 0, b[6-k] = -b[k], c[7-k] = -c[k]), so with a = |y| and
+        // t_k = sat((b_k - a) 2^60) = [a < b_k] for k = 4, 5, 6 (the product is exact,
+        // its sign decides, and any nonzero difference of two such floats saturates),
+        // T = t4 + t5 + t6 boundaries lie above a: the code is 7 - T for y >= 0 and T
+        // below, and |c| = c7 - t6 (c7 - c6) - t5 (c6 - c5) - t4 (c5 - c4), every partial
+        // sum an exact centroid.
+        constexpr float kBig = 1152921504606846976.f;        // 2^60
+        const float bb4 = cb.b[4] * kBig, bb5 = cb.b[5] * kBig, bb6 = cb.b[6] * kBig;
+        [[maybe_unused]] const float d3 = cb.c[7] - cb.c[6], d2 = cb.c[6] - cb.c[5], d1 = cb.c[5] - cb.c[4];
+        bool ok = true;
+        // sign words of tile jj (K): bit b of word w is z[32 w + b] >= 0
+        auto signs = [&](int jj) -> bool {
+            if (!warp_wait_r(bar(kRBarZFull + (jj & 1)), (uint32_t)((jj >> 1) & 1))) return false;
+            tc_fence_after();
+            const uint32_t zb = tl + 256u + (uint32_t)(128 * (jj & 1));
+            uint32_t sw0 = 0, sw1 = 0, sw2 = 0, sw3 = 0;
+#pragma unroll 1
+            for (int w = 0; w < 4; ++w) {
+                uint32_t z[32];
+                tc_ld32(zb + (uint32_t)(32 * w), z);
+                uint32_t word = 0;
+#pragma unroll
+                for (int bt = 0; bt < 32; ++bt) word |= (__uint_as_float(z[bt]) >= 0.f ? 1u : 0u) << bt;
+                sw0 = w == 0 ? word : sw0;
+                sw1 = w == 1 ? word : sw1;
+                sw2 = w == 2 ? word : sw2;
+                sw3 = w == 3 ? word : sw3;
+            }
+            const int64_t gv = row0_of(jj) + r;
+            if (gv < N) {
+                int64_t xoff;
+                uint8_t* blk;
+                int tau;
+                encode_locate(a, (uint32_t)gv, bb, xoff, blk, tau);
+                if (blk)
+                    *reinterpret_cast<uint4*>(blk + kBlockT * code_bytes(kRD) + tau * sign_bytes(kRD)) =
+                        make_uint4(sw0, sw1, sw2, sw3);
+            }
+            return true;
+        };
+        for (int j = 0; j < n; ++j) {
+            const int64_t gv = row0_of(j) + r;
+            if (!(ok = warp_wait_r(bar(kRBarYFull + (j & 1)), (uint32_t)((j >> 1) & 1)))) break;
+            tc_fence_after();
+            const uint32_t yb = tl + (uint32_t)(128 * (j & 1));
+            // ||Y||^2 = 128 ||x||^2
+            float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tc_ld32(yb + (uint32_t)(32 * c), v);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) s4[e & 3] = fmaf(__uint_as_float(v[e]), __uint_as_float(v[e]), s4[e & 3]);
+            }
+            const float ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+            const float nrm = sqrtf(ss * (1.f / 128.f));
+            const bool nz = ss > 0.f;
+            const float rcp = nz ? __frcp_rn(sqrtf(ss)) : 0.f;   // y = Y / ||Y||
+            // Codes in the token record: word 3 t + g holds, in nibble i, the code of slot
+            // position 8 g + i (bits 0-2) and bit g of the code of position 24 + i (bit 3).
+            // Position p of slot t is coordinate slot_coord(0, t, p), so chunk c (coordinates
+            // 32 c .. 32 c + 31) fills words 3 t + c for c < 3 and the bit-3 planes for c = 3;
+            // nibble i of slot t is the chunk's coordinate o(t, i) = 16 (i / 4) + 2 t + (i % 2)
+            // + 8 ((i / 2) % 2).
+            uint32_t wd[12];
+#pragma unroll
+            for (int i = 0; i < 12; ++i) wd[i] = 0u;
+            float g2 = 0.f;
+            // (K: the chunk loop stays rolled; unrolled, the code with the residual outgrows
+            // the instruction cache)
+#pragma unroll(IS_K ? 1 : 4)
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tc_ld32(yb + (uint32_t)(32 * c), v);
+                float cf[32];
+                [[maybe_unused]] uint32_t rh[16], rl[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    [[maybe_unused]] float rr[2];
+#pragma unroll
+                    for (int f = 0; f < 2; ++f) {
+                        const float y = __uint_as_float(v[e + f]) * rcp;
+                        const float av = fabsf(y);
+                        const float t4 = __saturatef(fmaf(av, -kBig, bb4));
+                        const float t5 = __saturatef(fmaf(av, -kBig, bb5));
+                        const float t6 = __saturatef(fmaf(av, -kBig, bb6));
+                        const float T = (t4 + t5) + t6;
+                        const float pos = (y >= 0.f) ? 1.f : 0.f;
+                        cf[e + f] = fmaf(pos, fmaf(T, -2.f, 7.f), T);
+                        if constexpr (IS_K) {
+                            float m = fmaf(-t6, d3, cb.c[7]);
+                            m = fmaf(-t5, d2, m);
+                            m = fmaf(-t4, d1, m);
+                            const float rv = nz ? y - m * fmaf(pos, 2.f, -1.f) : 0.f;
+                            g2 = fmaf(rv, rv, g2);
+                            rr[f] = rv * kRScale;
+                        }
+                    }
+                    if constexpr (IS_K) split_hilo(rr[0], rr[1], rh[e >> 1], rl[e >> 1]);
+                }
+                if constexpr (IS_K) {      // R over the chunk just read
+                    tc_st16(yb + (uint32_t)(32 * c), rh);
+                    tc_st16(yb + (uint32_t)(32 * c + 16), rl);
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    // nibbles 0-3 and 4-7 as exact float sums, read out of the mantissa (x + 2^23)
+                    const float lo = fmaf(cf[2 * t + 9], 4096.f, fmaf(cf[2 * t + 8], 256.f, fmaf(cf[2 * t + 1], 16.f, cf[2 * t])));
+                    const float hi =
+                        fmaf(cf[2 * t + 25], 4096.f, fmaf(cf[2 * t + 24], 256.f, fmaf(cf[2 * t + 17], 16.f, cf[2 * t + 16])));
+                    const uint32_t W = __byte_perm(__float_as_uint(lo + 8388608.f), __float_as_uint(hi + 8388608.f), 0x5410);
+                    // (register indices fixed at compile time, selected by the chunk)
+                    wd[3 * t + 0] = c == 0 ? W : c == 3 ? wd[3 * t + 0] | ((W & 0x11111111u) << 3) : wd[3 * t + 0];
+                    wd[3 * t + 1] = c == 1 ? W : c == 3 ? wd[3 * t + 1] | (((W >> 1) & 0x11111111u) << 3) : wd[3 * t + 1];
+                    wd[3 * t + 2] = c == 2 ? W : c == 3 ? wd[3 * t + 2] | (((W >> 2) & 0x11111111u) << 3) : wd[3 * t + 2];
+                }
+            }
+            if constexpr (IS_K) tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(kRBarRFull + (j & 1)));
+            if (gv < N) {
+                int64_t xoff;
+                uint8_t* blk;
+                int tau;
+                encode_locate(a, (uint32_t)gv, bb, xoff, blk, tau);
+                if (blk) {
+                    uint4* rec = reinterpret_cast<uint4*>(blk + tau * code_bytes(kRD));
+                    rec[0] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+                    rec[1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+                    rec[2] = make_uint4(wd[8], wd[9], wd[10], wd[11]);
+                    __half* nf = reinterpret_cast<__half*>(blk + kBlockT * (code_bytes(kRD) + (IS_K ? sign_bytes(kRD) : 0)));
+                    nf[tau] = __float2half_rn(nrm);
+                    if constexpr (IS_K) nf[kBlockT + tau] = __float2half_rn(sqrtf(g2));
+                }
+            }
+            if constexpr (IS_K) {          // the previous tile's projection ran meanwhile
+                if (j >= 1 && !(ok = signs(j - 1))) break;
+            }
+        }
+        if constexpr (IS_K) {
+            if (ok && n > 0) ok = signs(n - 1);
+        }
+        if (!ok && (tid & 31) == 0) atomicExch(a.err, 1);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tc_dealloc(tmem, S::kCols);
+    }
+    pdl_wait();                    // when chained: complete only after the previous kernel
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+template <int DT, bool IS_K>
+cudaError_t launch_rot_t(const CUtensorMap& tm, const EncArgs& a, int grid, bool pdl, cudaStream_t s) {
+    constexpr int smem = RotShape<IS_K>::kSmem;
+    cudaError_t e = set_smem_once<tq_encode_rot_kernel<DT, IS_K>>(smem);
+    if (e != cudaSuccess) return e;
+    if (pdl) return launch_pdl(tq_encode_rot_kernel<DT, IS_K>, dim3(grid), dim3(kRThreads), smem, s, tm, a);
+    tq_encode_rot_kernel<DT, IS_K><<<grid, kRThreads, smem, s>>>(tm, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_encode128_rot(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
+    if (dt != TQ_BF16 && dt != TQ_F16) return cudaErrorNotSupported;
+    const int64_t N = a.B * a.Hkv * a.Tnew;
+    if (N < kRotMinVectors || !a.vec16) return cudaErrorNotSupported;
+    // rows of the flattened input must be consecutive 256-byte rows
+    if (a.st != kRD || (a.Hkv > 1 && a.sh != a.Tnew * kRD) || (a.B > 1 && a.sb != a.Hkv * a.Tnew * kRD))
+        return cudaErrorNotSupported;
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    CUtensorMap tm;
+    const cuuint64_t dims[2] = {(cuuint64_t)kRD, (cuuint64_t)N};
+    const cuuint64_t strides[1] = {(cuuint64_t)kRD * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kRRows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(&tm, dt == TQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                           const_cast<void*>(a.x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorNotSupported;
+    const int64_t ntiles = (N + kRRows - 1) / kRRows;
+    const int grid = (int)(ntiles < num_sms ? ntiles : num_sms);
+    if (dt == TQ_BF16)
+        return is_k ? launch_rot_t<TQ_BF16, true>(tm, a, grid, pdl, s) : launch_rot_t<TQ_BF16, false>(tm, a, grid, pdl, s);
+    return is_k ? launch_rot_t<TQ_F16, true>(tm, a, grid, pdl, s) : launch_rot_t<TQ_F16, false>(tm, a, grid, pdl, s);
+}
+
+}  // namespace tqi

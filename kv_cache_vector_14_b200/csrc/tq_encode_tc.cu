@@ -320,21 +320,6 @@ __device__ __forceinline__ uint32_t pack_code_word(const uint8_t* rec, int w) {
     return main | (((tail >> g) & 0x11111111u) << 3);
 }
 
-// Input offset and cache block of vector gv (b, h, token order); blk is null
-// when a paged cache's table entry lies outside its pool.
-__device__ __forceinline__ void locate(const EncArgs& a, uint32_t gv, int64_t bb, int64_t& xoff, uint8_t*& blk,
-                                       int& tau) {
-    const uint32_t bh = fdiv(gv, a.fdT);
-    const uint32_t tt = gv - bh * (uint32_t)a.Tnew;
-    const uint32_t b = fdiv(bh, a.fdH);
-    const uint32_t hh = bh - b * (uint32_t)a.Hkv;
-    xoff = (int64_t)b * a.sb + (int64_t)hh * a.sh + (int64_t)tt * a.st;
-    const int64_t t = a.t0 + tt;
-    tau = (int)(t & 63);
-    const int64_t pb = cache_block(a.table, a.pool, a.NB, bh, t >> 6, a.err);
-    blk = pb >= 0 ? a.cache + pb * bb : nullptr;                   // null: nothing is written
-}
-
 // The 12 code words of each of the warp's four vectors (group g holds vector
 // g; my_rec is the code record of this lane's vector, null to skip) from the
 // staged bytes.
@@ -423,7 +408,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
             int64_t xoff;
             uint8_t* blk;
             int tau;
-            locate(a, (uint32_t)(r0 + v), bb, xoff, blk, tau);
+            encode_locate(a, (uint32_t)(r0 + v), bb, xoff, blk, tau);
             if (blk)
                 reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(kD) + tau * sign_bytes(kD))[warp >> 2] = word;
         }
@@ -446,7 +431,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) tq_encode_k128_tc_kernel(const
             int64_t xoff;
             uint8_t* blk;
             int tau;
-            locate(a, (uint32_t)(row0 + (valid ? v : r0)), bb, xoff, blk, tau);
+            encode_locate(a, (uint32_t)(row0 + (valid ? v : r0)), bb, xoff, blk, tau);
             GroupOut o;
             encode_group<DT, true>(a.x, xoff, valid, vec, l, dsg, a.cb, o);
             *reinterpret_cast<uint4*>(A + sw128_k_offset(v, 16 * l)) = make_uint4(o.rh[0], o.rh[1], o.rh[2], o.rh[3]);
@@ -531,7 +516,7 @@ __global__ void __launch_bounds__(kVWarps * 32, 3) tq_encode_v128_kernel(const E
         int64_t xoff;
         uint8_t* blk;
         int tau;
-        locate(a, (uint32_t)(valid ? gv0 + g : gv0), bb, xoff, blk, tau);
+        encode_locate(a, (uint32_t)(valid ? gv0 + g : gv0), bb, xoff, blk, tau);
         GroupOut o;
         encode_group<DT, false>(a.x, xoff, valid, vec, l, dsg, a.cb, o);
 #pragma unroll

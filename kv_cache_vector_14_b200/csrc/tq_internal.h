@@ -159,6 +159,21 @@ __device__ __forceinline__ int64_t cache_block(const int32_t* table, int64_t poo
     }
     return p;
 }
+
+// Input offset (elements) and cache block of vector gv (b, h, token order) of an
+// encode; blk is null when a paged cache's table entry lies outside its pool.
+__device__ __forceinline__ void encode_locate(const EncArgs& a, uint32_t gv, int64_t bb, int64_t& xoff, uint8_t*& blk,
+                                              int& tau) {
+    const uint32_t bh = fdiv(gv, a.fdT);
+    const uint32_t tt = gv - bh * (uint32_t)a.Tnew;
+    const uint32_t b = fdiv(bh, a.fdH);
+    const uint32_t hh = bh - b * (uint32_t)a.Hkv;
+    xoff = (int64_t)b * a.sb + (int64_t)hh * a.sh + (int64_t)tt * a.st;
+    const int64_t t = a.t0 + tt;
+    tau = (int)(t & 63);
+    const int64_t pb = cache_block(a.table, a.pool, a.NB, bh, t >> 6, a.err);
+    blk = pb >= 0 ? a.cache + pb * bb : nullptr;                   // null: nothing is written
+}
 #endif
 
 // Programmatic dependent launch: a kernel launched with launch_pdl may start
@@ -203,6 +218,9 @@ cudaError_t set_smem_once(int bytes) {
 cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl,
                           cudaStream_t s);
 cudaError_t launch_encode128(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s);
+// Bulk d = 128 encode of contiguous bf16 / fp16 input with the rotation on the
+// tensor cores; cudaErrorNotSupported when the call does not qualify.
+cudaError_t launch_encode128_rot(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s);
 // pdl: launched as a programmatic dependent of the previous kernel (fused
 // append-and-attend step); the kernels then complete only after it.
 cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, const float* dsign,

@@ -19,13 +19,17 @@
 //        holds <q', c[idx]> + gamma <u', 2 sigma - 1>)
 //   O[128 rows][128 coords] += [Phi | Plo] [Vdeq ; Vdeq]
 //       (A in tensor memory: the softmax weights p * nv, scaled by 2^-6, as
-//        fp16 hi and lo limbs; B in shared memory: the values' centroids, one row per
-//        coordinate along tokens)
-// Warp roles: warps 4-7 stage the cache blocks (bulk copies into a ring)
+//        fp16 hi and lo limbs; B in shared memory, MN-major: the values'
+//        centroids, one 256-byte row per token, the coordinates in the same
+//        slot order as the keys, so O's column 32 t + p is coordinate
+//        slot_coord(0, t, p))
+// Warp roles: warps 8-10 stage the cache blocks (bulk copies into a ring)
 // and expand the codes into the B operands (three buffers, so they run up to
-// two tiles ahead); warp 8 issues the mma (one thread); warps 0-3 own one row
-// each per thread (tensor-memory lane = row): they load S, apply the norms,
-// the causal mask and the online softmax, and write P over S in tensor memory.
+// two tiles ahead); warp 11 issues the mma (one thread); warps 0-7 own one
+// half row each per thread (tensor-memory lane = row; warpgroup h takes
+// tokens 32 h .. 32 h + 31 of a tile): they load S, apply the norms, the
+// causal mask and the online softmax (the two halves of a row exchange their
+// maxima through shared memory), and write P over S in tensor memory.
 // S and P have two tensor-memory buffers, so the tensor core computes the
 // scores of tile k + 1 while the softmax works on tile k; the mma of one
 // thread run in issue order, so S(k + 2) cannot overwrite P(k) before O += P(k)
@@ -44,7 +48,7 @@ constexpr int kPT = 64;                  // tokens per tile (one cache block)
 constexpr int kPRows = 128;              // query rows per CTA
 constexpr int kPRing = 3;                // raw block stages
 constexpr int kPBuf = 3;                 // B operand buffers
-constexpr int kSoftmaxThreads = 128, kProducerThreads = 128;
+constexpr int kSoftmaxThreads = 256, kProducerThreads = 96;      // two softmax warpgroups, three producer warps
 constexpr int kThreads = kSoftmaxThreads + kProducerThreads + 32;   // + the mma warp
 constexpr float kRescaleLog2 = 8.f;      // move the maximum used for P only when it grows by more than this
 constexpr float kPScale = 1.f / 64.f;    // P holds p nv 2^-6 (p <= 2^8, so fp16 holds it unless nv > 2^14)
@@ -52,8 +56,8 @@ constexpr float kPScale = 1.f / 64.f;    // P holds p nv 2^-6 (p <= 2^8, so fp16
 struct PtcShape {
     static constexpr int kKB = 64 * 48 + 64 * 16 + 256;     // K block bytes
     static constexpr int kVB = 64 * 48 + 128;                // V block bytes
-    // B buffers: keys [64 tok][128 coords] fp16, signs [64 tok][128 rows] fp16,
-    // values [128 coords][64 tok] fp16; 128-byte swizzled, K-major
+    // B buffers: keys [64 tok][128 coords] fp16, signs [64 tok][128 rows] fp16 (K-major),
+    // values [64 tok][128 coords] fp16 (MN-major); 128-byte swizzled, coordinates in slot order
     static constexpr int kOffK = 0;
     static constexpr int kOffS = 16384;
     static constexpr int kOffV = 32768;
@@ -63,7 +67,8 @@ struct PtcShape {
     static constexpr int kStage = kKB + kVB;
     static constexpr int kOffBar = kOffRing + kPRing * kStage;
     static constexpr int kNumBars = 16;
-    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kOffXchg = kOffBar + kNumBars * 8;  // row maxima [2 tiles][2 halves][128], sums [2][128]
+    static constexpr int kOffMisc = kOffXchg + 6 * 128 * 4;
     static constexpr int kSmem = kOffMisc + 64 + 1024;       // + slack to align the base
     // tensor memory: the query operand (4 x 64 columns), S / P (two buffers), O
     static constexpr int kColA = 0;
@@ -77,12 +82,12 @@ static_assert(PtcShape::kSmem <= 227 * 1024, "shared memory per CTA");
 // mbarriers (index into the barrier array)
 enum : int {
     kBarRing = 0,     // [3] raw stage filled (bulk copy bytes)
-    kBarBReady = 3,   // [3] B buffer built (128 producer arrivals)
+    kBarBReady = 3,   // [3] B buffer built (96 producer arrivals)
     kBarBFree = 6,    // [3] B buffer read by S and O of its tile (commit)
     kBarSFull = 9,    // [2] S computed into buffer x (commit)
-    kBarPReady = 11,  // [2] P written into buffer x (128 softmax arrivals)
+    kBarPReady = 11,  // [2] P written into buffer x (256 softmax arrivals)
     kBarODone = 13,   // O += P V of a tile done (commit)
-    kBarAReady = 14,  // query operand in tensor memory (128 softmax arrivals)
+    kBarAReady = 14,  // query operand in tensor memory (256 softmax arrivals)
     kBarDrain = 15,   // every mma issued by the mma thread done (commit, at exit)
 };
 
@@ -104,9 +109,6 @@ __device__ __forceinline__ bool bar_or(int id, int n, bool v) {
         : "r"((uint32_t)v), "r"(id), "r"(n)
         : "memory");
     return r != 0;
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 // warp-uniform bounded wait (the warp then runs warp-collective tensor-memory instructions)
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
@@ -171,36 +173,37 @@ __global__ void __launch_bounds__(kThreads, 1) tq_prefill_tc_kernel(const Prefil
     pdl_wait();                            // q' and u' come from the prologue kernel
 
     bool failed = false;
-    if (warp < 4) {
-        // ======================================== softmax warps: thread r = row r
-        const int r = tid;
-        const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+    if (warp < 8) {
+        // ======================================== softmax warps: thread = (row, half); warp w
+        // reaches tensor-memory lanes 32 (w % 4) .. +31, warpgroup h = w / 4 takes tokens
+        // 32 h .. 32 h + 31 of every tile and O columns 64 h .. 64 h + 63
+        const int hh = warp >> 2;
+        const int r = 32 * (warp & 3) + (tid & 31);
+        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        float* xm = reinterpret_cast<float*>(sm + S::kOffXchg);             // [2][2][128]
+        float* xl = xm + 4 * 128;                                            // [2][128]
         const int64_t grow = row0 + r;
         const bool rvalid = grow < nrows;
         const int64_t qi = rvalid ? grow / G : 0, qg = rvalid ? grow % G : 0;
         const int64_t qrow = ((int64_t)b * pa.Lq + qi) * a.Hq + (int64_t)hkv * G + qg;
         const int64_t lim = rvalid ? pa.T0 + qi + 1 : 0;          // tokens [0, lim) visible
-        // query operand: column c of each 64-column part holds K positions 2c, 2c + 1;
-        // K position kappa = 32 t + p is coordinate (JL row) slot_coord(0, t, p)
+        // query operand (warpgroup 0: q', warpgroup 1: u'): column c of each 64-column
+        // part holds K positions 2c, 2c + 1; K position kappa = 32 t + p is coordinate
+        // (JL row) slot_coord(0, t, p)
         {
-            const float* qp = a.qp + qrow * kPD;
-            const float* up = a.up + qrow * kPD;
+            const float* src = (hh == 0 ? a.qp : a.up) + qrow * kPD;
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {           // q', u'
-                const float* src = part == 0 ? qp : up;
+            for (int c0 = 0; c0 < 64; c0 += 16) {
+                uint32_t hi[16], lo[16];
 #pragma unroll
-                for (int c0 = 0; c0 < 64; c0 += 16) {
-                    uint32_t hi[16], lo[16];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const int kap = 2 * (c0 + c), t = kap >> 5, p = kap & 31;
-                        const float x0 = rvalid ? src[slot_coord(0, t, p)] : 0.f;
-                        const float x1 = rvalid ? src[slot_coord(0, t, p + 1)] : 0.f;
-                        split_hilo(x0, x1, hi[c], lo[c]);
-                    }
-                    tc_st16(tl + S::kColA + 128 * part + c0, hi);
-                    tc_st16(tl + S::kColA + 128 * part + 64 + c0, lo);
+                for (int c = 0; c < 16; ++c) {
+                    const int kap = 2 * (c0 + c), t = kap >> 5, p = kap & 31;
+                    const float x0 = rvalid ? src[slot_coord(0, t, p)] : 0.f;
+                    const float x1 = rvalid ? src[slot_coord(0, t, p + 1)] : 0.f;
+                    split_hilo(x0, x1, hi[c], lo[c]);
                 }
+                tc_st16(tl + S::kColA + 128 * hh + c0, hi);
+                tc_st16(tl + S::kColA + 128 * hh + 64 + c0, lo);
             }
             tc_wait_st();
             tc_fence_before();
@@ -211,49 +214,48 @@ __global__ void __launch_bounds__(kThreads, 1) tq_prefill_tc_kernel(const Prefil
         for (int k = 0; k < ntile; ++k) {
             const int x = k & 1;
             const uint32_t tx = tl + S::kColX + 64 * x;
-            // (failures are made warp-uniform: the tensor-memory loads and stores are warp-collective)
-            if (!warp_wait(bar(kBarSFull + x), (uint32_t)((k >> 1) & 1))) { failed = true; break; }
+            // A failed wait does not leave the loop at once: the two warpgroups meet at the
+            // row-maximum exchange below, which also ORs their failures, and leave together.
+            // (Within a warp the waits are uniform: the tensor-memory loads and stores are
+            // warp-collective.)
+            bool ok = !failed && warp_wait(bar(kBarSFull + x), (uint32_t)((k >> 1) & 1));
             tc_fence_after();
-            uint32_t sv[64];
-            {
-                uint32_t t32[32];
-                tc_ld32(tx, t32);
-#pragma unroll
-                for (int c = 0; c < 32; ++c) sv[c] = t32[c];
-                tc_ld32(tx + 32, t32);
-#pragma unroll
-                for (int c = 0; c < 32; ++c) sv[32 + c] = t32[c];
-            }
+            uint32_t sv[32];
+            tc_ld32(tx + 32 * hh, sv);
             // the tile's norms (written with its B operands)
-            if (!warp_wait(bar(kBarBReady + b3), (uint32_t)ph3)) { failed = true; break; }
-            const float4* sn4 = reinterpret_cast<const float4*>(scal + b3 * 128);
-            const int64_t tok0 = (int64_t)k * kPT;
-            const int vis = lim - tok0 >= kPT ? kPT : (int)(lim > tok0 ? lim - tok0 : 0);
-            float s[64];
+            ok = ok && warp_wait(bar(kBarBReady + b3), (uint32_t)ph3);
+            const float4* sn4 = reinterpret_cast<const float4*>(scal + b3 * 128 + 32 * hh);
+            const int64_t tok0 = (int64_t)k * kPT + 32 * hh;
+            const int vis = lim - tok0 >= 32 ? 32 : (int)(lim > tok0 ? lim - tok0 : 0);
+            float s[32];
 #pragma unroll
-            for (int t4 = 0; t4 < 16; ++t4) {
+            for (int t4 = 0; t4 < 8; ++t4) {
                 const float4 n4 = sn4[t4];
                 s[4 * t4 + 0] = __uint_as_float(sv[4 * t4 + 0]) * n4.x;
                 s[4 * t4 + 1] = __uint_as_float(sv[4 * t4 + 1]) * n4.y;
                 s[4 * t4 + 2] = __uint_as_float(sv[4 * t4 + 2]) * n4.z;
                 s[4 * t4 + 3] = __uint_as_float(sv[4 * t4 + 3]) * n4.w;
             }
-            if (vis < kPT) {
+            if (vis < 32) {
 #pragma unroll
-                for (int t = 0; t < 64; ++t)
+                for (int t = 0; t < 32; ++t)
                     if (t >= vis) s[t] = -INFINITY;
             }
             float mt = -INFINITY;
 #pragma unroll
-            for (int t = 0; t < 64; ++t) mt = fmaxf(mt, s[t]);
-            const float m_new = fmaxf(m_run, mt);
+            for (int t = 0; t < 32; ++t) mt = fmaxf(mt, s[t]);
+            xm[(x * 2 + hh) * 128 + r] = mt;
+            if (bar_or(2, kSoftmaxThreads, !ok)) { failed = true; break; }
+            mt = fmaxf(mt, xm[(x * 2 + (hh ^ 1)) * 128 + r]);
+            const float m_new = fmaxf(m_run, mt);             // the same in both halves of the row
             m_run = m_new;
-            // O += P(k-1) V(k-1) must be done before O is rescaled (and, for the
-            // barrier's phase tracking, every tile waits for it)
-            if (k > 0 && !warp_wait(bar(kBarODone), (uint32_t)((k - 1) & 1))) { failed = true; break; }
+            // O += P(k-1) V(k-1) must be done before O is rescaled (and, for the barrier's
+            // phase tracking, every tile waits for it); a failure here is acted on at the
+            // next exchange
+            if (k > 0 && !warp_wait(bar(kBarODone), (uint32_t)((k - 1) & 1))) failed = true;
             tc_fence_after();
             // Move this row's reference maximum when it grew by more than 2^8; O is rescaled
-            // by the warp as a whole, with factor 1 on the rows that keep theirs.
+            // by each warp as a whole, with factor 1 on the rows that keep theirs.
             float f = 1.f;
             if (m_new != -INFINITY && (m_used == -INFINITY || m_new > m_used + kRescaleLog2)) {
                 if (m_used != -INFINITY) {                    // O and l were built on m_used
@@ -264,21 +266,21 @@ __global__ void __launch_bounds__(kThreads, 1) tq_prefill_tc_kernel(const Prefil
             }
             if (__any_sync(kFull, f != 1.f)) {
 #pragma unroll
-                for (int c0 = 0; c0 < 128; c0 += 32) {
+                for (int c0 = 0; c0 < 64; c0 += 32) {
                     uint32_t ov[32];
-                    tc_ld32(tl + S::kColO + c0, ov);
+                    tc_ld32(tl + S::kColO + 64 * hh + c0, ov);
 #pragma unroll
                     for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * f);
-                    tc_st32(tl + S::kColO + c0, ov);
+                    tc_st32(tl + S::kColO + 64 * hh + c0, ov);
                 }
             }
             // P = 2^(s - m_used) nv 2^-6 over S: hi limbs in columns 0-31, lo limbs in
-            // 32-63 (tokens 2c, 2c + 1).  A row that has seen nothing yet (an absent
-            // row) keeps P = 0.
+            // 32-63 (tokens 2c, 2c + 1; this half: columns 16 h .. 16 h + 15 of each).
+            // A row that has seen nothing yet (an absent row) keeps P = 0.
             const float mu = m_used == -INFINITY ? 0.f : m_used;
-            uint32_t ph[32], plo[32];
+            uint32_t ph[16], plo[16];
 #pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) {
+            for (int c4 = 0; c4 < 8; ++c4) {
                 const float4 v4 = sn4[16 + c4];
                 const float p0 = fast_exp2(s[4 * c4 + 0] - mu), p1 = fast_exp2(s[4 * c4 + 1] - mu);
                 const float p2 = fast_exp2(s[4 * c4 + 2] - mu), p3 = fast_exp2(s[4 * c4 + 3] - mu);
@@ -286,8 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1) tq_prefill_tc_kernel(const Prefil
                 split_hilo(p0 * v4.x, p1 * v4.y, ph[2 * c4], plo[2 * c4]);
                 split_hilo(p2 * v4.z, p3 * v4.w, ph[2 * c4 + 1], plo[2 * c4 + 1]);
             }
-            tc_st32(tx, ph);
-            tc_st32(tx + 32, plo);
+            tc_st16(tx + 16 * hh, ph);
+            tc_st16(tx + 32 + 16 * hh, plo);
             tc_wait_st();
             tc_fence_before();
             mbar_arrive(bar(kBarPReady + x));
@@ -297,32 +299,36 @@ __global__ void __launch_bounds__(kThreads, 1) tq_prefill_tc_kernel(const Prefil
         if (!failed && !warp_wait(bar(kBarODone), (uint32_t)((ntile - 1) & 1))) failed = true;
         tc_fence_after();
         pdl_trigger();
+        xl[hh * 128 + r] = l;
+        // (every softmax thread gets here; a failure seen by any of them zeroes the CTA's rows)
+        if (bar_or(2, kSoftmaxThreads, failed)) failed = true;
         if (failed) atomicExch(a.err, 1);
-        // (the loads are warp-collective: every lane loads, valid rows store)
+        // (the loads are warp-collective: every lane loads, valid rows store).  O's column
+        // 32 t + p is coordinate slot_coord(0, t, p); positions 2i, 2i + 1 are adjacent
+        // coordinates.
         float* acc = a.part_acc + qrow * kPD;
 #pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) {
+        for (int c0 = 0; c0 < 64; c0 += 32) {
             uint32_t ov[32];
-            tc_ld32(tl + S::kColO + c0, ov);
+            tc_ld32(tl + S::kColO + 64 * hh + c0, ov);
+            const int t = 2 * hh + (c0 >> 5);
             if (rvalid) {
 #pragma unroll
-                for (int c = 0; c < 32; c += 4)
-                    *reinterpret_cast<float4*>(acc + c0 + c) =
-                        failed ? make_float4(0.f, 0.f, 0.f, 0.f)
-                               : make_float4(__uint_as_float(ov[c]) * (1.f / kPScale),
-                                             __uint_as_float(ov[c + 1]) * (1.f / kPScale),
-                                             __uint_as_float(ov[c + 2]) * (1.f / kPScale),
-                                             __uint_as_float(ov[c + 3]) * (1.f / kPScale));
+                for (int p = 0; p < 32; p += 2)
+                    *reinterpret_cast<float2*>(acc + slot_coord(0, t, p)) =
+                        failed ? make_float2(0.f, 0.f)
+                               : make_float2(__uint_as_float(ov[p]) * (1.f / kPScale),
+                                             __uint_as_float(ov[p + 1]) * (1.f / kPScale));
             }
         }
-        if (rvalid) {
+        if (rvalid && hh == 0) {
             a.part_ml[2 * qrow] = failed ? -INFINITY : m_used;
-            a.part_ml[2 * qrow + 1] = failed ? 0.f : l;
+            a.part_ml[2 * qrow + 1] = failed ? 0.f : xl[r] + xl[128 + r];
         }
-    } else if (warp < 8) {
-        // ======================================== producer warps: thread pt of 128
+    } else if (warp < 11) {
+        // ======================================== producer warps: thread pt of 96; item
+        // (token tau, slot group t) of the tile's 256
         const int pt = tid - kSoftmaxThreads;
-        const int tau = pt >> 1, hf = pt & 1;                   // token of the tile, half of its slots
         const uint32_t lut[4] = {a.cb.lut_lo[0], a.cb.lut_lo[1], a.cb.lut_hi[0], a.cb.lut_hi[1]};
         const uint32_t* pw = a.cb.pow2;
         int n_ring = ntile < kPRing ? ntile : kPRing;
@@ -340,11 +346,10 @@ __global__ void __launch_bounds__(kThreads, 1) tq_prefill_tc_kernel(const Prefil
                 uint8_t* Vt = sm + b3 * S::kBuf + S::kOffV;
                 const uint8_t* kb = st;
                 const uint8_t* vb = st + S::kKB;
-                const uint32_t gam = *reinterpret_cast<const uint16_t*>(kb + 64 * 64 + 128 + 2 * tau);
-                const uint32_t g2 = gam | (gam << 16);
-#pragma unroll
-                for (int tt = 0; tt < 2; ++tt) {
-                    const int t = 2 * hf + tt;
+                for (int it = pt; it < 4 * kPT; it += kProducerThreads) {
+                    const int tau = it >> 2, t = it & 3;
+                    const uint32_t gam = *reinterpret_cast<const uint16_t*>(kb + 64 * 64 + 128 + 2 * tau);
+                    const uint32_t g2 = gam | (gam << 16);
                     uint32_t sel[4], vsel[4];
                     code_selectors(kb + tau * 48 + 12 * t, pw, sel);
                     code_selectors(vb + tau * 48 + 12 * t, pw, vsel);
@@ -371,24 +376,21 @@ __global__ void __launch_bounds__(kThreads, 1) tq_prefill_tc_kernel(const Prefil
                         *reinterpret_cast<uint4*>(Sg + sw128_byte(tau, 2 * (32 * t + 8 * c), kPT)) =
                             make_uint4(xs[0], xs[1], xs[2], xs[3]);
                     }
-                    // values: row = coordinate, K position = token tau
+                    // values: row = token tau, positions 32 t .. 32 t + 31 (slot order, as the keys)
 #pragma unroll
-                    for (int kc = 0; kc < 8; ++kc) {
-                        uint32_t x0, x1;
-                        dequant4(sel_for(vsel, pw, kc), lut, x0, x1);
-                        const int p = 4 * kc;
-                        const uint32_t v4[4] = {x0 & 0xFFFFu, x0 >> 16, x1 & 0xFFFFu, x1 >> 16};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            *reinterpret_cast<uint16_t*>(Vt + sw128_byte(slot_coord(0, t, p + e), 2 * tau, kPD)) =
-                                (uint16_t)v4[e];
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t xv[4];
+                        dequant4(sel_for(vsel, pw, 2 * c), lut, xv[0], xv[1]);
+                        dequant4(sel_for(vsel, pw, 2 * c + 1), lut, xv[2], xv[3]);
+                        *reinterpret_cast<uint4*>(Vt + sw128_byte(tau, 2 * (32 * t + 8 * c), kPT)) =
+                            make_uint4(xv[0], xv[1], xv[2], xv[3]);
                     }
-                }
-                if (hf == 0) {             // the tile's per-token factors for the softmax
-                    scal[b3 * 128 + tau] =
-                        __half2float(*reinterpret_cast<const __half*>(kb + 64 * 64 + 2 * tau)) * a.scale_log2;
-                    scal[b3 * 128 + 64 + tau] =
-                        __half2float(*reinterpret_cast<const __half*>(vb + 64 * 48 + 2 * tau)) * kPScale;
+                    if (t == 0) {          // the tile's per-token factors for the softmax
+                        scal[b3 * 128 + tau] =
+                            __half2float(*reinterpret_cast<const __half*>(kb + 64 * 64 + 2 * tau)) * a.scale_log2;
+                        scal[b3 * 128 + 64 + tau] =
+                            __half2float(*reinterpret_cast<const __half*>(vb + 64 * 48 + 2 * tau)) * kPScale;
+                    }
                 }
                 fence_proxy_async();       // B operands written by threads, read by the tensor core
                 mbar_arrive(bar(kBarBReady + b3));
@@ -411,13 +413,16 @@ __global__ void __launch_bounds__(kThreads, 1) tq_prefill_tc_kernel(const Prefil
         }
     } else if ((tid & 31) == 0) {
         // ======================================== the mma thread
-        constexpr uint32_t kIdS = idesc_f16(128, kPT), kIdO = idesc_f16(128, kPD);
+        constexpr uint32_t kIdS = idesc_f16(128, kPT), kIdO = idesc_f16_bmn(128, kPD);
         auto mma_o = [&](int k) {          // O += P(k) V(k)
             const uint32_t vd = sbase + (uint32_t)((k % kPBuf) * S::kBuf + S::kOffV);
             const uint32_t pa_t = tmem + S::kColX + 64 * (k & 1);
+            // K step s: tokens 16 (s % 4) .. + 15 (two 8-token atoms); the coordinates
+            // 0-63 and 64-127 are the two halves of each token row, kPT * 128 bytes apart
 #pragma unroll
             for (int s = 0; s < 8; ++s)
-                tc_mma_f16_ts(tmem + S::kColO, pa_t + 8 * s, sw128_desc(vd + 32 * (s & 3)), kIdO,
+                tc_mma_f16_ts(tmem + S::kColO, pa_t + 8 * s,
+                              sw128_desc_mn(vd + 2048 * (s & 3), (uint32_t)(kPT * 128), 1024u), kIdO,
                               (k > 0 || s > 0) ? 1u : 0u);
             tc_commit(bar(kBarODone));
             tc_commit(bar(kBarBFree + k % kPBuf));

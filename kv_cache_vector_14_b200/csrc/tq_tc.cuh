@@ -51,21 +51,53 @@ __device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, 
         : "memory");
 }
 
-// Instruction descriptors (dense, both operands K-major): D format at bits
-// 4-5 (1 f32, 2 s32), A and B formats at bits 7-9 and 10-12 (f16 0; s8 1),
-// N / 8 at bits 17-22, M / 16 at bits 24-28.
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (fp16 or bf16 operands, as the instruction descriptor says)
+__device__ __forceinline__ void tc_mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 2-D tiled TMA load (no multicast) of box {c0.., c1..} into shared memory, completing on an mbarrier
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int c0, int c1, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+
+// Instruction descriptors (dense): D format at bits 4-5 (1 f32, 2 s32), A
+// and B formats at bits 7-9 and 10-12 (f16 0; s8 1), A and B major-ness at
+// bits 15 and 16 (0 K-major, 1 MN-major), N / 8 at bits 17-22, M / 16 at bits
+// 24-28.
 __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
     return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
     return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// f32 accumulate, A and B bf16 (format 1), both K-major
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) { return idesc_f16(M, N) | (1u << 7) | (1u << 10); }
+// the same with B MN-major (bit 16)
+__host__ __device__ constexpr uint32_t idesc_f16_bmn(int M, int N) { return idesc_f16(M, N) | (1u << 16); }
 
 // shared-memory operand descriptor: 128-byte swizzle, K-major, 8-row groups
 // 1024 bytes apart (leading offset unused for this layout), descriptor version 1
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// MN-major operand, 128-byte swizzle: a 1024-byte atom holds 8 consecutive K
+// indices, each a 128-byte row of 64 consecutive MN elements (16-bit); atoms
+// of the next 8 K indices are sbo bytes apart, the next 64 MN elements lbo
+// bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 // Byte offset of byte kb (0 .. 255) of row `row` in a K-major operand of
 // nrows rows held as 128-byte swizzled atoms: bytes 0..127 of every row in

@@ -172,6 +172,57 @@ def test_encode_zero_and_special_vectors(handles, prms):
     print(check_encode(prms[d], _x64(x), gk, gv))
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("paged", [False, True])
+def test_encode_tensor_core_rotation_path(handles, prms, dtype, paged):
+    """Bulk encodes of contiguous bf16 / fp16 input of at least 16384 vectors
+    (the rotation on the tensor cores, one vector per thread): 18000 vectors
+    (a ragged last tile), a token offset that straddles cache blocks, special
+    vectors (zero, one-hot, tiny, large, half-constant), contiguous and paged
+    caches; every vector against the oracle's encode, and tokens outside the
+    written range stay untouched."""
+    d, B, Hkv, T, t0 = 128, 1, 3, 6000, 37
+    Tcap, NB = 6080, 95
+    x = synthetic.gaussian((B, Hkv, T, d), seed=770 + len(dtype))
+    x[..., 5] *= 20.0
+    x[0, 0, 0] = 0.0
+    x[0, 0, 1] = 0.0
+    x[0, 0, 1, 7] = 3.0
+    x[0, 1, 2] = 1e-3
+    x[0, 1, 3] *= 1000.0
+    x[0, 2, 4] = 0.0
+    x[0, 2, 4, :64] = -2.0
+    x = synthetic.bf16_round(x) if dtype == "bf16" else x.astype(np.float16).astype(np.float32)
+    xt = torch_input(x, dtype)
+    assert xt.is_contiguous() and B * Hkv * T >= 16384
+    if paged:
+        pool = 2 * B * Hkv * NB + 3
+        perm = np.random.default_rng(11).permutation(pool).astype(np.int32)
+        kt = torch.from_numpy(perm[:B * Hkv * NB].reshape(B * Hkv, NB).copy()).cuda()
+        vt = torch.from_numpy(perm[B * Hkv * NB:2 * B * Hkv * NB].reshape(B * Hkv, NB).copy()).cuda()
+        kc = tq.Cache(d, True, B, Hkv, Tcap, block_table=kt, pool_blocks=pool)
+        vc = tq.Cache(d, False, B, Hkv, Tcap, block_table=vt, pool_blocks=pool)
+    else:
+        kc, vc = tq.Cache(d, True, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
+    tq.tq_encode_k(handles[d], xt, kc, t0)
+    tq.tq_encode_v(handles[d], xt, vc, t0)
+    torch.cuda.synchronize()
+    assert tq.tq_device_status(handles[d]) == tq.TQ_OK
+    if paged:                      # logical order, as a contiguous cache would hold it
+        kl, vl = tq.Cache(d, True, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
+        kl.buf.copy_(_gather_blocks(kc, kt))
+        vl.buf.copy_(_gather_blocks(vc, vt))
+        kc, vc = kl, vl
+    gk, gv = _flat(unpack_cache(kc, t0, T)), _flat(unpack_cache(vc, t0, T))
+    assert np.all(gk["idx"][0] == 4) and np.all(gk["sig"][0] == 1)
+    assert gk["nh"][0] == 0 and gk["gh"][0] == 0 and gv["nh"][0] == 0
+    print(check_encode(prms[d], _x64(x), gk, gv))
+    for c in (kc, vc):
+        u = unpack_cache(c, 0, Tcap)
+        for k, v in u.items():
+            assert not np.any(v[:, :t0]) and not np.any(v[:, t0 + T:]), k
+
+
 @pytest.mark.parametrize("d", [64, 128, 256])
 def test_append_one_token_at_a_time_equals_bulk(handles, d):
     """Bulk encodes (over 4 vectors per SM: the tiled kernel) and one-token
