@@ -66,7 +66,8 @@ def bf16_peak_tflops() -> float:
         return 1590.0
 
 
-DECODE_SOURCES = ("kv_cache_vector_14_b200/csrc/tq_decode_mma.cu", "kv_cache_vector_14_b200/csrc/tq_frag.cuh")
+DECODE_SOURCES = ("kv_cache_vector_14_b200/csrc/tq_decode_mma.cu", "kv_cache_vector_14_b200/csrc/tq_frag.cuh",
+                  "kv_cache_vector_14_b200/csrc/tq_internal.h")
 
 
 def source_sha(rels) -> str:

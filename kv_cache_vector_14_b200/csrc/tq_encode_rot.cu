@@ -13,8 +13,8 @@
 //     Y = X (H D)^T          (8 tcgen05.mma, M = N = 128, K = 16)
 // into tensor memory: H D has entries +-1, exact in bf16 and fp16, so every
 // product is exact and only the fp32 accumulation rounds (as the butterflies
-// of the per-lane path do).  Then each of 128 threads owns one vector (its
-// tensor-memory lane): ||Y||^2 = 128 ||x||^2 gives the norm, y = Y / ||Y|| the
+// of the per-lane path do).  Then each vector is quantised from its tensor-
+// memory lane: ||Y||^2 = 128 ||x||^2 gives the norm, y = Y / ||Y|| the
 // unit-sphere coordinates, the cell search and the centroid run on the FMA
 // pipe (saturated fused multiply-adds against the boundaries), and the codes
 // are packed into the token record.  For K, the residual r = y - c[idx] goes
@@ -22,10 +22,13 @@
 // (each 32-column chunk is overwritten only after it has been read), and the
 // tensor core computes the QJL projection from there:
 //     Z = R_hi S_hi^T + R_hi S_lo^T + R_lo S_hi^T   (24 tcgen05.mma, A in tensor memory)
-// whose sign bits are read out one tile later.  Warp 4 issues the TMA loads
-// (three tile buffers) and the mma (one thread); Y/R and Z are double-
-// buffered in tensor memory, so the rotation of the next tile and the
-// projection of this one overlap the quantisation.  Every wait is bounded.
+// whose sign bits are read out one tile later.  Two threads share a vector
+// (warps w and w + 4 reach the same tensor-memory lanes), each taking 64
+// coordinates; they add their halves of ||Y||^2 and gamma^2 and merge the
+// code words through shared memory.  Warp 8 issues the TMA loads (three tile
+// buffers) and the mma (one thread); Y/R and Z are double-buffered in tensor
+// memory, so the rotation of the next tile and the projection of this one
+// overlap the quantisation.  Every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -39,7 +42,7 @@ namespace {
 
 constexpr int kRD = 128;                  // head_dim
 constexpr int kRRows = 128;               // vectors per tile (tensor-memory lanes)
-constexpr int kRQuant = 128;              // quantiser threads, one vector each
+constexpr int kRQuant = 256;              // quantiser threads: two per vector (64 coordinates each)
 constexpr int kRThreads = kRQuant + 32;   // + the copy / mma warp
 constexpr int kRXBuf = 3;                 // input tile buffers
 constexpr int kRTile = kRRows * kRD * 2;  // one 16-bit 128 x 128 operand (32 KB)
@@ -52,7 +55,8 @@ struct RotShape {
     static constexpr int kOffS = kRTile;                         // K: JL operand, hi then lo limb
     static constexpr int kOffX = IS_K ? 3 * kRTile : kRTile;     // input tiles
     static constexpr int kOffBar = kOffX + kRXBuf * kRTile;
-    static constexpr int kOffMisc = kOffBar + 16 * 8;
+    static constexpr int kOffXchg = kOffBar + 16 * 8;            // per tile parity: ||Y||^2 halves, words, gamma^2
+    static constexpr int kOffMisc = kOffXchg + 2 * (2 * 128 + 12 * 128 + 128) * 4;
     static constexpr int kSmem = kOffMisc + 16 + 1024;           // + slack to align the base
     static constexpr int kCols = IS_K ? 512 : 256;               // Y/R x 2 (+ Z x 2)
 };
@@ -64,13 +68,29 @@ enum : int {
     kRBarXFull = 1,   // [3] input tile landed (TMA bytes)
     kRBarXFree = 4,   // [3] input tile read by its rotation (commit)
     kRBarYFull = 7,   // [2] Y computed (commit)
-    kRBarRFull = 9,   // [2] Y read and, for K, R written (128 quantiser arrivals)
+    kRBarRFull = 9,   // [2] Y read and, for K, R written (256 quantiser arrivals)
     kRBarZFull = 11,  // [2] Z computed (commit)
     kRBarDrain = 13,  // every mma of the mma thread done (commit, at exit)
 };
 
 __device__ __forceinline__ bool warp_wait_r(uint32_t bar, uint32_t parity) {
     return __all_sync(kFull, mbar_wait_bounded(bar, parity));
+}
+__device__ __forceinline__ void named_bar_r(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// barrier id over n threads that also ORs v across them (every thread gets the result)
+__device__ __forceinline__ bool bar_or_r(int id, int n, bool v) {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(res)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return res != 0;
 }
 
 template <int DT, bool IS_K>
@@ -114,7 +134,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
     // Rotation operand, row j (output coordinate), K index i (input coordinate):
     // (-1)^popcount(i & j) d_i, the Walsh-Hadamard matrix in natural order times
     // the random signs, as bf16 / fp16 +-1.
-    if (tid < kRQuant) {
+    if (tid < kRRows) {
         const int j = tid;
         const uint32_t one = DT == TQ_BF16 ? 0x3F80u : 0x3C00u;
 #pragma unroll 1
@@ -225,9 +245,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
             mbar_wait_bounded(bar(kRBarXFull + j % kRXBuf), (uint32_t)((j / kRXBuf) & 1));
         if (!ok) atomicExch(a.err, 1);
     } else if (tid < kRQuant) {
-        // ======================================== quantisers: thread r = vector r of the tile
-        const int r = tid;
-        const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+        // ======================================== quantisers: threads r and r + 128 share vector r
+        // of the tile (tensor-memory lane r); half h = tid / 128 takes coordinates 64 h .. 64 h + 63
+        const int hh = tid >> 7;
+        const int r = tid & 127;
+        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        float* xss = reinterpret_cast<float*>(sm + S::kOffXchg);            // [2][2][128]
+        uint32_t* xw = reinterpret_cast<uint32_t*>(xss + 2 * 2 * 128);       // [2][12][128]
+        float* xg = reinterpret_cast<float*>(xw + 2 * 12 * 128);             // [2][128]
         const Codebook& cb = a.cb;
         // Bucket index and centroid on the FMA pipe.  The codebook is antisymmetric
         // (b3 = 0, b[6-k] = -b[k], c[7-k] = -c[k]), so with a = |y| and
@@ -239,15 +264,15 @@ __global__ void __launch_bounds__(kRThreads, 1)
         constexpr float kBig = 1152921504606846976.f;        // 2^60
         const float bb4 = cb.b[4] * kBig, bb5 = cb.b[5] * kBig, bb6 = cb.b[6] * kBig;
         [[maybe_unused]] const float d3 = cb.c[7] - cb.c[6], d2 = cb.c[6] - cb.c[5], d1 = cb.c[5] - cb.c[4];
-        bool ok = true;
-        // sign words of tile jj (K): bit b of word w is z[32 w + b] >= 0
+        bool failed = false;
+        // sign words 2h, 2h + 1 of tile jj (K): bit b of word w is z[32 w + b] >= 0
         auto signs = [&](int jj) -> bool {
             if (!warp_wait_r(bar(kRBarZFull + (jj & 1)), (uint32_t)((jj >> 1) & 1))) return false;
             tc_fence_after();
-            const uint32_t zb = tl + 256u + (uint32_t)(128 * (jj & 1));
-            uint32_t sw0 = 0, sw1 = 0, sw2 = 0, sw3 = 0;
+            const uint32_t zb = tl + 256u + (uint32_t)(128 * (jj & 1) + 64 * hh);
+            uint32_t sw0 = 0, sw1 = 0;
 #pragma unroll 1
-            for (int w = 0; w < 4; ++w) {
+            for (int w = 0; w < 2; ++w) {
                 uint32_t z[32];
                 tc_ld32(zb + (uint32_t)(32 * w), z);
                 uint32_t word = 0;
@@ -255,8 +280,6 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 for (int bt = 0; bt < 32; ++bt) word |= (__uint_as_float(z[bt]) >= 0.f ? 1u : 0u) << bt;
                 sw0 = w == 0 ? word : sw0;
                 sw1 = w == 1 ? word : sw1;
-                sw2 = w == 2 ? word : sw2;
-                sw3 = w == 3 ? word : sw3;
             }
             const int64_t gv = row0_of(jj) + r;
             if (gv < N) {
@@ -265,45 +288,52 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 int tau;
                 encode_locate(a, (uint32_t)gv, bb, xoff, blk, tau);
                 if (blk)
-                    *reinterpret_cast<uint4*>(blk + kBlockT * code_bytes(kRD) + tau * sign_bytes(kRD)) =
-                        make_uint4(sw0, sw1, sw2, sw3);
+                    *reinterpret_cast<uint2*>(blk + kBlockT * code_bytes(kRD) + tau * sign_bytes(kRD) + 8 * hh) =
+                        make_uint2(sw0, sw1);
             }
             return true;
         };
         for (int j = 0; j < n; ++j) {
             const int64_t gv = row0_of(j) + r;
-            if (!(ok = warp_wait_r(bar(kRBarYFull + (j & 1)), (uint32_t)((j >> 1) & 1)))) break;
+            const int x = j & 1;
+            // A failed wait does not leave the loop at once: both halves of every vector meet
+            // at the exchange below, which also ORs their failures, and leave together.
+            // (Within a warp the waits are uniform: tensor-memory loads are warp-collective.)
+            const bool ok = !failed && warp_wait_r(bar(kRBarYFull + x), (uint32_t)((j >> 1) & 1));
             tc_fence_after();
-            const uint32_t yb = tl + (uint32_t)(128 * (j & 1));
-            // ||Y||^2 = 128 ||x||^2
+            const uint32_t yb = tl + (uint32_t)(128 * x + 64 * hh);
+            // ||Y||^2 = 128 ||x||^2, this half's 64 coordinates
             float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int cc = 0; cc < 2; ++cc) {
                 uint32_t v[32];
-                tc_ld32(yb + (uint32_t)(32 * c), v);
+                tc_ld32(yb + (uint32_t)(32 * cc), v);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) s4[e & 3] = fmaf(__uint_as_float(v[e]), __uint_as_float(v[e]), s4[e & 3]);
             }
-            const float ss = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+            xss[(x * 2 + hh) * 128 + r] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+            if (bar_or_r(1, kRQuant, !ok)) { failed = true; break; }
+            const float ss = xss[(x * 2) * 128 + r] + xss[(x * 2 + 1) * 128 + r];
             const float nrm = sqrtf(ss * (1.f / 128.f));
             const bool nz = ss > 0.f;
             const float rcp = nz ? __frcp_rn(sqrtf(ss)) : 0.f;   // y = Y / ||Y||
             // Codes in the token record: word 3 t + g holds, in nibble i, the code of slot
             // position 8 g + i (bits 0-2) and bit g of the code of position 24 + i (bit 3).
             // Position p of slot t is coordinate slot_coord(0, t, p), so chunk c (coordinates
-            // 32 c .. 32 c + 31) fills words 3 t + c for c < 3 and the bit-3 planes for c = 3;
+            // 32 c .. 32 c + 31) gives words 3 t + c for c < 3 and the bit-3 planes for c = 3;
             // nibble i of slot t is the chunk's coordinate o(t, i) = 16 (i / 4) + 2 t + (i % 2)
-            // + 8 ((i / 2) % 2).
-            uint32_t wd[12];
+            // + 8 ((i / 2) % 2).  ag[t] collects this half's part of word 3 t + g.
+            uint32_t a0[4], a1[4], a2[4];
 #pragma unroll
-            for (int i = 0; i < 12; ++i) wd[i] = 0u;
+            for (int t = 0; t < 4; ++t) a0[t] = a1[t] = a2[t] = 0u;
             float g2 = 0.f;
             // (K: the chunk loop stays rolled; unrolled, the code with the residual outgrows
             // the instruction cache)
-#pragma unroll(IS_K ? 1 : 4)
-            for (int c = 0; c < 4; ++c) {
+#pragma unroll(IS_K ? 1 : 2)
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * hh + cc;
                 uint32_t v[32];
-                tc_ld32(yb + (uint32_t)(32 * c), v);
+                tc_ld32(yb + (uint32_t)(32 * cc), v);
                 float cf[32];
                 [[maybe_unused]] uint32_t rh[16], rl[16];
 #pragma unroll
@@ -331,8 +361,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     if constexpr (IS_K) split_hilo(rr[0], rr[1], rh[e >> 1], rl[e >> 1]);
                 }
                 if constexpr (IS_K) {      // R over the chunk just read
-                    tc_st16(yb + (uint32_t)(32 * c), rh);
-                    tc_st16(yb + (uint32_t)(32 * c + 16), rl);
+                    tc_st16(yb + (uint32_t)(32 * cc), rh);
+                    tc_st16(yb + (uint32_t)(32 * cc + 16), rl);
                 }
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
@@ -342,37 +372,54 @@ __global__ void __launch_bounds__(kRThreads, 1)
                         fmaf(cf[2 * t + 25], 4096.f, fmaf(cf[2 * t + 24], 256.f, fmaf(cf[2 * t + 17], 16.f, cf[2 * t + 16])));
                     const uint32_t W = __byte_perm(__float_as_uint(lo + 8388608.f), __float_as_uint(hi + 8388608.f), 0x5410);
                     // (register indices fixed at compile time, selected by the chunk)
-                    wd[3 * t + 0] = c == 0 ? W : c == 3 ? wd[3 * t + 0] | ((W & 0x11111111u) << 3) : wd[3 * t + 0];
-                    wd[3 * t + 1] = c == 1 ? W : c == 3 ? wd[3 * t + 1] | (((W >> 1) & 0x11111111u) << 3) : wd[3 * t + 1];
-                    wd[3 * t + 2] = c == 2 ? W : c == 3 ? wd[3 * t + 2] | (((W >> 2) & 0x11111111u) << 3) : wd[3 * t + 2];
+                    a0[t] = c == 0 ? W : c == 3 ? (W & 0x11111111u) << 3 : a0[t];
+                    a1[t] = c == 1 ? W : c == 3 ? ((W >> 1) & 0x11111111u) << 3 : a1[t];
+                    a2[t] = c == 2 ? W : c == 3 ? a2[t] | (((W >> 2) & 0x11111111u) << 3) : a2[t];
                 }
             }
             if constexpr (IS_K) tc_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(kRBarRFull + (j & 1)));
-            if (gv < N) {
+            mbar_arrive(bar(kRBarRFull + x));
+            if (hh == 1) {
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    xw[(x * 12 + 3 * t + 0) * 128 + r] = a0[t];
+                    xw[(x * 12 + 3 * t + 1) * 128 + r] = a1[t];
+                    xw[(x * 12 + 3 * t + 2) * 128 + r] = a2[t];
+                }
+                xg[x * 128 + r] = g2;
+            }
+            named_bar_r(1, kRQuant);
+            if (hh == 0 && gv < N) {
                 int64_t xoff;
                 uint8_t* blk;
                 int tau;
                 encode_locate(a, (uint32_t)gv, bb, xoff, blk, tau);
                 if (blk) {
+                    uint32_t wd[12];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        wd[3 * t + 0] = a0[t] | xw[(x * 12 + 3 * t + 0) * 128 + r];
+                        wd[3 * t + 1] = a1[t] | xw[(x * 12 + 3 * t + 1) * 128 + r];
+                        wd[3 * t + 2] = a2[t] | xw[(x * 12 + 3 * t + 2) * 128 + r];
+                    }
                     uint4* rec = reinterpret_cast<uint4*>(blk + tau * code_bytes(kRD));
                     rec[0] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
                     rec[1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
                     rec[2] = make_uint4(wd[8], wd[9], wd[10], wd[11]);
                     __half* nf = reinterpret_cast<__half*>(blk + kBlockT * (code_bytes(kRD) + (IS_K ? sign_bytes(kRD) : 0)));
                     nf[tau] = __float2half_rn(nrm);
-                    if constexpr (IS_K) nf[kBlockT + tau] = __float2half_rn(sqrtf(g2));
+                    if constexpr (IS_K) nf[kBlockT + tau] = __float2half_rn(sqrtf(g2 + xg[x * 128 + r]));
                 }
             }
             if constexpr (IS_K) {          // the previous tile's projection ran meanwhile
-                if (j >= 1 && !(ok = signs(j - 1))) break;
+                if (j >= 1 && !signs(j - 1)) failed = true;      // acted on at the next exchange
             }
         }
         if constexpr (IS_K) {
-            if (ok && n > 0) ok = signs(n - 1);
+            if (!failed && n > 0 && !signs(n - 1)) failed = true;
         }
-        if (!ok && (tid & 31) == 0) atomicExch(a.err, 1);
+        if (failed && (tid & 31) == 0) atomicExch(a.err, 1);
     }
     tc_fence_before();
     __syncthreads();
