@@ -206,8 +206,10 @@ TQ_API tq_status tq_attend_decode_polar(const tq_handle* h, const void* q, tq_dt
 
 /* ---- chunked prefill ------------------------------------------------------ */
 
-/* Workspace bytes tq_attend_prefill needs (rotated queries and the per-row
- * softmax partials of B * Lq * Hq query rows).  0 on bad arguments. */
+/* Workspace bytes tq_attend_prefill needs (rotated queries and the softmax
+ * partials of B * Lq * Hq query rows; at head_dim 128 a row tile's tokens may
+ * be spread over several CTAs, each writing one partial, up to a bound that
+ * depends on the row count and the device's SM count).  0 on bad arguments. */
 TQ_API size_t tq_prefill_workspace_bytes(const tq_handle* h, int64_t B, int64_t Lq, int64_t Hq);
 
 /* Attention for a chunk of Lq new queries per sequence (q [B][Lq][Hq][d]
@@ -215,14 +217,17 @@ TQ_API size_t tq_prefill_workspace_bytes(const tq_handle* h, int64_t B, int64_t 
  * chunk attends over tokens [0, T0 + i] of its sequence, so the chunk's own K
  * and V must already be encoded at positions T0 .. T0 + Lq - 1.  Scores and
  * output as tq_attend_decode (the same estimator, in the page's K section and
- * hybrid V2+V3 section, with the QJL term evaluated on 16-bit fixed-point u');
- * out is fp32 [B][Lq][Hq][d].  With many queries per kv head the score and
- * value contractions are dense and run on tensor cores with the keys
- * dequantised once per 16 query rows (at d = 256 two CTAs share each 64 query
- * rows, each accumulating half of the value coordinates).  Supported: d in
- * {64, 128, 256}, any Hq/Hkv, B <= 65535, T0 + Lq <= Tcap; contiguous or
- * paged caches.  Errors: INVALID_ARG, UNSUPPORTED (grid limits), WORKSPACE,
- * CUDA. */
+ * hybrid V2+V3 section); out is fp32 [B][Lq][Hq][d].  With many queries per
+ * kv head the score and value contractions are dense and run on tensor cores:
+ * at d = 128 on tcgen05 with each 64-token block dequantised once per 128
+ * query rows (q' and u' as fp16 hi and lo limbs), the row tiles' token ranges
+ * spread evenly over one CTA per SM; at d = 64 and 256 on mma.sync tiles with
+ * the keys dequantised once per 16 query rows and the QJL term on 16-bit
+ * fixed-point u' (at d = 256 two CTAs share each 64 query rows, each
+ * accumulating half of the value coordinates).  Supported: d in {64, 128,
+ * 256}, any Hq/Hkv, B <= 65535, Lq Hq / Hkv <= 2^27, T0 + Lq <= Tcap;
+ * contiguous or paged caches.  Errors: INVALID_ARG, UNSUPPORTED (grid or size
+ * limits), WORKSPACE, CUDA. */
 TQ_API tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype qdtype, int64_t B, int64_t Lq,
                                    int64_t Hq, const tq_cache* kc, const tq_cache* vc, int64_t T0, float scale,
                                    float* out, void* ws, size_t ws_bytes, void* stream);

@@ -331,10 +331,17 @@ size_t tq_attend_workspace_bytes(const tq_handle* h, int64_t B, int64_t Hq, int6
     return p.bytes;
 }
 
+// Partials per row of a prefill call: the d = 128 kernel spreads row tiles over the SMs
+// and merges up to prefill_tc_split_cap partials per row; the others write one.
+static int prefill_splits(const tq_handle* h, int64_t rows) {
+    return h->d == 128 ? prefill_tc_split_cap(h->num_sms, rows) : 1;
+}
+
 size_t tq_prefill_workspace_bytes(const tq_handle* h, int64_t B, int64_t Lq, int64_t Hq) {
     if (!h || B < 0 || Lq < 0 || Hq <= 0) return 0;
     DecodePlan p;
-    layout_ws(h->d, (size_t)(B * Lq * Hq), 1, &p);
+    const int64_t rows = B * Lq * Hq;
+    layout_ws(h->d, (size_t)rows, prefill_splits(h, rows), &p);
     return p.bytes;
 }
 
@@ -350,6 +357,7 @@ tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype qdt, int
     const int G = (int)(Hq / Hkv);
     if (B > 65535 || Hkv > 65535) return TQ_ERR_UNSUPPORTED;          // grid limits
     if ((Lq * G + 63) / 64 * 2 >= ((int64_t)1 << 31)) return TQ_ERR_UNSUPPORTED;
+    if (Lq * G > ((int64_t)1 << 27)) return TQ_ERR_UNSUPPORTED;        // row tiles per sequence (host plan)
     if (B == 0 || Lq == 0) return TQ_OK;
     if (!q || !out || !ws || !aligned(q, dtype_size(qdt)) || !aligned(out, 16) || !aligned(ws, 256))
         return TQ_ERR_INVALID_ARG;
@@ -358,8 +366,9 @@ tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype qdt, int
     if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
     if (dev != h->device) return TQ_ERR_INVALID_ARG;
     const int64_t rows = B * Lq * Hq;
+    const int cap = prefill_splits(h, rows);
     DecodePlan p;
-    layout_ws(h->d, (size_t)rows, 1, &p);
+    layout_ws(h->d, (size_t)rows, cap, &p);
     if (ws_bytes < p.bytes) return TQ_ERR_WORKSPACE;
     uint8_t* w = static_cast<uint8_t*>(ws);
     DecArgs a{};
@@ -384,8 +393,11 @@ tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype qdt, int
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_prologue(h->d, q, qdt, rows, h->dsign, h->dST, const_cast<float*>(a.qp),
                                     const_cast<float*>(a.up), false, s);
-    if (e == cudaSuccess) e = launch_prefill(h->d, G, a, Lq, T0, s);
-    if (e == cudaSuccess) e = launch_combine(h->d, rows, 1, a.part_ml, a.part_acc, h->dsign, out, s);
+    int nsplit = 1;
+    if (e == cudaSuccess)
+        e = h->d == 128 ? launch_prefill_tc(G, a, Lq, T0, h->num_sms, cap, &nsplit, s)
+                        : launch_prefill(h->d, G, a, Lq, T0, s);
+    if (e == cudaSuccess) e = launch_combine(h->d, rows, nsplit, a.part_ml, a.part_acc, h->dsign, out, s);
     return cuda_status(e);
 }
 

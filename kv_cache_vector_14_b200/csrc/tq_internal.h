@@ -229,7 +229,11 @@ cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, cons
 // query i over tokens [0, T0 + i]; partials as one split of a.part_ml/part_acc.
 cudaError_t launch_prefill(int d, int G, const DecArgs& a, int64_t Lq, int64_t T0, cudaStream_t s);
 // head_dim 128: the tcgen05 form (tq_prefill_tc.cu)
-cudaError_t launch_prefill_tc(int G, const DecArgs& a, int64_t Lq, int64_t T0, cudaStream_t s);
+// d = 128 chunked prefill on tcgen05, one CTA per SM over the flattened tiles; the
+// partials go to nsplit slots per row (*nsplit_out, at most split_cap).
+int prefill_tc_split_cap(int num_sms, int64_t rows);
+cudaError_t launch_prefill_tc(int G, const DecArgs& a, int64_t Lq, int64_t T0, int num_sms, int split_cap,
+                              int* nsplit_out, cudaStream_t s);
 // qjl = false: PolarQuant-only K cache (V layout), scores without the QJL term.
 cudaError_t launch_decode(int d, int G, bool use_mma, bool qjl, const DecArgs& a, cudaStream_t s);
 cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml,

@@ -371,7 +371,7 @@ cudaError_t launch_prefill(int d, int G, const DecArgs& a, int64_t Lq, int64_t T
     if (!head_dim_ok(d) || G < 1) return cudaErrorInvalidValue;
     if (a.B * a.Hkv == 0 || Lq == 0) return cudaSuccess;
     if (d == 64) return launch_prefill_d<64>(G, a, Lq, T0, s);
-    return d == 128 ? launch_prefill_tc(G, a, Lq, T0, s) : launch_prefill_d<256>(G, a, Lq, T0, s);
+    return d == 256 ? launch_prefill_d<256>(G, a, Lq, T0, s) : cudaErrorInvalidValue;
 }
 
 }  // namespace tqi
