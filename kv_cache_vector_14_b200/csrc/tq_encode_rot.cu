@@ -22,13 +22,13 @@
 // (each 32-column chunk is overwritten only after it has been read), and the
 // tensor core computes the QJL projection from there:
 //     Z = R_hi S_hi^T + R_hi S_lo^T + R_lo S_hi^T   (24 tcgen05.mma, A in tensor memory)
-// whose sign bits are read out one tile later.  Two threads share a vector
-// (warps w and w + 4 reach the same tensor-memory lanes), each taking 64
-// coordinates; they add their halves of ||Y||^2 and gamma^2 and merge the
-// code words through shared memory.  Warp 8 issues the TMA loads (three tile
-// buffers) and the mma (one thread); Y/R and Z are double-buffered in tensor
-// memory, so the rotation of the next tile and the projection of this one
-// overlap the quantisation.  Every wait is bounded.
+// whose sign bits are read out one tile later.  Four threads share a vector
+// (warps w, w + 4, w + 8, w + 12 reach the same tensor-memory lanes), each
+// taking a 32-coordinate chunk; they add their parts of ||Y||^2 and gamma^2
+// and merge the code words through shared memory.  Warp 16 issues the TMA
+// loads (three tile buffers) and the mma (one thread); Y/R and Z are double-
+// buffered in tensor memory, so the rotation of the next tile and the
+// projection of this one overlap the quantisation.  Every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -42,7 +42,7 @@ namespace {
 
 constexpr int kRD = 128;                  // head_dim
 constexpr int kRRows = 128;               // vectors per tile (tensor-memory lanes)
-constexpr int kRQuant = 256;              // quantiser threads: two per vector (64 coordinates each)
+constexpr int kRQuant = 512;              // quantiser threads: four per vector (32 coordinates each)
 constexpr int kRThreads = kRQuant + 32;   // + the copy / mma warp
 constexpr int kRXBuf = 3;                 // input tile buffers
 constexpr int kRTile = kRRows * kRD * 2;  // one 16-bit 128 x 128 operand (32 KB)
@@ -55,8 +55,10 @@ struct RotShape {
     static constexpr int kOffS = kRTile;                         // K: JL operand, hi then lo limb
     static constexpr int kOffX = IS_K ? 3 * kRTile : kRTile;     // input tiles
     static constexpr int kOffBar = kOffX + kRXBuf * kRTile;
-    static constexpr int kOffXchg = kOffBar + 16 * 8;            // per tile parity: ||Y||^2 halves, words, gamma^2
-    static constexpr int kOffMisc = kOffXchg + 2 * (2 * 128 + 12 * 128 + 128) * 4;
+    // exchange between the four threads of a vector: ||Y||^2 and gamma^2 parts [4][128],
+    // code words of chunks 0-2 and bit-3 planes of chunk 3 [12][128] each
+    static constexpr int kOffXchg = kOffBar + 16 * 8;
+    static constexpr int kOffMisc = kOffXchg + (4 * 128 + 4 * 128 + 12 * 128 + 12 * 128) * 4;
     static constexpr int kSmem = kOffMisc + 16 + 1024;           // + slack to align the base
     static constexpr int kCols = IS_K ? 512 : 256;               // Y/R x 2 (+ Z x 2)
 };
@@ -68,7 +70,7 @@ enum : int {
     kRBarXFull = 1,   // [3] input tile landed (TMA bytes)
     kRBarXFree = 4,   // [3] input tile read by its rotation (commit)
     kRBarYFull = 7,   // [2] Y computed (commit)
-    kRBarRFull = 9,   // [2] Y read and, for K, R written (256 quantiser arrivals)
+    kRBarRFull = 9,   // [2] Y read and, for K, R written (512 quantiser arrivals)
     kRBarZFull = 11,  // [2] Z computed (commit)
     kRBarDrain = 13,  // every mma of the mma thread done (commit, at exit)
 };
@@ -181,13 +183,13 @@ __global__ void __launch_bounds__(kRThreads, 1)
             ok = mbar_wait_bounded(bar(kRBarB), 0u);
         }
         // Z(j) = R_hi S_hi^T + R_hi S_lo^T + R_lo S_hi^T.  R(j) lies in Y(j)'s columns:
-        // coordinates 32 c + 2 m, + 1 in column 32 c + m (hi) and 32 c + 16 + m (lo).
+        // coordinates 16 s + 2 m, + 1 in column 16 s + m (hi) and 16 s + 8 + m (lo).
         auto qjl = [&](int j) {
             const uint32_t rb = tmem + (uint32_t)(128 * (j & 1)), zd = tmem + 256u + (uint32_t)(128 * (j & 1));
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t koff = (uint32_t)((ks >> 2) * (kRRows * 128) + (ks & 3) * 32);
-                const uint32_t ahi = rb + (uint32_t)(32 * (ks >> 1) + 8 * (ks & 1)), alo = ahi + 16u;
+                const uint32_t ahi = rb + (uint32_t)(16 * ks), alo = ahi + 8u;
                 const uint64_t bhi = sw128_desc(sbase + (uint32_t)S::kOffS + koff);
                 const uint64_t blo = sw128_desc(sbase + (uint32_t)(S::kOffS + kRTile) + koff);
                 tc_mma_f16_ts(zd, ahi, bhi, kIdZ, ks > 0 ? 1u : 0u);
@@ -245,14 +247,15 @@ __global__ void __launch_bounds__(kRThreads, 1)
             mbar_wait_bounded(bar(kRBarXFull + j % kRXBuf), (uint32_t)((j / kRXBuf) & 1));
         if (!ok) atomicExch(a.err, 1);
     } else if (tid < kRQuant) {
-        // ======================================== quantisers: threads r and r + 128 share vector r
-        // of the tile (tensor-memory lane r); half h = tid / 128 takes coordinates 64 h .. 64 h + 63
-        const int hh = tid >> 7;
+        // ======================================== quantisers: threads r + 128 c (c = 0..3) share
+        // vector r of the tile (tensor-memory lane r); thread c takes coordinates 32 c .. 32 c + 31
+        const int cq = tid >> 7;
         const int r = tid & 127;
         const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-        float* xss = reinterpret_cast<float*>(sm + S::kOffXchg);            // [2][2][128]
-        uint32_t* xw = reinterpret_cast<uint32_t*>(xss + 2 * 2 * 128);       // [2][12][128]
-        float* xg = reinterpret_cast<float*>(xw + 2 * 12 * 128);             // [2][128]
+        float* xss = reinterpret_cast<float*>(sm + S::kOffXchg);            // [4][128]
+        float* xg = xss + 4 * 128;                                           // [4][128]
+        uint32_t* xw = reinterpret_cast<uint32_t*>(xg + 4 * 128);            // [12][128]
+        uint32_t* xp = xw + 12 * 128;                                        // [12][128]
         const Codebook& cb = a.cb;
         // Bucket index and centroid on the FMA pipe.  The codebook is antisymmetric
         // (b3 = 0, b[6-k] = -b[k], c[7-k] = -c[k]), so with a = |y| and
@@ -260,27 +263,27 @@ __global__ void __launch_bounds__(kRThreads, 1)
         // its sign decides, and any nonzero difference of two such floats saturates),
         // T = t4 + t5 + t6 boundaries lie above a: the code is 7 - T for y >= 0 and T
         // below, and |c| = c7 - t6 (c7 - c6) - t5 (c6 - c5) - t4 (c5 - c4), every partial
-        // sum an exact centroid.
+        // sum an exact centroid.  (Here the comparisons run on |Y| directly:
+        // t_k = sat(fma(|Y|, -2^60 / ||Y||, b_k 2^60)), one rounding, so the sign of
+        // b_k 2^60 - |Y| 2^60 / ||Y|| decides exactly; only the rounding of the per-vector
+        // factor differs from forming y first.  The residual is kept in units of 2^-12, with
+        // every constant scaled by a power of two.)
         constexpr float kBig = 1152921504606846976.f;        // 2^60
         const float bb4 = cb.b[4] * kBig, bb5 = cb.b[5] * kBig, bb6 = cb.b[6] * kBig;
-        [[maybe_unused]] const float d3 = cb.c[7] - cb.c[6], d2 = cb.c[6] - cb.c[5], d1 = cb.c[5] - cb.c[4];
+        [[maybe_unused]] const float d3 = (cb.c[7] - cb.c[6]) * kRScale, d2 = (cb.c[6] - cb.c[5]) * kRScale,
+                                     d1 = (cb.c[5] - cb.c[4]) * kRScale, c7 = cb.c[7] * kRScale;
         bool failed = false;
-        // sign words 2h, 2h + 1 of tile jj (K): bit b of word w is z[32 w + b] >= 0
+        [[maybe_unused]] bool nz_prev = true;                // the previous tile's vector is nonzero
+        // sign word cq of tile jj (K): bit b is z[32 cq + b] >= 0
         auto signs = [&](int jj) -> bool {
             if (!warp_wait_r(bar(kRBarZFull + (jj & 1)), (uint32_t)((jj >> 1) & 1))) return false;
             tc_fence_after();
-            const uint32_t zb = tl + 256u + (uint32_t)(128 * (jj & 1) + 64 * hh);
-            uint32_t sw0 = 0, sw1 = 0;
-#pragma unroll 1
-            for (int w = 0; w < 2; ++w) {
-                uint32_t z[32];
-                tc_ld32(zb + (uint32_t)(32 * w), z);
-                uint32_t word = 0;
+            uint32_t z[32];
+            tc_ld32(tl + 256u + (uint32_t)(128 * (jj & 1) + 32 * cq), z);
+            uint32_t word = 0;
 #pragma unroll
-                for (int bt = 0; bt < 32; ++bt) word |= (__uint_as_float(z[bt]) >= 0.f ? 1u : 0u) << bt;
-                sw0 = w == 0 ? word : sw0;
-                sw1 = w == 1 ? word : sw1;
-            }
+            for (int bt = 0; bt < 32; ++bt) word |= (__uint_as_float(z[bt]) >= 0.f ? 1u : 0u) << bt;
+            if (!nz_prev) word = 0xFFFFFFFFu;                // zero vector: z = 0, every sign bit 1
             const int64_t gv = row0_of(jj) + r;
             if (gv < N) {
                 int64_t xoff;
@@ -288,109 +291,100 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 int tau;
                 encode_locate(a, (uint32_t)gv, bb, xoff, blk, tau);
                 if (blk)
-                    *reinterpret_cast<uint2*>(blk + kBlockT * code_bytes(kRD) + tau * sign_bytes(kRD) + 8 * hh) =
-                        make_uint2(sw0, sw1);
+                    *reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(kRD) + tau * sign_bytes(kRD) + 4 * cq) = word;
             }
             return true;
         };
         for (int j = 0; j < n; ++j) {
             const int64_t gv = row0_of(j) + r;
-            const int x = j & 1;
-            // A failed wait does not leave the loop at once: both halves of every vector meet
-            // at the exchange below, which also ORs their failures, and leave together.
+            // A failed wait does not leave the loop at once: the four threads of every vector
+            // meet at the exchange below, which also ORs their failures, and leave together.
             // (Within a warp the waits are uniform: tensor-memory loads are warp-collective.)
-            const bool ok = !failed && warp_wait_r(bar(kRBarYFull + x), (uint32_t)((j >> 1) & 1));
+            const bool ok = !failed && warp_wait_r(bar(kRBarYFull + (j & 1)), (uint32_t)((j >> 1) & 1));
             tc_fence_after();
-            const uint32_t yb = tl + (uint32_t)(128 * x + 64 * hh);
-            // ||Y||^2 = 128 ||x||^2, this half's 64 coordinates
-            float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-            for (int cc = 0; cc < 2; ++cc) {
+            const uint32_t yb = tl + (uint32_t)(128 * (j & 1) + 32 * cq);
+            {                              // ||Y||^2 = 128 ||x||^2, this chunk's part
                 uint32_t v[32];
-                tc_ld32(yb + (uint32_t)(32 * cc), v);
+                tc_ld32(yb, v);
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int e = 0; e < 32; ++e) s4[e & 3] = fmaf(__uint_as_float(v[e]), __uint_as_float(v[e]), s4[e & 3]);
+                xss[cq * 128 + r] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
             }
-            xss[(x * 2 + hh) * 128 + r] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
             if (bar_or_r(1, kRQuant, !ok)) { failed = true; break; }
-            const float ss = xss[(x * 2) * 128 + r] + xss[(x * 2 + 1) * 128 + r];
+            const float ss = (xss[r] + xss[128 + r]) + (xss[256 + r] + xss[384 + r]);
             const float nrm = sqrtf(ss * (1.f / 128.f));
             const bool nz = ss > 0.f;
             const float rcp = nz ? __frcp_rn(sqrtf(ss)) : 0.f;   // y = Y / ||Y||
+            const float kneg = -kBig * rcp;
+            [[maybe_unused]] const float rcpS = rcp * kRScale;
             // Codes in the token record: word 3 t + g holds, in nibble i, the code of slot
             // position 8 g + i (bits 0-2) and bit g of the code of position 24 + i (bit 3).
-            // Position p of slot t is coordinate slot_coord(0, t, p), so chunk c (coordinates
-            // 32 c .. 32 c + 31) gives words 3 t + c for c < 3 and the bit-3 planes for c = 3;
-            // nibble i of slot t is the chunk's coordinate o(t, i) = 16 (i / 4) + 2 t + (i % 2)
-            // + 8 ((i / 2) % 2).  ag[t] collects this half's part of word 3 t + g.
-            uint32_t a0[4], a1[4], a2[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) a0[t] = a1[t] = a2[t] = 0u;
+            // Position p of slot t is coordinate slot_coord(0, t, p), so chunk c gives words
+            // 3 t + c for c < 3 and the bit-3 planes for c = 3; nibble i of slot t is the
+            // chunk's coordinate o(t, i) = 16 (i / 4) + 2 t + (i % 2) + 8 ((i / 2) % 2): half
+            // h of the chunk gives nibbles 4 h .. 4 h + 3.  W[t] collects the chunk's word of slot t.
+            uint32_t W[4] = {0u, 0u, 0u, 0u};
             float g2 = 0.f;
-            // (K: the chunk loop stays rolled; unrolled, the code with the residual outgrows
-            // the instruction cache)
 #pragma unroll(IS_K ? 1 : 2)
-            for (int cc = 0; cc < 2; ++cc) {
-                const int c = 2 * hh + cc;
-                uint32_t v[32];
-                tc_ld32(yb + (uint32_t)(32 * cc), v);
-                float cf[32];
-                [[maybe_unused]] uint32_t rh[16], rl[16];
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t v[16];
+                tc_ld16(yb + (uint32_t)(16 * h2), v);
+                float cf[16];
+                [[maybe_unused]] uint32_t rh[8], rl[8];
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
+                for (int e = 0; e < 16; e += 2) {
                     [[maybe_unused]] float rr[2];
 #pragma unroll
                     for (int f = 0; f < 2; ++f) {
-                        const float y = __uint_as_float(v[e + f]) * rcp;
-                        const float av = fabsf(y);
-                        const float t4 = __saturatef(fmaf(av, -kBig, bb4));
-                        const float t5 = __saturatef(fmaf(av, -kBig, bb5));
-                        const float t6 = __saturatef(fmaf(av, -kBig, bb6));
+                        // the sign of Y decides the side of the code and of the residual (Y = -0,
+                        // y = 0 on the boundary b3 = 0, counts as negative for both)
+                        const uint32_t ybits = v[e + f], sgn = ybits & 0x80000000u;
+                        const float av = __uint_as_float(ybits & 0x7FFFFFFFu);
+                        const float t4 = __saturatef(fmaf(av, kneg, bb4));
+                        const float t5 = __saturatef(fmaf(av, kneg, bb5));
+                        const float t6 = __saturatef(fmaf(av, kneg, bb6));
                         const float T = (t4 + t5) + t6;
-                        const float pos = (y >= 0.f) ? 1.f : 0.f;
-                        cf[e + f] = fmaf(pos, fmaf(T, -2.f, 7.f), T);
+                        // 7 - T above zero, T below: 3.5 +- (3.5 - T)
+                        cf[e + f] = 3.5f + __uint_as_float(__float_as_uint(3.5f - T) ^ sgn);
                         if constexpr (IS_K) {
-                            float m = fmaf(-t6, d3, cb.c[7]);
+                            float m = fmaf(-t6, d3, c7);                // |c| 2^12
                             m = fmaf(-t5, d2, m);
                             m = fmaf(-t4, d1, m);
-                            const float rv = nz ? y - m * fmaf(pos, 2.f, -1.f) : 0.f;
+                            const float rv = __uint_as_float(__float_as_uint(fmaf(av, rcpS, -m)) ^ sgn);   // r 2^12
                             g2 = fmaf(rv, rv, g2);
-                            rr[f] = rv * kRScale;
+                            rr[f] = rv;
                         }
                     }
                     if constexpr (IS_K) split_hilo(rr[0], rr[1], rh[e >> 1], rl[e >> 1]);
                 }
-                if constexpr (IS_K) {      // R over the chunk just read
-                    tc_st16(yb + (uint32_t)(32 * cc), rh);
-                    tc_st16(yb + (uint32_t)(32 * cc + 16), rl);
+                if constexpr (IS_K) {      // R over the columns just read: hi limbs, then lo
+                    tc_st8(yb + (uint32_t)(16 * h2), rh);
+                    tc_st8(yb + (uint32_t)(16 * h2 + 8), rl);
                 }
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
-                    // nibbles 0-3 and 4-7 as exact float sums, read out of the mantissa (x + 2^23)
-                    const float lo = fmaf(cf[2 * t + 9], 4096.f, fmaf(cf[2 * t + 8], 256.f, fmaf(cf[2 * t + 1], 16.f, cf[2 * t])));
-                    const float hi =
-                        fmaf(cf[2 * t + 25], 4096.f, fmaf(cf[2 * t + 24], 256.f, fmaf(cf[2 * t + 17], 16.f, cf[2 * t + 16])));
-                    const uint32_t W = __byte_perm(__float_as_uint(lo + 8388608.f), __float_as_uint(hi + 8388608.f), 0x5410);
-                    // (register indices fixed at compile time, selected by the chunk)
-                    a0[t] = c == 0 ? W : c == 3 ? (W & 0x11111111u) << 3 : a0[t];
-                    a1[t] = c == 1 ? W : c == 3 ? ((W >> 1) & 0x11111111u) << 3 : a1[t];
-                    a2[t] = c == 2 ? W : c == 3 ? a2[t] | (((W >> 2) & 0x11111111u) << 3) : a2[t];
+                    // four nibbles as an exact float sum, read out of the mantissa (x + 2^23)
+                    const float part = fmaf(cf[2 * t + 9], 4096.f, fmaf(cf[2 * t + 8], 256.f, fmaf(cf[2 * t + 1], 16.f, cf[2 * t])));
+                    const uint32_t bits = __float_as_uint(part + 8388608.f);
+                    W[t] = h2 == 0 ? bits : __byte_perm(W[t], bits, 0x5410);
                 }
             }
             if constexpr (IS_K) tc_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(kRBarRFull + x));
-            if (hh == 1) {
+            mbar_arrive(bar(kRBarRFull + (j & 1)));
+            if (cq < 3) {
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    xw[(x * 12 + 3 * t + 0) * 128 + r] = a0[t];
-                    xw[(x * 12 + 3 * t + 1) * 128 + r] = a1[t];
-                    xw[(x * 12 + 3 * t + 2) * 128 + r] = a2[t];
-                }
-                xg[x * 128 + r] = g2;
+                for (int t = 0; t < 4; ++t) xw[(3 * t + cq) * 128 + r] = W[t];
+            } else {
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+#pragma unroll
+                    for (int g = 0; g < 3; ++g) xp[(3 * t + g) * 128 + r] = ((W[t] >> g) & 0x11111111u) << 3;
             }
+            xg[cq * 128 + r] = g2;
             named_bar_r(1, kRQuant);
-            if (hh == 0 && gv < N) {
+            if (cq == 0 && gv < N) {
                 int64_t xoff;
                 uint8_t* blk;
                 int tau;
@@ -398,22 +392,22 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 if (blk) {
                     uint32_t wd[12];
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        wd[3 * t + 0] = a0[t] | xw[(x * 12 + 3 * t + 0) * 128 + r];
-                        wd[3 * t + 1] = a1[t] | xw[(x * 12 + 3 * t + 1) * 128 + r];
-                        wd[3 * t + 2] = a2[t] | xw[(x * 12 + 3 * t + 2) * 128 + r];
-                    }
+                    for (int k = 0; k < 12; ++k) wd[k] = xw[k * 128 + r] | xp[k * 128 + r];
                     uint4* rec = reinterpret_cast<uint4*>(blk + tau * code_bytes(kRD));
                     rec[0] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
                     rec[1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
                     rec[2] = make_uint4(wd[8], wd[9], wd[10], wd[11]);
                     __half* nf = reinterpret_cast<__half*>(blk + kBlockT * (code_bytes(kRD) + (IS_K ? sign_bytes(kRD) : 0)));
                     nf[tau] = __float2half_rn(nrm);
-                    if constexpr (IS_K) nf[kBlockT + tau] = __float2half_rn(sqrtf(g2 + xg[x * 128 + r]));
+                    if constexpr (IS_K) {        // gamma = ||r||; a zero vector has none
+                        const float gs = (xg[r] + xg[128 + r]) + (xg[256 + r] + xg[384 + r]);
+                        nf[kBlockT + tau] = __float2half_rn(nz ? sqrtf(gs) * (1.f / kRScale) : 0.f);
+                    }
                 }
             }
             if constexpr (IS_K) {          // the previous tile's projection ran meanwhile
                 if (j >= 1 && !signs(j - 1)) failed = true;      // acted on at the next exchange
+                nz_prev = nz;
             }
         }
         if constexpr (IS_K) {
