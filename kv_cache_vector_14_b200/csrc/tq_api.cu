@@ -257,6 +257,22 @@ tq_status tq_init(int head_dim, uint64_t seed, tq_handle** out) {
     // d = 128: the JL matrix as the B operand of the tensor-core encode, rows
     // permuted into sign-word order, fp16 hi and lo limbs of each fp32 entry
     std::vector<uint16_t> simg;
+    if (d == 64) {
+        // d = 64: rows in sign-word order (word r, bit l), the K index in the slot order of
+        // the bulk encode's rotated tile (16 t + p is coordinate slot_coord(0, t, p))
+        simg.assign((size_t)2 * 64 * d, 0);
+        for (int nr = 0; nr < d; ++nr) {
+            const int row = sign_row(d, nr >> 5, nr & 31);
+            for (int k = 0; k < d; ++k) {
+                const double sv = (double)h->hS[(size_t)row * d + slot_coord(0, k >> 4, k & 15)];
+                const uint16_t hi = double_to_half_bits(sv);
+                const uint16_t lo = double_to_half_bits(sv - half_bits_to_double(hi));
+                const size_t at = sw128_k_offset(nr, k) / 2;
+                simg[at] = hi;
+                simg[(size_t)64 * d + at] = lo;
+            }
+        }
+    }
     if (d == 128) {
         simg.assign((size_t)2 * kTcRows * d, 0);
         for (int n = 0; n < d; ++n) {

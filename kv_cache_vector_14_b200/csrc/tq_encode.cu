@@ -464,8 +464,11 @@ cudaError_t launch_encode(int d, bool is_k, tq_dtype dt, const EncArgs& a, int n
         const cudaError_t e = launch_encode128_rot(is_k, dt, a, num_sms, pdl, s);
         return e == cudaErrorNotSupported ? launch_encode128(is_k, dt, a, num_sms, pdl, s) : e;
     }
-    if (d == 64)
+    if (d == 64) {
+        const cudaError_t e = launch_encode64_rot(is_k, dt, a, num_sms, pdl, s);
+        if (e != cudaErrorNotSupported) return e;
         return is_k ? launch_enc_dt<64, true>(dt, a, num_sms, pdl, s) : launch_enc_dt<64, false>(dt, a, num_sms, pdl, s);
+    }
     if (d == 256)
         return is_k ? launch_enc_dt<256, true>(dt, a, num_sms, pdl, s) : launch_enc_dt<256, false>(dt, a, num_sms, pdl, s);
     return cudaErrorInvalidValue;

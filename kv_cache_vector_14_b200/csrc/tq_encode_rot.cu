@@ -1,5 +1,5 @@
-// TurboQuant K/V encode for head_dim 128 with the random rotation on the
-// 5th-generation tensor cores, for bulk encodes of contiguous bf16 / fp16
+// TurboQuant K/V encode for head_dim 128 and 64 with the random rotation on
+// the 5th-generation tensor cores, for bulk encodes of contiguous bf16 / fp16
 // input on sm_100a.
 //
 // Page "Apple Silicon向けSwiftLM、TurboQuant KVキャッシュ圧縮とSSD Expert
@@ -424,6 +424,330 @@ __global__ void __launch_bounds__(kRThreads, 1)
     pdl_wait();                    // when chained: complete only after the previous kernel
 }
 
+// ---------------------------------------------------------------- head_dim 64
+// The same scheme at d = 64: 128-vector tiles of 128-byte rows (one TMA box),
+// Y = X (H D)^T with 4 tcgen05.mma (N = 64), the rotation's rows in slot order
+// (Y's column 16 t + p is coordinate slot_coord(0, t, p), position p of slot t
+// of the d = 64 record; the JL operand's K index follows), and two threads per
+// vector (warps w and w + 4), each owning two 16-position slots: a thread
+// writes its slots' code words and halfwords and its sign word itself, and
+// only ||Y||^2 and gamma^2 are added across the two.  Two CTAs fit an SM
+// (256 tensor-memory columns each).
+constexpr int k6D = 64;
+constexpr int k6Quant = 256;                 // two threads per vector
+constexpr int k6Threads = k6Quant + 32;
+constexpr int k6Tile = kRRows * k6D * 2;     // 16 KB
+constexpr int k6Op = 64 * k6D * 2;           // a 64 x 64 16-bit operand (8 KB)
+
+template <bool IS_K>
+struct Rot64Shape {
+    static constexpr int kOffM = 0;                              // rotation operand H D (rows in slot order)
+    static constexpr int kOffS = k6Op;                           // K: JL operand, hi then lo limb
+    static constexpr int kOffX = IS_K ? 3 * k6Op : k6Op;         // input tiles
+    static constexpr int kOffBar = kOffX + kRXBuf * k6Tile;
+    static constexpr int kOffXchg = kOffBar + 16 * 8;            // ||Y||^2 and gamma^2 parts [2 tiles][2][128] each
+    static constexpr int kOffMisc = kOffXchg + 2 * (2 * 2 * 128) * 4;
+    static constexpr int kSmem = kOffMisc + 16 + 1024;
+    static constexpr int kCols = 256;                            // Y/R x 2 at 0, 64; Z x 2 at 128, 192
+};
+
+template <int DT, bool IS_K>
+__global__ void __launch_bounds__(k6Threads, 2)
+    tq_encode_rot64_kernel(const __grid_constant__ CUtensorMap tmap, const EncArgs a) {
+    using S = Rot64Shape<IS_K>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + S::kOffBar);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + S::kOffMisc);
+    pdl_trigger();                 // a chained kernel may start (it waits for this one's writes)
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int64_t N = a.B * a.Hkv * a.Tnew;
+    const int64_t ntiles = (N + kRRows - 1) / kRRows;
+    const int n = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);   // this CTA's tiles
+    auto row0_of = [&](int j) { return ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kRRows; };
+    const int64_t bb = block_bytes(k6D, IS_K);
+
+    if (tid == 0) {
+        mbar_init(bar(kRBarB), 1);
+        for (int i = 0; i < kRXBuf; ++i) {
+            mbar_init(bar(kRBarXFull + i), 1);
+            mbar_init(bar(kRBarXFree + i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(kRBarYFull + i), 1);
+            mbar_init(bar(kRBarRFull + i), k6Quant);
+            mbar_init(bar(kRBarZFull + i), 1);
+        }
+        mbar_init(bar(kRBarDrain), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc_alloc(smem_u32(tmem_slot), S::kCols);
+        tc_relinquish();
+    }
+    // Rotation operand row nr (Y's column nr), K index i: (-1)^popcount(i & j) d_i with
+    // j = slot_coord(0, nr / 16, nr % 16), as bf16 / fp16 +-1.
+    if (tid < 64) {
+        const int j = slot_coord(0, tid >> 4, tid & 15);
+        const uint32_t one = DT == TQ_BF16 ? 0x3F80u : 0x3C00u;
+#pragma unroll 1
+        for (int i0 = 0; i0 < k6D; i0 += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                uint32_t h2[2];
+#pragma unroll
+                for (int f = 0; f < 2; ++f) {
+                    const int i = i0 + 2 * e + f;
+                    const uint32_t neg = ((uint32_t)__popc(i & j) & 1u) ^ (__ldg(a.dsign + i) < 0.f ? 1u : 0u);
+                    h2[f] = one | (neg << 15);
+                }
+                w[e] = h2[0] | (h2[1] << 16);
+            }
+            *reinterpret_cast<uint4*>(sm + S::kOffM + sw128_byte(tid, 2 * i0, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async();           // written by threads, read by the tensor core
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (tid == k6Quant) {
+        // ======================================== copy and mma thread
+        constexpr uint32_t kIdY = DT == TQ_BF16 ? idesc_bf16(kRRows, k6D) : idesc_f16(kRRows, k6D);
+        constexpr uint32_t kIdZ = idesc_f16(kRRows, k6D);
+        auto load = [&](int j) {       // input tile j -> buffer j % 3 (one 64-column box)
+            const int bx = j % kRXBuf;
+            const uint32_t dst = sbase + (uint32_t)(S::kOffX + bx * k6Tile), br = bar(kRBarXFull + bx);
+            mbar_expect_tx(br, (uint32_t)k6Tile);
+            tma_load_2d(dst, &tmap, 0, (int)row0_of(j), br);
+        };
+        int n_load = n < kRXBuf ? n : kRXBuf;
+        for (int j = 0; j < n_load; ++j) load(j);
+        bool ok = true;
+        if constexpr (IS_K) {
+            mbar_expect_tx(bar(kRBarB), (uint32_t)(2 * k6Op));
+            bulk_g2s(sbase + (uint32_t)S::kOffS, a.bimg, (uint32_t)(2 * k6Op), bar(kRBarB));
+            ok = mbar_wait_bounded(bar(kRBarB), 0u);
+        }
+        // Z(j) = R_hi S_hi^T + R_hi S_lo^T + R_lo S_hi^T over the coordinates in slot order.
+        // R(j) lies in Y(j)'s columns: K positions 16 s + 2 m, + 1 in column 16 s + m (hi)
+        // and 16 s + 8 + m (lo).
+        auto qjl = [&](int j) {
+            const uint32_t rb = tmem + (uint32_t)(64 * (j & 1)), zd = tmem + 128u + (uint32_t)(64 * (j & 1));
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint32_t ahi = rb + (uint32_t)(16 * ks), alo = ahi + 8u;
+                const uint64_t bhi = sw128_desc(sbase + (uint32_t)S::kOffS + 32u * ks);
+                const uint64_t blo = sw128_desc(sbase + (uint32_t)(S::kOffS + k6Op) + 32u * ks);
+                tc_mma_f16_ts(zd, ahi, bhi, kIdZ, ks > 0 ? 1u : 0u);
+                tc_mma_f16_ts(zd, ahi, blo, kIdZ, 1u);
+                tc_mma_f16_ts(zd, alo, bhi, kIdZ, 1u);
+            }
+            tc_commit(bar(kRBarZFull + (j & 1)));
+        };
+        for (int j = 0; ok && j < n; ++j) {
+            const int bx = j % kRXBuf;
+            if (!(ok = mbar_wait_bounded(bar(kRBarXFull + bx), (uint32_t)((j / kRXBuf) & 1)))) break;
+            if (j >= 2 && !(ok = mbar_wait_bounded(bar(kRBarRFull + (j & 1)), (uint32_t)(((j - 2) >> 1) & 1)))) break;
+            tc_fence_after();
+            const uint32_t xa = sbase + (uint32_t)(S::kOffX + bx * k6Tile);
+            const uint32_t yd = tmem + (uint32_t)(64 * (j & 1));
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                tc_mma_f16_ss(yd, sw128_desc(xa + 32u * ks), sw128_desc(sbase + (uint32_t)S::kOffM + 32u * ks), kIdY,
+                              ks > 0 ? 1u : 0u);
+            tc_commit(bar(kRBarYFull + (j & 1)));
+            tc_commit(bar(kRBarXFree + bx));
+            if constexpr (IS_K) {
+                if (j >= 1) {
+                    if (!(ok = mbar_wait_bounded(bar(kRBarRFull + ((j - 1) & 1)), (uint32_t)(((j - 1) >> 1) & 1))))
+                        break;
+                    tc_fence_after();
+                    qjl(j - 1);
+                }
+            }
+            if (j >= 1 && j + 2 < n) {
+                if (!(ok = mbar_wait_bounded(bar(kRBarXFree + (j - 1) % kRXBuf), (uint32_t)(((j - 1) / kRXBuf) & 1))))
+                    break;
+                load(j + 2);
+                ++n_load;
+            }
+        }
+        if constexpr (IS_K) {
+            if (ok && n > 0) {
+                if ((ok = mbar_wait_bounded(bar(kRBarRFull + ((n - 1) & 1)), (uint32_t)(((n - 1) >> 1) & 1)))) {
+                    tc_fence_after();
+                    qjl(n - 1);
+                }
+            }
+        }
+        tc_commit(bar(kRBarDrain));
+        mbar_wait_bounded(bar(kRBarDrain), 0u);
+        for (int j = n_load > kRXBuf ? n_load - kRXBuf : 0; j < n_load; ++j)
+            mbar_wait_bounded(bar(kRBarXFull + j % kRXBuf), (uint32_t)((j / kRXBuf) & 1));
+        if (!ok) atomicExch(a.err, 1);
+    } else if (tid < k6Quant) {
+        // ======================================== quantisers: threads r and r + 128 share vector r
+        // (tensor-memory lane r); thread h owns slots 2 h, 2 h + 1, Y's columns 32 h .. 32 h + 31
+        const int hv = tid >> 7;
+        const int r = tid & 127;
+        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        float* xss = reinterpret_cast<float*>(sm + S::kOffXchg);            // [2][2][128]
+        [[maybe_unused]] float* xg = xss + 2 * 2 * 128;                      // [2][2][128]
+        const Codebook& cb = a.cb;
+        // the cell search and residual of the d = 128 kernel, with this head_dim's codebook
+        constexpr float kBig = 1152921504606846976.f;        // 2^60
+        const float bb4 = cb.b[4] * kBig, bb5 = cb.b[5] * kBig, bb6 = cb.b[6] * kBig;
+        [[maybe_unused]] const float d3 = (cb.c[7] - cb.c[6]) * kRScale, d2 = (cb.c[6] - cb.c[5]) * kRScale,
+                                     d1 = (cb.c[5] - cb.c[4]) * kRScale, c7 = cb.c[7] * kRScale;
+        bool failed = false;
+        [[maybe_unused]] bool nz_prev = true;                // the previous tile's vector is nonzero
+        // sign word hv of tile jj (K): bit b is z[32 hv + b] >= 0
+        auto signs = [&](int jj) -> bool {
+            if (!warp_wait_r(bar(kRBarZFull + (jj & 1)), (uint32_t)((jj >> 1) & 1))) return false;
+            tc_fence_after();
+            uint32_t z[32];
+            tc_ld32(tl + 128u + (uint32_t)(64 * (jj & 1) + 32 * hv), z);
+            uint32_t word = 0;
+#pragma unroll
+            for (int bt = 0; bt < 32; ++bt) word |= (__uint_as_float(z[bt]) >= 0.f ? 1u : 0u) << bt;
+            if (!nz_prev) word = 0xFFFFFFFFu;                // zero vector: z = 0, every sign bit 1
+            const int64_t gv = row0_of(jj) + r;
+            if (gv < N) {
+                int64_t xoff;
+                uint8_t* blk;
+                int tau;
+                encode_locate(a, (uint32_t)gv, bb, xoff, blk, tau);
+                if (blk)
+                    *reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(k6D) + tau * sign_bytes(k6D) + 4 * hv) = word;
+            }
+            return true;
+        };
+        for (int j = 0; j < n; ++j) {
+            const int64_t gv = row0_of(j) + r;
+            const int x = j & 1;
+            // A failed wait does not leave the loop at once: both threads of every vector meet
+            // at the exchange below, which also ORs their failures, and leave together.
+            const bool ok = !failed && warp_wait_r(bar(kRBarYFull + x), (uint32_t)((j >> 1) & 1));
+            tc_fence_after();
+            const uint32_t yb = tl + (uint32_t)(64 * x + 32 * hv);
+            {                              // ||Y||^2 = 64 ||x||^2, this thread's part
+                uint32_t v[32];
+                tc_ld32(yb, v);
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int e = 0; e < 32; ++e) s4[e & 3] = fmaf(__uint_as_float(v[e]), __uint_as_float(v[e]), s4[e & 3]);
+                xss[(x * 2 + hv) * 128 + r] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+            }
+            if (bar_or_r(1, k6Quant, !ok)) { failed = true; break; }
+            const float ss = xss[(x * 2) * 128 + r] + xss[(x * 2 + 1) * 128 + r];
+            const float nrm = sqrtf(ss * (1.f / 64.f));
+            const bool nz = ss > 0.f;
+            const float rcp = nz ? __frcp_rn(sqrtf(ss)) : 0.f;   // y = Y / ||Y||
+            const float kneg = -kBig * rcp;
+            [[maybe_unused]] const float rcpS = rcp * kRScale;
+            // d = 64 record, slot t: word t holds in nibble i the code of position i (bits 0-2)
+            // and, for i < 4 bit 0, for i >= 4 bit 1 of the code of position 12 + i % 4 (bit 3);
+            // halfword t holds the codes of positions 8..11 and bit 2 of those of 12..15.
+            uint32_t wd0 = 0, wd1 = 0, hw0 = 0, hw1 = 0;
+            float g2 = 0.f;
+#pragma unroll(IS_K ? 1 : 2)
+            for (int h2 = 0; h2 < 2; ++h2) {           // slot 2 hv + h2
+                uint32_t v[16];
+                tc_ld16(yb + (uint32_t)(16 * h2), v);
+                float cf[16];
+                [[maybe_unused]] uint32_t rh[8], rl[8];
+#pragma unroll
+                for (int e = 0; e < 16; e += 2) {
+                    [[maybe_unused]] float rr[2];
+#pragma unroll
+                    for (int f = 0; f < 2; ++f) {
+                        const uint32_t ybits = v[e + f], sgn = ybits & 0x80000000u;
+                        const float av = __uint_as_float(ybits & 0x7FFFFFFFu);
+                        const float t4 = __saturatef(fmaf(av, kneg, bb4));
+                        const float t5 = __saturatef(fmaf(av, kneg, bb5));
+                        const float t6 = __saturatef(fmaf(av, kneg, bb6));
+                        const float T = (t4 + t5) + t6;
+                        cf[e + f] = 3.5f + __uint_as_float(__float_as_uint(3.5f - T) ^ sgn);
+                        if constexpr (IS_K) {
+                            float m = fmaf(-t6, d3, c7);
+                            m = fmaf(-t5, d2, m);
+                            m = fmaf(-t4, d1, m);
+                            const float rv = __uint_as_float(__float_as_uint(fmaf(av, rcpS, -m)) ^ sgn);
+                            g2 = fmaf(rv, rv, g2);
+                            rr[f] = rv;
+                        }
+                    }
+                    if constexpr (IS_K) split_hilo(rr[0], rr[1], rh[e >> 1], rl[e >> 1]);
+                }
+                if constexpr (IS_K) {
+                    tc_st8(yb + (uint32_t)(16 * h2), rh);
+                    tc_st8(yb + (uint32_t)(16 * h2 + 8), rl);
+                }
+                // nibble sums as exact floats, read out of the mantissa (x + 2^23)
+                const float n0 = fmaf(cf[3], 4096.f, fmaf(cf[2], 256.f, fmaf(cf[1], 16.f, cf[0])));
+                const float n1 = fmaf(cf[7], 4096.f, fmaf(cf[6], 256.f, fmaf(cf[5], 16.f, cf[4])));
+                const float n2 = fmaf(cf[11], 4096.f, fmaf(cf[10], 256.f, fmaf(cf[9], 16.f, cf[8])));
+                const float n3 = fmaf(cf[15], 4096.f, fmaf(cf[14], 256.f, fmaf(cf[13], 16.f, cf[12])));
+                const uint32_t na = __byte_perm(__float_as_uint(n0 + 8388608.f), __float_as_uint(n1 + 8388608.f), 0x5410);
+                const uint32_t nb = __float_as_uint(n2 + 8388608.f) & 0xFFFFu;
+                const uint32_t nc = __float_as_uint(n3 + 8388608.f) & 0xFFFFu;
+                const uint32_t w = na | ((nc & 0x1111u) << 3) | (((nc >> 1) & 0x1111u) << 19);
+                const uint32_t hw = nb | (((nc >> 2) & 0x1111u) << 3);
+                wd0 = h2 == 0 ? w : wd0;
+                wd1 = h2 == 1 ? w : wd1;
+                hw0 = h2 == 0 ? hw : hw0;
+                hw1 = h2 == 1 ? hw : hw1;
+            }
+            if constexpr (IS_K) tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(kRBarRFull + x));
+            if constexpr (IS_K) xg[(x * 2 + hv) * 128 + r] = g2;
+            uint8_t* blk = nullptr;
+            int tau = 0;
+            if (gv < N) {
+                int64_t xoff;
+                encode_locate(a, (uint32_t)gv, bb, xoff, blk, tau);
+                if (blk) {
+                    uint8_t* rec = blk + tau * code_bytes(k6D);
+                    *reinterpret_cast<uint2*>(rec + 8 * hv) = make_uint2(wd0, wd1);     // words 2 hv, 2 hv + 1
+                    *reinterpret_cast<uint32_t*>(rec + 16 + 4 * hv) = hw0 | (hw1 << 16);    // their halfwords
+                    if (hv == 0)
+                        reinterpret_cast<__half*>(blk + kBlockT * (code_bytes(k6D) + (IS_K ? sign_bytes(k6D) : 0)))[tau] =
+                            __float2half_rn(nrm);
+                }
+            }
+            if constexpr (IS_K) {
+                named_bar_r(1, k6Quant);   // both gamma^2 parts are written
+                if (hv == 0 && blk) {
+                    const float gs = xg[(x * 2) * 128 + r] + xg[(x * 2 + 1) * 128 + r];
+                    reinterpret_cast<__half*>(blk + kBlockT * (code_bytes(k6D) + sign_bytes(k6D)))[kBlockT + tau] =
+                        __float2half_rn(nz ? sqrtf(gs) * (1.f / kRScale) : 0.f);     // a zero vector has no residual
+                }
+                if (j >= 1 && !signs(j - 1)) failed = true;      // acted on at the next exchange
+                nz_prev = nz;
+            }
+        }
+        if constexpr (IS_K) {
+            if (!failed && n > 0 && !signs(n - 1)) failed = true;
+        }
+        if (failed && (tid & 31) == 0) atomicExch(a.err, 1);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tc_dealloc(tmem, S::kCols);
+    }
+    pdl_wait();                    // when chained: complete only after the previous kernel
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -447,27 +771,52 @@ cudaError_t launch_rot_t(const CUtensorMap& tm, const EncArgs& a, int grid, bool
     return cudaGetLastError();
 }
 
-}  // namespace
+template <int DT, bool IS_K>
+cudaError_t launch_rot64_t(const CUtensorMap& tm, const EncArgs& a, int grid, bool pdl, cudaStream_t s) {
+    constexpr int smem = Rot64Shape<IS_K>::kSmem;
+    cudaError_t e = set_smem_once<tq_encode_rot64_kernel<DT, IS_K>>(smem);
+    if (e != cudaSuccess) return e;
+    if (pdl) return launch_pdl(tq_encode_rot64_kernel<DT, IS_K>, dim3(grid), dim3(k6Threads), smem, s, tm, a);
+    tq_encode_rot64_kernel<DT, IS_K><<<grid, k6Threads, smem, s>>>(tm, a);
+    return cudaGetLastError();
+}
 
-cudaError_t launch_encode128_rot(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
-    if (dt != TQ_BF16 && dt != TQ_F16) return cudaErrorNotSupported;
+// 2-D tensor map over the flattened [N, d] input when its rows are consecutive (16-bit
+// elements, 16-byte aligned); false when the call does not qualify.
+bool rot_tensor_map(int d, tq_dtype dt, const EncArgs& a, CUtensorMap* tm) {
+    if (dt != TQ_BF16 && dt != TQ_F16) return false;
     const int64_t N = a.B * a.Hkv * a.Tnew;
-    if (N < kRotMinVectors || !a.vec16) return cudaErrorNotSupported;
-    // rows of the flattened input must be consecutive 256-byte rows
-    if (a.st != kRD || (a.Hkv > 1 && a.sh != a.Tnew * kRD) || (a.B > 1 && a.sb != a.Hkv * a.Tnew * kRD))
-        return cudaErrorNotSupported;
+    if (N < kRotMinVectors || !a.vec16) return false;
+    if (a.st != d || (a.Hkv > 1 && a.sh != a.Tnew * d) || (a.B > 1 && a.sb != a.Hkv * a.Tnew * d)) return false;
     const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-    if (!enc) return cudaErrorNotSupported;
-    CUtensorMap tm;
-    const cuuint64_t dims[2] = {(cuuint64_t)kRD, (cuuint64_t)N};
-    const cuuint64_t strides[1] = {(cuuint64_t)kRD * 2};
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)N};
+    const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)kRRows};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(&tm, dt == TQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                           const_cast<void*>(a.x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorNotSupported;
+    return enc(tm, dt == TQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+               const_cast<void*>(a.x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_encode64_rot(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
+    CUtensorMap tm;
+    if (!a.bimg || !rot_tensor_map(k6D, dt, a, &tm)) return cudaErrorNotSupported;
+    const int64_t N = a.B * a.Hkv * a.Tnew;
+    const int64_t ntiles = (N + kRRows - 1) / kRRows;
+    const int grid = (int)(ntiles < 2 * (int64_t)num_sms ? ntiles : 2 * (int64_t)num_sms);
+    if (dt == TQ_BF16)
+        return is_k ? launch_rot64_t<TQ_BF16, true>(tm, a, grid, pdl, s) : launch_rot64_t<TQ_BF16, false>(tm, a, grid, pdl, s);
+    return is_k ? launch_rot64_t<TQ_F16, true>(tm, a, grid, pdl, s) : launch_rot64_t<TQ_F16, false>(tm, a, grid, pdl, s);
+}
+
+cudaError_t launch_encode128_rot(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
+    CUtensorMap tm;
+    if (!rot_tensor_map(kRD, dt, a, &tm)) return cudaErrorNotSupported;
+    const int64_t N = a.B * a.Hkv * a.Tnew;
     const int64_t ntiles = (N + kRRows - 1) / kRRows;
     const int grid = (int)(ntiles < num_sms ? ntiles : num_sms);
     if (dt == TQ_BF16)

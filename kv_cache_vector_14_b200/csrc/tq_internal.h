@@ -114,7 +114,8 @@ struct EncArgs {
     int64_t pool;             // pool blocks of a paged cache
     const float* dsign;       // [d] +-1
     const float* sthr;        // [d][d/32][32] JL matrix, encode lane order
-    const uint8_t* bimg;      // d = 128: JL matrix as tensor-core operand (hi, lo fp16 limbs)
+    const uint8_t* bimg;      // JL matrix as tensor-core operand (hi, lo fp16 limbs; d = 128: K index =
+                              // coordinate; d = 64: K index in slot order), rows in sign-word order
     int* err;                 // device check word
     int vec16;                // every input row starts on a 16-byte boundary
     FastDiv fdT, fdH;         // division by Tnew and by Hkv (vector counts below 2^31)
@@ -221,6 +222,7 @@ cudaError_t launch_encode128(bool is_k, tq_dtype dt, const EncArgs& a, int num_s
 // Bulk d = 128 encode of contiguous bf16 / fp16 input with the rotation on the
 // tensor cores; cudaErrorNotSupported when the call does not qualify.
 cudaError_t launch_encode128_rot(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s);
+cudaError_t launch_encode64_rot(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s);
 // pdl: launched as a programmatic dependent of the previous kernel (fused
 // append-and-attend step); the kernels then complete only after it.
 cudaError_t launch_prologue(int d, const void* q, tq_dtype dt, int64_t BHq, const float* dsign,

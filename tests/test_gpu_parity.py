@@ -172,18 +172,19 @@ def test_encode_zero_and_special_vectors(handles, prms):
     print(check_encode(prms[d], _x64(x), gk, gv))
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("paged", [False, True])
-def test_encode_tensor_core_rotation_path(handles, prms, dtype, paged):
+def test_encode_tensor_core_rotation_path(handles, prms, d, dtype, paged):
     """Bulk encodes of contiguous bf16 / fp16 input of at least 16384 vectors
-    (the rotation on the tensor cores, one vector per thread): 18000 vectors
-    (a ragged last tile), a token offset that straddles cache blocks, special
-    vectors (zero, one-hot, tiny, large, half-constant), contiguous and paged
-    caches; every vector against the oracle's encode, and tokens outside the
-    written range stay untouched."""
-    d, B, Hkv, T, t0 = 128, 1, 3, 6000, 37
+    (the rotation on the tensor cores, quantisation from tensor memory) at
+    head_dim 64 and 128: 18000 vectors (a ragged last tile), a token offset that
+    straddles cache blocks, special vectors (zero, one-hot, tiny, large,
+    half-constant), contiguous and paged caches; every vector against the
+    oracle's encode, and tokens outside the written range stay untouched."""
+    B, Hkv, T, t0 = 1, 3, 6000, 37
     Tcap, NB = 6080, 95
-    x = synthetic.gaussian((B, Hkv, T, d), seed=770 + len(dtype))
+    x = synthetic.gaussian((B, Hkv, T, d), seed=770 + len(dtype) + d)
     x[..., 5] *= 20.0
     x[0, 0, 0] = 0.0
     x[0, 0, 1] = 0.0
@@ -191,7 +192,7 @@ def test_encode_tensor_core_rotation_path(handles, prms, dtype, paged):
     x[0, 1, 2] = 1e-3
     x[0, 1, 3] *= 1000.0
     x[0, 2, 4] = 0.0
-    x[0, 2, 4, :64] = -2.0
+    x[0, 2, 4, :d // 2] = -2.0
     x = synthetic.bf16_round(x) if dtype == "bf16" else x.astype(np.float16).astype(np.float32)
     xt = torch_input(x, dtype)
     assert xt.is_contiguous() and B * Hkv * T >= 16384
