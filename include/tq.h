@@ -313,8 +313,15 @@ TQ_API tq_status tq_set_decode_events(tq_handle* h, void* ev_start, void* ev_sto
 TQ_API tq_status tq_set_wait_limit(tq_handle* h, int first_wait);
 
 /* Diagnostics: choose the decode kernel of later tq_attend_decode calls on this
- * handle: 0 = automatic (tensor-core kernel where supported), 1 = the SIMT
- * kernel.  Changes the workspace size tq_attend_workspace_bytes reports. */
+ * handle: 0 = automatic (tensor-core kernel where supported, with the work
+ * partition its cost model prefers), 1 = the SIMT kernel, 2 = the tensor-core
+ * kernel on the uniform split grid only, 3 = the tensor-core kernel on the
+ * stream-K grid wherever that fits (sequences of one length, no more
+ * (batch, kv head, head group) units than CTA slots, partial slots within the
+ * workspace bound).  Paths 0, 2 and 3 give the same outputs up to the fp32
+ * order of the softmax merge.  Changes the workspace size
+ * tq_attend_workspace_bytes reports (path 1).  Errors: INVALID_ARG (NULL h,
+ * path outside 0..3). */
 TQ_API tq_status tq_set_decode_path(tq_handle* h, int path);
 
 /* Name of the kernel path tq_attend_decode uses for these sizes on this handle

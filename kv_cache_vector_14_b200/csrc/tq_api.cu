@@ -26,10 +26,11 @@ int64_t split_loop_bound(int64_t cap, int64_t pairs, int64_t nchunk) {
     return bound < nchunk ? bound : nchunk;
 }
 
-int choose_nsplit(int64_t cap, int warps, int64_t pairs, int64_t nchunk) {
-    // A CTA also pays a fixed cost (constants, barrier set-up, the merge of its
-    // warps, the partial it writes), about kSetup chunk-steps per warp.
-    const double kSetup = 2.0;
+// A CTA also pays a fixed cost (constants, barrier set-up, the merge of its
+// warps, the partial it writes), about kSetup chunk-steps per warp.
+constexpr double kSetup = 2.0;
+
+int choose_nsplit(int64_t cap, int warps, int64_t pairs, int64_t nchunk, double* steps = nullptr) {
     const int64_t hi = split_loop_bound(cap, pairs, nchunk);
     const double ideal = (double)pairs * nchunk / ((double)cap * warps);
     int64_t best = 1;
@@ -41,9 +42,49 @@ int choose_nsplit(int64_t cap, int warps, int64_t pairs, int64_t nchunk) {
         const int64_t waves = (pairs * used + cap - 1) / cap;
         const double t = (double)waves * ((double)((per + warps - 1) / warps) + kSetup);
         const double eff = ideal / t;
-        if (eff > best_eff + 1e-12) { best_eff = eff; best = ns; }
+        if (eff > best_eff + 1e-12) { best_eff = eff; best = ns; if (steps) *steps = t; }
     }
     return (int)best;
+}
+
+// Stream-K plan for sequences of one length: nC CTAs take equal shares of the
+// units' chunks laid end to end (units x nck in all).  With nC >= units a
+// share spans at most two units; the kernel then divides the CTA's warps
+// between them in proportion to their chunks.  Returns the modelled
+// chunk-steps of the slowest CTA (plus the fixed cost) and the partial slots
+// a unit needs (the CTAs that overlap it), or -1 when the shape does not fit.
+double streamk_plan(int64_t cap, int warps, int64_t units, int64_t nck, int64_t* nC_out, int* slots_out) {
+    const int64_t N = units * nck;
+    const int64_t nC = cap < N ? cap : N;
+    if (nC < units || nC <= 0) return -1.0;
+    double worst = 0.0;
+    for (int64_t c = 0; c < nC; ++c) {
+        const int64_t lo = c * N / nC, hi = (c + 1) * N / nC;
+        const int64_t u0 = lo / nck, u1 = (hi - 1) / nck;
+        if (hi <= lo || u1 - u0 > 1) return -1.0;
+        double t;
+        if (u1 == u0) {
+            t = (double)((hi - lo + warps - 1) / warps);
+        } else {   // the kernel's division of the warps: the best of the splits
+            const int64_t cut = (u0 + 1) * nck, nA = cut - lo, nB = hi - cut;
+            int64_t bt = -1;
+            for (int k = 1; k < warps; ++k) {
+                const int64_t ta = (nA + k - 1) / k, tb = (nB + warps - k - 1) / (warps - k);
+                const int64_t tk = ta > tb ? ta : tb;
+                if (bt < 0 || tk < bt) bt = tk;
+            }
+            t = (double)bt;
+        }
+        worst = t > worst ? t : worst;
+    }
+    int64_t slots = 0;
+    for (int64_t u = 0; u < units; ++u) {
+        const int64_t cf = ((u * nck + 1) * nC - 1) / N, cl = ((u * nck + nck) * nC - 1) / N;
+        slots = cl - cf + 1 > slots ? cl - cf + 1 : slots;
+    }
+    *nC_out = nC;
+    *slots_out = (int)slots;
+    return worst + kSetup;
 }
 
 struct DecodePlan {
@@ -51,6 +92,7 @@ struct DecodePlan {
     bool use_mma = false;
     int nsplit = 0;
     int64_t split_tokens = 0;
+    int64_t sk_ctas = 0, sk_nck = 0;     // stream-K grid (sk_ctas > 0)
     size_t off_qp = 0, off_up = 0, off_ml = 0, off_acc = 0, bytes = 0;
 };
 
@@ -63,19 +105,37 @@ void layout_ws(int d, size_t BHq, int nsplit, DecodePlan* p) {
     p->bytes = off;
 }
 
+// upper_bound: the plan whose workspace bounds every call up to Tmax tokens.
+// equal_len: every sequence has Tmax tokens (no per-sequence lengths), which
+// lets the tensor-core kernel take the stream-K grid when it models faster.
 bool make_plan(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t Tmax, DecodePlan* p,
-               bool upper_bound) {
+               bool upper_bound, bool equal_len = false) {
     if (!h || B < 0 || Hq <= 0 || Hkv <= 0 || Tmax < 0 || Hq % Hkv) return false;
     const int d = h->d;
     p->G = (int)(Hq / Hkv);
-    p->use_mma = !h->force_simt && mma_supported(d, p->G);
+    p->use_mma = h->decode_path != 1 && mma_supported(d, p->G);
     const int64_t pairs = B * Hkv > 0 ? B * Hkv * decode_head_groups(p->use_mma, p->G) : 1;
     const int64_t cap = (int64_t)h->num_sms * decode_ctas_per_sm(p->use_mma);
     const int chunk = decode_chunk_tokens(d, p->use_mma);
     const int64_t nchunk = Tmax > 0 ? (Tmax + chunk - 1) / chunk : 1;
+    const int warps = decode_warps(p->use_mma, p->G);
+    double t_split = 0.0;
     p->nsplit = upper_bound ? (int)split_loop_bound(cap, pairs, nchunk)
-                            : choose_nsplit(cap, decode_warps(p->use_mma, p->G), pairs, nchunk);
+                            : choose_nsplit(cap, warps, pairs, nchunk, &t_split);
     p->split_tokens = ((nchunk + p->nsplit - 1) / p->nsplit) * chunk;
+    p->sk_ctas = p->sk_nck = 0;
+    if (!upper_bound && equal_len && p->use_mma && Tmax > 0 && B * Hkv > 0) {
+        int64_t nC = 0;
+        int slots = 0;
+        const double t_sk = streamk_plan(cap, warps, pairs, nchunk, &nC, &slots);
+        // the workspace of any call was sized by the split count bound
+        const bool faster = h->decode_path == 3 || (h->decode_path == 0 && t_sk < t_split);
+        if (t_sk > 0.0 && faster && slots <= split_loop_bound(cap, pairs, nchunk)) {
+            p->nsplit = slots;
+            p->sk_ctas = nC;
+            p->sk_nck = nchunk;
+        }
+    }
     layout_ws(d, (size_t)(B * Hq), p->nsplit, p);
     return true;
 }
@@ -148,7 +208,7 @@ tq_status prepare_attend(const tq_handle* h, const void* q, tq_dtype qdt, int64_
     if (cudaGetDevice(&dev) != cudaSuccess) return TQ_ERR_CUDA;
     if (dev != h->device) return TQ_ERR_INVALID_ARG;
     const int64_t Tmax = seq_lens ? kc->Tcap : T;
-    if (!make_plan(h, B, Hq, Hkv, Tmax, p, false)) return TQ_ERR_INVALID_ARG;
+    if (!make_plan(h, B, Hq, Hkv, Tmax, p, false, seq_lens == nullptr)) return TQ_ERR_INVALID_ARG;
     if (ws_bytes < p->bytes) return TQ_ERR_WORKSPACE;
     uint8_t* w = static_cast<uint8_t*>(ws);
     *a = DecArgs{};
@@ -167,6 +227,9 @@ tq_status prepare_attend(const tq_handle* h, const void* q, tq_dtype qdt, int64_
     a->B = B; a->Hq = Hq; a->Hkv = Hkv;
     a->nsplit = p->nsplit;
     a->split_tokens = p->split_tokens;
+    a->sk_ctas = (int)p->sk_ctas;
+    a->sk_nck = p->sk_nck;
+    a->sk_total = p->sk_nck * B * Hkv * decode_head_groups(p->use_mma, p->G);
     a->scale_log2 = scale * kLog2e;
     a->part_ml = reinterpret_cast<float*>(w + p->off_ml);
     a->part_acc = reinterpret_cast<float*>(w + p->off_acc);
@@ -419,7 +482,7 @@ tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype qdt, int
 
 const char* tq_attend_path(const tq_handle* h, int64_t Hq, int64_t Hkv) {
     if (!h || Hq <= 0 || Hkv <= 0 || Hq % Hkv) return "invalid";
-    return (!h->force_simt && mma_supported(h->d, (int)(Hq / Hkv))) ? "mma" : "simt";
+    return (h->decode_path != 1 && mma_supported(h->d, (int)(Hq / Hkv))) ? "mma" : "simt";
 }
 
 tq_status tq_attend_decode(const tq_handle* h, const void* q, tq_dtype qdt, int64_t B, int64_t Hq,
@@ -488,8 +551,8 @@ tq_status tq_set_wait_limit(tq_handle* h, int first_wait) {
 }
 
 tq_status tq_set_decode_path(tq_handle* h, int path) {
-    if (!h || path < 0 || path > 1) return TQ_ERR_INVALID_ARG;
-    h->force_simt = path;
+    if (!h || path < 0 || path > 3) return TQ_ERR_INVALID_ARG;
+    h->decode_path = path;
     return TQ_OK;
 }
 

@@ -61,6 +61,20 @@ __device__ __forceinline__ int64_t staged_block(const int32_t* table, const int3
     }
     return p;
 }
+// Warps given to the first of two units sharing a stream-K CTA (nA and nB
+// chunks): the split with the fewest chunk-steps for the slower group.
+template <int NW>
+__device__ __forceinline__ int streamk_split(int64_t nA, int64_t nB) {
+    int best = 1;
+    int64_t bt = INT64_MAX;
+    for (int k = 1; k < NW; ++k) {
+        const int64_t ta = (nA + k - 1) / k, tb = (nB + NW - k - 1) / (NW - k);
+        const int64_t t = ta > tb ? ta : tb;
+        if (t < bt) { bt = t; best = k; }
+    }
+    return best;
+}
+
 // Token-row orientation: each mma tile has 16 tokens on M and the (head,
 // hi|lo) columns on N (NT n-tiles of 4 heads), so no M rows are wasted:
 //   scores  S[16 tok][8] += Kdeq[16 tok][16 coords] * Q'[16 coords][8]   (D/16 coordinate chunks, fp16)
@@ -75,6 +89,7 @@ template <int D, int NT, int NW, bool QJL>
 __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs a, int G) {
     using C = Cfg<D, QJL>;
     constexpr int kKC = C::kKC;
+    constexpr int kSBGroup = 2 * NT * kKC * 32;   // uint2 entries of one group's q'/u' fragments (d = 256)
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)NW * kStages * C::kStageB);
     // per-warp (max, sum) of each head for the merge: [NW][8][2]
@@ -88,33 +103,94 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gr = lane >> 2, tq4 = lane & 3;
     uint8_t* ring = smem + (size_t)warp * kStages * C::kStageB;
-    const int split = blockIdx.x, b = blockIdx.z;
     const int hgroups = (G + 7) >> 3;
-    const int hkv = blockIdx.y / hgroups;
-    const int g0 = (blockIdx.y - hkv * hgroups) * 8;          // first query head of this CTA's group
-    const int Gl = G - g0 < 8 ? G - g0 : 8;                    // query heads in the group
-    const int64_t hbase = (int64_t)b * a.Hq + (int64_t)hkv * G + g0;
 
-    int64_t Tb = a.seq_lens ? (int64_t)a.seq_lens[b] : a.T;
+    // ---------------- this CTA's work: one or two (unit, token range) groups.
+    // A unit is (batch, kv head, query-head group).  Uniform split grid: one
+    // group, unit (blockIdx.z, blockIdx.y), split blockIdx.x.  Stream-K: the
+    // CTA's chunk range lies in at most two units; its warps are divided
+    // between them in proportion to their chunks (warps [0, kA) and [kA, NW)),
+    // and each group writes one partial slot of its unit: slot c - (first CTA
+    // of the unit).  The CTA holding a unit's last chunk also writes the
+    // unit's unused slots as empty partials.
+    int ngrp = 1, kA = NW;
+    int64_t unitA = 0, s0A = 0, s1A = 0, unitB = 0, s0B = 0, s1B = 0;   // group 0 (A) and group 1 (B)
+    int slotA = 0, slotB = 0;
+    bool endA = false, endB = false;
+    int64_t Tb = a.seq_lens ? (int64_t)a.seq_lens[blockIdx.z] : a.T;
     Tb = Tb < 0 ? 0 : (Tb > a.Tcap ? a.Tcap : Tb);
-    const int64_t s0 = (int64_t)split * a.split_tokens;
-    const int64_t s1 = (s0 + a.split_tokens < Tb) ? s0 + a.split_tokens : Tb;
+    if (a.sk_ctas == 0) {
+        unitA = (int64_t)blockIdx.z * a.Hkv * hgroups + blockIdx.y;
+        s0A = (int64_t)blockIdx.x * a.split_tokens;
+        s1A = (s0A + a.split_tokens < Tb) ? s0A + a.split_tokens : Tb;
+        slotA = blockIdx.x;
+    } else {
+        const int64_t N = a.sk_total, nck = a.sk_nck, nC = a.sk_ctas, c = blockIdx.x;
+        const int64_t lo = c * N / nC, hi = (c + 1) * N / nC;
+        const int64_t u0 = lo / nck, u1 = (hi - 1) / nck;
+        const int64_t cut = (u0 + 1) * nck < hi ? (u0 + 1) * nck : hi;
+        auto tok = [&](int64_t x, int64_t u) {                 // chunk x of unit u as a token bound
+            const int64_t t = (x - u * nck) * C::kChunk;
+            return t < Tb ? t : Tb;
+        };
+        auto first_cta = [&](int64_t u) { return (int)(((u * nck + 1) * nC - 1) / N); };
+        unitA = u0;
+        s0A = tok(lo, u0);
+        s1A = tok(cut, u0);
+        slotA = (int)c - first_cta(u0);
+        endA = cut == (u0 + 1) * nck;
+        if (u1 != u0) {
+            kA = streamk_split<NW>(cut - lo, hi - cut);
+            ngrp = 2;
+            unitB = u1;
+            s0B = tok(cut, u1);
+            s1B = tok(hi, u1);
+            slotB = (int)c - first_cta(u1);
+            endB = hi == (u1 + 1) * nck;
+        }
+    }
+    const int grp = warp < kA ? 0 : 1;
+    const int wi = grp ? warp - kA : warp;                     // this warp among its group's
+    const int nw = grp ? NW - kA : kA;
+    auto unit_rows = [&](int g, int64_t& hb, int& gl, int64_t& sq) {
+        const int64_t u = g ? unitB : unitA;
+        const int64_t bk = u / hgroups;                          // b * Hkv + kv head
+        const int hg = (int)(u - bk * hgroups);
+        const int64_t bb = bk / a.Hkv, kv = bk - bb * a.Hkv;
+        gl = G - 8 * hg < 8 ? G - 8 * hg : 8;
+        hb = bb * a.Hq + kv * G + 8 * hg;
+        sq = bk;
+    };
+    int64_t hbase, seq;
+    int Gl;
+    unit_rows(grp, hbase, Gl, seq);
+    const int64_t s0 = grp ? s0B : s0A, s1 = grp ? s1B : s1A;
     const int nchunk = s1 > s0 ? (int)((s1 - s0 + C::kChunk - 1) / C::kChunk) : 0;
-    const int nmine = nchunk > warp ? (nchunk - warp + NW - 1) / NW : 0;
-    const int64_t seq = (int64_t)b * a.Hkv + hkv;
-    // A paged cache's table entries for this split go to shared memory first (one
-    // coalesced load per CTA), so the per-chunk lookups that feed the bulk copies
-    // do not wait on global memory; longer splits keep the direct lookups.
-    const int64_t lb0 = s0 >> 6;
-    const int ntab = s1 > s0 ? (int)(((s1 + 63) >> 6) - lb0) : 0;
-    const bool staged = (a.ktable || a.vtable) && ntab <= kTabMax;
+    const int nmine = nchunk > wi ? (nchunk - wi + nw - 1) / nw : 0;
+    // A paged cache's table entries for the CTA's token ranges go to shared
+    // memory first (one coalesced load per CTA), so the per-chunk lookups that
+    // feed the bulk copies do not wait on global memory; longer ranges keep the
+    // direct lookups.
+    const int64_t lb0A = s0A >> 6, lb0B = s0B >> 6;
+    const int ntabA = s1A > s0A ? (int)(((s1A + 63) >> 6) - lb0A) : 0;
+    const int ntabB = ngrp == 2 && s1B > s0B ? (int)(((s1B + 63) >> 6) - lb0B) : 0;
+    const bool staged = (a.ktable || a.vtable) && ntabA + ntabB <= kTabMax;
     if (staged) {
-        for (int i = threadIdx.x; i < ntab; i += NW * 32) {
-            sTab[i] = a.ktable ? __ldg(a.ktable + seq * a.NB + lb0 + i) : 0;
-            sTab[kTabMax + i] = a.vtable ? __ldg(a.vtable + seq * a.NB + lb0 + i) : 0;
+        for (int g = 0; g < ngrp; ++g) {
+            int64_t hb_, sq_;
+            int gl_;
+            unit_rows(g, hb_, gl_, sq_);
+            const int off = g ? ntabA : 0, n = g ? ntabB : ntabA;
+            const int64_t l0 = g ? lb0B : lb0A;
+            for (int i = threadIdx.x; i < n; i += NW * 32) {
+                sTab[off + i] = a.ktable ? __ldg(a.ktable + sq_ * a.NB + l0 + i) : 0;
+                sTab[kTabMax + off + i] = a.vtable ? __ldg(a.vtable + sq_ * a.NB + l0 + i) : 0;
+            }
         }
         __syncthreads();
     }
+    const int64_t lb0 = grp ? lb0B : lb0A;
+    const int toff = grp ? ntabA : 0;
     const int64_t kbb = block_bytes(D, QJL), vbb = block_bytes(D, false);
 
     if (lane == 0)
@@ -124,18 +200,18 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
 
     // cache blocks (K, V) of this warp's chunk i; a paged cache reads its block table
     auto blocks_of = [&](int i, int64_t& kblk, int64_t& vblk) {
-        const int64_t t0 = s0 + (int64_t)(warp + i * NW) * C::kChunk;
+        const int64_t t0 = s0 + (int64_t)(wi + i * nw) * C::kChunk;
         if (staged) {
-            kblk = staged_block(a.ktable, sTab, a.kpool, seq * a.NB + (t0 >> 6), (int)((t0 >> 6) - lb0), a.err);
-            vblk = staged_block(a.vtable, sTab + kTabMax, a.vpool, seq * a.NB + (t0 >> 6), (int)((t0 >> 6) - lb0),
-                                a.err);
+            const int ti = (int)((t0 >> 6) - lb0) + toff;
+            kblk = staged_block(a.ktable, sTab, a.kpool, seq * a.NB + (t0 >> 6), ti, a.err);
+            vblk = staged_block(a.vtable, sTab + kTabMax, a.vpool, seq * a.NB + (t0 >> 6), ti, a.err);
         } else {
             kblk = cache_block(a.ktable, a.kpool, a.NB, seq, t0 >> 6, a.err);
             vblk = cache_block(a.vtable, a.vpool, a.NB, seq, t0 >> 6, a.err);
         }
     };
     auto issue = [&](int i, int64_t kblk, int64_t vblk) {
-        const int64_t t0 = s0 + (int64_t)(warp + i * NW) * C::kChunk;     // multiple of the chunk
+        const int64_t t0 = s0 + (int64_t)(wi + i * nw) * C::kChunk;     // multiple of the chunk
         const int sub = (int)((t0 & 63) / C::kChunk);
         const uint8_t* kb = a.kc + (kblk >= 0 ? kblk : 0) * kbb;    // a bad table entry reads block 0
         const uint8_t* vb = a.vc + (vblk >= 0 ? vblk : 0) * vbb;
@@ -156,7 +232,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     };
     // chunks holding tokens that a chained encode writes are fetched only after pdl_wait
     auto fresh = [&](int i) {
-        const int64_t t0 = s0 + (int64_t)(warp + i * NW) * C::kChunk;
+        const int64_t t0 = s0 + (int64_t)(wi + i * nw) * C::kChunk;
         return t0 < a.fresh_hi && a.fresh_lo < t0 + C::kChunk;
     };
     if (lane == 0) {
@@ -188,11 +264,11 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
 
     // B-operand fragment of k-step kc: column n = gr of n-tile nt is head
     // 4 nt + gr / 2, limb gr % 2; rows 16 kc + 2 tq4 (+1), +8 (+9)
-    auto b_frag = [&](const float* base, int nt, int kc, uint32_t& r0, uint32_t& r1) {
+    auto b_frag = [&](const float* base, int64_t hb, int gl, int nt, int kc, uint32_t& r0, uint32_t& r1) {
         const int hcol = 4 * nt + (gr >> 1);
         float x[4] = {0.f, 0.f, 0.f, 0.f};
-        if (hcol < Gl) {
-            const float* p = base + (hbase + hcol) * D + 16 * kc + 2 * tq4;
+        if (hcol < gl) {
+            const float* p = base + (hb + hcol) * D + 16 * kc + 2 * tq4;
             x[0] = p[0]; x[1] = p[1]; x[2] = p[8]; x[3] = p[9];
         }
         uint32_t h0, l0, h1, l1;
@@ -206,16 +282,23 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int kc = 0; kc < kKC; ++kc) b_frag(a.qp, nt, kc, bq[nt][kc][0], bq[nt][kc][1]);
+            for (int kc = 0; kc < kKC; ++kc) b_frag(a.qp, hbase, Gl, nt, kc, bq[nt][kc][0], bq[nt][kc][1]);
     } else {
-        for (int kc = warp; kc < kKC; kc += NW)
+        // q' fragments of each group's unit, in that group's copy of sB
+        for (int idx = warp; idx < ngrp * kKC; idx += NW) {
+            const int g = idx >= kKC ? 1 : 0, kc = idx - g * kKC;
+            int64_t hb_, sq_;
+            int gl_;
+            unit_rows(g, hb_, gl_, sq_);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 uint32_t r0, r1;
-                b_frag(a.qp, nt, kc, r0, r1);
-                sB[(nt * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
+                b_frag(a.qp, hb_, gl_, nt, kc, r0, r1);
+                sB[(size_t)g * kSBGroup + (nt * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
             }
+        }
     }
+    [[maybe_unused]] const uint2* sBw = sB + (size_t)grp * kSBGroup;   // this warp's group's operands
     // QJL term on int8 operands.  u' of each head is taken to 16-bit fixed point,
     // u_int = rint(u' kQ / max|u'|), as two signed byte limbs (256 hi + lo): B column
     // n = gr of n-tile nt is head 4 nt + gr / 2, limb gr % 2.  The A operand byte e
@@ -266,8 +349,8 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                 if constexpr (C::kBRegs) {
                     iu[nt][kb][0] = w[0];
                     iu[nt][kb][1] = w[1];
-                } else if (warp == 0) {
-                    sB[((NT + nt) * kKC + kb) * 32 + lane] = make_uint2(w[0], w[1]);
+                } else if (wi == 0) {
+                    sB[(size_t)grp * kSBGroup + ((NT + nt) * kKC + kb) * 32 + lane] = make_uint2(w[0], w[1]);
                 }
             }
             usum += __shfl_xor_sync(kFull, usum, 1);
@@ -310,7 +393,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
             break;
         }
         const uint8_t* st = ring + (i % kStages) * C::kStageB;
-        const int64_t tok0 = s0 + (int64_t)(warp + i * NW) * C::kChunk;
+        const int64_t tok0 = s0 + (int64_t)(wi + i * nw) * C::kChunk;
         const int nvalid = (int)((s1 - tok0) < C::kChunk ? (s1 - tok0) : C::kChunk);
 
         // one 16-token tile; PARTIAL masks tokens beyond nvalid (only the last
@@ -348,7 +431,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                     if constexpr (C::kBRegs) {
                         mma16816(acc[nt], ka, bq[nt][kc][0], bq[nt][kc][1]);
                     } else {
-                        const uint2 fq = sB[(nt * kKC + kc) * 32 + lane];
+                        const uint2 fq = sBw[(nt * kKC + kc) * 32 + lane];
                         mma16816(acc[nt], ka, fq.x, fq.y);
                     }
                 }
@@ -364,7 +447,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                             if constexpr (C::kBRegs) {
                                 imma16832(accS[nt], sg, iu[nt][kb][0], iu[nt][kb][1]);
                             } else {
-                                const uint2 fu = sB[((NT + nt) * kKC + kb) * 32 + lane];
+                                const uint2 fu = sBw[((NT + nt) * kKC + kb) * 32 + lane];
                                 imma16832(accS[nt], sg, fu.x, fu.y);
                             }
                         }
@@ -492,29 +575,43 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         }
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < Gl * D; idx += NW * 32) {
-        const int g = idx / D, j = idx % D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, sML[(w * 8 + g) * 2]);
-        float L = 0.f, A = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                const float mw = sML[(w * 8 + g) * 2];
-                if (mw == -INFINITY) continue;                    // empty or failed warp
-                const float* wb = reinterpret_cast<const float*>(smem + (size_t)w * kStages * C::kStageB) + g * D;
-                const float f = exp2f(mw - M);
-                L = fmaf(f, sML[(w * 8 + g) * 2 + 1], L);
-                A = fmaf(f, wb[j], A);
+    for (int g = 0; g < ngrp; ++g) {
+        int64_t hb_, sq_;
+        int gl_;
+        unit_rows(g, hb_, gl_, sq_);
+        const int w0 = g ? kA : 0, w1 = g ? NW : kA;
+        for (int idx = threadIdx.x; idx < gl_ * D; idx += NW * 32) {
+            const int h = idx / D, j = idx % D;
+            float M = -INFINITY;
+            for (int w = w0; w < w1; ++w) M = fmaxf(M, sML[(w * 8 + h) * 2]);
+            float L = 0.f, A = 0.f;
+            if (M != -INFINITY) {
+                for (int w = w0; w < w1; ++w) {
+                    const float mw = sML[(w * 8 + h) * 2];
+                    if (mw == -INFINITY) continue;                    // empty or failed warp
+                    const float* wb = reinterpret_cast<const float*>(smem + (size_t)w * kStages * C::kStageB) + h * D;
+                    const float f = exp2f(mw - M);
+                    L = fmaf(f, sML[(w * 8 + h) * 2 + 1], L);
+                    A = fmaf(f, wb[j], A);
+                }
             }
-        }
-        const int64_t bh = hbase + g;
-        const int64_t pidx = bh * a.nsplit + split;
-        a.part_acc[pidx * D + j] = A;
-        if (j == 0) {
-            a.part_ml[2 * pidx] = M;
-            a.part_ml[2 * pidx + 1] = L;
+            const int slot = g ? slotB : slotA;
+            const int64_t pidx = (hb_ + h) * a.nsplit + slot;
+            a.part_acc[pidx * D + j] = A;
+            if (j == 0) {
+                a.part_ml[2 * pidx] = M;
+                a.part_ml[2 * pidx + 1] = L;
+            }
+            // the CTA holding the unit's last chunk empties the unit's unused slots
+            if (g ? endB : endA)
+                for (int sp = slot + 1; sp < a.nsplit; ++sp) {
+                    const int64_t e = (hb_ + h) * a.nsplit + sp;
+                    a.part_acc[e * D + j] = 0.f;
+                    if (j == 0) {
+                        a.part_ml[2 * e] = -INFINITY;
+                        a.part_ml[2 * e + 1] = 0.f;
+                    }
+                }
         }
     }
 }
@@ -529,11 +626,12 @@ cudaError_t launch_mma_t(const DecArgs& a, int G, cudaStream_t s) {
     using C = Cfg<D, QJL>;
     const size_t smem = (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
                         (size_t)NW * 8 * 2 * sizeof(float) + 2 * kTabMax * sizeof(int32_t) +
-                        (C::kBRegs ? 0 : (size_t)2 * NT * C::kKC * 32 * sizeof(uint2));
+                        (C::kBRegs ? 0 : (size_t)2 * 2 * NT * C::kKC * 32 * sizeof(uint2));
     auto kern = tq_decode_mma_kernel<D, NT, NW, QJL>;
     cudaError_t e = set_smem_once<tq_decode_mma_kernel<D, NT, NW, QJL>>((int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(a.nsplit, (unsigned)(a.Hkv * ((G + 7) / 8)), (unsigned)a.B);
+    const dim3 grid = a.sk_ctas > 0 ? dim3((unsigned)a.sk_ctas)
+                                    : dim3(a.nsplit, (unsigned)(a.Hkv * ((G + 7) / 8)), (unsigned)a.B);
     return launch_pdl(kern, grid, dim3(NW * 32), smem, s, a, G);
 }
 

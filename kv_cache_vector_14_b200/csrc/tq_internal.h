@@ -135,8 +135,14 @@ struct DecArgs {
     int64_t T;                // used when seq_lens is null
     int64_t Tcap;
     int64_t B, Hq, Hkv;
-    int nsplit;
-    int64_t split_tokens;     // tokens per split, multiple of 64
+    int nsplit;               // partial slots per query head
+    int64_t split_tokens;     // tokens per split, multiple of 64 (uniform split grid)
+    // Stream-K grid (sk_ctas > 0; equal-length sequences only): the units
+    // (batch, kv head, query-head group) laid end to end, sk_nck chunks each
+    // (sk_total in all), and CTA c takes chunks [c sk_total / sk_ctas,
+    // (c + 1) sk_total / sk_ctas), at most two units' worth.
+    int sk_ctas;
+    int64_t sk_nck, sk_total;
     float scale_log2;         // softmax scale * log2(e)
     float* part_ml;           // [B*Hq][nsplit][2] (running max in log2 units, sum)
     float* part_acc;          // [B*Hq][nsplit][d] rotated-domain accumulators
@@ -265,6 +271,6 @@ struct tq_handle {
     tqi::Codebook cb{};
     cudaEvent_t ev_start = nullptr;   // optional timing of the split-K kernel
     cudaEvent_t ev_stop = nullptr;
-    int force_simt = 0;               // diagnostics: always use the SIMT decode kernel
+    int decode_path = 0;              // diagnostics: 0 auto, 1 SIMT, 2 tensor-core uniform splits, 3 tensor-core stream-K
     int first_wait = -1;              // diagnostics: try count of the decode's first ring wait (< 0: full bound)
 };

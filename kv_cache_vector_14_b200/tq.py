@@ -310,8 +310,11 @@ def tq_set_wait_limit(h, first_wait: int) -> None:
 
 
 def tq_set_decode_path(h, path: str) -> None:
-    """"auto" (tensor-core kernel where supported) or "simt"."""
-    _check(lib().tq_set_decode_path(h, {"auto": 0, "simt": 1}[path]), "tq_set_decode_path")
+    """"auto" (tensor-core kernel where supported, cost-model partition), "simt",
+    "split" (tensor-core kernel, uniform split grid) or "streamk" (tensor-core
+    kernel, stream-K grid wherever it fits)."""
+    _check(lib().tq_set_decode_path(h, {"auto": 0, "simt": 1, "split": 2, "streamk": 3}[path]),
+           "tq_set_decode_path")
 
 
 def tq_attend_path(h, Hq: int, Hkv: int) -> str:

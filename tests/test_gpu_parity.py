@@ -673,6 +673,72 @@ def test_attend_query_dtypes(decode_path, handles, prms, qdt):
     assert err.max() <= ATT_TOL
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("G", [1, 4, 12])
+@pytest.mark.parametrize("paged", [False, True])
+def test_streamk_partition_matches_split_and_oracle(handles, prms, d, G, paged):
+    """The stream-K grid (equal shares of the units' chunks laid end to end,
+    CTAs that straddle two units with their warps divided between them, a
+    partial slot per overlapping CTA, unused slots emptied by the unit's last
+    CTA) against the uniform split grid of the same kernel (1e-5) and against
+    the oracle, with head groups (G = 12), paged caches and a ragged tail; then
+    a fused append step on the stream-K grid equals the separate calls bit for
+    bit."""
+    h = handles[d]
+    B, Hkv, T, Tcap = 3, 5, 3001, 3072
+    Hq, NB = Hkv * G, Tcap // 64
+    x = synthetic.gaussian((2, B, Hkv, T + 1, d), seed=90 + d + G)
+    xt = torch_input(x, "bf16")
+    kc, vc = tq.Cache(d, True, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
+    if paged:
+        pool = 2 * B * Hkv * NB + 3
+        perm = np.random.default_rng(d + G).permutation(pool).astype(np.int32)
+        kt = torch.from_numpy(perm[:B * Hkv * NB].reshape(B * Hkv, NB).copy()).cuda()
+        vt = torch.from_numpy(perm[B * Hkv * NB:2 * B * Hkv * NB].reshape(B * Hkv, NB).copy()).cuda()
+        ka = tq.Cache(d, True, B, Hkv, Tcap, block_table=kt, pool_blocks=pool)
+        va = tq.Cache(d, False, B, Hkv, Tcap, block_table=vt, pool_blocks=pool)
+    else:
+        ka, va = tq.Cache(d, True, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
+    for k_, v_ in ((kc, vc), (ka, va)) if paged else ((ka, va),):
+        tq.tq_encode_k(h, xt[0, :, :, :T], k_, 0)
+        tq.tq_encode_v(h, xt[1, :, :, :T], v_, 0)
+    if not paged:
+        kc, vc = ka, va
+    q = synthetic.gaussian((B, Hq, d), seed=91)
+    qt = torch_input(q, "f32")
+    ws = torch.empty(tq.tq_attend_workspace_bytes(h, B, Hq, Hkv, Tcap), dtype=torch.uint8, device="cuda")
+    scale = 1.0 / np.sqrt(d)
+    outs = {}
+    try:
+        for path in ("split", "streamk"):
+            tq.tq_set_decode_path(h, path)
+            out = torch.full((B, Hq, d), float("nan"), dtype=torch.float32, device="cuda")
+            tq.tq_attend_decode(h, qt, ka, va, out, ws, T=T, scale=scale)
+            outs[path] = out.cpu().numpy()
+        # one fused append step on the stream-K grid against the separate calls
+        ref = torch.empty((B, Hq, d), dtype=torch.float32, device="cuda")
+        fused = torch.full((B, Hq, d), float("nan"), dtype=torch.float32, device="cuda")
+        kb, vb = ka.buf.clone(), va.buf.clone()
+        tq.tq_encode_k(h, xt[0, :, :, T:T + 1], ka, T)
+        tq.tq_encode_v(h, xt[1, :, :, T:T + 1], va, T)
+        tq.tq_attend_decode(h, qt, ka, va, ref, ws, T=T + 1, scale=scale)
+        ka.buf.copy_(kb)
+        va.buf.copy_(vb)
+        tq.tq_append_attend(h, xt[0, :, :, T:T + 1], xt[1, :, :, T:T + 1], ka, va, T, qt, fused, ws, scale=scale)
+        torch.cuda.synchronize()
+    finally:
+        tq.tq_set_decode_path(h, "auto")
+    assert np.all(np.isfinite(outs["streamk"]))
+    assert rel_err_rows(outs["streamk"], outs["split"]).max() <= 1e-5
+    oref = oracle_attend(prms[d], q.astype(np.float64), unpack_cache(kc, 0, T), unpack_cache(vc, 0, T), Hkv,
+                         [T] * B, scale)
+    err = rel_err_rows(outs["streamk"], oref)
+    print("stream-K max rel err", err.max())
+    assert err.max() <= ATT_TOL
+    assert torch.equal(fused, ref)
+    assert tq.tq_device_status(h) == tq.TQ_OK
+
+
 def test_split_count_invariance(decode_path, handles):
     """Different split plans (by T, or by Tcap through seq_lens) agree within 1e-5."""
     d, B, Hq, Hkv, T, Tcap = 128, 2, 8, 2, 3000, 8192
