@@ -63,9 +63,9 @@ __global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t B
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int64_t h0 = (int64_t)blockIdx.x * QH;
     const int rc = blockIdx.y;
-    for (int i = t; i < D * kRC / 4; i += D) {
+    for (int i = t; i < D * kRC / 4; i += D) {          // in flight during the rotation below
         const int jr = i / (kRC / 4), c4 = i % (kRC / 4);
-        reinterpret_cast<float4*>(sst)[i] = __ldg(reinterpret_cast<const float4*>(ST + (size_t)jr * D + rc * kRC) + c4);
+        cp_async16(reinterpret_cast<float4*>(sst) + i, reinterpret_cast<const float4*>(ST + (size_t)jr * D + rc * kRC) + c4);
     }
     const float ds = dsign[t];
 #pragma unroll
@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t B
     const float inv = 1.0f / sqrtf((float)D);
 #pragma unroll
     for (int k = 0; k < QH; ++k) v[k * D + t] *= inv;
+    cp_async_wait_all();
     __syncthreads();
     float acc[QH];
 #pragma unroll

@@ -316,14 +316,15 @@ __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(con
     const int rg0 = blockIdx.y * RG;                // first row group of this CTA
     if (threadIdx.x < 8) sC[threadIdx.x] = a.cb.c[threadIdx.x];
     {
-        // this CTA's rows of the lane-ordered JL matrix: RG*32 floats per column
+        // this CTA's rows of the lane-ordered JL matrix: RG*32 floats per column,
+        // all copies in flight at once (they overlap the vector's load and rotation)
         const float4* src = reinterpret_cast<const float4*>(a.sthr);
         for (int i = threadIdx.x; i < D * RG * 8; i += kSmallWarps * 32) {
             const int j = i / (RG * 8), c = i % (RG * 8);
-            reinterpret_cast<float4*>(sS)[i] = __ldg(src + ((size_t)j * R + rg0) * 8 + c);
+            cp_async16(reinterpret_cast<float4*>(sS) + i, src + ((size_t)j * R + rg0) * 8 + c);
         }
     }
-    __syncthreads();
+    __syncthreads();                                 // sC
     const int64_t N = a.B * a.Hkv * a.Tnew;
     const int64_t gv0 = (int64_t)blockIdx.x * kSmallWarps + warp;
     const bool valid = gv0 < N;
@@ -376,6 +377,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32) tq_encode_k_small_kernel(con
         scode[warp][stage_at<D>(j)] = (uint8_t)code;
     }
     g2 = warp_sum(g2);
+    cp_async_wait_all();
+    __syncthreads();                                 // this CTA's rows of S are staged
     const bool writer = wr && blockIdx.y == 0;
     if (writer && lane == 0) {
         const int64_t norm_off = kBlockT * code_bytes(D) + kBlockT * sign_bytes(D);

@@ -27,6 +27,15 @@ __device__ __forceinline__ uint64_t global_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
+// 16-byte copy global -> shared that does not pass through registers
+// (cp.async, cache-global); many of them are in flight at once and one
+// cp_async_wait_all() waits for all of this thread's.  Both addresses 16-byte
+// aligned.
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst_smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 #endif
 
 // Codebook passed by value to every kernel (it lands in the constant bank).
