@@ -48,11 +48,12 @@ int choose_nsplit(int64_t cap, int warps, int64_t pairs, int64_t nchunk, double*
 }
 
 // Stream-K plan for sequences of one length: nC CTAs take equal shares of the
-// units' chunks laid end to end (units x nck in all).  With nC >= units a
-// share spans at most two units; the kernel then divides the CTA's warps
-// between them in proportion to their chunks.  Returns the modelled
-// chunk-steps of the slowest CTA (plus the fixed cost) and the partial slots
-// a unit needs (the CTAs that overlap it), or -1 when the shape does not fit.
+// units' chunks laid end to end (units x nck in all), and each warp a
+// contiguous run of its CTA's share.  With nC >= units a share spans at most
+// two units, so at most one warp per CTA crosses into the next unit (it pays
+// about half a chunk-step to switch).  Returns the modelled chunk-steps of the
+// slowest CTA (plus the fixed cost) and the partial slots a unit needs (the
+// CTAs that overlap it), or -1 when the shape does not fit.
 double streamk_plan(int64_t cap, int warps, int64_t units, int64_t nck, int64_t* nC_out, int* slots_out) {
     const int64_t N = units * nck;
     const int64_t nC = cap < N ? cap : N;
@@ -62,19 +63,7 @@ double streamk_plan(int64_t cap, int warps, int64_t units, int64_t nck, int64_t*
         const int64_t lo = c * N / nC, hi = (c + 1) * N / nC;
         const int64_t u0 = lo / nck, u1 = (hi - 1) / nck;
         if (hi <= lo || u1 - u0 > 1) return -1.0;
-        double t;
-        if (u1 == u0) {
-            t = (double)((hi - lo + warps - 1) / warps);
-        } else {   // the kernel's division of the warps: the best of the splits
-            const int64_t cut = (u0 + 1) * nck, nA = cut - lo, nB = hi - cut;
-            int64_t bt = -1;
-            for (int k = 1; k < warps; ++k) {
-                const int64_t ta = (nA + k - 1) / k, tb = (nB + warps - k - 1) / (warps - k);
-                const int64_t tk = ta > tb ? ta : tb;
-                if (bt < 0 || tk < bt) bt = tk;
-            }
-            t = (double)bt;
-        }
+        const double t = (double)((hi - lo + warps - 1) / warps) + (u1 != u0 ? 0.5 : 0.0);
         worst = t > worst ? t : worst;
     }
     int64_t slots = 0;

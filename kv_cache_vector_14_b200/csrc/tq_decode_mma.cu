@@ -61,18 +61,17 @@ __device__ __forceinline__ int64_t staged_block(const int32_t* table, const int3
     }
     return p;
 }
-// Warps given to the first of two units sharing a stream-K CTA (nA and nB
-// chunks): the split with the fewest chunk-steps for the slower group.
-template <int NW>
-__device__ __forceinline__ int streamk_split(int64_t nA, int64_t nB) {
-    int best = 1;
-    int64_t bt = INT64_MAX;
-    for (int k = 1; k < NW; ++k) {
-        const int64_t ta = (nA + k - 1) / k, tb = (nB + NW - k - 1) / (NW - k);
-        const int64_t t = ta > tb ? ta : tb;
-        if (t < bt) { bt = t; best = k; }
+// Pool block of table row `row` (= sequence * blocks per sequence + logical
+// block) of a paged cache, or `row` itself for a contiguous cache; an entry
+// outside the pool sets the check word and gives -1, as cache_block does.
+__device__ __forceinline__ int64_t table_block(const int32_t* table, int64_t pool, int64_t row, int* err) {
+    if (!table) return row;
+    const int32_t p = __ldg(table + row);
+    if (p < 0 || (int64_t)p >= pool) {
+        atomicExch(err, 1);
+        return -1;
     }
-    return best;
+    return p;
 }
 
 // Token-row orientation: each mma tile has 16 tokens on M and the (head,
@@ -89,34 +88,45 @@ template <int D, int NT, int NW, bool QJL>
 __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs a, int G) {
     using C = Cfg<D, QJL>;
     constexpr int kKC = C::kKC;
-    constexpr int kSBGroup = 2 * NT * kKC * 32;   // uint2 entries of one group's q'/u' fragments (d = 256)
+    constexpr int kSBGroup = 2 * NT * kKC * 32;   // uint2 entries of one unit's q'/u' fragments
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)NW * kStages * C::kStageB);
     // per-warp (max, sum) of each head for the merge: [NW][8][2]
     float* sML = reinterpret_cast<float*>(smem + (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8);
-    // d = 256: q'/u' fragments per (operand, n-tile, k-step, lane), filled once per CTA
-    // paged caches: the split's slice of the K and V block tables, [2][kTabMax]
+    // paged caches: the CTA's slices of the K and V block tables, [2][kTabMax]
+    // q'/u' fragments per (unit group, operand, n-tile, k-step, lane), filled once per CTA
     int32_t* sTab = reinterpret_cast<int32_t*>(smem + (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
                                                (size_t)NW * 8 * 2 * sizeof(float));
     uint2* sB = reinterpret_cast<uint2*>(smem + (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
                                          (size_t)NW * 8 * 2 * sizeof(float) + 2 * kTabMax * sizeof(int32_t));
+    // u' factors per (unit group, kind, head): [2][2][8]
+    float* sF = reinterpret_cast<float*>(sB + 2 * kSBGroup);
+    // the crossing warp's unit-A result: accumulators [8][D], (max, sum) [8][2]
+    float* xacc = sF + 2 * 2 * 8;
+    float* xml = xacc + 8 * D;
+    int64_t* sU = reinterpret_cast<int64_t*>(xml + 8 * 2);     // [NW][2][4] unit descriptors
+    int* sMerge = reinterpret_cast<int*>(sU + NW * 8);          // [8] CTA merge facts
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gr = lane >> 2, tq4 = lane & 3;
     uint8_t* ring = smem + (size_t)warp * kStages * C::kStageB;
     const int hgroups = (G + 7) >> 3;
 
-    // ---------------- this CTA's work: one or two (unit, token range) groups.
-    // A unit is (batch, kv head, query-head group).  Uniform split grid: one
-    // group, unit (blockIdx.z, blockIdx.y), split blockIdx.x.  Stream-K: the
-    // CTA's chunk range lies in at most two units; its warps are divided
-    // between them in proportion to their chunks (warps [0, kA) and [kA, NW)),
-    // and each group writes one partial slot of its unit: slot c - (first CTA
-    // of the unit).  The CTA holding a unit's last chunk also writes the
-    // unit's unused slots as empty partials.
-    int ngrp = 1, kA = NW;
-    int64_t unitA = 0, s0A = 0, s1A = 0, unitB = 0, s0B = 0, s1B = 0;   // group 0 (A) and group 1 (B)
-    int slotA = 0, slotB = 0;
-    bool endA = false, endB = false;
+    // ---------------- this CTA's work.  A unit is (batch, kv head, query-head
+    // group).  Uniform split grid: unit (blockIdx.z, blockIdx.y), the tokens of
+    // split blockIdx.x, chunks dealt to the warps in turn.  Stream-K: the CTA's
+    // chunk range [lo, hi) of the units laid end to end lies in at most two
+    // units, A and then B from chunk `cut`; warp w takes the contiguous chunks
+    // [lo + w S / NW, lo + (w + 1) S / NW), S = hi - lo, so at most one warp
+    // crosses from A to B, and it keeps its A result in shared memory (xacc,
+    // xml) for the merge.  The CTA writes one partial slot of each unit it
+    // touches, c - (first CTA of the unit); the CTA holding a unit's last chunk
+    // also empties the unit's unused slots.
+    int64_t unitA = 0, unitB = 0, s0A = 0, s1A = 0, s0B = 0, s1B = 0;   // token ranges of A and B
+    int64_t cut = INT64_MAX, xw0 = 0, nck = 1;
+    int slotA = 0, slotB = 0, ngrp = 1, nmine = 0, ipart = 0;
+    bool endA = false, endB = false, firstB = false;
+    int aEnd = NW, bBeg = NW;          // merge: warps [0, aEnd) feed unit A, [bBeg, NW) unit B
+    bool aX = false;                   // the crossing warp's unit-A result feeds unit A too
     int64_t Tb = a.seq_lens ? (int64_t)a.seq_lens[blockIdx.z] : a.T;
     Tb = Tb < 0 ? 0 : (Tb > a.Tcap ? a.Tcap : Tb);
     if (a.sk_ctas == 0) {
@@ -124,11 +134,14 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         s0A = (int64_t)blockIdx.x * a.split_tokens;
         s1A = (s0A + a.split_tokens < Tb) ? s0A + a.split_tokens : Tb;
         slotA = blockIdx.x;
+        const int nchunk = s1A > s0A ? (int)((s1A - s0A + C::kChunk - 1) / C::kChunk) : 0;
+        nmine = nchunk > warp ? (nchunk - warp + NW - 1) / NW : 0;
+        ipart = nmine;
     } else {
-        const int64_t N = a.sk_total, nck = a.sk_nck, nC = a.sk_ctas, c = blockIdx.x;
-        const int64_t lo = c * N / nC, hi = (c + 1) * N / nC;
-        const int64_t u0 = lo / nck, u1 = (hi - 1) / nck;
-        const int64_t cut = (u0 + 1) * nck < hi ? (u0 + 1) * nck : hi;
+        const int64_t N = a.sk_total, nC = a.sk_ctas, c = blockIdx.x;
+        nck = a.sk_nck;
+        const int64_t lo = c * N / nC, hi = (c + 1) * N / nC, S = hi - lo;
+        const int64_t u0 = lo / nck, u1 = (hi - 1) / nck, nxt = (u0 + 1) * nck;
         auto tok = [&](int64_t x, int64_t u) {                 // chunk x of unit u as a token bound
             const int64_t t = (x - u * nck) * C::kChunk;
             return t < Tb ? t : Tb;
@@ -136,22 +149,34 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         auto first_cta = [&](int64_t u) { return (int)(((u * nck + 1) * nC - 1) / N); };
         unitA = u0;
         s0A = tok(lo, u0);
-        s1A = tok(cut, u0);
+        s1A = tok(nxt < hi ? nxt : hi, u0);
         slotA = (int)c - first_cta(u0);
-        endA = cut == (u0 + 1) * nck;
+        endA = nxt <= hi;
         if (u1 != u0) {
-            kA = streamk_split<NW>(cut - lo, hi - cut);
             ngrp = 2;
+            cut = nxt;
             unitB = u1;
-            s0B = tok(cut, u1);
+            s0B = tok(nxt, u1);
             s1B = tok(hi, u1);
             slotB = (int)c - first_cta(u1);
             endB = hi == (u1 + 1) * nck;
         }
+        auto wlo = [&](int w) { return lo + (int64_t)w * S / NW; };
+        xw0 = wlo(warp);
+        const int64_t xw1 = wlo(warp + 1);
+        nmine = (int)(xw1 - xw0);
+        firstB = xw0 >= cut;
+        ipart = (xw0 < cut && cut < xw1) ? (int)(cut - xw0) : nmine;
+        if (ngrp == 2)
+            for (int w = 0; w < NW; ++w) {
+                const int64_t a0 = wlo(w), a1 = wlo(w + 1);
+                if (a0 >= cut || cut < a1) {
+                    aEnd = bBeg = w;
+                    aX = a0 < cut;
+                    break;
+                }
+            }
     }
-    const int grp = warp < kA ? 0 : 1;
-    const int wi = grp ? warp - kA : warp;                     // this warp among its group's
-    const int nw = grp ? NW - kA : kA;
     auto unit_rows = [&](int g, int64_t& hb, int& gl, int64_t& sq) {
         const int64_t u = g ? unitB : unitA;
         const int64_t bk = u / hgroups;                          // b * Hkv + kv head
@@ -161,12 +186,10 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         hb = bb * a.Hq + kv * G + 8 * hg;
         sq = bk;
     };
-    int64_t hbase, seq;
-    int Gl;
-    unit_rows(grp, hbase, Gl, seq);
-    const int64_t s0 = grp ? s0B : s0A, s1 = grp ? s1B : s1A;
-    const int nchunk = s1 > s0 ? (int)((s1 - s0 + C::kChunk - 1) / C::kChunk) : 0;
-    const int nmine = nchunk > wi ? (nchunk - wi + nw - 1) / nw : 0;
+    int64_t hbA, seqA, hbB = 0, seqB = 0;
+    int GlA, GlB = 0;
+    unit_rows(0, hbA, GlA, seqA);
+    if (ngrp == 2) unit_rows(1, hbB, GlB, seqB);
     // A paged cache's table entries for the CTA's token ranges go to shared
     // memory first (one coalesced load per CTA), so the per-chunk lookups that
     // feed the bulk copies do not wait on global memory; longer ranges keep the
@@ -177,11 +200,8 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     const bool staged = (a.ktable || a.vtable) && ntabA + ntabB <= kTabMax;
     if (staged) {
         for (int g = 0; g < ngrp; ++g) {
-            int64_t hb_, sq_;
-            int gl_;
-            unit_rows(g, hb_, gl_, sq_);
             const int off = g ? ntabA : 0, n = g ? ntabB : ntabA;
-            const int64_t l0 = g ? lb0B : lb0A;
+            const int64_t l0 = g ? lb0B : lb0A, sq_ = g ? seqB : seqA;
             for (int i = threadIdx.x; i < n; i += NW * 32) {
                 sTab[off + i] = a.ktable ? __ldg(a.ktable + sq_ * a.NB + l0 + i) : 0;
                 sTab[kTabMax + off + i] = a.vtable ? __ldg(a.vtable + sq_ * a.NB + l0 + i) : 0;
@@ -189,29 +209,66 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         }
         __syncthreads();
     }
-    const int64_t lb0 = grp ? lb0B : lb0A;
-    const int toff = grp ? ntabA : 0;
     const int64_t kbb = block_bytes(D, QJL), vbb = block_bytes(D, false);
-
-    if (lane == 0)
+    // Unit descriptors in shared memory, read by the producer lane per chunk,
+    // at the crossing and in the merge (registers stay with the main loop):
+    // per warp and unit group, block-table row of logical block 0, offset of
+    // the staged table slice, first query row, query heads.  CTA-wide merge
+    // facts in sMerge (written by thread 0, read after the next barrier).
+    int64_t* myU = sU + warp * 8;
+    if (lane == 0) {
+        myU[0] = seqA * a.NB;
+        myU[1] = -lb0A;
+        myU[2] = hbA;
+        myU[3] = GlA;
+        myU[4] = seqB * a.NB;
+        myU[5] = ntabA - lb0B;
+        myU[6] = hbB;
+        myU[7] = GlB;
         for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&bars[warp * kStages + s]), 1);
+    }
+    if (threadIdx.x == 0) {
+        sMerge[0] = ngrp; sMerge[1] = aEnd; sMerge[2] = bBeg; sMerge[3] = aX;
+        sMerge[4] = slotA; sMerge[5] = slotB; sMerge[6] = endA; sMerge[7] = endB;
+    }
     fence_mbar_init();
     __syncwarp();
+    // chunk i of this warp is chunk (i < icut ? offA : offB) + i step of its unit
+    int offA, offB = 0, icut, step;
+    if (a.sk_ctas == 0) {
+        offA = (int)(s0A / C::kChunk) + warp;
+        icut = nmine;
+        step = NW;
+    } else {
+        offA = (int)(xw0 - unitA * nck);
+        offB = (int)(xw0 - unitB * nck);
+        icut = firstB ? 0 : ipart;
+        step = 1;
+    }
 
+    // token offset of this warp's chunk i in its unit, and whether the unit is B
+    auto chunk_at = [&](int i, bool& inB) -> int64_t {
+        inB = i >= icut;
+        return (int64_t)((inB ? offB : offA) + i * step) * C::kChunk;
+    };
     // cache blocks (K, V) of this warp's chunk i; a paged cache reads its block table
     auto blocks_of = [&](int i, int64_t& kblk, int64_t& vblk) {
-        const int64_t t0 = s0 + (int64_t)(wi + i * nw) * C::kChunk;
+        bool inB;
+        const int64_t t0 = chunk_at(i, inB);
+        const int64_t* u = myU + (inB ? 4 : 0);
+        const int64_t row = u[0] + (t0 >> 6);
         if (staged) {
-            const int ti = (int)((t0 >> 6) - lb0) + toff;
-            kblk = staged_block(a.ktable, sTab, a.kpool, seq * a.NB + (t0 >> 6), ti, a.err);
-            vblk = staged_block(a.vtable, sTab + kTabMax, a.vpool, seq * a.NB + (t0 >> 6), ti, a.err);
+            const int ti = (int)((t0 >> 6) + u[1]);
+            kblk = staged_block(a.ktable, sTab, a.kpool, row, ti, a.err);
+            vblk = staged_block(a.vtable, sTab + kTabMax, a.vpool, row, ti, a.err);
         } else {
-            kblk = cache_block(a.ktable, a.kpool, a.NB, seq, t0 >> 6, a.err);
-            vblk = cache_block(a.vtable, a.vpool, a.NB, seq, t0 >> 6, a.err);
+            kblk = table_block(a.ktable, a.kpool, row, a.err);
+            vblk = table_block(a.vtable, a.vpool, row, a.err);
         }
     };
     auto issue = [&](int i, int64_t kblk, int64_t vblk) {
-        const int64_t t0 = s0 + (int64_t)(wi + i * nw) * C::kChunk;     // multiple of the chunk
+        bool inB;
+        const int64_t t0 = chunk_at(i, inB);                          // multiple of the chunk
         const int sub = (int)((t0 & 63) / C::kChunk);
         const uint8_t* kb = a.kc + (kblk >= 0 ? kblk : 0) * kbb;    // a bad table entry reads block 0
         const uint8_t* vb = a.vc + (vblk >= 0 ? vblk : 0) * vbb;
@@ -232,7 +289,8 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     };
     // chunks holding tokens that a chained encode writes are fetched only after pdl_wait
     auto fresh = [&](int i) {
-        const int64_t t0 = s0 + (int64_t)(wi + i * nw) * C::kChunk;
+        bool inB;
+        const int64_t t0 = chunk_at(i, inB);
         return t0 < a.fresh_hi && a.fresh_lo < t0 + C::kChunk;
     };
     if (lane == 0) {
@@ -277,28 +335,17 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         r0 = (gr & 1) ? l0 : h0;
         r1 = (gr & 1) ? l1 : h1;
     };
-    uint32_t bq[C::kBRegs ? NT : 1][C::kBRegs ? kKC : 1][2];
-    if constexpr (C::kBRegs) {
+    // The q' fragments of each unit the CTA touches go to sB (group g: unit A
+    // or B), filled by all warps; so do the u' words and factors below.
+    for (int idx = warp; idx < ngrp * kKC; idx += NW) {
+        const int g = idx >= kKC ? 1 : 0, kc = idx - g * kKC;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int kc = 0; kc < kKC; ++kc) b_frag(a.qp, hbase, Gl, nt, kc, bq[nt][kc][0], bq[nt][kc][1]);
-    } else {
-        // q' fragments of each group's unit, in that group's copy of sB
-        for (int idx = warp; idx < ngrp * kKC; idx += NW) {
-            const int g = idx >= kKC ? 1 : 0, kc = idx - g * kKC;
-            int64_t hb_, sq_;
-            int gl_;
-            unit_rows(g, hb_, gl_, sq_);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                uint32_t r0, r1;
-                b_frag(a.qp, hb_, gl_, nt, kc, r0, r1);
-                sB[(size_t)g * kSBGroup + (nt * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
-            }
+        for (int nt = 0; nt < NT; ++nt) {
+            uint32_t r0, r1;
+            b_frag(a.qp, g ? hbB : hbA, g ? GlB : GlA, nt, kc, r0, r1);
+            sB[(size_t)g * kSBGroup + (nt * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
         }
     }
-    [[maybe_unused]] const uint2* sBw = sB + (size_t)grp * kSBGroup;   // this warp's group's operands
     // QJL term on int8 operands.  u' of each head is taken to 16-bit fixed point,
     // u_int = rint(u' kQ / max|u'|), as two signed byte limbs (256 hi + lo): B column
     // n = gr of n-tile nt is head 4 nt + gr / 2, limb gr % 2.  The A operand byte e
@@ -307,21 +354,21 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     // byte e holds u_int of that bit's JL row.  With acc = sum of the products,
     // sum_i u'_i (2 sigma_i - 1) = (max|u'| / kQ) (-acc / 64 - sum_i u_int_i), exact
     // up to the fixed point of u' (the term is scaled by gamma ~ 0.18 of the score).
+    // The words of (unit g, n-tile nt) go to sB, and the factors of head h to
+    // sF[g][0][h] (scale_log2 max|u'| / (64 kQ)) and sF[g][1][h] (64 sum u_int).
     constexpr int kKB = D / 32;
     constexpr float kQ = 32000.f;
-    [[maybe_unused]] uint32_t iu[QJL && C::kBRegs ? NT : 1][QJL && C::kBRegs ? kKB : 1][2];
-    [[maybe_unused]] float fS[NT], uS[NT];   // factors of this lane's own head 4 nt + tq4
     if constexpr (QJL) {
         auto row_of = [&](int kb, int half, int e) {
             const int bit = 8 * e + 7 - 2 * (kb & 3) - half;
             if constexpr (D == 64) return slot_coord(0, tq4, e < 2 ? bit : bit - 20);   // h | h << 20
             return slot_coord(kb >> 2, tq4, bit < 16 ? 2 * bit : 2 * (bit - 16) + 1);
         };
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
+        for (int idx = warp; idx < ngrp * NT; idx += NW) {
+            const int g = idx >= NT ? 1 : 0, nt = idx - g * NT;
             const int hcol = 4 * nt + (gr >> 1);
-            const bool live = hcol < Gl;
-            const float* up = a.up + (hbase + (live ? hcol : 0)) * D;
+            const bool hlive = hcol < (g ? GlB : GlA);
+            const float* up = a.up + ((g ? hbB : hbA) + (hlive ? hcol : 0)) * D;
             float um = 0.f;
 #pragma unroll
             for (int kb = 0; kb < kKB; ++kb)
@@ -331,7 +378,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                     for (int e = 0; e < 4; ++e) um = fmaxf(um, fabsf(up[row_of(kb, hf, e)]));
             um = fmaxf(um, __shfl_xor_sync(kFull, um, 1));
             um = fmaxf(um, __shfl_xor_sync(kFull, um, 2));
-            if (!live) um = 0.f;
+            if (!hlive) um = 0.f;
             const float fu = um > 0.f ? kQ / um : 0.f;
             int usum = 0;
 #pragma unroll
@@ -346,40 +393,105 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                         w[hf] |= (uint32_t)(uint8_t)(int8_t)((gr & 1) ? lo : (ui - lo) >> 8) << (8 * e);
                         usum += ui;
                     }
-                if constexpr (C::kBRegs) {
-                    iu[nt][kb][0] = w[0];
-                    iu[nt][kb][1] = w[1];
-                } else if (wi == 0) {
-                    sB[(size_t)grp * kSBGroup + ((NT + nt) * kKC + kb) * 32 + lane] = make_uint2(w[0], w[1]);
-                }
+                sB[(size_t)g * kSBGroup + ((NT + nt) * kKC + kb) * 32 + lane] = make_uint2(w[0], w[1]);
             }
             usum += __shfl_xor_sync(kFull, usum, 1);
             usum += __shfl_xor_sync(kFull, usum, 2);
-            // this lane's score columns are head 4 nt + tq4, whose factors sit in lane 8 tq4
-            fS[nt] = a.scale_log2 * (__shfl_sync(kFull, um, 8 * tq4) / kQ) * (1.f / 64.f);
-            uS[nt] = 64.f * (float)__shfl_sync(kFull, usum, 8 * tq4);
+            if ((gr & 1) == 0 && tq4 == 0) {
+                sF[(g * 2) * 8 + hcol] = a.scale_log2 * (um / kQ) * (1.f / 64.f);
+                sF[(g * 2 + 1) * 8 + hcol] = 64.f * (float)usum;
+            }
         }
     }
-    if constexpr (!C::kBRegs) __syncthreads();
+    // the crossing warp's unit-A result starts empty (it stays so if a wait fails before the crossing)
+    if (ipart < nmine && lane < 8) {
+        xml[2 * lane] = -INFINITY;
+        xml[2 * lane + 1] = 0.f;
+    }
+    __syncthreads();
     const uint32_t lut[4] = {a.cb.lut_lo[0], a.cb.lut_lo[1], a.cb.lut_hi[0], a.cb.lut_hi[1]};
     const uint32_t* pw = a.cb.pow2;
     [[maybe_unused]] const uint32_t m64 = pw[20] | 1u;    // d = 64 sign widening factor
 
+    // ---------------- this warp's unit: operands and softmax state
+    int64_t hbase = hbA;
+    int Gl = GlA;
+    uint32_t bq[C::kBRegs ? NT : 1][C::kBRegs ? kKC : 1][2];
+    [[maybe_unused]] uint32_t iu[QJL && C::kBRegs ? NT : 1][QJL && C::kBRegs ? kKB : 1][2];
+    [[maybe_unused]] float fS[NT], uS[NT];   // factors of this lane's own head 4 nt + tq4
+    [[maybe_unused]] const uint2* sBw = sB;  // this warp's unit's fragments in sB
     float o[NT][kKC][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int mt = 0; mt < kKC; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
     float mrun[NT], lrun[NT], live[NT];
+    auto load_unit = [&](int g) {
+        hbase = myU[4 * g + 2];
+        Gl = (int)myU[4 * g + 3];
+        sBw = sB + (size_t)g * kSBGroup;
+        if constexpr (C::kBRegs) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        mrun[nt] = -INFINITY;
-        lrun[nt] = 0.f;
-        live[nt] = (4 * nt + tq4 < Gl) ? 1.f : 0.f;   // this lane's head exists
-    }
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int kc = 0; kc < kKC; ++kc) {
+                    const uint2 v = sBw[(nt * kKC + kc) * 32 + lane];
+                    bq[nt][kc][0] = v.x;
+                    bq[nt][kc][1] = v.y;
+                }
+            if constexpr (QJL) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int kb = 0; kb < kKB; ++kb) {
+                        const uint2 v = sBw[((NT + nt) * kKC + kb) * 32 + lane];
+                        iu[nt][kb][0] = v.x;
+                        iu[nt][kb][1] = v.y;
+                    }
+            }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            if constexpr (QJL) {
+                fS[nt] = sF[(g * 2) * 8 + 4 * nt + tq4];
+                uS[nt] = sF[(g * 2 + 1) * 8 + 4 * nt + tq4];
+            }
+            live[nt] = (4 * nt + tq4 < Gl) ? 1.f : 0.f;   // this lane's head exists
+            mrun[nt] = -INFINITY;
+            lrun[nt] = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < kKC; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+        }
+    };
+    // softmax sums over the lanes of a head, then the result of the unit in
+    // hand: accumulators to acc_dst [8][D] (if write_acc), (max, sum) of every
+    // head this lane serves to ml_dst [8][2] (max -inf where the head is absent)
+    auto finish_unit = [&](bool failed_, float* acc_dst, float* ml_dst, bool write_acc) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            if (failed_) { mrun[nt] = -INFINITY; lrun[nt] = 0.f; }
+            lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 4);
+            lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 8);
+            lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 16);
+            const int h = 4 * nt + tq4;
+            const bool hl = h < Gl;
+            if (hl && write_acc) {
+#pragma unroll
+                for (int mt = 0; mt < kKC; ++mt) {
+                    acc_dst[h * D + 16 * mt + gr] = o[nt][mt][0] + o[nt][mt][1];
+                    acc_dst[h * D + 16 * mt + 8 + gr] = o[nt][mt][2] + o[nt][mt][3];
+                }
+            }
+            if (gr == 0) {
+                ml_dst[h * 2] = hl ? mrun[nt] : -INFINITY;
+                ml_dst[h * 2 + 1] = hl ? lrun[nt] : 0.f;
+            }
+        }
+    };
+    load_unit(firstB ? 1 : 0);
     bool failed = false, drained = true;
 
     for (int i = 0; i < nmine; ++i) {
+        if (i == ipart) {                     // this warp crosses from unit A to unit B
+            finish_unit(false, xacc, xml, true);
+            load_unit(1);
+        }
         const uint32_t bar = smem_u32(&bars[warp * kStages + (i % kStages)]);
         const bool ok = mbar_wait_bounded(bar, (uint32_t)((i / kStages) & 1), i == 0 ? a.first_wait : kWaitLimit);
         if (__any_sync(kFull, !ok)) {         // warp-uniform: no lane may run on alone into mma.sync
@@ -393,11 +505,12 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
             break;
         }
         const uint8_t* st = ring + (i % kStages) * C::kStageB;
-        const int64_t tok0 = s0 + (int64_t)(wi + i * nw) * C::kChunk;
-        const int nvalid = (int)((s1 - tok0) < C::kChunk ? (s1 - tok0) : C::kChunk);
+        bool inB_;
+        const int64_t tok0 = chunk_at(i, inB_);
+        const int nvalid = (int)((Tb - tok0) < C::kChunk ? (Tb - tok0) : C::kChunk);
 
         // one 16-token tile; PARTIAL masks tokens beyond nvalid (only the last
-        // chunk of a split can be partial)
+        // chunk of a sequence can be partial)
         auto tile = [&](const int kt, auto partial_tag) {
             constexpr bool PARTIAL = decltype(partial_tag)::value;
             const int tA = kt * 16 + gr, tB = tA + 8;            // this lane's two tokens
@@ -542,47 +655,23 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
             if (i + kStages + 1 < nmine) blocks_of(i + kStages + 1, next_k, next_v);
         }
     }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        if (failed) { mrun[nt] = -INFINITY; lrun[nt] = 0.f; }
-        lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 4);
-        lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 8);
-        lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 16);
-    }
-
     pdl_trigger();                        // the combine kernel may start launching
-    // ---------------- merge the warps of the CTA into one partial per head.  Each
-    // warp's (max, sum) go to sML; its accumulators to its own ring, unless a
-    // failed wait left copies of unknown state there (then the warp is skipped:
-    // its max is -inf and its accumulators are never read).
+    // ---------------- merge the warps of the CTA into one partial per unit and
+    // head.  Each warp's (max, sum) go to sML; its accumulators to its own
+    // ring, unless a failed wait left copies of unknown state there (then the
+    // warp is skipped: its max is -inf and its accumulators are never read).
     __syncwarp();
-    float* wbuf = reinterpret_cast<float*>(ring);             // [Gl][D], in this warp's own ring
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int h = 4 * nt + tq4;
-        if (h < Gl) {
-            if (drained) {
-#pragma unroll
-                for (int mt = 0; mt < kKC; ++mt) {
-                    wbuf[h * D + 16 * mt + gr] = o[nt][mt][0] + o[nt][mt][1];
-                    wbuf[h * D + 16 * mt + 8 + gr] = o[nt][mt][2] + o[nt][mt][3];
-                }
-            }
-            if (gr == 0) {
-                sML[(warp * 8 + h) * 2] = mrun[nt];
-                sML[(warp * 8 + h) * 2 + 1] = lrun[nt];
-            }
-        }
-    }
+    finish_unit(failed, reinterpret_cast<float*>(ring), sML + warp * 16, drained);
     __syncthreads();
-    for (int g = 0; g < ngrp; ++g) {
-        int64_t hb_, sq_;
-        int gl_;
-        unit_rows(g, hb_, gl_, sq_);
-        const int w0 = g ? kA : 0, w1 = g ? NW : kA;
+    const int ngrp_ = sMerge[0];
+    for (int g = 0; g < ngrp_; ++g) {
+        const int64_t hb_ = myU[4 * g + 2];
+        const int gl_ = (int)myU[4 * g + 3];
+        const int w0 = g ? sMerge[2] : 0, w1 = g ? NW : sMerge[1];
+        const bool withx = g == 0 && sMerge[3];                  // the crossing warp's unit-A result
         for (int idx = threadIdx.x; idx < gl_ * D; idx += NW * 32) {
             const int h = idx / D, j = idx % D;
-            float M = -INFINITY;
+            float M = withx ? xml[2 * h] : -INFINITY;
             for (int w = w0; w < w1; ++w) M = fmaxf(M, sML[(w * 8 + h) * 2]);
             float L = 0.f, A = 0.f;
             if (M != -INFINITY) {
@@ -594,8 +683,13 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                     L = fmaf(f, sML[(w * 8 + h) * 2 + 1], L);
                     A = fmaf(f, wb[j], A);
                 }
+                if (withx && xml[2 * h] != -INFINITY) {
+                    const float f = exp2f(xml[2 * h] - M);
+                    L = fmaf(f, xml[2 * h + 1], L);
+                    A = fmaf(f, xacc[h * D + j], A);
+                }
             }
-            const int slot = g ? slotB : slotA;
+            const int slot = sMerge[4 + g];
             const int64_t pidx = (hb_ + h) * a.nsplit + slot;
             a.part_acc[pidx * D + j] = A;
             if (j == 0) {
@@ -603,7 +697,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                 a.part_ml[2 * pidx + 1] = L;
             }
             // the CTA holding the unit's last chunk empties the unit's unused slots
-            if (g ? endB : endA)
+            if (sMerge[6 + g])
                 for (int sp = slot + 1; sp < a.nsplit; ++sp) {
                     const int64_t e = (hb_ + h) * a.nsplit + sp;
                     a.part_acc[e * D + j] = 0.f;
@@ -626,7 +720,8 @@ cudaError_t launch_mma_t(const DecArgs& a, int G, cudaStream_t s) {
     using C = Cfg<D, QJL>;
     const size_t smem = (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
                         (size_t)NW * 8 * 2 * sizeof(float) + 2 * kTabMax * sizeof(int32_t) +
-                        (C::kBRegs ? 0 : (size_t)2 * 2 * NT * C::kKC * 32 * sizeof(uint2));
+                        (size_t)2 * 2 * NT * C::kKC * 32 * sizeof(uint2) + (2 * 2 * 8 + 8 * D + 8 * 2) * sizeof(float) +
+                        (size_t)NW * 8 * sizeof(int64_t) + 8 * sizeof(int);
     auto kern = tq_decode_mma_kernel<D, NT, NW, QJL>;
     cudaError_t e = set_smem_once<tq_decode_mma_kernel<D, NT, NW, QJL>>((int)smem);
     if (e != cudaSuccess) return e;
