@@ -43,8 +43,8 @@ ENCODE_BYTES_PER_VECTOR = {("k", 128): 68, ("v", 128): 50}
 # DRAM traffic of the split-K kernel (read + write bytes per launch) from one
 # ncu capture, valid only while the kernel sources are unchanged (sha256 over
 # DECODE_SOURCES at capture time).
-NCU_TRAFFIC = {"source_sha256": "450a46948ff11fe5206caa997eed3f1119bc86c5f4a417dd2f0d4f08baa4c620",
-               "bytes_per_launch": 386805504 + 4402944,
+NCU_TRAFFIC = {"source_sha256": "9dea2855e972859fe222f09c7b134fb799e12bb9fe07c2dd9a6fc472589762ae",
+               "bytes_per_launch": 387275520 + 3267840,
                "capture": "profiles/tq_decode_mma_d128_long_context_b4_hq16_hkv8_t102400.md"}
 
 
