@@ -48,6 +48,8 @@ constexpr int kRXBuf = 3;                 // input tile buffers
 constexpr int kRTile = kRRows * kRD * 2;  // one 16-bit 128 x 128 operand (32 KB)
 constexpr int64_t kRotMinVectors = 16384; // smaller encodes keep the per-lane kernels
 constexpr float kRScale = 4096.f;         // residual scale before the fp16 split
+// 3.5 (1 + 16 + 256 + 4096): the offset of four nibbles whose codes are held as code - 3.5
+constexpr float kNib35 = 15291.5f;
 
 template <bool IS_K>
 struct RotShape {
@@ -58,7 +60,10 @@ struct RotShape {
     // exchange between the four threads of a vector: ||Y||^2 and gamma^2 parts [4][128],
     // code words of chunks 0-2 and bit-3 planes of chunk 3 [12][128] each
     static constexpr int kOffXchg = kOffBar + 16 * 8;
-    static constexpr int kOffMisc = kOffXchg + (4 * 128 + 4 * 128 + 12 * 128 + 12 * 128) * 4;
+    // K: address of each vector's sign words, per tile parity [2][128] (written with the
+    // record, used for the projection's signs one tile later)
+    static constexpr int kOffSgn = kOffXchg + (4 * 128 + 4 * 128 + 12 * 128 + 12 * 128) * 4;
+    static constexpr int kOffMisc = kOffSgn + (IS_K ? 2 * 128 * 8 : 0);
     static constexpr int kSmem = kOffMisc + 16 + 1024;           // + slack to align the base
     static constexpr int kCols = IS_K ? 512 : 256;               // Y/R x 2 (+ Z x 2)
 };
@@ -256,6 +261,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         float* xg = xss + 4 * 128;                                           // [4][128]
         uint32_t* xw = reinterpret_cast<uint32_t*>(xg + 4 * 128);            // [12][128]
         uint32_t* xp = xw + 12 * 128;                                        // [12][128]
+        [[maybe_unused]] uint8_t** sgn_at = reinterpret_cast<uint8_t**>(sm + S::kOffSgn);   // K: [2][128]
         const Codebook& cb = a.cb;
         // Bucket index and centroid on the FMA pipe.  The codebook is antisymmetric
         // (b3 = 0, b[6-k] = -b[k], c[7-k] = -c[k]), so with a = |y| and
@@ -280,19 +286,16 @@ __global__ void __launch_bounds__(kRThreads, 1)
             tc_fence_after();
             uint32_t z[32];
             tc_ld32(tl + 256u + (uint32_t)(128 * (jj & 1) + 32 * cq), z);
+            // the sign bits of z[31] .. z[0] shifted in one by one (one funnel shift each),
+            // then inverted: bit b = 1 when z[b] >= 0 (a z of -0 would give 0; the
+            // accumulation never yields one for a nonzero vector)
             uint32_t word = 0;
 #pragma unroll
-            for (int bt = 0; bt < 32; ++bt) word |= (__uint_as_float(z[bt]) >= 0.f ? 1u : 0u) << bt;
+            for (int bt = 31; bt >= 0; --bt) word = __funnelshift_l(z[bt], word, 1);
+            word = ~word;
             if (!nz_prev) word = 0xFFFFFFFFu;                // zero vector: z = 0, every sign bit 1
-            const int64_t gv = row0_of(jj) + r;
-            if (gv < N) {
-                int64_t xoff;
-                uint8_t* blk;
-                int tau;
-                encode_locate(a, (uint32_t)gv, bb, xoff, blk, tau);
-                if (blk)
-                    *reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(kRD) + tau * sign_bytes(kRD) + 4 * cq) = word;
-            }
+            uint8_t* sp = sgn_at[(jj & 1) * 128 + r];            // null: no record to write
+            if (sp) *reinterpret_cast<uint32_t*>(sp + 4 * cq) = word;
             return true;
         };
         for (int j = 0; j < n; ++j) {
@@ -345,8 +348,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
                         const float t5 = __saturatef(fmaf(av, kneg, bb5));
                         const float t6 = __saturatef(fmaf(av, kneg, bb6));
                         const float T = (t4 + t5) + t6;
-                        // 7 - T above zero, T below: 3.5 +- (3.5 - T)
-                        cf[e + f] = 3.5f + __uint_as_float(__float_as_uint(3.5f - T) ^ sgn);
+                        // 7 - T above zero, T below: 3.5 +- (3.5 - T); the 3.5 of all four
+                        // nibbles is added once in the sum below (kNib35)
+                        cf[e + f] = __uint_as_float(__float_as_uint(3.5f - T) ^ sgn);
                         if constexpr (IS_K) {
                             float m = fmaf(-t6, d3, c7);                // |c| 2^12
                             m = fmaf(-t5, d2, m);
@@ -365,7 +369,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
                     // four nibbles as an exact float sum, read out of the mantissa (x + 2^23)
-                    const float part = fmaf(cf[2 * t + 9], 4096.f, fmaf(cf[2 * t + 8], 256.f, fmaf(cf[2 * t + 1], 16.f, cf[2 * t])));
+                    const float part = fmaf(cf[2 * t + 9], 4096.f,
+                                            fmaf(cf[2 * t + 8], 256.f, fmaf(cf[2 * t + 1], 16.f, cf[2 * t] + kNib35)));
                     const uint32_t bits = __float_as_uint(part + 8388608.f);
                     W[t] = h2 == 0 ? bits : __byte_perm(W[t], bits, 0x5410);
                 }
@@ -384,11 +389,13 @@ __global__ void __launch_bounds__(kRThreads, 1)
             }
             xg[cq * 128 + r] = g2;
             named_bar_r(1, kRQuant);
-            if (cq == 0 && gv < N) {
+            if (cq == 0) {
                 int64_t xoff;
-                uint8_t* blk;
-                int tau;
-                encode_locate(a, (uint32_t)gv, bb, xoff, blk, tau);
+                uint8_t* blk = nullptr;
+                int tau = 0;
+                if (gv < N) encode_locate(a, (uint32_t)gv, bb, xoff, blk, tau);
+                if constexpr (IS_K)
+                    sgn_at[(j & 1) * 128 + r] = blk ? blk + kBlockT * code_bytes(kRD) + tau * sign_bytes(kRD) : nullptr;
                 if (blk) {
                     uint32_t wd[12];
 #pragma unroll
@@ -608,25 +615,23 @@ __global__ void __launch_bounds__(k6Threads, 2)
                                      d1 = (cb.c[5] - cb.c[4]) * kRScale, c7 = cb.c[7] * kRScale;
         bool failed = false;
         [[maybe_unused]] bool nz_prev = true;                // the previous tile's vector is nonzero
+        // K: address of the sign words of this thread's vector in the previous tile (null: none)
+        [[maybe_unused]] uint8_t* sgn_prev = nullptr;
         // sign word hv of tile jj (K): bit b is z[32 hv + b] >= 0
         auto signs = [&](int jj) -> bool {
             if (!warp_wait_r(bar(kRBarZFull + (jj & 1)), (uint32_t)((jj >> 1) & 1))) return false;
             tc_fence_after();
             uint32_t z[32];
             tc_ld32(tl + 128u + (uint32_t)(64 * (jj & 1) + 32 * hv), z);
+            // the sign bits of z[31] .. z[0] shifted in one by one (one funnel shift each),
+            // then inverted: bit b = 1 when z[b] >= 0 (a z of -0 would give 0; the
+            // accumulation never yields one for a nonzero vector)
             uint32_t word = 0;
 #pragma unroll
-            for (int bt = 0; bt < 32; ++bt) word |= (__uint_as_float(z[bt]) >= 0.f ? 1u : 0u) << bt;
+            for (int bt = 31; bt >= 0; --bt) word = __funnelshift_l(z[bt], word, 1);
+            word = ~word;
             if (!nz_prev) word = 0xFFFFFFFFu;                // zero vector: z = 0, every sign bit 1
-            const int64_t gv = row0_of(jj) + r;
-            if (gv < N) {
-                int64_t xoff;
-                uint8_t* blk;
-                int tau;
-                encode_locate(a, (uint32_t)gv, bb, xoff, blk, tau);
-                if (blk)
-                    *reinterpret_cast<uint32_t*>(blk + kBlockT * code_bytes(k6D) + tau * sign_bytes(k6D) + 4 * hv) = word;
-            }
+            if (sgn_prev) *reinterpret_cast<uint32_t*>(sgn_prev + 4 * hv) = word;
             return true;
         };
         for (int j = 0; j < n; ++j) {
@@ -674,7 +679,7 @@ __global__ void __launch_bounds__(k6Threads, 2)
                         const float t5 = __saturatef(fmaf(av, kneg, bb5));
                         const float t6 = __saturatef(fmaf(av, kneg, bb6));
                         const float T = (t4 + t5) + t6;
-                        cf[e + f] = 3.5f + __uint_as_float(__float_as_uint(3.5f - T) ^ sgn);
+                        cf[e + f] = __uint_as_float(__float_as_uint(3.5f - T) ^ sgn);   // code - 3.5
                         if constexpr (IS_K) {
                             float m = fmaf(-t6, d3, c7);
                             m = fmaf(-t5, d2, m);
@@ -691,10 +696,10 @@ __global__ void __launch_bounds__(k6Threads, 2)
                     tc_st8(yb + (uint32_t)(16 * h2 + 8), rl);
                 }
                 // nibble sums as exact floats, read out of the mantissa (x + 2^23)
-                const float n0 = fmaf(cf[3], 4096.f, fmaf(cf[2], 256.f, fmaf(cf[1], 16.f, cf[0])));
-                const float n1 = fmaf(cf[7], 4096.f, fmaf(cf[6], 256.f, fmaf(cf[5], 16.f, cf[4])));
-                const float n2 = fmaf(cf[11], 4096.f, fmaf(cf[10], 256.f, fmaf(cf[9], 16.f, cf[8])));
-                const float n3 = fmaf(cf[15], 4096.f, fmaf(cf[14], 256.f, fmaf(cf[13], 16.f, cf[12])));
+                const float n0 = fmaf(cf[3], 4096.f, fmaf(cf[2], 256.f, fmaf(cf[1], 16.f, cf[0] + kNib35)));
+                const float n1 = fmaf(cf[7], 4096.f, fmaf(cf[6], 256.f, fmaf(cf[5], 16.f, cf[4] + kNib35)));
+                const float n2 = fmaf(cf[11], 4096.f, fmaf(cf[10], 256.f, fmaf(cf[9], 16.f, cf[8] + kNib35)));
+                const float n3 = fmaf(cf[15], 4096.f, fmaf(cf[14], 256.f, fmaf(cf[13], 16.f, cf[12] + kNib35)));
                 const uint32_t na = __byte_perm(__float_as_uint(n0 + 8388608.f), __float_as_uint(n1 + 8388608.f), 0x5410);
                 const uint32_t nb = __float_as_uint(n2 + 8388608.f) & 0xFFFFu;
                 const uint32_t nc = __float_as_uint(n3 + 8388608.f) & 0xFFFFu;
@@ -731,6 +736,7 @@ __global__ void __launch_bounds__(k6Threads, 2)
                         __float2half_rn(nz ? sqrtf(gs) * (1.f / kRScale) : 0.f);     // a zero vector has no residual
                 }
                 if (j >= 1 && !signs(j - 1)) failed = true;      // acted on at the next exchange
+                sgn_prev = blk ? blk + kBlockT * code_bytes(k6D) + tau * sign_bytes(k6D) : nullptr;
                 nz_prev = nz;
             }
         }
