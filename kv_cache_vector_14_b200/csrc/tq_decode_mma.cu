@@ -27,8 +27,9 @@
 //
 // Data movement: each warp owns a ring of STAGES shared-memory buffers of a
 // chunk of tokens (32 at d = 128, 16 at d = 256; K codes, signs, norms,
-// gammas, V codes, norms: six bulk copies, cp.async.bulk with an mbarrier
-// transaction count, no multicast).  Waits are bounded: on timeout the kernel
+// gammas, V codes, norms: six bulk copies issued by six lanes at once,
+// cp.async.bulk with an mbarrier transaction count, no multicast).  Waits are
+// bounded: on timeout the kernel
 // sets the handle's check word, waits (bounded) for its own copies, and
 // contributes an empty partial.
 //
@@ -266,6 +267,28 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
             vblk = table_block(a.vtable, a.vpool, row, a.err);
         }
     };
+    // A stage is six bulk copies (four without the QJL bit): K codes, K signs, K
+    // norms, gammas, V codes, V norms of one chunk.  Lane k issues copy k, so a
+    // stage costs the warp one copy instruction rather than six in a row: its
+    // source offset in the K or V block for sub-chunk 0, the step per sub-chunk,
+    // its place in the stage and its size.
+    constexpr int kCopies = QJL ? 6 : 4;
+    int cp_off = 0, cp_step = 0, cp_dst = 0, cp_size = 0;
+    bool cp_v = false;
+    {
+        constexpr int cb = C::kCodeB, sb = C::kSignB, ch = C::kChunk;
+        const int k = QJL ? lane : (lane == 0 ? 0 : lane == 1 ? 2 : lane + 2);   // without QJL: 0, 2, 4, 5
+        switch (k) {
+            case 0: cp_off = 0; cp_step = ch * cb; cp_dst = C::kOffKc; cp_size = ch * cb; break;
+            case 1: cp_off = 64 * cb; cp_step = ch * sb; cp_dst = C::kOffKs; cp_size = ch * sb; break;
+            case 2: cp_off = QJL ? 64 * (cb + sb) : 64 * cb; cp_step = 2 * ch; cp_dst = C::kOffKn; cp_size = 2 * ch; break;
+            case 3: cp_off = 64 * (cb + sb) + 128; cp_step = 2 * ch; cp_dst = C::kOffKg; cp_size = 2 * ch; break;
+            case 4: cp_off = 0; cp_step = ch * cb; cp_dst = C::kOffVc; cp_size = ch * cb; cp_v = true; break;
+            case 5: cp_off = 64 * cb; cp_step = 2 * ch; cp_dst = C::kOffVn; cp_size = 2 * ch; cp_v = true; break;
+            default: break;
+        }
+    }
+    // every lane of the warp: lane 0 arms the stage's barrier, then lanes 0 .. kCopies - 1 copy
     auto issue = [&](int i, int64_t kblk, int64_t vblk) {
         bool inB;
         const int64_t t0 = chunk_at(i, inB);                          // multiple of the chunk
@@ -274,18 +297,10 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         const uint8_t* vb = a.vc + (vblk >= 0 ? vblk : 0) * vbb;
         uint8_t* st = ring + (i % kStages) * C::kStageB;
         const uint32_t bar = smem_u32(&bars[warp * kStages + (i % kStages)]);
-        constexpr int cb = C::kCodeB, sb = C::kSignB, ch = C::kChunk;
-        mbar_expect_tx(bar, C::kStageB);
-        bulk_g2s(smem_u32(st + C::kOffKc), kb + sub * ch * cb, ch * cb, bar);
-        if constexpr (QJL) {
-            bulk_g2s(smem_u32(st + C::kOffKs), kb + 64 * cb + sub * ch * sb, ch * sb, bar);
-            bulk_g2s(smem_u32(st + C::kOffKn), kb + 64 * (cb + sb) + sub * 2 * ch, 2 * ch, bar);
-            bulk_g2s(smem_u32(st + C::kOffKg), kb + 64 * (cb + sb) + 128 + sub * 2 * ch, 2 * ch, bar);
-        } else {
-            bulk_g2s(smem_u32(st + C::kOffKn), kb + 64 * cb + sub * 2 * ch, 2 * ch, bar);
-        }
-        bulk_g2s(smem_u32(st + C::kOffVc), vb + sub * ch * cb, ch * cb, bar);
-        bulk_g2s(smem_u32(st + C::kOffVn), vb + 64 * cb + sub * 2 * ch, 2 * ch, bar);
+        if (lane == 0) mbar_expect_tx(bar, C::kStageB);
+        __syncwarp();
+        if (lane < kCopies)
+            bulk_g2s(smem_u32(st + cp_dst), (cp_v ? vb : kb) + cp_off + sub * cp_step, (uint32_t)cp_size, bar);
     };
     // chunks holding tokens that a chained encode writes are fetched only after pdl_wait
     auto fresh = [&](int i) {
@@ -293,16 +308,14 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         const int64_t t0 = chunk_at(i, inB);
         return t0 < a.fresh_hi && a.fresh_lo < t0 + C::kChunk;
     };
-    if (lane == 0) {
-        for (int i = 0; i < kStages && i < nmine; ++i)
-            if (!fresh(i)) {
-                int64_t kb_, vb_;
-                blocks_of(i, kb_, vb_);
-                issue(i, kb_, vb_);
-            }
-    }
+    for (int i = 0; i < kStages && i < nmine; ++i)      // warp-uniform
+        if (!fresh(i)) {
+            int64_t kb_, vb_;
+            blocks_of(i, kb_, vb_);
+            issue(i, kb_, vb_);
+        }
     pdl_wait();                           // q' and u' come from the prologue kernel
-    if (lane == 0) {
+    {
         bool any = false;
         for (int i = 0; i < kStages && i < nmine; ++i) any |= fresh(i);
         if (any) {
@@ -318,7 +331,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     // blocks of the next chunk to issue, looked up one chunk ahead so that a
     // block-table load overlaps a chunk of work
     int64_t next_k = 0, next_v = 0;
-    if (lane == 0 && kStages < nmine) blocks_of(kStages, next_k, next_v);
+    if (kStages < nmine) blocks_of(kStages, next_k, next_v);
 
     // B-operand fragment of k-step kc: column n = gr of n-tile nt is head
     // 4 nt + gr / 2, limb gr % 2; rows 16 kc + 2 tq4 (+1), +8 (+9)
@@ -649,7 +662,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
             if (C::kTiles > 1 && nvalid > 16) tile(1, std::true_type{});
         }
         __syncwarp();
-        if (lane == 0 && i + kStages < nmine) {
+        if (i + kStages < nmine) {            // warp-uniform
             fence_proxy_async();
             issue(i + kStages, next_k, next_v);
             if (i + kStages + 1 < nmine) blocks_of(i + kStages + 1, next_k, next_v);
