@@ -43,8 +43,8 @@ ENCODE_BYTES_PER_VECTOR = {("k", 128): 68, ("v", 128): 50}
 # DRAM traffic of the split-K kernel (read + write bytes per launch) from one
 # ncu capture, valid only while the kernel sources are unchanged (sha256 over
 # DECODE_SOURCES at capture time).
-NCU_TRAFFIC = {"source_sha256": "9dea2855e972859fe222f09c7b134fb799e12bb9fe07c2dd9a6fc472589762ae",
-               "bytes_per_launch": 387275520 + 3267840,
+NCU_TRAFFIC = {"source_sha256": "6da3cad98699ac616c052b36e1404f6bf38b4db37cc10f60268107e9b23e1e95",
+               "bytes_per_launch": 387273472 + 3273984,
                "capture": "profiles/tq_decode_mma_d128_long_context_b4_hq16_hkv8_t102400.md"}
 
 
@@ -847,15 +847,29 @@ def run_ours(args, rank: int, world: int, dist):
                               "decode_path": path}), flush=True)
         return
 
-    # ---- end to end: pinned host inputs copied in, the output read back, every step
-    kh = k_new.cpu().pin_memory()
-    vh = v_new.cpu().pin_memory()
-    qh = q.cpu().pin_memory()
+    # ---- end to end: pinned host inputs copied in, the output read back, every step.
+    # The step's new K, V and query sit in one pinned host buffer and go to the
+    # device in one copy (one transfer instead of three on the step's stream).
+    parts = [k_new.contiguous(), v_new.contiguous(), q.contiguous()]
+    offs, off = [], 0
+    for t_ in parts:
+        offs.append(off)
+        off += (t_.numel() * t_.element_size() + 255) // 256 * 256
+    hbuf = torch.empty(off, dtype=torch.uint8).pin_memory()
+    dbuf = torch.empty(off, dtype=torch.uint8, device=dev)
+    views_h, views_d = [], []
+    for t_, o_ in zip(parts, offs):
+        nb = t_.numel() * t_.element_size()
+        views_h.append(hbuf[o_:o_ + nb].view(t_.dtype).view(t_.shape))
+        views_d.append(dbuf[o_:o_ + nb].view(t_.dtype).view(t_.shape))
+    for vh_, t_ in zip(views_h, parts):
+        vh_.copy_(t_.cpu())
+    kh, vh, qh = views_h
+    kd, vd, qd = views_d
     oh = torch.empty_like(out, device="cpu").pin_memory()
-    kd, vd, qd = torch.empty_like(k_new), torch.empty_like(v_new), torch.empty_like(q)
     n_e2e = max(1, min(args.steps, 2000))
     for _ in range(3):
-        kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True); qd.copy_(qh, non_blocking=True)
+        dbuf.copy_(hbuf, non_blocking=True)
         step(kd, vd, qd, out)
         oh.copy_(out, non_blocking=True)
     torch.cuda.synchronize()
@@ -863,7 +877,7 @@ def run_ours(args, rank: int, world: int, dist):
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2.record()
     for _ in range(n_e2e):
-        kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True); qd.copy_(qh, non_blocking=True)
+        dbuf.copy_(hbuf, non_blocking=True)
         step(kd, vd, qd, out)
         oh.copy_(out, non_blocking=True)
     e3.record()
@@ -871,7 +885,7 @@ def run_ours(args, rank: int, world: int, dist):
     ms_e2e_local = e2.elapsed_time(e3) / n_e2e
     ms_e2e = max_over_ranks(ms_e2e_local, dist, dev)
     e2e_value = whole_job_rate(bytes_step, ms_e2e_local * 1e-3, world, dist, dev) / 1e9
-    h2d = (kh.numel() + vh.numel()) * 4 + qh.numel() * 2
+    h2d = hbuf.numel()                  # the one packed copy (K and V fp32, q bf16, 256-byte aligned parts)
     d2h = oh.numel() * 4
 
     tq.tq_attend_decode(h, q, kc, vc, out, ws, T=T, scale=w.scale)     # QJL output for the quality check
