@@ -16,8 +16,10 @@ bool dtype_ok(int dt) { return dt == TQ_F32 || dt == TQ_BF16 || dt == TQ_F16; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Split count for decode.  Work is `pairs` sequences of nchunk chunks; a CTA
-// handles `per` consecutive chunks spread over its warps, so its time is
-// ceil(per / warps) chunk-steps and the kernel's time is waves * that.  The
+// handles `per` consecutive chunks spread over its warps.  Its warps share one
+// SM and interleave, so its time follows the SM's work, per / warps chunk-steps
+// (at least one: a warp's own chunk is the shortest time), and the kernel's
+// time is waves * that.  The
 // count maximising ideal / actual time wins (ties: fewer partials).  The loop
 // bound is also the workspace's upper bound (split_upper_bound).
 int64_t split_loop_bound(int64_t cap, int64_t pairs, int64_t nchunk) {
@@ -29,6 +31,11 @@ int64_t split_loop_bound(int64_t cap, int64_t pairs, int64_t nchunk) {
 // A CTA also pays a fixed cost (constants, barrier set-up, the merge of its
 // warps, the partial it writes), about kSetup chunk-steps per warp.
 constexpr double kSetup = 2.0;
+// chunk-steps of a CTA with `chunks` chunks over `warps` warps (see above)
+double chunk_steps(int64_t chunks, int warps) {
+    const double t = (double)chunks / warps;
+    return t > 1.0 ? t : 1.0;
+}
 
 int choose_nsplit(int64_t cap, int warps, int64_t pairs, int64_t nchunk, double* steps = nullptr) {
     const int64_t hi = split_loop_bound(cap, pairs, nchunk);
@@ -40,7 +47,7 @@ int choose_nsplit(int64_t cap, int warps, int64_t pairs, int64_t nchunk, double*
         const int64_t used = (nchunk + per - 1) / per;
         if (used != ns) continue;
         const int64_t waves = (pairs * used + cap - 1) / cap;
-        const double t = (double)waves * ((double)((per + warps - 1) / warps) + kSetup);
+        const double t = (double)waves * (chunk_steps(per, warps) + kSetup);
         const double eff = ideal / t;
         if (eff > best_eff + 1e-12) { best_eff = eff; best = ns; if (steps) *steps = t; }
     }
@@ -51,7 +58,7 @@ int choose_nsplit(int64_t cap, int warps, int64_t pairs, int64_t nchunk, double*
 // units' chunks laid end to end (units x nck in all), and each warp a
 // contiguous run of its CTA's share.  With nC >= units a share spans at most
 // two units, so at most one warp per CTA crosses into the next unit (it pays
-// about half a chunk-step to switch).  Returns the modelled chunk-steps of the
+// a tenth of a chunk-step or so to switch).  Returns the modelled chunk-steps of the
 // slowest CTA (plus the fixed cost) and the partial slots a unit needs (the
 // CTAs that overlap it), or -1 when the shape does not fit.
 double streamk_plan(int64_t cap, int warps, int64_t units, int64_t nck, int64_t* nC_out, int* slots_out) {
@@ -63,7 +70,7 @@ double streamk_plan(int64_t cap, int warps, int64_t units, int64_t nck, int64_t*
         const int64_t lo = c * N / nC, hi = (c + 1) * N / nC;
         const int64_t u0 = lo / nck, u1 = (hi - 1) / nck;
         if (hi <= lo || u1 - u0 > 1) return -1.0;
-        const double t = (double)((hi - lo + warps - 1) / warps) + (u1 != u0 ? 0.5 : 0.0);
+        const double t = chunk_steps(hi - lo, warps) + (u1 != u0 ? 0.1 : 0.0);
         worst = t > worst ? t : worst;
     }
     int64_t slots = 0;
@@ -73,7 +80,10 @@ double streamk_plan(int64_t cap, int warps, int64_t units, int64_t nck, int64_t*
     }
     *nC_out = nC;
     *slots_out = (int)slots;
-    return worst + kSetup;
+    // a stream-K CTA's set-up is longer (its share's bounds and the slots of two
+    // units): ~0.6 chunk-steps more, measured on the GQA, long-context and
+    // append-and-attend workloads against their uniform grids
+    return worst + kSetup + 0.6;
 }
 
 struct DecodePlan {
