@@ -739,6 +739,41 @@ def test_streamk_partition_matches_split_and_oracle(handles, prms, d, G, paged):
     assert tq.tq_device_status(h) == tq.TQ_OK
 
 
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_streamk_polar_only_k(handles, prms, d):
+    """PolarQuant-only K (no QJL bit) on the stream-K grid against the uniform
+    grid (1e-5) and the oracle with gamma = 0, sequences of one length with a
+    ragged tail, two query heads per kv head."""
+    h = handles[d]
+    B, Hkv, G, T, Tcap = 2, 5, 2, 2501, 2560
+    Hq = Hkv * G
+    xk = torch_input(synthetic.gaussian((B, Hkv, Tcap, d), seed=81 + d), "bf16")
+    xv = torch_input(synthetic.gaussian((B, Hkv, Tcap, d), seed=82 + d), "bf16")
+    kc, vc = tq.Cache(d, False, B, Hkv, Tcap), tq.Cache(d, False, B, Hkv, Tcap)
+    tq.tq_encode_v(h, xk, kc, 0)
+    tq.tq_encode_v(h, xv, vc, 0)
+    q = synthetic.gaussian((B, Hq, d), seed=83)
+    ws = torch.empty(tq.tq_attend_workspace_bytes(h, B, Hq, Hkv, Tcap), dtype=torch.uint8, device="cuda")
+    scale = 1.0 / np.sqrt(d)
+    outs = {}
+    try:
+        for path in ("split", "streamk"):
+            tq.tq_set_decode_path(h, path)
+            out = torch.full((B, Hq, d), float("nan"), dtype=torch.float32, device="cuda")
+            tq.tq_attend_decode_polar(h, torch_input(q, "f32"), kc, vc, out, ws, T=T, scale=scale)
+            outs[path] = out.cpu().numpy()
+    finally:
+        tq.tq_set_decode_path(h, "auto")
+    assert rel_err_rows(outs["streamk"], outs["split"]).max() <= 1e-5
+    ku, vu = unpack_cache(kc, 0, T), unpack_cache(vc, 0, T)
+    ku = {"idx": ku["idx"], "nh": ku["nh"], "sig": np.ones(ku["idx"].shape, np.uint8), "gh": np.zeros_like(ku["nh"])}
+    ref = oracle_attend(prms[d], q.astype(np.float64), ku, vu, Hkv, [T] * B, scale)
+    err = rel_err_rows(outs["streamk"], ref)
+    print("stream-K polar-only K max rel err", err.max())
+    assert err.max() <= ATT_TOL
+    assert tq.tq_device_status(h) == tq.TQ_OK
+
+
 def test_split_count_invariance(decode_path, handles):
     """Different split plans (by T, or by Tcap through seq_lens) agree within 1e-5."""
     d, B, Hq, Hkv, T, Tcap = 128, 2, 8, 2, 3000, 8192
@@ -768,12 +803,15 @@ def test_group_heads_equal_separate_heads(decode_path, handles):
 
 
 @pytest.mark.parametrize("d,G", [(128, 4), (128, 2), (64, 2), (256, 4), (128, 8)])
-def test_bounded_wait_give_up_path(handles, prms, d, G):
+@pytest.mark.parametrize("path", ["auto", "streamk"])
+def test_bounded_wait_give_up_path(handles, prms, d, G, path):
     """Every wait in the attention kernel is bounded.  With the first-wait
     budget set to zero polls every warp gives up at its first staged chunk: the
     call completes, the check word reports the failed wait, the outputs are
     finite (the warps' tokens are left out), and after the budget is restored
-    the same handle computes the attention again and matches the oracle."""
+    the same handle computes the attention again and matches the oracle.  Also
+    on the stream-K grid, where some warps give up before crossing into a
+    second sequence."""
     h = handles[d]
     B, Hkv, T = 2, 2, 777
     Hq, Tcap = Hkv * G, 832
@@ -784,15 +822,18 @@ def test_bounded_wait_give_up_path(handles, prms, d, G):
     q = synthetic.gaussian((B, Hq, d), seed=18)
     assert tq.tq_device_status(h) == tq.TQ_OK
     try:
+        tq.tq_set_decode_path(h, path)
         tq.tq_set_wait_limit(h, 0)
         out = attend_gpu(h, torch_input(q, "f32"), kc, vc, T=T, scale=0.1)
         assert tq.tq_device_status(h) == tq.TQ_ERR_DEVICE_CHECK
         assert torch.isfinite(out).all()
+        tq.tq_set_wait_limit(h, -1)
+        assert tq.tq_device_status(h) == tq.TQ_OK
+        out = attend_gpu(h, torch_input(q, "f32"), kc, vc, T=T, scale=0.1).cpu().numpy()
+        assert tq.tq_device_status(h) == tq.TQ_OK
     finally:
         tq.tq_set_wait_limit(h, -1)
-    assert tq.tq_device_status(h) == tq.TQ_OK
-    out = attend_gpu(h, torch_input(q, "f32"), kc, vc, T=T, scale=0.1).cpu().numpy()
-    assert tq.tq_device_status(h) == tq.TQ_OK
+        tq.tq_set_decode_path(h, "auto")
     ref = oracle_attend(prms[d], q.astype(np.float64), unpack_cache(kc, 0, Tcap), unpack_cache(vc, 0, Tcap), Hkv,
                         [T] * B, 0.1)
     assert rel_err_rows(out, ref).max() <= ATT_TOL
