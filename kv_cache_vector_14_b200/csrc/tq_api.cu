@@ -304,6 +304,20 @@ tq_status tq_init(int head_dim, uint64_t seed, tq_handle** out) {
     h->cb.lut_lo[0] = lo[0]; h->cb.lut_lo[1] = lo[1];
     h->cb.lut_hi[0] = hi[0]; h->cb.lut_hi[1] = hi[1];
     for (int k = 0; k < 32; ++k) h->cb.pow2[k] = 1u << k;
+    // integer byte limbs of c 2^14 (exact when each fp16 centroid is a multiple of 2^-14)
+    h->cb.k8 = 1;
+    uint32_t l8[2] = {0, 0}, h8[2] = {0, 0};
+    for (int k = 0; k < 8; ++k) {
+        const double ci = half_bits_to_double(double_to_half_bits((double)h->hc[k])) * 16384.0;
+        const long long v = std::llround(ci);
+        if ((double)v != ci || v > 32767 || v < -32768) h->cb.k8 = 0;
+        const int lo8 = (int)(((v + 128) & 255) - 128), hi8 = (int)((v - lo8) / 256);
+        if (hi8 < -128 || hi8 > 127) h->cb.k8 = 0;
+        l8[k >> 2] |= (uint32_t)(uint8_t)(int8_t)lo8 << (8 * (k & 3));
+        h8[k >> 2] |= (uint32_t)(uint8_t)(int8_t)hi8 << (8 * (k & 3));
+    }
+    h->cb.lut8_lo[0] = l8[0]; h->cb.lut8_lo[1] = l8[1];
+    h->cb.lut8_hi[0] = h8[0]; h->cb.lut8_hi[1] = h8[1];
 
     std::vector<float> sign(d), st((size_t)d * d), sthr((size_t)d * d);
     for (int j = 0; j < d; ++j) sign[j] = (float)h->hD[j];

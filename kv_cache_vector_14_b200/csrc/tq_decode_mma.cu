@@ -85,10 +85,11 @@ __device__ __forceinline__ int64_t table_block(const int32_t* table, int64_t poo
 // and output rows belong to head t (and head 4 + t when NT = 2).  A kv head
 // with more than 8 query heads is served by ceil(G / 8) CTAs (grid.y = Hkv x
 // head groups), each taking up to 8 of its query heads.
-template <int D, int NT, int NW, bool QJL>
+template <int D, int NT, int NW, bool QJL, bool K8>
 __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs a, int G) {
     using C = Cfg<D, QJL>;
     constexpr int kKC = C::kKC;
+    static_assert(!K8 || (D == 128 && NT == 1), "int8 key operands: head_dim 128, up to two heads per kv head");
     constexpr int kSBGroup = 2 * NT * kKC * 32;   // uint2 entries of one unit's q'/u' fragments
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)NW * kStages * C::kStageB);
@@ -100,10 +101,10 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                                                (size_t)NW * 8 * 2 * sizeof(float));
     uint2* sB = reinterpret_cast<uint2*>(smem + (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
                                          (size_t)NW * 8 * 2 * sizeof(float) + 2 * kTabMax * sizeof(int32_t));
-    // u' factors per (unit group, kind, head): [2][2][8]
+    // score factors per (unit group, kind, head): [2][3][8] (u' factor, u' sum, int8 q' factor)
     float* sF = reinterpret_cast<float*>(sB + 2 * kSBGroup);
     // the crossing warp's unit-A result: accumulators [8][D], (max, sum) [8][2]
-    float* xacc = sF + 2 * 2 * 8;
+    float* xacc = sF + 2 * 3 * 8;
     float* xml = xacc + 8 * D;
     int64_t* sU = reinterpret_cast<int64_t*>(xml + 8 * 2);     // [NW][2][4] unit descriptors
     int* sMerge = reinterpret_cast<int*>(sU + NW * 8);          // [8] CTA merge facts
@@ -350,13 +351,57 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     };
     // The q' fragments of each unit the CTA touches go to sB (group g: unit A
     // or B), filled by all warps; so do the u' words and factors below.
-    for (int idx = warp; idx < ngrp * kKC; idx += NW) {
+    for (int idx = warp; !K8 && idx < ngrp * kKC; idx += NW) {
         const int g = idx >= kKC ? 1 : 0, kc = idx - g * kKC;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             uint32_t r0, r1;
             b_frag(a.qp, g ? hbB : hbA, g ? GlB : GlA, nt, kc, r0, r1);
             sB[(size_t)g * kSBGroup + (nt * kKC + kc) * 32 + lane] = make_uint2(r0, r1);
+        }
+    }
+    // int8 key operands (K8, up to two heads): q' of each head in 22-bit fixed
+    // point, q_int = rint(q' 2^22 / max|q'|) = l0 + 256 l1 + 65536 l2 (signed byte
+    // limbs); B column n = gr is head gr / 4, limb gr % 4 (limb 3 zero).  K-block w
+    // of the m16n8k32 operand: rows 4 tq4 + e and 16 + 4 tq4 + e are positions
+    // 8 w + e and 8 w + 4 + e of slot tq4, i.e. coordinates 32 w + 2 tq4 + o(e)
+    // and 32 w + 16 + 2 tq4 + o(e), o = (0, 1, 8, 9).  The factor of head h,
+    // scale_log2 max|q'| 2^-22 2^-14 (the keys are c 2^14), goes to sF[g][2][h].
+    if constexpr (K8) {
+        for (int g = warp; g < ngrp; g += NW) {
+            const int hq = gr >> 2, lq = gr & 3;
+            const int gl_ = g ? GlB : GlA;
+            const float* qrow = a.qp + ((g ? hbB : hbA) + (hq < gl_ ? hq : 0)) * D;
+            float qv[4][8];
+            float qm = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int o = (e & 1) + 8 * ((e >> 1) & 1);
+                    qv[w][e] = qrow[32 * w + 16 * (e >> 2) + 2 * tq4 + o];
+                    qm = fmaxf(qm, fabsf(qv[w][e]));
+                }
+            qm = fmaxf(qm, __shfl_xor_sync(kFull, qm, 1));
+            qm = fmaxf(qm, __shfl_xor_sync(kFull, qm, 2));
+            if (hq >= gl_) qm = 0.f;
+            const float fq = qm > 0.f ? 4194304.f / qm : 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                uint32_t b2[2] = {0u, 0u};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int qi = __float2int_rn(qv[w][e] * fq);
+                    const int l0 = ((qi + 128) & 255) - 128;
+                    const int r1 = (qi - l0) >> 8;
+                    const int l1 = ((r1 + 128) & 255) - 128;
+                    const int l2 = (r1 - l1) >> 8;
+                    const int limb = lq == 0 ? l0 : lq == 1 ? l1 : lq == 2 ? l2 : 0;
+                    b2[e >> 2] |= (uint32_t)(uint8_t)(int8_t)limb << (8 * (e & 3));
+                }
+                sB[(size_t)g * kSBGroup + w * 32 + lane] = make_uint2(b2[0], b2[1]);
+            }
+            if (lq == 0 && tq4 == 0) sF[(g * 3 + 2) * 8 + hq] = a.scale_log2 * (qm * (1.f / 4194304.f)) * (1.f / 16384.f);
         }
     }
     // QJL term on int8 operands.  u' of each head is taken to 16-bit fixed point,
@@ -368,7 +413,8 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     // sum_i u'_i (2 sigma_i - 1) = (max|u'| / kQ) (-acc / 64 - sum_i u_int_i), exact
     // up to the fixed point of u' (the term is scaled by gamma ~ 0.18 of the score).
     // The words of (unit g, n-tile nt) go to sB, and the factors of head h to
-    // sF[g][0][h] (scale_log2 max|u'| / (64 kQ)) and sF[g][1][h] (64 sum u_int).
+    // sF[g][0][h] (scale_log2 max|u'| / (64 kQ)) and sF[g][1][h] (64 sum u_int).  With int8
+    // key operands (K8) the columns are head gr / 4, limb gr % 4 (limbs 2, 3 zero).
     constexpr int kKB = D / 32;
     constexpr float kQ = 32000.f;
     if constexpr (QJL) {
@@ -379,8 +425,9 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         };
         for (int idx = warp; idx < ngrp * NT; idx += NW) {
             const int g = idx >= NT ? 1 : 0, nt = idx - g * NT;
-            const int hcol = 4 * nt + (gr >> 1);
+            const int hcol = K8 ? (gr >> 2) : 4 * nt + (gr >> 1);
             const bool hlive = hcol < (g ? GlB : GlA);
+            const bool zcol = K8 && (gr & 3) >= 2;               // K8: limb columns 2, 3 are zero
             const float* up = a.up + ((g ? hbB : hbA) + (hlive ? hcol : 0)) * D;
             float um = 0.f;
 #pragma unroll
@@ -403,16 +450,17 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                     for (int e = 0; e < 4; ++e) {
                         const int ui = __float2int_rn(up[row_of(kb, hf, e)] * fu);
                         const int lo = ((ui + 128) & 255) - 128;
-                        w[hf] |= (uint32_t)(uint8_t)(int8_t)((gr & 1) ? lo : (ui - lo) >> 8) << (8 * e);
+                        const int lb = (gr & 1) ? lo : (ui - lo) >> 8;
+                        w[hf] |= (uint32_t)(uint8_t)(int8_t)(zcol ? 0 : lb) << (8 * e);
                         usum += ui;
                     }
                 sB[(size_t)g * kSBGroup + ((NT + nt) * kKC + kb) * 32 + lane] = make_uint2(w[0], w[1]);
             }
             usum += __shfl_xor_sync(kFull, usum, 1);
             usum += __shfl_xor_sync(kFull, usum, 2);
-            if ((gr & 1) == 0 && tq4 == 0) {
-                sF[(g * 2) * 8 + hcol] = a.scale_log2 * (um / kQ) * (1.f / 64.f);
-                sF[(g * 2 + 1) * 8 + hcol] = 64.f * (float)usum;
+            if ((gr & (K8 ? 3 : 1)) == 0 && tq4 == 0) {
+                sF[(g * 3) * 8 + hcol] = a.scale_log2 * (um / kQ) * (1.f / 64.f);
+                sF[(g * 3 + 1) * 8 + hcol] = 64.f * (float)usum;
             }
         }
     }
@@ -423,6 +471,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     }
     __syncthreads();
     const uint32_t lut[4] = {a.cb.lut_lo[0], a.cb.lut_lo[1], a.cb.lut_hi[0], a.cb.lut_hi[1]};
+    [[maybe_unused]] const uint32_t l8[4] = {a.cb.lut8_lo[0], a.cb.lut8_lo[1], a.cb.lut8_hi[0], a.cb.lut8_hi[1]};
     const uint32_t* pw = a.cb.pow2;
     [[maybe_unused]] const uint32_t m64 = pw[20] | 1u;    // d = 64 sign widening factor
 
@@ -432,6 +481,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
     uint32_t bq[C::kBRegs ? NT : 1][C::kBRegs ? kKC : 1][2];
     [[maybe_unused]] uint32_t iu[QJL && C::kBRegs ? NT : 1][QJL && C::kBRegs ? kKB : 1][2];
     [[maybe_unused]] float fS[NT], uS[NT];   // factors of this lane's own head 4 nt + tq4
+    [[maybe_unused]] float fK = 0.f;         // K8: factor of this lane's head's integer key score
     [[maybe_unused]] const uint2* sBw = sB;  // this warp's unit's fragments in sB
     float o[NT][kKC][4];
     float mrun[NT], lrun[NT], live[NT];
@@ -443,7 +493,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int kc = 0; kc < kKC; ++kc) {
+                for (int kc = 0; kc < (K8 ? 4 : kKC); ++kc) {     // K8: the four k-blocks' q' limbs
                     const uint2 v = sBw[(nt * kKC + kc) * 32 + lane];
                     bq[nt][kc][0] = v.x;
                     bq[nt][kc][1] = v.y;
@@ -461,11 +511,16 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
+            // this lane's head: 4 nt + tq4, or with int8 keys tq4 / 2 (even lanes own it,
+            // odd lanes hold the same score and contribute nothing)
+            const int hh = K8 ? (tq4 >> 1) : 4 * nt + tq4;
+            const bool own = !K8 || (tq4 & 1) == 0;
             if constexpr (QJL) {
-                fS[nt] = sF[(g * 2) * 8 + 4 * nt + tq4];
-                uS[nt] = sF[(g * 2 + 1) * 8 + 4 * nt + tq4];
+                fS[nt] = own ? sF[(g * 3) * 8 + hh] : 0.f;
+                uS[nt] = own ? sF[(g * 3 + 1) * 8 + hh] : 0.f;
             }
-            live[nt] = (4 * nt + tq4 < Gl) ? 1.f : 0.f;   // this lane's head exists
+            if constexpr (K8) fK = sF[(g * 3 + 2) * 8 + hh];
+            live[nt] = (own && hh < Gl) ? 1.f : 0.f;      // this lane's head exists
             mrun[nt] = -INFINITY;
             lrun[nt] = 0.f;
 #pragma unroll
@@ -482,8 +537,9 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
             lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 4);
             lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 8);
             lrun[nt] += __shfl_xor_sync(kFull, lrun[nt], 16);
-            const int h = 4 * nt + tq4;
-            const bool hl = h < Gl;
+            const int h = K8 ? (tq4 >> 1) : 4 * nt + tq4;
+            const bool own = !K8 || (tq4 & 1) == 0;
+            const bool hl = own && h < Gl;
             if (hl && write_acc) {
 #pragma unroll
                 for (int mt = 0; mt < kKC; ++mt) {
@@ -491,7 +547,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                     acc_dst[h * D + 16 * mt + 8 + gr] = o[nt][mt][2] + o[nt][mt][3];
                 }
             }
-            if (gr == 0) {
+            if (gr == 0 && own) {
                 ml_dst[h * 2] = hl ? mrun[nt] : -INFINITY;
                 ml_dst[h * 2 + 1] = hl ? lrun[nt] : 0.f;
             }
@@ -546,37 +602,63 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                 acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
                 accS[nt][0] = accS[nt][1] = accS[nt][2] = accS[nt][3] = 0;
             }
-#pragma unroll
-            for (int kc = 0; kc < kKC; ++kc) {
-                const int sl = kc >> 3, kk = kc & 7;
-                uint32_t ka[4];
-                dequant4(sel_for(selA[sl], pw, kk), lut, ka[0], ka[2]);
-                dequant4(sel_for(selB[sl], pw, kk), lut, ka[1], ka[3]);
+            // QJL term: int8 m16n8k32 over one k32 block of sign bits
+            [[maybe_unused]] auto sign_mma = [&](int kb, int sl) {
+                const int k4 = kb & 3;
+                const uint32_t sg[4] = {shl_m(sgA[sl], pw, 2 * k4) & 0x80808080u,
+                                        shl_m(sgB[sl], pw, 2 * k4) & 0x80808080u,
+                                        shl_m(sgA[sl], pw, 2 * k4 + 1) & 0x80808080u,
+                                        shl_m(sgB[sl], pw, 2 * k4 + 1) & 0x80808080u};
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     if constexpr (C::kBRegs) {
-                        mma16816(acc[nt], ka, bq[nt][kc][0], bq[nt][kc][1]);
+                        imma16832(accS[nt], sg, iu[nt][kb][0], iu[nt][kb][1]);
                     } else {
-                        const uint2 fq = sBw[(nt * kKC + kc) * 32 + lane];
-                        mma16816(acc[nt], ka, fq.x, fq.y);
+                        const uint2 fu = sBw[((NT + nt) * kKC + kb) * 32 + lane];
+                        imma16832(accS[nt], sg, fu.x, fu.y);
                     }
                 }
-                if constexpr (QJL) {
-                    if ((kc & 1) == 0) {                        // one k32 block of signs per two k-steps
-                        const int kb = kc >> 1, k4 = kb & 3;
-                        const uint32_t sg[4] = {shl_m(sgA[sl], pw, 2 * k4) & 0x80808080u,
-                                                shl_m(sgB[sl], pw, 2 * k4) & 0x80808080u,
-                                                shl_m(sgA[sl], pw, 2 * k4 + 1) & 0x80808080u,
-                                                shl_m(sgB[sl], pw, 2 * k4 + 1) & 0x80808080u};
+            };
+            if constexpr (K8) {
+                // keys as int8 limbs of c 2^14: one prmt gives four codes' limb bytes,
+                // which are the m16n8k32 A operand rows as they stand (no interleave)
+                int accK[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            if constexpr (C::kBRegs) {
-                                imma16832(accS[nt], sg, iu[nt][kb][0], iu[nt][kb][1]);
-                            } else {
-                                const uint2 fu = sBw[((NT + nt) * kKC + kb) * 32 + lane];
-                                imma16832(accS[nt], sg, fu.x, fu.y);
-                            }
+                for (int w = 0; w < 4; ++w) {
+                    const uint32_t sa = selA[0][w], sb = selB[0][w];
+                    const uint32_t sah = shr_m(sa, pw, 16), sbh = shr_m(sb, pw, 16);
+                    const uint32_t alo[4] = {__byte_perm(l8[0], l8[1], sa), __byte_perm(l8[0], l8[1], sb),
+                                             __byte_perm(l8[0], l8[1], sah), __byte_perm(l8[0], l8[1], sbh)};
+                    const uint32_t ahi[4] = {__byte_perm(l8[2], l8[3], sa), __byte_perm(l8[2], l8[3], sb),
+                                             __byte_perm(l8[2], l8[3], sah), __byte_perm(l8[2], l8[3], sbh)};
+                    imma16832(accK[0], alo, bq[0][w][0], bq[0][w][1]);
+                    imma16832(accK[1], ahi, bq[0][w][0], bq[0][w][1]);
+                    if constexpr (QJL) sign_mma(w, 0);
+                }
+                // this lane's columns 2 tq4, 2 tq4 + 1 are q' limbs 2 (tq4 & 1), + 1 of head tq4 / 2
+                const float w0 = (tq4 & 1) ? 65536.f : 1.f, w1 = (tq4 & 1) ? 0.f : 256.f;
+                acc[0][0] = fmaf((float)accK[1][0], w0, fmaf((float)accK[1][1], w1, 0.f)) * 256.f +
+                            fmaf((float)accK[0][0], w0, (float)accK[0][1] * w1);
+                acc[0][2] = fmaf((float)accK[1][2], w0, fmaf((float)accK[1][3], w1, 0.f)) * 256.f +
+                            fmaf((float)accK[0][2], w0, (float)accK[0][3] * w1);
+            } else {
+#pragma unroll
+                for (int kc = 0; kc < kKC; ++kc) {
+                    const int sl = kc >> 3, kk = kc & 7;
+                    uint32_t ka[4];
+                    dequant4(sel_for(selA[sl], pw, kk), lut, ka[0], ka[2]);
+                    dequant4(sel_for(selB[sl], pw, kk), lut, ka[1], ka[3]);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        if constexpr (C::kBRegs) {
+                            mma16816(acc[nt], ka, bq[nt][kc][0], bq[nt][kc][1]);
+                        } else {
+                            const uint2 fq = sBw[(nt * kKC + kc) * 32 + lane];
+                            mma16816(acc[nt], ka, fq.x, fq.y);
                         }
+                    }
+                    if constexpr (QJL) {
+                        if ((kc & 1) == 0) sign_mma(kc >> 1, sl);   // one k32 block of signs per two k-steps
                     }
                 }
             }
@@ -598,12 +680,17 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
             uint32_t pb[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                float sA = a.scale_log2 * (acc[nt][0] + acc[nt][1]);
-                float sB_ = a.scale_log2 * (acc[nt][2] + acc[nt][3]);
+                float sA = K8 ? fK * acc[nt][0] : a.scale_log2 * (acc[nt][0] + acc[nt][1]);
+                float sB_ = K8 ? fK * acc[nt][2] : a.scale_log2 * (acc[nt][2] + acc[nt][3]);
                 if constexpr (QJL) {
                     // + gamma (max|u'| / kQ) (-acc / 64 - sum u_int), acc = 256 hi-limb + lo-limb column
+                    // (K8: zero on the odd lanes, whose factors are zero)
                     sA = fmaf(-gAf * fS[nt], (float)(accS[nt][0] * 256 + accS[nt][1]) + uS[nt], sA);
                     sB_ = fmaf(-gBf * fS[nt], (float)(accS[nt][2] * 256 + accS[nt][3]) + uS[nt], sB_);
+                }
+                if constexpr (K8) {             // the head's q' limbs sit on lanes tq4 and tq4 ^ 1
+                    sA += __shfl_xor_sync(kFull, sA, 1);
+                    sB_ += __shfl_xor_sync(kFull, sB_, 1);
                 }
                 sA *= nkA.x;
                 sB_ *= nkA.y;
@@ -728,15 +815,15 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
 constexpr int kNW1 = 16;   // warps per CTA, up to 4 heads per kv head (one n-tile)
 constexpr int kNW2 = 8;    // warps per CTA, 8 heads per kv head (two n-tiles, more registers)
 
-template <int D, int NT, int NW, bool QJL>
+template <int D, int NT, int NW, bool QJL, bool K8 = false>
 cudaError_t launch_mma_t(const DecArgs& a, int G, cudaStream_t s) {
     using C = Cfg<D, QJL>;
     const size_t smem = (size_t)NW * kStages * C::kStageB + (size_t)NW * kStages * 8 +
                         (size_t)NW * 8 * 2 * sizeof(float) + 2 * kTabMax * sizeof(int32_t) +
-                        (size_t)2 * 2 * NT * C::kKC * 32 * sizeof(uint2) + (2 * 2 * 8 + 8 * D + 8 * 2) * sizeof(float) +
+                        (size_t)2 * 2 * NT * C::kKC * 32 * sizeof(uint2) + (2 * 3 * 8 + 8 * D + 8 * 2) * sizeof(float) +
                         (size_t)NW * 8 * sizeof(int64_t) + 8 * sizeof(int);
-    auto kern = tq_decode_mma_kernel<D, NT, NW, QJL>;
-    cudaError_t e = set_smem_once<tq_decode_mma_kernel<D, NT, NW, QJL>>((int)smem);
+    auto kern = tq_decode_mma_kernel<D, NT, NW, QJL, K8>;
+    cudaError_t e = set_smem_once<tq_decode_mma_kernel<D, NT, NW, QJL, K8>>((int)smem);
     if (e != cudaSuccess) return e;
     const dim3 grid = a.sk_ctas > 0 ? dim3((unsigned)a.sk_ctas)
                                     : dim3(a.nsplit, (unsigned)(a.Hkv * ((G + 7) / 8)), (unsigned)a.B);
@@ -747,8 +834,11 @@ template <bool QJL>
 cudaError_t launch_mma_q(int d, int G, const DecArgs& a, cudaStream_t s) {
     if (d == 64)
         return G <= 4 ? launch_mma_t<64, 1, kNW1, QJL>(a, G, s) : launch_mma_t<64, 2, kNW2, QJL>(a, G, s);
-    if (d == 128)
+    if (d == 128) {
+        // up to two heads per kv head: keys as int8 limbs (half the byte look-ups)
+        if (G <= 2 && a.cb.k8) return launch_mma_t<128, 1, kNW1, QJL, true>(a, G, s);
         return G <= 4 ? launch_mma_t<128, 1, kNW1, QJL>(a, G, s) : launch_mma_t<128, 2, kNW2, QJL>(a, G, s);
+    }
     return G <= 4 ? launch_mma_t<256, 1, kNW1, QJL>(a, G, s) : launch_mma_t<256, 2, kNW2, QJL>(a, G, s);
 }
 

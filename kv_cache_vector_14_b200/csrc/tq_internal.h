@@ -45,6 +45,12 @@ struct Codebook {
     uint32_t lut_lo[2]; // low bytes of the fp16 bit patterns of c[0..7]
     uint32_t lut_hi[2]; // high bytes of the fp16 bit patterns of c[0..7]
     uint32_t pow2[32];  // 1 << k: shifts done as integer multiplies (FMA pipe, not ALU)
+    // The centroids as exact integers c 2^14 = 256 hi + lo (signed byte limbs),
+    // when every one is an integer of at most 15 bits (int8 key operands):
+    // byte k of lut8_lo / lut8_hi is the lo / hi limb of c[k].
+    uint32_t lut8_lo[2];
+    uint32_t lut8_hi[2];
+    int k8;             // 1: the limbs above are exact
 };
 
 // Host-side generation of the constants (tq_params.cpp).
