@@ -23,7 +23,15 @@
 // look-up tables of the fp16 centroids (lo bytes, hi bytes), and its sign
 // bits come as one word of which a shift and a mask keep four signs, one per
 // operand byte.  Value fragments are produced key-style and transposed in
-// registers (movmatrix).
+// registers (movmatrix).  With at most two query heads per kv head at
+// head_dim 128 (K8) the keys enter as int8 limbs of the integer centroids
+// c 2^14 instead (one prmt per four codes and limb, no interleave) against q'
+// in 22-bit fixed point as three byte limbs.
+//
+// Work partition: a uniform split of every (batch, kv head, head group) unit
+// (grid = splits x units), or a stream-K grid over all units' chunks laid end
+// to end (grid = CTAs, each warp a contiguous run of chunks, at most one warp
+// per CTA crossing into a second unit); the host's cost model picks.
 //
 // Data movement: each warp owns a ring of STAGES shared-memory buffers of a
 // chunk of tokens (32 at d = 128, 16 at d = 256; K codes, signs, norms,
