@@ -754,6 +754,239 @@ __global__ void __launch_bounds__(k6Threads, 2)
     pdl_wait();                    // when chained: complete only after the previous kernel
 }
 
+// ---------------------------------------------------------------- head_dim 128, V, two threads per vector
+// The V encode at d = 128 with the d = 64 kernel's organisation: Y = X (H D)^T
+// with the rotation's rows in slot order (Y's column 32 t + p is coordinate
+// slot_coord(0, t, p), position p of slot t), two threads per vector (warps w
+// and w + 4), each owning two 32-position slots: a thread builds its slots'
+// three code words (Wa, Wb, Wc of each slot, the bit-3 planes from positions
+// 24..31 included) in registers and stores its 24 bytes of the record itself,
+// so the two threads meet once per tile, for ||Y||^2.  Two input buffers and
+// 256 tensor-memory columns (Y x 2), so two CTAs fit an SM.
+constexpr int kVQuant = 256;                 // two threads per vector
+constexpr int kVThreads = kVQuant + 32;
+constexpr int kVXBuf = 2;                    // input tile buffers
+
+struct RotVShape {
+    static constexpr int kOffM = 0;                              // rotation operand H D (rows in slot order)
+    static constexpr int kOffX = kRTile;                         // input tiles
+    static constexpr int kOffBar = kOffX + kVXBuf * kRTile;
+    static constexpr int kOffXchg = kOffBar + 16 * 8;            // ||Y||^2 parts [2 tiles][2][128]
+    static constexpr int kOffMisc = kOffXchg + 2 * 2 * 128 * 4;
+    static constexpr int kSmem = kOffMisc + 16 + 1024;
+    static constexpr int kCols = 256;                            // Y x 2 at 0, 128
+};
+static_assert(2 * (RotVShape::kSmem + 1024) <= 228 * 1024, "two CTAs per SM");
+
+template <int DT>
+__global__ void __launch_bounds__(kVThreads, 2)
+    tq_encode_rotv_kernel(const __grid_constant__ CUtensorMap tmap, const EncArgs a) {
+    using S = RotVShape;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + S::kOffBar);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + S::kOffMisc);
+    pdl_trigger();                 // a chained kernel may start (it waits for this one's writes)
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int64_t N = a.B * a.Hkv * a.Tnew;
+    const int64_t ntiles = (N + kRRows - 1) / kRRows;
+    const int n = (int)((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);   // this CTA's tiles
+    auto row0_of = [&](int j) { return ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kRRows; };
+    const int64_t bb = block_bytes(kRD, false);
+
+    if (tid == 0) {
+        for (int i = 0; i < kVXBuf; ++i) {
+            mbar_init(bar(kRBarXFull + i), 1);
+            mbar_init(bar(kRBarXFree + i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(kRBarYFull + i), 1);
+            mbar_init(bar(kRBarRFull + i), kVQuant);
+        }
+        mbar_init(bar(kRBarDrain), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc_alloc(smem_u32(tmem_slot), S::kCols);
+        tc_relinquish();
+    }
+    // Rotation operand row nr (Y's column nr), K index i: (-1)^popcount(i & j) d_i with
+    // j = slot_coord(0, nr / 32, nr % 32), as bf16 / fp16 +-1.
+    if (tid < kRRows) {
+        const int j = slot_coord(0, tid >> 5, tid & 31);
+        const uint32_t one = DT == TQ_BF16 ? 0x3F80u : 0x3C00u;
+#pragma unroll 1
+        for (int i0 = 0; i0 < kRD; i0 += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                uint32_t h2[2];
+#pragma unroll
+                for (int f = 0; f < 2; ++f) {
+                    const int i = i0 + 2 * e + f;
+                    const uint32_t neg = ((uint32_t)__popc(i & j) & 1u) ^ (__ldg(a.dsign + i) < 0.f ? 1u : 0u);
+                    h2[f] = one | (neg << 15);
+                }
+                w[e] = h2[0] | (h2[1] << 16);
+            }
+            *reinterpret_cast<uint4*>(sm + S::kOffM + sw128_byte(tid, 2 * i0, kRD)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async();           // written by threads, read by the tensor core
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (tid == kVQuant) {
+        // ======================================== copy and mma thread
+        constexpr uint32_t kIdY = DT == TQ_BF16 ? idesc_bf16(kRRows, kRD) : idesc_f16(kRRows, kRD);
+        auto load = [&](int j) {       // input tile j -> buffer j % 2 (two 64-column boxes)
+            const int bx = j % kVXBuf;
+            const uint32_t dst = sbase + (uint32_t)(S::kOffX + bx * kRTile), br = bar(kRBarXFull + bx);
+            mbar_expect_tx(br, (uint32_t)kRTile);
+            const int r0 = (int)row0_of(j);
+            tma_load_2d(dst, &tmap, 0, r0, br);
+            tma_load_2d(dst + kRTile / 2, &tmap, 64, r0, br);
+        };
+        int n_load = n < kVXBuf ? n : kVXBuf;
+        for (int j = 0; j < n_load; ++j) load(j);
+        bool ok = true;
+        for (int j = 0; ok && j < n; ++j) {
+            const int bx = j % kVXBuf;
+            if (!(ok = mbar_wait_bounded(bar(kRBarXFull + bx), (uint32_t)((j / kVXBuf) & 1)))) break;
+            // Y(j) overwrites buffer j % 2: the quantisers are done with tile j - 2 there
+            if (j >= 2 && !(ok = mbar_wait_bounded(bar(kRBarRFull + (j & 1)), (uint32_t)(((j - 2) >> 1) & 1)))) break;
+            tc_fence_after();
+            const uint32_t xa = sbase + (uint32_t)(S::kOffX + bx * kRTile);
+            const uint32_t yd = tmem + (uint32_t)(128 * (j & 1));
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t koff = (uint32_t)((ks >> 2) * (kRRows * 128) + (ks & 3) * 32);
+                tc_mma_f16_ss(yd, sw128_desc(xa + koff), sw128_desc(sbase + (uint32_t)S::kOffM + koff), kIdY,
+                              ks > 0 ? 1u : 0u);
+            }
+            tc_commit(bar(kRBarYFull + (j & 1)));
+            tc_commit(bar(kRBarXFree + bx));
+            // tile j + 1 goes into tile j - 1's buffer once that tile's rotation is done
+            if (j >= 1 && j + 1 < n) {
+                if (!(ok = mbar_wait_bounded(bar(kRBarXFree + (j - 1) % kVXBuf), (uint32_t)(((j - 1) / kVXBuf) & 1))))
+                    break;
+                load(j + 1);
+                ++n_load;
+            }
+        }
+        // every mma and copy this thread issued is done before shared and tensor memory are
+        // released (only the last load into each buffer can still be in flight)
+        tc_commit(bar(kRBarDrain));
+        mbar_wait_bounded(bar(kRBarDrain), 0u);
+        for (int j = n_load > kVXBuf ? n_load - kVXBuf : 0; j < n_load; ++j)
+            mbar_wait_bounded(bar(kRBarXFull + j % kVXBuf), (uint32_t)((j / kVXBuf) & 1));
+        if (!ok) atomicExch(a.err, 1);
+    } else if (tid < kVQuant) {
+        // ======================================== quantisers: threads r and r + 128 share vector r
+        // (tensor-memory lane r); thread h owns slots 2 h, 2 h + 1, Y's columns 64 h .. 64 h + 63
+        const int hv = tid >> 7;
+        const int r = tid & 127;
+        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        float* xss = reinterpret_cast<float*>(sm + S::kOffXchg);            // [2][2][128]
+        const Codebook& cb = a.cb;
+        // the cell search of the four-thread kernel
+        constexpr float kBig = 1152921504606846976.f;        // 2^60
+        const float bb4 = cb.b[4] * kBig, bb5 = cb.b[5] * kBig, bb6 = cb.b[6] * kBig;
+        bool failed = false;
+        for (int j = 0; j < n; ++j) {
+            const int64_t gv = row0_of(j) + r;
+            const int x = j & 1;
+            // A failed wait does not leave the loop at once: both threads of every vector meet
+            // at the exchange below, which also ORs their failures, and leave together.
+            const bool ok = !failed && warp_wait_r(bar(kRBarYFull + x), (uint32_t)((j >> 1) & 1));
+            tc_fence_after();
+            const uint32_t yb = tl + (uint32_t)(128 * x + 64 * hv);
+            {                              // ||Y||^2 = 128 ||x||^2, this thread's part
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    uint32_t v[32];
+                    tc_ld32(yb + (uint32_t)(32 * q), v);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        s4[e & 3] = fmaf(__uint_as_float(v[e]), __uint_as_float(v[e]), s4[e & 3]);
+                }
+                xss[(x * 2 + hv) * 128 + r] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+            }
+            if (bar_or_r(1, kVQuant, !ok)) { failed = true; break; }
+            const float ss = xss[(x * 2) * 128 + r] + xss[(x * 2 + 1) * 128 + r];
+            const float nrm = sqrtf(ss * (1.f / 128.f));
+            const float rcp = ss > 0.f ? __frcp_rn(sqrtf(ss)) : 0.f;   // y = Y / ||Y||
+            const float kneg = -kBig * rcp;
+            // slot 2 hv + s2: word a holds in nibble k the code of position k (bits 0-2) and
+            // bit 0 of the code of position 24 + k (bit 3); words b, c positions 8 + k, 16 + k
+            // and bits 1, 2 of the code of 24 + k
+            uint32_t wd[6];
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2) {
+                uint32_t nib[4];       // nibble words of positions 0-7, 8-15, 16-23, 24-31
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t v[16];
+                    tc_ld16(yb + (uint32_t)(32 * s2 + 16 * h2), v);
+                    float cf[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const uint32_t ybits = v[e], sgn = ybits & 0x80000000u;
+                        const float av = __uint_as_float(ybits & 0x7FFFFFFFu);
+                        const float t4 = __saturatef(fmaf(av, kneg, bb4));
+                        const float t5 = __saturatef(fmaf(av, kneg, bb5));
+                        const float t6 = __saturatef(fmaf(av, kneg, bb6));
+                        const float T = (t4 + t5) + t6;
+                        cf[e] = __uint_as_float(__float_as_uint(3.5f - T) ^ sgn);   // code - 3.5
+                    }
+                    // nibble sums as exact floats, read out of the mantissa (x + 2^23)
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const float lo = fmaf(cf[8 * q + 3], 4096.f,
+                                              fmaf(cf[8 * q + 2], 256.f, fmaf(cf[8 * q + 1], 16.f, cf[8 * q] + kNib35)));
+                        const float hi = fmaf(cf[8 * q + 7], 4096.f,
+                                              fmaf(cf[8 * q + 6], 256.f, fmaf(cf[8 * q + 5], 16.f, cf[8 * q + 4] + kNib35)));
+                        nib[2 * h2 + q] = __byte_perm(__float_as_uint(lo + 8388608.f), __float_as_uint(hi + 8388608.f), 0x5410);
+                    }
+                }
+                const uint32_t p3 = nib[3];
+#pragma unroll
+                for (int g = 0; g < 3; ++g) wd[3 * s2 + g] = nib[g] | (((p3 >> g) & 0x11111111u) << 3);
+            }
+            tc_fence_before();
+            mbar_arrive(bar(kRBarRFull + x));
+            if (gv < N) {
+                int64_t xoff;
+                uint8_t* blk;
+                int tau;
+                encode_locate(a, (uint32_t)gv, bb, xoff, blk, tau);
+                if (blk) {
+                    uint2* rec = reinterpret_cast<uint2*>(blk + tau * code_bytes(kRD) + 24 * hv);   // slots 2 hv, 2 hv + 1
+                    rec[0] = make_uint2(wd[0], wd[1]);
+                    rec[1] = make_uint2(wd[2], wd[3]);
+                    rec[2] = make_uint2(wd[4], wd[5]);
+                    if (hv == 0) reinterpret_cast<__half*>(blk + kBlockT * code_bytes(kRD))[tau] = __float2half_rn(nrm);
+                }
+            }
+        }
+        if (failed && (tid & 31) == 0) atomicExch(a.err, 1);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tc_dealloc(tmem, S::kCols);
+    }
+    pdl_wait();                    // when chained: complete only after the previous kernel
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -774,6 +1007,16 @@ cudaError_t launch_rot_t(const CUtensorMap& tm, const EncArgs& a, int grid, bool
     if (e != cudaSuccess) return e;
     if (pdl) return launch_pdl(tq_encode_rot_kernel<DT, IS_K>, dim3(grid), dim3(kRThreads), smem, s, tm, a);
     tq_encode_rot_kernel<DT, IS_K><<<grid, kRThreads, smem, s>>>(tm, a);
+    return cudaGetLastError();
+}
+
+template <int DT>
+cudaError_t launch_rotv_t(const CUtensorMap& tm, const EncArgs& a, int grid, bool pdl, cudaStream_t s) {
+    constexpr int smem = RotVShape::kSmem;
+    cudaError_t e = set_smem_once<tq_encode_rotv_kernel<DT>>(smem);
+    if (e != cudaSuccess) return e;
+    if (pdl) return launch_pdl(tq_encode_rotv_kernel<DT>, dim3(grid), dim3(kVThreads), smem, s, tm, a);
+    tq_encode_rotv_kernel<DT><<<grid, kVThreads, smem, s>>>(tm, a);
     return cudaGetLastError();
 }
 
@@ -825,9 +1068,11 @@ cudaError_t launch_encode128_rot(bool is_k, tq_dtype dt, const EncArgs& a, int n
     const int64_t N = a.B * a.Hkv * a.Tnew;
     const int64_t ntiles = (N + kRRows - 1) / kRRows;
     const int grid = (int)(ntiles < num_sms ? ntiles : num_sms);
-    if (dt == TQ_BF16)
-        return is_k ? launch_rot_t<TQ_BF16, true>(tm, a, grid, pdl, s) : launch_rot_t<TQ_BF16, false>(tm, a, grid, pdl, s);
-    return is_k ? launch_rot_t<TQ_F16, true>(tm, a, grid, pdl, s) : launch_rot_t<TQ_F16, false>(tm, a, grid, pdl, s);
+    if (!is_k) {                   // V: two threads per vector, two CTAs per SM
+        const int gv = (int)(ntiles < 2 * num_sms ? ntiles : 2 * num_sms);
+        return dt == TQ_BF16 ? launch_rotv_t<TQ_BF16>(tm, a, gv, pdl, s) : launch_rotv_t<TQ_F16>(tm, a, gv, pdl, s);
+    }
+    return dt == TQ_BF16 ? launch_rot_t<TQ_BF16, true>(tm, a, grid, pdl, s) : launch_rot_t<TQ_F16, true>(tm, a, grid, pdl, s);
 }
 
 }  // namespace tqi
