@@ -324,6 +324,21 @@ TQ_API tq_status tq_set_wait_limit(tq_handle* h, int first_wait);
  * path outside 0..3). */
 TQ_API tq_status tq_set_decode_path(tq_handle* h, int path);
 
+/* Diagnostics, host only (no device or handle needed): the work partition the
+ * tensor-core decode takes for a call of these sizes (head_dim, B sequences,
+ * Hq / Hkv heads, T tokens) on a GPU with num_sms SMs, automatic path.
+ * equal_len != 0: every sequence has T tokens (a call without seq_lens; only
+ * then is the stream-K grid considered), else T is the cache capacity.
+ * Outputs: *nsplit partial slots per query head; *split_tokens tokens per
+ * split of the uniform grid; *streamk_ctas the CTAs of the stream-K grid (0:
+ * the uniform grid is used) and *streamk_chunks the chunks of one (batch, kv
+ * head, query-head group) unit that it divides; *chunk_tokens tokens per chunk.
+ * Errors: INVALID_ARG (head_dim not 64/128/256, sizes as tq_attend_decode
+ * rejects them, num_sms < 1, a NULL output). */
+TQ_API tq_status tq_decode_plan(int num_sms, int head_dim, int64_t B, int64_t Hq, int64_t Hkv, int64_t T,
+                                int equal_len, int* nsplit, int64_t* split_tokens, int64_t* streamk_ctas,
+                                int64_t* streamk_chunks, int* chunk_tokens);
+
 /* Name of the kernel path tq_attend_decode uses for these sizes on this handle
  * ("mma" or "simt"); static string. */
 TQ_API const char* tq_attend_path(const tq_handle* h, int64_t Hq, int64_t Hkv);

@@ -107,14 +107,14 @@ void layout_ws(int d, size_t BHq, int nsplit, DecodePlan* p) {
 // upper_bound: the plan whose workspace bounds every call up to Tmax tokens.
 // equal_len: every sequence has Tmax tokens (no per-sequence lengths), which
 // lets the tensor-core kernel take the stream-K grid when it models faster.
-bool make_plan(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t Tmax, DecodePlan* p,
-               bool upper_bound, bool equal_len = false) {
-    if (!h || B < 0 || Hq <= 0 || Hkv <= 0 || Tmax < 0 || Hq % Hkv) return false;
-    const int d = h->d;
+// The plan for head_dim d on a GPU of num_sms SMs; decode_path as tq_set_decode_path.
+bool make_plan_core(int d, int num_sms, int decode_path, int64_t B, int64_t Hq, int64_t Hkv, int64_t Tmax,
+                    DecodePlan* p, bool upper_bound, bool equal_len) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Tmax < 0 || Hq % Hkv || num_sms < 1) return false;
     p->G = (int)(Hq / Hkv);
-    p->use_mma = h->decode_path != 1 && mma_supported(d, p->G);
+    p->use_mma = decode_path != 1 && mma_supported(d, p->G);
     const int64_t pairs = B * Hkv > 0 ? B * Hkv * decode_head_groups(p->use_mma, p->G) : 1;
-    const int64_t cap = (int64_t)h->num_sms * decode_ctas_per_sm(p->use_mma);
+    const int64_t cap = (int64_t)num_sms * decode_ctas_per_sm(p->use_mma);
     const int chunk = decode_chunk_tokens(d, p->use_mma);
     const int64_t nchunk = Tmax > 0 ? (Tmax + chunk - 1) / chunk : 1;
     const int warps = decode_warps(p->use_mma, p->G);
@@ -128,7 +128,7 @@ bool make_plan(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t T
         int slots = 0;
         const double t_sk = streamk_plan(cap, warps, pairs, nchunk, &nC, &slots);
         // the workspace of any call was sized by the split count bound
-        const bool faster = h->decode_path == 3 || (h->decode_path == 0 && t_sk < t_split);
+        const bool faster = decode_path == 3 || (decode_path == 0 && t_sk < t_split);
         if (t_sk > 0.0 && faster && slots <= split_loop_bound(cap, pairs, nchunk)) {
             p->nsplit = slots;
             p->sk_ctas = nC;
@@ -137,6 +137,11 @@ bool make_plan(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t T
     }
     layout_ws(d, (size_t)(B * Hq), p->nsplit, p);
     return true;
+}
+
+bool make_plan(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t Tmax, DecodePlan* p,
+               bool upper_bound, bool equal_len = false) {
+    return h && make_plan_core(h->d, h->num_sms, h->decode_path, B, Hq, Hkv, Tmax, p, upper_bound, equal_len);
 }
 
 tq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
@@ -415,6 +420,21 @@ tq_status tq_encode_k(const tq_handle* h, const void* x, tq_dtype dt, int64_t B,
 tq_status tq_encode_v(const tq_handle* h, const void* x, tq_dtype dt, int64_t B, int64_t Hkv, int64_t Tnew,
                       int64_t sb, int64_t sh, int64_t st, const tq_cache* vc, int64_t t0, void* stream) {
     return encode_common(h, x, dt, B, Hkv, Tnew, sb, sh, st, vc, t0, stream, false);
+}
+
+tq_status tq_decode_plan(int num_sms, int head_dim, int64_t B, int64_t Hq, int64_t Hkv, int64_t T, int equal_len,
+                         int* nsplit, int64_t* split_tokens, int64_t* streamk_ctas, int64_t* streamk_chunks,
+                         int* chunk_tokens) {
+    if (!nsplit || !split_tokens || !streamk_ctas || !streamk_chunks || !chunk_tokens) return TQ_ERR_INVALID_ARG;
+    if (!head_dim_ok(head_dim) || T < 0) return TQ_ERR_INVALID_ARG;
+    DecodePlan p;
+    if (!make_plan_core(head_dim, num_sms, 0, B, Hq, Hkv, T, &p, false, equal_len != 0)) return TQ_ERR_INVALID_ARG;
+    *nsplit = p.nsplit;
+    *split_tokens = p.split_tokens;
+    *streamk_ctas = p.sk_ctas;
+    *streamk_chunks = p.sk_nck;
+    *chunk_tokens = decode_chunk_tokens(head_dim, p.use_mma);
+    return TQ_OK;
 }
 
 size_t tq_attend_workspace_bytes(const tq_handle* h, int64_t B, int64_t Hq, int64_t Hkv, int64_t Tmax) {

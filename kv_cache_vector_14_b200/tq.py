@@ -24,7 +24,7 @@ EXPORTED = ("tq_params_host", "tq_init", "tq_destroy", "tq_get_params", "tq_head
             "tq_cache_bytes", "tq_encode_k", "tq_encode_v", "tq_attend_workspace_bytes", "tq_attend_decode",
             "tq_append_attend", "tq_prefill_workspace_bytes", "tq_attend_prefill", "tq_attend_decode_polar",
             "tq_attend_decode_static", "tq_device_status", "tq_set_decode_events", "tq_set_decode_path", "tq_set_wait_limit", "tq_attend_path",
-            "tq_status_string")
+            "tq_decode_plan", "tq_status_string")
 
 
 class TQError(RuntimeError):
@@ -97,6 +97,9 @@ def lib() -> C.CDLL:
             L.tq_set_wait_limit.restype = st
             L.tq_attend_path.argtypes = [P, i64, i64]
             L.tq_attend_path.restype = C.c_char_p
+            L.tq_decode_plan.argtypes = [i32, i32, i64, i64, i64, i64, i32, C.POINTER(i32), C.POINTER(i64),
+                                         C.POINTER(i64), C.POINTER(i64), C.POINTER(i32)]
+            L.tq_decode_plan.restype = st
             L.tq_status_string.argtypes = [i32]
             L.tq_status_string.restype = C.c_char_p
             _lib = L
@@ -319,3 +322,15 @@ def tq_set_decode_path(h, path: str) -> None:
 
 def tq_attend_path(h, Hq: int, Hkv: int) -> str:
     return lib().tq_attend_path(h, Hq, Hkv).decode()
+
+
+def tq_decode_plan(num_sms: int, d: int, B: int, Hq: int, Hkv: int, T: int, equal_len: bool = True) -> dict:
+    """The decode work partition for these sizes on a GPU of num_sms SMs (host only):
+    partial slots per query head, tokens per uniform split, stream-K CTAs (0: the
+    uniform grid) and chunks per unit, tokens per chunk."""
+    ns, ct = C.c_int32(), C.c_int32()
+    stt, skc, skn = C.c_int64(), C.c_int64(), C.c_int64()
+    _check(lib().tq_decode_plan(num_sms, d, B, Hq, Hkv, T, int(equal_len), C.byref(ns), C.byref(stt), C.byref(skc),
+                                C.byref(skn), C.byref(ct)), "tq_decode_plan")
+    return {"nsplit": ns.value, "split_tokens": stt.value, "streamk_ctas": skc.value, "streamk_chunks": skn.value,
+            "chunk_tokens": ct.value}
