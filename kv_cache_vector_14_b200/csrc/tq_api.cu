@@ -175,6 +175,7 @@ tq_status prepare_encode(const tq_handle* h, const void* x, tq_dtype dt, int64_t
     a->table = c->block_table;
     a->pool = c->pool_blocks;
     a->dsign = h->dsign; a->sthr = h->dSThr; a->bimg = h->dSB; a->err = h->derr; a->cb = h->cb;
+    for (int i = 0; i < 4; ++i) a->dneg[i] = h->dneg[i];
     const int64_t es = (int64_t)dtype_size(dt);
     a->vec16 = (aligned(x, 16) && (sb * es) % 16 == 0 && (sh * es) % 16 == 0 && (st * es) % 16 == 0) ? 1 : 0;
     a->fdT = make_fastdiv((uint32_t)Tnew);
@@ -326,6 +327,8 @@ tq_status tq_init(int head_dim, uint64_t seed, tq_handle** out) {
 
     std::vector<float> sign(d), st((size_t)d * d), sthr((size_t)d * d);
     for (int j = 0; j < d; ++j) sign[j] = (float)h->hD[j];
+    for (int j = 0; j < d; ++j)
+        if (h->hD[j] < 0) h->dneg[j >> 5] |= 1u << (j & 31);
     for (int i = 0; i < d; ++i)
         for (int j = 0; j < d; ++j) st[(size_t)j * d + i] = h->hS[(size_t)i * d + j];
     const int R = d / 32;

@@ -100,6 +100,28 @@ __device__ __forceinline__ bool bar_or_r(int id, int n, bool v) {
     return res != 0;
 }
 
+// Eight entries (K indices i0 .. i0 + 7, i0 a multiple of 8) of row j of the rotation
+// operand, (-1)^popcount(i & j) d_i as 16-bit +-1 (one: the bit pattern of 1.0).  The bits
+// of i0 and of i - i0 < 8 are disjoint, so popcount(i & j) is popcount(i0 & j) plus that of
+// (i - i0) & j: the chunk's sign bits are the byte of d's sign mask at i0, XOR the parity
+// pattern of j & 7 over k = 0..7 (bit k: popcount(k & j) odd), XOR all ones when i0 & j has
+// odd parity.  dword holds the sign bits of d_{32 (i0 / 32)} .. d_{32 (i0 / 32) + 31}.
+__device__ __forceinline__ uint4 rot_chunk(int j, int i0, uint32_t dword, uint32_t one) {
+    const uint32_t low = ((j & 1) ? 0xAAu : 0u) ^ ((j & 2) ? 0xCCu : 0u) ^ ((j & 4) ? 0xF0u : 0u);
+    const uint32_t neg = ((dword >> (i0 & 31)) ^ low ^ ((__popc(i0 & j) & 1) ? 0xFFu : 0u)) & 0xFFu;
+    const uint32_t one2 = one | (one << 16);
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w[e] = one2 | (((neg >> (2 * e)) & 1u) << 15) | (((neg >> (2 * e + 1)) & 1u) << 31);
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// word i0 / 32 of the sign mask (a select chain: no dynamic index into the parameters)
+__device__ __forceinline__ uint32_t dneg_word(const EncArgs& a, int i0) {
+    const int k = i0 >> 5;
+    return k == 0 ? a.dneg[0] : k == 1 ? a.dneg[1] : k == 2 ? a.dneg[2] : a.dneg[3];
+}
+
 template <int DT, bool IS_K>
 __global__ void __launch_bounds__(kRThreads, 1)
     tq_encode_rot_kernel(const __grid_constant__ CUtensorMap tmap, const EncArgs a) {
@@ -120,7 +142,18 @@ __global__ void __launch_bounds__(kRThreads, 1)
     auto row0_of = [&](int j) { return ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kRRows; };
     const int64_t bb = block_bytes(kRD, IS_K);
 
-    if (tid == 0) {
+    auto load = [&](int j) {           // input tile j -> buffer j % 3 (two 64-column boxes)
+        const int bx = j % kRXBuf;
+        const uint32_t dst = sbase + (uint32_t)(S::kOffX + bx * kRTile), br = bar(kRBarXFull + bx);
+        mbar_expect_tx(br, (uint32_t)kRTile);
+        const int r0 = (int)row0_of(j);
+        tma_load_2d(dst, &tmap, 0, r0, br);
+        tma_load_2d(dst + kRTile / 2, &tmap, 64, r0, br);
+    };
+    int n_load = n < kRXBuf ? n : kRXBuf;
+    // The copy thread sets up the barriers and starts the JL operand copy and the first
+    // input tiles before the rest of the set-up, which their latency then covers.
+    if (tid == kRQuant) {
         mbar_init(bar(kRBarB), 1);
         for (int i = 0; i < kRXBuf; ++i) {
             mbar_init(bar(kRBarXFull + i), 1);
@@ -133,6 +166,12 @@ __global__ void __launch_bounds__(kRThreads, 1)
         }
         mbar_init(bar(kRBarDrain), 1);
         fence_mbar_init();
+        if constexpr (IS_K) {
+            mbar_expect_tx(bar(kRBarB), (uint32_t)(2 * kRTile));
+            bulk_g2s(sbase + (uint32_t)S::kOffS, a.bimg, (uint32_t)(2 * kRTile), bar(kRBarB));
+        }
+        if (a.wait_x) pdl_wait();      // the input and the cache are the previous kernel's to finish
+        for (int j = 0; j < n_load; ++j) load(j);
     }
     if (warp == 0) {
         tc_alloc(smem_u32(tmem_slot), S::kCols);
@@ -140,25 +179,15 @@ __global__ void __launch_bounds__(kRThreads, 1)
     }
     // Rotation operand, row j (output coordinate), K index i (input coordinate):
     // (-1)^popcount(i & j) d_i, the Walsh-Hadamard matrix in natural order times
-    // the random signs, as bf16 / fp16 +-1.
-    if (tid < kRRows) {
-        const int j = tid;
-        const uint32_t one = DT == TQ_BF16 ? 0x3F80u : 0x3C00u;
-#pragma unroll 1
-        for (int i0 = 0; i0 < kRD; i0 += 8) {
-            uint32_t w[4];
+    // the random signs, as bf16 / fp16 +-1; eight entries per store, four per thread.
+    if (tid < kRQuant) {
+        const int i0 = (tid & 15) * 8;
+        const uint32_t dw = dneg_word(a, i0), one = DT == TQ_BF16 ? 0x3F80u : 0x3C00u;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                uint32_t h2[2];
-#pragma unroll
-                for (int f = 0; f < 2; ++f) {
-                    const int i = i0 + 2 * e + f;
-                    const uint32_t neg = ((uint32_t)__popc(i & j) & 1u) ^ (__ldg(a.dsign + i) < 0.f ? 1u : 0u);
-                    h2[f] = one | (neg << 15);
-                }
-                w[e] = h2[0] | (h2[1] << 16);
-            }
-            *reinterpret_cast<uint4*>(sm + S::kOffM + sw128_byte(j, 2 * i0, kRD)) = make_uint4(w[0], w[1], w[2], w[3]);
+        static_assert((kRRows * kRD / 8) % kRQuant == 0 && kRQuant % 16 == 0, "whole chunks per thread");
+        for (int m = 0; m < kRRows * kRD / 8 / kRQuant; ++m) {
+            const int j = (tid >> 4) + (kRQuant / 16) * m;
+            *reinterpret_cast<uint4*>(sm + S::kOffM + sw128_byte(j, 2 * i0, kRD)) = rot_chunk(j, i0, dw, one);
         }
         fence_proxy_async();           // written by threads, read by the tensor core
     }
@@ -171,22 +200,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
         // ======================================== copy and mma thread
         constexpr uint32_t kIdY = DT == TQ_BF16 ? idesc_bf16(kRRows, kRD) : idesc_f16(kRRows, kRD);
         constexpr uint32_t kIdZ = idesc_f16(kRRows, kRD);
-        auto load = [&](int j) {       // input tile j -> buffer j % 3 (two 64-column boxes)
-            const int bx = j % kRXBuf;
-            const uint32_t dst = sbase + (uint32_t)(S::kOffX + bx * kRTile), br = bar(kRBarXFull + bx);
-            mbar_expect_tx(br, (uint32_t)kRTile);
-            const int r0 = (int)row0_of(j);
-            tma_load_2d(dst, &tmap, 0, r0, br);
-            tma_load_2d(dst + kRTile / 2, &tmap, 64, r0, br);
-        };
-        int n_load = n < kRXBuf ? n : kRXBuf;
-        for (int j = 0; j < n_load; ++j) load(j);
         bool ok = true;
-        if constexpr (IS_K) {
-            mbar_expect_tx(bar(kRBarB), (uint32_t)(2 * kRTile));
-            bulk_g2s(sbase + (uint32_t)S::kOffS, a.bimg, (uint32_t)(2 * kRTile), bar(kRBarB));
-            ok = mbar_wait_bounded(bar(kRBarB), 0u);
-        }
+        if constexpr (IS_K) ok = mbar_wait_bounded(bar(kRBarB), 0u);
         // Z(j) = R_hi S_hi^T + R_hi S_lo^T + R_lo S_hi^T.  R(j) lies in Y(j)'s columns:
         // coordinates 16 s + 2 m, + 1 in column 16 s + m (hi) and 16 s + 8 + m (lo).
         auto qjl = [&](int j) {
@@ -303,6 +318,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
             // A failed wait does not leave the loop at once: the four threads of every vector
             // meet at the exchange below, which also ORs their failures, and leave together.
             // (Within a warp the waits are uniform: tensor-memory loads are warp-collective.)
+            // Every exchange stays within a vector's four threads, so its barrier (id 1 + q)
+            // spans only the four warps of lane quarter q and the quarters run out of step:
+            // while one waits at its barrier the others issue.
             const bool ok = !failed && warp_wait_r(bar(kRBarYFull + (j & 1)), (uint32_t)((j >> 1) & 1));
             tc_fence_after();
             const uint32_t yb = tl + (uint32_t)(128 * (j & 1) + 32 * cq);
@@ -314,7 +332,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                 for (int e = 0; e < 32; ++e) s4[e & 3] = fmaf(__uint_as_float(v[e]), __uint_as_float(v[e]), s4[e & 3]);
                 xss[cq * 128 + r] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
             }
-            if (bar_or_r(1, kRQuant, !ok)) { failed = true; break; }
+            if (bar_or_r(1 + (warp & 3), 4 * 32, !ok)) { failed = true; break; }
             const float ss = (xss[r] + xss[128 + r]) + (xss[256 + r] + xss[384 + r]);
             const float nrm = sqrtf(ss * (1.f / 128.f));
             const bool nz = ss > 0.f;
@@ -388,7 +406,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
                     for (int g = 0; g < 3; ++g) xp[(3 * t + g) * 128 + r] = ((W[t] >> g) & 0x11111111u) << 3;
             }
             xg[cq * 128 + r] = g2;
-            named_bar_r(1, kRQuant);
+            named_bar_r(1 + (warp & 3), 4 * 32);
             if (cq == 0) {
                 int64_t xoff;
                 uint8_t* blk = nullptr;
@@ -478,7 +496,15 @@ __global__ void __launch_bounds__(k6Threads, 2)
     auto row0_of = [&](int j) { return ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kRRows; };
     const int64_t bb = block_bytes(k6D, IS_K);
 
-    if (tid == 0) {
+    auto load = [&](int j) {           // input tile j -> buffer j % 3 (one 64-column box)
+        const int bx = j % kRXBuf;
+        const uint32_t dst = sbase + (uint32_t)(S::kOffX + bx * k6Tile), br = bar(kRBarXFull + bx);
+        mbar_expect_tx(br, (uint32_t)k6Tile);
+        tma_load_2d(dst, &tmap, 0, (int)row0_of(j), br);
+    };
+    int n_load = n < kRXBuf ? n : kRXBuf;
+    // barriers, the JL operand copy and the first input tiles first (as at d = 128)
+    if (tid == k6Quant) {
         mbar_init(bar(kRBarB), 1);
         for (int i = 0; i < kRXBuf; ++i) {
             mbar_init(bar(kRBarXFull + i), 1);
@@ -491,31 +517,29 @@ __global__ void __launch_bounds__(k6Threads, 2)
         }
         mbar_init(bar(kRBarDrain), 1);
         fence_mbar_init();
+        if constexpr (IS_K) {
+            mbar_expect_tx(bar(kRBarB), (uint32_t)(2 * k6Op));
+            bulk_g2s(sbase + (uint32_t)S::kOffS, a.bimg, (uint32_t)(2 * k6Op), bar(kRBarB));
+        }
+        if (a.wait_x) pdl_wait();      // the input and the cache are the previous kernel's to finish
+        for (int j = 0; j < n_load; ++j) load(j);
     }
     if (warp == 0) {
         tc_alloc(smem_u32(tmem_slot), S::kCols);
         tc_relinquish();
     }
     // Rotation operand row nr (Y's column nr), K index i: (-1)^popcount(i & j) d_i with
-    // j = slot_coord(0, nr / 16, nr % 16), as bf16 / fp16 +-1.
-    if (tid < 64) {
-        const int j = slot_coord(0, tid >> 4, tid & 15);
-        const uint32_t one = DT == TQ_BF16 ? 0x3F80u : 0x3C00u;
-#pragma unroll 1
-        for (int i0 = 0; i0 < k6D; i0 += 8) {
-            uint32_t w[4];
+    // j = slot_coord(0, nr / 16, nr % 16), as bf16 / fp16 +-1; eight entries per store,
+    // two per thread.
+    if (tid < k6Quant) {
+        const int i0 = (tid & 7) * 8;
+        const uint32_t dw = dneg_word(a, i0), one = DT == TQ_BF16 ? 0x3F80u : 0x3C00u;
+        static_assert((64 * k6D / 8) % k6Quant == 0 && k6Quant % 8 == 0, "whole chunks per thread");
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                uint32_t h2[2];
-#pragma unroll
-                for (int f = 0; f < 2; ++f) {
-                    const int i = i0 + 2 * e + f;
-                    const uint32_t neg = ((uint32_t)__popc(i & j) & 1u) ^ (__ldg(a.dsign + i) < 0.f ? 1u : 0u);
-                    h2[f] = one | (neg << 15);
-                }
-                w[e] = h2[0] | (h2[1] << 16);
-            }
-            *reinterpret_cast<uint4*>(sm + S::kOffM + sw128_byte(tid, 2 * i0, 64)) = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int m = 0; m < 64 * k6D / 8 / k6Quant; ++m) {
+            const int nr = (tid >> 3) + (k6Quant / 8) * m;
+            const int j = slot_coord(0, nr >> 4, nr & 15);
+            *reinterpret_cast<uint4*>(sm + S::kOffM + sw128_byte(nr, 2 * i0, 64)) = rot_chunk(j, i0, dw, one);
         }
         fence_proxy_async();           // written by threads, read by the tensor core
     }
@@ -528,20 +552,8 @@ __global__ void __launch_bounds__(k6Threads, 2)
         // ======================================== copy and mma thread
         constexpr uint32_t kIdY = DT == TQ_BF16 ? idesc_bf16(kRRows, k6D) : idesc_f16(kRRows, k6D);
         constexpr uint32_t kIdZ = idesc_f16(kRRows, k6D);
-        auto load = [&](int j) {       // input tile j -> buffer j % 3 (one 64-column box)
-            const int bx = j % kRXBuf;
-            const uint32_t dst = sbase + (uint32_t)(S::kOffX + bx * k6Tile), br = bar(kRBarXFull + bx);
-            mbar_expect_tx(br, (uint32_t)k6Tile);
-            tma_load_2d(dst, &tmap, 0, (int)row0_of(j), br);
-        };
-        int n_load = n < kRXBuf ? n : kRXBuf;
-        for (int j = 0; j < n_load; ++j) load(j);
         bool ok = true;
-        if constexpr (IS_K) {
-            mbar_expect_tx(bar(kRBarB), (uint32_t)(2 * k6Op));
-            bulk_g2s(sbase + (uint32_t)S::kOffS, a.bimg, (uint32_t)(2 * k6Op), bar(kRBarB));
-            ok = mbar_wait_bounded(bar(kRBarB), 0u);
-        }
+        if constexpr (IS_K) ok = mbar_wait_bounded(bar(kRBarB), 0u);
         // Z(j) = R_hi S_hi^T + R_hi S_lo^T + R_lo S_hi^T over the coordinates in slot order.
         // R(j) lies in Y(j)'s columns: K positions 16 s + 2 m, + 1 in column 16 s + m (hi)
         // and 16 s + 8 + m (lo).
@@ -639,6 +651,7 @@ __global__ void __launch_bounds__(k6Threads, 2)
             const int x = j & 1;
             // A failed wait does not leave the loop at once: both threads of every vector meet
             // at the exchange below, which also ORs their failures, and leave together.
+            // The exchange barrier (id 1 + q) spans only the two warps of lane quarter q.
             const bool ok = !failed && warp_wait_r(bar(kRBarYFull + x), (uint32_t)((j >> 1) & 1));
             tc_fence_after();
             const uint32_t yb = tl + (uint32_t)(64 * x + 32 * hv);
@@ -650,7 +663,7 @@ __global__ void __launch_bounds__(k6Threads, 2)
                 for (int e = 0; e < 32; ++e) s4[e & 3] = fmaf(__uint_as_float(v[e]), __uint_as_float(v[e]), s4[e & 3]);
                 xss[(x * 2 + hv) * 128 + r] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
             }
-            if (bar_or_r(1, k6Quant, !ok)) { failed = true; break; }
+            if (bar_or_r(1 + (warp & 3), 2 * 32, !ok)) { failed = true; break; }
             const float ss = xss[(x * 2) * 128 + r] + xss[(x * 2 + 1) * 128 + r];
             const float nrm = sqrtf(ss * (1.f / 64.f));
             const bool nz = ss > 0.f;
@@ -729,7 +742,7 @@ __global__ void __launch_bounds__(k6Threads, 2)
                 }
             }
             if constexpr (IS_K) {
-                named_bar_r(1, k6Quant);   // both gamma^2 parts are written
+                named_bar_r(1 + (warp & 3), 2 * 32);   // both gamma^2 parts are written
                 if (hv == 0 && blk) {
                     const float gs = xg[(x * 2) * 128 + r] + xg[(x * 2 + 1) * 128 + r];
                     reinterpret_cast<__half*>(blk + kBlockT * (code_bytes(k6D) + sign_bytes(k6D)))[kBlockT + tau] =
@@ -798,7 +811,17 @@ __global__ void __launch_bounds__(kVThreads, 2)
     auto row0_of = [&](int j) { return ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kRRows; };
     const int64_t bb = block_bytes(kRD, false);
 
-    if (tid == 0) {
+    auto load = [&](int j) {           // input tile j -> buffer j % 2 (two 64-column boxes)
+        const int bx = j % kVXBuf;
+        const uint32_t dst = sbase + (uint32_t)(S::kOffX + bx * kRTile), br = bar(kRBarXFull + bx);
+        mbar_expect_tx(br, (uint32_t)kRTile);
+        const int r0 = (int)row0_of(j);
+        tma_load_2d(dst, &tmap, 0, r0, br);
+        tma_load_2d(dst + kRTile / 2, &tmap, 64, r0, br);
+    };
+    int n_load = n < kVXBuf ? n : kVXBuf;
+    // barriers and the first input tiles first (as in the K kernel)
+    if (tid == kVQuant) {
         for (int i = 0; i < kVXBuf; ++i) {
             mbar_init(bar(kRBarXFull + i), 1);
             mbar_init(bar(kRBarXFree + i), 1);
@@ -809,31 +832,25 @@ __global__ void __launch_bounds__(kVThreads, 2)
         }
         mbar_init(bar(kRBarDrain), 1);
         fence_mbar_init();
+        if (a.wait_x) pdl_wait();      // the input and the cache are the previous kernel's to finish
+        for (int j = 0; j < n_load; ++j) load(j);
     }
     if (warp == 0) {
         tc_alloc(smem_u32(tmem_slot), S::kCols);
         tc_relinquish();
     }
     // Rotation operand row nr (Y's column nr), K index i: (-1)^popcount(i & j) d_i with
-    // j = slot_coord(0, nr / 32, nr % 32), as bf16 / fp16 +-1.
-    if (tid < kRRows) {
-        const int j = slot_coord(0, tid >> 5, tid & 31);
-        const uint32_t one = DT == TQ_BF16 ? 0x3F80u : 0x3C00u;
-#pragma unroll 1
-        for (int i0 = 0; i0 < kRD; i0 += 8) {
-            uint32_t w[4];
+    // j = slot_coord(0, nr / 32, nr % 32), as bf16 / fp16 +-1; eight entries per store,
+    // eight per thread.
+    if (tid < kVQuant) {
+        const int i0 = (tid & 15) * 8;
+        const uint32_t dw = dneg_word(a, i0), one = DT == TQ_BF16 ? 0x3F80u : 0x3C00u;
+        static_assert((kRRows * kRD / 8) % kVQuant == 0 && kVQuant % 16 == 0, "whole chunks per thread");
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                uint32_t h2[2];
-#pragma unroll
-                for (int f = 0; f < 2; ++f) {
-                    const int i = i0 + 2 * e + f;
-                    const uint32_t neg = ((uint32_t)__popc(i & j) & 1u) ^ (__ldg(a.dsign + i) < 0.f ? 1u : 0u);
-                    h2[f] = one | (neg << 15);
-                }
-                w[e] = h2[0] | (h2[1] << 16);
-            }
-            *reinterpret_cast<uint4*>(sm + S::kOffM + sw128_byte(tid, 2 * i0, kRD)) = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int m = 0; m < kRRows * kRD / 8 / kVQuant; ++m) {
+            const int nr = (tid >> 4) + (kVQuant / 16) * m;
+            const int j = slot_coord(0, nr >> 5, nr & 31);
+            *reinterpret_cast<uint4*>(sm + S::kOffM + sw128_byte(nr, 2 * i0, kRD)) = rot_chunk(j, i0, dw, one);
         }
         fence_proxy_async();           // written by threads, read by the tensor core
     }
@@ -845,16 +862,6 @@ __global__ void __launch_bounds__(kVThreads, 2)
     if (tid == kVQuant) {
         // ======================================== copy and mma thread
         constexpr uint32_t kIdY = DT == TQ_BF16 ? idesc_bf16(kRRows, kRD) : idesc_f16(kRRows, kRD);
-        auto load = [&](int j) {       // input tile j -> buffer j % 2 (two 64-column boxes)
-            const int bx = j % kVXBuf;
-            const uint32_t dst = sbase + (uint32_t)(S::kOffX + bx * kRTile), br = bar(kRBarXFull + bx);
-            mbar_expect_tx(br, (uint32_t)kRTile);
-            const int r0 = (int)row0_of(j);
-            tma_load_2d(dst, &tmap, 0, r0, br);
-            tma_load_2d(dst + kRTile / 2, &tmap, 64, r0, br);
-        };
-        int n_load = n < kVXBuf ? n : kVXBuf;
-        for (int j = 0; j < n_load; ++j) load(j);
         bool ok = true;
         for (int j = 0; ok && j < n; ++j) {
             const int bx = j % kVXBuf;
@@ -904,6 +911,7 @@ __global__ void __launch_bounds__(kVThreads, 2)
             const int x = j & 1;
             // A failed wait does not leave the loop at once: both threads of every vector meet
             // at the exchange below, which also ORs their failures, and leave together.
+            // The exchange barrier (id 1 + q) spans only the two warps of lane quarter q.
             const bool ok = !failed && warp_wait_r(bar(kRBarYFull + x), (uint32_t)((j >> 1) & 1));
             tc_fence_after();
             const uint32_t yb = tl + (uint32_t)(128 * x + 64 * hv);
@@ -919,7 +927,7 @@ __global__ void __launch_bounds__(kVThreads, 2)
                 }
                 xss[(x * 2 + hv) * 128 + r] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
             }
-            if (bar_or_r(1, kVQuant, !ok)) { failed = true; break; }
+            if (bar_or_r(1 + (warp & 3), 2 * 32, !ok)) { failed = true; break; }
             const float ss = xss[(x * 2) * 128 + r] + xss[(x * 2 + 1) * 128 + r];
             const float nrm = sqrtf(ss * (1.f / 128.f));
             const float rcp = ss > 0.f ? __frcp_rn(sqrtf(ss)) : 0.f;   // y = Y / ||Y||
@@ -1049,11 +1057,24 @@ bool rot_tensor_map(int d, tq_dtype dt, const EncArgs& a, CUtensorMap* tm) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Every launch is a programmatic dependent of the previous kernel on the stream, so that the
+// set-up (barriers, tensor memory, the rotation operand, the JL operand copy) overlaps that
+// kernel's end.  A chained launch (pdl: the previous kernel writes neither this input nor the
+// cache range) loads at once; any other waits for the previous kernel before its first input
+// load, and every write of the kernel follows that load.
+EncArgs dependent_args(const EncArgs& a, bool chained) {
+    EncArgs b = a;
+    b.wait_x = chained ? 0 : 1;
+    return b;
+}
+
 }  // namespace
 
-cudaError_t launch_encode64_rot(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
+cudaError_t launch_encode64_rot(bool is_k, tq_dtype dt, const EncArgs& a0, int num_sms, bool pdl, cudaStream_t s) {
     CUtensorMap tm;
-    if (!a.bimg || !rot_tensor_map(k6D, dt, a, &tm)) return cudaErrorNotSupported;
+    if (!a0.bimg || !rot_tensor_map(k6D, dt, a0, &tm)) return cudaErrorNotSupported;
+    const EncArgs a = dependent_args(a0, pdl);
+    pdl = true;
     const int64_t N = a.B * a.Hkv * a.Tnew;
     const int64_t ntiles = (N + kRRows - 1) / kRRows;
     const int grid = (int)(ntiles < 2 * (int64_t)num_sms ? ntiles : 2 * (int64_t)num_sms);
@@ -1062,9 +1083,11 @@ cudaError_t launch_encode64_rot(bool is_k, tq_dtype dt, const EncArgs& a, int nu
     return is_k ? launch_rot64_t<TQ_F16, true>(tm, a, grid, pdl, s) : launch_rot64_t<TQ_F16, false>(tm, a, grid, pdl, s);
 }
 
-cudaError_t launch_encode128_rot(bool is_k, tq_dtype dt, const EncArgs& a, int num_sms, bool pdl, cudaStream_t s) {
+cudaError_t launch_encode128_rot(bool is_k, tq_dtype dt, const EncArgs& a0, int num_sms, bool pdl, cudaStream_t s) {
     CUtensorMap tm;
-    if (!rot_tensor_map(kRD, dt, a, &tm)) return cudaErrorNotSupported;
+    if (!rot_tensor_map(kRD, dt, a0, &tm)) return cudaErrorNotSupported;
+    const EncArgs a = dependent_args(a0, pdl);
+    pdl = true;
     const int64_t N = a.B * a.Hkv * a.Tnew;
     const int64_t ntiles = (N + kRRows - 1) / kRRows;
     const int grid = (int)(ntiles < num_sms ? ntiles : num_sms);

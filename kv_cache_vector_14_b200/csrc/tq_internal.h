@@ -133,6 +133,10 @@ struct EncArgs {
                               // coordinate; d = 64: K index in slot order), rows in sign-word order
     int* err;                 // device check word
     int vec16;                // every input row starts on a 16-byte boundary
+    int wait_x;               // launched as a programmatic dependent of a kernel that may write the
+                              // input or the cache: wait for it (griddepcontrol.wait) before the first
+                              // input load (tensor-core encodes)
+    uint32_t dneg[4];         // bit i of word i / 32: d_i < 0 (head_dim up to 128)
     FastDiv fdT, fdH;         // division by Tnew and by Hkv (vector counts below 2^31)
     Codebook cb;
 };
@@ -282,6 +286,7 @@ struct tq_handle {
     float* dST = nullptr;     // [d][m] transposed S (query prologue)
     float* dSThr = nullptr;   // [d][d/32][32] encode lane order
     uint8_t* dSB = nullptr;   // d = 128: JL operand image for the tensor-core encode (64 KB)
+    uint32_t dneg[8] = {};    // bit i of word i / 32: d_i < 0
     int* derr = nullptr;
     tqi::Codebook cb{};
     cudaEvent_t ev_start = nullptr;   // optional timing of the split-K kernel
