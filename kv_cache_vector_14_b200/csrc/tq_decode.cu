@@ -45,9 +45,11 @@ __device__ void smem_fwht(float* v) {
 
 // ---------------------------------------------------------------- prologue
 // q' = H D q / sqrt(d) and up = sqrt(pi/2)/m * S q'.  A CTA takes QH = D / kRC
-// query heads and one chunk of kRC rows of S: it transforms its heads in
-// shared memory and stages the kRC columns of S^T it needs (one L2 read of S
-// per head group).  Warp w then sums coordinates [32 w, 32 w + 32) for row
+// query heads and one chunk of kRC rows of S: warp k transforms head k in
+// registers (coordinate lane + 32 r in element r; butterflies over the lane
+// bits by shuffles, then over r, the levels in the same order as a butterfly
+// over the whole index, so the sums are the same) while the kRC columns of
+// S^T it needs are staged (one L2 read of S per head group).  Warp w then sums coordinates [32 w, 32 w + 32) for row
 // `lane` of the chunk and all QH heads at once (each staged S value is read
 // once per CTA), and the QH partial sums of every output are added in warp
 // order.  The CTAs of row chunk 0 also store q'.
@@ -63,21 +65,37 @@ __global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t B
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int64_t h0 = (int64_t)blockIdx.x * QH;
     const int rc = blockIdx.y;
+    // the query loads go out first: the rotation waits for them, not for S
+    constexpr int R = D / 32;
+    const int64_t hw = h0 + warp;                        // this warp's head
+    float x[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) x[r] = (hw < BHq) ? load_q<DT>(q, hw * D + lane + 32 * r) : 0.f;
     for (int i = t; i < D * kRC / 4; i += D) {          // in flight during the rotation below
         const int jr = i / (kRC / 4), c4 = i % (kRC / 4);
         cp_async16(reinterpret_cast<float4*>(sst) + i, reinterpret_cast<const float4*>(ST + (size_t)jr * D + rc * kRC) + c4);
     }
-    const float ds = dsign[t];
 #pragma unroll
-    for (int k = 0; k < QH; ++k) {
-        const int64_t h = h0 + k;
-        v[k * D + t] = (h < BHq) ? ds * load_q<DT>(q, h * D + t) : 0.f;
-    }
-    __syncthreads();
-    smem_fwht<D, QH>(v);
+    for (int r = 0; r < R; ++r) x[r] *= dsign[lane + 32 * r];
+#pragma unroll
+    for (int hb = 1; hb < 32; hb <<= 1)
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const float p = __shfl_xor_sync(kFull, x[r], hb);
+            x[r] = (lane & hb) ? (p - x[r]) : (x[r] + p);
+        }
+#pragma unroll
+    for (int hb = 1; hb < R; hb <<= 1)
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+            if ((r & hb) == 0) {
+                const float u = x[r], w = x[r | hb];
+                x[r] = u + w;
+                x[r | hb] = u - w;
+            }
     const float inv = 1.0f / sqrtf((float)D);
 #pragma unroll
-    for (int k = 0; k < QH; ++k) v[k * D + t] *= inv;
+    for (int r = 0; r < R; ++r) v[warp * D + lane + 32 * r] = x[r] * inv;
     cp_async_wait_all();
     __syncthreads();
     float acc[QH];
@@ -333,6 +351,8 @@ __global__ void __launch_bounds__(D) tq_combine_kernel(const float* part_ml, con
 template <int D, int DT>
 cudaError_t launch_prologue_t(dim3 grid, bool pdl, const void* q, int64_t BHq, const float* dsign, const float* st,
                               float* qp, float* up, cudaStream_t s) {
+    const cudaError_t e = set_carveout_once<tq_prologue_kernel<D, DT>>();
+    if (e != cudaSuccess) return e;
     if (pdl) return launch_pdl(tq_prologue_kernel<D, DT>, grid, dim3(D), 0, s, q, BHq, dsign, st, qp, up);
     tq_prologue_kernel<D, DT><<<grid, D, 0, s>>>(q, BHq, dsign, st, qp, up);
     return cudaGetLastError();
@@ -390,6 +410,9 @@ cudaError_t launch_decode_simt(int d, int G, bool qjl, const DecArgs& a, cudaStr
 cudaError_t launch_combine(int d, int64_t BHq, int nsplit, const float* part_ml, const float* part_acc,
                            const float* dsign, float* out, cudaStream_t s) {
     if (BHq == 0) return cudaSuccess;
+    cudaError_t e = d == 64 ? set_carveout_once<tq_combine_kernel<64>>()
+                    : d == 128 ? set_carveout_once<tq_combine_kernel<128>>() : set_carveout_once<tq_combine_kernel<256>>();
+    if (e != cudaSuccess) return e;
     if (d == 64)
         return launch_pdl(tq_combine_kernel<64>, dim3((unsigned)BHq), dim3(64), 0, s, part_ml, part_acc, nsplit, dsign, out);
     if (d == 128)

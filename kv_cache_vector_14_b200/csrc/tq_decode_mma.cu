@@ -317,26 +317,7 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
         const int64_t t0 = chunk_at(i, inB);
         return t0 < a.fresh_hi && a.fresh_lo < t0 + C::kChunk;
     };
-    for (int i = 0; i < kStages && i < nmine; ++i)      // warp-uniform
-        if (!fresh(i)) {
-            int64_t kb_, vb_;
-            blocks_of(i, kb_, vb_);
-            issue(i, kb_, vb_);
-        }
     pdl_wait();                           // q' and u' come from the prologue kernel
-    {
-        bool any = false;
-        for (int i = 0; i < kStages && i < nmine; ++i) any |= fresh(i);
-        if (any) {
-            asm volatile("fence.proxy.async;" ::: "memory");
-            for (int i = 0; i < kStages && i < nmine; ++i)
-                if (fresh(i)) {
-                    int64_t kb_, vb_;
-                    blocks_of(i, kb_, vb_);
-                    issue(i, kb_, vb_);
-                }
-        }
-    }
     // blocks of the next chunk to issue, looked up one chunk ahead so that a
     // block-table load overlaps a chunk of work
     int64_t next_k = 0, next_v = 0;
@@ -470,6 +451,16 @@ __global__ void __launch_bounds__(NW * 32, 1) tq_decode_mma_kernel(const DecArgs
                 sF[(g * 3) * 8 + hcol] = a.scale_log2 * (um / kQ) * (1.f / 64.f);
                 sF[(g * 3 + 1) * 8 + hcol] = 64.f * (float)usum;
             }
+        }
+    }
+    {
+        bool any = false;
+        for (int i = 0; i < kStages && i < nmine; ++i) any |= fresh(i);
+        if (any) asm volatile("fence.proxy.async;" ::: "memory");
+        for (int i = 0; i < kStages && i < nmine; ++i) {
+            int64_t kb_, vb_;
+            blocks_of(i, kb_, vb_);
+            issue(i, kb_, vb_);
         }
     }
     // the crossing warp's unit-A result starts empty (it stays so if a wait fails before the crossing)

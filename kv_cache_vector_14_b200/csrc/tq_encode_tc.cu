@@ -552,6 +552,8 @@ cudaError_t launch_t(bool is_k, const EncArgs& a, int num_sms, bool pdl, cudaStr
     const int64_t ctas = (nquads + kVWarps - 1) / kVWarps;
     const int64_t cap = (int64_t)num_sms * 8;
     const unsigned grid = (unsigned)(ctas < cap ? ctas : cap);
+    const cudaError_t e = set_carveout_once<tq_encode_v128_kernel<DT>>();
+    if (e != cudaSuccess) return e;
     if (pdl) return launch_pdl(tq_encode_v128_kernel<DT>, dim3(grid), dim3(kVWarps * 32), 0, s, a);
     tq_encode_v128_kernel<DT><<<grid, kVWarps * 32, 0, s>>>(a);
     return cudaGetLastError();

@@ -236,6 +236,27 @@ cudaError_t set_smem_once(int bytes) {
     const unsigned long long bit = 1ull << (dev & 63);
     if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
     e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    // the largest carveout too, as set_carveout_once below gives the step's other kernels
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(Kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
+
+// Ask once per device and process for the largest shared-memory carveout.  The
+// kernels of one decode step (appends, prologue, split-K, combine) then find the
+// SMs configured alike, so a programmatic dependent's CTAs start without an SM
+// being reconfigured, and a kernel with little shared memory fits as many CTAs
+// per SM as its registers allow.
+template <auto Kern>
+cudaError_t set_carveout_once() {
+    static std::atomic<unsigned long long> done{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
     return e;
 }
