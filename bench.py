@@ -43,8 +43,8 @@ ENCODE_BYTES_PER_VECTOR = {("k", 128): 68, ("v", 128): 50}
 # DRAM traffic of the split-K kernel (read + write bytes per launch) from one
 # ncu capture, valid only while the kernel sources are unchanged (sha256 over
 # DECODE_SOURCES at capture time).
-NCU_TRAFFIC = {"source_sha256": "5c049d98fcda1a7fe56dd10f33487846439c36083a776b102f2a97a27b3632ef",
-               "bytes_per_launch": 387300864 + 3434240,
+NCU_TRAFFIC = {"source_sha256": "b92fbfb91599ce7faae1a3c9cf92f313b8878332d27044e65647f74a8e4377fc",
+               "bytes_per_launch": 387270144 + 3134208,
                "capture": "profiles/tq_decode_mma_d128_long_context_b4_hq16_hkv8_t102400.md"}
 
 
