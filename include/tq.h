@@ -147,6 +147,10 @@ TQ_API size_t tq_cache_bytes(int head_dim, int is_k, int64_t B, int64_t Hkv, int
  * takes the upper cell), and for K the residual's norm gamma (fp16) and the
  * sign bits of S * residual are stored.  A zero vector stores code 4, gamma 0,
  * all signs 1.  Tokens outside [t0, t0+Tnew) are not touched.
+ * Stream order holds as for any launch.  A bulk encode of 16-bit input (at
+ * d = 64 and 128, at least 16384 contiguous vectors) starts its set-up while
+ * the previous kernel on the stream finishes, and it waits for that kernel
+ * before it reads x or writes the cache.
  * Errors: INVALID_ARG (NULL pointers, B/Hkv mismatch with the cache, Tnew < 0,
  * t0 < 0, t0 + Tnew > Tcap, misaligned x or cache), CUDA. */
 TQ_API tq_status tq_encode_k(const tq_handle* h, const void* x, tq_dtype dtype, int64_t B, int64_t Hkv,
