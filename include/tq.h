@@ -251,9 +251,9 @@ TQ_API tq_status tq_attend_prefill(const tq_handle* h, const void* q, tq_dtype q
  * tq_attend_decode (ws sized by tq_attend_workspace_bytes(h, B, Hq, Hkv,
  * t0 + Tnew)).  The kernels are chained with programmatic dependent launch:
  * the query prologue runs alongside the encodes and the attention kernel
- * prefetches every cached chunk except the ones holding the new tokens
- * before they are written; every kernel completes only after the one before
- * it, so the next work on the stream sees the finished step.
+ * sets up while they run, reading the cache only after they complete; every
+ * kernel completes only after the one before it, so the next work on the
+ * stream sees the finished step.
  * Errors: those of tq_encode_k and tq_attend_decode (checked before any
  * launch). */
 TQ_API tq_status tq_append_attend(const tq_handle* h, const void* k_new, const void* v_new, tq_dtype kv_dtype,

@@ -562,8 +562,8 @@ tq_status tq_append_attend(const tq_handle* h, const void* k_new, const void* v_
     if (chained) {
         // K encode as a plain launch, V encode and the prologue as its
         // programmatic dependents (each completes only after its predecessor);
-        // the split-K kernel prefetches every chunk but the appended tokens'
-        // before it waits.
+        // the split-K kernel sets up while they run and reads the cache and
+        // the query operands after it waits.
         e = launch_encode(h->d, true, kv_dtype, ek, h->num_sms, false, s);
         if (e == cudaSuccess) e = launch_encode(h->d, false, kv_dtype, ev, h->num_sms, true, s);
         a.fresh_lo = t0;

@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(D) tq_prologue_kernel(const void* q, int64_t B
     constexpr int QH = D / kRC;                           // heads per CTA = warps per CTA
     __shared__ __align__(16) float v[QH * D];
     __shared__ __align__(16) float sst[D * kRC];          // sst[j][i] = S[rc*kRC + i][j]; then partial sums
-    pdl_trigger();                                        // the split-K kernel may start its prefetch
+    pdl_trigger();                                        // the split-K kernel may start its set-up
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int64_t h0 = (int64_t)blockIdx.x * QH;
     const int rc = blockIdx.y;
